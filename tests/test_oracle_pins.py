@@ -1,0 +1,444 @@
+"""Pins for the CPU oracle: checks against what the pages and the mathematics fix, never against the
+oracle's own formulas retyped.  CPU only.
+
+Each test names the plausible mistake it would catch.
+"""
+import numpy as np
+import pytest
+from scipy.special import expit
+
+import oracle
+from bit_quantized_mamba_b200 import inputs
+
+
+def unpack_pm1(bits: np.ndarray) -> np.ndarray:
+    """Independent unpack: numpy's little-endian bit order over the little-endian words."""
+    d_out, words = bits.shape
+    b = np.unpackbits(bits.view(np.uint8).reshape(d_out, words * 4), axis=1, bitorder="little")
+    return b.astype(np.int64) * 2 - 1
+
+
+def pack_pm1(signs: np.ndarray) -> np.ndarray:
+    """Independent pack of a +-1 matrix into LSB-first uint32 words."""
+    d_out, d_in = signs.shape
+    by = np.packbits((signs > 0).astype(np.uint8), axis=1, bitorder="little")
+    return np.ascontiguousarray(by).view(np.uint32).reshape(d_out, d_in // 32)
+
+
+# ------------------------------------------------------------------------------------- sign expansion
+
+def test_sign_exhaustive_byte_patterns():
+    """Every byte pattern in every byte lane: catches a wrong bit order (MSB-first), a wrong word index
+    or an inverted sign convention."""
+    rows = np.arange(256, dtype=np.uint32)
+    bits = np.zeros((256, 2), np.uint32)
+    for lane in range(4):
+        bits[:, 0] |= rows << (8 * lane)
+    bits[:, 1] = ~bits[:, 0]
+    for o in range(256):
+        for i in range(64):
+            word, j = divmod(i, 32)
+            byte_val = o if word == 0 else (255 - o)
+            expected = 1 if (byte_val >> (j % 8)) & 1 else -1
+            assert oracle.sign(bits, 64, o, i) == expected, (o, i)
+
+
+def test_sign_random_round_trip():
+    g = np.random.default_rng(11)
+    signs = g.choice(np.array([-1, 1]), size=(24, 96))
+    bits = pack_pm1(signs)
+    for o in range(24):
+        for i in range(96):
+            assert oracle.sign(bits, 96, o, i) == signs[o, i]
+
+
+# ------------------------------------------------------------------------------------------ quantizer
+
+def test_quantize_absmax_and_error_bound():
+    g = np.random.default_rng(5)
+    x = g.standard_normal((6, 1000)).astype(np.float32) * np.float32(3.0)
+    q, s = oracle.quantize(x)
+    for b in range(6):
+        k = np.argmax(np.abs(x[b]))
+        assert abs(int(q[b, k])) == 127 and np.sign(q[b, k]) == np.sign(x[b, k])
+        assert np.all(np.abs(q[b]) <= 127)
+        err = np.abs(x[b].astype(np.float64) - float(s[b]) * q[b].astype(np.float64))
+        assert err.max() <= float(s[b]) / 2 * (1 + 2.0 ** -18)
+        # s is absmax/127 to fp32 precision
+        assert abs(float(s[b]) * 127 - np.abs(x[b]).max()) <= 1e-6 * np.abs(x[b]).max()
+
+
+def test_quantize_round_half_even_ties():
+    """absmax 127 gives s == 1 exactly, so codes are rint(x): ties must go to even."""
+    x = np.array([[127.0, 2.5, 3.5, -2.5, 0.5, -0.5, 1.5, 126.5]], np.float32)
+    q, s = oracle.quantize(x)
+    assert s[0] == 1.0
+    assert q[0].tolist() == [127, 2, 4, -2, 0, 0, 2, 126]
+
+
+def test_quantize_power_of_two_invariance():
+    g = np.random.default_rng(6)
+    x = g.standard_normal((3, 513)).astype(np.float32)
+    q, s = oracle.quantize(x)
+    for k in (-7, -1, 3, 10):
+        q2, s2 = oracle.quantize(x * np.float32(2.0 ** k))
+        assert np.array_equal(q, q2)
+        assert np.array_equal(s2, s * np.float32(2.0 ** k))
+
+
+def test_quantize_zero_row():
+    q, s = oracle.quantize(np.zeros((2, 64), np.float32))
+    assert np.all(q == 0) and np.all(s == 0)
+
+
+def test_quantize_matches_ieee_fp32_division():
+    """The fp64-then-round division equals numpy's IEEE fp32 division (no double-rounding slip)."""
+    g = np.random.default_rng(7)
+    x = g.standard_normal((50, 4096)).astype(np.float32)
+    q, s = oracle.quantize(x)
+    for b in range(50):
+        m = np.abs(x[b]).max()
+        s32 = np.float32(m) / np.float32(127.0)
+        assert s32 == s[b]
+        r = (x[b] / s32).astype(np.float32)
+        assert np.array_equal(np.clip(np.rint(r), -127, 127).astype(np.int8), q[b])
+
+
+# --------------------------------------------------------------------------------- scaffold GEMV
+
+@pytest.fixture(scope="module")
+def tiny():
+    return inputs.tiny_linear(0)
+
+
+def test_gemv_brute_force_tiny(tiny):
+    """acc equals an explicit +-1 integer matmul (the brute-force tiny GEMV)."""
+    L = oracle.Linear.from_dict(tiny["linear"])
+    out = oracle.linear_decode(L, tiny["x"])
+    S = unpack_pm1(L.bits)
+    q = out["xq"][0].astype(np.int64)
+    assert np.array_equal(out["acc"][0].astype(np.int64), S @ q)
+    # identity acc = 2*sum_{bit=1} q - sum q
+    ones = (S > 0).astype(np.int64)
+    assert np.array_equal(out["acc"][0], 2 * (ones @ q) - q.sum())
+
+
+def test_gemv_bit_flip_negates_and_all_ones(tiny):
+    L = oracle.Linear.from_dict(tiny["linear"])
+    base = oracle.linear_decode(L, tiny["x"])
+    d = dict(tiny["linear"])
+    d["bits"] = ~L.bits
+    flipped = oracle.linear_decode(oracle.Linear.from_dict(d), tiny["x"])
+    assert np.array_equal(flipped["acc"], -base["acc"])
+    d["bits"] = np.full_like(L.bits, 0xFFFFFFFF)
+    allones = oracle.linear_decode(oracle.Linear.from_dict(d), tiny["x"])
+    assert np.all(allones["acc"][0] == base["xq"][0].astype(np.int64).sum())
+
+
+def test_gemv_one_hot_input(tiny):
+    L = oracle.Linear.from_dict(tiny["linear"])
+    S = unpack_pm1(L.bits)
+    for j in (0, 31, 32, 200, 255):
+        x = np.zeros((1, 256), np.float32)
+        x[0, j] = -2.0
+        out = oracle.linear_decode(L, x)
+        assert out["xq"][0, j] == -127
+        assert np.array_equal(out["acc"][0], -127 * S[:, j])
+
+
+# ------------------------------------------------------------------------------------------- LoRA
+
+def test_lora_rank0_equals_scaffold_alone(tiny):
+    """r = 0 gives the scaffold alone; W_A = 0 gives the same, bit for bit."""
+    d = dict(tiny["linear"])
+    full = oracle.linear_decode(oracle.Linear.from_dict(d), tiny["x"])
+    r0 = dict(d, lora_b=np.zeros((0, 256), np.int8), lora_b_scale=np.zeros(0, np.float32),
+              lora_a=np.zeros((512, 0), np.int8))
+    out0 = oracle.linear_decode(oracle.Linear.from_dict(r0), tiny["x"])
+    wa0 = dict(d, lora_a=np.zeros_like(d["lora_a"]))
+    outa = oracle.linear_decode(oracle.Linear.from_dict(wa0), tiny["x"])
+    assert np.array_equal(out0["y"], outa["y"])
+    assert np.array_equal(out0["acc"], full["acc"])
+    s = float(out0["xscale"][0])
+    expect = (out0["acc"][0].astype(np.float64) * s * d["w_scale"].astype(np.float64))
+    assert np.allclose(out0["y"][0], expect, rtol=2e-7, atol=0)
+    assert not np.array_equal(full["y"], out0["y"])  # the LoRA term is not silently dropped
+
+
+def test_lora_one_hot_down_rows(tiny):
+    d = dict(tiny["linear"])
+    cols = [3, 17, 100, 255, 0, 64, 128, 129, 5, 6, 7, 8, 9, 10, 11, 12]
+    lb = np.zeros((16, 256), np.int8)
+    for r, c in enumerate(cols):
+        lb[r, c] = 1
+    out = oracle.linear_decode(oracle.Linear.from_dict(dict(d, lora_b=lb)), tiny["x"])
+    assert np.array_equal(out["t"][0], out["xq"][0, cols].astype(np.int32))
+
+
+def test_lora_epilogue_real_number_formula(tiny):
+    """y = acc*s*sW + sA * W_A @ (t*sB*s) to fp32 accuracy: catches a transposed W_A, a missing scale or
+    a wrong-sign term."""
+    d = tiny["linear"]
+    L = oracle.Linear.from_dict(d)
+    out = oracle.linear_decode(L, tiny["x"])
+    s = float(out["xscale"][0])
+    t = (unpack_t := out["t"][0].astype(np.float64))
+    assert np.array_equal(unpack_t, d["lora_b"].astype(np.int64) @ out["xq"][0].astype(np.int64))
+    tf = t * d["lora_b_scale"].astype(np.float64) * s
+    y = (out["acc"][0] * s * d["w_scale"].astype(np.float64)
+         + d["lora_a_scale"].astype(np.float64) * (d["lora_a"].astype(np.float64) @ tf))
+    assert np.allclose(out["y"][0], y, rtol=1e-6, atol=1e-7)
+
+
+# ------------------------------------------------------------------------------------------- conv
+
+def silu(v):
+    return v * expit(v)
+
+
+def test_conv_stepped_equals_textbook_convolution():
+    g = np.random.default_rng(9)
+    T, Cn = 11, 8
+    x = g.standard_normal((T, Cn)).astype(np.float32)
+    w = g.normal(0, 0.5, (Cn, 4)).astype(np.float32)
+    b = g.normal(0, 0.1, Cn).astype(np.float32)
+    state = np.zeros((1, Cn, 3), np.float32)
+    outs = np.stack([oracle.conv_step(state, w, b, x[t:t + 1])[0] for t in range(T)])
+    for c in range(Cn):
+        # causal conv: out[t] = sum_k w[c,k] * x[t-3+k]  (numpy full convolution with reversed taps)
+        pre = np.convolve(x[:, c].astype(np.float64), w[c, ::-1].astype(np.float64))[:T] + b[c]
+        assert np.allclose(outs[:, c], silu(pre), rtol=1e-6, atol=1e-7)
+    assert np.array_equal(state[0], x[-3:].T)
+
+
+def test_conv_impulse_reproduces_taps():
+    Cn = 5
+    w = np.arange(20, dtype=np.float32).reshape(Cn, 4) / 10 - 1
+    b = np.zeros(Cn, np.float32)
+    state = np.zeros((1, Cn, 3), np.float32)
+    for t in range(6):
+        x = np.ones((1, Cn), np.float32) if t == 0 else np.zeros((1, Cn), np.float32)
+        out = oracle.conv_step(state, w, b, x)[0]
+        expect = silu(w[:, 3 - t].astype(np.float64)) if t < 4 else np.zeros(Cn)
+        assert np.allclose(out, expect, rtol=1e-6, atol=1e-8)
+
+
+# -------------------------------------------------------------------------------------------- SSM
+
+def softplus(v):
+    return np.logaddexp(0.0, v)
+
+
+def ssd_dual_form(x, dt_raw, A_log, dt_bias, D, Bm, Cm, G):
+    """Quadratic (attention-like) form of the selective SSM over a whole sequence, fp64:
+    y_t = sum_{s<=t} (prod_{k=s+1..t} a_k) * dt_s * (C_t . B_s) * x_s + D * x_t."""
+    T, H, P = x.shape
+    N = Bm.shape[-1]
+    dt = softplus(dt_raw.astype(np.float64) + dt_bias.astype(np.float64))  # [T,H]
+    a = np.exp(dt * -np.exp(A_log.astype(np.float64)))                     # [T,H]
+    y = np.zeros((T, H, P))
+    for h in range(H):
+        g = h // (H // G)
+        for t in range(T):
+            for s in range(t + 1):
+                decay = np.prod(a[s + 1:t + 1, h])
+                cb = float(Cm[t, g].astype(np.float64) @ Bm[s, g].astype(np.float64))
+                y[t, h] += decay * dt[s, h] * cb * x[s, h].astype(np.float64)
+            y[t, h] += D[h] * x[t, h]
+    return y
+
+
+@pytest.mark.parametrize("H,G", [(2, 1), (4, 2)])
+def test_ssm_stepped_equals_dual_form(H, G):
+    g = np.random.default_rng(13 + H)
+    T, P, N = 12, 3, 5
+    x = g.standard_normal((T, H, P)).astype(np.float32)
+    dt_raw = g.standard_normal((T, H)).astype(np.float32)
+    A_log = g.uniform(0, 1.5, H).astype(np.float32)
+    dt_bias = g.uniform(-2, 0, H).astype(np.float32)
+    D = g.uniform(0.5, 1.5, H).astype(np.float32)
+    Bm = g.standard_normal((T, G, N)).astype(np.float32)
+    Cm = g.standard_normal((T, G, N)).astype(np.float32)
+    state = np.zeros((1, H, P, N), np.float32)
+    ys = np.stack([oracle.ssm_step(state, x[t].reshape(1, -1), dt_raw[t:t + 1], A_log, dt_bias, D,
+                                   Bm[t:t + 1], Cm[t:t + 1]).reshape(H, P) for t in range(T)])
+    ref = ssd_dual_form(x, dt_raw, A_log, dt_bias, D, Bm, Cm, G)
+    assert np.allclose(ys, ref, rtol=1e-5, atol=1e-5)
+
+
+def test_ssm_constant_input_geometric_closed_form():
+    H, P, N, T = 1, 2, 3, 9
+    x = np.array([[0.7, -1.3]], np.float32)
+    Bv = np.array([[[0.5, -0.25, 1.0]]], np.float32)
+    Cv = np.array([[[1.5, 2.0, -0.5]]], np.float32)
+    dt_raw = np.array([[0.3]], np.float32)
+    A_log = np.array([0.2], np.float32)
+    dt_bias = np.array([-1.0], np.float32)
+    D = np.array([0.9], np.float32)
+    state = np.zeros((1, H, P, N), np.float32)
+    for _ in range(T):
+        y = oracle.ssm_step(state, x, dt_raw, A_log, dt_bias, D, Bv, Cv)
+    dt = softplus(-0.7)
+    a = np.exp(dt * -np.exp(0.2))
+    S = dt * x[0][:, None].astype(np.float64) * Bv[0, 0][None, :] * (1 - a ** T) / (1 - a)
+    assert np.allclose(state[0, 0], S, rtol=1e-5)
+    assert np.allclose(y[0], S @ Cv[0, 0] + 0.9 * x[0], rtol=1e-5)
+
+
+def test_ssm_dt_to_zero_freezes_state():
+    g = np.random.default_rng(21)
+    H, P, N = 2, 4, 8
+    state = g.standard_normal((1, H, P, N)).astype(np.float32)
+    before = state.copy()
+    x = g.standard_normal((1, H * P)).astype(np.float32)
+    Bv = g.standard_normal((1, 1, N)).astype(np.float32)
+    Cv = g.standard_normal((1, 1, N)).astype(np.float32)
+    D = np.array([0.5, 1.25], np.float32)
+    y = oracle.ssm_step(state, x, np.zeros((1, H), np.float32), np.zeros(H, np.float32),
+                        np.full(H, -60.0, np.float32), D, Bv, Cv)
+    assert np.array_equal(state, before)
+    ref = before[0] @ Cv[0, 0].astype(np.float64) + (np.repeat(D, P) * x[0]).reshape(H, P)
+    assert np.allclose(y[0].reshape(H, P), ref, rtol=1e-6, atol=1e-6)
+
+
+def test_ssm_dA_to_zero_is_memoryless():
+    g = np.random.default_rng(22)
+    H, P, N = 2, 3, 4
+    state = g.standard_normal((1, H, P, N)).astype(np.float32) * 100
+    x = g.standard_normal((1, H * P)).astype(np.float32)
+    Bv = g.standard_normal((1, 1, N)).astype(np.float32)
+    Cv = g.standard_normal((1, 1, N)).astype(np.float32)
+    D = np.zeros(H, np.float32)
+    y = oracle.ssm_step(state, x, np.zeros((1, H), np.float32), np.full(H, 6.0, np.float32),
+                        np.full(H, 2.0, np.float32), D, Bv, Cv)
+    dt = softplus(2.0)
+    S = dt * x[0].reshape(H, P, 1).astype(np.float64) * Bv[0, 0].astype(np.float64)
+    assert np.allclose(state[0], S, rtol=1e-6)
+    assert np.allclose(y[0].reshape(H, P), S @ Cv[0, 0].astype(np.float64), rtol=1e-5, atol=1e-6)
+
+
+# --------------------------------------------------------------------------------- norms and gate
+
+def test_rmsnorm_constant_row_reconstructs_weight():
+    g = np.random.default_rng(30)
+    w = g.uniform(0.5, 1.5, 256).astype(np.float32)
+    for c in (-3.0, 0.25, 40.0):
+        h = np.full((1, 256), c, np.float32)
+        q, s = oracle.rmsnorm_quantize(h, w)
+        u = np.sign(c) * w.astype(np.float64) / np.sqrt(1 + 1e-5 / c ** 2)
+        assert np.all(np.abs(s[0] * q[0] - u) <= s[0] / 2 * 1.0001)
+
+
+def test_rmsnorm_fold_matches_explicit_normalization_away_from_ties():
+    """Quantizing the explicitly normalized row gives the same codes except within 1e-4 of a rounding
+    tie, and the scale is the explicit one to fp32 precision."""
+    g = np.random.default_rng(31)
+    h = (g.standard_normal((8, 2048)) * 3).astype(np.float32)
+    w = g.uniform(0.5, 1.5, 2048).astype(np.float32)
+    q, s = oracle.rmsnorm_quantize(h, w)
+    for b in range(8):
+        hb = h[b].astype(np.float64)
+        u = hb / np.sqrt(np.mean(hb ** 2) + 1e-5) * w
+        m = np.abs(u).max()
+        r = u / (m / 127)
+        near_tie = np.abs(np.abs(r - np.floor(r)) - 0.5) < 1e-4
+        exact = np.rint(r).astype(np.int64)
+        assert np.all((exact == q[b]) | near_tie)
+        assert abs(s[b] - m / 127) <= 1e-6 * m / 127
+
+
+def test_gate_silu_against_logistic():
+    g = np.random.default_rng(32)
+    y = g.standard_normal(1000).astype(np.float32)
+    z = (g.standard_normal(1000) * 4).astype(np.float32)
+    out = oracle.gate(y, z)
+    assert np.allclose(out, y * (z * expit(z.astype(np.float64))), rtol=1e-6, atol=1e-9)
+
+
+# ------------------------------------------------------------------------------------ layer wiring
+
+SMALL = dict(d_model=64, nheads=4, headdim=16, d_state=16, ngroups=1, rank=4)
+
+
+def _oracle_layer(ld):
+    lay = dict(ld)
+    lay["in_proj"] = oracle.Linear.from_dict(ld["in_proj"])
+    lay["out_proj"] = oracle.Linear.from_dict(ld["out_proj"])
+    return lay
+
+
+def test_layer_zero_out_proj_keeps_residual():
+    m = inputs.decode_model(seed=40, n_layers=1, n_tokens=2, **SMALL)
+    ld = m["layers"][0]
+    ld["out_proj"]["w_scale"][:] = 0
+    ld["out_proj"]["lora_a_scale"][:] = 0
+    lay = _oracle_layer(ld)
+    conv, ssm = inputs.zero_states(1, 1, 4, 16, 16, 1)
+    h = m["emb"][0].copy()
+    h0 = h.copy()
+    taps = oracle.layer_decode(lay, h, conv[0], ssm[0], taps=True)
+    assert np.array_equal(h, h0)
+    assert np.any(ssm[0] != 0) and np.any(taps["y"] != 0)
+
+
+def test_layer_composition_of_pinned_steps():
+    """The layer equals the pinned steps wired as: norm+quant -> in_proj -> split z|x|B|C|dt -> conv ->
+    SSM -> gate -> norm+quant -> out_proj -> residual."""
+    m = inputs.decode_model(seed=41, n_layers=1, n_tokens=3, **SMALL)
+    lay = _oracle_layer(m["layers"][0])
+    E, N = 64, 16
+    conv_a, ssm_a = inputs.zero_states(1, 1, 4, 16, 16, 1)
+    conv_b, ssm_b = conv_a.copy(), ssm_a.copy()
+    for t in range(3):
+        h_a = m["emb"][t].copy()
+        oracle.layer_decode(lay, h_a, conv_a[0], ssm_a[0])
+        h_b = m["emb"][t].copy()
+        q, s = oracle.rmsnorm_quantize(h_b, lay["norm_w"])
+        zx, _, _ = oracle.linear_core(lay["in_proj"], q[0], s[0])
+        z, xbc, dt = zx[:E], zx[E:E + E + 2 * N], zx[E + E + 2 * N:]
+        xc = oracle.conv_step(conv_b[0], lay["conv_w"], lay["conv_b"], xbc[None])[0]
+        y = oracle.ssm_step(ssm_b[0], xc[None, :E], dt[None], lay["A_log"], lay["dt_bias"], lay["D"],
+                            xc[None, E:E + N], xc[None, E + N:])[0]
+        gg = oracle.gate(y, z)
+        q2, s2 = oracle.rmsnorm_quantize(gg[None], lay["gnorm_w"])
+        out, _, _ = oracle.linear_core(lay["out_proj"], q2[0], s2[0])
+        h_b = (h_b[0] + out).astype(np.float32)
+        assert np.array_equal(h_a[0], h_b)
+        assert np.array_equal(ssm_a, ssm_b) and np.array_equal(conv_a, conv_b)
+
+
+# ------------------------------------------------------------------------------------------ LM head
+
+def test_lm_head_brute_force():
+    g = np.random.default_rng(50)
+    W = g.integers(-127, 128, (300, 128), dtype=np.int8)
+    sr = g.uniform(1e-4, 1e-3, 300).astype(np.float32)
+    x = g.standard_normal(128).astype(np.float32)
+    logits, acc = oracle.lm_head(W, sr, x)
+    q, s = oracle.quantize(x[None])
+    assert np.array_equal(acc, W.astype(np.int64) @ q[0].astype(np.int64))
+    assert np.allclose(logits, acc.astype(np.float64) * float(s[0]) * sr, rtol=2e-7)
+    rows = np.array([299, 0, 17])
+    l2, a2 = oracle.lm_head(W, sr, x, rows)
+    assert np.array_equal(a2, acc[rows]) and np.array_equal(l2, logits[rows])
+
+
+# ------------------------------------------------------------------------------------- shape pins
+
+def test_model_size_and_composition_pin():
+    """The 1.3B shapes reproduce the printed size split of the 278 MB model (56% scaffold, 37%
+    embedding/LM head, 4% LoRA, rest other) and 1 bit per scaffold weight (8x less than int8)."""
+    total = 278e6
+    L, Dm, E, Nst, H = inputs.N_LAYERS, inputs.D_MODEL, inputs.D_INNER, inputs.D_STATE, inputs.N_HEADS
+    d_ip = inputs.D_IN_PROJ
+    assert d_ip == 2 * E + 2 * Nst + H == 8512
+    scaffold_weights = L * (d_ip * Dm + Dm * E)
+    scaffold_bytes = scaffold_weights / 8
+    lm_bytes = inputs.VOCAB * Dm
+    lora_bytes = L * (inputs.RANK * Dm + d_ip * inputs.RANK + inputs.RANK * E + Dm * inputs.RANK)
+    assert round(100 * scaffold_bytes / total) == 56
+    assert round(100 * lm_bytes / total) == 37
+    assert 4 <= 100 * lora_bytes / total < 5
+    other = total - scaffold_bytes - lm_bytes - lora_bytes
+    assert 2 <= 100 * other / total < 3.5
+    assert scaffold_weights / scaffold_bytes == 8
