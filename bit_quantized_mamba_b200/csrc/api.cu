@@ -1,0 +1,362 @@
+// C ABI of libdfssm (declared in include/dfssm.h): argument validation and kernel launches.
+
+#include <cstdio>
+#include <cstring>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace {
+
+thread_local char g_last_cuda_error[256] = "";
+
+int cuda_fail(cudaError_t e) {
+  std::snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "%s: %s", cudaGetErrorName(e),
+                cudaGetErrorString(e));
+  return DFSSM_ECUDA;
+}
+
+inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+int check_linear(const dfssm_linear_t* L) {
+  if (!L) return DFSSM_EINVAL;
+  if (L->d_out < 1 || L->d_in < 32 || L->d_in % 32 != 0 || L->d_in > 8192) return DFSSM_EINVAL;
+  if (L->rank < 0 || L->rank > DFSSM_MAX_RANK) return DFSSM_EINVAL;
+  if (!L->bits || !L->w_scale) return DFSSM_EINVAL;
+  if (L->rank > 0 && (!L->lora_b || !L->lora_b_scale || !L->lora_a || !L->lora_a_scale))
+    return DFSSM_EINVAL;
+  if (!aligned(L->bits, 16) || !aligned(L->w_scale, 4)) return DFSSM_EALIGN;
+  if (L->rank > 0) {
+    if (!aligned(L->lora_b, 4) || !aligned(L->lora_b_scale, 4) || !aligned(L->lora_a_scale, 4))
+      return DFSSM_EALIGN;
+    if (L->rank == DFSSM_MAX_RANK && !aligned(L->lora_a, 16)) return DFSSM_EALIGN;
+  }
+  return DFSSM_OK;
+}
+
+size_t linear_decode_ws(int B, int d_in) { return dfssm::quant_scratch_bytes(B, d_in); }
+
+struct LayerWs {
+  float* zxbcdt;  // [B][d_ip]
+  float* xc;      // [B][C]
+  float* g;       // [B][E]
+  dfssm::QuantScratch qs;
+};
+
+size_t layer_ws_bytes(int B, int d_model, int E, int C, int d_ip) {
+  const int nmax = d_model > E ? d_model : E;
+  return align256(sizeof(float) * (size_t)B * d_ip) + align256(sizeof(float) * (size_t)B * C) +
+         align256(sizeof(float) * (size_t)B * E) + dfssm::quant_scratch_bytes(B, nmax);
+}
+
+LayerWs carve_layer_ws(void* base, int B, int d_model, int E, int C, int d_ip) {
+  char* p = static_cast<char*>(base);
+  LayerWs w;
+  w.zxbcdt = reinterpret_cast<float*>(p);
+  p += align256(sizeof(float) * (size_t)B * d_ip);
+  w.xc = reinterpret_cast<float*>(p);
+  p += align256(sizeof(float) * (size_t)B * C);
+  w.g = reinterpret_cast<float*>(p);
+  p += align256(sizeof(float) * (size_t)B * E);
+  const int nmax = d_model > E ? d_model : E;
+  w.qs = dfssm::carve_quant_scratch(p, B, nmax);
+  return w;
+}
+
+bool device_ok() {
+  static int ok = -1;
+  if (ok < 0) {
+    int dev = 0, major = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) {
+      cudaGetLastError();
+      ok = 0;
+    } else {
+      ok = (major == 10) ? 1 : 0;
+    }
+  }
+  return ok == 1;
+}
+
+dfssm::GemvArgs gemv_args(const dfssm_linear_t* L, int B, const dfssm::QuantScratch& qs) {
+  dfssm::GemvArgs g{};
+  g.bits = L->bits;
+  g.w_scale = L->w_scale;
+  g.lora_a = L->lora_a;
+  g.lora_a_scale = L->lora_a_scale;
+  g.lora_b_scale = L->lora_b_scale;
+  g.rank = L->rank;
+  g.d_out = L->d_out;
+  g.d_in = L->d_in;
+  g.B = B;
+  g.in = qs;
+  return g;
+}
+
+}  // namespace
+
+extern "C" {
+
+int dfssm_abi_version(void) { return DFSSM_ABI_VERSION; }
+
+const char* dfssm_status_string(int s) {
+  switch (s) {
+    case DFSSM_OK: return "ok";
+    case DFSSM_EINVAL: return "invalid argument";
+    case DFSSM_EALIGN: return "misaligned pointer";
+    case DFSSM_EUNSUPPORTED: return "unsupported configuration";
+    case DFSSM_ECUDA: return "CUDA error";
+    case DFSSM_ETIMEOUT: return "device wait timed out";
+    case DFSSM_EDEVICE: return "no usable sm_100 device";
+    case DFSSM_EWORKSPACE: return "workspace missing, too small or misaligned";
+    default: return "unknown status";
+  }
+}
+
+const char* dfssm_last_cuda_error(void) { return g_last_cuda_error; }
+
+size_t dfssm_workspace_size(int op, int a, int b, int c) {
+  switch (op) {
+    case DFSSM_OP_LINEAR_DECODE:
+      if (a < 1 || a > DFSSM_MAX_BATCH || b < 32 || b % 32 || b > 8192) return 0;
+      return linear_decode_ws(a, b);
+    case DFSSM_OP_LINEAR_PREFILL:
+      if (a < 1 || b < 128 || b % 128 || c < 1) return 0;
+      return dfssm::prefill_workspace_bytes(a, b, c);
+    case DFSSM_OP_LAYER_DECODE: {
+      if (a < 1 || a > DFSSM_MAX_BATCH || b < 32 || c < 32) return 0;
+      // conv channels and in_proj rows depend on d_state/ngroups/nheads; size for the largest
+      // supported (2*ngroups*d_state <= 2048, nheads <= 1024).
+      const int C = c + 2048, d_ip = 2 * c + 2048 + 1024;
+      return layer_ws_bytes(a, b, c, C, d_ip);
+    }
+    case DFSSM_OP_LM_HEAD:
+      if (b < 16 || b % 16 || b > 8192 || c < 1) return 0;
+      return dfssm::quant_scratch_bytes(1, b);
+    default: return 0;
+  }
+}
+
+int dfssm_pack_signs(const int8_t* signs, int d_out, int d_in, uint32_t* bits) {
+  if (!signs || !bits || d_out < 1 || d_in < 32 || d_in % 32) return DFSSM_EINVAL;
+  const int words = d_in / 32;
+  for (int o = 0; o < d_out; ++o) {
+    for (int w = 0; w < words; ++w) {
+      uint32_t v = 0;
+      for (int j = 0; j < 32; ++j)
+        if (signs[(size_t)o * d_in + 32 * w + j] > 0) v |= (1u << j);
+      bits[(size_t)o * words + w] = v;
+    }
+  }
+  return DFSSM_OK;
+}
+
+int dfssm_linear_decode(const dfssm_linear_t* lin, const float* x, int B, float* y, void* workspace,
+                        size_t ws_bytes, const dfssm_debug_t* dbg, void* stream) {
+  int st = check_linear(lin);
+  if (st) return st;
+  if (!x || !y || B < 1) return DFSSM_EINVAL;
+  if (B > DFSSM_MAX_BATCH) return DFSSM_EUNSUPPORTED;
+  if (!aligned(x, 16) || !aligned(y, 4)) return DFSSM_EALIGN;
+  if (!workspace || !aligned(workspace, 256) || ws_bytes < linear_decode_ws(B, lin->d_in))
+    return DFSSM_EWORKSPACE;
+  if (!device_ok()) return DFSSM_EDEVICE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  dfssm::QuantScratch qs = dfssm::carve_quant_scratch(workspace, B, lin->d_in);
+  dfssm::QuantArgs qa{};
+  qa.x = x;
+  qa.ldx = lin->d_in;
+  qa.norm_w = nullptr;
+  qa.n = lin->d_in;
+  qa.B = B;
+  qa.lora_b = lin->lora_b;
+  qa.rank = lin->rank;
+  qa.permute = true;
+  qa.out = qs;
+  if (dbg) {
+    qa.dbg_xq = dbg->xq;
+    qa.dbg_s = dbg->xscale;
+    qa.dbg_t = dbg->lora_t;
+  }
+  cudaError_t e = dfssm::launch_quant(qa, s);
+  if (e != cudaSuccess) return cuda_fail(e);
+  dfssm::GemvArgs ga = gemv_args(lin, B, qs);
+  ga.y = y;
+  ga.ldy = lin->d_out;
+  ga.dbg_acc = dbg ? dbg->acc : nullptr;
+  e = dfssm::launch_gemv(ga, s);
+  if (e != cudaSuccess) return cuda_fail(e);
+  return DFSSM_OK;
+}
+
+int dfssm_conv_step(float* conv_state, const float* w, const float* b, const float* x_in, float* x_out,
+                    int B, int C, void* stream) {
+  if (!conv_state || !w || !b || !x_in || !x_out || B < 1 || C < 1) return DFSSM_EINVAL;
+  if (!aligned(w, 16) || !aligned(conv_state, 4)) return DFSSM_EALIGN;
+  if (!device_ok()) return DFSSM_EDEVICE;
+  dfssm::ConvArgs a{conv_state, w, b, x_in, C, x_out, C, B, C};
+  cudaError_t e = dfssm::launch_conv(a, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? DFSSM_OK : cuda_fail(e);
+}
+
+int dfssm_ssm_step(float* ssm_state, const float* x, const float* dt_raw, const float* A_log,
+                   const float* dt_bias, const float* D, const float* Bm, const float* Cm, float* y,
+                   int B, int H, int P, int N, int G, void* stream) {
+  if (!ssm_state || !x || !dt_raw || !A_log || !dt_bias || !D || !Bm || !Cm || !y) return DFSSM_EINVAL;
+  if (B < 1 || H < 1 || P < 1 || N < 4 || G < 1 || H % G) return DFSSM_EINVAL;
+  if (N % 4 || N > 512) return DFSSM_EUNSUPPORTED;
+  if (!aligned(ssm_state, 16) || !aligned(Bm, 16) || !aligned(Cm, 16)) return DFSSM_EALIGN;
+  if (!device_ok()) return DFSSM_EDEVICE;
+  dfssm::SsmArgs a{};
+  a.state = ssm_state;
+  a.x = x;
+  a.ldx = H * P;
+  a.dt_raw = dt_raw;
+  a.lddt = H;
+  a.A_log = A_log;
+  a.dt_bias = dt_bias;
+  a.D = D;
+  a.Bm = Bm;
+  a.Cm = Cm;
+  a.ldbc = G * N;
+  a.y = y;
+  a.ldy = H * P;
+  a.z = nullptr;
+  a.B = B;
+  a.H = H;
+  a.P = P;
+  a.N = N;
+  a.G = G;
+  cudaError_t e = dfssm::launch_ssm(a, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? DFSSM_OK : cuda_fail(e);
+}
+
+int dfssm_layer_decode(const dfssm_layer_t* layers, int n_layers, const dfssm_dims_t* dims,
+                       float* hidden, float* const* conv_states, float* const* ssm_states, int B,
+                       void* workspace, size_t ws_bytes, void* stream) {
+  if (!layers || !dims || !hidden || !conv_states || !ssm_states) return DFSSM_EINVAL;
+  if (n_layers < 1 || B < 1) return DFSSM_EINVAL;
+  if (n_layers > DFSSM_MAX_LAYERS || B > DFSSM_MAX_BATCH) return DFSSM_EUNSUPPORTED;
+  const int Dm = dims->d_model, H = dims->nheads, P = dims->headdim, N = dims->d_state,
+            G = dims->ngroups;
+  if (Dm < 32 || Dm % 32 || H < 1 || P < 1 || N < 4 || G < 1 || H % G) return DFSSM_EINVAL;
+  const int E = H * P;
+  const int C = E + 2 * G * N;
+  const int d_ip = 2 * E + 2 * G * N + H;
+  if (E % 32 || N % 4 || N > 512 || Dm > 8192 || E > 8192 || 2 * G * N > 2048 || H > 1024)
+    return DFSSM_EUNSUPPORTED;
+  if (!aligned(hidden, 16)) return DFSSM_EALIGN;
+  for (int l = 0; l < n_layers; ++l) {
+    const dfssm_layer_t& Ly = layers[l];
+    int st = check_linear(&Ly.in_proj);
+    if (st) return st;
+    st = check_linear(&Ly.out_proj);
+    if (st) return st;
+    if (Ly.in_proj.d_out != d_ip || Ly.in_proj.d_in != Dm || Ly.out_proj.d_out != Dm ||
+        Ly.out_proj.d_in != E)
+      return DFSSM_EINVAL;
+    if (!Ly.conv_w || !Ly.conv_b || !Ly.A_log || !Ly.dt_bias || !Ly.D || !Ly.norm_w || !Ly.gnorm_w)
+      return DFSSM_EINVAL;
+    if (!conv_states[l] || !ssm_states[l]) return DFSSM_EINVAL;
+    if (!aligned(Ly.conv_w, 16) || !aligned(ssm_states[l], 16)) return DFSSM_EALIGN;
+  }
+  if (!workspace || !aligned(workspace, 256) || ws_bytes < layer_ws_bytes(B, Dm, E, C, d_ip))
+    return DFSSM_EWORKSPACE;
+  if (!device_ok()) return DFSSM_EDEVICE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  LayerWs w = carve_layer_ws(workspace, B, Dm, E, C, d_ip);
+  cudaError_t e = cudaSuccess;
+  for (int l = 0; l < n_layers && e == cudaSuccess; ++l) {
+    const dfssm_layer_t& Ly = layers[l];
+    // pre-norm + quantize + LoRA-down
+    dfssm::QuantArgs qa{};
+    qa.x = hidden;
+    qa.ldx = Dm;
+    qa.norm_w = Ly.norm_w;
+    qa.n = Dm;
+    qa.B = B;
+    qa.lora_b = Ly.in_proj.lora_b;
+    qa.rank = Ly.in_proj.rank;
+    qa.permute = true;
+    qa.out = w.qs;
+    e = dfssm::launch_quant(qa, s);
+    if (e != cudaSuccess) break;
+    // in_proj
+    dfssm::GemvArgs ga = gemv_args(&Ly.in_proj, B, w.qs);
+    ga.y = w.zxbcdt;
+    ga.ldy = d_ip;
+    e = dfssm::launch_gemv(ga, s);
+    if (e != cudaSuccess) break;
+    // conv over x|B|C
+    dfssm::ConvArgs ca{conv_states[l], Ly.conv_w, Ly.conv_b, w.zxbcdt + E, d_ip, w.xc, C, B, C};
+    e = dfssm::launch_conv(ca, s);
+    if (e != cudaSuccess) break;
+    // SSM + gate
+    dfssm::SsmArgs sa{};
+    sa.state = ssm_states[l];
+    sa.x = w.xc;
+    sa.ldx = C;
+    sa.dt_raw = w.zxbcdt + E + C;
+    sa.lddt = d_ip;
+    sa.A_log = Ly.A_log;
+    sa.dt_bias = Ly.dt_bias;
+    sa.D = Ly.D;
+    sa.Bm = w.xc + E;
+    sa.Cm = w.xc + E + G * N;
+    sa.ldbc = C;
+    sa.y = w.g;
+    sa.ldy = E;
+    sa.z = w.zxbcdt;
+    sa.ldz = d_ip;
+    sa.B = B;
+    sa.H = H;
+    sa.P = P;
+    sa.N = N;
+    sa.G = G;
+    e = dfssm::launch_ssm(sa, s);
+    if (e != cudaSuccess) break;
+    // gated norm + quantize + LoRA-down
+    qa.x = w.g;
+    qa.ldx = E;
+    qa.norm_w = Ly.gnorm_w;
+    qa.n = E;
+    qa.lora_b = Ly.out_proj.lora_b;
+    qa.rank = Ly.out_proj.rank;
+    e = dfssm::launch_quant(qa, s);
+    if (e != cudaSuccess) break;
+    // out_proj + residual
+    ga = gemv_args(&Ly.out_proj, B, w.qs);
+    ga.resid = hidden;
+    ga.ldr = Dm;
+    e = dfssm::launch_gemv(ga, s);
+  }
+  return e == cudaSuccess ? DFSSM_OK : cuda_fail(e);
+}
+
+int dfssm_lm_head(const int8_t* W, const float* s_row, int V, int d, const float* x, float* logits,
+                  int32_t* acc, void* workspace, size_t ws_bytes, void* stream) {
+  if (!W || !s_row || !x || !logits || V < 1 || d < 16 || d % 16) return DFSSM_EINVAL;
+  if (d > 8192) return DFSSM_EUNSUPPORTED;
+  if (!aligned(W, 16) || !aligned(x, 4)) return DFSSM_EALIGN;
+  if (!workspace || !aligned(workspace, 256) || ws_bytes < dfssm::quant_scratch_bytes(1, d))
+    return DFSSM_EWORKSPACE;
+  if (!device_ok()) return DFSSM_EDEVICE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  dfssm::QuantScratch qs = dfssm::carve_quant_scratch(workspace, 1, d);
+  dfssm::QuantArgs qa{};
+  qa.x = x;
+  qa.ldx = d;
+  qa.n = d;
+  qa.B = 1;
+  qa.rank = 0;
+  qa.permute = false;
+  qa.out = qs;
+  cudaError_t e = dfssm::launch_quant(qa, s);
+  if (e != cudaSuccess) return cuda_fail(e);
+  dfssm::Int8GemvArgs ia{W, s_row, V, d, qs, logits, acc};
+  e = dfssm::launch_int8_gemv(ia, s);
+  return e == cudaSuccess ? DFSSM_OK : cuda_fail(e);
+}
+
+}  // extern "C"

@@ -1,0 +1,117 @@
+// Internal device helpers shared by the libdfssm kernels (sm_100a only).
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "../../include/dfssm.h"
+
+#if defined(__CUDA_ARCH__) && (__CUDA_ARCH__ < 1000)
+#error "libdfssm is built for sm_100a only"
+#endif
+
+namespace dfssm {
+
+constexpr int kWarp = 32;
+
+// ---------------------------------------------------------------- programmatic dependent launch
+// A kernel launched with programmatic stream serialization may start before the previous kernel of the
+// stream has finished.  Everything it reads that an earlier kernel may write (activations, states,
+// workspace) and everything it writes must come after pdl_wait(); only immutable weights may be
+// fetched before it.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// ---------------------------------------------------------------- loads
+// Streaming 16-byte load of read-only data that is used once (weights): not allocated in L1.
+__device__ __forceinline__ uint4 ld_stream_u4(const void* p) {
+  uint4 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "l"(p));
+  return r;
+}
+__device__ __forceinline__ uint32_t ld_stream_u32(const void* p) {
+  uint32_t r;
+  asm volatile("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(r) : "l"(p));
+  return r;
+}
+__device__ __forceinline__ float4 ld_stream_f4(const void* p) {
+  float4 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(r.x), "=f"(r.y), "=f"(r.z), "=f"(r.w)
+               : "l"(p));
+  return r;
+}
+// 16-byte load of data that is read once and then overwritten by this thread (SSM state): no L1.
+__device__ __forceinline__ float4 ld_evict_first_f4(const void* p) {
+  float4 r;
+  asm volatile("ld.global.L1::no_allocate.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(r.x), "=f"(r.y), "=f"(r.z), "=f"(r.w)
+               : "l"(p));
+  return r;
+}
+__device__ __forceinline__ void st_f4(void* p, float4 v) {
+  asm volatile("st.global.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(v.x), "f"(v.y), "f"(v.z),
+               "f"(v.w)
+               : "memory");
+}
+
+// ---------------------------------------------------------------- integer dot products
+// d = c + sum_j a.u8[j] * b.s8[j]   (a unsigned bytes, b signed bytes)
+__device__ __forceinline__ int dp4a_us(uint32_t a, uint32_t b, int c) {
+  int d;
+  asm("dp4a.u32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+// d = c + sum_j a.s8[j] * b.s8[j]
+__device__ __forceinline__ int dp4a_ss(uint32_t a, uint32_t b, int c) {
+  int d;
+  asm("dp4a.s32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+
+// ---------------------------------------------------------------- exact-rounding float helpers
+// Products and sums that feed a quantizer must be single IEEE operations (never contracted to FMA).
+__device__ __forceinline__ float fmul(float a, float b) { return __fmul_rn(a, b); }
+__device__ __forceinline__ float fadd(float a, float b) { return __fadd_rn(a, b); }
+__device__ __forceinline__ double dmul(double a, double b) { return __dmul_rn(a, b); }
+__device__ __forceinline__ double dadd(double a, double b) { return __dadd_rn(a, b); }
+
+// SiLU evaluated in fp64 and rounded once: v / (1 + exp(-v)).
+__device__ __forceinline__ float silu_f64(float v) {
+  const double d = (double)v;
+  return __double2float_rn(__ddiv_rn(d, __dadd_rn(1.0, exp(-d))));
+}
+
+// Per-token quantization code of v for scale s0 > 0: clamp(rint(fl32(v / s0)), -127, 127).
+__device__ __forceinline__ int quant_code(float v, float s0) {
+  float r = rintf(__fdiv_rn(v, s0));
+  r = fminf(fmaxf(r, -127.0f), 127.0f);
+  return (int)r;
+}
+
+// Position of natural-order activation index i inside the dp4a-friendly permuted layout: within each
+// 32-element block, word k (k = 0..7) holds elements k, k+8, k+16, k+24 in its four bytes.  With that
+// layout, (w & (0x01010101 << k)) selects exactly the sign bits that pair with word k.
+__device__ __forceinline__ int perm_index(int i) {
+  const int j = i & 31;
+  return (i & ~31) + ((j & 7) << 2) + (j >> 3);
+}
+
+// ---------------------------------------------------------------- block reductions
+template <typename T>
+__device__ __forceinline__ T warp_sum(T v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+}  // namespace dfssm

@@ -1,0 +1,101 @@
+// Internal host-side interfaces between the C-ABI layer (api.cu) and the kernel files.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace dfssm {
+
+// Scratch carved from the caller's workspace for one quantize -> linear hand-off.
+struct QuantScratch {
+  int8_t* q;     // [B][n] codes (dp4a-permuted or natural order)
+  float* s;      // [B] per-token scale
+  int32_t* sumq; // [B] sum of the codes of each token
+  int32_t* t;    // [B][16] LoRA-down accumulators
+};
+size_t quant_scratch_bytes(int B, int n);
+QuantScratch carve_quant_scratch(void* base, int B, int n);
+
+struct QuantArgs {
+  const float* x;
+  int ldx;                 // row stride of x (elements)
+  const float* norm_w;     // non-NULL: RMSNorm(eps 1e-5) folded into the scale
+  int n;                   // row length
+  int B;
+  const int8_t* lora_b;    // [rank][n] or NULL
+  int rank;
+  bool permute;            // dp4a-permuted layout (scaffold GEMV) or natural (int8 GEMV)
+  QuantScratch out;
+  int8_t* dbg_xq;          // optional taps
+  float* dbg_s;
+  int32_t* dbg_t;
+};
+cudaError_t launch_quant(const QuantArgs& a, cudaStream_t st);
+
+struct GemvArgs {
+  const uint32_t* bits;
+  const float* w_scale;
+  const int8_t* lora_a;
+  const float* lora_a_scale;
+  const float* lora_b_scale;
+  int rank, d_out, d_in, B;
+  QuantScratch in;
+  float* y;
+  int ldy;
+  float* resid;            // non-NULL: resid = fl32(resid + y) instead of writing y
+  int ldr;
+  int32_t* dbg_acc;        // [B][d_out] or NULL
+};
+cudaError_t launch_gemv(const GemvArgs& a, cudaStream_t st);
+
+struct ConvArgs {
+  float* state;            // [B][C][3]
+  const float* w;          // [C][4]
+  const float* bias;       // [C]
+  const float* x_in;
+  int ldx;
+  float* x_out;
+  int ldo;
+  int B, C;
+};
+cudaError_t launch_conv(const ConvArgs& a, cudaStream_t st);
+
+struct SsmArgs {
+  float* state;            // [B][H][P][N]
+  const float* x;          // [B][ldx], head-major H*P
+  int ldx;
+  const float* dt_raw;     // [B][lddt]
+  int lddt;
+  const float* A_log;
+  const float* dt_bias;
+  const float* D;
+  const float* Bm;         // [B][ldbc] rows, group g at offset g*N
+  const float* Cm;
+  int ldbc;
+  float* y;                // [B][ldy]
+  int ldy;
+  const float* z;          // optional gate input [B][ldz]: y is replaced by fl32(y * SiLU(z))
+  int ldz;
+  int B, H, P, N, G;
+};
+cudaError_t launch_ssm(const SsmArgs& a, cudaStream_t st);
+
+struct Int8GemvArgs {
+  const int8_t* W;
+  const float* s_row;
+  int V, d;
+  QuantScratch in;          // natural-order codes of one token
+  float* logits;
+  int32_t* acc;
+};
+cudaError_t launch_int8_gemv(const Int8GemvArgs& a, cudaStream_t st);
+
+int num_sms();
+
+}  // namespace dfssm
+
+namespace dfssm {
+// Prefill (tcgen05) workspace requirement for M tokens of a d_in -> d_out linear.
+size_t prefill_workspace_bytes(int M, int d_in, int d_out);
+}  // namespace dfssm

@@ -1,0 +1,272 @@
+"""Thin ctypes binding of libdfssm (include/dfssm.h): argument marshalling only.
+
+Every compute step runs in the CUDA library; this module only turns torch tensors (device memory,
+allocated by the caller) into pointers, picks the current torch stream and raises on a negative status.
+There is no fallback: if the library or a CUDA device is missing, the calls raise.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+
+import numpy as np
+import torch
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libdfssm.so")
+
+OP_LINEAR_DECODE = 1
+OP_LINEAR_PREFILL = 2
+OP_LAYER_DECODE = 3
+OP_LM_HEAD = 4
+MAX_RANK = 16
+MAX_BATCH = 16
+MAX_LAYERS = 64
+
+STATUS = {0: "DFSSM_OK", -1: "DFSSM_EINVAL", -2: "DFSSM_EALIGN", -3: "DFSSM_EUNSUPPORTED",
+          -4: "DFSSM_ECUDA", -5: "DFSSM_ETIMEOUT", -6: "DFSSM_EDEVICE", -7: "DFSSM_EWORKSPACE"}
+
+
+class DfssmError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        msg = f"{fn} returned {STATUS.get(status, status)}"
+        if status == -4:
+            msg += f" ({lib().dfssm_last_cuda_error().decode()})"
+        super().__init__(msg)
+        self.status = status
+
+
+class LinearT(C.Structure):
+    _fields_ = [("d_out", C.c_int32), ("d_in", C.c_int32), ("rank", C.c_int32),
+                ("bits", C.c_void_p), ("w_scale", C.c_void_p), ("lora_b", C.c_void_p),
+                ("lora_b_scale", C.c_void_p), ("lora_a", C.c_void_p), ("lora_a_scale", C.c_void_p)]
+
+
+class DebugT(C.Structure):
+    _fields_ = [("acc", C.c_void_p), ("lora_t", C.c_void_p), ("xq", C.c_void_p),
+                ("xscale", C.c_void_p)]
+
+
+class DimsT(C.Structure):
+    _fields_ = [("d_model", C.c_int32), ("nheads", C.c_int32), ("headdim", C.c_int32),
+                ("d_state", C.c_int32), ("ngroups", C.c_int32)]
+
+
+class LayerT(C.Structure):
+    _fields_ = [("in_proj", LinearT), ("out_proj", LinearT), ("conv_w", C.c_void_p),
+                ("conv_b", C.c_void_p), ("A_log", C.c_void_p), ("dt_bias", C.c_void_p),
+                ("D", C.c_void_p), ("norm_w", C.c_void_p), ("gnorm_w", C.c_void_p)]
+
+
+_lib = None
+
+# name -> (restype, argtypes); every function that include/dfssm.h declares.
+_P, _I, _Z = C.c_void_p, C.c_int, C.c_size_t
+SIGNATURES = {
+    "dfssm_workspace_size": (_Z, [_I, _I, _I, _I]),
+    "dfssm_linear_decode": (_I, [_P, _P, _I, _P, _P, _Z, _P, _P]),
+    "dfssm_linear_prefill": (_I, [_P, _P, _I, _P, _P, _Z, _P, _P]),
+    "dfssm_conv_step": (_I, [_P, _P, _P, _P, _P, _I, _I, _P]),
+    "dfssm_ssm_step": (_I, [_P] * 9 + [_I] * 5 + [_P]),
+    "dfssm_layer_decode": (_I, [_P, _I, _P, _P, _P, _P, _I, _P, _Z, _P]),
+    "dfssm_lm_head": (_I, [_P, _P, _I, _I, _P, _P, _P, _P, _Z, _P]),
+    "dfssm_pack_signs": (_I, [_P, _I, _I, _P]),
+    "dfssm_status_string": (C.c_char_p, [_I]),
+    "dfssm_last_cuda_error": (C.c_char_p, []),
+    "dfssm_abi_version": (_I, []),
+}
+
+
+def lib():
+    """Load libdfssm.so (built in-tree by bit_quantized_mamba_b200.build); raise if it is missing."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"libdfssm.so not built ({LIB_PATH}); run __graft_entry__.build()")
+        L = C.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            f = getattr(L, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = L
+    return _lib
+
+
+def _check(fn: str, status: int):
+    if status != 0:
+        raise DfssmError(fn, status)
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("expected a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError("expected a contiguous tensor")
+    return t.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def workspace_size(op: int, a: int, b: int, c: int) -> int:
+    return int(lib().dfssm_workspace_size(op, a, b, c))
+
+
+def workspace(nbytes: int, device="cuda") -> torch.Tensor:
+    """Caller-owned scratch (torch allocations are 512-byte aligned)."""
+    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+
+
+class Linear:
+    """Device copy of one scaffold+LoRA linear (see dfssm_linear_t)."""
+
+    def __init__(self, bits, w_scale, lora_b, lora_b_scale, lora_a, lora_a_scale):
+        self.bits, self.w_scale = bits, w_scale
+        self.lora_b, self.lora_b_scale = lora_b, lora_b_scale
+        self.lora_a, self.lora_a_scale = lora_a, lora_a_scale
+        self.d_out = bits.shape[0]
+        self.d_in = bits.shape[1] * 32
+        self.rank = lora_b.shape[0] if lora_b is not None else 0
+        self._c = LinearT(self.d_out, self.d_in, self.rank, _ptr(bits), _ptr(w_scale),
+                          _ptr(lora_b) if self.rank else None,
+                          _ptr(lora_b_scale) if self.rank else None,
+                          _ptr(lora_a) if self.rank else None, _ptr(lora_a_scale) if self.rank else None)
+
+    @classmethod
+    def from_host(cls, d: dict, device="cuda"):
+        t = {k: torch.from_numpy(np.ascontiguousarray(v)).to(device) for k, v in d.items()
+             if k != "bits"}
+        # the sign words travel as int32 (same bytes); only their address reaches the library
+        bits = torch.from_numpy(np.ascontiguousarray(d["bits"]).view(np.int32)).to(device)
+        return cls(bits, t["w_scale"], t["lora_b"], t["lora_b_scale"], t["lora_a"], t["lora_a_scale"])
+
+    def cstruct(self) -> LinearT:
+        return self._c
+
+
+def linear_decode(lin: Linear, x: torch.Tensor, y: torch.Tensor | None = None, ws=None,
+                  debug: dict | None = None, stream=None) -> torch.Tensor:
+    B = x.shape[0]
+    if y is None:
+        y = torch.empty((B, lin.d_out), dtype=torch.float32, device=x.device)
+    if ws is None:
+        ws = workspace(workspace_size(OP_LINEAR_DECODE, B, lin.d_in, lin.d_out), x.device)
+    dbg = None
+    if debug is not None:
+        dbg = DebugT(*(_ptr(debug.get(k)) for k in ("acc", "lora_t", "xq", "xscale")))
+    _check("dfssm_linear_decode", lib().dfssm_linear_decode(
+        C.byref(lin.cstruct()), _ptr(x), B, _ptr(y), _ptr(ws), ws.numel(),
+        C.byref(dbg) if dbg is not None else None, _stream(stream)))
+    return y
+
+
+def linear_prefill(lin: Linear, x: torch.Tensor, y: torch.Tensor | None = None, ws=None,
+                   debug: dict | None = None, stream=None) -> torch.Tensor:
+    M = x.shape[0]
+    if y is None:
+        y = torch.empty((M, lin.d_out), dtype=torch.float32, device=x.device)
+    if ws is None:
+        ws = workspace(workspace_size(OP_LINEAR_PREFILL, M, lin.d_in, lin.d_out), x.device)
+    dbg = None
+    if debug is not None:
+        dbg = DebugT(*(_ptr(debug.get(k)) for k in ("acc", "lora_t", "xq", "xscale")))
+    _check("dfssm_linear_prefill", lib().dfssm_linear_prefill(
+        C.byref(lin.cstruct()), _ptr(x), M, _ptr(y), _ptr(ws), ws.numel(),
+        C.byref(dbg) if dbg is not None else None, _stream(stream)))
+    return y
+
+
+def conv_step(conv_state, w, b, x_in, x_out=None, stream=None):
+    B, Cn = x_in.shape
+    if x_out is None:
+        x_out = torch.empty_like(x_in)
+    _check("dfssm_conv_step", lib().dfssm_conv_step(_ptr(conv_state), _ptr(w), _ptr(b), _ptr(x_in),
+                                                    _ptr(x_out), B, Cn, _stream(stream)))
+    return x_out
+
+
+def ssm_step(ssm_state, x, dt_raw, A_log, dt_bias, D, Bm, Cm, y=None, stream=None):
+    B, H, P, N = ssm_state.shape
+    G = Bm.numel() // (B * N)
+    if y is None:
+        y = torch.empty((B, H * P), dtype=torch.float32, device=x.device)
+    _check("dfssm_ssm_step", lib().dfssm_ssm_step(
+        _ptr(ssm_state), _ptr(x), _ptr(dt_raw), _ptr(A_log), _ptr(dt_bias), _ptr(D), _ptr(Bm),
+        _ptr(Cm), _ptr(y), B, H, P, N, G, _stream(stream)))
+    return y
+
+
+class Layer:
+    """Device copy of one DF-SSM Mamba-2 layer (see dfssm_layer_t)."""
+
+    VEC = ("conv_w", "conv_b", "A_log", "dt_bias", "D", "norm_w", "gnorm_w")
+
+    def __init__(self, in_proj: Linear, out_proj: Linear, **vec):
+        self.in_proj, self.out_proj = in_proj, out_proj
+        for k in self.VEC:
+            setattr(self, k, vec[k])
+        self._c = LayerT(in_proj.cstruct(), out_proj.cstruct(), *(_ptr(vec[k]) for k in self.VEC))
+
+    @classmethod
+    def from_host(cls, d: dict, device="cuda"):
+        vec = {k: torch.from_numpy(np.ascontiguousarray(d[k])).to(device) for k in cls.VEC}
+        return cls(Linear.from_host(d["in_proj"], device), Linear.from_host(d["out_proj"], device),
+                   **vec)
+
+    def cstruct(self) -> LayerT:
+        return self._c
+
+
+class LayerStack:
+    """Layers plus their per-layer conv/SSM state tensors, marshalled once for repeated decode calls."""
+
+    def __init__(self, layers: list[Layer], dims: dict, conv_states: list, ssm_states: list):
+        n = len(layers)
+        self.layers, self.conv_states, self.ssm_states = layers, conv_states, ssm_states
+        self.dims = DimsT(dims["d_model"], dims["nheads"], dims["headdim"], dims["d_state"],
+                          dims["ngroups"])
+        self.d_model = dims["d_model"]
+        self.d_inner = dims["nheads"] * dims["headdim"]
+        self._layers = (LayerT * n)(*(L.cstruct() for L in layers))
+        self._conv = (C.c_void_p * n)(*(_ptr(t) for t in conv_states))
+        self._ssm = (C.c_void_p * n)(*(_ptr(t) for t in ssm_states))
+        self.n = n
+
+
+def layer_decode(stack: LayerStack, hidden: torch.Tensor, ws=None, stream=None) -> torch.Tensor:
+    """One decode step of every layer of the stack; hidden [B][d_model] is updated in place."""
+    B = hidden.shape[0]
+    if ws is None:
+        ws = workspace(workspace_size(OP_LAYER_DECODE, B, stack.d_model, stack.d_inner),
+                       hidden.device)
+    _check("dfssm_layer_decode", lib().dfssm_layer_decode(
+        stack._layers, stack.n, C.byref(stack.dims), _ptr(hidden), stack._conv, stack._ssm, B,
+        _ptr(ws), ws.numel(), _stream(stream)))
+    return hidden
+
+
+def lm_head(W, s_row, x, logits=None, acc=None, ws=None, stream=None):
+    V, d = W.shape
+    if logits is None:
+        logits = torch.empty(V, dtype=torch.float32, device=x.device)
+    if ws is None:
+        ws = workspace(workspace_size(OP_LM_HEAD, 1, d, V), x.device)
+    _check("dfssm_lm_head", lib().dfssm_lm_head(_ptr(W), _ptr(s_row), V, d, _ptr(x), _ptr(logits),
+                                                _ptr(acc), _ptr(ws), ws.numel(), _stream(stream)))
+    return logits
+
+
+def pack_signs(signs: np.ndarray) -> np.ndarray:
+    """Host: +-1 int8 [d_out][d_in] -> LSB-first uint32 words [d_out][d_in/32]."""
+    signs = np.ascontiguousarray(signs, dtype=np.int8)
+    d_out, d_in = signs.shape
+    bits = np.zeros((d_out, d_in // 32), np.uint32)
+    _check("dfssm_pack_signs", lib().dfssm_pack_signs(signs.ctypes.data, d_out, d_in,
+                                                      bits.ctypes.data))
+    return bits

@@ -1,0 +1,194 @@
+/*
+ * dfssm.h — C ABI of libdfssm, the B200 (sm_100a) implementation of the DF-SSM decode/prefill hot path.
+ *
+ * DF-SSM ("Density Field State Space Models: 1-Bit Distillation, Efficient Inference, and Knowledge
+ * Organization in Mamba-2", arXiv 2606.10932) compresses Mamba-2 so that in_proj and out_proj are a
+ * frozen 1-bit sign scaffold with per-output-channel scales, applied to per-token int8 activations with
+ * int32 accumulation, plus an int8 rank-16 LoRA correction (gist.science technical summary, §2.B "Frozen
+ * Scaffold with LoRA Correction" and §2.C "Optimized Inference Pipeline").  The stateful ops are the
+ * width-4 causal-conv shift register and the per-head SSM recurrence (same summary, §2.C).  The Mamba-2
+ * block equations are those of the cited Mamba-2/SSD layer (mlsanity citation map, "Builds on").
+ *
+ * Conventions for every entry point:
+ *   - Pointers documented as "device" must point to memory of the current CUDA device.  The caller owns
+ *     every buffer; the library allocates no device memory.  Scratch comes from a caller-provided
+ *     workspace of at least dfssm_workspace_size(...) bytes, 256-byte aligned.
+ *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy default stream).  Inputs
+ *     must not be modified, and outputs not read, until the stream reaches the call.  Weights and
+ *     parameters must be fully written before the call is enqueued (kernels may read them before they
+ *     wait on the preceding kernel of the stream).
+ *   - Arguments are validated before anything is launched; on a negative status nothing was enqueued.
+ *   - Calls that share a workspace must not overlap on the GPU.  The library keeps no global state
+ *     beyond cached device attributes, so calls on different streams with different workspaces may run
+ *     concurrently.
+ *   - fp32 values that feed an int8 quantizer are computed as single correctly rounded fp32 operations,
+ *     with sums and transcendental functions evaluated in fp64 and rounded once, so that quantization
+ *     codes are reproducible by a plain CPU evaluation of the same definitions.
+ */
+#ifndef DFSSM_H_
+#define DFSSM_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define DFSSM_ABI_VERSION 1
+#define DFSSM_MAX_RANK 16
+#define DFSSM_MAX_BATCH 16
+#define DFSSM_MAX_LAYERS 64
+
+typedef enum {
+  DFSSM_OK = 0,
+  DFSSM_EINVAL = -1,       /* bad size, NULL pointer or inconsistent arguments                      */
+  DFSSM_EALIGN = -2,       /* a pointer is not aligned as documented                                */
+  DFSSM_EUNSUPPORTED = -3, /* valid, but outside what this build implements (e.g. B > 16)           */
+  DFSSM_ECUDA = -4,        /* a CUDA runtime call failed; see dfssm_last_cuda_error()                */
+  DFSSM_ETIMEOUT = -5,     /* a device-side wait ran out of its iteration budget                    */
+  DFSSM_EDEVICE = -6,      /* no usable sm_100 device                                               */
+  DFSSM_EWORKSPACE = -7    /* workspace NULL, too small or misaligned                               */
+} dfssm_status;
+
+/*
+ * One DF-SSM linear: y = scaffold(x) + LoRA(x) (technical summary §2.B–C).
+ *   bits          device u32 [d_out][d_in/32], row-major.  Bit j of word w of row o is the sign of weight
+ *                 (o, 32w+j): set = +1, clear = -1 (least significant bit first).  16-byte aligned.
+ *   w_scale       device f32 [d_out]   per-output-channel scaffold scale sW
+ *   lora_b        device i8  [rank][d_in]   W_B, row-major; 4-byte aligned
+ *   lora_b_scale  device f32 [rank]    per-row scale of W_B
+ *   lora_a        device i8  [d_out][rank]  W_A, row-major
+ *   lora_a_scale  device f32 [d_out]   per-row scale of W_A
+ * Constraints: d_in % 32 == 0, d_in <= 8192, d_out >= 1, 0 <= rank <= 16.  rank == 0 means no LoRA
+ * (lora_* may then be NULL).
+ * Computes, for each token b with (q, s) its per-token int8 quantization:
+ *   acc[o] = sum_i sign(o,i) q[i]  (int32),   t[r] = sum_i W_B[r,i] q[i]  (int32)
+ *   tf[r]  = fl32(t[r] sB[r] s),  y[o] = fl32(acc[o] s sW[o] + sA[o] sum_r W_A[o,r] tf[r])   (fp64 inside)
+ */
+typedef struct {
+  int32_t d_out, d_in, rank;
+  const uint32_t* bits;
+  const float* w_scale;
+  const int8_t* lora_b;
+  const float* lora_b_scale;
+  const int8_t* lora_a;
+  const float* lora_a_scale;
+} dfssm_linear_t;
+
+/* Optional device taps of the integer intermediates (any member may be NULL). */
+typedef struct {
+  int32_t* acc;   /* [B][d_out]  scaffold accumulators                                    */
+  int32_t* lora_t;/* [B][rank]   LoRA-down accumulators                                   */
+  int8_t* xq;     /* [B][d_in]   quantized activations, natural order                     */
+  float* xscale;  /* [B]         per-token scale s                                         */
+} dfssm_debug_t;
+
+/* Workspace sizing.  `op` selects the entry point; the remaining arguments are that entry point's
+ * sizes as listed; unused ones are ignored.  Returns 0 for invalid sizes. */
+enum {
+  DFSSM_OP_LINEAR_DECODE = 1,  /* a = B,  b = d_in,  c = d_out                         */
+  DFSSM_OP_LINEAR_PREFILL = 2, /* a = M,  b = d_in,  c = d_out                         */
+  DFSSM_OP_LAYER_DECODE = 3,   /* a = B,  b = d_model, c = d_inner (nheads*headdim)     */
+  DFSSM_OP_LM_HEAD = 4         /* a = 1,  b = d,     c = V                             */
+};
+size_t dfssm_workspace_size(int op, int a, int b, int c);
+
+/*
+ * Batch-B decode of one linear (scaffold GEMV + fused int8 LoRA), technical summary §2.B–C.
+ *   x   device f32 [B][d_in] (16-byte aligned),  y device f32 [B][d_out]
+ *   1 <= B <= 16.  dbg may be NULL.  workspace: dfssm_workspace_size(DFSSM_OP_LINEAR_DECODE, B, d_in, d_out).
+ */
+int dfssm_linear_decode(const dfssm_linear_t* lin, const float* x, int B, float* y, void* workspace,
+                        size_t ws_bytes, const dfssm_debug_t* dbg, void* stream);
+
+/*
+ * M-token prefill of one linear on int8 tcgen05 tensor cores (technical summary §2.C: the scaffold
+ * matmul on INT8 tensor cores).  Same math as dfssm_linear_decode, per row of x.
+ *   x device f32 [M][d_in], y device f32 [M][d_out], M >= 1.  d_in % 128 == 0 required.
+ *   Integer results (dbg->acc, dbg->lora_t, dbg->xq, dbg->xscale) are exact; y is fp32 to within
+ *   1e-6 relative of the fp64 epilogue (the prefill epilogue uses fp32 fused multiply-add).
+ */
+int dfssm_linear_prefill(const dfssm_linear_t* lin, const float* x, int M, float* y, void* workspace,
+                         size_t ws_bytes, const dfssm_debug_t* dbg, void* stream);
+
+/*
+ * Width-4 stateful shift-register causal convolution, one decode step, with SiLU (technical summary §2.C
+ * "stateful shift register (convolution)").
+ *   conv_state device f32 [B][C][3]  (the last three inputs, oldest first; updated in place)
+ *   w device f32 [C][4] (w[c][3] multiplies the current input), b device f32 [C]
+ *   x_in device f32 [B][C], x_out device f32 [B][C]   (x_out = SiLU(b + sum_k w[c,k] window_k))
+ */
+int dfssm_conv_step(float* conv_state, const float* w, const float* b, const float* x_in, float* x_out,
+                    int B, int C, void* stream);
+
+/*
+ * Mamba-2 SSM state update and readout for one decode step (technical summary §2.C "SSM recurrence").
+ *   ssm_state device f32 [B][H][P][N] (updated in place), x device f32 [B][H*P], dt_raw device f32 [B][H],
+ *   A_log, dt_bias, D device f32 [H], Bm, Cm device f32 [B][G][N], y device f32 [B][H*P].
+ *   dt = softplus(dt_raw + dt_bias); dA = exp(dt * -exp(A_log));
+ *   S = dA S + (dt x) B;  y = S . C + D x.      Requires H % G == 0, N % 4 == 0, N <= 512.
+ */
+int dfssm_ssm_step(float* ssm_state, const float* x, const float* dt_raw, const float* A_log,
+                   const float* dt_bias, const float* D, const float* Bm, const float* Cm, float* y,
+                   int B, int H, int P, int N, int G, void* stream);
+
+/* Shape of a DF-SSM Mamba-2 layer.  d_inner = nheads*headdim; conv channels = d_inner + 2*ngroups*d_state;
+ * in_proj rows = 2*d_inner + 2*ngroups*d_state + nheads, ordered z | x | B | C | dt. */
+typedef struct {
+  int32_t d_model, nheads, headdim, d_state, ngroups;
+} dfssm_dims_t;
+
+/* Parameters of one layer (all device pointers). */
+typedef struct {
+  dfssm_linear_t in_proj;   /* d_out = 2*d_inner + 2*ngroups*d_state + nheads, d_in = d_model */
+  dfssm_linear_t out_proj;  /* d_out = d_model, d_in = d_inner                               */
+  const float* conv_w;      /* [conv channels][4] */
+  const float* conv_b;      /* [conv channels]    */
+  const float* A_log;       /* [nheads] */
+  const float* dt_bias;     /* [nheads] */
+  const float* D;           /* [nheads] */
+  const float* norm_w;      /* [d_model]  pre-mixer RMSNorm weight, eps 1e-5 */
+  const float* gnorm_w;     /* [d_inner]  gated RMSNorm weight, eps 1e-5    */
+} dfssm_layer_t;
+
+/*
+ * One decode step (one token per sequence) through n_layers DF-SSM Mamba-2 layers.
+ *   layers       HOST array [n_layers] (read during the call only)
+ *   hidden       device f32 [B][d_model]; the residual stream, updated in place
+ *   conv_states  HOST array [n_layers] of device f32 [B][conv channels][3]
+ *   ssm_states   HOST array [n_layers] of device f32 [B][nheads][headdim][d_state]
+ * Per layer: (q,s) = quant(RMSNorm(h)); zxbcdt = in_proj; x|B|C = SiLU(conv(xBC)); y = SSM(x, dt, B, C);
+ * g = y*SiLU(z); (q',s') = quant(RMSNorm(g)); h += out_proj.   1 <= B <= 16, n_layers <= 64.
+ * workspace: dfssm_workspace_size(DFSSM_OP_LAYER_DECODE, B, d_model, d_inner).
+ */
+int dfssm_layer_decode(const dfssm_layer_t* layers, int n_layers, const dfssm_dims_t* dims,
+                       float* hidden, float* const* conv_states, float* const* ssm_states, int B,
+                       void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * Int8 LM head on one token (technical summary §2.B: int8 LM head with per-row scaling).
+ *   W device i8 [V][d] (16-byte aligned, d % 16 == 0), s_row device f32 [V], x device f32 [d],
+ *   logits device f32 [V].   logits[v] = fl32(acc[v] s s_row[v]), acc[v] = sum_i W[v,i] q[i].
+ *   acc (device i32 [V]) may be NULL.  workspace: dfssm_workspace_size(DFSSM_OP_LM_HEAD, 1, d, V).
+ */
+int dfssm_lm_head(const int8_t* W, const float* s_row, int V, int d, const float* x, float* logits,
+                  int32_t* acc, void* workspace, size_t ws_bytes, void* stream);
+
+/* Host helper: pack a +-1 int8 matrix [d_out][d_in] (row-major, host) into the bit layout above
+ * (host u32 [d_out][d_in/32]).  Any value > 0 maps to a set bit. */
+int dfssm_pack_signs(const int8_t* signs, int d_out, int d_in, uint32_t* bits);
+
+/* Text for a status code (static storage). */
+const char* dfssm_status_string(int status);
+
+/* The last CUDA error string recorded by a DFSSM_ECUDA return on this thread (static storage). */
+const char* dfssm_last_cuda_error(void);
+
+/* DFSSM_ABI_VERSION of the loaded library. */
+int dfssm_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* DFSSM_H_ */

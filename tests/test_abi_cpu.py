@@ -1,0 +1,86 @@
+"""Host-side checks of the C ABI (no GPU): the library builds, loads, exports every function that
+include/dfssm.h declares, and validates arguments before touching a device."""
+import ctypes as C
+import os
+import re
+
+import numpy as np
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "dfssm.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(dfssm_[a-z0-9_]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    from bit_quantized_mamba_b200 import build, dfssm
+    build.build()
+    return dfssm.lib()
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ("dfssm_linear_decode", "dfssm_linear_prefill", "dfssm_conv_step",
+                     "dfssm_ssm_step", "dfssm_layer_decode"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(L):
+    from bit_quantized_mamba_b200 import dfssm
+    names = declared_functions()
+    for n in names:
+        assert hasattr(L, n), f"{n} declared in dfssm.h but not exported"
+    assert set(names) == set(dfssm.SIGNATURES), "binding and header disagree"
+    assert L.dfssm_abi_version() == 1
+
+
+def test_status_strings(L):
+    assert L.dfssm_status_string(0) == b"ok"
+    assert L.dfssm_status_string(-7).startswith(b"workspace")
+
+
+def test_workspace_sizes(L):
+    from bit_quantized_mamba_b200 import dfssm
+    assert dfssm.workspace_size(dfssm.OP_LINEAR_DECODE, 1, 2048, 8512) >= 2048 + 16 * 16 * 4
+    assert dfssm.workspace_size(dfssm.OP_LINEAR_DECODE, 17, 2048, 8512) == 0
+    assert dfssm.workspace_size(dfssm.OP_LINEAR_DECODE, 1, 100, 8512) == 0
+    assert dfssm.workspace_size(dfssm.OP_LAYER_DECODE, 1, 2048, 4096) > 8512 * 4
+    assert dfssm.workspace_size(dfssm.OP_LM_HEAD, 1, 2048, 50288) >= 2048
+
+
+def test_argument_validation_precedes_device_use(L):
+    """Invalid arguments are rejected on the host (these calls would fault if they reached a device)."""
+    from bit_quantized_mamba_b200 import dfssm
+    lin = dfssm.LinearT(512, 100, 16, 16, 16, 16, 16, 16, 16)  # d_in not a multiple of 32
+    assert L.dfssm_linear_decode(C.byref(lin), 16, 1, 16, 256, 1 << 20, None, None) == -1
+    lin = dfssm.LinearT(512, 256, 17, 16, 16, 16, 16, 16, 16)  # rank > 16
+    assert L.dfssm_linear_decode(C.byref(lin), 16, 1, 16, 256, 1 << 20, None, None) == -1
+    lin = dfssm.LinearT(512, 256, 16, 8, 16, 16, 16, 16, 16)   # bits misaligned
+    assert L.dfssm_linear_decode(C.byref(lin), 16, 1, 16, 256, 1 << 20, None, None) == -2
+    lin = dfssm.LinearT(512, 256, 16, 16, 16, 16, 16, 16, 16)
+    assert L.dfssm_linear_decode(C.byref(lin), 16, 17, 16, 256, 1 << 20, None, None) == -3
+    assert L.dfssm_linear_decode(C.byref(lin), 16, 1, 16, None, 1 << 20, None, None) == -7
+    assert L.dfssm_linear_decode(C.byref(lin), 16, 1, 16, 256, 10, None, None) == -7
+    assert L.dfssm_linear_decode(None, 16, 1, 16, 256, 1 << 20, None, None) == -1
+    assert L.dfssm_ssm_step(16, 16, 16, 16, 16, 16, 16, 16, 16, 1, 3, 4, 8, 2, None) == -1  # H % G
+    assert L.dfssm_ssm_step(16, 16, 16, 16, 16, 16, 16, 16, 16, 1, 4, 4, 6, 1, None) == -3  # N % 4
+    assert L.dfssm_conv_step(None, 16, 16, 16, 16, 1, 8, None) == -1
+    assert L.dfssm_lm_head(16, 16, 10, 24, 16, 16, None, 256, 1 << 20, None) == -1  # d % 16
+
+
+def test_pack_signs_matches_oracle_bit_layout(L):
+    """The host packer writes the documented layout (checked against the oracle's independent unpack)."""
+    import oracle
+    from bit_quantized_mamba_b200 import dfssm
+    g = np.random.default_rng(3)
+    signs = g.choice(np.array([-1, 1], np.int8), size=(7, 96))
+    bits = dfssm.pack_signs(signs)
+    for o in range(7):
+        for i in range(96):
+            assert oracle.sign(bits, 96, o, i) == signs[o, i]

@@ -1,0 +1,242 @@
+"""Parity of the CUDA path (through the C ABI) with the CPU oracle, on the same seeded inputs.
+
+Bar: integer intermediates (scaffold accumulators, LoRA-down accumulators, int8 codes) bit-exact; fp32
+outputs and states within max|d| <= 1e-3 * (1 + |ref|).  The library evaluates every fp32 value that
+feeds a quantizer exactly as the oracle defines it, so the fp32 results are also expected to be
+bit-identical except for rare last-bit differences of fp64 reductions; the tests report that count.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from bit_quantized_mamba_b200 import inputs
+
+pytestmark = pytest.mark.gpu
+
+RTOL = 1e-3
+
+
+def assert_tol(gpu, ref, what):
+    gpu = np.asarray(gpu, np.float64)
+    ref = np.asarray(ref, np.float64)
+    assert gpu.shape == ref.shape, what
+    bad = np.abs(gpu - ref) > RTOL * (1 + np.abs(ref))
+    assert not bad.any(), (f"{what}: {bad.sum()} of {bad.size} outside tolerance; max |d| = "
+                           f"{np.abs(gpu - ref).max():.3e}")
+    return int((gpu != ref).sum())
+
+
+@pytest.fixture(scope="module")
+def dev():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from bit_quantized_mamba_b200 import build, dfssm
+    build.build()
+    dfssm.lib()
+    return torch.device("cuda:0")
+
+
+def to_dev(a, dev):
+    return torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+
+
+def run_linear(lin_host, x, dev):
+    from bit_quantized_mamba_b200 import dfssm
+    L = dfssm.Linear.from_host(lin_host, dev)
+    B = x.shape[0]
+    dbg = dict(acc=torch.zeros((B, L.d_out), dtype=torch.int32, device=dev),
+               lora_t=torch.zeros((B, max(L.rank, 1)), dtype=torch.int32, device=dev),
+               xq=torch.zeros((B, L.d_in), dtype=torch.int8, device=dev),
+               xscale=torch.zeros(B, dtype=torch.float32, device=dev))
+    y = dfssm.linear_decode(L, to_dev(x, dev), debug=dbg)
+    torch.cuda.synchronize()
+    out = {k: v.cpu().numpy() for k, v in dbg.items()}
+    out["lora_t"] = out["lora_t"][:, :L.rank]
+    out["y"] = y.cpu().numpy()
+    return out
+
+
+def compare_linear(g, r, what):
+    assert np.array_equal(g["xq"], r["xq"]), f"{what}: int8 codes differ"
+    assert np.array_equal(g["xscale"], r["xscale"]), f"{what}: scales differ"
+    assert np.array_equal(g["lora_t"], r["t"]), f"{what}: LoRA-down accumulators differ"
+    assert np.array_equal(g["acc"], r["acc"]), f"{what}: scaffold accumulators differ"
+    return assert_tol(g["y"], r["y"], what)
+
+
+def test_linear_tiny(dev):
+    d = inputs.tiny_linear(0)
+    g = run_linear(d["linear"], d["x"], dev)
+    r = oracle.linear_decode(oracle.Linear.from_dict(d["linear"]), d["x"])
+    assert compare_linear(g, r, "tiny") == 0
+
+
+def _rand_linear(seed, d_out, d_in, rank):
+    gen = np.random.default_rng(seed)
+    return inputs.linear(gen, d_out, d_in, rank) if rank else dict(
+        inputs.linear(gen, d_out, d_in, 1), lora_b=np.zeros((0, d_in), np.int8),
+        lora_b_scale=np.zeros(0, np.float32), lora_a=np.zeros((d_out, 0), np.int8))
+
+
+@pytest.mark.parametrize("d_out,d_in,rank,B", [
+    (1, 32, 0, 1), (33, 64, 1, 2), (127, 96, 7, 3), (129, 160, 16, 5), (512, 256, 16, 16),
+    (300, 384, 16, 4), (257, 1024, 16, 1), (1000, 8192, 16, 2), (8512, 2048, 16, 3),
+    (2048, 4096, 16, 16), (77, 512, 16, 1)])
+def test_linear_shapes(dev, d_out, d_in, rank, B):
+    lin = _rand_linear(d_out * 7 + d_in + rank + B, d_out, d_in, rank)
+    gen = np.random.default_rng(B)
+    x = inputs.normal(gen, (B, d_in)) * np.float32(2.5)
+    if B > 1:
+        x[1] = 0.0  # an all-zero token: s = 0, q = 0
+    g = run_linear(lin, x, dev)
+    r = oracle.linear_decode(oracle.Linear.from_dict(lin), x)
+    assert compare_linear(g, r, f"{d_out}x{d_in} r{rank} B{B}") == 0
+
+
+@pytest.mark.parametrize("which", ["in_proj", "out_proj"])
+def test_linear_full_stacks(dev, which):
+    """The 48-copy in_proj / out_proj workloads at B = 1, 4, 16: every copy's codes checked, copies
+    0 and 47 fully against the oracle, the others on 64 sampled rows."""
+    from bit_quantized_mamba_b200 import dfssm
+    data = inputs.in_proj_stack() if which == "in_proj" else inputs.out_proj_stack()
+    lins = [dfssm.Linear.from_host(l, dev) for l in data["linears"]]
+    gen = np.random.default_rng(99)
+    for B in (1, 4, 16):
+        x = data["x"][:B]
+        xd = to_dev(x, dev)
+        ys, accs, xqs = [], [], []
+        for L in lins:
+            dbg = dict(acc=torch.zeros((B, L.d_out), dtype=torch.int32, device=dev),
+                       xq=torch.zeros((B, L.d_in), dtype=torch.int8, device=dev))
+            ys.append(dfssm.linear_decode(L, xd, debug=dbg))
+            accs.append(dbg["acc"])
+            xqs.append(dbg["xq"])
+        torch.cuda.synchronize()
+        rq, rs = oracle.quantize(x)
+        for c, host in enumerate(data["linears"]):
+            assert np.array_equal(xqs[c].cpu().numpy(), rq)
+            OL = oracle.Linear.from_dict(host)
+            y = ys[c].cpu().numpy()
+            acc = accs[c].cpu().numpy()
+            if c in (0, len(lins) - 1):
+                r = oracle.linear_decode(OL, x)
+                assert np.array_equal(acc, r["acc"]), (which, B, c)
+                assert assert_tol(y, r["y"], f"{which} B{B} copy{c}") == 0
+            else:
+                rows = np.sort(gen.choice(OL.d_out, 64, replace=False))
+                for b in range(B):
+                    ry, racc = oracle.linear_rows(OL, rq[b], rs[b], rows)
+                    assert np.array_equal(acc[b, rows], racc), (which, B, c, b)
+                    assert assert_tol(y[b, rows], ry, f"{which} B{B} copy{c}") == 0
+
+
+def test_conv_step(dev):
+    from bit_quantized_mamba_b200 import dfssm
+    gen = np.random.default_rng(5)
+    B, Cn = 2, inputs.CONV_CH
+    w = gen.normal(0, 0.1, (Cn, 4)).astype(np.float32)
+    b = gen.normal(0, 0.1, Cn).astype(np.float32)
+    st_ref = np.zeros((B, Cn, 3), np.float32)
+    st = torch.zeros((B, Cn, 3), dtype=torch.float32, device=dev)
+    wd, bd = to_dev(w, dev), to_dev(b, dev)
+    mism = 0
+    for t in range(6):
+        x = inputs.normal(gen, (B, Cn)) * np.float32(3)
+        out = dfssm.conv_step(st, wd, bd, to_dev(x, dev)).cpu().numpy()
+        ref = oracle.conv_step(st_ref, w, b, x)
+        mism += assert_tol(out, ref, f"conv step {t}")
+        assert np.array_equal(st.cpu().numpy(), st_ref)
+    assert mism <= 2
+
+
+@pytest.mark.parametrize("B,H,P,N,G", [(2, 64, 64, 128, 1), (3, 8, 16, 32, 2), (1, 6, 5, 12, 3)])
+def test_ssm_step(dev, B, H, P, N, G):
+    from bit_quantized_mamba_b200 import dfssm
+    gen = np.random.default_rng(H * N + G)
+    A_log = gen.uniform(0, 2.7, H).astype(np.float32)
+    dt_bias = gen.uniform(-4, -1, H).astype(np.float32)
+    D = gen.uniform(0.5, 1.5, H).astype(np.float32)
+    st_ref = (gen.standard_normal((B, H, P, N)) * 0.5).astype(np.float32)
+    st = to_dev(st_ref, dev)
+    pd = [to_dev(a, dev) for a in (A_log, dt_bias, D)]
+    mism = 0
+    for t in range(4):
+        x = inputs.normal(gen, (B, H * P))
+        dt_raw = (inputs.normal(gen, (B, H)) * np.float32(2)).astype(np.float32)
+        Bm = inputs.normal(gen, (B, G, N))
+        Cm = inputs.normal(gen, (B, G, N))
+        y = dfssm.ssm_step(st, to_dev(x, dev), to_dev(dt_raw, dev), *pd, to_dev(Bm, dev),
+                           to_dev(Cm, dev)).cpu().numpy()
+        yr = oracle.ssm_step(st_ref, x, dt_raw, A_log, dt_bias, D, Bm, Cm)
+        mism += assert_tol(y, yr, f"ssm y {t}")
+        mism += assert_tol(st.cpu().numpy(), st_ref, f"ssm state {t}")
+    assert mism <= 4
+
+
+SMALL = dict(d_model=256, nheads=8, headdim=32, d_state=64, ngroups=1, rank=16)
+
+
+def _stack(model, dims, B, dev):
+    from bit_quantized_mamba_b200 import dfssm
+    n = len(model["layers"])
+    conv, ssm = inputs.zero_states(B, n, dims["nheads"], dims["headdim"], dims["d_state"],
+                                   dims["ngroups"])
+    layers = [dfssm.Layer.from_host(l, dev) for l in model["layers"]]
+    conv_d = [to_dev(conv[i], dev) for i in range(n)]
+    ssm_d = [to_dev(ssm[i], dev) for i in range(n)]
+    stack = dfssm.LayerStack(layers, dims, conv_d, ssm_d)
+    olayers = []
+    for l in model["layers"]:
+        ol = dict(l)
+        ol["in_proj"] = oracle.Linear.from_dict(l["in_proj"])
+        ol["out_proj"] = oracle.Linear.from_dict(l["out_proj"])
+        olayers.append(ol)
+    return stack, olayers, conv, ssm
+
+
+def _decode_compare(dev, model, dims, B, n_tokens, final_only=False):
+    from bit_quantized_mamba_b200 import dfssm
+    stack, olayers, conv, ssm = _stack(model, dims, B, dev)
+    n = len(olayers)
+    mism = 0
+    ws = dfssm.workspace(dfssm.workspace_size(dfssm.OP_LAYER_DECODE, B, dims["d_model"],
+                                              dims["nheads"] * dims["headdim"]), dev)
+    for t in range(n_tokens):
+        h_ref = np.ascontiguousarray(model["emb"][t][:B])
+        h = to_dev(h_ref, dev)
+        dfssm.layer_decode(stack, h, ws)
+        for l in range(n):
+            oracle.layer_decode(olayers[l], h_ref, conv[l], ssm[l])
+        if not final_only or t == n_tokens - 1:
+            torch.cuda.synchronize()
+            mism += assert_tol(h.cpu().numpy(), h_ref, f"hidden after token {t}")
+    for l in range(n):
+        mism += assert_tol(stack.ssm_states[l].cpu().numpy(), ssm[l], f"ssm state layer {l}")
+        mism += assert_tol(stack.conv_states[l].cpu().numpy(), conv[l], f"conv state layer {l}")
+    return mism
+
+
+def test_layer_decode_small_stack(dev):
+    model = inputs.decode_model(seed=7, n_layers=4, n_tokens=6, batch=2, **SMALL)
+    assert _decode_compare(dev, model, SMALL, 2, 6) <= 8
+
+
+def test_layer_decode_full_48x64(dev):
+    """The full 48-layer Mamba-2-1.3B-shaped stack, batch 1, 64 free-running decode steps."""
+    model = inputs.decode_model(seed=3)
+    dims = dict(d_model=2048, nheads=64, headdim=64, d_state=128, ngroups=1)
+    mism = _decode_compare(dev, model, dims, 1, 64, final_only=True)
+    print(f"48x64 decode: {mism} fp32 values differ in the last bits (all within tolerance)")
+
+
+def test_lm_head(dev):
+    from bit_quantized_mamba_b200 import dfssm
+    p = inputs.prefill(seed=4, m=4)
+    x = p["x_in"][-1]
+    W = to_dev(p["lm_w"], dev)
+    acc = torch.zeros(W.shape[0], dtype=torch.int32, device=dev)
+    logits = dfssm.lm_head(W, to_dev(p["lm_s"], dev), to_dev(x, dev), acc=acc).cpu().numpy()
+    rl, racc = oracle.lm_head(p["lm_w"], p["lm_s"], x)
+    assert np.array_equal(acc.cpu().numpy(), racc)
+    assert assert_tol(logits, rl, "lm head") == 0
