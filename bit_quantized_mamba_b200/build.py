@@ -13,7 +13,8 @@ OBJ = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libdfssm.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
-FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC,-O2", "--expt-relaxed-constexpr"]
+INCLUDE = os.path.join(os.path.dirname(HERE), "include")
+FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC,-O2", "--expt-relaxed-constexpr", "-I", INCLUDE]
 
 
 def sources():

@@ -44,14 +44,20 @@ struct LayerWs {
   dfssm::QuantScratch qs;
 };
 
-size_t layer_ws_bytes(int B, int d_model, int E, int C, int d_ip) {
+size_t chain_ws_bytes(int B, int d_model, int E, int C, int d_ip) {
   const int nmax = d_model > E ? d_model : E;
   return align256(sizeof(float) * (size_t)B * d_ip) + align256(sizeof(float) * (size_t)B * C) +
          align256(sizeof(float) * (size_t)B * E) + dfssm::quant_scratch_bytes(B, nmax);
 }
 
+// Layer-decode workspace: [fused-kernel region][per-op chain region].  The fused region comes first so
+// that its error word sits at a fixed offset (dfssm_device_status).
+size_t layer_ws_bytes(int B, int d_model, int E, int C, int d_ip) {
+  return align256(dfssm::fused_decode_workspace_bytes()) + chain_ws_bytes(B, d_model, E, C, d_ip);
+}
+
 LayerWs carve_layer_ws(void* base, int B, int d_model, int E, int C, int d_ip) {
-  char* p = static_cast<char*>(base);
+  char* p = static_cast<char*>(base) + align256(dfssm::fused_decode_workspace_bytes());
   LayerWs w;
   w.zxbcdt = reinterpret_cast<float*>(p);
   p += align256(sizeof(float) * (size_t)B * d_ip);
@@ -63,6 +69,9 @@ LayerWs carve_layer_ws(void* base, int B, int d_model, int E, int C, int d_ip) {
   w.qs = dfssm::carve_quant_scratch(p, B, nmax);
   return w;
 }
+
+// Clock budget of one device-side wait of the fused decode kernel (about 1 s at 2 GHz).
+constexpr long long kSpinLimitCycles = 2000000000LL;
 
 bool device_ok() {
   static int ok = -1;
@@ -265,6 +274,11 @@ int dfssm_layer_decode(const dfssm_layer_t* layers, int n_layers, const dfssm_di
     return DFSSM_EWORKSPACE;
   if (!device_ok()) return DFSSM_EDEVICE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (dfssm::fused_decode_supported(*dims, B, layers, n_layers)) {
+    const cudaError_t fe = dfssm::launch_fused_decode(layers, n_layers, hidden, conv_states, ssm_states,
+                                                      workspace, s, kSpinLimitCycles);
+    return fe == cudaSuccess ? DFSSM_OK : cuda_fail(fe);
+  }
   LayerWs w = carve_layer_ws(workspace, B, Dm, E, C, d_ip);
   cudaError_t e = cudaSuccess;
   for (int l = 0; l < n_layers && e == cudaSuccess; ++l) {
@@ -331,6 +345,24 @@ int dfssm_layer_decode(const dfssm_layer_t* layers, int n_layers, const dfssm_di
     ga.ldr = Dm;
     e = dfssm::launch_gemv(ga, s);
   }
+  return e == cudaSuccess ? DFSSM_OK : cuda_fail(e);
+}
+
+int dfssm_device_status(void* workspace, void* stream) {
+  if (!workspace || !aligned(workspace, 256)) return DFSSM_EWORKSPACE;
+  if (!device_ok()) return DFSSM_EDEVICE;
+  int code = 0;
+  const int e = dfssm::read_device_error(workspace, static_cast<cudaStream_t>(stream), &code);
+  if (e) return cuda_fail(static_cast<cudaError_t>(e));
+  return code ? DFSSM_ETIMEOUT : DFSSM_OK;
+}
+
+int dfssm_selftest_timeout(void* workspace, size_t ws_bytes, void* stream) {
+  if (!workspace || !aligned(workspace, 256) || ws_bytes < dfssm::fused_decode_workspace_bytes())
+    return DFSSM_EWORKSPACE;
+  if (!device_ok()) return DFSSM_EDEVICE;
+  const cudaError_t e =
+      dfssm::launch_timeout_selftest(workspace, static_cast<cudaStream_t>(stream), 2000000LL);
   return e == cudaSuccess ? DFSSM_OK : cuda_fail(e);
 }
 

@@ -4,7 +4,7 @@
 #include <cstdint>
 #include <cuda_runtime.h>
 
-#include "../../include/dfssm.h"
+#include "dfssm.h"
 
 #if defined(__CUDA_ARCH__) && (__CUDA_ARCH__ < 1000)
 #error "libdfssm is built for sm_100a only"
@@ -99,6 +99,56 @@ __device__ __forceinline__ int quant_code(float v, float s0) {
 __device__ __forceinline__ int perm_index(int i) {
   const int j = i & 31;
   return (i & ~31) + ((j & 7) << 2) + (j >> 3);
+}
+
+// ---------------------------------------------------------------- the method's arithmetic
+// These few functions fix the rounding sequence of every fp32 value the decode path stores; all
+// kernels (the per-op kernels and the fused decode kernel) use them, so both paths agree bit for bit.
+
+// Linear output for one (token, row): fl32(acc*s*sW + sA * sum_r W_A[r]*tf[r]), fp64 in this order.
+__device__ __forceinline__ float linear_out(int acc, float s, float sW, float sA, const int8_t* wa,
+                                            const float* tf, int rank) {
+  double lora = 0.0;
+  for (int r = 0; r < rank; ++r) lora = dadd(lora, dmul((double)wa[r], (double)tf[r]));
+  const double scaffold = dmul(dmul((double)acc, (double)s), (double)sW);
+  const double corr = rank > 0 ? dmul((double)sA, lora) : 0.0;
+  return __double2float_rn(dadd(scaffold, corr));
+}
+
+// LoRA intermediate tf = fl32(t * sB * s) (fp64).
+__device__ __forceinline__ float lora_tf(int t, float sB, float s) {
+  return __double2float_rn(dmul(dmul((double)t, (double)sB), (double)s));
+}
+
+// Scale of RMSNorm+quantize: fl32(s0 / sqrt(ss/n + 1e-5)) (fp64).
+__device__ __forceinline__ float rms_scale(float s0, double ss, int n) {
+  const double rms = __dsqrt_rn(__dadd_rn(__ddiv_rn(ss, (double)n), 1e-5));
+  return __double2float_rn(__ddiv_rn((double)s0, rms));
+}
+
+// Conv pre-activation fl32(b + w0*s0 + w1*s1 + w2*s2 + w3*x) (fp64, this order), then SiLU.
+__device__ __forceinline__ float conv_out(float4 w, float bias, float s0, float s1, float s2, float x) {
+  double e = (double)bias;
+  e = dadd(e, dmul((double)w.x, (double)s0));
+  e = dadd(e, dmul((double)w.y, (double)s1));
+  e = dadd(e, dmul((double)w.z, (double)s2));
+  e = dadd(e, dmul((double)w.w, (double)x));
+  return silu_f64(__double2float_rn(e));
+}
+
+// dt = fl32(softplus(fl32(dt_raw + dt_bias))), softplus(v) = v for v > 20 else log1p(exp(v)) (fp64).
+__device__ __forceinline__ float ssm_dt(float dt_raw, float dt_bias) {
+  const float v = fadd(dt_raw, dt_bias);
+  return v > 20.0f ? v : __double2float_rn(log1p(exp((double)v)));
+}
+// dA = fl32(exp(fl32(dt * fl32(-exp(A_log))))) (fp64 transcendental functions).
+__device__ __forceinline__ float ssm_dA(float dt, float A_log) {
+  const float A = __double2float_rn(-exp((double)A_log));
+  return __double2float_rn(exp((double)fmul(dt, A)));
+}
+// One state element: fl32(fl32(dA*S) + fl32(dtx*B)).
+__device__ __forceinline__ float ssm_state(float dA, float S, float dtx, float Bn) {
+  return fadd(fmul(dA, S), fmul(dtx, Bn));
 }
 
 // ---------------------------------------------------------------- block reductions

@@ -1,0 +1,700 @@
+// Fused persistent decode of a DF-SSM Mamba-2 stack: one cooperative launch carries one token through
+// every layer (gist.science technical summary of DF-SSM, §2.C: batch-1 decode of the 1-bit scaffold with
+// int8 LoRA, the conv shift register and the SSM recurrence; the pages capture the 48-layer forward as a
+// CUDA graph — here the whole forward is one kernel, so no launch sits between layers).
+//
+// One CTA per SM owns a fixed slice of every layer:
+//   * ~E/NC SSM rows (h,p): their SSM state rows, the matching z and x rows of in_proj, the conv
+//     channels of those x rows;
+//   * ~320/NC of the rows every CTA needs (B, C and dt rows of in_proj), whose scaffold accumulators it
+//     publishes;
+//   * ~d_model/NC rows of out_proj and the matching entries of the residual stream.
+// The weights and states of a CTA's slice are loaded into registers and shared memory at the start of
+// the layer (and prefetched into L2 one layer ahead), before the CTA waits on anything, so the HBM stream
+// overlaps the dependency chain.  Cross-CTA hand-offs go through global memory with monotonically
+// increasing counters (arrive = fence + atomic add; wait = bounded acquire spin).  A wait that runs past
+// its clock budget records DFSSM_ETIMEOUT in the workspace error word and the CTA returns.
+//
+// All arithmetic goes through the functions in common.cuh, so the results are those of the per-op path.
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace dfssm {
+namespace fused {
+
+constexpr int DM = 2048, E = 4096, H = 64, P = 64, N = 128, R = 16;
+constexpr int CC = E + 2 * N;           // conv channels: x | B | C
+constexpr int DIP = 2 * E + 2 * N + H;  // in_proj rows: z | x | B | C | dt
+constexpr int SH0 = 2 * E;              // first row needed by every CTA (B rows, then C, then dt)
+constexpr int NSH = 2 * N + H;          // 320 such rows
+constexpr int NT = 512, NW = NT / 32;
+constexpr int MAX_IN = 64, MAX_OUT = 16, MAX_SSM = 32;
+constexpr int NUM_T_PRODUCERS = R;      // CTAs [0, 16) produce t_in, [16, 32) produce t_out
+constexpr int kAuxThread = 32;         // computes the RMS scale while thread 0 polls
+
+enum { CTR_H = 0, CTR_BC, CTR_G, CTR_TOUT, N_CTR };
+constexpr int CTR_STRIDE = 32;          // one 128-byte line per counter
+
+struct LayerPtrs {
+  const uint32_t* in_bits;
+  const float* in_ws;
+  const int8_t* in_lb;
+  const float* in_lbs;
+  const int8_t* in_la;
+  const float* in_las;
+  const uint32_t* out_bits;
+  const float* out_ws;
+  const int8_t* out_lb;
+  const float* out_lbs;
+  const int8_t* out_la;
+  const float* out_las;
+  const float* conv_w;
+  const float* conv_b;
+  const float* A_log;
+  const float* dt_bias;
+  const float* D;
+  const float* norm_w;
+  const float* gnorm_w;
+  float* conv_state;
+  float* ssm_state;
+};
+
+struct Params {
+  LayerPtrs L[DFSSM_MAX_LAYERS];
+  int n_layers;
+  float* hidden;
+  int* ctr;
+  int* err;
+  int* status;
+  int* tin;
+  int* tout;
+  int* sacc;
+  float* gbuf;
+  long long spin_limit;
+};
+
+// ------------------------------------------------------------------------------ workspace layout
+// [counters N_CTR x 128 B][abort word 128 B][status word 128 B][t_in 16][t_out 16][sacc 320][gbuf 4096]
+// The counters and the abort word are cleared before every launch; the status word is sticky: a timed
+// out wait stores kTimeoutMagic there, and only dfssm_device_status clears it.
+constexpr size_t OFF_CTR = 0;
+constexpr size_t OFF_ERR = OFF_CTR + N_CTR * CTR_STRIDE * 4;
+constexpr size_t OFF_STATUS = OFF_ERR + 128;
+constexpr size_t CLEAR_BYTES = OFF_STATUS;  // counters + abort word
+constexpr size_t OFF_TIN = OFF_STATUS + 128;
+constexpr size_t OFF_TOUT = OFF_TIN + 64;
+constexpr size_t OFF_SACC = OFF_TOUT + 64;
+constexpr size_t OFF_GBUF = OFF_SACC + ((NSH * 4 + 255) / 256) * 256;
+constexpr size_t WS_BYTES = OFF_GBUF + E * 4;
+
+// ------------------------------------------------------------------------------ synchronisation
+
+__device__ __forceinline__ int ld_acquire(const int* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ int ld_relaxed(const int* p) {
+  int v;
+  asm volatile("ld.relaxed.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+constexpr int kTimeoutMagic = 0x7E0D1E57;
+
+// All threads of the CTA: returns once *ctr >= target.  Returns false (for every thread) when the
+// clock budget ran out (the abort and status words are then set) or another CTA already aborted.
+// Thread 0 polls with relaxed loads and finishes with an acquire fence; the CTA barrier then orders
+// the other threads' reads after it.
+__device__ bool block_wait(const int* ctr, int target, int* err, int* status, long long limit,
+                           int* sflag) {
+  if (threadIdx.x == 0) {
+    int ok = 1;
+    if (ld_relaxed(ctr) < target) {
+      const long long t0 = clock64();
+      unsigned it = 0;
+      while (ld_relaxed(ctr) < target) {
+        if ((++it & 15u) == 0) {
+          if (ld_relaxed(err) != 0) {
+            ok = 0;
+            break;
+          }
+          if (clock64() - t0 > limit) {
+            atomicExch(err, 1);
+            atomicExch(status, kTimeoutMagic);
+            ok = 0;
+            break;
+          }
+        }
+      }
+    }
+    if (ok) asm volatile("fence.acq_rel.gpu;" ::: "memory");
+    *sflag = ok;
+  }
+  __syncthreads();
+  return *sflag != 0;
+}
+
+// All threads of the CTA: count one arrival after every global write the CTA made so far (the CTA
+// barrier orders them before thread 0's release).
+__device__ __forceinline__ void block_arrive(int* ctr) {
+  __syncthreads();
+  if (threadIdx.x == 0) asm volatile("red.release.gpu.global.add.s32 [%0], 1;" ::"l"(ctr) : "memory");
+}
+
+__device__ __forceinline__ void prefetch_l2(const void* p, unsigned bytes) {
+  if (bytes >= 16)
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes & ~15u) : "memory");
+}
+
+// One prefetch per 128-byte line of [p, p + bytes) (the first line is aligned down inside the array).
+__device__ __forceinline__ void prefetch_lines(const void* p, unsigned bytes) {
+  const char* a = reinterpret_cast<const char*>(reinterpret_cast<uintptr_t>(p) & ~uintptr_t(127));
+  const char* e = reinterpret_cast<const char*>(p) + bytes;
+  for (; a < e; a += 128) asm volatile("prefetch.global.L2 [%0];" ::"l"(a) : "memory");
+}
+
+// ------------------------------------------------------------------------------ block reductions
+
+struct Red2 {
+  double ss;
+  float m;
+};
+
+__device__ __forceinline__ Red2 block_sum_max(double ss, float m, double* rd, float* rf) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  ss = warp_sum(ss);
+  m = warp_max(m);
+  if (lane == 0) {
+    rd[w] = ss;
+    rf[w] = m;
+  }
+  __syncthreads();
+  double s2 = lane < NW ? rd[lane] : 0.0;
+  float m2 = lane < NW ? rf[lane] : 0.0f;
+  s2 = warp_sum(s2);
+  m2 = warp_max(m2);
+  __syncthreads();  // rd/rf may be reused right after
+  return Red2{s2, m2};
+}
+
+__device__ __forceinline__ int block_sum_int(int v, int* ri) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  v = warp_sum(v);
+  if (lane == 0) ri[w] = v;
+  __syncthreads();
+  int t = lane < NW ? ri[lane] : 0;
+  t = warp_sum(t);
+  __syncthreads();
+  return t;
+}
+
+// Shared-memory position of natural activation index i: the dp4a-permuted codes of 128-input segment
+// `seg` occupy eight 16-byte chunks, and chunk v of every segment is stored contiguously across the
+// NSEG segments (byte (v * NSEG + seg) * 16 + pos % 16), so the lanes that each own one segment read
+// consecutive chunks without bank conflicts.
+template <int NSEG>
+__device__ __forceinline__ int seg_index(int i) {
+  const int seg = i >> 7;
+  const int pos = perm_index(i) & 127;
+  return ((pos >> 4) * NSEG + seg) * 16 + (pos & 15);
+}
+
+// Sum over bit=1 positions of q for 128 weights (one uint4 of sign bits) against the permuted codes of
+// their segment; chunk v of the segment is qp4[v * NSEG].
+template <int NSEG>
+__device__ __forceinline__ int bits_dot(uint4 w, const uint4* qp4) {
+  int acc8[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) acc8[k] = 0;
+  const uint32_t w4[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const uint4 qa = qp4[(2 * j) * NSEG], qb = qp4[(2 * j + 1) * NSEG];
+    const uint32_t qp[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
+#pragma unroll
+    for (int k = 0; k < 8; ++k) acc8[k] = dp4a_us(w4[j] & (0x01010101u << k), qp[k], acc8[k]);
+  }
+  int S = 0;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) S += acc8[k] >> k;
+  return S;
+}
+
+// ------------------------------------------------------------------------------ the kernel
+
+__global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ Params p) {
+  __shared__ __align__(16) int8_t q_perm[E];
+  __shared__ __align__(16) int8_t q_nat[E];
+  __shared__ double red_d[NW];
+  __shared__ float red_f[NW];
+  __shared__ int red_i[NW];
+  __shared__ int sflag;
+  __shared__ float tf[R];
+  __shared__ float s_scale;
+  __shared__ int s_sumq;
+  // in_proj rows owned by this CTA (slot order: shared rows, z rows, x rows)
+  __shared__ int acc_in[MAX_IN];
+  __shared__ float in_sw[MAX_IN], in_sa[MAX_IN];
+  __shared__ __align__(16) int8_t in_wa[MAX_IN][R];
+  // the 320 rows every CTA needs
+  __shared__ float sh_sw[NSH], sh_sa[NSH];
+  __shared__ __align__(16) int8_t sh_wa[NSH][R];
+  __shared__ float4 bc_w[2 * N];
+  __shared__ float bc_b[2 * N];
+  __shared__ float bc_st[2 * N][3];
+  __shared__ float bc_new[2 * N];
+  __shared__ __align__(16) float Bsm[N];
+  __shared__ __align__(16) float Csm[N];
+  // SSM rows
+  __shared__ float zsm[MAX_SSM], xsm[MAX_SSM];
+  __shared__ float dtv[2], dAv[2], Dv[2];
+  // out_proj rows
+  __shared__ int acc_out[MAX_OUT];
+  __shared__ float o_sw[MAX_OUT], o_sa[MAX_OUT];
+  __shared__ __align__(16) int8_t o_wa[MAX_OUT][R];
+
+  const int c = blockIdx.x, NC = gridDim.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+
+  // ---- fixed ownership
+  const int rs0 = (int)((long long)c * E / NC), rs1 = (int)((long long)(c + 1) * E / NC);
+  const int n_ssm = rs1 - rs0;
+  const int sh0 = c * NSH / NC, sh1 = (c + 1) * NSH / NC, n_sh = sh1 - sh0;
+  const int ro0 = c * DM / NC, ro1 = (c + 1) * DM / NC, n_out = ro1 - ro0;
+  const int n_in = n_sh + 2 * n_ssm;
+  const int hA = rs0 / P;  // first head of this CTA's SSM rows (at most two heads)
+  auto in_row = [&](int slot) -> int {
+    if (slot < n_sh) return SH0 + sh0 + slot;
+    const int j = slot - n_sh;
+    return j < n_ssm ? rs0 + j : E + rs0 + (j - n_ssm);
+  };
+
+  // per-thread GEMV / SSM positions
+  const int li_in = lane & 15;
+  const int slot_in[2] = {warp * 2 + (lane >> 4), 32 + warp * 2 + (lane >> 4)};
+  const int slot_out = warp;  // out_proj: one row per warp, 32 lanes x 128 weights
+  const int ssm_slot[2] = {warp, NW + warp};
+
+  for (int l = 0; l < p.n_layers; ++l) {
+    const LayerPtrs& Lp = p.L[l];
+
+    // ---------------------------------------------------------------- loads for the whole layer
+    if (tid < 2 && l + 1 < p.n_layers) {
+      // this CTA's slice of the next layer, and (spread over CTAs 0..31) the parts every CTA reads
+      const LayerPtrs& Nx = p.L[l + 1];
+      if (tid == 0) {
+        prefetch_l2(Nx.in_bits + (size_t)(SH0 + sh0) * (DM / 32), n_sh * (DM / 8));
+        prefetch_l2(Nx.in_bits + (size_t)rs0 * (DM / 32), n_ssm * (DM / 8));
+        prefetch_l2(Nx.in_bits + (size_t)(E + rs0) * (DM / 32), n_ssm * (DM / 8));
+        prefetch_l2(Nx.out_bits + (size_t)ro0 * (E / 32), n_out * (E / 8));
+        prefetch_l2(Nx.ssm_state + (size_t)rs0 * N, n_ssm * N * 4);
+        prefetch_l2(Nx.in_la + (size_t)rs0 * R, n_ssm * R);
+        prefetch_l2(Nx.in_la + (size_t)(E + rs0) * R, n_ssm * R);
+        prefetch_l2(Nx.out_la + (size_t)ro0 * R, n_out * R);
+        prefetch_l2(Nx.conv_w + (size_t)rs0 * 4, n_ssm * 16);
+      } else {
+        prefetch_lines(Nx.in_ws + rs0, n_ssm * 4);
+        prefetch_lines(Nx.in_ws + E + rs0, n_ssm * 4);
+        prefetch_lines(Nx.in_las + rs0, n_ssm * 4);
+        prefetch_lines(Nx.in_las + E + rs0, n_ssm * 4);
+        prefetch_lines(Nx.out_ws + ro0, n_out * 4);
+        prefetch_lines(Nx.out_las + ro0, n_out * 4);
+        prefetch_lines(Nx.conv_b + rs0, n_ssm * 4);
+        prefetch_lines(Nx.conv_state + (size_t)rs0 * 3, n_ssm * 12);
+        if (c < NUM_T_PRODUCERS) prefetch_l2(Nx.in_lb + (size_t)c * DM, DM);
+        else if (c < 2 * NUM_T_PRODUCERS) prefetch_l2(Nx.out_lb + (size_t)(c - NUM_T_PRODUCERS) * E, E);
+        switch (c) {
+          case 0: prefetch_l2(Nx.norm_w, DM * 4); break;
+          case 1: prefetch_l2(Nx.gnorm_w, E * 4); break;
+          case 2:
+            prefetch_lines(Nx.in_ws + SH0, NSH * 4);
+            prefetch_lines(Nx.in_las + SH0, NSH * 4);
+            prefetch_l2(Nx.in_la + (size_t)SH0 * R, NSH * R);
+            break;
+          case 3:
+            prefetch_l2(Nx.conv_w + (size_t)E * 4, 2 * N * 16);
+            prefetch_lines(Nx.conv_b + E, 2 * N * 4);
+            prefetch_lines(Nx.conv_state + (size_t)E * 3, 2 * N * 12);
+            break;
+          case 4:
+            prefetch_lines(Nx.dt_bias, H * 4);
+            prefetch_lines(Nx.A_log, H * 4);
+            prefetch_lines(Nx.D, H * 4);
+            prefetch_lines(Nx.in_lbs, R * 4);
+            prefetch_lines(Nx.out_lbs, R * 4);
+            break;
+          default: break;
+        }
+      }
+    }
+    uint4 w_in[2], w_out;
+#pragma unroll
+    for (int ps = 0; ps < 2; ++ps) {
+      const int slot = slot_in[ps];
+      w_in[ps] = slot < n_in ? ld_stream_u4(Lp.in_bits + (size_t)in_row(slot) * (DM / 32) + li_in * 4)
+                             : make_uint4(0, 0, 0, 0);
+    }
+    w_out = slot_out < n_out ? ld_stream_u4(Lp.out_bits + (size_t)(ro0 + slot_out) * (E / 32) + lane * 4)
+                             : make_uint4(0, 0, 0, 0);
+    float4 sv[2];
+#pragma unroll
+    for (int ps = 0; ps < 2; ++ps) {
+      const int rr = ssm_slot[ps];
+      sv[ps] = rr < n_ssm ? ld_evict_first_f4(Lp.ssm_state + (size_t)(rs0 + rr) * N + lane * 4)
+                          : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    float nw[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) nw[k] = __ldg(Lp.norm_w + tid + k * NT);
+    uint32_t wb_in = 0;
+    uint2 wb_out = make_uint2(0, 0);
+    if (c < NUM_T_PRODUCERS) wb_in = ld_stream_u32(Lp.in_lb + (size_t)c * DM + 4 * tid);
+    if (c >= NUM_T_PRODUCERS && c < 2 * NUM_T_PRODUCERS) {
+      const int8_t* rowp = Lp.out_lb + (size_t)(c - NUM_T_PRODUCERS) * E + 8 * tid;
+      wb_out = make_uint2(ld_stream_u32(rowp), ld_stream_u32(rowp + 4));
+    }
+    // epilogue parameters into shared memory
+    if (tid < n_in) {
+      const int row = in_row(tid);
+      in_sw[tid] = __ldg(Lp.in_ws + row);
+      in_sa[tid] = __ldg(Lp.in_las + row);
+      *reinterpret_cast<uint4*>(in_wa[tid]) = ld_stream_u4(Lp.in_la + (size_t)row * R);
+    }
+    if (tid < NSH) {
+      const int row = SH0 + tid;
+      sh_sw[tid] = __ldg(Lp.in_ws + row);
+      sh_sa[tid] = __ldg(Lp.in_las + row);
+      *reinterpret_cast<uint4*>(sh_wa[tid]) = __ldg(reinterpret_cast<const uint4*>(Lp.in_la) + row);
+    }
+    if (tid < 2 * N) {
+      const int ch = E + tid;
+      bc_w[tid] = __ldg(reinterpret_cast<const float4*>(Lp.conv_w) + ch);
+      bc_b[tid] = __ldg(Lp.conv_b + ch);
+      bc_st[tid][0] = __ldcg(Lp.conv_state + (size_t)ch * 3 + 0);
+      bc_st[tid][1] = __ldcg(Lp.conv_state + (size_t)ch * 3 + 1);
+      bc_st[tid][2] = __ldcg(Lp.conv_state + (size_t)ch * 3 + 2);
+    }
+    if (tid < n_out) {
+      const int row = ro0 + tid;
+      o_sw[tid] = __ldg(Lp.out_ws + row);
+      o_sa[tid] = __ldg(Lp.out_las + row);
+      *reinterpret_cast<uint4*>(o_wa[tid]) = ld_stream_u4(Lp.out_la + (size_t)row * R);
+    }
+    // own x channels: conv taps, bias, state (thread NSH + j handles channel rs0 + j)
+    float4 cw = make_float4(0.f, 0.f, 0.f, 0.f);
+    float cb = 0.f, cs0 = 0.f, cs1 = 0.f, cs2 = 0.f;
+    if (tid >= NSH && tid - NSH < n_ssm) {
+      const int ch = rs0 + (tid - NSH);
+      cw = __ldg(reinterpret_cast<const float4*>(Lp.conv_w) + ch);
+      cb = __ldg(Lp.conv_b + ch);
+      cs0 = Lp.conv_state[(size_t)ch * 3 + 0];
+      cs1 = Lp.conv_state[(size_t)ch * 3 + 1];
+      cs2 = Lp.conv_state[(size_t)ch * 3 + 2];
+    }
+    if (tid < 2) {
+      const int h = hA + tid;
+      if (h < H) Dv[tid] = __ldg(Lp.D + h);
+    }
+
+    // ---------------------------------------------------------------- phase A: h -> in_proj
+    if (l > 0 && !block_wait(p.ctr + CTR_H * CTR_STRIDE, NC * l, p.err, p.status, p.spin_limit, &sflag)) return;
+    double ssA;
+    float s0A;
+    {
+      float hv[4], v[4];
+      double ss = 0.0;
+      float m = 0.0f;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        hv[k] = __ldcg(p.hidden + tid + k * NT);
+        ss += (double)hv[k] * (double)hv[k];
+        v[k] = fmul(hv[k], nw[k]);
+        m = fmaxf(m, fabsf(v[k]));
+      }
+      const Red2 r = block_sum_max(ss, m, red_d, red_f);
+      const float s0 = r.m == 0.0f ? 0.0f : __fdiv_rn(r.m, 127.0f);
+      int sq = 0;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int i = tid + k * NT;
+        const int code = r.m == 0.0f ? 0 : quant_code(v[k], s0);
+        q_nat[i] = (int8_t)code;
+        q_perm[seg_index<DM / 128>(i)] = (int8_t)code;
+        sq += code;
+      }
+      sq = block_sum_int(sq, red_i);  // its internal barriers also publish q_nat / q_perm
+      if (tid == 0) s_sumq = sq;
+      ssA = r.ss;
+      s0A = s0;
+    }
+    // LoRA-down producers: t_in[c] = sum_i W_B[c,i] q_i.  It is written before this CTA's B/C arrival,
+    // so a CTA that has seen every B/C arrival also sees every t_in.
+    if (c < NUM_T_PRODUCERS) {
+      const int t = block_sum_int(dp4a_ss(wb_in, reinterpret_cast<const uint32_t*>(q_nat)[tid], 0),
+                                  red_i);
+      if (tid == 0) p.tin[c] = t;
+    }
+    __syncthreads();
+    const int sumq_in = s_sumq;
+    // scaffold GEMV over the owned rows; pass 0 holds the rows every CTA needs
+    {
+      const uint4* qp4 = reinterpret_cast<const uint4*>(q_perm) + li_in;
+#pragma unroll
+      for (int ps = 0; ps < 2; ++ps) {
+        int S = bits_dot<DM / 128>(w_in[ps], qp4);
+#pragma unroll
+        for (int o = 8; o > 0; o >>= 1) S += __shfl_xor_sync(0xffffffffu, S, o);
+        if (li_in == 0 && slot_in[ps] < n_in) acc_in[slot_in[ps]] = 2 * S - sumq_in;
+        if (ps == 0) {
+          __syncthreads();
+          if (tid < n_sh) p.sacc[sh0 + tid] = acc_in[tid];
+          block_arrive(p.ctr + CTR_BC * CTR_STRIDE);
+        }
+      }
+    }
+    if (tid == kAuxThread) s_scale = rms_scale(s0A, ssA, DM);
+    if (!block_wait(p.ctr + CTR_BC * CTR_STRIDE, NC * (l + 1), p.err, p.status, p.spin_limit, &sflag))
+      return;
+    const float s_in = s_scale;
+    if (tid < R) tf[tid] = lora_tf(__ldcg(p.tin + tid), __ldg(Lp.in_lbs + tid), s_in);
+    __syncthreads();
+    if (tid < NSH) {
+      // rows every CTA needs: B, C (conv + SiLU) and dt of this CTA's heads
+      const float y = linear_out(__ldcg(p.sacc + tid), s_in, sh_sw[tid], sh_sa[tid], sh_wa[tid], tf, R);
+      if (tid < 2 * N) {
+        bc_new[tid] = y;
+        const float xc = conv_out(bc_w[tid], bc_b[tid], bc_st[tid][0], bc_st[tid][1], bc_st[tid][2], y);
+        if (tid < N) Bsm[tid] = xc;
+        else Csm[tid - N] = xc;
+      } else {
+        const int h = tid - 2 * N;
+        if (h == hA || h == hA + 1) {
+          const float dt = ssm_dt(y, __ldg(Lp.dt_bias + h));
+          dtv[h - hA] = dt;
+          dAv[h - hA] = ssm_dA(dt, __ldg(Lp.A_log + h));
+        }
+      }
+    } else if (tid - NSH < n_ssm) {
+      // the owned z rows (gate value SiLU(z) kept) and x rows (conv of the owned x channels)
+      const int j = tid - NSH;
+      const int sz = n_sh + j, sx = n_sh + n_ssm + j;
+      zsm[j] = silu_f64(linear_out(acc_in[sz], s_in, in_sw[sz], in_sa[sz], in_wa[sz], tf, R));
+      const float xr = linear_out(acc_in[sx], s_in, in_sw[sx], in_sa[sx], in_wa[sx], tf, R);
+      xsm[j] = conv_out(cw, cb, cs0, cs1, cs2, xr);
+      float* st = Lp.conv_state + (size_t)(rs0 + j) * 3;
+      st[0] = cs1;
+      st[1] = cs2;
+      st[2] = xr;
+    }
+    __syncthreads();
+
+    // ---------------------------------------------------------------- phase B: SSM + gate
+#pragma unroll
+    for (int ps = 0; ps < 2; ++ps) {
+      const int rr = ssm_slot[ps];
+      if (rr < n_ssm) {
+        const int hp = rs0 + rr;
+        const int hi = hp / P - hA;
+        const float dt = dtv[hi], dA = dAv[hi];
+        const float xv = xsm[rr];
+        const float dtx = fmul(dt, xv);
+        const float4 b4 = reinterpret_cast<const float4*>(Bsm)[lane];
+        const float4 c4 = reinterpret_cast<const float4*>(Csm)[lane];
+        float4 s4 = sv[ps];
+        s4.x = ssm_state(dA, s4.x, dtx, b4.x);
+        s4.y = ssm_state(dA, s4.y, dtx, b4.y);
+        s4.z = ssm_state(dA, s4.z, dtx, b4.z);
+        s4.w = ssm_state(dA, s4.w, dtx, b4.w);
+        double acc = (double)s4.x * (double)c4.x;
+        acc = fma((double)s4.y, (double)c4.y, acc);
+        acc = fma((double)s4.z, (double)c4.z, acc);
+        acc = fma((double)s4.w, (double)c4.w, acc);
+        st_f4(Lp.ssm_state + (size_t)hp * N + lane * 4, s4);
+        acc = warp_sum(acc);
+        if (lane == 0) {
+          const float y = __double2float_rn(dadd(acc, dmul((double)Dv[hi], (double)xv)));
+          p.gbuf[hp] = fmul(y, zsm[rr]);
+        }
+      }
+    }
+    block_arrive(p.ctr + CTR_G * CTR_STRIDE);
+
+    // ---------------------------------------------------------------- phase C: gated norm -> out_proj
+    float gw[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) gw[k] = __ldg(Lp.gnorm_w + tid + k * NT);
+    if (!block_wait(p.ctr + CTR_G * CTR_STRIDE, NC * (l + 1), p.err, p.status, p.spin_limit, &sflag)) return;
+    // every CTA has now read the old B/C conv state: the owners of those rows shift it
+    for (int j = tid; j < n_sh; j += NT) {
+      const int k = sh0 + j;
+      if (k < 2 * N) {
+        float* st = Lp.conv_state + (size_t)(E + k) * 3;
+        st[0] = bc_st[k][1];
+        st[1] = bc_st[k][2];
+        st[2] = bc_new[k];
+      }
+    }
+    {
+      float v[8];
+      double ss = 0.0;
+      float m = 0.0f;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const float g = __ldcg(p.gbuf + tid + k * NT);
+        ss += (double)g * (double)g;
+        v[k] = fmul(g, gw[k]);
+        m = fmaxf(m, fabsf(v[k]));
+      }
+      const Red2 r = block_sum_max(ss, m, red_d, red_f);
+      const float s0 = r.m == 0.0f ? 0.0f : __fdiv_rn(r.m, 127.0f);
+      int sq = 0;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const int i = tid + k * NT;
+        const int code = r.m == 0.0f ? 0 : quant_code(v[k], s0);
+        q_nat[i] = (int8_t)code;
+        q_perm[seg_index<E / 128>(i)] = (int8_t)code;
+        sq += code;
+      }
+      sq = block_sum_int(sq, red_i);
+      if (tid == 0) s_sumq = sq;
+      ssA = r.ss;
+      s0A = s0;
+    }
+    if (c >= NUM_T_PRODUCERS && c < 2 * NUM_T_PRODUCERS) {
+      const uint2 qq = reinterpret_cast<const uint2*>(q_nat)[tid];
+      const int t = block_sum_int(dp4a_ss(wb_out.y, qq.y, dp4a_ss(wb_out.x, qq.x, 0)), red_i);
+      if (tid == 0) p.tout[c - NUM_T_PRODUCERS] = t;
+      block_arrive(p.ctr + CTR_TOUT * CTR_STRIDE);
+    }
+    __syncthreads();
+    {
+      const uint4* qp4 = reinterpret_cast<const uint4*>(q_perm) + lane;
+      int S = bits_dot<E / 128>(w_out, qp4);
+      S = warp_sum(S);
+      if (lane == 0 && slot_out < n_out) acc_out[slot_out] = 2 * S - s_sumq;
+    }
+    if (tid == kAuxThread) s_scale = rms_scale(s0A, ssA, E);
+    if (!block_wait(p.ctr + CTR_TOUT * CTR_STRIDE, NUM_T_PRODUCERS * (l + 1), p.err, p.status, p.spin_limit,
+                    &sflag))
+      return;
+    const float s_out = s_scale;
+    if (tid < R) tf[tid] = lora_tf(__ldcg(p.tout + tid), __ldg(Lp.out_lbs + tid), s_out);
+    __syncthreads();
+    if (tid < n_out) {
+      const int o = ro0 + tid;
+      const float y = linear_out(acc_out[tid], s_out, o_sw[tid], o_sa[tid], o_wa[tid], tf, R);
+      p.hidden[o] = fadd(__ldcg(p.hidden + o), y);
+    }
+    block_arrive(p.ctr + CTR_H * CTR_STRIDE);
+  }
+}
+
+// Waits on a counter that nothing increments, with a short budget: exercises the timeout path.
+__global__ void timeout_selftest_kernel(int* ctr, int* err, int* status, long long limit) {
+  __shared__ int sflag;
+  block_wait(ctr, 1, err, status, limit, &sflag);
+}
+
+}  // namespace fused
+
+size_t fused_decode_workspace_bytes() { return fused::WS_BYTES; }
+
+bool fused_decode_supported(const dfssm_dims_t& d, int B, const dfssm_layer_t* layers, int n) {
+  if (B != 1 || d.d_model != fused::DM || d.nheads != fused::H || d.headdim != fused::P ||
+      d.d_state != fused::N || d.ngroups != 1)
+    return false;
+  for (int l = 0; l < n; ++l)
+    if (layers[l].in_proj.rank != fused::R || layers[l].out_proj.rank != fused::R) return false;
+  const int nc = num_sms();
+  // ownership limits: in_proj rows per CTA <= 64, out_proj rows <= 16, SSM rows <= 32, and the two
+  // groups of LoRA-down producers must exist
+  if (nc < 133 || nc > 1024) return false;
+  int coop = 0, dev = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev);
+  return coop != 0;
+}
+
+cudaError_t launch_fused_decode(const dfssm_layer_t* layers, int n_layers, float* hidden,
+                                float* const* conv_states, float* const* ssm_states, void* ws,
+                                cudaStream_t st, long long spin_limit) {
+  static_assert(sizeof(fused::Params) < 32000, "kernel parameter block too large");
+  fused::Params p;  // copied into the launch
+  for (int l = 0; l < n_layers; ++l) {
+    const dfssm_layer_t& Ly = layers[l];
+    fused::LayerPtrs& q = p.L[l];
+    q.in_bits = Ly.in_proj.bits;
+    q.in_ws = Ly.in_proj.w_scale;
+    q.in_lb = Ly.in_proj.lora_b;
+    q.in_lbs = Ly.in_proj.lora_b_scale;
+    q.in_la = Ly.in_proj.lora_a;
+    q.in_las = Ly.in_proj.lora_a_scale;
+    q.out_bits = Ly.out_proj.bits;
+    q.out_ws = Ly.out_proj.w_scale;
+    q.out_lb = Ly.out_proj.lora_b;
+    q.out_lbs = Ly.out_proj.lora_b_scale;
+    q.out_la = Ly.out_proj.lora_a;
+    q.out_las = Ly.out_proj.lora_a_scale;
+    q.conv_w = Ly.conv_w;
+    q.conv_b = Ly.conv_b;
+    q.A_log = Ly.A_log;
+    q.dt_bias = Ly.dt_bias;
+    q.D = Ly.D;
+    q.norm_w = Ly.norm_w;
+    q.gnorm_w = Ly.gnorm_w;
+    q.conv_state = conv_states[l];
+    q.ssm_state = ssm_states[l];
+  }
+  char* base = static_cast<char*>(ws);
+  p.n_layers = n_layers;
+  p.hidden = hidden;
+  p.ctr = reinterpret_cast<int*>(base + fused::OFF_CTR);
+  p.err = reinterpret_cast<int*>(base + fused::OFF_ERR);
+  p.status = reinterpret_cast<int*>(base + fused::OFF_STATUS);
+  p.tin = reinterpret_cast<int*>(base + fused::OFF_TIN);
+  p.tout = reinterpret_cast<int*>(base + fused::OFF_TOUT);
+  p.sacc = reinterpret_cast<int*>(base + fused::OFF_SACC);
+  p.gbuf = reinterpret_cast<float*>(base + fused::OFF_GBUF);
+  p.spin_limit = spin_limit;
+  cudaError_t e = cudaMemsetAsync(p.ctr, 0, fused::CLEAR_BYTES, st);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(num_sms());
+  cfg.blockDim = dim3(fused::NT);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, fused::decode_kernel, p);
+}
+
+cudaError_t launch_timeout_selftest(void* ws, cudaStream_t st, long long spin_limit) {
+  char* base = static_cast<char*>(ws);
+  int* ctr = reinterpret_cast<int*>(base + fused::OFF_CTR);
+  int* err = reinterpret_cast<int*>(base + fused::OFF_ERR);
+  int* status = reinterpret_cast<int*>(base + fused::OFF_STATUS);
+  cudaError_t e = cudaMemsetAsync(ctr, 0, fused::CLEAR_BYTES, st);
+  if (e != cudaSuccess) return e;
+  fused::timeout_selftest_kernel<<<1, 32, 0, st>>>(ctr, err, status, spin_limit);
+  return cudaGetLastError();
+}
+
+int read_device_error(void* ws, cudaStream_t st, int* code) {
+  char* base = static_cast<char*>(ws);
+  int* status = reinterpret_cast<int*>(base + fused::OFF_STATUS);
+  int h = 0;
+  cudaError_t e = cudaMemcpyAsync(&h, status, sizeof(int), cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e == cudaSuccess) e = cudaMemsetAsync(status, 0, sizeof(int), st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  *code = (h == fused::kTimeoutMagic) ? 1 : 0;
+  return e == cudaSuccess ? 0 : (int)e;
+}
+
+}  // namespace dfssm

@@ -98,4 +98,15 @@ int num_sms();
 namespace dfssm {
 // Prefill (tcgen05) workspace requirement for M tokens of a d_in -> d_out linear.
 size_t prefill_workspace_bytes(int M, int d_in, int d_out);
+
+// Fused persistent decode (one cooperative launch per token through all layers).
+size_t fused_decode_workspace_bytes();
+bool fused_decode_supported(const dfssm_dims_t& d, int B, const dfssm_layer_t* layers, int n);
+cudaError_t launch_fused_decode(const dfssm_layer_t* layers, int n_layers, float* hidden,
+                                float* const* conv_states, float* const* ssm_states, void* ws,
+                                cudaStream_t st, long long spin_limit);
+// Launches a kernel that waits on a counter nothing increments, with the given clock budget.
+cudaError_t launch_timeout_selftest(void* ws, cudaStream_t st, long long spin_limit);
+// Reads and clears the device error word of a fused-decode workspace region (synchronises st).
+int read_device_error(void* ws, cudaStream_t st, int* code);
 }  // namespace dfssm

@@ -168,11 +168,7 @@ __global__ void __launch_bounds__(kQuantThreads) quant_kernel(QuantArgs a) {
     }
   }
   if (tid == 0) {
-    float s = s0;
-    if (a.norm_w) {
-      const double rms = __dsqrt_rn(__dadd_rn(__ddiv_rn(ss, (double)a.n), 1e-5));
-      s = __double2float_rn(__ddiv_rn((double)s0, rms));
-    }
+    const float s = a.norm_w ? rms_scale(s0, ss, a.n) : s0;
     a.out.s[b] = s;
     if (a.dbg_s) a.dbg_s[b] = s;
   }
@@ -187,15 +183,11 @@ cudaError_t launch_quant(const QuantArgs& a, cudaStream_t st) {
 
 constexpr int kGemvThreads = 256;
 
-// LoRA-up epilogue for one (token b, row o); fp64 in the oracle's order.
+// LoRA-up epilogue for one (token b, row o).
 __device__ __forceinline__ void gemv_epilogue(const GemvArgs& a, int b, int row, int acc, float sW,
                                               float sA, const int8_t* wa, const float* tf,
                                               float s) {
-  double lora = 0.0;
-  for (int r = 0; r < a.rank; ++r) lora = dadd(lora, dmul((double)wa[r], (double)tf[r]));
-  const double scaffold = dmul(dmul((double)acc, (double)s), (double)sW);
-  const double corr = a.rank > 0 ? dmul((double)sA, lora) : 0.0;
-  const float yv = __double2float_rn(dadd(scaffold, corr));
+  const float yv = linear_out(acc, s, sW, sA, wa, tf, a.rank);
   if (a.resid) {
     float* h = a.resid + (size_t)b * a.ldr + row;
     *h = fadd(*h, yv);
@@ -214,10 +206,7 @@ __device__ __forceinline__ void gemv_stage(const GemvArgs& a, uint4* qsm, float 
   if (threadIdx.x < nb * DFSSM_MAX_RANK) {
     const int b = threadIdx.x / DFSSM_MAX_RANK, r = threadIdx.x % DFSSM_MAX_RANK;
     float v = 0.0f;
-    if (r < a.rank)
-      v = __double2float_rn(
-          dmul(dmul((double)a.in.t[b * DFSSM_MAX_RANK + r], (double)a.lora_b_scale[r]),
-               (double)a.in.s[b]));
+    if (r < a.rank) v = lora_tf(a.in.t[b * DFSSM_MAX_RANK + r], a.lora_b_scale[r], a.in.s[b]);
     tf[b][r] = v;
   }
   if (threadIdx.x < nb) {

@@ -47,13 +47,7 @@ __global__ void __launch_bounds__(256) conv_step_kernel(ConvArgs a) {
   float* st = a.state + (size_t)idx * 3;
   const float s0 = st[0], s1 = st[1], s2 = st[2];
   const float xv = a.x_in[(size_t)b * a.ldx + c];
-  double e = (double)bias;
-  e = dadd(e, dmul((double)w.x, (double)s0));
-  e = dadd(e, dmul((double)w.y, (double)s1));
-  e = dadd(e, dmul((double)w.z, (double)s2));
-  e = dadd(e, dmul((double)w.w, (double)xv));
-  const float pre = __double2float_rn(e);
-  a.x_out[(size_t)b * a.ldo + c] = silu_f64(pre);
+  a.x_out[(size_t)b * a.ldo + c] = conv_out(w, bias, s0, s1, s2, xv);
   st[0] = s1;
   st[1] = s2;
   st[2] = xv;
@@ -69,10 +63,6 @@ cudaError_t launch_conv(const ConvArgs& a, cudaStream_t st) {
 //   v = fl32(dt_raw + dt_bias); dt = fl32(softplus(v)); A = fl32(-exp(A_log)); dA = fl32(exp(fl32(dt*A)))
 //   dtx = fl32(dt*x);  S <- fl32(fl32(dA*S) + fl32(dtx*B));  y = fl32(sum_n S*C + D*x)  (fp64 sum)
 // Optional gate: y <- fl32(y * fl32(SiLU(z))).
-
-__device__ __forceinline__ float softplus_f64(float v) {
-  return v > 20.0f ? v : __double2float_rn(log1p(exp((double)v)));
-}
 
 __global__ void __launch_bounds__(256) ssm_step_kernel(SsmArgs a) {
   const int warp_g = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
@@ -94,10 +84,8 @@ __global__ void __launch_bounds__(256) ssm_step_kernel(SsmArgs a) {
   pdl_wait();
   if (!valid) return;
 
-  const float v = fadd(a.dt_raw[(size_t)b * a.lddt + h], dt_bias);
-  const float dt = softplus_f64(v);
-  const float A = __double2float_rn(-exp((double)A_log));
-  const float dA = __double2float_rn(exp((double)fmul(dt, A)));
+  const float dt = ssm_dt(a.dt_raw[(size_t)b * a.lddt + h], dt_bias);
+  const float dA = ssm_dA(dt, A_log);
   const float xv = a.x[(size_t)b * a.ldx + hp];
   const float dtx = fmul(dt, xv);
 
@@ -109,10 +97,10 @@ __global__ void __launch_bounds__(256) ssm_step_kernel(SsmArgs a) {
     float4 s4 = ld_evict_first_f4(S + 4 * n4);
     const float4 b4 = *reinterpret_cast<const float4*>(Bg + 4 * n4);
     const float4 c4 = *reinterpret_cast<const float4*>(Cg + 4 * n4);
-    s4.x = fadd(fmul(dA, s4.x), fmul(dtx, b4.x));
-    s4.y = fadd(fmul(dA, s4.y), fmul(dtx, b4.y));
-    s4.z = fadd(fmul(dA, s4.z), fmul(dtx, b4.z));
-    s4.w = fadd(fmul(dA, s4.w), fmul(dtx, b4.w));
+    s4.x = ssm_state(dA, s4.x, dtx, b4.x);
+    s4.y = ssm_state(dA, s4.y, dtx, b4.y);
+    s4.z = ssm_state(dA, s4.z, dtx, b4.z);
+    s4.w = ssm_state(dA, s4.w, dtx, b4.w);
     acc = fma((double)s4.x, (double)c4.x, acc);  // products of two fp32 are exact in fp64
     acc = fma((double)s4.y, (double)c4.y, acc);
     acc = fma((double)s4.z, (double)c4.z, acc);

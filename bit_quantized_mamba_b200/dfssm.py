@@ -70,6 +70,8 @@ SIGNATURES = {
     "dfssm_layer_decode": (_I, [_P, _I, _P, _P, _P, _P, _I, _P, _Z, _P]),
     "dfssm_lm_head": (_I, [_P, _P, _I, _I, _P, _P, _P, _P, _Z, _P]),
     "dfssm_pack_signs": (_I, [_P, _I, _I, _P]),
+    "dfssm_device_status": (_I, [_P, _P]),
+    "dfssm_selftest_timeout": (_I, [_P, _Z, _P]),
     "dfssm_status_string": (C.c_char_p, [_I]),
     "dfssm_last_cuda_error": (C.c_char_p, []),
     "dfssm_abi_version": (_I, []),
@@ -119,8 +121,8 @@ def workspace_size(op: int, a: int, b: int, c: int) -> int:
 
 
 def workspace(nbytes: int, device="cuda") -> torch.Tensor:
-    """Caller-owned scratch (torch allocations are 512-byte aligned)."""
-    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+    """Caller-owned scratch, zero-filled (torch allocations are 512-byte aligned)."""
+    return torch.zeros(max(int(nbytes), 256), dtype=torch.uint8, device=device)
 
 
 class Linear:
@@ -249,6 +251,16 @@ def layer_decode(stack: LayerStack, hidden: torch.Tensor, ws=None, stream=None) 
         stack._layers, stack.n, C.byref(stack.dims), _ptr(hidden), stack._conv, stack._ssm, B,
         _ptr(ws), ws.numel(), _stream(stream)))
     return hidden
+
+
+def device_status(ws, stream=None) -> int:
+    """Synchronise the stream, read and clear the fused-decode error word: 0 (DFSSM_OK) or -5."""
+    return int(lib().dfssm_device_status(_ptr(ws), _stream(stream)))
+
+
+def selftest_timeout(ws, stream=None) -> None:
+    _check("dfssm_selftest_timeout", lib().dfssm_selftest_timeout(_ptr(ws), ws.numel(),
+                                                                  _stream(stream)))
 
 
 def lm_head(W, s_row, x, logits=None, acc=None, ws=None, stream=None):

@@ -175,6 +175,21 @@ int dfssm_layer_decode(const dfssm_layer_t* layers, int n_layers, const dfssm_di
 int dfssm_lm_head(const int8_t* W, const float* s_row, int V, int d, const float* x, float* logits,
                   int32_t* acc, void* workspace, size_t ws_bytes, void* stream);
 
+/*
+ * Device-side failure detection of dfssm_layer_decode.  The fused decode kernel (batch 1, Mamba-2-1.3B
+ * shape) hands data between its CTAs through counters in the workspace; every wait has a clock budget
+ * (about one second).  A wait that runs out makes every CTA of that launch return early (its outputs are
+ * then incomplete) and records a sticky status word in the workspace; each new launch starts with fresh
+ * counters.  dfssm_device_status synchronises `stream`, reads and clears the status word, and returns
+ * DFSSM_OK or DFSSM_ETIMEOUT.  No device trap or fault is ever raised.
+ */
+int dfssm_device_status(void* workspace, void* stream);
+
+/* Diagnostic: launch a one-warp kernel that waits, with a budget of about 1 ms, on a workspace counter
+ * that nothing increments, so that the next dfssm_device_status returns DFSSM_ETIMEOUT.  workspace as
+ * for dfssm_layer_decode. */
+int dfssm_selftest_timeout(void* workspace, size_t ws_bytes, void* stream);
+
 /* Host helper: pack a +-1 int8 matrix [d_out][d_in] (row-major, host) into the bit layout above
  * (host u32 [d_out][d_in/32]).  Any value > 0 maps to a set bit. */
 int dfssm_pack_signs(const int8_t* signs, int d_out, int d_in, uint32_t* bits);

@@ -240,3 +240,37 @@ def test_lm_head(dev):
     rl, racc = oracle.lm_head(p["lm_w"], p["lm_s"], x)
     assert np.array_equal(acc.cpu().numpy(), racc)
     assert assert_tol(logits, rl, "lm head") == 0
+
+
+FULL = dict(d_model=2048, nheads=64, headdim=64, d_state=128, ngroups=1)
+
+
+def test_layer_decode_fused_few_layers(dev):
+    """Batch 1 at the 1.3B shape runs the fused persistent kernel: 3 layers x 5 tokens."""
+    model = inputs.decode_model(seed=12, n_layers=3, n_tokens=5)
+    assert _decode_compare(dev, model, FULL, 1, 5) <= 4
+
+
+def test_layer_decode_chain_full_dims_batch2(dev):
+    """Batch 2 at the 1.3B shape runs the per-op kernel chain."""
+    model = inputs.decode_model(seed=13, n_layers=2, n_tokens=3, batch=2)
+    assert _decode_compare(dev, model, FULL, 2, 3) <= 4
+
+
+def test_device_wait_timeout_is_reported(dev):
+    """A device-side wait that can never complete runs out of its budget, records DFSSM_ETIMEOUT and
+    returns; the status read clears it and the workspace is usable again."""
+    from bit_quantized_mamba_b200 import dfssm
+    ws = dfssm.workspace(dfssm.workspace_size(dfssm.OP_LAYER_DECODE, 1, 2048, 4096), dev)
+    assert dfssm.device_status(ws) == 0
+    dfssm.selftest_timeout(ws)
+    assert dfssm.device_status(ws) == -5
+    assert dfssm.device_status(ws) == 0
+    model = inputs.decode_model(seed=14, n_layers=1, n_tokens=1)
+    stack, olayers, conv, ssm = _stack(model, FULL, 1, dev)
+    h = to_dev(model["emb"][0], dev)
+    dfssm.layer_decode(stack, h, ws)
+    assert dfssm.device_status(ws) == 0
+    h_ref = np.ascontiguousarray(model["emb"][0])
+    oracle.layer_decode(olayers[0], h_ref, conv[0], ssm[0])
+    assert_tol(h.cpu().numpy(), h_ref, "decode after a reported timeout")
