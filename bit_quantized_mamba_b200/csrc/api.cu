@@ -105,6 +105,8 @@ dfssm::GemvArgs gemv_args(const dfssm_linear_t* L, int B, const dfssm::QuantScra
 
 }  // namespace
 
+int dfssm::record_cuda_failure(cudaError_t e) { return cuda_fail(e); }
+
 extern "C" {
 
 int dfssm_abi_version(void) { return DFSSM_ABI_VERSION; }

@@ -109,4 +109,6 @@ cudaError_t launch_fused_decode(const dfssm_layer_t* layers, int n_layers, float
 cudaError_t launch_timeout_selftest(void* ws, cudaStream_t st, long long spin_limit);
 // Reads and clears the device error word of a fused-decode workspace region (synchronises st).
 int read_device_error(void* ws, cudaStream_t st, int* code);
+// Records e as the text returned by dfssm_last_cuda_error (this thread) and returns DFSSM_ECUDA.
+int record_cuda_failure(cudaError_t e);
 }  // namespace dfssm

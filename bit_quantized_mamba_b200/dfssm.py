@@ -65,6 +65,7 @@ SIGNATURES = {
     "dfssm_workspace_size": (_Z, [_I, _I, _I, _I]),
     "dfssm_linear_decode": (_I, [_P, _P, _I, _P, _P, _Z, _P, _P]),
     "dfssm_linear_prefill": (_I, [_P, _P, _I, _P, _P, _Z, _P, _P]),
+    "dfssm_linear_decode_noalloc": (_I, [_P, _P, _I, _P, _P, _P]),
     "dfssm_conv_step": (_I, [_P, _P, _P, _P, _P, _I, _I, _P]),
     "dfssm_ssm_step": (_I, [_P] * 9 + [_I] * 5 + [_P]),
     "dfssm_layer_decode": (_I, [_P, _I, _P, _P, _P, _P, _I, _P, _Z, _P]),
@@ -165,6 +166,21 @@ def linear_decode(lin: Linear, x: torch.Tensor, y: torch.Tensor | None = None, w
     _check("dfssm_linear_decode", lib().dfssm_linear_decode(
         C.byref(lin.cstruct()), _ptr(x), B, _ptr(y), _ptr(ws), ws.numel(),
         C.byref(dbg) if dbg is not None else None, _stream(stream)))
+    return y
+
+
+def linear_decode_noalloc(lin: Linear, x: torch.Tensor, y: torch.Tensor | None = None,
+                          debug: dict | None = None, stream=None) -> torch.Tensor:
+    """dfssm_linear_decode without a workspace (the library keeps a fixed scratch array per device)."""
+    B = x.shape[0]
+    if y is None:
+        y = torch.empty((B, lin.d_out), dtype=torch.float32, device=x.device)
+    dbg = None
+    if debug is not None:
+        dbg = DebugT(*(_ptr(debug.get(k)) for k in ("acc", "lora_t", "xq", "xscale")))
+    _check("dfssm_linear_decode_noalloc", lib().dfssm_linear_decode_noalloc(
+        C.byref(lin.cstruct()), _ptr(x), B, _ptr(y), C.byref(dbg) if dbg is not None else None,
+        _stream(stream)))
     return y
 
 

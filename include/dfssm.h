@@ -103,6 +103,23 @@ int dfssm_linear_decode(const dfssm_linear_t* lin, const float* x, int B, float*
                         size_t ws_bytes, const dfssm_debug_t* dbg, void* stream);
 
 /*
+ * dfssm_linear_decode for callers that cannot allocate device memory.  The paper has no counterpart: this
+ * is a deployment variant of the same computation, with the same arguments and results except that there
+ * is no workspace.  It serves code that may only hand the library its inputs and outputs — a plugin whose
+ * host process owns every device allocation, or a real-time loop that must not call cudaMalloc because it
+ * can block and synchronise the device.
+ *   Limits: 1 <= B <= 16 and d_in <= 8192; larger sizes return DFSSM_EUNSUPPORTED before anything runs.
+ *   Scratch: a fixed 132,608-byte array in the library's own device memory, held by every device that
+ *   loads the library until the process exits.  The call allocates and frees nothing.
+ *   Set-up: the first call on a device looks up that array's device address (cudaGetSymbolAddress, with
+ *   that device current) and caches it; make that first call before any stream capture.
+ *   Sharing: all calls on a device use the same array.  Each call writes everything it reads there, so
+ *   nothing needs clearing, but calls that overlap on the GPU (unordered streams) race: order them.
+ */
+int dfssm_linear_decode_noalloc(const dfssm_linear_t* lin, const float* x, int B, float* y,
+                                const dfssm_debug_t* dbg, void* stream);
+
+/*
  * M-token prefill of one linear on int8 tcgen05 tensor cores (technical summary §2.C: the scaffold
  * matmul on INT8 tensor cores).  Same math as dfssm_linear_decode, per row of x.
  *   x device f32 [M][d_in], y device f32 [M][d_out], M >= 1.  d_in % 128 == 0 required.
