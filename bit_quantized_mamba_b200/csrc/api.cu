@@ -182,13 +182,14 @@ int dfssm_linear_decode(const dfssm_linear_t* lin, const float* x, int B, float*
   qa.n = lin->d_in;
   qa.B = B;
   qa.lora_b = lin->lora_b;
+  qa.lora_b_scale = lin->lora_b_scale;
   qa.rank = lin->rank;
   qa.permute = true;
   qa.out = qs;
   if (dbg) {
     qa.dbg_xq = dbg->xq;
     qa.dbg_s = dbg->xscale;
-    qa.dbg_t = dbg->lora_t;
+    qa.dbg_tf = dbg->lora_tf;
   }
   cudaError_t e = dfssm::launch_quant(qa, s);
   if (e != cudaSuccess) return cuda_fail(e);
@@ -293,6 +294,7 @@ int dfssm_layer_decode(const dfssm_layer_t* layers, int n_layers, const dfssm_di
     qa.n = Dm;
     qa.B = B;
     qa.lora_b = Ly.in_proj.lora_b;
+    qa.lora_b_scale = Ly.in_proj.lora_b_scale;
     qa.rank = Ly.in_proj.rank;
     qa.permute = true;
     qa.out = w.qs;
@@ -338,6 +340,7 @@ int dfssm_layer_decode(const dfssm_layer_t* layers, int n_layers, const dfssm_di
     qa.norm_w = Ly.gnorm_w;
     qa.n = E;
     qa.lora_b = Ly.out_proj.lora_b;
+    qa.lora_b_scale = Ly.out_proj.lora_b_scale;
     qa.rank = Ly.out_proj.rank;
     e = dfssm::launch_quant(qa, s);
     if (e != cudaSuccess) break;

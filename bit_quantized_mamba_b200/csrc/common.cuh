@@ -92,6 +92,15 @@ __device__ __forceinline__ int quant_code(float v, float s0) {
   r = fminf(fmaxf(r, -127.0f), 127.0f);
   return (int)r;
 }
+// Same code, computed as rint(v * fl32(1/s0)) unless that product lies within 1e-3 of a rounding
+// boundary: |v/s0| <= 127, and both v*fl32(1/s0) and fl32(v/s0) are within 2e-5 of v/s0, so away from a
+// boundary they round to the same integer; near one, the IEEE division decides.
+__device__ __forceinline__ int quant_code_fast(float v, float s0, float inv_s0) {
+  const float t = v * inv_s0;
+  const float k = rintf(t);
+  if (fabsf(t - k) < 0.499f) return (int)fminf(fmaxf(k, -127.0f), 127.0f);
+  return quant_code(v, s0);
+}
 
 // Position of natural-order activation index i inside the dp4a-friendly permuted layout: within each
 // 32-element block, word k (k = 0..7) holds elements k, k+8, k+16, k+24 in its four bytes.  With that
@@ -115,14 +124,23 @@ __device__ __forceinline__ float linear_out(int acc, float s, float sW, float sA
   return __double2float_rn(dadd(scaffold, corr));
 }
 
-// LoRA intermediate tf = fl32(t * sB * s) (fp64).
-__device__ __forceinline__ float lora_tf(int t, float sB, float s) {
-  return __double2float_rn(dmul(dmul((double)t, (double)sB), (double)s));
+// Exact fp64 value of a 32-bit integer without the (slow) integer-to-double conversion unit:
+// 2^52 + 2^31 + w read as a double, minus 2^52 + 2^31.
+__device__ __forceinline__ double int_to_f64(int w) {
+  return __hiloint2double(0x43300000, w ^ (int)0x80000000) - 4503601774854144.0;
 }
 
-// Scale of RMSNorm+quantize: fl32(s0 / sqrt(ss/n + 1e-5)) (fp64).
-__device__ __forceinline__ float rms_scale(float s0, double ss, int n) {
-  const double rms = __dsqrt_rn(__dadd_rn(__ddiv_rn(ss, (double)n), 1e-5));
+// LoRA intermediate tf = fl32(u * sB / rms) (fp64), u = sum_i W_B[r,i] v_i; rms = 1 for a plain linear.
+__device__ __forceinline__ float lora_tf(double u, float sB, double rms) {
+  return __double2float_rn(__ddiv_rn(dmul(u, (double)sB), rms));
+}
+
+// RMS of a row with sum of squares ss: sqrt(ss/n + 1e-5) (fp64); the quantizer scale of the normalized
+// row is fl32(s0 / rms).
+__device__ __forceinline__ double rms_of(double ss, int n) {
+  return __dsqrt_rn(__dadd_rn(__ddiv_rn(ss, (double)n), 1e-5));
+}
+__device__ __forceinline__ float rms_scale(float s0, double rms) {
   return __double2float_rn(__ddiv_rn((double)s0, rms));
 }
 

@@ -12,8 +12,10 @@
 // The weights and states of a CTA's slice are loaded into registers and shared memory at the start of
 // the layer (and prefetched into L2 one layer ahead), before the CTA waits on anything, so the HBM stream
 // overlaps the dependency chain.  Cross-CTA hand-offs go through global memory with monotonically
-// increasing counters (arrive = fence + atomic add; wait = bounded acquire spin).  A wait that runs past
-// its clock budget records DFSSM_ETIMEOUT in the workspace error word and the CTA returns.
+// increasing counters (arrive = CTA barrier + release add; wait = bounded relaxed spin + acquire fence),
+// three per layer.  The LoRA down-projection is linear in its fp32 input, so each CTA publishes its
+// partial sums over the rows it owns next to those rows, and no separate hand-off is needed for it.  A wait
+// that runs past its clock budget records DFSSM_ETIMEOUT in the workspace status word and the CTA returns.
 //
 // All arithmetic goes through the functions in common.cuh, so the results are those of the per-op path.
 
@@ -24,16 +26,14 @@ namespace dfssm {
 namespace fused {
 
 constexpr int DM = 2048, E = 4096, H = 64, P = 64, N = 128, R = 16;
-constexpr int CC = E + 2 * N;           // conv channels: x | B | C
-constexpr int DIP = 2 * E + 2 * N + H;  // in_proj rows: z | x | B | C | dt
-constexpr int SH0 = 2 * E;              // first row needed by every CTA (B rows, then C, then dt)
+constexpr int SH0 = 2 * E;              // first in_proj row every CTA needs (B rows, then C, then dt)
 constexpr int NSH = 2 * N + H;          // 320 such rows
-constexpr int NT = 512, NW = NT / 32;
+constexpr int NT = 512, NW = NT / 32;   // NW == R: warp r computes LoRA row r's partial sums
 constexpr int MAX_IN = 64, MAX_OUT = 16, MAX_SSM = 32;
-constexpr int NUM_T_PRODUCERS = R;      // CTAs [0, 16) produce t_in, [16, 32) produce t_out
-constexpr int kAuxThread = 32;         // computes the RMS scale while thread 0 polls
+constexpr int MIN_CTAS = 133, MAX_CTAS = 256;
+static_assert(NW == R, "one warp per LoRA row");
 
-enum { CTR_H = 0, CTR_BC, CTR_G, CTR_TOUT, N_CTR };
+enum { CTR_H = 0, CTR_BC, CTR_G, N_CTR };
 constexpr int CTR_STRIDE = 32;          // one 128-byte line per counter
 
 struct LayerPtrs {
@@ -67,34 +67,29 @@ struct Params {
   int* ctr;
   int* err;
   int* status;
-  int* tin;
-  int* tout;
   int* sacc;
   float* gbuf;
+  double* upin;   // [NC][R] LoRA-down partial sums of the next in_proj (one row per CTA)
+  double* upout;  // [NC][R] LoRA-down partial sums of out_proj
   long long spin_limit;
 };
 
 // ------------------------------------------------------------------------------ workspace layout
-// [counters N_CTR x 128 B][abort word 128 B][status word 128 B][t_in 16][t_out 16][sacc 320][gbuf 4096]
+// [counters N_CTR x 128 B][abort word 128 B][status word 128 B][sacc 320][gbuf 4096][upin][upout]
 // The counters and the abort word are cleared before every launch; the status word is sticky: a timed
 // out wait stores kTimeoutMagic there, and only dfssm_device_status clears it.
 constexpr size_t OFF_CTR = 0;
 constexpr size_t OFF_ERR = OFF_CTR + N_CTR * CTR_STRIDE * 4;
 constexpr size_t OFF_STATUS = OFF_ERR + 128;
 constexpr size_t CLEAR_BYTES = OFF_STATUS;  // counters + abort word
-constexpr size_t OFF_TIN = OFF_STATUS + 128;
-constexpr size_t OFF_TOUT = OFF_TIN + 64;
-constexpr size_t OFF_SACC = OFF_TOUT + 64;
+constexpr size_t OFF_SACC = OFF_STATUS + 128;
 constexpr size_t OFF_GBUF = OFF_SACC + ((NSH * 4 + 255) / 256) * 256;
-constexpr size_t WS_BYTES = OFF_GBUF + E * 4;
+constexpr size_t OFF_UIN = OFF_GBUF + E * 4;
+constexpr size_t OFF_UOUT = OFF_UIN + MAX_CTAS * R * 8;
+constexpr size_t WS_BYTES = OFF_UOUT + MAX_CTAS * R * 8;
 
 // ------------------------------------------------------------------------------ synchronisation
 
-__device__ __forceinline__ int ld_acquire(const int* p) {
-  int v;
-  asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
-}
 __device__ __forceinline__ int ld_relaxed(const int* p) {
   int v;
   asm volatile("ld.relaxed.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
@@ -155,40 +150,20 @@ __device__ __forceinline__ void prefetch_lines(const void* p, unsigned bytes) {
   for (; a < e; a += 128) asm volatile("prefetch.global.L2 [%0];" ::"l"(a) : "memory");
 }
 
-// ------------------------------------------------------------------------------ block reductions
-
-struct Red2 {
-  double ss;
-  float m;
-};
-
-__device__ __forceinline__ Red2 block_sum_max(double ss, float m, double* rd, float* rf) {
-  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-  ss = warp_sum(ss);
-  m = warp_max(m);
-  if (lane == 0) {
-    rd[w] = ss;
-    rf[w] = m;
-  }
-  __syncthreads();
-  double s2 = lane < NW ? rd[lane] : 0.0;
-  float m2 = lane < NW ? rf[lane] : 0.0f;
-  s2 = warp_sum(s2);
-  m2 = warp_max(m2);
-  __syncthreads();  // rd/rf may be reused right after
-  return Red2{s2, m2};
+// Asynchronous global -> shared copies (completion awaited with cp_async_wait_all before a barrier).
+__device__ __forceinline__ void cp_async4(void* dst, const void* src) {
+  const unsigned d = (unsigned)__cvta_generic_to_shared(dst);
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(d), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  const unsigned d = (unsigned)__cvta_generic_to_shared(dst);
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
 }
 
-__device__ __forceinline__ int block_sum_int(int v, int* ri) {
-  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-  v = warp_sum(v);
-  if (lane == 0) ri[w] = v;
-  __syncthreads();
-  int t = lane < NW ? ri[lane] : 0;
-  t = warp_sum(t);
-  __syncthreads();
-  return t;
-}
+// ------------------------------------------------------------------------------ GEMV inner loop
 
 // Shared-memory position of natural activation index i: the dp4a-permuted codes of 128-input segment
 // `seg` occupy eight 16-byte chunks, and chunk v of every segment is stored contiguously across the
@@ -222,18 +197,34 @@ __device__ __forceinline__ int bits_dot(uint4 w, const uint4* qp4) {
   return S;
 }
 
+// Sum of one LoRA row's partial sums: thread t adds the partials of row t % R from every CTA
+// (t + NT k); a warp then holds row r in lanes r and r + 16.
+__device__ __forceinline__ double gather_partials(const double* part, int NC) {
+  double u = 0.0;
+  for (int j = threadIdx.x; j < NC * R; j += NT) u += __ldcg(part + j);
+  return u + __shfl_xor_sync(0xffffffffu, u, 16);
+}
+
 // ------------------------------------------------------------------------------ the kernel
+//
+// Per layer (three hand-offs):
+//   A  wait h    -> RMSNorm+quantize h, LoRA-down from the partials, scaffold GEMV of the owned rows;
+//                   the B/C/dt rows' accumulators are published first (arrive B/C)
+//   B  wait B/C  -> epilogues (B/C conv, dt, own z gate, own x conv), SSM of the owned rows, g of the
+//                   owned rows and their LoRA-down partial sums published (arrive g)
+//   C  wait g    -> gated RMSNorm+quantize, out_proj GEMV of the owned rows, residual; the next layer's
+//                   in_proj LoRA-down partial sums over the owned rows published (arrive h)
+// A prologue publishes the first layer's in_proj partial sums from the input hidden state.
 
 __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ Params p) {
   __shared__ __align__(16) int8_t q_perm[E];
-  __shared__ __align__(16) int8_t q_nat[E];
   __shared__ double red_d[NW];
   __shared__ float red_f[NW];
   __shared__ int red_i[NW];
+  __shared__ double red_u[NW][R];
   __shared__ int sflag;
   __shared__ float tf[R];
   __shared__ float s_scale;
-  __shared__ int s_sumq;
   // in_proj rows owned by this CTA (slot order: shared rows, z rows, x rows)
   __shared__ int acc_in[MAX_IN];
   __shared__ float in_sw[MAX_IN], in_sa[MAX_IN];
@@ -241,18 +232,18 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ P
   // the 320 rows every CTA needs
   __shared__ float sh_sw[NSH], sh_sa[NSH];
   __shared__ __align__(16) int8_t sh_wa[NSH][R];
-  __shared__ float4 bc_w[2 * N];
+  __shared__ __align__(16) float4 bc_w[2 * N];
   __shared__ float bc_b[2 * N];
   __shared__ float bc_st[2 * N][3];
   __shared__ float bc_new[2 * N];
   __shared__ __align__(16) float Bsm[N];
   __shared__ __align__(16) float Csm[N];
   // SSM rows
-  __shared__ float zsm[MAX_SSM], xsm[MAX_SSM];
+  __shared__ float zsm[MAX_SSM], xsm[MAX_SSM], gsm[MAX_SSM];
   __shared__ float dtv[2], dAv[2], Dv[2];
   // out_proj rows
   __shared__ int acc_out[MAX_OUT];
-  __shared__ float o_sw[MAX_OUT], o_sa[MAX_OUT];
+  __shared__ float o_sw[MAX_OUT], o_sa[MAX_OUT], h_old[MAX_OUT], h_new[MAX_OUT];
   __shared__ __align__(16) int8_t o_wa[MAX_OUT][R];
 
   const int c = blockIdx.x, NC = gridDim.x;
@@ -270,19 +261,34 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ P
     const int j = slot - n_sh;
     return j < n_ssm ? rs0 + j : E + rs0 + (j - n_ssm);
   };
-
-  // per-thread GEMV / SSM positions
   const int li_in = lane & 15;
   const int slot_in[2] = {warp * 2 + (lane >> 4), 32 + warp * 2 + (lane >> 4)};
   const int slot_out = warp;  // out_proj: one row per warp, 32 lanes x 128 weights
   const int ssm_slot[2] = {warp, NW + warp};
+  const int dt_head = tid - 2 * N;  // threads [256, 320) own the dt rows
+  const bool dt_own = tid >= 2 * N && tid < NSH && (dt_head == hA || dt_head == hA + 1);
+
+  // ---- prologue: the first layer's in_proj LoRA-down partial sums over this CTA's hidden rows
+  {
+    const LayerPtrs& L0 = p.L[0];
+    double part = 0.0;
+    if (lane < n_out) {
+      const int o = ro0 + lane;
+      const float v = fmul(__ldcg(p.hidden + o), __ldg(L0.norm_w + o));
+      part = int_to_f64((int)L0.in_lb[(size_t)warp * DM + o]) * (double)v;
+    }
+    part = warp_sum(part);
+    if (lane == 0) p.upin[c * R + warp] = part;
+    block_arrive(p.ctr + CTR_H * CTR_STRIDE);
+  }
 
   for (int l = 0; l < p.n_layers; ++l) {
     const LayerPtrs& Lp = p.L[l];
+    const bool has_next = l + 1 < p.n_layers;
 
     // ---------------------------------------------------------------- loads for the whole layer
-    if (tid < 2 && l + 1 < p.n_layers) {
-      // this CTA's slice of the next layer, and (spread over CTAs 0..31) the parts every CTA reads
+    if (tid < 2 && has_next) {
+      // this CTA's slice of the next layer, and (spread over CTAs 0..4) the parts every CTA reads
       const LayerPtrs& Nx = p.L[l + 1];
       if (tid == 0) {
         prefetch_l2(Nx.in_bits + (size_t)(SH0 + sh0) * (DM / 32), n_sh * (DM / 8));
@@ -303,8 +309,6 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ P
         prefetch_lines(Nx.out_las + ro0, n_out * 4);
         prefetch_lines(Nx.conv_b + rs0, n_ssm * 4);
         prefetch_lines(Nx.conv_state + (size_t)rs0 * 3, n_ssm * 12);
-        if (c < NUM_T_PRODUCERS) prefetch_l2(Nx.in_lb + (size_t)c * DM, DM);
-        else if (c < 2 * NUM_T_PRODUCERS) prefetch_l2(Nx.out_lb + (size_t)(c - NUM_T_PRODUCERS) * E, E);
         switch (c) {
           case 0: prefetch_l2(Nx.norm_w, DM * 4); break;
           case 1: prefetch_l2(Nx.gnorm_w, E * 4); break;
@@ -329,6 +333,7 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ P
         }
       }
     }
+    // registers: sign bits, SSM state rows, norm weights, LoRA columns of the owned rows
     uint4 w_in[2], w_out;
 #pragma unroll
     for (int ps = 0; ps < 2; ++ps) {
@@ -345,42 +350,28 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ P
       sv[ps] = rr < n_ssm ? ld_evict_first_f4(Lp.ssm_state + (size_t)(rs0 + rr) * N + lane * 4)
                           : make_float4(0.f, 0.f, 0.f, 0.f);
     }
-    float nw[4];
+    float nw[4], gw[8];
 #pragma unroll
     for (int k = 0; k < 4; ++k) nw[k] = __ldg(Lp.norm_w + tid + k * NT);
-    uint32_t wb_in = 0;
-    uint2 wb_out = make_uint2(0, 0);
-    if (c < NUM_T_PRODUCERS) wb_in = ld_stream_u32(Lp.in_lb + (size_t)c * DM + 4 * tid);
-    if (c >= NUM_T_PRODUCERS && c < 2 * NUM_T_PRODUCERS) {
-      const int8_t* rowp = Lp.out_lb + (size_t)(c - NUM_T_PRODUCERS) * E + 8 * tid;
-      wb_out = make_uint2(ld_stream_u32(rowp), ld_stream_u32(rowp + 4));
+#pragma unroll
+    for (int k = 0; k < 8; ++k) gw[k] = __ldg(Lp.gnorm_w + tid + k * NT);
+    // warp r, lane j: out_proj LoRA column of owned SSM row j, and the next in_proj LoRA column of owned
+    // hidden row j (with its next norm weight)
+    int wbo = 0, wbi_next = 0;
+    float gw_own = 0.f, nw_next = 0.f;
+    if (lane < n_ssm) {
+      wbo = (int)Lp.out_lb[(size_t)warp * E + rs0 + lane];
+      gw_own = __ldg(Lp.gnorm_w + rs0 + lane);
     }
-    // epilogue parameters into shared memory
-    if (tid < n_in) {
-      const int row = in_row(tid);
-      in_sw[tid] = __ldg(Lp.in_ws + row);
-      in_sa[tid] = __ldg(Lp.in_las + row);
-      *reinterpret_cast<uint4*>(in_wa[tid]) = ld_stream_u4(Lp.in_la + (size_t)row * R);
+    if (has_next && lane < n_out) {
+      const LayerPtrs& Nx = p.L[l + 1];
+      wbi_next = (int)Nx.in_lb[(size_t)warp * DM + ro0 + lane];
+      nw_next = __ldg(Nx.norm_w + ro0 + lane);
     }
-    if (tid < NSH) {
-      const int row = SH0 + tid;
-      sh_sw[tid] = __ldg(Lp.in_ws + row);
-      sh_sa[tid] = __ldg(Lp.in_las + row);
-      *reinterpret_cast<uint4*>(sh_wa[tid]) = __ldg(reinterpret_cast<const uint4*>(Lp.in_la) + row);
-    }
-    if (tid < 2 * N) {
-      const int ch = E + tid;
-      bc_w[tid] = __ldg(reinterpret_cast<const float4*>(Lp.conv_w) + ch);
-      bc_b[tid] = __ldg(Lp.conv_b + ch);
-      bc_st[tid][0] = __ldcg(Lp.conv_state + (size_t)ch * 3 + 0);
-      bc_st[tid][1] = __ldcg(Lp.conv_state + (size_t)ch * 3 + 1);
-      bc_st[tid][2] = __ldcg(Lp.conv_state + (size_t)ch * 3 + 2);
-    }
-    if (tid < n_out) {
-      const int row = ro0 + tid;
-      o_sw[tid] = __ldg(Lp.out_ws + row);
-      o_sa[tid] = __ldg(Lp.out_las + row);
-      *reinterpret_cast<uint4*>(o_wa[tid]) = ld_stream_u4(Lp.out_la + (size_t)row * R);
+    float lbs_in = 0.f, lbs_out = 0.f;
+    if (tid < R) {
+      lbs_in = __ldg(Lp.in_lbs + tid);
+      lbs_out = __ldg(Lp.out_lbs + tid);
     }
     // own x channels: conv taps, bias, state (thread NSH + j handles channel rs0 + j)
     float4 cw = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -393,51 +384,99 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ P
       cs1 = Lp.conv_state[(size_t)ch * 3 + 1];
       cs2 = Lp.conv_state[(size_t)ch * 3 + 2];
     }
-    if (tid < 2) {
-      const int h = hA + tid;
-      if (h < H) Dv[tid] = __ldg(Lp.D + h);
+    float dtb = 0.f, A_h = 0.f;
+    if (dt_own) {
+      dtb = __ldg(Lp.dt_bias + dt_head);
+      A_h = __double2float_rn(-exp((double)__ldg(Lp.A_log + dt_head)));
     }
+    // epilogue parameters into shared memory, asynchronously
+    if (tid < n_in) {
+      const int row = in_row(tid);
+      cp_async4(&in_sw[tid], Lp.in_ws + row);
+      cp_async4(&in_sa[tid], Lp.in_las + row);
+      cp_async16(in_wa[tid], Lp.in_la + (size_t)row * R);
+    }
+    if (tid < NSH) {
+      const int row = SH0 + tid;
+      cp_async4(&sh_sw[tid], Lp.in_ws + row);
+      cp_async4(&sh_sa[tid], Lp.in_las + row);
+      cp_async16(sh_wa[tid], Lp.in_la + (size_t)row * R);
+    }
+    if (tid < 2 * N) {
+      const int ch = E + tid;
+      cp_async16(&bc_w[tid], Lp.conv_w + (size_t)ch * 4);
+      cp_async4(&bc_b[tid], Lp.conv_b + ch);
+      cp_async4(&bc_st[tid][0], Lp.conv_state + (size_t)ch * 3 + 0);
+      cp_async4(&bc_st[tid][1], Lp.conv_state + (size_t)ch * 3 + 1);
+      cp_async4(&bc_st[tid][2], Lp.conv_state + (size_t)ch * 3 + 2);
+    }
+    if (tid < n_out) {
+      const int row = ro0 + tid;
+      cp_async4(&o_sw[tid], Lp.out_ws + row);
+      cp_async4(&o_sa[tid], Lp.out_las + row);
+      cp_async16(o_wa[tid], Lp.out_la + (size_t)row * R);
+    }
+    if (tid < 2 && hA + tid < H) cp_async4(&Dv[tid], Lp.D + hA + tid);
+    cp_async_wait_all();
 
     // ---------------------------------------------------------------- phase A: h -> in_proj
-    if (l > 0 && !block_wait(p.ctr + CTR_H * CTR_STRIDE, NC * l, p.err, p.status, p.spin_limit, &sflag)) return;
-    double ssA;
-    float s0A;
+    if (!block_wait(p.ctr + CTR_H * CTR_STRIDE, NC * (l + 1), p.err, p.status, p.spin_limit, &sflag))
+      return;
     {
-      float hv[4], v[4];
+      float v[4];
       double ss = 0.0;
       float m = 0.0f;
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
-        hv[k] = __ldcg(p.hidden + tid + k * NT);
-        ss += (double)hv[k] * (double)hv[k];
-        v[k] = fmul(hv[k], nw[k]);
+        const float hv = __ldcg(p.hidden + tid + k * NT);
+        ss += (double)hv * (double)hv;
+        v[k] = fmul(hv, nw[k]);
         m = fmaxf(m, fabsf(v[k]));
       }
-      const Red2 r = block_sum_max(ss, m, red_d, red_f);
-      const float s0 = r.m == 0.0f ? 0.0f : __fdiv_rn(r.m, 127.0f);
+      if (tid < n_out) h_old[tid] = __ldcg(p.hidden + ro0 + tid);
+      const double u = gather_partials(p.upin, NC);
+      ss = warp_sum(ss);
+      m = warp_max(m);
+      if (lane == 0) {
+        red_d[warp] = ss;
+        red_f[warp] = m;
+      }
+      if (lane < R) red_u[warp][lane] = u;
+      __syncthreads();
+      ss = 0.0;
+      m = 0.0f;
+#pragma unroll
+      for (int w = 0; w < NW; ++w) {
+        ss += red_d[w];
+        m = fmaxf(m, red_f[w]);
+      }
+      const float s0 = m == 0.0f ? 0.0f : __fdiv_rn(m, 127.0f);
+      const float inv_s0 = m == 0.0f ? 0.0f : __frcp_rn(s0);
       int sq = 0;
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
-        const int i = tid + k * NT;
-        const int code = r.m == 0.0f ? 0 : quant_code(v[k], s0);
-        q_nat[i] = (int8_t)code;
-        q_perm[seg_index<DM / 128>(i)] = (int8_t)code;
+        const int code = m == 0.0f ? 0 : quant_code_fast(v[k], s0, inv_s0);
+        q_perm[seg_index<DM / 128>(tid + k * NT)] = (int8_t)code;
         sq += code;
       }
-      sq = block_sum_int(sq, red_i);  // its internal barriers also publish q_nat / q_perm
-      if (tid == 0) s_sumq = sq;
-      ssA = r.ss;
-      s0A = s0;
+      sq = warp_sum(sq);
+      if (lane == 0) red_i[warp] = sq;
+      if (tid <= R) {
+        const double rms = rms_of(ss, DM);
+        if (tid < R) {
+          double ut = 0.0;
+#pragma unroll
+          for (int w = 0; w < NW; ++w) ut += red_u[w][tid];
+          tf[tid] = lora_tf(ut, lbs_in, rms);
+        } else {
+          s_scale = rms_scale(s0, rms);
+        }
+      }
+      __syncthreads();
     }
-    // LoRA-down producers: t_in[c] = sum_i W_B[c,i] q_i.  It is written before this CTA's B/C arrival,
-    // so a CTA that has seen every B/C arrival also sees every t_in.
-    if (c < NUM_T_PRODUCERS) {
-      const int t = block_sum_int(dp4a_ss(wb_in, reinterpret_cast<const uint32_t*>(q_nat)[tid], 0),
-                                  red_i);
-      if (tid == 0) p.tin[c] = t;
-    }
-    __syncthreads();
-    const int sumq_in = s_sumq;
+    int sumq = 0;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) sumq += red_i[w];
     // scaffold GEMV over the owned rows; pass 0 holds the rows every CTA needs
     {
       const uint4* qp4 = reinterpret_cast<const uint4*>(q_perm) + li_in;
@@ -446,7 +485,7 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ P
         int S = bits_dot<DM / 128>(w_in[ps], qp4);
 #pragma unroll
         for (int o = 8; o > 0; o >>= 1) S += __shfl_xor_sync(0xffffffffu, S, o);
-        if (li_in == 0 && slot_in[ps] < n_in) acc_in[slot_in[ps]] = 2 * S - sumq_in;
+        if (li_in == 0 && slot_in[ps] < n_in) acc_in[slot_in[ps]] = 2 * S - sumq;
         if (ps == 0) {
           __syncthreads();
           if (tid < n_sh) p.sacc[sh0 + tid] = acc_in[tid];
@@ -454,12 +493,11 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ P
         }
       }
     }
-    if (tid == kAuxThread) s_scale = rms_scale(s0A, ssA, DM);
+
+    // ---------------------------------------------------------------- phase B: epilogues + SSM
     if (!block_wait(p.ctr + CTR_BC * CTR_STRIDE, NC * (l + 1), p.err, p.status, p.spin_limit, &sflag))
       return;
     const float s_in = s_scale;
-    if (tid < R) tf[tid] = lora_tf(__ldcg(p.tin + tid), __ldg(Lp.in_lbs + tid), s_in);
-    __syncthreads();
     if (tid < NSH) {
       // rows every CTA needs: B, C (conv + SiLU) and dt of this CTA's heads
       const float y = linear_out(__ldcg(p.sacc + tid), s_in, sh_sw[tid], sh_sa[tid], sh_wa[tid], tf, R);
@@ -468,13 +506,10 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ P
         const float xc = conv_out(bc_w[tid], bc_b[tid], bc_st[tid][0], bc_st[tid][1], bc_st[tid][2], y);
         if (tid < N) Bsm[tid] = xc;
         else Csm[tid - N] = xc;
-      } else {
-        const int h = tid - 2 * N;
-        if (h == hA || h == hA + 1) {
-          const float dt = ssm_dt(y, __ldg(Lp.dt_bias + h));
-          dtv[h - hA] = dt;
-          dAv[h - hA] = ssm_dA(dt, __ldg(Lp.A_log + h));
-        }
+      } else if (dt_own) {
+        const float dt = ssm_dt(y, dtb);
+        dtv[dt_head - hA] = dt;
+        dAv[dt_head - hA] = __double2float_rn(exp((double)fmul(dt, A_h)));
       }
     } else if (tid - NSH < n_ssm) {
       // the owned z rows (gate value SiLU(z) kept) and x rows (conv of the owned x channels)
@@ -489,11 +524,11 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ P
       st[2] = xr;
     }
     __syncthreads();
-
-    // ---------------------------------------------------------------- phase B: SSM + gate
+    float4 snew[2];
 #pragma unroll
     for (int ps = 0; ps < 2; ++ps) {
       const int rr = ssm_slot[ps];
+      snew[ps] = sv[ps];
       if (rr < n_ssm) {
         const int hp = rs0 + rr;
         const int hi = hp / P - hA;
@@ -507,25 +542,36 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ P
         s4.y = ssm_state(dA, s4.y, dtx, b4.y);
         s4.z = ssm_state(dA, s4.z, dtx, b4.z);
         s4.w = ssm_state(dA, s4.w, dtx, b4.w);
+        snew[ps] = s4;
         double acc = (double)s4.x * (double)c4.x;
         acc = fma((double)s4.y, (double)c4.y, acc);
         acc = fma((double)s4.z, (double)c4.z, acc);
         acc = fma((double)s4.w, (double)c4.w, acc);
-        st_f4(Lp.ssm_state + (size_t)hp * N + lane * 4, s4);
         acc = warp_sum(acc);
         if (lane == 0) {
           const float y = __double2float_rn(dadd(acc, dmul((double)Dv[hi], (double)xv)));
-          p.gbuf[hp] = fmul(y, zsm[rr]);
+          const float g = fmul(y, zsm[rr]);
+          gsm[rr] = g;
+          p.gbuf[hp] = g;
         }
       }
     }
+    __syncthreads();
+    {
+      // out_proj LoRA-down partial sums over the owned rows of g: warp r, lane j
+      double part = 0.0;
+      if (lane < n_ssm) part = int_to_f64(wbo) * (double)fmul(gsm[lane], gw_own);
+      part = warp_sum(part);
+      if (lane == 0) p.upout[c * R + warp] = part;
+    }
     block_arrive(p.ctr + CTR_G * CTR_STRIDE);
+#pragma unroll
+    for (int ps = 0; ps < 2; ++ps)
+      if (ssm_slot[ps] < n_ssm) st_f4(Lp.ssm_state + (size_t)(rs0 + ssm_slot[ps]) * N + lane * 4, snew[ps]);
 
     // ---------------------------------------------------------------- phase C: gated norm -> out_proj
-    float gw[8];
-#pragma unroll
-    for (int k = 0; k < 8; ++k) gw[k] = __ldg(Lp.gnorm_w + tid + k * NT);
-    if (!block_wait(p.ctr + CTR_G * CTR_STRIDE, NC * (l + 1), p.err, p.status, p.spin_limit, &sflag)) return;
+    if (!block_wait(p.ctr + CTR_G * CTR_STRIDE, NC * (l + 1), p.err, p.status, p.spin_limit, &sflag))
+      return;
     // every CTA has now read the old B/C conv state: the owners of those rows shift it
     for (int j = tid; j < n_sh; j += NT) {
       const int k = sh0 + j;
@@ -547,46 +593,69 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ P
         v[k] = fmul(g, gw[k]);
         m = fmaxf(m, fabsf(v[k]));
       }
-      const Red2 r = block_sum_max(ss, m, red_d, red_f);
-      const float s0 = r.m == 0.0f ? 0.0f : __fdiv_rn(r.m, 127.0f);
+      const double u = gather_partials(p.upout, NC);
+      ss = warp_sum(ss);
+      m = warp_max(m);
+      if (lane == 0) {
+        red_d[warp] = ss;
+        red_f[warp] = m;
+      }
+      if (lane < R) red_u[warp][lane] = u;
+      __syncthreads();
+      ss = 0.0;
+      m = 0.0f;
+#pragma unroll
+      for (int w = 0; w < NW; ++w) {
+        ss += red_d[w];
+        m = fmaxf(m, red_f[w]);
+      }
+      const float s0 = m == 0.0f ? 0.0f : __fdiv_rn(m, 127.0f);
+      const float inv_s0 = m == 0.0f ? 0.0f : __frcp_rn(s0);
       int sq = 0;
 #pragma unroll
       for (int k = 0; k < 8; ++k) {
-        const int i = tid + k * NT;
-        const int code = r.m == 0.0f ? 0 : quant_code(v[k], s0);
-        q_nat[i] = (int8_t)code;
-        q_perm[seg_index<E / 128>(i)] = (int8_t)code;
+        const int code = m == 0.0f ? 0 : quant_code_fast(v[k], s0, inv_s0);
+        q_perm[seg_index<E / 128>(tid + k * NT)] = (int8_t)code;
         sq += code;
       }
-      sq = block_sum_int(sq, red_i);
-      if (tid == 0) s_sumq = sq;
-      ssA = r.ss;
-      s0A = s0;
+      sq = warp_sum(sq);
+      if (lane == 0) red_i[warp] = sq;
+      if (tid <= R) {
+        const double rms = rms_of(ss, E);
+        if (tid < R) {
+          double ut = 0.0;
+#pragma unroll
+          for (int w = 0; w < NW; ++w) ut += red_u[w][tid];
+          tf[tid] = lora_tf(ut, lbs_out, rms);
+        } else {
+          s_scale = rms_scale(s0, rms);
+        }
+      }
+      __syncthreads();
     }
-    if (c >= NUM_T_PRODUCERS && c < 2 * NUM_T_PRODUCERS) {
-      const uint2 qq = reinterpret_cast<const uint2*>(q_nat)[tid];
-      const int t = block_sum_int(dp4a_ss(wb_out.y, qq.y, dp4a_ss(wb_out.x, qq.x, 0)), red_i);
-      if (tid == 0) p.tout[c - NUM_T_PRODUCERS] = t;
-      block_arrive(p.ctr + CTR_TOUT * CTR_STRIDE);
-    }
-    __syncthreads();
+    sumq = 0;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) sumq += red_i[w];
     {
       const uint4* qp4 = reinterpret_cast<const uint4*>(q_perm) + lane;
       int S = bits_dot<E / 128>(w_out, qp4);
       S = warp_sum(S);
-      if (lane == 0 && slot_out < n_out) acc_out[slot_out] = 2 * S - s_sumq;
+      if (lane == 0 && slot_out < n_out) acc_out[slot_out] = 2 * S - sumq;
     }
-    if (tid == kAuxThread) s_scale = rms_scale(s0A, ssA, E);
-    if (!block_wait(p.ctr + CTR_TOUT * CTR_STRIDE, NUM_T_PRODUCERS * (l + 1), p.err, p.status, p.spin_limit,
-                    &sflag))
-      return;
-    const float s_out = s_scale;
-    if (tid < R) tf[tid] = lora_tf(__ldcg(p.tout + tid), __ldg(Lp.out_lbs + tid), s_out);
     __syncthreads();
     if (tid < n_out) {
-      const int o = ro0 + tid;
-      const float y = linear_out(acc_out[tid], s_out, o_sw[tid], o_sa[tid], o_wa[tid], tf, R);
-      p.hidden[o] = fadd(__ldcg(p.hidden + o), y);
+      const float y = linear_out(acc_out[tid], s_scale, o_sw[tid], o_sa[tid], o_wa[tid], tf, R);
+      const float hn = fadd(h_old[tid], y);
+      p.hidden[ro0 + tid] = hn;
+      h_new[tid] = hn;
+    }
+    if (has_next) {
+      // the next layer's in_proj LoRA-down partial sums over the owned rows of h: warp r, lane j
+      __syncthreads();
+      double part = 0.0;
+      if (lane < n_out) part = int_to_f64(wbi_next) * (double)fmul(h_new[lane], nw_next);
+      part = warp_sum(part);
+      if (lane == 0) p.upin[c * R + warp] = part;
     }
     block_arrive(p.ctr + CTR_H * CTR_STRIDE);
   }
@@ -609,9 +678,9 @@ bool fused_decode_supported(const dfssm_dims_t& d, int B, const dfssm_layer_t* l
   for (int l = 0; l < n; ++l)
     if (layers[l].in_proj.rank != fused::R || layers[l].out_proj.rank != fused::R) return false;
   const int nc = num_sms();
-  // ownership limits: in_proj rows per CTA <= 64, out_proj rows <= 16, SSM rows <= 32, and the two
-  // groups of LoRA-down producers must exist
-  if (nc < 133 || nc > 1024) return false;
+  // ownership limits: in_proj rows per CTA <= 64, out_proj rows <= 16, SSM rows <= 32; partial-sum
+  // buffers sized for MAX_CTAS
+  if (nc < fused::MIN_CTAS || nc > fused::MAX_CTAS) return false;
   int coop = 0, dev = 0;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev);
@@ -654,8 +723,8 @@ cudaError_t launch_fused_decode(const dfssm_layer_t* layers, int n_layers, float
   p.ctr = reinterpret_cast<int*>(base + fused::OFF_CTR);
   p.err = reinterpret_cast<int*>(base + fused::OFF_ERR);
   p.status = reinterpret_cast<int*>(base + fused::OFF_STATUS);
-  p.tin = reinterpret_cast<int*>(base + fused::OFF_TIN);
-  p.tout = reinterpret_cast<int*>(base + fused::OFF_TOUT);
+  p.upin = reinterpret_cast<double*>(base + fused::OFF_UIN);
+  p.upout = reinterpret_cast<double*>(base + fused::OFF_UOUT);
   p.sacc = reinterpret_cast<int*>(base + fused::OFF_SACC);
   p.gbuf = reinterpret_cast<float*>(base + fused::OFF_GBUF);
   p.spin_limit = spin_limit;

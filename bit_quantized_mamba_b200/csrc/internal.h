@@ -12,7 +12,7 @@ struct QuantScratch {
   int8_t* q;     // [B][n] codes (dp4a-permuted or natural order)
   float* s;      // [B] per-token scale
   int32_t* sumq; // [B] sum of the codes of each token
-  int32_t* t;    // [B][16] LoRA-down accumulators
+  float* tf;     // [B][16] LoRA intermediate (entries >= rank are 0)
 };
 size_t quant_scratch_bytes(int B, int n);
 QuantScratch carve_quant_scratch(void* base, int B, int n);
@@ -24,12 +24,13 @@ struct QuantArgs {
   int n;                   // row length
   int B;
   const int8_t* lora_b;    // [rank][n] or NULL
+  const float* lora_b_scale;
   int rank;
   bool permute;            // dp4a-permuted layout (scaffold GEMV) or natural (int8 GEMV)
   QuantScratch out;
   int8_t* dbg_xq;          // optional taps
   float* dbg_s;
-  int32_t* dbg_t;
+  float* dbg_tf;
 };
 cudaError_t launch_quant(const QuantArgs& a, cudaStream_t st);
 

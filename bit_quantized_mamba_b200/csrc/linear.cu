@@ -22,7 +22,7 @@ static inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 size_t quant_scratch_bytes(int B, int n) {
   return align256((size_t)B * n) + align256(sizeof(float) * 16) + align256(sizeof(int32_t) * 16) +
-         align256(sizeof(int32_t) * 16 * 16);
+         align256(sizeof(float) * 16 * 16);
 }
 
 QuantScratch carve_quant_scratch(void* base, int B, int n) {
@@ -34,7 +34,7 @@ QuantScratch carve_quant_scratch(void* base, int B, int n) {
   p += align256(sizeof(float) * 16);
   s.sumq = reinterpret_cast<int32_t*>(p);
   p += align256(sizeof(int32_t) * 16);
-  s.t = reinterpret_cast<int32_t*>(p);
+  s.tf = reinterpret_cast<float*>(p);
   return s;
 }
 
@@ -67,8 +67,8 @@ static cudaError_t launch_pdl(Kern k, dim3 grid, dim3 block, size_t smem, cudaSt
 
 // ------------------------------------------------------------------------------- quantize kernel
 // One CTA per token.  v = x (or fl32(x*norm_w) when the RMSNorm is folded in); s0 = fl32(absmax/127);
-// q = clamp(rint(fl32(v/s0)), +-127); s = s0 (or fl32(s0 / sqrt(sum x^2 / n + 1e-5)) in fp64);
-// t[r] = sum_i W_B[r,i] q_i.
+// q = clamp(rint(fl32(v/s0)), +-127); rms = 1 (or sqrt(sum x^2 / n + 1e-5) in fp64); s = fl32(s0/rms);
+// LoRA down on the fp32 input: tf[r] = fl32((sum_i W_B[r,i] v_i) sB[r] / rms), the sum in fp64.
 
 constexpr int kQuantThreads = 512;
 
@@ -77,10 +77,10 @@ __global__ void __launch_bounds__(kQuantThreads) quant_kernel(QuantArgs a) {
   pdl_wait();
   extern __shared__ __align__(16) unsigned char smem[];
   float* v = reinterpret_cast<float*>(smem);
-  int8_t* qs = reinterpret_cast<int8_t*>(v + a.n);
   __shared__ double red_d[kQuantThreads / 32];
   __shared__ float red_f[kQuantThreads / 32];
-  __shared__ int red_i[kQuantThreads / 32][DFSSM_MAX_RANK + 1];
+  __shared__ int red_i[kQuantThreads / 32];
+  __shared__ double red_u[kQuantThreads / 32][DFSSM_MAX_RANK];
   const int b = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
   constexpr int NW = kQuantThreads / 32;
@@ -105,77 +105,76 @@ __global__ void __launch_bounds__(kQuantThreads) quant_kernel(QuantArgs a) {
     red_d[wid] = ss;
   }
   __syncthreads();
-  if (wid == 0) {
-    float mm = lane < NW ? red_f[lane] : 0.0f;
-    double sd = lane < NW ? red_d[lane] : 0.0;
-    mm = warp_max(mm);
-    sd = warp_sum(sd);
-    if (lane == 0) {
-      red_f[0] = mm;
-      red_d[0] = sd;
-    }
+  m = 0.0f;
+  ss = 0.0;
+  for (int w = 0; w < NW; ++w) {
+    m = fmaxf(m, red_f[w]);
+    ss += red_d[w];
   }
-  __syncthreads();
-  m = red_f[0];
-  ss = red_d[0];
   const float s0 = (m == 0.0f) ? 0.0f : __fdiv_rn(m, 127.0f);
+  const float inv_s0 = (m == 0.0f) ? 0.0f : __frcp_rn(s0);
 
   int8_t* qout = a.out.q + (size_t)b * a.n;
   int sq = 0;
   for (int i = tid; i < a.n; i += kQuantThreads) {
-    const int c = (m == 0.0f) ? 0 : quant_code(v[i], s0);
-    qs[i] = (int8_t)c;
+    const int c = (m == 0.0f) ? 0 : quant_code_fast(v[i], s0, inv_s0);
     sq += c;
     qout[a.permute ? perm_index(i) : i] = (int8_t)c;
     if (a.dbg_xq) a.dbg_xq[(size_t)b * a.n + i] = (int8_t)c;
   }
-  __syncthreads();
 
-  // LoRA down: t[r] = sum_i W_B[r,i] q_i, four bytes per dp4a.
-  int tr[DFSSM_MAX_RANK];
+  // LoRA down on the fp32 input, four inputs per step (products int8 x fp32 are exact in fp64).
+  double u[DFSSM_MAX_RANK];
 #pragma unroll
-  for (int r = 0; r < DFSSM_MAX_RANK; ++r) tr[r] = 0;
+  for (int r = 0; r < DFSSM_MAX_RANK; ++r) u[r] = 0.0;
   if (a.rank > 0) {
-    const uint32_t* q4 = reinterpret_cast<const uint32_t*>(qs);
     for (int w = tid; w < a.n / 4; w += kQuantThreads) {
-      const uint32_t qq = q4[w];
+      const float4 v4 = reinterpret_cast<const float4*>(v)[w];
+      const double vd[4] = {(double)v4.x, (double)v4.y, (double)v4.z, (double)v4.w};
 #pragma unroll
       for (int r = 0; r < DFSSM_MAX_RANK; ++r) {
         if (r < a.rank) {
           const uint32_t wb = ld_stream_u32(a.lora_b + (size_t)r * a.n + 4 * (size_t)w);
-          tr[r] = dp4a_ss(wb, qq, tr[r]);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int wj = (int)(int8_t)(wb >> (8 * j));
+            u[r] = fma(int_to_f64(wj), vd[j], u[r]);
+          }
         }
       }
     }
   }
   sq = warp_sum(sq);
 #pragma unroll
-  for (int r = 0; r < DFSSM_MAX_RANK; ++r) tr[r] = warp_sum(tr[r]);
+  for (int r = 0; r < DFSSM_MAX_RANK; ++r) u[r] = warp_sum(u[r]);
   if (lane == 0) {
+    red_i[wid] = sq;
 #pragma unroll
-    for (int r = 0; r < DFSSM_MAX_RANK; ++r) red_i[wid][r] = tr[r];
-    red_i[wid][DFSSM_MAX_RANK] = sq;
+    for (int r = 0; r < DFSSM_MAX_RANK; ++r) red_u[wid][r] = u[r];
   }
   __syncthreads();
-  if (tid <= DFSSM_MAX_RANK) {
-    int tot = 0;
-    for (int w = 0; w < NW; ++w) tot += red_i[w][tid];
-    if (tid == DFSSM_MAX_RANK) {
-      a.out.sumq[b] = tot;
-    } else {
-      a.out.t[b * DFSSM_MAX_RANK + tid] = tot;
-      if (a.dbg_t && tid < a.rank) a.dbg_t[(size_t)b * a.rank + tid] = tot;
-    }
+  const double rms = a.norm_w ? rms_of(ss, a.n) : 1.0;
+  if (tid < DFSSM_MAX_RANK) {
+    double tot = 0.0;
+    for (int w = 0; w < NW; ++w) tot += red_u[w][tid];
+    const float tf = tid < a.rank ? lora_tf(tot, a.lora_b_scale[tid], rms) : 0.0f;
+    a.out.tf[b * DFSSM_MAX_RANK + tid] = tf;
+    if (a.dbg_tf && tid < a.rank) a.dbg_tf[(size_t)b * a.rank + tid] = tf;
   }
-  if (tid == 0) {
-    const float s = a.norm_w ? rms_scale(s0, ss, a.n) : s0;
+  if (tid == DFSSM_MAX_RANK) {
+    int tot = 0;
+    for (int w = 0; w < NW; ++w) tot += red_i[w];
+    a.out.sumq[b] = tot;
+  }
+  if (tid == DFSSM_MAX_RANK + 1) {
+    const float s = a.norm_w ? rms_scale(s0, rms) : s0;
     a.out.s[b] = s;
     if (a.dbg_s) a.dbg_s[b] = s;
   }
 }
 
 cudaError_t launch_quant(const QuantArgs& a, cudaStream_t st) {
-  const size_t smem = (size_t)a.n * 5;  // <= 40 KB for n <= 8192
+  const size_t smem = (size_t)a.n * 4;  // <= 32 KB for n <= 8192
   return launch_pdl(quant_kernel, dim3(a.B), dim3(kQuantThreads), smem, st, a);
 }
 
@@ -206,7 +205,7 @@ __device__ __forceinline__ void gemv_stage(const GemvArgs& a, uint4* qsm, float 
   if (threadIdx.x < nb * DFSSM_MAX_RANK) {
     const int b = threadIdx.x / DFSSM_MAX_RANK, r = threadIdx.x % DFSSM_MAX_RANK;
     float v = 0.0f;
-    if (r < a.rank) v = lora_tf(a.in.t[b * DFSSM_MAX_RANK + r], a.lora_b_scale[r], a.in.s[b]);
+    if (r < a.rank) v = a.in.tf[b * DFSSM_MAX_RANK + r];
     tf[b][r] = v;
   }
   if (threadIdx.x < nb) {

@@ -10,8 +10,8 @@
 //
 // The array (kScratchBytes, enough for B <= 16 tokens of d_in <= 8192) is a module global: every device
 // that loads the library holds it until the process exits.  All calls on a device share it and each call
-// overwrites it before reading it (the quantize kernel writes every code, scale, code sum and LoRA-down
-// sum that the GEMV kernel then reads), so nothing has to start at zero; two calls that overlap on the GPU
+// overwrites it before reading it (the quantize kernel writes every code, scale, code sum and LoRA
+// intermediate that the GEMV kernel then reads), so nothing has to start at zero; two calls that overlap on the GPU
 // (different streams, no ordering between them) race on it.
 //
 // In host code the array's name is only a host-side stand-in, not a device address.  The device address
@@ -104,13 +104,14 @@ extern "C" int dfssm_linear_decode_noalloc(const dfssm_linear_t* lin, const floa
   qa.n = lin->d_in;
   qa.B = B;
   qa.lora_b = lin->lora_b;
+  qa.lora_b_scale = lin->lora_b_scale;
   qa.rank = lin->rank;
   qa.permute = true;
   qa.out = qs;
   if (dbg) {
     qa.dbg_xq = dbg->xq;
     qa.dbg_s = dbg->xscale;
-    qa.dbg_t = dbg->lora_t;
+    qa.dbg_tf = dbg->lora_tf;
   }
   cudaError_t e = dfssm::launch_quant(qa, s);
   if (e != cudaSuccess) return dfssm::record_cuda_failure(e);

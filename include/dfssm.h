@@ -62,9 +62,10 @@ typedef enum {
  *   lora_a_scale  device f32 [d_out]   per-row scale of W_A
  * Constraints: d_in % 32 == 0, d_in <= 8192, d_out >= 1, 0 <= rank <= 16.  rank == 0 means no LoRA
  * (lora_* may then be NULL).
- * Computes, for each token b with (q, s) its per-token int8 quantization:
- *   acc[o] = sum_i sign(o,i) q[i]  (int32),   t[r] = sum_i W_B[r,i] q[i]  (int32)
- *   tf[r]  = fl32(t[r] sB[r] s),  y[o] = fl32(acc[o] s sW[o] + sA[o] sum_r W_A[o,r] tf[r])   (fp64 inside)
+ * Computes, for each token b with input x and (q, s) its per-token int8 quantization:
+ *   acc[o] = sum_i sign(o,i) q[i]  (int32, exact)
+ *   tf[r]  = fl32((sum_i W_B[r,i] x[i]) sB[r])           (LoRA down on the fp32 input, fp64 sum)
+ *   y[o]   = fl32(acc[o] s sW[o] + sA[o] sum_r W_A[o,r] tf[r])   (fp64 inside)
  */
 typedef struct {
   int32_t d_out, d_in, rank;
@@ -76,10 +77,10 @@ typedef struct {
   const float* lora_a_scale;
 } dfssm_linear_t;
 
-/* Optional device taps of the integer intermediates (any member may be NULL). */
+/* Optional device taps of the intermediates (any member may be NULL). */
 typedef struct {
-  int32_t* acc;   /* [B][d_out]  scaffold accumulators                                    */
-  int32_t* lora_t;/* [B][rank]   LoRA-down accumulators                                   */
+  int32_t* acc;   /* [B][d_out]  scaffold accumulators (int32, exact)                      */
+  float* lora_tf; /* [B][rank]   LoRA intermediate tf                                      */
   int8_t* xq;     /* [B][d_in]   quantized activations, natural order                     */
   float* xscale;  /* [B]         per-token scale s                                         */
 } dfssm_debug_t;
@@ -123,8 +124,8 @@ int dfssm_linear_decode_noalloc(const dfssm_linear_t* lin, const float* x, int B
  * M-token prefill of one linear on int8 tcgen05 tensor cores (technical summary §2.C: the scaffold
  * matmul on INT8 tensor cores).  Same math as dfssm_linear_decode, per row of x.
  *   x device f32 [M][d_in], y device f32 [M][d_out], M >= 1.  d_in % 128 == 0 required.
- *   Integer results (dbg->acc, dbg->lora_t, dbg->xq, dbg->xscale) are exact; y is fp32 to within
- *   1e-6 relative of the fp64 epilogue (the prefill epilogue uses fp32 fused multiply-add).
+ *   dbg->acc, dbg->xq and dbg->xscale are exact; tf and y are fp32 to within 1e-6 relative of the fp64
+ *   definition (the prefill epilogue uses fp32 fused multiply-add).
  */
 int dfssm_linear_prefill(const dfssm_linear_t* lin, const float* x, int M, float* y, void* workspace,
                          size_t ws_bytes, const dfssm_debug_t* dbg, void* stream);
@@ -175,8 +176,10 @@ typedef struct {
  *   hidden       device f32 [B][d_model]; the residual stream, updated in place
  *   conv_states  HOST array [n_layers] of device f32 [B][conv channels][3]
  *   ssm_states   HOST array [n_layers] of device f32 [B][nheads][headdim][d_state]
- * Per layer: (q,s) = quant(RMSNorm(h)); zxbcdt = in_proj; x|B|C = SiLU(conv(xBC)); y = SSM(x, dt, B, C);
- * g = y*SiLU(z); (q',s') = quant(RMSNorm(g)); h += out_proj.   1 <= B <= 16, n_layers <= 64.
+ * Per layer: (q,s) = quant(RMSNorm(h)); zxbcdt = in_proj (LoRA on RMSNorm(h)); x|B|C = SiLU(conv(xBC));
+ * y = SSM(x, dt, B, C); g = y*SiLU(z); (q',s') = quant(RMSNorm(g)); h += out_proj.  The RMS factor is
+ * folded into the quantizer scale and the LoRA intermediate: s = fl32(s0/rms), tf = fl32(u sB / rms)
+ * with v = fl32(h w) quantized and u = W_B v.   1 <= B <= 16, n_layers <= 64.
  * workspace: dfssm_workspace_size(DFSSM_OP_LAYER_DECODE, B, d_model, d_inner).
  */
 int dfssm_layer_decode(const dfssm_layer_t* layers, int n_layers, const dfssm_dims_t* dims,

@@ -35,11 +35,12 @@ def _declare(L):
     L.oracle_sign.restype = _I
     L.oracle_quantize.argtypes = [_P, _I, _I, _P, _P]
     L.oracle_linear_decode.argtypes = [_I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _I, _P, _P, _P, _P, _P]
-    L.oracle_linear_core.argtypes = [_I, _I, _I, _P, _P, _P, _P, _P, _P, _P, C.c_float, _P, _P, _P]
-    L.oracle_linear_rows.argtypes = [_I, _I, _I, _P, _P, _P, _P, _P, _P, _P, C.c_float, _P, _I, _P, _P]
+    L.oracle_lora_down.argtypes = [_I, _I, _P, _P, _P, C.c_double, _P]
+    L.oracle_linear_core.argtypes = [_I, _I, _I, _P, _P, _P, _P, _P, C.c_float, _P, _P, _P]
+    L.oracle_linear_rows.argtypes = [_I, _I, _I, _P, _P, _P, _P, _P, C.c_float, _P, _P, _I, _P, _P]
     L.oracle_conv_step.argtypes = [_P, _P, _P, _P, _P, _I, _I]
     L.oracle_ssm_step.argtypes = [_P] * 9 + [_I] * 5
-    L.oracle_rmsnorm_quantize.argtypes = [_P, _P, _I, _I, _P, _P]
+    L.oracle_rmsnorm_quantize.argtypes = [_P, _P, _I, _I, _P, _P, _P, _P]
     L.oracle_gate.argtypes = [_P, _P, _P, _I]
     L.oracle_layer_decode.argtypes = [_I] * 7 + [_P] * 12 + [_P] * 7 + [_P] * 3 + [_P, _P]
     L.oracle_lm_head.argtypes = [_P, _P, _I, _I, _P, _P, _I, _P, _P]
@@ -101,37 +102,51 @@ class Linear:
 
 
 def linear_decode(L: Linear, x: np.ndarray):
-    """Quantize each row of x and apply the linear. Returns dict(y, acc, t, xq, xscale)."""
+    """Quantize each row of x and apply the linear. Returns dict(y, acc, tf, xq, xscale)."""
     x = _c(np.atleast_2d(x), np.float32)
     B = x.shape[0]
     assert x.shape[1] == L.d_in
     y = np.zeros((B, L.d_out), np.float32)
     acc = np.zeros((B, L.d_out), np.int32)
-    t = np.zeros((B, max(L.rank, 1)), np.int32)
+    tf = np.zeros((B, max(L.rank, 1)), np.float32)
     xq = np.zeros((B, L.d_in), np.int8)
     xs = np.zeros(B, np.float32)
-    lib().oracle_linear_decode(*L._args(), _p(x), B, _p(y), _p(acc), _p(t), _p(xq), _p(xs))
-    return dict(y=y, acc=acc, t=t[:, :L.rank], xq=xq, xscale=xs)
+    lib().oracle_linear_decode(*L._args(), _p(x), B, _p(y), _p(acc), _p(tf), _p(xq), _p(xs))
+    return dict(y=y, acc=acc, tf=tf[:, :L.rank], xq=xq, xscale=xs)
 
 
-def linear_core(L: Linear, q: np.ndarray, s: float):
-    """The linear on one pre-quantized row q (int8) with scale s. Returns (y, acc, t)."""
+def lora_down(L: Linear, v: np.ndarray, rms: float = 1.0) -> np.ndarray:
+    """LoRA intermediate tf[r] = fl32((sum_i W_B[r,i] v_i) * sB[r] / rms) of one input row v."""
+    v = _c(v, np.float32).reshape(L.d_in)
+    tf = np.zeros(max(L.rank, 1), np.float32)
+    a = L._args()
+    lib().oracle_lora_down(L.d_in, L.rank, a[5], a[6], _p(v), float(rms), _p(tf))
+    return tf[:L.rank]
+
+
+def linear_core(L: Linear, q: np.ndarray, s: float, tf: np.ndarray):
+    """The linear on one pre-quantized row q (int8) with scale s and LoRA intermediate tf.
+    Returns (y, acc)."""
     q = _c(q, np.int8).reshape(L.d_in)
+    tf = _c(tf, np.float32).reshape(-1) if L.rank else np.zeros(1, np.float32)
     y = np.zeros(L.d_out, np.float32)
     acc = np.zeros(L.d_out, np.int32)
-    t = np.zeros(max(L.rank, 1), np.int32)
-    lib().oracle_linear_core(*L._args(), _p(q), C.c_float(float(s)), _p(acc), _p(t), _p(y))
-    return y, acc, t[:L.rank]
+    a = L._args()
+    lib().oracle_linear_core(L.d_out, L.d_in, L.rank, a[3], a[4], a[7], a[8], _p(q),
+                             C.c_float(float(s)), _p(tf), _p(acc), _p(y))
+    return y, acc
 
 
-def linear_rows(L: Linear, q: np.ndarray, s: float, rows):
+def linear_rows(L: Linear, q: np.ndarray, s: float, tf: np.ndarray, rows):
     """Only the listed output rows of the linear on pre-quantized q. Returns (y, acc)."""
     q = _c(q, np.int8).reshape(L.d_in)
+    tf = _c(tf, np.float32).reshape(-1) if L.rank else np.zeros(1, np.float32)
     rows = _c(rows, np.int32)
     y = np.zeros(len(rows), np.float32)
     acc = np.zeros(len(rows), np.int32)
-    lib().oracle_linear_rows(*L._args(), _p(q), C.c_float(float(s)), _p(rows), len(rows), _p(acc),
-                             _p(y))
+    a = L._args()
+    lib().oracle_linear_rows(L.d_out, L.d_in, L.rank, a[3], a[4], a[7], a[8], _p(q),
+                             C.c_float(float(s)), _p(tf), _p(rows), len(rows), _p(acc), _p(y))
     return y, acc
 
 
@@ -165,13 +180,16 @@ def ssm_step(ssm_state, x, dt_raw, A_log, dt_bias, D, Bm, Cm):
 
 
 def rmsnorm_quantize(h, w):
+    """RMSNorm folded into the quantizer. Returns (q [B][n], s [B], v [B][n], rms [B])."""
     h = _c(np.atleast_2d(h), np.float32)
     B, n = h.shape
     w = _c(w, np.float32)
     q = np.zeros((B, n), np.int8)
     s = np.zeros(B, np.float32)
-    lib().oracle_rmsnorm_quantize(_p(h), _p(w), B, n, _p(q), _p(s))
-    return q, s
+    v = np.zeros((B, n), np.float32)
+    rms = np.zeros(B, np.float64)
+    lib().oracle_rmsnorm_quantize(_p(h), _p(w), B, n, _p(q), _p(s), _p(v), _p(rms))
+    return q, s, v, rms
 
 
 def gate(y, z):

@@ -70,23 +70,28 @@ void quantize_row(const float* v, int n, int8_t* q, float* s_out) {
   *s_out = s;
 }
 
-// Linear layer on an already-quantized row: 1-bit scaffold + int8 rank-r LoRA ([TS-2B], [TS-2C]).
-//   acc[o] = sum_i sign(o,i) * q[i]                       (exact integer; fits int32)
-//   t[r]   = sum_i W_B[r,i] * q[i]                        (exact integer)
-//   tf[r]  = fl32(t[r] * sB[r] * s)                       (reading (iii): LoRA intermediate kept fp32)
-//   y[o]   = fl32(acc[o]*s*sW[o] + sA[o] * sum_r W_A[o,r]*tf[r])
-// Reading (iv): per-row scales for W_B (rank rows) and W_A (d_out rows).
-void linear_core(int d_out, int d_in, int rank, const uint32_t* bits, const float* w_scale,
-                 const int8_t* lora_b, const float* lora_b_scale, const int8_t* lora_a,
-                 const float* lora_a_scale, const int8_t* q, float s, int32_t* acc_out,
-                 int32_t* t_out, float* y) {
-  std::vector<float> tf((size_t)(rank > 0 ? rank : 1));
+// LoRA down-projection of the linear's fp32 input ([TS-2B]: the LoRA matrices W_A, W_B are int8 with
+// per-row scales; a LoRA module applies W_A (W_B x) to the layer input x).  Reading (iii): the LoRA sees
+// the same input as the layer, not its int8 codes, and its intermediate stays fp32:
+//   u[r]  = sum_i W_B[r,i] * v[i]             (fp64; every product int8 x fp32 is exact)
+//   tf[r] = fl32(u[r] * sB[r] / rms)          (rms = 1 for a plain linear; the RMS of the norm when the
+//                                              layer input is RMSNorm(h) and v = fl32(h*w))
+void lora_down(int d_in, int rank, const int8_t* lora_b, const float* lora_b_scale, const float* v,
+               double rms, float* tf) {
   for (int r = 0; r < rank; ++r) {
-    int64_t sum = 0;
-    for (int i = 0; i < d_in; ++i) sum += (int64_t)lora_b[(size_t)r * d_in + i] * (int64_t)q[i];
-    if (t_out) t_out[r] = (int32_t)sum;
-    tf[r] = r32((double)sum * (double)lora_b_scale[r] * (double)s);
+    double u = 0.0;
+    for (int i = 0; i < d_in; ++i) u += (double)lora_b[(size_t)r * d_in + i] * (double)v[i];
+    tf[r] = r32(u * (double)lora_b_scale[r] / rms);
   }
+}
+
+// Scaffold + LoRA-up on an already-quantized row ([TS-2B], [TS-2C]); reading (iv): per-row scales for
+// W_B (rank rows) and W_A (d_out rows).
+//   acc[o] = sum_i sign(o,i) * q[i]                       (exact integer; fits int32)
+//   y[o]   = fl32(acc[o]*s*sW[o] + sA[o] * sum_r W_A[o,r]*tf[r])
+void linear_core(int d_out, int d_in, int rank, const uint32_t* bits, const float* w_scale,
+                 const int8_t* lora_a, const float* lora_a_scale, const int8_t* q, float s,
+                 const float* tf, int32_t* acc_out, float* y) {
 #pragma omp parallel for schedule(static)
   for (int o = 0; o < d_out; ++o) {
     int64_t a = 0;
@@ -103,15 +108,18 @@ void linear_core(int d_out, int d_in, int rank, const uint32_t* bits, const floa
 // Mamba-2 pre-mixer RMSNorm followed by the per-token quantizer (reading: eps = 1e-5, weight per
 // channel).  The quantizer is invariant to a positive scalar factor of its input — q(c*v) = q(v) and
 // s(c*v) = c*s(v) in exact arithmetic — so the RMS factor is folded into the scale:
-//   v_i = fl32(h_i * w_i);  (q, s0) = quantize(v);  s = fl32(s0 / sqrt(sum_i h_i^2 / n + eps)).
-void rmsnorm_quantize(const float* h, const float* w, int n, double eps, int8_t* q, float* s_out,
-                      float* v_scratch) {
+//   v_i = fl32(h_i * w_i);  (q, s0) = quantize(v);  rms = sqrt(sum_i h_i^2 / n + eps);  s = fl32(s0 / rms).
+// Returns rms (fp64) and leaves v in v_out for the LoRA down-projection.
+double rmsnorm_quantize(const float* h, const float* w, int n, double eps, int8_t* q, float* s_out,
+                        float* v_out) {
   double ss = 0.0;
   for (int i = 0; i < n; ++i) ss += (double)h[i] * (double)h[i];
-  for (int i = 0; i < n; ++i) v_scratch[i] = r32((double)h[i] * (double)w[i]);
+  for (int i = 0; i < n; ++i) v_out[i] = r32((double)h[i] * (double)w[i]);
   float s0 = 0.0f;
-  quantize_row(v_scratch, n, q, &s0);
-  *s_out = r32((double)s0 / std::sqrt(ss / (double)n + eps));
+  quantize_row(v_out, n, q, &s0);
+  const double rms = std::sqrt(ss / (double)n + eps);
+  *s_out = r32((double)s0 / rms);
+  return rms;
 }
 
 inline double silu64(double v) { return v / (1.0 + std::exp(-v)); }
@@ -120,7 +128,7 @@ inline double silu64(double v) { return v / (1.0 + std::exp(-v)); }
 
 extern "C" {
 
-int oracle_abi_version(void) { return 1; }
+int oracle_abi_version(void) { return 2; }
 
 // Pinned by: exhaustive byte-pattern round trip against an independent packer, brute force.
 int oracle_sign(const uint32_t* bits, int d_in, int o, int i) { return unpack_sign(bits, d_in, o, i); }
@@ -138,40 +146,43 @@ void oracle_quantize(const float* x, int B, int n, int8_t* q, float* s) {
 void oracle_linear_decode(int d_out, int d_in, int rank, const uint32_t* bits, const float* w_scale,
                           const int8_t* lora_b, const float* lora_b_scale, const int8_t* lora_a,
                           const float* lora_a_scale, const float* x, int B, float* y,
-                          int32_t* acc, int32_t* t, int8_t* xq, float* xscale) {
+                          int32_t* acc, float* tf_out, int8_t* xq, float* xscale) {
   std::vector<int8_t> q((size_t)d_in);
+  std::vector<float> tf((size_t)(rank > 0 ? rank : 1));
   for (int b = 0; b < B; ++b) {
     float s = 0.0f;
-    quantize_row(x + (size_t)b * d_in, d_in, q.data(), &s);
+    const float* xb = x + (size_t)b * d_in;
+    quantize_row(xb, d_in, q.data(), &s);
     if (xq) std::memcpy(xq + (size_t)b * d_in, q.data(), (size_t)d_in);
     if (xscale) xscale[b] = s;
-    linear_core(d_out, d_in, rank, bits, w_scale, lora_b, lora_b_scale, lora_a, lora_a_scale,
-                q.data(), s, acc ? acc + (size_t)b * d_out : nullptr,
-                t ? t + (size_t)b * (rank > 0 ? rank : 1) : nullptr, y + (size_t)b * d_out);
+    lora_down(d_in, rank, lora_b, lora_b_scale, xb, 1.0, tf.data());
+    if (tf_out)
+      for (int r = 0; r < rank; ++r) tf_out[(size_t)b * rank + r] = tf[r];
+    linear_core(d_out, d_in, rank, bits, w_scale, lora_a, lora_a_scale, q.data(), s, tf.data(),
+                acc ? acc + (size_t)b * d_out : nullptr, y + (size_t)b * d_out);
   }
 }
 
-// Same linear on pre-quantized rows (used for teacher-forced and sampled checks).
+// LoRA down-projection alone (see lora_down): tf[r] for input v and divisor rms.
+void oracle_lora_down(int d_in, int rank, const int8_t* lora_b, const float* lora_b_scale,
+                      const float* v, double rms, float* tf) {
+  lora_down(d_in, rank, lora_b, lora_b_scale, v, rms, tf);
+}
+
+// Scaffold + LoRA-up on pre-quantized codes q with scale s and LoRA intermediate tf (teacher-forced and
+// sampled checks).
 void oracle_linear_core(int d_out, int d_in, int rank, const uint32_t* bits, const float* w_scale,
-                        const int8_t* lora_b, const float* lora_b_scale, const int8_t* lora_a,
-                        const float* lora_a_scale, const int8_t* q, float s, int32_t* acc,
-                        int32_t* t, float* y) {
-  linear_core(d_out, d_in, rank, bits, w_scale, lora_b, lora_b_scale, lora_a, lora_a_scale, q, s, acc,
-              t, y);
+                        const int8_t* lora_a, const float* lora_a_scale, const int8_t* q, float s,
+                        const float* tf, int32_t* acc, float* y) {
+  linear_core(d_out, d_in, rank, bits, w_scale, lora_a, lora_a_scale, q, s, tf, acc, y);
 }
 
 // Sampled rows of the linear: only output rows listed in `rows` are computed (y[k] for rows[k]).
-// Used for the full-size prefill and LM-head checks, where a whole oracle pass is too slow.
+// Used for the full-size prefill and multi-copy checks, where a whole oracle pass is too slow.
 void oracle_linear_rows(int d_out, int d_in, int rank, const uint32_t* bits, const float* w_scale,
-                        const int8_t* lora_b, const float* lora_b_scale, const int8_t* lora_a,
-                        const float* lora_a_scale, const int8_t* q, float s, const int* rows,
-                        int n_rows, int32_t* acc, float* y) {
-  std::vector<float> tf((size_t)(rank > 0 ? rank : 1));
-  for (int r = 0; r < rank; ++r) {
-    int64_t sum = 0;
-    for (int i = 0; i < d_in; ++i) sum += (int64_t)lora_b[(size_t)r * d_in + i] * (int64_t)q[i];
-    tf[r] = r32((double)sum * (double)lora_b_scale[r] * (double)s);
-  }
+                        const int8_t* lora_a, const float* lora_a_scale, const int8_t* q, float s,
+                        const float* tf, const int* rows, int n_rows, int32_t* acc, float* y) {
+  (void)d_out;
   for (int k = 0; k < n_rows; ++k) {
     const int o = rows[k];
     int64_t a = 0;
@@ -257,13 +268,17 @@ void oracle_ssm_step(float* ssm_state, const float* x, const float* dt_raw, cons
   }
 }
 
-// Pre-mixer RMSNorm + per-token quantization of B rows (the RMS factor folded into the scale).
+// Pre-mixer RMSNorm + per-token quantization of B rows (the RMS factor folded into the scale); also
+// returns v = fl32(h*w) [B][n] and rms [B] for the LoRA down-projection.
 // Pinned by: a constant row reconstructs w*sign(c); codes agree with quantizing the explicitly
 // normalized row away from rounding ties; scale relation.
-void oracle_rmsnorm_quantize(const float* h, const float* w, int B, int n, int8_t* q, float* s) {
-  std::vector<float> v((size_t)n);
-  for (int b = 0; b < B; ++b)
-    rmsnorm_quantize(h + (size_t)b * n, w, n, 1e-5, q + (size_t)b * n, s + b, v.data());
+void oracle_rmsnorm_quantize(const float* h, const float* w, int B, int n, int8_t* q, float* s,
+                             float* v, double* rms) {
+  for (int b = 0; b < B; ++b) {
+    const double r = rmsnorm_quantize(h + (size_t)b * n, w, n, 1e-5, q + (size_t)b * n, s + b,
+                                      v + (size_t)b * n);
+    if (rms) rms[b] = r;
+  }
 }
 
 // Gate of the Mamba-2 output: g = fl32(y * fl32(SiLU(z))) (reading (ix): gate before the norm).
@@ -277,12 +292,12 @@ void oracle_gate(const float* y, const float* z, float* g, int n) {
 
 // One Mamba-2 layer decode step with the DF-SSM linears, B rows, the layer's residual stream h
 // updated in place.  Wiring (reading; the Mamba-2 block [MAP] with the DF-SSM linears [TS-2B]):
-//   (q, s)  = rmsnorm_quantize(h, norm_w)
-//   zxbcdt  = in_proj(q, s)                      (reading (v): order z | x | B | C | dt)
+//   (q, s)  = rmsnorm_quantize(h, norm_w);  tf = lora_down(fl32(h*norm_w)) / rms
+//   zxbcdt  = in_proj(q, s, tf)                  (reading (v): order z | x | B | C | dt)
 //   xc      = conv_step(xBC)                     (SiLU applied to x, B and C channels)
 //   y       = ssm_step(xc.x, dt, xc.B, xc.C)
-//   g       = gate(y, z);  (q', s') = rmsnorm_quantize(g, gnorm_w)
-//   h       = fl32(h + out_proj(q', s'))
+//   g       = gate(y, z);  (q', s') = rmsnorm_quantize(g, gnorm_w);  tf' = lora_down(...) / rms'
+//   h       = fl32(h + out_proj(q', s', tf'))
 // Shapes: D = d_model, E = d_inner = H*P, C = E + 2*G*N conv channels, in_proj rows 2E + 2GN + H.
 // Pinned by: composition of the separately pinned steps in this order; a zero out_proj scale leaves
 // h unchanged.
@@ -304,13 +319,14 @@ void oracle_layer_decode(int B, int Dm, int H, int P, int N, int G, int rank,
   std::vector<int8_t> q((size_t)(E > Dm ? E : Dm));
   std::vector<float> v((size_t)(E > Dm ? E : Dm));
   std::vector<float> zx((size_t)d_ip), xbc((size_t)C), xc((size_t)C), dt((size_t)H), y((size_t)E),
-      g((size_t)E), out((size_t)Dm);
+      g((size_t)E), out((size_t)Dm), tf((size_t)(rank > 0 ? rank : 1));
   for (int b = 0; b < B; ++b) {
     float* hb = h + (size_t)b * Dm;
     float s = 0.0f;
-    rmsnorm_quantize(hb, norm_w, Dm, 1e-5, q.data(), &s, v.data());
-    linear_core(d_ip, Dm, rank, in_bits, in_ws, in_lb, in_lbs, in_la, in_las, q.data(), s, nullptr,
-                nullptr, zx.data());
+    double rms = rmsnorm_quantize(hb, norm_w, Dm, 1e-5, q.data(), &s, v.data());
+    lora_down(Dm, rank, in_lb, in_lbs, v.data(), rms, tf.data());
+    linear_core(d_ip, Dm, rank, in_bits, in_ws, in_la, in_las, q.data(), s, tf.data(), nullptr,
+                zx.data());
     if (tap_zxbcdt) std::memcpy(tap_zxbcdt + (size_t)b * d_ip, zx.data(), sizeof(float) * d_ip);
     std::memcpy(xbc.data(), zx.data() + E, sizeof(float) * C);
     std::memcpy(dt.data(), zx.data() + E + C, sizeof(float) * H);
@@ -319,9 +335,10 @@ void oracle_layer_decode(int B, int Dm, int H, int P, int N, int G, int rank,
                     xc.data() + E, xc.data() + E + G * N, y.data(), 1, H, P, N, G);
     if (tap_y) std::memcpy(tap_y + (size_t)b * E, y.data(), sizeof(float) * E);
     oracle_gate(y.data(), zx.data(), g.data(), E);
-    rmsnorm_quantize(g.data(), gnorm_w, E, 1e-5, q.data(), &s, v.data());
-    linear_core(Dm, E, rank, out_bits, out_ws, out_lb, out_lbs, out_la, out_las, q.data(), s,
-                nullptr, nullptr, out.data());
+    rms = rmsnorm_quantize(g.data(), gnorm_w, E, 1e-5, q.data(), &s, v.data());
+    lora_down(E, rank, out_lb, out_lbs, v.data(), rms, tf.data());
+    linear_core(Dm, E, rank, out_bits, out_ws, out_la, out_las, q.data(), s, tf.data(), nullptr,
+                out.data());
     for (int i = 0; i < Dm; ++i) hb[i] = r32((double)hb[i] + (double)out[i]);
   }
 }

@@ -166,28 +166,40 @@ def test_lora_rank0_equals_scaffold_alone(tiny):
 
 
 def test_lora_one_hot_down_rows(tiny):
+    """A one-hot W_B row picks one input: tf[r] = fl32(x_j * sB[r]) (the LoRA sees the fp32 input)."""
     d = dict(tiny["linear"])
     cols = [3, 17, 100, 255, 0, 64, 128, 129, 5, 6, 7, 8, 9, 10, 11, 12]
     lb = np.zeros((16, 256), np.int8)
     for r, c in enumerate(cols):
         lb[r, c] = 1
     out = oracle.linear_decode(oracle.Linear.from_dict(dict(d, lora_b=lb)), tiny["x"])
-    assert np.array_equal(out["t"][0], out["xq"][0, cols].astype(np.int32))
+    expect = (tiny["x"][0, cols].astype(np.float64) * d["lora_b_scale"].astype(np.float64))
+    assert np.array_equal(out["tf"][0], expect.astype(np.float32))
 
 
 def test_lora_epilogue_real_number_formula(tiny):
-    """y = acc*s*sW + sA * W_A @ (t*sB*s) to fp32 accuracy: catches a transposed W_A, a missing scale or
-    a wrong-sign term."""
+    """y = acc*s*sW + sA * W_A @ ((W_B @ x) * sB) to fp32 accuracy: catches a transposed W_A or W_B, a
+    missing scale or a wrong-sign term."""
     d = tiny["linear"]
     L = oracle.Linear.from_dict(d)
     out = oracle.linear_decode(L, tiny["x"])
     s = float(out["xscale"][0])
-    t = (unpack_t := out["t"][0].astype(np.float64))
-    assert np.array_equal(unpack_t, d["lora_b"].astype(np.int64) @ out["xq"][0].astype(np.int64))
-    tf = t * d["lora_b_scale"].astype(np.float64) * s
+    u = d["lora_b"].astype(np.float64) @ tiny["x"][0].astype(np.float64)
+    tf = u * d["lora_b_scale"].astype(np.float64)
+    assert np.allclose(out["tf"][0], tf, rtol=1e-6, atol=0)
     y = (out["acc"][0] * s * d["w_scale"].astype(np.float64)
          + d["lora_a_scale"].astype(np.float64) * (d["lora_a"].astype(np.float64) @ tf))
     assert np.allclose(out["y"][0], y, rtol=1e-6, atol=1e-7)
+
+
+def test_lora_down_rms_divisor_and_linearity(tiny):
+    """tf(v, rms) = tf(v) / rms to fp32 accuracy, and tf is linear in v (doubling v doubles tf exactly)."""
+    L = oracle.Linear.from_dict(tiny["linear"])
+    v = tiny["x"][0]
+    t1 = oracle.lora_down(L, v).astype(np.float64)
+    t3 = oracle.lora_down(L, v, rms=3.0).astype(np.float64)
+    assert np.allclose(t3, t1 / 3.0, rtol=2e-7)
+    assert np.array_equal(oracle.lora_down(L, v * np.float32(2)), (t1 * 2).astype(np.float32))
 
 
 # ------------------------------------------------------------------------------------------- conv
@@ -324,7 +336,8 @@ def test_rmsnorm_constant_row_reconstructs_weight():
     w = g.uniform(0.5, 1.5, 256).astype(np.float32)
     for c in (-3.0, 0.25, 40.0):
         h = np.full((1, 256), c, np.float32)
-        q, s = oracle.rmsnorm_quantize(h, w)
+        q, s, _, rms = oracle.rmsnorm_quantize(h, w)
+        assert abs(rms[0] - np.sqrt(c * c + 1e-5)) <= 1e-12 * abs(c)
         u = np.sign(c) * w.astype(np.float64) / np.sqrt(1 + 1e-5 / c ** 2)
         assert np.all(np.abs(s[0] * q[0] - u) <= s[0] / 2 * 1.0001)
 
@@ -335,7 +348,8 @@ def test_rmsnorm_fold_matches_explicit_normalization_away_from_ties():
     g = np.random.default_rng(31)
     h = (g.standard_normal((8, 2048)) * 3).astype(np.float32)
     w = g.uniform(0.5, 1.5, 2048).astype(np.float32)
-    q, s = oracle.rmsnorm_quantize(h, w)
+    q, s, v, rms = oracle.rmsnorm_quantize(h, w)
+    assert np.array_equal(v, (h.astype(np.float64) * w).astype(np.float32))
     for b in range(8):
         hb = h[b].astype(np.float64)
         u = hb / np.sqrt(np.mean(hb ** 2) + 1e-5) * w
@@ -382,8 +396,8 @@ def test_layer_zero_out_proj_keeps_residual():
 
 
 def test_layer_composition_of_pinned_steps():
-    """The layer equals the pinned steps wired as: norm+quant -> in_proj -> split z|x|B|C|dt -> conv ->
-    SSM -> gate -> norm+quant -> out_proj -> residual."""
+    """The layer equals the pinned steps wired as: norm+quant (+ LoRA down on the normalized input) ->
+    in_proj -> split z|x|B|C|dt -> conv -> SSM -> gate -> norm+quant -> out_proj -> residual."""
     m = inputs.decode_model(seed=41, n_layers=1, n_tokens=3, **SMALL)
     lay = _oracle_layer(m["layers"][0])
     E, N = 64, 16
@@ -393,15 +407,17 @@ def test_layer_composition_of_pinned_steps():
         h_a = m["emb"][t].copy()
         oracle.layer_decode(lay, h_a, conv_a[0], ssm_a[0])
         h_b = m["emb"][t].copy()
-        q, s = oracle.rmsnorm_quantize(h_b, lay["norm_w"])
-        zx, _, _ = oracle.linear_core(lay["in_proj"], q[0], s[0])
+        q, s, v, rms = oracle.rmsnorm_quantize(h_b, lay["norm_w"])
+        tf = oracle.lora_down(lay["in_proj"], v[0], rms[0])
+        zx, _ = oracle.linear_core(lay["in_proj"], q[0], s[0], tf)
         z, xbc, dt = zx[:E], zx[E:E + E + 2 * N], zx[E + E + 2 * N:]
         xc = oracle.conv_step(conv_b[0], lay["conv_w"], lay["conv_b"], xbc[None])[0]
         y = oracle.ssm_step(ssm_b[0], xc[None, :E], dt[None], lay["A_log"], lay["dt_bias"], lay["D"],
                             xc[None, E:E + N], xc[None, E + N:])[0]
         gg = oracle.gate(y, z)
-        q2, s2 = oracle.rmsnorm_quantize(gg[None], lay["gnorm_w"])
-        out, _, _ = oracle.linear_core(lay["out_proj"], q2[0], s2[0])
+        q2, s2, v2, rms2 = oracle.rmsnorm_quantize(gg[None], lay["gnorm_w"])
+        tf2 = oracle.lora_down(lay["out_proj"], v2[0], rms2[0])
+        out, _ = oracle.linear_core(lay["out_proj"], q2[0], s2[0], tf2)
         h_b = (h_b[0] + out).astype(np.float32)
         assert np.array_equal(h_a[0], h_b)
         assert np.array_equal(ssm_a, ssm_b) and np.array_equal(conv_a, conv_b)
