@@ -30,8 +30,11 @@ constexpr int SH0 = 2 * E;              // first in_proj row every CTA needs (B 
 constexpr int NSH = 2 * N + H;          // 320 such rows
 constexpr int NT = 512, NW = NT / 32;   // NW == R: warp r computes LoRA row r's partial sums
 constexpr int MAX_IN = 64, MAX_OUT = 16, MAX_SSM = 32;
-constexpr int MIN_CTAS = 133, MAX_CTAS = 256;
+constexpr int MIN_CTAS = 137, MAX_CTAS = 256;  // >= 137: at most 15 out_proj rows per CTA
 static_assert(NW == R, "one warp per LoRA row");
+constexpr int kPrefetchThread = 32;     // warp 1 issues the next layer's L2 prefetches
+constexpr int kChainWarp = NW - 1;      // warp 15 computes the fp64 scale chain (no out_proj row)
+constexpr int kChainBase = kChainWarp * 32;
 
 enum { CTR_H = 0, CTR_BC, CTR_G, N_CTR };
 constexpr int CTR_STRIDE = 32;          // one 128-byte line per counter
@@ -200,9 +203,32 @@ __device__ __forceinline__ int bits_dot(uint4 w, const uint4* qp4) {
 // Sum of one LoRA row's partial sums: thread t adds the partials of row t % R from every CTA
 // (t + NT k); a warp then holds row r in lanes r and r + 16.
 __device__ __forceinline__ double gather_partials(const double* part, int NC) {
+  constexpr int K = MAX_CTAS * R / NT;  // all loads in flight at once
+  double pv[K];
+#pragma unroll
+  for (int k = 0; k < K; ++k) {
+    const int j = threadIdx.x + k * NT;
+    pv[k] = j < NC * R ? __ldcg(part + j) : 0.0;
+  }
   double u = 0.0;
-  for (int j = threadIdx.x; j < NC * R; j += NT) u += __ldcg(part + j);
+#pragma unroll
+  for (int k = 0; k < K; ++k) u += pv[k];
   return u + __shfl_xor_sync(0xffffffffu, u, 16);
+}
+
+// The fp64 scale chain of one RMSNorm+quantize: thread k < R computes the LoRA intermediate of row k
+// from the per-warp partial sums, thread R the quantizer scale.
+__device__ __forceinline__ void scale_chain(int k, double ss, float s0, int n, float lbs,
+                                            const double (*red_u)[R], float* tf, float* s_scale) {
+  const double rms = rms_of(ss, n);
+  if (k < R) {
+    double ut = 0.0;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) ut += red_u[w][k];
+    tf[k] = lora_tf(ut, lbs, rms);
+  } else {
+    *s_scale = rms_scale(s0, rms);
+  }
 }
 
 // ------------------------------------------------------------------------------ the kernel
@@ -237,7 +263,7 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ P
   __shared__ float bc_st[2 * N][3];
   __shared__ float bc_new[2 * N];
   __shared__ __align__(16) float Bsm[N];
-  __shared__ __align__(16) float Csm[N];
+  __shared__ __align__(16) double Cd[N];
   // SSM rows
   __shared__ float zsm[MAX_SSM], xsm[MAX_SSM], gsm[MAX_SSM];
   __shared__ float dtv[2], dAv[2], Dv[2];
@@ -287,10 +313,11 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ P
     const bool has_next = l + 1 < p.n_layers;
 
     // ---------------------------------------------------------------- loads for the whole layer
-    if (tid < 2 && has_next) {
-      // this CTA's slice of the next layer, and (spread over CTAs 0..4) the parts every CTA reads
+    if ((tid == kPrefetchThread || tid == kPrefetchThread + 1) && has_next) {
+      // this CTA's slice of the next layer, and (spread over CTAs 0..4) the parts every CTA reads.
+      // Issued by warp 1: a bulk prefetch stalls its thread, and thread 0 polls the counters.
       const LayerPtrs& Nx = p.L[l + 1];
-      if (tid == 0) {
+      if (tid == kPrefetchThread) {
         prefetch_l2(Nx.in_bits + (size_t)(SH0 + sh0) * (DM / 32), n_sh * (DM / 8));
         prefetch_l2(Nx.in_bits + (size_t)rs0 * (DM / 32), n_ssm * (DM / 8));
         prefetch_l2(Nx.in_bits + (size_t)(E + rs0) * (DM / 32), n_ssm * (DM / 8));
@@ -369,9 +396,9 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ P
       nw_next = __ldg(Nx.norm_w + ro0 + lane);
     }
     float lbs_in = 0.f, lbs_out = 0.f;
-    if (tid < R) {
-      lbs_in = __ldg(Lp.in_lbs + tid);
-      lbs_out = __ldg(Lp.out_lbs + tid);
+    if (tid >= kChainBase && tid < kChainBase + R) {
+      lbs_in = __ldg(Lp.in_lbs + tid - kChainBase);
+      lbs_out = __ldg(Lp.out_lbs + tid - kChainBase);
     }
     // own x channels: conv taps, bias, state (thread NSH + j handles channel rs0 + j)
     float4 cw = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -422,6 +449,8 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ P
     // ---------------------------------------------------------------- phase A: h -> in_proj
     if (!block_wait(p.ctr + CTR_H * CTR_STRIDE, NC * (l + 1), p.err, p.status, p.spin_limit, &sflag))
       return;
+    double ssA;
+    float s0A;
     {
       float v[4];
       double ss = 0.0;
@@ -461,18 +490,9 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ P
       }
       sq = warp_sum(sq);
       if (lane == 0) red_i[warp] = sq;
-      if (tid <= R) {
-        const double rms = rms_of(ss, DM);
-        if (tid < R) {
-          double ut = 0.0;
-#pragma unroll
-          for (int w = 0; w < NW; ++w) ut += red_u[w][tid];
-          tf[tid] = lora_tf(ut, lbs_in, rms);
-        } else {
-          s_scale = rms_scale(s0, rms);
-        }
-      }
       __syncthreads();
+      ssA = ss;
+      s0A = s0;
     }
     int sumq = 0;
 #pragma unroll
@@ -493,6 +513,10 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ P
         }
       }
     }
+    // the fp64 scale chain (RMS, LoRA intermediate, quantizer scale), off the GEMV's critical path: the
+    // chain warp has no pass-1 rows, and the epilogue needs the results only after the B/C wait
+    if (tid >= kChainBase && tid <= kChainBase + R) scale_chain(tid - kChainBase, ssA, s0A, DM, lbs_in,
+                                                              red_u, tf, &s_scale);
 
     // ---------------------------------------------------------------- phase B: epilogues + SSM
     if (!block_wait(p.ctr + CTR_BC * CTR_STRIDE, NC * (l + 1), p.err, p.status, p.spin_limit, &sflag))
@@ -505,7 +529,7 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ P
         bc_new[tid] = y;
         const float xc = conv_out(bc_w[tid], bc_b[tid], bc_st[tid][0], bc_st[tid][1], bc_st[tid][2], y);
         if (tid < N) Bsm[tid] = xc;
-        else Csm[tid - N] = xc;
+        else Cd[tid - N] = (double)xc;
       } else if (dt_own) {
         const float dt = ssm_dt(y, dtb);
         dtv[dt_head - hA] = dt;
@@ -536,17 +560,18 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ P
         const float xv = xsm[rr];
         const float dtx = fmul(dt, xv);
         const float4 b4 = reinterpret_cast<const float4*>(Bsm)[lane];
-        const float4 c4 = reinterpret_cast<const float4*>(Csm)[lane];
+        const double2 c01 = reinterpret_cast<const double2*>(Cd)[2 * lane];
+        const double2 c23 = reinterpret_cast<const double2*>(Cd)[2 * lane + 1];
         float4 s4 = sv[ps];
         s4.x = ssm_state(dA, s4.x, dtx, b4.x);
         s4.y = ssm_state(dA, s4.y, dtx, b4.y);
         s4.z = ssm_state(dA, s4.z, dtx, b4.z);
         s4.w = ssm_state(dA, s4.w, dtx, b4.w);
         snew[ps] = s4;
-        double acc = (double)s4.x * (double)c4.x;
-        acc = fma((double)s4.y, (double)c4.y, acc);
-        acc = fma((double)s4.z, (double)c4.z, acc);
-        acc = fma((double)s4.w, (double)c4.w, acc);
+        double acc = (double)s4.x * c01.x;
+        acc = fma((double)s4.y, c01.y, acc);
+        acc = fma((double)s4.z, c23.x, acc);
+        acc = fma((double)s4.w, c23.y, acc);
         acc = warp_sum(acc);
         if (lane == 0) {
           const float y = __double2float_rn(dadd(acc, dmul((double)Dv[hi], (double)xv)));
@@ -620,27 +645,20 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ P
       }
       sq = warp_sum(sq);
       if (lane == 0) red_i[warp] = sq;
-      if (tid <= R) {
-        const double rms = rms_of(ss, E);
-        if (tid < R) {
-          double ut = 0.0;
+      if (warp == kChainWarp) {
+        // publish this warp's codes to the GEMV warps without waiting, then run the scale chain
+        asm volatile("bar.arrive 1, %0;" ::"n"(NT) : "memory");
+        if (lane <= R) scale_chain(lane, ss, s0, E, lbs_out, red_u, tf, &s_scale);
+      } else {
+        asm volatile("bar.sync 1, %0;" ::"n"(NT) : "memory");
+        int sumq_c = 0;
 #pragma unroll
-          for (int w = 0; w < NW; ++w) ut += red_u[w][tid];
-          tf[tid] = lora_tf(ut, lbs_out, rms);
-        } else {
-          s_scale = rms_scale(s0, rms);
-        }
+        for (int w = 0; w < NW; ++w) sumq_c += red_i[w];
+        const uint4* qp4 = reinterpret_cast<const uint4*>(q_perm) + lane;
+        int S = bits_dot<E / 128>(w_out, qp4);
+        S = warp_sum(S);
+        if (lane == 0 && slot_out < n_out) acc_out[slot_out] = 2 * S - sumq_c;
       }
-      __syncthreads();
-    }
-    sumq = 0;
-#pragma unroll
-    for (int w = 0; w < NW; ++w) sumq += red_i[w];
-    {
-      const uint4* qp4 = reinterpret_cast<const uint4*>(q_perm) + lane;
-      int S = bits_dot<E / 128>(w_out, qp4);
-      S = warp_sum(S);
-      if (lane == 0 && slot_out < n_out) acc_out[slot_out] = 2 * S - sumq;
     }
     __syncthreads();
     if (tid < n_out) {
