@@ -1,17 +1,445 @@
-// Prefill of one DF-SSM linear on int8 tcgen05 tensor cores (placeholder until the kernel lands).
+// M-token prefill of one DF-SSM linear on the 5th-generation (tcgen05) int8 tensor cores
+// (gist.science technical summary of DF-SSM, §2.C: "1-bit packed weights are expanded on-the-fly to int8
+// and processed via ... INT8 tensor cores").  At M = 2048 tokens the scaffold matmul is a dense
+// contraction, so it runs as an int8 GEMM with int32 accumulation in tensor memory:
+//   1. quantize every token (per-token absmax int8 codes, natural order) and its fp64 LoRA
+//      down-projection (the decode path's quantize kernel, one CTA per token);
+//   2. expand the packed sign bits once to +-1 int8 rows in the workspace;
+//   3. acc[m][n] = sum_k q[m][k] w[n][k] on tcgen05.mma kind::i8 (128x256 tiles, K steps of 128 bytes,
+//      TMA loads with 128-byte swizzle into a 4-stage shared-memory ring, accumulator in TMEM), then
+//      the epilogue reads TMEM and writes y[m][n] = acc s[m] sW[n] + sA[n] sum_r W_A[n][r] tf[m][r].
+// The integer accumulators are exact; the epilogue is fp32 with fused multiply-add.
+//
+// Every wait on an mbarrier is bounded: a wait that runs out of budget sets the workspace error word,
+// the CTA stops issuing work, waits (bounded) for its copies in flight, frees its tensor memory and
+// returns.
+
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <cstdio>
+#include <mutex>
+
 #include "common.cuh"
 #include "internal.h"
 
 namespace dfssm {
-size_t prefill_workspace_bytes(int M, int d_in, int d_out) {
-  (void)M; (void)d_in; (void)d_out;
-  return 256;
+namespace prefill {
+
+constexpr int BM = 128, BN = 256, BK = 128;  // tile; BK bytes = BK int8 elements
+constexpr int STAGES = 4;
+constexpr int UMMA_K = 32;                   // K of one kind::i8 MMA
+constexpr int A_BYTES = BM * BK, B_BYTES = BN * BK, STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int NT = 192;                      // warp 0 TMA, warp 1 MMA + TMEM owner, warps 2..5 epilogue
+constexpr int TMEM_COLS = BN;                // 128 lanes x 256 int32 columns
+constexpr size_t SMEM_BYTES = (size_t)STAGES * STAGE_BYTES + 1024 /* align */ + 256 /* barriers */;
+constexpr long long kWaitBudget = 4000000000LL;  // clock cycles per wait (~2 s)
+
+struct EpiArgs {
+  const float* s;       // [M] per-token scale
+  const float* tf;      // [M][16] LoRA intermediate
+  const float* w_scale; // [N]
+  const float* la_scale;// [N]
+  const int8_t* la;     // [N][rank]
+  int rank;
+  float* y;             // [M][N]
+  int32_t* acc;         // [M][N] or null
+  int M, N, K;
+  int* err;
+};
+
+// ------------------------------------------------------------------------------ PTX helpers
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
 }
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait for the given phase parity; false when the budget ran out or another role aborted.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity)) {
+    if (*abort_flag) return false;
+    if (clock64() - t0 > kWaitBudget) return false;
+  }
+  return true;
+}
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int c0, int c1,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
+      "[%4];" ::"r"(smem_u32(dst)),
+      "l"(map), "r"(c0), "r"(c1), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// K-major operand in 128-byte-swizzled rows of 128 bytes: 8-row groups 1024 bytes apart.
+__device__ __forceinline__ uint64_t umma_desc_k_sw128(uint32_t smem_addr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((smem_addr >> 4) & 0x3FFFu);  // start address (16-byte units)
+  d |= (uint64_t)1 << 16;                        // leading byte offset (unused with swizzle)
+  d |= (uint64_t)(1024 >> 4) << 32;              // stride byte offset: next 8-row group
+  d |= (uint64_t)1 << 46;                        // descriptor version for sm_100
+  d |= (uint64_t)2 << 61;                        // 128-byte swizzle
+  return d;
+}
+// kind::i8 instruction descriptor: D s32, A s8, B s8, both K-major, M = BM, N = BN.
+constexpr uint32_t kIdesc = (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
+                            ((uint32_t)(BM >> 4) << 24);
+
+__device__ __forceinline__ void umma_i8(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t accum) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(kIdesc), "r"(accum)
+      : "memory");
+}
+__device__ __forceinline__ void umma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   smem_u32(bar))
+               : "memory");
+}
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, "
+      "[%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
+        "=r"(r[15])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// ------------------------------------------------------------------------------ kernels
+
+// w8[n][k] = +1 for a set sign bit, -1 otherwise.  One thread per 32-bit word (32 weights).
+__global__ void expand_bits_kernel(const uint32_t* __restrict__ bits, int8_t* __restrict__ w8,
+                                   long long words) {
+  const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= words) return;
+  const uint32_t w = bits[i];
+  uint32_t out[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const uint32_t nib = (w >> (4 * j)) & 0xFu;
+    uint32_t v = 0;
+#pragma unroll
+    for (int b = 0; b < 4; ++b) v |= (((nib >> b) & 1u) ? 0x01u : 0xFFu) << (8 * b);
+    out[j] = v;
+  }
+  uint4* dst = reinterpret_cast<uint4*>(w8 + i * 32);
+  dst[0] = make_uint4(out[0], out[1], out[2], out[3]);
+  dst[1] = make_uint4(out[4], out[5], out[6], out[7]);
+}
+
+__global__ void __launch_bounds__(NT, 1)
+    gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
+                const EpiArgs ep) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+  uint64_t* empty = full + STAGES;
+  uint64_t* tmem_full = empty + STAGES;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(tmem_full + 1);
+  __shared__ int abort_flag;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n0 = blockIdx.x * BN, m0 = blockIdx.y * BM;
+  const int kblocks = ep.K / BK;
+
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(tmem_full, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(tmem_holder)),
+                 "r"(TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+  __syncthreads();
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+  const uint32_t tmem_base = *tmem_holder;
+
+  if (warp == 0 && lane == 0) {
+    // ---- TMA producer
+    int issued = 0;
+    for (int kb = 0; kb < kblocks; ++kb) {
+      const int s = kb % STAGES;
+      if (kb >= STAGES && !mbar_wait(&empty[s], ((kb / STAGES) - 1) & 1, &abort_flag)) {
+        abort_flag = 1;
+        break;
+      }
+      unsigned char* a_dst = smem + s * STAGE_BYTES;
+      unsigned char* b_dst = a_dst + A_BYTES;
+      mbar_expect_tx(&full[s], STAGE_BYTES);
+      tma_load_2d(a_dst, &map_a, kb * BK, m0, &full[s]);
+      tma_load_2d(b_dst, &map_b, kb * BK, n0, &full[s]);
+      ++issued;
+    }
+    // copies still in flight complete before this CTA may exit
+    for (int kb = (issued > STAGES ? issued - STAGES : 0); kb < issued; ++kb)
+      mbar_wait(&full[kb % STAGES], (kb / STAGES) & 1, &abort_flag);
+  } else if (warp == 1 && lane == 0) {
+    // ---- MMA issuer: one thread issues every tcgen05.mma of the tile
+    bool ok = true;
+    for (int kb = 0; kb < kblocks && ok; ++kb) {
+      const int s = kb % STAGES;
+      if (!mbar_wait(&full[s], (kb / STAGES) & 1, &abort_flag)) {
+        abort_flag = 1;
+        ok = false;
+        break;
+      }
+      asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+      const uint32_t a_addr = smem_u32(smem + s * STAGE_BYTES);
+      const uint32_t b_addr = a_addr + A_BYTES;
+#pragma unroll
+      for (int kk = 0; kk < BK / UMMA_K; ++kk)
+        umma_i8(tmem_base, umma_desc_k_sw128(a_addr + kk * UMMA_K), umma_desc_k_sw128(b_addr + kk * UMMA_K),
+                (kb > 0 || kk > 0) ? 1u : 0u);
+      umma_commit(&empty[s]);  // frees the stage once these MMAs have read it
+    }
+    umma_commit(tmem_full);    // accumulator complete (also signals after an abort)
+  } else if (warp >= 2) {
+    // ---- epilogue: warp w reads TMEM lanes [32 (w % 4), +32) = tile rows
+    const int q = warp & 3;
+    const int row = q * 32 + lane;
+    const int m = m0 + row;
+    const bool ok = mbar_wait(tmem_full, 0, &abort_flag);
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+    if (!ok || abort_flag) {
+      if (lane == 0) atomicExch(ep.err, 1);
+    } else {
+      float sm = 0.f;
+      float tfm[DFSSM_MAX_RANK];
+#pragma unroll
+      for (int r = 0; r < DFSSM_MAX_RANK; ++r) tfm[r] = 0.f;
+      if (m < ep.M) {
+        sm = ep.s[m];
+#pragma unroll
+        for (int r = 0; r < DFSSM_MAX_RANK; ++r) tfm[r] = ep.tf[(size_t)m * DFSSM_MAX_RANK + r];
+      }
+      for (int c0 = 0; c0 < BN; c0 += 16) {
+        uint32_t v[16];
+        tmem_ld16(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)c0, v);
+        if (m >= ep.M) continue;
+        float out[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const int n = n0 + c0 + j;
+          float yv = 0.f;
+          if (n < ep.N) {
+            const int acc = (int)v[j];
+            float lora = 0.f;
+            if (ep.rank == DFSSM_MAX_RANK) {
+              const uint4 wa4 = __ldg(reinterpret_cast<const uint4*>(ep.la) + n);
+              const int8_t* wa = reinterpret_cast<const int8_t*>(&wa4);
+#pragma unroll
+              for (int r = 0; r < DFSSM_MAX_RANK; ++r) lora = fmaf((float)wa[r], tfm[r], lora);
+            } else {
+              for (int r = 0; r < ep.rank; ++r) lora = fmaf((float)ep.la[(size_t)n * ep.rank + r], tfm[r], lora);
+            }
+            yv = fmaf((float)acc, sm * __ldg(ep.w_scale + n), ep.rank > 0 ? __ldg(ep.la_scale + n) * lora : 0.f);
+            if (ep.acc) ep.acc[(size_t)m * ep.N + n] = acc;
+          }
+          out[j] = yv;
+        }
+        float* yrow = ep.y + (size_t)m * ep.N + n0 + c0;
+        if (n0 + c0 + 16 <= ep.N && (ep.N % 4) == 0) {
+#pragma unroll
+          for (int j = 0; j < 16; j += 4)
+            *reinterpret_cast<float4*>(yrow + j) = make_float4(out[j], out[j + 1], out[j + 2], out[j + 3]);
+        } else {
+          for (int j = 0; j < 16 && n0 + c0 + j < ep.N; ++j) yrow[j] = out[j];
+        }
+      }
+    }
+  }
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+  __syncthreads();
+  if (abort_flag && threadIdx.x == 0) atomicExch(ep.err, 1);
+  if (warp == 1) {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(TMEM_COLS)
+                 : "memory");
+  }
+}
+
+// ------------------------------------------------------------------------------ host side
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// Row-major int8 matrix [rows][K] viewed as a 2-D tensor (K innermost) with box {BK, box_rows}.
+bool make_map(CUtensorMap* map, const void* base, int rows, int K, int box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)K};
+  cuuint32_t box[2] = {(cuuint32_t)BK, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides,
+                        box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+inline size_t al256(size_t x) { return (x + 255) & ~size_t(255); }
+
+struct Ws {
+  int8_t* xq;
+  float* s;
+  int32_t* sumq;
+  float* tf;
+  int8_t* w8;
+  int* err;
+};
+
+size_t ws_bytes(int M, int K, int N) {
+  return al256((size_t)M * K) + al256((size_t)M * 4) * 2 + al256((size_t)M * 16 * 4) +
+         al256((size_t)N * K) + 256;
+}
+
+Ws carve(void* base, int M, int K, int N) {
+  char* p = static_cast<char*>(base);
+  Ws w;
+  w.xq = reinterpret_cast<int8_t*>(p);
+  p += al256((size_t)M * K);
+  w.s = reinterpret_cast<float*>(p);
+  p += al256((size_t)M * 4);
+  w.sumq = reinterpret_cast<int32_t*>(p);
+  p += al256((size_t)M * 4);
+  w.tf = reinterpret_cast<float*>(p);
+  p += al256((size_t)M * 16 * 4);
+  w.w8 = reinterpret_cast<int8_t*>(p);
+  p += al256((size_t)N * K);
+  w.err = reinterpret_cast<int*>(p);
+  return w;
+}
+
+}  // namespace prefill
+
+size_t prefill_workspace_bytes(int M, int d_in, int d_out) { return prefill::ws_bytes(M, d_in, d_out); }
+
 }  // namespace dfssm
 
 extern "C" int dfssm_linear_prefill(const dfssm_linear_t* lin, const float* x, int M, float* y,
                                     void* workspace, size_t ws_bytes, const dfssm_debug_t* dbg,
                                     void* stream) {
-  (void)lin; (void)x; (void)M; (void)y; (void)workspace; (void)ws_bytes; (void)dbg; (void)stream;
-  return DFSSM_EUNSUPPORTED;
+  using namespace dfssm;
+  if (!lin || !x || !y || M < 1) return DFSSM_EINVAL;
+  if (lin->d_out < 1 || lin->d_in < 128 || lin->d_in % 128 || lin->d_in > 8192) return DFSSM_EINVAL;
+  if (lin->rank < 0 || lin->rank > DFSSM_MAX_RANK) return DFSSM_EINVAL;
+  if (!lin->bits || !lin->w_scale) return DFSSM_EINVAL;
+  if (lin->rank > 0 && (!lin->lora_b || !lin->lora_b_scale || !lin->lora_a || !lin->lora_a_scale))
+    return DFSSM_EINVAL;
+  if ((reinterpret_cast<uintptr_t>(lin->bits) & 15) || (reinterpret_cast<uintptr_t>(x) & 15) ||
+      (reinterpret_cast<uintptr_t>(y) & 15))
+    return DFSSM_EALIGN;
+  if (lin->rank == DFSSM_MAX_RANK && (reinterpret_cast<uintptr_t>(lin->lora_a) & 15)) return DFSSM_EALIGN;
+  if (lin->rank > 0 && (reinterpret_cast<uintptr_t>(lin->lora_b) & 3)) return DFSSM_EALIGN;
+  const int K = lin->d_in, N = lin->d_out;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255) ||
+      ws_bytes < prefill::ws_bytes(M, K, N))
+    return DFSSM_EWORKSPACE;
+  int dev = 0, major = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess || major != 10)
+    return DFSSM_EDEVICE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  prefill::Ws w = prefill::carve(workspace, M, K, N);
+
+  // 1. per-token quantization and LoRA down-projection
+  QuantArgs qa{};
+  qa.x = x;
+  qa.ldx = K;
+  qa.norm_w = nullptr;
+  qa.n = K;
+  qa.B = M;
+  qa.lora_b = lin->lora_b;
+  qa.lora_b_scale = lin->lora_b_scale;
+  qa.rank = lin->rank;
+  qa.permute = false;
+  qa.out.q = w.xq;
+  qa.out.s = w.s;
+  qa.out.sumq = w.sumq;
+  qa.out.tf = w.tf;
+  if (dbg) {
+    qa.dbg_xq = dbg->xq;
+    qa.dbg_s = dbg->xscale;
+    qa.dbg_tf = dbg->lora_tf;
+  }
+  cudaError_t e = launch_quant(qa, st);
+  if (e != cudaSuccess) return record_cuda_failure(e);
+  // 2. +-1 int8 weights
+  const long long words = (long long)N * (K / 32);
+  prefill::expand_bits_kernel<<<(unsigned)((words + 255) / 256), 256, 0, st>>>(lin->bits, w.w8, words);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return record_cuda_failure(e);
+  e = cudaMemsetAsync(w.err, 0, sizeof(int), st);
+  if (e != cudaSuccess) return record_cuda_failure(e);
+  // 3. tcgen05 GEMM + epilogue
+  CUtensorMap map_a, map_b;
+  if (!prefill::make_map(&map_a, w.xq, M, K, prefill::BM) || !prefill::make_map(&map_b, w.w8, N, K, prefill::BN))
+    return DFSSM_EUNSUPPORTED;
+  prefill::EpiArgs ep{};
+  ep.s = w.s;
+  ep.tf = w.tf;
+  ep.w_scale = lin->w_scale;
+  ep.la_scale = lin->lora_a_scale;
+  ep.la = lin->lora_a;
+  ep.rank = lin->rank;
+  ep.y = y;
+  ep.acc = dbg ? dbg->acc : nullptr;
+  ep.M = M;
+  ep.N = N;
+  ep.K = K;
+  ep.err = w.err;
+  static bool attr_done = false;
+  if (!attr_done) {
+    e = cudaFuncSetAttribute(prefill::gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)prefill::SMEM_BYTES);
+    if (e != cudaSuccess) return record_cuda_failure(e);
+    attr_done = true;
+  }
+  dim3 grid((N + prefill::BN - 1) / prefill::BN, (M + prefill::BM - 1) / prefill::BM);
+  prefill::gemm_kernel<<<grid, prefill::NT, prefill::SMEM_BYTES, st>>>(map_a, map_b, ep);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return record_cuda_failure(e);
+  return DFSSM_OK;
 }

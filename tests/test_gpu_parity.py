@@ -274,3 +274,55 @@ def test_device_wait_timeout_is_reported(dev):
     h_ref = np.ascontiguousarray(model["emb"][0])
     oracle.layer_decode(olayers[0], h_ref, conv[0], ssm[0])
     assert_tol(h.cpu().numpy(), h_ref, "decode after a reported timeout")
+
+
+def _prefill_compare(dev, lin_host, x, rows):
+    """Prefill through the C ABI vs the oracle: int8 codes and scales of every token exact; scaffold
+    accumulators exact and the LoRA intermediate / outputs within tolerance on the listed rows."""
+    from bit_quantized_mamba_b200 import dfssm
+    L = dfssm.Linear.from_host(lin_host, dev)
+    M = x.shape[0]
+    dbg = dict(acc=torch.zeros((M, L.d_out), dtype=torch.int32, device=dev),
+               lora_tf=torch.zeros((M, L.rank), dtype=torch.float32, device=dev),
+               xq=torch.zeros((M, L.d_in), dtype=torch.int8, device=dev),
+               xscale=torch.zeros(M, dtype=torch.float32, device=dev))
+    y = dfssm.linear_prefill(L, to_dev(x, dev), debug=dbg)
+    torch.cuda.synchronize()
+    OL = oracle.Linear.from_dict(lin_host)
+    rq, rs = oracle.quantize(x)
+    assert np.array_equal(dbg["xq"].cpu().numpy(), rq), "prefill int8 codes differ"
+    assert np.array_equal(dbg["xscale"].cpu().numpy(), rs), "prefill scales differ"
+    yg, accg, tfg = y.cpu().numpy(), dbg["acc"].cpu().numpy(), dbg["lora_tf"].cpu().numpy()
+    for m in rows:
+        tf = oracle.lora_down(OL, x[m])
+        assert_tol(tfg[m], tf, f"prefill tf row {m}")
+        yr, accr = oracle.linear_core(OL, rq[m], rs[m], tf)
+        assert np.array_equal(accg[m], accr), f"prefill scaffold accumulators differ at row {m}"
+        assert_tol(yg[m], yr, f"prefill y row {m}")
+
+
+def test_prefill_ragged_small(dev):
+    """M and d_out not multiples of the 128 x 256 tile; every row checked."""
+    gen = np.random.default_rng(61)
+    lin = inputs.linear(gen, 300, 256, 16)
+    x = inputs.normal(gen, (200, 256)) * np.float32(2)
+    x[7] = 0.0
+    _prefill_compare(dev, lin, x, range(200))
+
+
+def test_prefill_rank_below_16(dev):
+    gen = np.random.default_rng(62)
+    lin = inputs.linear(gen, 256, 384, 5)
+    x = inputs.normal(gen, (130, 384))
+    _prefill_compare(dev, lin, x, range(130))
+
+
+@pytest.mark.parametrize("which", ["in_proj", "out_proj"])
+def test_prefill_full_size(dev, which):
+    """The 2048-token prefill of the in_proj / out_proj-shaped linears: every token's codes, 12 sampled
+    tokens across all output columns."""
+    p = inputs.prefill(seed=4, m=2048, vocab=16)
+    lin = p["in_proj"] if which == "in_proj" else p["out_proj"]
+    x = p["x_in"] if which == "in_proj" else p["x_out"]
+    rows = [0, 1, 127, 128, 129, 511, 1000, 1023, 1024, 1500, 2046, 2047]
+    _prefill_compare(dev, lin, x, rows)
