@@ -37,6 +37,14 @@ BYTES_LAYER = (BYTES_IN_PROJ + BYTES_OUT_PROJ + 4352 * 5 * 4 + 4352 * 3 * 4 * 2
 BYTES_TOKEN = 48 * BYTES_LAYER
 
 
+def peaks_bf16():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["bf16_tflops"])
+    except Exception:
+        return 1590.0
+
+
 def peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -281,38 +289,102 @@ def run_ours(args, rank, world, local_rank):
     e2e_ms = max_over_ranks(e0.elapsed_time(e1))
     e2e_value = world * N_TOKENS * e2e_steps / (e2e_ms / 1e3)
 
-    # ---- scaffold GEMV sweep: 48 in_proj / out_proj copies, L2 flushed before each pass
+    # ---- scaffold GEMV sweep: 48 in_proj / out_proj copies through dfssm_linear_decode, captured in
+    # a CUDA graph (48 calls = 96 kernels, PDL-chained); L2 flushed before each timed replay
     hbm, peak_kind = peaks()
     flush = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device=dev)
     gemv = {}
-    for which, data_fn, nbytes in (("in_proj", inputs.in_proj_stack, BYTES_IN_PROJ),
-                                   ("out_proj", inputs.out_proj_stack, BYTES_OUT_PROJ)):
-        data = data_fn()
-        lins = [dfssm.Linear.from_host(l, dev) for l in data["linears"]]
-        xd = torch.from_numpy(data["x"]).to(dev)
-        for B in (1, 4, 16):
-            y = torch.empty((B, lins[0].d_out), dtype=torch.float32, device=dev)
-            gws = dfssm.workspace(dfssm.workspace_size(dfssm.OP_LINEAR_DECODE, B, lins[0].d_in,
-                                                       lins[0].d_out), dev)
-            xb = xd[:B].contiguous()
-            tot = 0.0
-            reps = 5
+    if not args.no_extras:
+        for which, data_fn, nbytes in (("in_proj", inputs.in_proj_stack, BYTES_IN_PROJ),
+                                       ("out_proj", inputs.out_proj_stack, BYTES_OUT_PROJ)):
+            data = data_fn()
+            lins = [dfssm.Linear.from_host(l, dev) for l in data["linears"]]
+            xd = torch.from_numpy(data["x"]).to(dev)
+            for B in (1, 4, 16):
+                y = torch.empty((B, lins[0].d_out), dtype=torch.float32, device=dev)
+                gws = dfssm.workspace(dfssm.workspace_size(dfssm.OP_LINEAR_DECODE, B, lins[0].d_in,
+                                                           lins[0].d_out), dev)
+                xb = xd[:B].contiguous()
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.stream(stream):
+                    for L in lins:  # warm every launch configuration before capture
+                        dfssm.linear_decode(L, xb, y, gws, stream=torch.cuda.current_stream())
+                    torch.cuda.synchronize()
+                    with torch.cuda.graph(g, stream=stream):
+                        for L in lins:
+                            dfssm.linear_decode(L, xb, y, gws, stream=torch.cuda.current_stream())
+                tot, reps = 0.0, 10
+                with torch.cuda.stream(stream):
+                    for r in range(reps + 2):
+                        flush.fill_(r & 0xFF)
+                        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                        a.record()
+                        g.replay()
+                        b.record()
+                        b.synchronize()
+                        if r >= 2:
+                            tot += a.elapsed_time(b)
+                del g
+                us_per_call = tot / reps / len(lins) * 1e3
+                gbs = nbytes / (us_per_call * 1e-6) / 1e9
+                gemv[f"{which}_B{B}"] = {"us_per_call": round(us_per_call, 3), "GB_s": round(gbs, 1),
+                                         "frac_of_measured_hbm": round(gbs / hbm, 3)}
+            del lins
+
+    # ---- prefill (2048 tokens) on tcgen05 int8, and the int8 LM head on the last token
+    prefill = {}
+    if not args.no_extras:
+        pdata = inputs.prefill(seed=4, m=2048)
+        int8_peak = 2.0 * peaks_bf16()  # int8 dense = 2x bf16 dense (nominal ratio)
+        for which, xkey in (("in_proj", "x_in"), ("out_proj", "x_out")):
+            L = dfssm.Linear.from_host(pdata[which], dev)
+            xin = torch.from_numpy(pdata[xkey]).to(dev)
+            M = xin.shape[0]
+            yp = torch.empty((M, L.d_out), dtype=torch.float32, device=dev)
+            pws = dfssm.workspace(dfssm.workspace_size(dfssm.OP_LINEAR_PREFILL, M, L.d_in, L.d_out), dev)
             with torch.cuda.stream(stream):
-                for r in range(reps + 1):
+                for r in range(3):
+                    dfssm.linear_prefill(L, xin, yp, pws, stream=torch.cuda.current_stream())
+                torch.cuda.synchronize()
+                tot, reps = 0.0, 10
+                for r in range(reps):
                     flush.fill_(r & 0xFF)
                     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
                     a.record()
-                    for L in lins:
-                        dfssm.linear_decode(L, xb, y, gws, stream=torch.cuda.current_stream())
+                    dfssm.linear_prefill(L, xin, yp, pws, stream=torch.cuda.current_stream())
                     b.record()
                     b.synchronize()
-                    if r > 0:
-                        tot += a.elapsed_time(b)
-            us_per_call = tot / reps / len(lins) * 1e3
-            gbs = nbytes / (us_per_call * 1e-6) / 1e9
-            gemv[f"{which}_B{B}"] = {"us_per_call": round(us_per_call, 3), "GB_s": round(gbs, 1),
-                                     "frac_of_measured_hbm": round(gbs / hbm, 3)}
-        del lins
+                    tot += a.elapsed_time(b)
+            ms = tot / reps
+            tops = 2.0 * M * L.d_out * L.d_in / (ms * 1e-3) / 1e12
+            prefill[which] = {"ms_per_call": round(ms, 4), "int8_TOPS": round(tops, 1),
+                              "frac_of_int8_peak": round(tops / int8_peak, 3)}
+        W = torch.from_numpy(pdata["lm_w"]).to(dev)
+        srow = torch.from_numpy(pdata["lm_s"]).to(dev)
+        xl = torch.from_numpy(pdata["x_in"][-1].copy()).to(dev)
+        logits = torch.empty(W.shape[0], dtype=torch.float32, device=dev)
+        lws = dfssm.workspace(dfssm.workspace_size(dfssm.OP_LM_HEAD, 1, W.shape[1], W.shape[0]), dev)
+        with torch.cuda.stream(stream):
+            for r in range(3):
+                dfssm.lm_head(W, srow, xl, logits, ws=lws, stream=torch.cuda.current_stream())
+            torch.cuda.synchronize()
+            tot, reps = 0.0, 10
+            for r in range(reps):
+                flush.fill_(r & 0xFF)
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record()
+                dfssm.lm_head(W, srow, xl, logits, ws=lws, stream=torch.cuda.current_stream())
+                b.record()
+                b.synchronize()
+                tot += a.elapsed_time(b)
+        ms = tot / reps
+        lm_bytes = W.numel() + 4 * W.shape[0]
+        prefill["lm_head"] = {"ms_per_call": round(ms, 4),
+                              "GB_s": round(lm_bytes / (ms * 1e-3) / 1e9, 1),
+                              "frac_of_measured_hbm": round(lm_bytes / (ms * 1e-3) / 1e9 / hbm, 3)}
+        prefill["int8_peak_TOPS"] = round(int8_peak, 1)
+        prefill["int8_peak_kind"] = "measured bf16 burst x 2 (nominal int8/bf16 ratio)"
+        del W
     del flush
     torch.cuda.synchronize()
 
@@ -335,6 +407,7 @@ def run_ours(args, rank, world, local_rank):
         "algorithmic_GB_s": BYTES_TOKEN * N_TOKENS / (ms_per_step * 1e-3) / 1e9,
         "roofline": roofline,
         "scaffold_gemv": gemv,
+        "prefill": prefill,
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": N_TOKENS * 2048 * 4,
                 "d2h_bytes_per_step": 2048 * 4},
         "gpu_launches": args.steps * N_TOKENS,
@@ -352,6 +425,22 @@ def run_ours(args, rank, world, local_rank):
     graph = None
 
 
+def run_prefill_profile(args):
+    """Eager prefill calls for an ncu launch list (no timing is reported)."""
+    import torch
+    from bit_quantized_mamba_b200 import build, dfssm, inputs
+    build.build()
+    dev = torch.device("cuda", 0)
+    p = inputs.prefill(seed=4, m=2048, vocab=16)
+    L = dfssm.Linear.from_host(p["in_proj"], dev)
+    x = torch.from_numpy(p["x_in"]).to(dev)
+    y = torch.empty((x.shape[0], L.d_out), dtype=torch.float32, device=dev)
+    ws = dfssm.workspace(dfssm.workspace_size(dfssm.OP_LINEAR_PREFILL, x.shape[0], L.d_in, L.d_out), dev)
+    for _ in range(args.warmup + 1):
+        dfssm.linear_prefill(L, x, y, ws)
+    torch.cuda.synchronize()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -360,6 +449,10 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the GEMV sweep, prefill and LM-head measurements")
+    ap.add_argument("--ncu-prefill", action="store_true",
+                    help="profiling mode: run the 2048-token in_proj prefill --warmup + 1 times and exit")
     ap.add_argument("--ncu", action="store_true",
                     help="profiling mode: decode --warmup tokens then one more token, eagerly, and exit")
     args = ap.parse_args()
@@ -370,6 +463,9 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", 0))
     if args.impl == "reference":
         run_reference(args, rank)
+        return
+    if args.ncu_prefill:
+        run_prefill_profile(args)
         return
     if world > 1:
         import datetime

@@ -373,8 +373,11 @@ static cudaError_t launch_fast(const GemvArgs& a, cudaStream_t st) {
   const size_t smem = (size_t)a.B * a.d_in;
   auto k = gemv_kernel<LPR, NSEG, BT>;
   if (smem > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
+    // once per instantiation (the largest size any call can need), not per launch, so that launches
+    // can be captured in a CUDA graph
+    static const cudaError_t set = cudaFuncSetAttribute(
+        k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)(DFSSM_MAX_BATCH * 8192));
+    if (set != cudaSuccess) return set;
   }
   return launch_pdl(k, dim3((a.d_out + RPC - 1) / RPC), dim3(kGemvThreads), smem, st, a);
 }
@@ -385,8 +388,9 @@ static cudaError_t launch_generic(const GemvArgs& a, cudaStream_t st) {
   const size_t smem = (size_t)a.B * a.d_in;
   auto k = gemv_generic_kernel<BT>;
   if (smem > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
+    static const cudaError_t set = cudaFuncSetAttribute(
+        k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)(DFSSM_MAX_BATCH * 8192));
+    if (set != cudaSuccess) return set;
   }
   return launch_pdl(k, dim3((a.d_out + RPC - 1) / RPC), dim3(kGemvThreads), smem, st, a);
 }

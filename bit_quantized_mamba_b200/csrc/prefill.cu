@@ -2,12 +2,13 @@
 // (gist.science technical summary of DF-SSM, §2.C: "1-bit packed weights are expanded on-the-fly to int8
 // and processed via ... INT8 tensor cores").  At M = 2048 tokens the scaffold matmul is a dense
 // contraction, so it runs as an int8 GEMM with int32 accumulation in tensor memory:
-//   1. quantize every token (per-token absmax int8 codes, natural order) and its fp64 LoRA
-//      down-projection (the decode path's quantize kernel, one CTA per token);
+//   1. quantize every token (per-token absmax int8 codes, natural order, exactly as in decode) and its
+//      LoRA down-projection (fp32, one warp per token);
 //   2. expand the packed sign bits once to +-1 int8 rows in the workspace;
 //   3. acc[m][n] = sum_k q[m][k] w[n][k] on tcgen05.mma kind::i8 (128x256 tiles, K steps of 128 bytes,
-//      TMA loads with 128-byte swizzle into a 4-stage shared-memory ring, accumulator in TMEM), then
-//      the epilogue reads TMEM and writes y[m][n] = acc s[m] sW[n] + sA[n] sum_r W_A[n][r] tf[m][r].
+//      TMA loads with 128-byte swizzle into a 4-stage shared-memory ring, two TMEM accumulators in a
+//      persistent kernel), then the epilogue reads TMEM and writes
+//      y[m][n] = acc s[m] sW[n] + sA[n] sum_r W_A[n][r] tf[m][r] while the next tile accumulates.
 // The integer accumulators are exact; the epilogue is fp32 with fused multiply-add.
 //
 // Every wait on an mbarrier is bounded: a wait that runs out of budget sets the workspace error word,
@@ -27,12 +28,9 @@ namespace dfssm {
 namespace prefill {
 
 constexpr int BM = 128, BN = 256, BK = 128;  // tile; BK bytes = BK int8 elements
-constexpr int STAGES = 4;
+constexpr int STAGES = 3;
 constexpr int UMMA_K = 32;                   // K of one kind::i8 MMA
 constexpr int A_BYTES = BM * BK, B_BYTES = BN * BK, STAGE_BYTES = A_BYTES + B_BYTES;
-constexpr int NT = 192;                      // warp 0 TMA, warp 1 MMA + TMEM owner, warps 2..5 epilogue
-constexpr int TMEM_COLS = BN;                // 128 lanes x 256 int32 columns
-constexpr size_t SMEM_BYTES = (size_t)STAGES * STAGE_BYTES + 1024 /* align */ + 256 /* barriers */;
 constexpr long long kWaitBudget = 4000000000LL;  // clock cycles per wait (~2 s)
 
 struct EpiArgs {
@@ -127,6 +125,12 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+// Exact fp32 value of a small integer (|w| < 2^22) without the conversion unit: the bit pattern of
+// 1.5 * 2^23 plus w is the float 1.5 * 2^23 + w.
+__device__ __forceinline__ float int8_to_f32(int w) {
+  return __int_as_float(0x4B400000 + w) - 12582912.0f;
+}
+
 // ------------------------------------------------------------------------------ kernels
 
 // w8[n][k] = +1 for a set sign bit, -1 otherwise.  One thread per 32-bit word (32 weights).
@@ -149,7 +153,84 @@ __global__ void expand_bits_kernel(const uint32_t* __restrict__ bits, int8_t* __
   dst[1] = make_uint4(out[4], out[5], out[6], out[7]);
 }
 
-__global__ void __launch_bounds__(NT, 1)
+// Quantization for the prefill: one warp per token.  Codes (natural order) and scale exactly as the
+// decode quantizer; the LoRA down-projection u = W_B x runs in fp32 with W_B staged in shared memory
+// (the prefill output is checked to tolerance, its integer accumulators exactly).
+constexpr int QW = 8;  // tokens (warps) per CTA
+__global__ void __launch_bounds__(QW * 32) prefill_quant_kernel(const float* __restrict__ x, int M, int K,
+                                                               const int8_t* __restrict__ lora_b,
+                                                               const float* __restrict__ lora_b_scale,
+                                                               int rank, int8_t* __restrict__ xq,
+                                                               float* __restrict__ s_out,
+                                                               float* __restrict__ tf_out,
+                                                               int8_t* dbg_xq, float* dbg_s, float* dbg_tf) {
+  extern __shared__ __align__(16) unsigned char sm[];
+  int8_t* wb = reinterpret_cast<int8_t*>(sm);  // [rank][K]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int i = threadIdx.x * 4; i < rank * K; i += blockDim.x * 4)
+    *reinterpret_cast<uint32_t*>(wb + i) = __ldg(reinterpret_cast<const uint32_t*>(lora_b + i));
+  __syncthreads();
+  const int m = blockIdx.x * QW + warp;
+  if (m >= M) return;
+  const float* xr = x + (size_t)m * K;
+  float m_abs = 0.0f;
+  for (int i = lane * 4; i < K; i += 128) {
+    const float4 v = __ldg(reinterpret_cast<const float4*>(xr + i));
+    m_abs = fmaxf(m_abs, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
+  }
+  m_abs = warp_max(m_abs);
+  const float s0 = m_abs == 0.0f ? 0.0f : __fdiv_rn(m_abs, 127.0f);
+  const float inv_s0 = m_abs == 0.0f ? 0.0f : __frcp_rn(s0);
+  float u[DFSSM_MAX_RANK];
+#pragma unroll
+  for (int r = 0; r < DFSSM_MAX_RANK; ++r) u[r] = 0.0f;
+  for (int i = lane * 4; i < K; i += 128) {
+    const float4 v = __ldg(reinterpret_cast<const float4*>(xr + i));
+    const float vv[4] = {v.x, v.y, v.z, v.w};
+    uint32_t packed = 0;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int c = m_abs == 0.0f ? 0 : quant_code_fast(vv[j], s0, inv_s0);
+      packed |= (uint32_t)(uint8_t)(int8_t)c << (8 * j);
+    }
+    *reinterpret_cast<uint32_t*>(xq + (size_t)m * K + i) = packed;
+    if (dbg_xq) *reinterpret_cast<uint32_t*>(dbg_xq + (size_t)m * K + i) = packed;
+#pragma unroll
+    for (int r = 0; r < DFSSM_MAX_RANK; ++r) {
+      if (r < rank) {
+        const uint32_t w4 = *reinterpret_cast<const uint32_t*>(wb + (size_t)r * K + i);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) u[r] = fmaf(int8_to_f32((int)(int8_t)(w4 >> (8 * j))), vv[j], u[r]);
+      }
+    }
+  }
+#pragma unroll
+  for (int r = 0; r < DFSSM_MAX_RANK; ++r) u[r] = warp_sum(u[r]);
+  if (lane < DFSSM_MAX_RANK) {
+    float uv = 0.0f;
+#pragma unroll
+    for (int r = 0; r < DFSSM_MAX_RANK; ++r)
+      if (r == lane) uv = u[r];
+    const float t = lane < rank ? uv * __ldg(lora_b_scale + lane) : 0.0f;
+    tf_out[(size_t)m * DFSSM_MAX_RANK + lane] = t;
+    if (dbg_tf && lane < rank) dbg_tf[(size_t)m * rank + lane] = t;
+  }
+  if (lane == 0) {
+    s_out[m] = s0;
+    if (dbg_s) dbg_s[m] = s0;
+  }
+}
+
+// Persistent tcgen05 GEMM: one CTA per SM walks the output tiles; warp 0 streams A/B stages with TMA,
+// warp 1 issues the MMAs into one of two TMEM accumulators, warps 2..9 drain the other accumulator (two
+// warps per 32-lane TMEM quadrant, each taking half of the 256 columns), so a tile's epilogue overlaps
+// the next tile's main loop.
+constexpr int EPI_WARPS = 8;
+constexpr int PNT = 64 + EPI_WARPS * 32;   // 320 threads
+constexpr int PTMEM_COLS = 2 * BN;         // two 256-column accumulators
+constexpr size_t PSMEM_BYTES = (size_t)STAGES * STAGE_BYTES + 1024 + 512 + 2 * BN * (16 * 4 + 8);
+
+__global__ void __launch_bounds__(PNT, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
                 const EpiArgs ep) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -157,12 +238,18 @@ __global__ void __launch_bounds__(NT, 1)
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
   uint64_t* empty = full + STAGES;
-  uint64_t* tmem_full = empty + STAGES;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(tmem_full + 1);
+  uint64_t* acc_full = empty + STAGES;     // [2] MMA -> epilogue
+  uint64_t* acc_empty = acc_full + 2;      // [2] epilogue -> MMA
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(acc_empty + 2);
+  // per-accumulator column parameters of the tile being drained: W_A rows (as fp32), sW, sA
+  float* col_wa = reinterpret_cast<float*>(smem + STAGES * STAGE_BYTES + 512);      // [2][BN][16]
+  float* col_sw = col_wa + 2 * BN * 16;                                             // [2][BN]
+  float* col_sa = col_sw + 2 * BN;                                                  // [2][BN]
   __shared__ int abort_flag;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n0 = blockIdx.x * BN, m0 = blockIdx.y * BM;
+  const int tiles_n = (ep.N + BN - 1) / BN, tiles_m = (ep.M + BM - 1) / BM;
+  const int tiles = tiles_n * tiles_m;
   const int kblocks = ep.K / BK;
 
   if (threadIdx.x == 0) {
@@ -171,13 +258,16 @@ __global__ void __launch_bounds__(NT, 1)
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    mbar_init(tmem_full, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], EPI_WARPS);
+    }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                      smem_u32(tmem_holder)),
-                 "r"(TMEM_COLS)
+                 "r"(PTMEM_COLS)
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
@@ -187,87 +277,132 @@ __global__ void __launch_bounds__(NT, 1)
   const uint32_t tmem_base = *tmem_holder;
 
   if (warp == 0 && lane == 0) {
-    // ---- TMA producer
-    int issued = 0;
-    for (int kb = 0; kb < kblocks; ++kb) {
-      const int s = kb % STAGES;
-      if (kb >= STAGES && !mbar_wait(&empty[s], ((kb / STAGES) - 1) & 1, &abort_flag)) {
-        abort_flag = 1;
-        break;
-      }
-      unsigned char* a_dst = smem + s * STAGE_BYTES;
-      unsigned char* b_dst = a_dst + A_BYTES;
-      mbar_expect_tx(&full[s], STAGE_BYTES);
-      tma_load_2d(a_dst, &map_a, kb * BK, m0, &full[s]);
-      tma_load_2d(b_dst, &map_b, kb * BK, n0, &full[s]);
-      ++issued;
-    }
-    // copies still in flight complete before this CTA may exit
-    for (int kb = (issued > STAGES ? issued - STAGES : 0); kb < issued; ++kb)
-      mbar_wait(&full[kb % STAGES], (kb / STAGES) & 1, &abort_flag);
-  } else if (warp == 1 && lane == 0) {
-    // ---- MMA issuer: one thread issues every tcgen05.mma of the tile
+    // ---- TMA producer: k-blocks of every tile of this CTA, through the stage ring
+    int it = 0;
     bool ok = true;
-    for (int kb = 0; kb < kblocks && ok; ++kb) {
-      const int s = kb % STAGES;
-      if (!mbar_wait(&full[s], (kb / STAGES) & 1, &abort_flag)) {
+    for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
+      const int n0 = (t % tiles_n) * BN, m0 = (t / tiles_n) * BM;
+      for (int kb = 0; kb < kblocks; ++kb, ++it) {
+        const int s = it % STAGES;
+        if (it >= STAGES && !mbar_wait(&empty[s], ((it / STAGES) - 1) & 1, &abort_flag)) {
+          abort_flag = 1;
+          ok = false;
+          break;
+        }
+        unsigned char* a_dst = smem + s * STAGE_BYTES;
+        mbar_expect_tx(&full[s], STAGE_BYTES);
+        tma_load_2d(a_dst, &map_a, kb * BK, m0, &full[s]);
+        tma_load_2d(a_dst + A_BYTES, &map_b, kb * BK, n0, &full[s]);
+      }
+    }
+    // the last stages' copies land before this CTA may exit
+    for (int j = (it > STAGES ? it - STAGES : 0); j < it; ++j)
+      mbar_wait(&full[j % STAGES], (j / STAGES) & 1, &abort_flag);
+  } else if (warp == 1 && lane == 0) {
+    // ---- MMA issuer
+    int it = 0, local = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x, ++local) {
+      const int buf = local & 1;
+      if (local >= 2 && !mbar_wait(&acc_empty[buf], ((local >> 1) - 1) & 1, &abort_flag)) {
         abort_flag = 1;
-        ok = false;
         break;
       }
       asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-      const uint32_t a_addr = smem_u32(smem + s * STAGE_BYTES);
-      const uint32_t b_addr = a_addr + A_BYTES;
+      const uint32_t d_tmem = tmem_base + (uint32_t)(buf * BN);
+      for (int kb = 0; kb < kblocks; ++kb, ++it) {
+        const int s = it % STAGES;
+        if (!mbar_wait(&full[s], (it / STAGES) & 1, &abort_flag)) {
+          abort_flag = 1;
+          ok = false;
+          break;
+        }
+        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+        const uint32_t a_addr = smem_u32(smem + s * STAGE_BYTES);
+        const uint32_t b_addr = a_addr + A_BYTES;
 #pragma unroll
-      for (int kk = 0; kk < BK / UMMA_K; ++kk)
-        umma_i8(tmem_base, umma_desc_k_sw128(a_addr + kk * UMMA_K), umma_desc_k_sw128(b_addr + kk * UMMA_K),
-                (kb > 0 || kk > 0) ? 1u : 0u);
-      umma_commit(&empty[s]);  // frees the stage once these MMAs have read it
+        for (int kk = 0; kk < BK / UMMA_K; ++kk)
+          umma_i8(d_tmem, umma_desc_k_sw128(a_addr + kk * UMMA_K), umma_desc_k_sw128(b_addr + kk * UMMA_K),
+                  (kb > 0 || kk > 0) ? 1u : 0u);
+        umma_commit(&empty[s]);
+      }
+      umma_commit(&acc_full[buf]);
     }
-    umma_commit(tmem_full);    // accumulator complete (also signals after an abort)
   } else if (warp >= 2) {
-    // ---- epilogue: warp w reads TMEM lanes [32 (w % 4), +32) = tile rows
+    // ---- epilogue: warp e = warp - 2 drains TMEM lanes [32 (warp % 4), +32) and column half e / 4
+    const int e = warp - 2;
     const int q = warp & 3;
-    const int row = q * 32 + lane;
-    const int m = m0 + row;
-    const bool ok = mbar_wait(tmem_full, 0, &abort_flag);
-    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-    if (!ok || abort_flag) {
-      if (lane == 0) atomicExch(ep.err, 1);
-    } else {
+    const int half = e >> 2;
+    const int etid = threadIdx.x - 64;  // 0..255
+    int local = 0;
+    for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++local) {
+      const int buf = local & 1;
+      const int n0 = (t % tiles_n) * BN, m0 = (t / tiles_n) * BM;
+      // column parameters of this tile, staged once per tile by the 256 epilogue threads
+      {
+        const int n = n0 + etid;
+        float* wa_dst = col_wa + (size_t)(buf * BN + etid) * 16;
+        if (n < ep.N && ep.rank == DFSSM_MAX_RANK) {
+          const uint4 w4 = __ldg(reinterpret_cast<const uint4*>(ep.la) + n);
+          const uint32_t wv[4] = {w4.x, w4.y, w4.z, w4.w};
+#pragma unroll
+          for (int r = 0; r < 16; ++r) wa_dst[r] = int8_to_f32((int)(int8_t)(wv[r >> 2] >> (8 * (r & 3))));
+        } else {
+          for (int r = 0; r < 16; ++r)
+            wa_dst[r] = (n < ep.N && r < ep.rank) ? (float)ep.la[(size_t)n * ep.rank + r] : 0.0f;
+        }
+        col_sw[buf * BN + etid] = n < ep.N ? __ldg(ep.w_scale + n) : 0.0f;
+        col_sa[buf * BN + etid] = (n < ep.N && ep.rank > 0) ? __ldg(ep.la_scale + n) : 0.0f;
+      }
+      asm volatile("bar.sync 1, %0;" ::"n"(EPI_WARPS * 32) : "memory");
+      const int row = q * 32 + lane;
+      const int m = m0 + row;
       float sm = 0.f;
       float tfm[DFSSM_MAX_RANK];
 #pragma unroll
       for (int r = 0; r < DFSSM_MAX_RANK; ++r) tfm[r] = 0.f;
       if (m < ep.M) {
-        sm = ep.s[m];
+        sm = __ldg(ep.s + m);
+        const float4* tp = reinterpret_cast<const float4*>(ep.tf + (size_t)m * DFSSM_MAX_RANK);
 #pragma unroll
-        for (int r = 0; r < DFSSM_MAX_RANK; ++r) tfm[r] = ep.tf[(size_t)m * DFSSM_MAX_RANK + r];
+        for (int r4 = 0; r4 < 4; ++r4) {
+          const float4 v = __ldg(tp + r4);
+          tfm[4 * r4] = v.x;
+          tfm[4 * r4 + 1] = v.y;
+          tfm[4 * r4 + 2] = v.z;
+          tfm[4 * r4 + 3] = v.w;
+        }
       }
-      for (int c0 = 0; c0 < BN; c0 += 16) {
+      // every epilogue warp runs every tile iteration (the named barrier above counts on it); after an
+      // abort the accumulator is simply not read
+      const bool ok = !abort_flag && mbar_wait(&acc_full[buf], (local >> 1) & 1, &abort_flag);
+      asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+      if (!ok) {
+        abort_flag = 1;
+        if (lane == 0) atomicExch(ep.err, 1);
+      }
+      for (int cc = 0; ok && cc < BN / 2; cc += 16) {
+        const int c0 = half * (BN / 2) + cc;
         uint32_t v[16];
-        tmem_ld16(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)c0, v);
+        tmem_ld16(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * BN + c0), v);
         if (m >= ep.M) continue;
         float out[16];
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
-          const int n = n0 + c0 + j;
-          float yv = 0.f;
-          if (n < ep.N) {
-            const int acc = (int)v[j];
-            float lora = 0.f;
-            if (ep.rank == DFSSM_MAX_RANK) {
-              const uint4 wa4 = __ldg(reinterpret_cast<const uint4*>(ep.la) + n);
-              const int8_t* wa = reinterpret_cast<const int8_t*>(&wa4);
+          const int cidx = buf * BN + c0 + j;
+          const float4* wa4 = reinterpret_cast<const float4*>(col_wa + (size_t)cidx * 16);
+          float lora = 0.f;
 #pragma unroll
-              for (int r = 0; r < DFSSM_MAX_RANK; ++r) lora = fmaf((float)wa[r], tfm[r], lora);
-            } else {
-              for (int r = 0; r < ep.rank; ++r) lora = fmaf((float)ep.la[(size_t)n * ep.rank + r], tfm[r], lora);
-            }
-            yv = fmaf((float)acc, sm * __ldg(ep.w_scale + n), ep.rank > 0 ? __ldg(ep.la_scale + n) * lora : 0.f);
-            if (ep.acc) ep.acc[(size_t)m * ep.N + n] = acc;
+          for (int r4 = 0; r4 < 4; ++r4) {
+            const float4 w = wa4[r4];
+            lora = fmaf(w.x, tfm[4 * r4], lora);
+            lora = fmaf(w.y, tfm[4 * r4 + 1], lora);
+            lora = fmaf(w.z, tfm[4 * r4 + 2], lora);
+            lora = fmaf(w.w, tfm[4 * r4 + 3], lora);
           }
-          out[j] = yv;
+          const int acc = (int)v[j];
+          out[j] = fmaf((float)acc, sm * col_sw[cidx], col_sa[cidx] * lora);
+          if (ep.acc && n0 + c0 + j < ep.N) ep.acc[(size_t)m * ep.N + n0 + c0 + j] = acc;
         }
         float* yrow = ep.y + (size_t)m * ep.N + n0 + c0;
         if (n0 + c0 + 16 <= ep.N && (ep.N % 4) == 0) {
@@ -278,6 +413,12 @@ __global__ void __launch_bounds__(NT, 1)
           for (int j = 0; j < 16 && n0 + c0 + j < ep.N; ++j) yrow[j] = out[j];
         }
       }
+      // this warp's reads of the accumulator are complete: release it to the MMA warp
+      asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+      __syncwarp();
+      if (lane == 0)
+        asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&acc_empty[buf]))
+                     : "memory");
     }
   }
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
@@ -285,7 +426,7 @@ __global__ void __launch_bounds__(NT, 1)
   if (abort_flag && threadIdx.x == 0) atomicExch(ep.err, 1);
   if (warp == 1) {
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(TMEM_COLS)
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(PTMEM_COLS)
                  : "memory");
   }
 }
@@ -384,27 +525,19 @@ extern "C" int dfssm_linear_prefill(const dfssm_linear_t* lin, const float* x, i
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   prefill::Ws w = prefill::carve(workspace, M, K, N);
 
-  // 1. per-token quantization and LoRA down-projection
-  QuantArgs qa{};
-  qa.x = x;
-  qa.ldx = K;
-  qa.norm_w = nullptr;
-  qa.n = K;
-  qa.B = M;
-  qa.lora_b = lin->lora_b;
-  qa.lora_b_scale = lin->lora_b_scale;
-  qa.rank = lin->rank;
-  qa.permute = false;
-  qa.out.q = w.xq;
-  qa.out.s = w.s;
-  qa.out.sumq = w.sumq;
-  qa.out.tf = w.tf;
-  if (dbg) {
-    qa.dbg_xq = dbg->xq;
-    qa.dbg_s = dbg->xscale;
-    qa.dbg_tf = dbg->lora_tf;
+  // 1. per-token quantization and LoRA down-projection (one warp per token)
+  const size_t qsmem = (size_t)lin->rank * K;
+  static bool qattr = false;
+  if (!qattr) {
+    const cudaError_t ea = cudaFuncSetAttribute(prefill::prefill_quant_kernel,
+                                                cudaFuncAttributeMaxDynamicSharedMemorySize, 16 * 8192);
+    if (ea != cudaSuccess) return record_cuda_failure(ea);
+    qattr = true;
   }
-  cudaError_t e = launch_quant(qa, st);
+  prefill::prefill_quant_kernel<<<(M + prefill::QW - 1) / prefill::QW, prefill::QW * 32, qsmem, st>>>(
+      x, M, K, lin->lora_b, lin->lora_b_scale, lin->rank, w.xq, w.s, w.tf, dbg ? dbg->xq : nullptr,
+      dbg ? dbg->xscale : nullptr, dbg ? dbg->lora_tf : nullptr);
+  cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return record_cuda_failure(e);
   // 2. +-1 int8 weights
   const long long words = (long long)N * (K / 32);
@@ -433,12 +566,13 @@ extern "C" int dfssm_linear_prefill(const dfssm_linear_t* lin, const float* x, i
   static bool attr_done = false;
   if (!attr_done) {
     e = cudaFuncSetAttribute(prefill::gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)prefill::SMEM_BYTES);
+                             (int)prefill::PSMEM_BYTES);
     if (e != cudaSuccess) return record_cuda_failure(e);
     attr_done = true;
   }
-  dim3 grid((N + prefill::BN - 1) / prefill::BN, (M + prefill::BM - 1) / prefill::BM);
-  prefill::gemm_kernel<<<grid, prefill::NT, prefill::SMEM_BYTES, st>>>(map_a, map_b, ep);
+  const int tiles = ((N + prefill::BN - 1) / prefill::BN) * ((M + prefill::BM - 1) / prefill::BM);
+  const int grid = tiles < num_sms() ? tiles : num_sms();
+  prefill::gemm_kernel<<<grid, prefill::PNT, prefill::PSMEM_BYTES, st>>>(map_a, map_b, ep);
   e = cudaGetLastError();
   if (e != cudaSuccess) return record_cuda_failure(e);
   return DFSSM_OK;
