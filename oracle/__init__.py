@@ -35,7 +35,7 @@ def _declare(L):
     L.oracle_sign.restype = _I
     L.oracle_quantize.argtypes = [_P, _I, _I, _P, _P]
     L.oracle_linear_decode.argtypes = [_I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _I, _P, _P, _P, _P, _P]
-    L.oracle_lora_down.argtypes = [_I, _I, _P, _P, _P, C.c_double, _P]
+    L.oracle_lora_down.argtypes = [_I, _I, _P, _P, _P, C.c_float, _P, _P]
     L.oracle_linear_core.argtypes = [_I, _I, _I, _P, _P, _P, _P, _P, C.c_float, _P, _P, _P]
     L.oracle_linear_rows.argtypes = [_I, _I, _I, _P, _P, _P, _P, _P, C.c_float, _P, _P, _I, _P, _P]
     L.oracle_conv_step.argtypes = [_P, _P, _P, _P, _P, _I, _I]
@@ -102,26 +102,28 @@ class Linear:
 
 
 def linear_decode(L: Linear, x: np.ndarray):
-    """Quantize each row of x and apply the linear. Returns dict(y, acc, tf, xq, xscale)."""
+    """Quantize each row of x and apply the linear. Returns dict(y, acc, t, xq, xscale)."""
     x = _c(np.atleast_2d(x), np.float32)
     B = x.shape[0]
     assert x.shape[1] == L.d_in
     y = np.zeros((B, L.d_out), np.float32)
     acc = np.zeros((B, L.d_out), np.int32)
-    tf = np.zeros((B, max(L.rank, 1)), np.float32)
+    t = np.zeros((B, max(L.rank, 1)), np.int32)
     xq = np.zeros((B, L.d_in), np.int8)
     xs = np.zeros(B, np.float32)
-    lib().oracle_linear_decode(*L._args(), _p(x), B, _p(y), _p(acc), _p(tf), _p(xq), _p(xs))
-    return dict(y=y, acc=acc, tf=tf[:, :L.rank], xq=xq, xscale=xs)
+    lib().oracle_linear_decode(*L._args(), _p(x), B, _p(y), _p(acc), _p(t), _p(xq), _p(xs))
+    return dict(y=y, acc=acc, t=t.reshape(-1)[:B * L.rank].reshape(B, L.rank), xq=xq, xscale=xs)
 
 
-def lora_down(L: Linear, v: np.ndarray, rms: float = 1.0) -> np.ndarray:
-    """LoRA intermediate tf[r] = fl32((sum_i W_B[r,i] v_i) * sB[r] / rms) of one input row v."""
-    v = _c(v, np.float32).reshape(L.d_in)
+def lora_down(L: Linear, q: np.ndarray, s: float):
+    """LoRA down-projection of one row of codes q (int8) with scale s:
+    t[r] = sum_i W_B[r,i] q_i (int32) and tf[r] = fl32(t[r] * sB[r] * s). Returns (t, tf)."""
+    q = _c(q, np.int8).reshape(L.d_in)
+    t = np.zeros(max(L.rank, 1), np.int32)
     tf = np.zeros(max(L.rank, 1), np.float32)
     a = L._args()
-    lib().oracle_lora_down(L.d_in, L.rank, a[5], a[6], _p(v), float(rms), _p(tf))
-    return tf[:L.rank]
+    lib().oracle_lora_down(L.d_in, L.rank, a[5], a[6], _p(q), C.c_float(float(s)), _p(t), _p(tf))
+    return t[:L.rank], tf[:L.rank]
 
 
 def linear_core(L: Linear, q: np.ndarray, s: float, tf: np.ndarray):

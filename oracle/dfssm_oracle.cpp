@@ -70,18 +70,19 @@ void quantize_row(const float* v, int n, int8_t* q, float* s_out) {
   *s_out = s;
 }
 
-// LoRA down-projection of the linear's fp32 input ([TS-2B]: the LoRA matrices W_A, W_B are int8 with
-// per-row scales; a LoRA module applies W_A (W_B x) to the layer input x).  Reading (iii): the LoRA sees
-// the same input as the layer, not its int8 codes, and its intermediate stays fp32:
-//   u[r]  = sum_i W_B[r,i] * v[i]             (fp64; every product int8 x fp32 is exact)
-//   tf[r] = fl32(u[r] * sB[r] / rms)          (rms = 1 for a plain linear; the RMS of the norm when the
-//                                              layer input is RMSNorm(h) and v = fl32(h*w))
-void lora_down(int d_in, int rank, const int8_t* lora_b, const float* lora_b_scale, const float* v,
-               double rms, float* tf) {
+// LoRA down-projection ([TS-2B]: a rank-16 LoRA module W_A (W_B x) with int8 matrices and per-row
+// scales, applied to the layer input; [TS-2C]: the linear's input is the per-token int8 activation of the
+// INT8 scaffold matmul).  Reading (iii): W_B multiplies the same int8 codes q as the scaffold, with int32
+// accumulation, and the intermediate stays fp32 (it is not requantized):
+//   t[r]  = sum_i W_B[r,i] * q[i]              (exact integer; |t| <= 127*127*d_in fits int32)
+//   tf[r] = fl32(t[r] * sB[r] * s)             (fp64, this order; s the input's quantizer scale)
+void lora_down(int d_in, int rank, const int8_t* lora_b, const float* lora_b_scale, const int8_t* q,
+               float s, int32_t* t_out, float* tf) {
   for (int r = 0; r < rank; ++r) {
-    double u = 0.0;
-    for (int i = 0; i < d_in; ++i) u += (double)lora_b[(size_t)r * d_in + i] * (double)v[i];
-    tf[r] = r32(u * (double)lora_b_scale[r] / rms);
+    int64_t t = 0;
+    for (int i = 0; i < d_in; ++i) t += (int64_t)lora_b[(size_t)r * d_in + i] * (int64_t)q[i];
+    if (t_out) t_out[r] = (int32_t)t;
+    tf[r] = r32((double)t * (double)lora_b_scale[r] * (double)s);
   }
 }
 
@@ -109,7 +110,7 @@ void linear_core(int d_out, int d_in, int rank, const uint32_t* bits, const floa
 // channel).  The quantizer is invariant to a positive scalar factor of its input — q(c*v) = q(v) and
 // s(c*v) = c*s(v) in exact arithmetic — so the RMS factor is folded into the scale:
 //   v_i = fl32(h_i * w_i);  (q, s0) = quantize(v);  rms = sqrt(sum_i h_i^2 / n + eps);  s = fl32(s0 / rms).
-// Returns rms (fp64) and leaves v in v_out for the LoRA down-projection.
+// Returns rms (fp64) and leaves v = fl32(h*w) in v_out.
 double rmsnorm_quantize(const float* h, const float* w, int n, double eps, int8_t* q, float* s_out,
                         float* v_out) {
   double ss = 0.0;
@@ -128,7 +129,7 @@ inline double silu64(double v) { return v / (1.0 + std::exp(-v)); }
 
 extern "C" {
 
-int oracle_abi_version(void) { return 2; }
+int oracle_abi_version(void) { return 3; }
 
 // Pinned by: exhaustive byte-pattern round trip against an independent packer, brute force.
 int oracle_sign(const uint32_t* bits, int d_in, int o, int i) { return unpack_sign(bits, d_in, o, i); }
@@ -141,32 +142,30 @@ void oracle_quantize(const float* x, int B, int n, int8_t* q, float* s) {
 
 // dfssm linear decode: quantize each of the B rows of x, then the scaffold + LoRA linear.
 // Pinned by: brute-force +-1 integer matmul, 2*sum_{bit=1} q - sum q identity, bit-flip negation,
-// one-hot inputs, rank-0 == scaffold alone, W_A == 0 == scaffold alone, one-hot W_B rows, the real-number
-// epilogue formula.
+// one-hot inputs, rank-0 == scaffold alone, W_A == 0 == scaffold alone, one-hot W_B rows, brute-force
+// integer LoRA-down, the real-number epilogue formula.
 void oracle_linear_decode(int d_out, int d_in, int rank, const uint32_t* bits, const float* w_scale,
                           const int8_t* lora_b, const float* lora_b_scale, const int8_t* lora_a,
                           const float* lora_a_scale, const float* x, int B, float* y,
-                          int32_t* acc, float* tf_out, int8_t* xq, float* xscale) {
+                          int32_t* acc, int32_t* t_out, int8_t* xq, float* xscale) {
   std::vector<int8_t> q((size_t)d_in);
   std::vector<float> tf((size_t)(rank > 0 ? rank : 1));
   for (int b = 0; b < B; ++b) {
     float s = 0.0f;
-    const float* xb = x + (size_t)b * d_in;
-    quantize_row(xb, d_in, q.data(), &s);
+    quantize_row(x + (size_t)b * d_in, d_in, q.data(), &s);
     if (xq) std::memcpy(xq + (size_t)b * d_in, q.data(), (size_t)d_in);
     if (xscale) xscale[b] = s;
-    lora_down(d_in, rank, lora_b, lora_b_scale, xb, 1.0, tf.data());
-    if (tf_out)
-      for (int r = 0; r < rank; ++r) tf_out[(size_t)b * rank + r] = tf[r];
+    lora_down(d_in, rank, lora_b, lora_b_scale, q.data(), s, t_out ? t_out + (size_t)b * rank : nullptr,
+              tf.data());
     linear_core(d_out, d_in, rank, bits, w_scale, lora_a, lora_a_scale, q.data(), s, tf.data(),
                 acc ? acc + (size_t)b * d_out : nullptr, y + (size_t)b * d_out);
   }
 }
 
-// LoRA down-projection alone (see lora_down): tf[r] for input v and divisor rms.
+// LoRA down-projection alone (see lora_down): t[r] and tf[r] for codes q with scale s.
 void oracle_lora_down(int d_in, int rank, const int8_t* lora_b, const float* lora_b_scale,
-                      const float* v, double rms, float* tf) {
-  lora_down(d_in, rank, lora_b, lora_b_scale, v, rms, tf);
+                      const int8_t* q, float s, int32_t* t, float* tf) {
+  lora_down(d_in, rank, lora_b, lora_b_scale, q, s, t, tf);
 }
 
 // Scaffold + LoRA-up on pre-quantized codes q with scale s and LoRA intermediate tf (teacher-forced and
@@ -269,7 +268,7 @@ void oracle_ssm_step(float* ssm_state, const float* x, const float* dt_raw, cons
 }
 
 // Pre-mixer RMSNorm + per-token quantization of B rows (the RMS factor folded into the scale); also
-// returns v = fl32(h*w) [B][n] and rms [B] for the LoRA down-projection.
+// returns v = fl32(h*w) [B][n] and rms [B].
 // Pinned by: a constant row reconstructs w*sign(c); codes agree with quantizing the explicitly
 // normalized row away from rounding ties; scale relation.
 void oracle_rmsnorm_quantize(const float* h, const float* w, int B, int n, int8_t* q, float* s,
@@ -292,11 +291,11 @@ void oracle_gate(const float* y, const float* z, float* g, int n) {
 
 // One Mamba-2 layer decode step with the DF-SSM linears, B rows, the layer's residual stream h
 // updated in place.  Wiring (reading; the Mamba-2 block [MAP] with the DF-SSM linears [TS-2B]):
-//   (q, s)  = rmsnorm_quantize(h, norm_w);  tf = lora_down(fl32(h*norm_w)) / rms
+//   (q, s)  = rmsnorm_quantize(h, norm_w);  tf = lora_down(q, s)
 //   zxbcdt  = in_proj(q, s, tf)                  (reading (v): order z | x | B | C | dt)
 //   xc      = conv_step(xBC)                     (SiLU applied to x, B and C channels)
 //   y       = ssm_step(xc.x, dt, xc.B, xc.C)
-//   g       = gate(y, z);  (q', s') = rmsnorm_quantize(g, gnorm_w);  tf' = lora_down(...) / rms'
+//   g       = gate(y, z);  (q', s') = rmsnorm_quantize(g, gnorm_w);  tf' = lora_down(q', s')
 //   h       = fl32(h + out_proj(q', s', tf'))
 // Shapes: D = d_model, E = d_inner = H*P, C = E + 2*G*N conv channels, in_proj rows 2E + 2GN + H.
 // Pinned by: composition of the separately pinned steps in this order; a zero out_proj scale leaves
@@ -323,8 +322,8 @@ void oracle_layer_decode(int B, int Dm, int H, int P, int N, int G, int rank,
   for (int b = 0; b < B; ++b) {
     float* hb = h + (size_t)b * Dm;
     float s = 0.0f;
-    double rms = rmsnorm_quantize(hb, norm_w, Dm, 1e-5, q.data(), &s, v.data());
-    lora_down(Dm, rank, in_lb, in_lbs, v.data(), rms, tf.data());
+    rmsnorm_quantize(hb, norm_w, Dm, 1e-5, q.data(), &s, v.data());
+    lora_down(Dm, rank, in_lb, in_lbs, q.data(), s, nullptr, tf.data());
     linear_core(d_ip, Dm, rank, in_bits, in_ws, in_la, in_las, q.data(), s, tf.data(), nullptr,
                 zx.data());
     if (tap_zxbcdt) std::memcpy(tap_zxbcdt + (size_t)b * d_ip, zx.data(), sizeof(float) * d_ip);
@@ -335,8 +334,8 @@ void oracle_layer_decode(int B, int Dm, int H, int P, int N, int G, int rank,
                     xc.data() + E, xc.data() + E + G * N, y.data(), 1, H, P, N, G);
     if (tap_y) std::memcpy(tap_y + (size_t)b * E, y.data(), sizeof(float) * E);
     oracle_gate(y.data(), zx.data(), g.data(), E);
-    rms = rmsnorm_quantize(g.data(), gnorm_w, E, 1e-5, q.data(), &s, v.data());
-    lora_down(E, rank, out_lb, out_lbs, v.data(), rms, tf.data());
+    rmsnorm_quantize(g.data(), gnorm_w, E, 1e-5, q.data(), &s, v.data());
+    lora_down(E, rank, out_lb, out_lbs, q.data(), s, nullptr, tf.data());
     linear_core(Dm, E, rank, out_bits, out_ws, out_la, out_las, q.data(), s, tf.data(), nullptr,
                 out.data());
     for (int i = 0; i < Dm; ++i) hb[i] = r32((double)hb[i] + (double)out[i]);

@@ -166,40 +166,66 @@ def test_lora_rank0_equals_scaffold_alone(tiny):
 
 
 def test_lora_one_hot_down_rows(tiny):
-    """A one-hot W_B row picks one input: tf[r] = fl32(x_j * sB[r]) (the LoRA sees the fp32 input)."""
+    """A one-hot W_B row picks one activation code: t[r] = q_j exactly, tf[r] = fl32(q_j * sB[r] * s)."""
     d = dict(tiny["linear"])
     cols = [3, 17, 100, 255, 0, 64, 128, 129, 5, 6, 7, 8, 9, 10, 11, 12]
     lb = np.zeros((16, 256), np.int8)
     for r, c in enumerate(cols):
         lb[r, c] = 1
     out = oracle.linear_decode(oracle.Linear.from_dict(dict(d, lora_b=lb)), tiny["x"])
-    expect = (tiny["x"][0, cols].astype(np.float64) * d["lora_b_scale"].astype(np.float64))
-    assert np.array_equal(out["tf"][0], expect.astype(np.float32))
+    q = out["xq"][0]
+    assert np.array_equal(out["t"][0], q[cols].astype(np.int32))
+    s = float(out["xscale"][0])
+    t, tf = oracle.lora_down(oracle.Linear.from_dict(dict(d, lora_b=lb)), q, s)
+    expect = q[cols].astype(np.float64) * d["lora_b_scale"].astype(np.float64) * s
+    assert np.allclose(tf, expect, rtol=2 ** -24, atol=0)
+
+
+def test_lora_down_brute_force_integer():
+    """t = W_B q is the exact integer product (numpy int64 matmul) for random and extreme codes, and
+    negating q negates t."""
+    g = np.random.default_rng(12)
+    for d_in in (32, 256, 4096):
+        lb = g.integers(-127, 128, (16, d_in), dtype=np.int8)
+        L = oracle.Linear(np.zeros((4, d_in // 32), np.uint32), np.ones(4, np.float32), lb,
+                          np.ones(16, np.float32), np.zeros((4, 16), np.int8), np.ones(4, np.float32))
+        for q in (g.integers(-127, 128, d_in, dtype=np.int8), np.full(d_in, 127, np.int8),
+                  np.full(d_in, -127, np.int8)):
+            t, _ = oracle.lora_down(L, q, 1.0)
+            expect = lb.astype(np.int64) @ q.astype(np.int64)
+            assert np.array_equal(t.astype(np.int64), expect)
+            tn, _ = oracle.lora_down(L, (-q.astype(np.int16)).astype(np.int8), 1.0)
+            assert np.array_equal(tn, -t)
 
 
 def test_lora_epilogue_real_number_formula(tiny):
-    """y = acc*s*sW + sA * W_A @ ((W_B @ x) * sB) to fp32 accuracy: catches a transposed W_A or W_B, a
-    missing scale or a wrong-sign term."""
+    """y = acc*s*sW + sA * W_A @ ((W_B @ q) * sB * s) to fp32 accuracy: catches a transposed W_A or W_B,
+    a missing scale or a wrong-sign term."""
     d = tiny["linear"]
     L = oracle.Linear.from_dict(d)
     out = oracle.linear_decode(L, tiny["x"])
     s = float(out["xscale"][0])
-    u = d["lora_b"].astype(np.float64) @ tiny["x"][0].astype(np.float64)
-    tf = u * d["lora_b_scale"].astype(np.float64)
-    assert np.allclose(out["tf"][0], tf, rtol=1e-6, atol=0)
+    t = d["lora_b"].astype(np.int64) @ out["xq"][0].astype(np.int64)
+    assert np.array_equal(out["t"][0].astype(np.int64), t)
+    tf = t * d["lora_b_scale"].astype(np.float64) * s
     y = (out["acc"][0] * s * d["w_scale"].astype(np.float64)
          + d["lora_a_scale"].astype(np.float64) * (d["lora_a"].astype(np.float64) @ tf))
     assert np.allclose(out["y"][0], y, rtol=1e-6, atol=1e-7)
 
 
-def test_lora_down_rms_divisor_and_linearity(tiny):
-    """tf(v, rms) = tf(v) / rms to fp32 accuracy, and tf is linear in v (doubling v doubles tf exactly)."""
+def test_lora_power_of_two_input_scaling(tiny):
+    """Scaling x by 2^k leaves the codes and t unchanged and scales tf and y by exactly 2^k (the LoRA
+    intermediate carries the input's quantizer scale s)."""
     L = oracle.Linear.from_dict(tiny["linear"])
-    v = tiny["x"][0]
-    t1 = oracle.lora_down(L, v).astype(np.float64)
-    t3 = oracle.lora_down(L, v, rms=3.0).astype(np.float64)
-    assert np.allclose(t3, t1 / 3.0, rtol=2e-7)
-    assert np.array_equal(oracle.lora_down(L, v * np.float32(2)), (t1 * 2).astype(np.float32))
+    a = oracle.linear_decode(L, tiny["x"])
+    for k in (-3, 5):
+        b = oracle.linear_decode(L, tiny["x"] * np.float32(2.0 ** k))
+        assert np.array_equal(a["xq"], b["xq"]) and np.array_equal(a["t"], b["t"])
+        assert np.array_equal(b["xscale"], (a["xscale"] * np.float32(2.0 ** k)).astype(np.float32))
+        _, tfa = oracle.lora_down(L, a["xq"][0], float(a["xscale"][0]))
+        _, tfb = oracle.lora_down(L, b["xq"][0], float(b["xscale"][0]))
+        assert np.array_equal(tfb, (tfa * np.float32(2.0 ** k)).astype(np.float32))
+        assert np.array_equal(b["y"], (a["y"] * np.float32(2.0 ** k)).astype(np.float32))
 
 
 # ------------------------------------------------------------------------------------------- conv
@@ -396,7 +422,7 @@ def test_layer_zero_out_proj_keeps_residual():
 
 
 def test_layer_composition_of_pinned_steps():
-    """The layer equals the pinned steps wired as: norm+quant (+ LoRA down on the normalized input) ->
+    """The layer equals the pinned steps wired as: norm+quant (+ LoRA down on the codes) ->
     in_proj -> split z|x|B|C|dt -> conv -> SSM -> gate -> norm+quant -> out_proj -> residual."""
     m = inputs.decode_model(seed=41, n_layers=1, n_tokens=3, **SMALL)
     lay = _oracle_layer(m["layers"][0])
@@ -408,7 +434,7 @@ def test_layer_composition_of_pinned_steps():
         oracle.layer_decode(lay, h_a, conv_a[0], ssm_a[0])
         h_b = m["emb"][t].copy()
         q, s, v, rms = oracle.rmsnorm_quantize(h_b, lay["norm_w"])
-        tf = oracle.lora_down(lay["in_proj"], v[0], rms[0])
+        _, tf = oracle.lora_down(lay["in_proj"], q[0], s[0])
         zx, _ = oracle.linear_core(lay["in_proj"], q[0], s[0], tf)
         z, xbc, dt = zx[:E], zx[E:E + E + 2 * N], zx[E + E + 2 * N:]
         xc = oracle.conv_step(conv_b[0], lay["conv_w"], lay["conv_b"], xbc[None])[0]
@@ -416,7 +442,7 @@ def test_layer_composition_of_pinned_steps():
                             xc[None, E:E + N], xc[None, E + N:])[0]
         gg = oracle.gate(y, z)
         q2, s2, v2, rms2 = oracle.rmsnorm_quantize(gg[None], lay["gnorm_w"])
-        tf2 = oracle.lora_down(lay["out_proj"], v2[0], rms2[0])
+        _, tf2 = oracle.lora_down(lay["out_proj"], q2[0], s2[0])
         out, _ = oracle.linear_core(lay["out_proj"], q2[0], s2[0], tf2)
         h_b = (h_b[0] + out).astype(np.float32)
         assert np.array_equal(h_a[0], h_b)
