@@ -189,7 +189,7 @@ int dfssm_linear_decode(const dfssm_linear_t* lin, const float* x, int B, float*
   if (dbg) {
     qa.dbg_xq = dbg->xq;
     qa.dbg_s = dbg->xscale;
-    qa.dbg_tf = dbg->lora_tf;
+    qa.dbg_t = dbg->lora_t;
   }
   cudaError_t e = dfssm::launch_quant(qa, s);
   if (e != cudaSuccess) return cuda_fail(e);

@@ -130,9 +130,10 @@ __device__ __forceinline__ double int_to_f64(int w) {
   return __hiloint2double(0x43300000, w ^ (int)0x80000000) - 4503601774854144.0;
 }
 
-// LoRA intermediate tf = fl32(u * sB / rms) (fp64), u = sum_i W_B[r,i] v_i; rms = 1 for a plain linear.
-__device__ __forceinline__ float lora_tf(double u, float sB, double rms) {
-  return __double2float_rn(__ddiv_rn(dmul(u, (double)sB), rms));
+// LoRA intermediate tf = fl32(t * sB * s) (fp64, this order): t = sum_i W_B[r,i] q_i is the exact int32
+// LoRA-down of the int8 codes q, s the codes' quantizer scale.
+__device__ __forceinline__ float lora_tf(int t, float sB, float s) {
+  return __double2float_rn(dmul(dmul(int_to_f64(t), (double)sB), (double)s));
 }
 
 // RMS of a row with sum of squares ss: sqrt(ss/n + 1e-5) (fp64); the quantizer scale of the normalized

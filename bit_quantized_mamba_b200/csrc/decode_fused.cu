@@ -13,9 +13,10 @@
 // the layer (and prefetched into L2 one layer ahead), before the CTA waits on anything, so the HBM stream
 // overlaps the dependency chain.  Cross-CTA hand-offs go through global memory with monotonically
 // increasing counters (arrive = CTA barrier + release add; wait = bounded relaxed spin + acquire fence),
-// three per layer.  The LoRA down-projection is linear in its fp32 input, so each CTA publishes its
-// partial sums over the rows it owns next to those rows, and no separate hand-off is needed for it.  A wait
-// that runs past its clock budget records DFSSM_ETIMEOUT in the workspace status word and the CTA returns.
+// three per layer.  Every CTA quantizes the whole h (and g) itself, so it also computes the LoRA
+// down-projection t = W_B q of the codes itself (exact int32 dp4a against W_B staged in shared memory)
+// and no hand-off is needed for it.  A wait that runs past its clock budget records DFSSM_ETIMEOUT in the
+// workspace status word and the CTA returns.
 //
 // All arithmetic goes through the functions in common.cuh, so the results are those of the per-op path.
 
@@ -72,13 +73,11 @@ struct Params {
   int* status;
   int* sacc;
   float* gbuf;
-  double* upin;   // [NC][R] LoRA-down partial sums of the next in_proj (one row per CTA)
-  double* upout;  // [NC][R] LoRA-down partial sums of out_proj
   long long spin_limit;
 };
 
 // ------------------------------------------------------------------------------ workspace layout
-// [counters N_CTR x 128 B][abort word 128 B][status word 128 B][sacc 320][gbuf 4096][upin][upout]
+// [counters N_CTR x 128 B][abort word 128 B][status word 128 B][sacc 320][gbuf 4096]
 // The counters and the abort word are cleared before every launch; the status word is sticky: a timed
 // out wait stores kTimeoutMagic there, and only dfssm_device_status clears it.
 constexpr size_t OFF_CTR = 0;
@@ -87,9 +86,9 @@ constexpr size_t OFF_STATUS = OFF_ERR + 128;
 constexpr size_t CLEAR_BYTES = OFF_STATUS;  // counters + abort word
 constexpr size_t OFF_SACC = OFF_STATUS + 128;
 constexpr size_t OFF_GBUF = OFF_SACC + ((NSH * 4 + 255) / 256) * 256;
-constexpr size_t OFF_UIN = OFF_GBUF + E * 4;
-constexpr size_t OFF_UOUT = OFF_UIN + MAX_CTAS * R * 8;
-constexpr size_t WS_BYTES = OFF_UOUT + MAX_CTAS * R * 8;
+constexpr size_t WS_BYTES = OFF_GBUF + E * 4;
+// dynamic shared memory: W_B of in_proj [R][DM] and of out_proj [R][E]
+constexpr int WB_BYTES = R * (DM + E);
 
 // ------------------------------------------------------------------------------ synchronisation
 
@@ -200,35 +199,22 @@ __device__ __forceinline__ int bits_dot(uint4 w, const uint4* qp4) {
   return S;
 }
 
-// Sum of one LoRA row's partial sums: thread t adds the partials of row t % R from every CTA
-// (t + NT k); a warp then holds row r in lanes r and r + 16.
-__device__ __forceinline__ double gather_partials(const double* part, int NC) {
-  constexpr int K = MAX_CTAS * R / NT;  // all loads in flight at once
-  double pv[K];
+// LoRA down-projection row r = warp: t[r] = sum_i W_B[r,i] q_i over NCH 16-byte chunks, lane taking
+// chunks lane, lane + 32, ... of the natural-order codes and of W_B row r (conflict-free in shared memory).
+template <int NCH>
+__device__ __forceinline__ int lora_row(const int8_t* wb_row, const int8_t* qn, int lane) {
+  const uint4* w4 = reinterpret_cast<const uint4*>(wb_row);
+  const uint4* q4 = reinterpret_cast<const uint4*>(qn);
+  int t = 0;
 #pragma unroll
-  for (int k = 0; k < K; ++k) {
-    const int j = threadIdx.x + k * NT;
-    pv[k] = j < NC * R ? __ldcg(part + j) : 0.0;
+  for (int k = 0; k < NCH / 32; ++k) {
+    const uint4 w = w4[lane + 32 * k], q = q4[lane + 32 * k];
+    t = dp4a_ss(w.x, q.x, t);
+    t = dp4a_ss(w.y, q.y, t);
+    t = dp4a_ss(w.z, q.z, t);
+    t = dp4a_ss(w.w, q.w, t);
   }
-  double u = 0.0;
-#pragma unroll
-  for (int k = 0; k < K; ++k) u += pv[k];
-  return u + __shfl_xor_sync(0xffffffffu, u, 16);
-}
-
-// The fp64 scale chain of one RMSNorm+quantize: thread k < R computes the LoRA intermediate of row k
-// from the per-warp partial sums, thread R the quantizer scale.
-__device__ __forceinline__ void scale_chain(int k, double ss, float s0, int n, float lbs,
-                                            const double (*red_u)[R], float* tf, float* s_scale) {
-  const double rms = rms_of(ss, n);
-  if (k < R) {
-    double ut = 0.0;
-#pragma unroll
-    for (int w = 0; w < NW; ++w) ut += red_u[w][k];
-    tf[k] = lora_tf(ut, lbs, rms);
-  } else {
-    *s_scale = rms_scale(s0, rms);
-  }
+  return __reduce_add_sync(0xffffffffu, t);
 }
 
 // ------------------------------------------------------------------------------ the kernel
@@ -239,15 +225,19 @@ __device__ __forceinline__ void scale_chain(int k, double ss, float s0, int n, f
 //   B  wait B/C  -> epilogues (B/C conv, dt, own z gate, own x conv), SSM of the owned rows, g of the
 //                   owned rows and their LoRA-down partial sums published (arrive g)
 //   C  wait g    -> gated RMSNorm+quantize, out_proj GEMV of the owned rows, residual; the next layer's
-//                   in_proj LoRA-down partial sums over the owned rows published (arrive h)
-// A prologue publishes the first layer's in_proj partial sums from the input hidden state.
+//                   (arrive h)
+// The first layer reads the input hidden state directly (it is complete before the launch).
 
 __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ Params p) {
+  extern __shared__ __align__(16) int8_t wb_sm[];  // W_B of in_proj [R][DM], then of out_proj [R][E]
+  int8_t* const wb_in = wb_sm;
+  int8_t* const wb_out = wb_sm + R * DM;
   __shared__ __align__(16) int8_t q_perm[E];
+  __shared__ __align__(16) int8_t q_nat[E];
   __shared__ double red_d[NW];
   __shared__ float red_f[NW];
   __shared__ int red_i[NW];
-  __shared__ double red_u[NW][R];
+  __shared__ int t_sm[R];
   __shared__ int sflag;
   __shared__ float tf[R];
   __shared__ float s_scale;
@@ -265,11 +255,11 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ P
   __shared__ __align__(16) float Bsm[N];
   __shared__ __align__(16) double Cd[N];
   // SSM rows
-  __shared__ float zsm[MAX_SSM], xsm[MAX_SSM], gsm[MAX_SSM];
+  __shared__ float zsm[MAX_SSM], xsm[MAX_SSM];
   __shared__ float dtv[2], dAv[2], Dv[2];
   // out_proj rows
   __shared__ int acc_out[MAX_OUT];
-  __shared__ float o_sw[MAX_OUT], o_sa[MAX_OUT], h_old[MAX_OUT], h_new[MAX_OUT];
+  __shared__ float o_sw[MAX_OUT], o_sa[MAX_OUT], h_old[MAX_OUT];
   __shared__ __align__(16) int8_t o_wa[MAX_OUT][R];
 
   const int c = blockIdx.x, NC = gridDim.x;
@@ -293,20 +283,6 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ P
   const int ssm_slot[2] = {warp, NW + warp};
   const int dt_head = tid - 2 * N;  // threads [256, 320) own the dt rows
   const bool dt_own = tid >= 2 * N && tid < NSH && (dt_head == hA || dt_head == hA + 1);
-
-  // ---- prologue: the first layer's in_proj LoRA-down partial sums over this CTA's hidden rows
-  {
-    const LayerPtrs& L0 = p.L[0];
-    double part = 0.0;
-    if (lane < n_out) {
-      const int o = ro0 + lane;
-      const float v = fmul(__ldcg(p.hidden + o), __ldg(L0.norm_w + o));
-      part = int_to_f64((int)L0.in_lb[(size_t)warp * DM + o]) * (double)v;
-    }
-    part = warp_sum(part);
-    if (lane == 0) p.upin[c * R + warp] = part;
-    block_arrive(p.ctr + CTR_H * CTR_STRIDE);
-  }
 
   for (int l = 0; l < p.n_layers; ++l) {
     const LayerPtrs& Lp = p.L[l];
@@ -356,6 +332,8 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ P
             prefetch_lines(Nx.in_lbs, R * 4);
             prefetch_lines(Nx.out_lbs, R * 4);
             break;
+          case 5: prefetch_l2(Nx.in_lb, R * DM); break;
+          case 6: prefetch_l2(Nx.out_lb, R * E); break;
           default: break;
         }
       }
@@ -382,19 +360,6 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ P
     for (int k = 0; k < 4; ++k) nw[k] = __ldg(Lp.norm_w + tid + k * NT);
 #pragma unroll
     for (int k = 0; k < 8; ++k) gw[k] = __ldg(Lp.gnorm_w + tid + k * NT);
-    // warp r, lane j: out_proj LoRA column of owned SSM row j, and the next in_proj LoRA column of owned
-    // hidden row j (with its next norm weight)
-    int wbo = 0, wbi_next = 0;
-    float gw_own = 0.f, nw_next = 0.f;
-    if (lane < n_ssm) {
-      wbo = (int)Lp.out_lb[(size_t)warp * E + rs0 + lane];
-      gw_own = __ldg(Lp.gnorm_w + rs0 + lane);
-    }
-    if (has_next && lane < n_out) {
-      const LayerPtrs& Nx = p.L[l + 1];
-      wbi_next = (int)Nx.in_lb[(size_t)warp * DM + ro0 + lane];
-      nw_next = __ldg(Nx.norm_w + ro0 + lane);
-    }
     float lbs_in = 0.f, lbs_out = 0.f;
     if (tid >= kChainBase && tid < kChainBase + R) {
       lbs_in = __ldg(Lp.in_lbs + tid - kChainBase);
@@ -444,10 +409,13 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ P
       cp_async16(o_wa[tid], Lp.out_la + (size_t)row * R);
     }
     if (tid < 2 && hA + tid < H) cp_async4(&Dv[tid], Lp.D + hA + tid);
+    // W_B of both linears (every CTA computes t = W_B q itself)
+    for (int k = tid; k < R * DM / 16; k += NT) cp_async16(wb_in + 16 * k, Lp.in_lb + 16 * (size_t)k);
+    for (int k = tid; k < R * E / 16; k += NT) cp_async16(wb_out + 16 * k, Lp.out_lb + 16 * (size_t)k);
     cp_async_wait_all();
 
     // ---------------------------------------------------------------- phase A: h -> in_proj
-    if (!block_wait(p.ctr + CTR_H * CTR_STRIDE, NC * (l + 1), p.err, p.status, p.spin_limit, &sflag))
+    if (l > 0 && !block_wait(p.ctr + CTR_H * CTR_STRIDE, NC * l, p.err, p.status, p.spin_limit, &sflag))
       return;
     double ssA;
     float s0A;
@@ -463,14 +431,12 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ P
         m = fmaxf(m, fabsf(v[k]));
       }
       if (tid < n_out) h_old[tid] = __ldcg(p.hidden + ro0 + tid);
-      const double u = gather_partials(p.upin, NC);
       ss = warp_sum(ss);
       m = warp_max(m);
       if (lane == 0) {
         red_d[warp] = ss;
         red_f[warp] = m;
       }
-      if (lane < R) red_u[warp][lane] = u;
       __syncthreads();
       ss = 0.0;
       m = 0.0f;
@@ -486,6 +452,7 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ P
       for (int k = 0; k < 4; ++k) {
         const int code = m == 0.0f ? 0 : quant_code_fast(v[k], s0, inv_s0);
         q_perm[seg_index<DM / 128>(tid + k * NT)] = (int8_t)code;
+        q_nat[tid + k * NT] = (int8_t)code;
         sq += code;
       }
       sq = warp_sum(sq);
@@ -510,13 +477,17 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ P
           __syncthreads();
           if (tid < n_sh) p.sacc[sh0 + tid] = acc_in[tid];
           block_arrive(p.ctr + CTR_BC * CTR_STRIDE);
+          // LoRA down of the codes: warp r computes t[r]
+          const int t = lora_row<DM / 16>(wb_in + warp * DM, q_nat, lane);
+          if (lane == 0) t_sm[warp] = t;
         }
       }
     }
-    // the fp64 scale chain (RMS, LoRA intermediate, quantizer scale), off the GEMV's critical path: the
+    // the fp64 scale chain (RMS, quantizer scale, LoRA intermediate), off the GEMV's critical path: the
     // chain warp has no pass-1 rows, and the epilogue needs the results only after the B/C wait
-    if (tid >= kChainBase && tid <= kChainBase + R) scale_chain(tid - kChainBase, ssA, s0A, DM, lbs_in,
-                                                              red_u, tf, &s_scale);
+    if (tid == kChainBase + R) s_scale = rms_scale(s0A, rms_of(ssA, DM));
+    __syncthreads();
+    if (tid >= kChainBase && tid < kChainBase + R) tf[tid - kChainBase] = lora_tf(t_sm[tid - kChainBase], lbs_in, s_scale);
 
     // ---------------------------------------------------------------- phase B: epilogues + SSM
     if (!block_wait(p.ctr + CTR_BC * CTR_STRIDE, NC * (l + 1), p.err, p.status, p.spin_limit, &sflag))
@@ -576,18 +547,9 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ P
         if (lane == 0) {
           const float y = __double2float_rn(dadd(acc, dmul((double)Dv[hi], (double)xv)));
           const float g = fmul(y, zsm[rr]);
-          gsm[rr] = g;
           p.gbuf[hp] = g;
         }
       }
-    }
-    __syncthreads();
-    {
-      // out_proj LoRA-down partial sums over the owned rows of g: warp r, lane j
-      double part = 0.0;
-      if (lane < n_ssm) part = int_to_f64(wbo) * (double)fmul(gsm[lane], gw_own);
-      part = warp_sum(part);
-      if (lane == 0) p.upout[c * R + warp] = part;
     }
     block_arrive(p.ctr + CTR_G * CTR_STRIDE);
 #pragma unroll
@@ -618,14 +580,12 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ P
         v[k] = fmul(g, gw[k]);
         m = fmaxf(m, fabsf(v[k]));
       }
-      const double u = gather_partials(p.upout, NC);
       ss = warp_sum(ss);
       m = warp_max(m);
       if (lane == 0) {
         red_d[warp] = ss;
         red_f[warp] = m;
       }
-      if (lane < R) red_u[warp][lane] = u;
       __syncthreads();
       ss = 0.0;
       m = 0.0f;
@@ -641,16 +601,19 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ P
       for (int k = 0; k < 8; ++k) {
         const int code = m == 0.0f ? 0 : quant_code_fast(v[k], s0, inv_s0);
         q_perm[seg_index<E / 128>(tid + k * NT)] = (int8_t)code;
+        q_nat[tid + k * NT] = (int8_t)code;
         sq += code;
       }
       sq = warp_sum(sq);
       if (lane == 0) red_i[warp] = sq;
+      __syncthreads();
+      // LoRA down of the codes (warp r: t[r]); the GEMV warps then take one out_proj row each, and the
+      // chain warp (no out_proj row) computes the quantizer scale
+      const int t = lora_row<E / 16>(wb_out + warp * E, q_nat, lane);
+      if (lane == 0) t_sm[warp] = t;
       if (warp == kChainWarp) {
-        // publish this warp's codes to the GEMV warps without waiting, then run the scale chain
-        asm volatile("bar.arrive 1, %0;" ::"n"(NT) : "memory");
-        if (lane <= R) scale_chain(lane, ss, s0, E, lbs_out, red_u, tf, &s_scale);
+        if (lane == 0) s_scale = rms_scale(s0, rms_of(ss, E));
       } else {
-        asm volatile("bar.sync 1, %0;" ::"n"(NT) : "memory");
         int sumq_c = 0;
 #pragma unroll
         for (int w = 0; w < NW; ++w) sumq_c += red_i[w];
@@ -661,19 +624,12 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ P
       }
     }
     __syncthreads();
+    if (tid >= kChainBase && tid < kChainBase + R) tf[tid - kChainBase] = lora_tf(t_sm[tid - kChainBase], lbs_out, s_scale);
+    __syncthreads();
     if (tid < n_out) {
       const float y = linear_out(acc_out[tid], s_scale, o_sw[tid], o_sa[tid], o_wa[tid], tf, R);
       const float hn = fadd(h_old[tid], y);
       p.hidden[ro0 + tid] = hn;
-      h_new[tid] = hn;
-    }
-    if (has_next) {
-      // the next layer's in_proj LoRA-down partial sums over the owned rows of h: warp r, lane j
-      __syncthreads();
-      double part = 0.0;
-      if (lane < n_out) part = int_to_f64(wbi_next) * (double)fmul(h_new[lane], nw_next);
-      part = warp_sum(part);
-      if (lane == 0) p.upin[c * R + warp] = part;
     }
     block_arrive(p.ctr + CTR_H * CTR_STRIDE);
   }
@@ -741,8 +697,6 @@ cudaError_t launch_fused_decode(const dfssm_layer_t* layers, int n_layers, float
   p.ctr = reinterpret_cast<int*>(base + fused::OFF_CTR);
   p.err = reinterpret_cast<int*>(base + fused::OFF_ERR);
   p.status = reinterpret_cast<int*>(base + fused::OFF_STATUS);
-  p.upin = reinterpret_cast<double*>(base + fused::OFF_UIN);
-  p.upout = reinterpret_cast<double*>(base + fused::OFF_UOUT);
   p.sacc = reinterpret_cast<int*>(base + fused::OFF_SACC);
   p.gbuf = reinterpret_cast<float*>(base + fused::OFF_GBUF);
   p.spin_limit = spin_limit;
@@ -751,7 +705,11 @@ cudaError_t launch_fused_decode(const dfssm_layer_t* layers, int n_layers, float
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(num_sms());
   cfg.blockDim = dim3(fused::NT);
-  cfg.dynamicSmemBytes = 0;
+  // set once (not per launch, so that launches can be captured in a CUDA graph)
+  static const cudaError_t attr_set = cudaFuncSetAttribute(
+      fused::decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, fused::WB_BYTES);
+  if (attr_set != cudaSuccess) return attr_set;
+  cfg.dynamicSmemBytes = fused::WB_BYTES;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeCooperative;

@@ -30,7 +30,7 @@ struct QuantArgs {
   QuantScratch out;
   int8_t* dbg_xq;          // optional taps
   float* dbg_s;
-  float* dbg_tf;
+  int32_t* dbg_t;          // [B][rank] exact LoRA-down t
 };
 cudaError_t launch_quant(const QuantArgs& a, cudaStream_t st);
 

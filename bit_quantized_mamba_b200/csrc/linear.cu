@@ -67,8 +67,8 @@ static cudaError_t launch_pdl(Kern k, dim3 grid, dim3 block, size_t smem, cudaSt
 
 // ------------------------------------------------------------------------------- quantize kernel
 // One CTA per token.  v = x (or fl32(x*norm_w) when the RMSNorm is folded in); s0 = fl32(absmax/127);
-// q = clamp(rint(fl32(v/s0)), +-127); rms = 1 (or sqrt(sum x^2 / n + 1e-5) in fp64); s = fl32(s0/rms);
-// LoRA down on the fp32 input: tf[r] = fl32((sum_i W_B[r,i] v_i) sB[r] / rms), the sum in fp64.
+// q = clamp(rint(fl32(v/s0)), +-127); rms = 1 (or sqrt(sum x^2 / n + 1e-5) in fp64); s = fl32(s0/rms).
+// LoRA down on the codes: t[r] = sum_i W_B[r,i] q_i (int32, dp4a), tf[r] = fl32(t[r] sB[r] s).
 
 constexpr int kQuantThreads = 512;
 
@@ -76,11 +76,12 @@ __global__ void __launch_bounds__(kQuantThreads) quant_kernel(QuantArgs a) {
   pdl_launch_dependents();
   pdl_wait();
   extern __shared__ __align__(16) unsigned char smem[];
-  float* v = reinterpret_cast<float*>(smem);
+  float* v = reinterpret_cast<float*>(smem);                       // [n]
+  int8_t* qn = reinterpret_cast<int8_t*>(smem + (size_t)a.n * 4);  // [n] natural-order codes
   __shared__ double red_d[kQuantThreads / 32];
   __shared__ float red_f[kQuantThreads / 32];
   __shared__ int red_i[kQuantThreads / 32];
-  __shared__ double red_u[kQuantThreads / 32][DFSSM_MAX_RANK];
+  __shared__ int t_sm[DFSSM_MAX_RANK];
   const int b = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
   constexpr int NW = kQuantThreads / 32;
@@ -119,47 +120,32 @@ __global__ void __launch_bounds__(kQuantThreads) quant_kernel(QuantArgs a) {
   for (int i = tid; i < a.n; i += kQuantThreads) {
     const int c = (m == 0.0f) ? 0 : quant_code_fast(v[i], s0, inv_s0);
     sq += c;
+    qn[i] = (int8_t)c;
     qout[a.permute ? perm_index(i) : i] = (int8_t)c;
     if (a.dbg_xq) a.dbg_xq[(size_t)b * a.n + i] = (int8_t)c;
   }
-
-  // LoRA down on the fp32 input, four inputs per step (products int8 x fp32 are exact in fp64).
-  double u[DFSSM_MAX_RANK];
-#pragma unroll
-  for (int r = 0; r < DFSSM_MAX_RANK; ++r) u[r] = 0.0;
-  if (a.rank > 0) {
-    for (int w = tid; w < a.n / 4; w += kQuantThreads) {
-      const float4 v4 = reinterpret_cast<const float4*>(v)[w];
-      const double vd[4] = {(double)v4.x, (double)v4.y, (double)v4.z, (double)v4.w};
-#pragma unroll
-      for (int r = 0; r < DFSSM_MAX_RANK; ++r) {
-        if (r < a.rank) {
-          const uint32_t wb = ld_stream_u32(a.lora_b + (size_t)r * a.n + 4 * (size_t)w);
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const int wj = (int)(int8_t)(wb >> (8 * j));
-            u[r] = fma(int_to_f64(wj), vd[j], u[r]);
-          }
-        }
-      }
-    }
-  }
   sq = warp_sum(sq);
-#pragma unroll
-  for (int r = 0; r < DFSSM_MAX_RANK; ++r) u[r] = warp_sum(u[r]);
-  if (lane == 0) {
-    red_i[wid] = sq;
-#pragma unroll
-    for (int r = 0; r < DFSSM_MAX_RANK; ++r) red_u[wid][r] = u[r];
+  if (lane == 0) red_i[wid] = sq;
+  __syncthreads();
+  // LoRA down: warp r computes t[r] over 4-byte words of W_B row r and of the codes.
+  for (int r = wid; r < a.rank; r += NW) {
+    const uint32_t* wb = reinterpret_cast<const uint32_t*>(a.lora_b + (size_t)r * a.n);
+    const uint32_t* q4 = reinterpret_cast<const uint32_t*>(qn);
+    int part = 0;
+    for (int w = lane; w < a.n / 4; w += 32) part = dp4a_ss(ld_stream_u32(wb + w), q4[w], part);
+    part = __reduce_add_sync(0xffffffffu, part);
+    if (lane == 0) t_sm[r] = part;
   }
   __syncthreads();
   const double rms = a.norm_w ? rms_of(ss, a.n) : 1.0;
+  const float s = a.norm_w ? rms_scale(s0, rms) : s0;
   if (tid < DFSSM_MAX_RANK) {
-    double tot = 0.0;
-    for (int w = 0; w < NW; ++w) tot += red_u[w][tid];
-    const float tf = tid < a.rank ? lora_tf(tot, a.lora_b_scale[tid], rms) : 0.0f;
+    float tf = 0.0f;
+    if (tid < a.rank) {
+      tf = lora_tf(t_sm[tid], a.lora_b_scale[tid], s);
+      if (a.dbg_t) a.dbg_t[(size_t)b * a.rank + tid] = t_sm[tid];
+    }
     a.out.tf[b * DFSSM_MAX_RANK + tid] = tf;
-    if (a.dbg_tf && tid < a.rank) a.dbg_tf[(size_t)b * a.rank + tid] = tf;
   }
   if (tid == DFSSM_MAX_RANK) {
     int tot = 0;
@@ -167,14 +153,13 @@ __global__ void __launch_bounds__(kQuantThreads) quant_kernel(QuantArgs a) {
     a.out.sumq[b] = tot;
   }
   if (tid == DFSSM_MAX_RANK + 1) {
-    const float s = a.norm_w ? rms_scale(s0, rms) : s0;
     a.out.s[b] = s;
     if (a.dbg_s) a.dbg_s[b] = s;
   }
 }
 
 cudaError_t launch_quant(const QuantArgs& a, cudaStream_t st) {
-  const size_t smem = (size_t)a.n * 4;  // <= 32 KB for n <= 8192
+  const size_t smem = (size_t)a.n * 5;  // <= 40 KB for n <= 8192
   return launch_pdl(quant_kernel, dim3(a.B), dim3(kQuantThreads), smem, st, a);
 }
 

@@ -111,7 +111,7 @@ extern "C" int dfssm_linear_decode_noalloc(const dfssm_linear_t* lin, const floa
   if (dbg) {
     qa.dbg_xq = dbg->xq;
     qa.dbg_s = dbg->xscale;
-    qa.dbg_tf = dbg->lora_tf;
+    qa.dbg_t = dbg->lora_t;
   }
   cudaError_t e = dfssm::launch_quant(qa, s);
   if (e != cudaSuccess) return dfssm::record_cuda_failure(e);

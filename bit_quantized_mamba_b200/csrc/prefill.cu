@@ -154,8 +154,8 @@ __global__ void expand_bits_kernel(const uint32_t* __restrict__ bits, int8_t* __
 }
 
 // Quantization for the prefill: one warp per token.  Codes (natural order) and scale exactly as the
-// decode quantizer; the LoRA down-projection u = W_B x runs in fp32 with W_B staged in shared memory
-// (the prefill output is checked to tolerance, its integer accumulators exactly).
+// decode quantizer; the LoRA down-projection t = W_B q on the codes (int32, dp4a) with W_B staged in
+// shared memory, and tf = fl32(t sB s) rounded as in the decode path.
 constexpr int QW = 8;  // tokens (warps) per CTA
 __global__ void __launch_bounds__(QW * 32) prefill_quant_kernel(const float* __restrict__ x, int M, int K,
                                                                const int8_t* __restrict__ lora_b,
@@ -163,7 +163,7 @@ __global__ void __launch_bounds__(QW * 32) prefill_quant_kernel(const float* __r
                                                                int rank, int8_t* __restrict__ xq,
                                                                float* __restrict__ s_out,
                                                                float* __restrict__ tf_out,
-                                                               int8_t* dbg_xq, float* dbg_s, float* dbg_tf) {
+                                                               int8_t* dbg_xq, float* dbg_s, int32_t* dbg_t) {
   extern __shared__ __align__(16) unsigned char sm[];
   int8_t* wb = reinterpret_cast<int8_t*>(sm);  // [rank][K]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -181,9 +181,9 @@ __global__ void __launch_bounds__(QW * 32) prefill_quant_kernel(const float* __r
   m_abs = warp_max(m_abs);
   const float s0 = m_abs == 0.0f ? 0.0f : __fdiv_rn(m_abs, 127.0f);
   const float inv_s0 = m_abs == 0.0f ? 0.0f : __frcp_rn(s0);
-  float u[DFSSM_MAX_RANK];
+  int u[DFSSM_MAX_RANK];
 #pragma unroll
-  for (int r = 0; r < DFSSM_MAX_RANK; ++r) u[r] = 0.0f;
+  for (int r = 0; r < DFSSM_MAX_RANK; ++r) u[r] = 0;
   for (int i = lane * 4; i < K; i += 128) {
     const float4 v = __ldg(reinterpret_cast<const float4*>(xr + i));
     const float vv[4] = {v.x, v.y, v.z, v.w};
@@ -196,24 +196,19 @@ __global__ void __launch_bounds__(QW * 32) prefill_quant_kernel(const float* __r
     *reinterpret_cast<uint32_t*>(xq + (size_t)m * K + i) = packed;
     if (dbg_xq) *reinterpret_cast<uint32_t*>(dbg_xq + (size_t)m * K + i) = packed;
 #pragma unroll
-    for (int r = 0; r < DFSSM_MAX_RANK; ++r) {
-      if (r < rank) {
-        const uint32_t w4 = *reinterpret_cast<const uint32_t*>(wb + (size_t)r * K + i);
-#pragma unroll
-        for (int j = 0; j < 4; ++j) u[r] = fmaf(int8_to_f32((int)(int8_t)(w4 >> (8 * j))), vv[j], u[r]);
-      }
-    }
+    for (int r = 0; r < DFSSM_MAX_RANK; ++r)
+      if (r < rank) u[r] = dp4a_ss(*reinterpret_cast<const uint32_t*>(wb + (size_t)r * K + i), packed, u[r]);
   }
 #pragma unroll
-  for (int r = 0; r < DFSSM_MAX_RANK; ++r) u[r] = warp_sum(u[r]);
+  for (int r = 0; r < DFSSM_MAX_RANK; ++r) u[r] = __reduce_add_sync(0xffffffffu, u[r]);
   if (lane < DFSSM_MAX_RANK) {
-    float uv = 0.0f;
+    int tv = 0;
 #pragma unroll
     for (int r = 0; r < DFSSM_MAX_RANK; ++r)
-      if (r == lane) uv = u[r];
-    const float t = lane < rank ? uv * __ldg(lora_b_scale + lane) : 0.0f;
-    tf_out[(size_t)m * DFSSM_MAX_RANK + lane] = t;
-    if (dbg_tf && lane < rank) dbg_tf[(size_t)m * rank + lane] = t;
+      if (r == lane) tv = u[r];
+    const float tf = lane < rank ? lora_tf(tv, __ldg(lora_b_scale + lane), s0) : 0.0f;
+    tf_out[(size_t)m * DFSSM_MAX_RANK + lane] = tf;
+    if (dbg_t && lane < rank) dbg_t[(size_t)m * rank + lane] = tv;
   }
   if (lane == 0) {
     s_out[m] = s0;
@@ -536,7 +531,7 @@ extern "C" int dfssm_linear_prefill(const dfssm_linear_t* lin, const float* x, i
   }
   prefill::prefill_quant_kernel<<<(M + prefill::QW - 1) / prefill::QW, prefill::QW * 32, qsmem, st>>>(
       x, M, K, lin->lora_b, lin->lora_b_scale, lin->rank, w.xq, w.s, w.tf, dbg ? dbg->xq : nullptr,
-      dbg ? dbg->xscale : nullptr, dbg ? dbg->lora_tf : nullptr);
+      dbg ? dbg->xscale : nullptr, dbg ? dbg->lora_t : nullptr);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return record_cuda_failure(e);
   // 2. +-1 int8 weights

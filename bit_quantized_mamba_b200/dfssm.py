@@ -42,7 +42,7 @@ class LinearT(C.Structure):
 
 
 class DebugT(C.Structure):
-    _fields_ = [("acc", C.c_void_p), ("lora_tf", C.c_void_p), ("xq", C.c_void_p),
+    _fields_ = [("acc", C.c_void_p), ("lora_t", C.c_void_p), ("xq", C.c_void_p),
                 ("xscale", C.c_void_p)]
 
 
@@ -162,7 +162,7 @@ def linear_decode(lin: Linear, x: torch.Tensor, y: torch.Tensor | None = None, w
         ws = workspace(workspace_size(OP_LINEAR_DECODE, B, lin.d_in, lin.d_out), x.device)
     dbg = None
     if debug is not None:
-        dbg = DebugT(*(_ptr(debug.get(k)) for k in ("acc", "lora_tf", "xq", "xscale")))
+        dbg = DebugT(*(_ptr(debug.get(k)) for k in ("acc", "lora_t", "xq", "xscale")))
     _check("dfssm_linear_decode", lib().dfssm_linear_decode(
         C.byref(lin.cstruct()), _ptr(x), B, _ptr(y), _ptr(ws), ws.numel(),
         C.byref(dbg) if dbg is not None else None, _stream(stream)))
@@ -177,7 +177,7 @@ def linear_decode_noalloc(lin: Linear, x: torch.Tensor, y: torch.Tensor | None =
         y = torch.empty((B, lin.d_out), dtype=torch.float32, device=x.device)
     dbg = None
     if debug is not None:
-        dbg = DebugT(*(_ptr(debug.get(k)) for k in ("acc", "lora_tf", "xq", "xscale")))
+        dbg = DebugT(*(_ptr(debug.get(k)) for k in ("acc", "lora_t", "xq", "xscale")))
     _check("dfssm_linear_decode_noalloc", lib().dfssm_linear_decode_noalloc(
         C.byref(lin.cstruct()), _ptr(x), B, _ptr(y), C.byref(dbg) if dbg is not None else None,
         _stream(stream)))
@@ -193,7 +193,7 @@ def linear_prefill(lin: Linear, x: torch.Tensor, y: torch.Tensor | None = None, 
         ws = workspace(workspace_size(OP_LINEAR_PREFILL, M, lin.d_in, lin.d_out), x.device)
     dbg = None
     if debug is not None:
-        dbg = DebugT(*(_ptr(debug.get(k)) for k in ("acc", "lora_tf", "xq", "xscale")))
+        dbg = DebugT(*(_ptr(debug.get(k)) for k in ("acc", "lora_t", "xq", "xscale")))
     _check("dfssm_linear_prefill", lib().dfssm_linear_prefill(
         C.byref(lin.cstruct()), _ptr(x), M, _ptr(y), _ptr(ws), ws.numel(),
         C.byref(dbg) if dbg is not None else None, _stream(stream)))

@@ -35,7 +35,7 @@
 extern "C" {
 #endif
 
-#define DFSSM_ABI_VERSION 1
+#define DFSSM_ABI_VERSION 2
 #define DFSSM_MAX_RANK 16
 #define DFSSM_MAX_BATCH 16
 #define DFSSM_MAX_LAYERS 64
@@ -64,7 +64,8 @@ typedef enum {
  * (lora_* may then be NULL).
  * Computes, for each token b with input x and (q, s) its per-token int8 quantization:
  *   acc[o] = sum_i sign(o,i) q[i]  (int32, exact)
- *   tf[r]  = fl32((sum_i W_B[r,i] x[i]) sB[r])           (LoRA down on the fp32 input, fp64 sum)
+ *   t[r]   = sum_i W_B[r,i] q[i]  (int32, exact)           (LoRA down on the same int8 codes)
+ *   tf[r]  = fl32(t[r] sB[r] s)                            (fp64 inside, this order)
  *   y[o]   = fl32(acc[o] s sW[o] + sA[o] sum_r W_A[o,r] tf[r])   (fp64 inside)
  */
 typedef struct {
@@ -80,7 +81,7 @@ typedef struct {
 /* Optional device taps of the intermediates (any member may be NULL). */
 typedef struct {
   int32_t* acc;   /* [B][d_out]  scaffold accumulators (int32, exact)                      */
-  float* lora_tf; /* [B][rank]   LoRA intermediate tf                                      */
+  int32_t* lora_t; /* [B][rank]  LoRA-down accumulators t (int32, exact)                  */
   int8_t* xq;     /* [B][d_in]   quantized activations, natural order                     */
   float* xscale;  /* [B]         per-token scale s                                         */
 } dfssm_debug_t;

@@ -37,7 +37,7 @@ def test_library_exports_every_declared_symbol(L):
     for n in names:
         assert hasattr(L, n), f"{n} declared in dfssm.h but not exported"
     assert set(names) == set(dfssm.SIGNATURES), "binding and header disagree"
-    assert L.dfssm_abi_version() == 1
+    assert L.dfssm_abi_version() == 2
 
 
 def test_status_strings(L):

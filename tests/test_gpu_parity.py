@@ -46,13 +46,13 @@ def run_linear(lin_host, x, dev):
     L = dfssm.Linear.from_host(lin_host, dev)
     B = x.shape[0]
     dbg = dict(acc=torch.zeros((B, L.d_out), dtype=torch.int32, device=dev),
-               lora_tf=torch.zeros((B, max(L.rank, 1)), dtype=torch.float32, device=dev),
+               lora_t=torch.zeros((B, max(L.rank, 1)), dtype=torch.int32, device=dev),
                xq=torch.zeros((B, L.d_in), dtype=torch.int8, device=dev),
                xscale=torch.zeros(B, dtype=torch.float32, device=dev))
     y = dfssm.linear_decode(L, to_dev(x, dev), debug=dbg)
     torch.cuda.synchronize()
     out = {k: v.cpu().numpy() for k, v in dbg.items()}
-    out["lora_tf"] = out["lora_tf"][:, :L.rank]
+    out["lora_t"] = out["lora_t"][:, :L.rank]
     out["y"] = y.cpu().numpy()
     return out
 
@@ -61,7 +61,8 @@ def compare_linear(g, r, what):
     assert np.array_equal(g["xq"], r["xq"]), f"{what}: int8 codes differ"
     assert np.array_equal(g["xscale"], r["xscale"]), f"{what}: scales differ"
     assert np.array_equal(g["acc"], r["acc"]), f"{what}: scaffold accumulators differ"
-    return assert_tol(g["lora_tf"], r["tf"], what + " tf") + assert_tol(g["y"], r["y"], what)
+    assert np.array_equal(g["lora_t"], r["t"]), f"{what}: LoRA-down accumulators differ"
+    return assert_tol(g["y"], r["y"], what)
 
 
 def test_linear_tiny(dev):
@@ -125,7 +126,7 @@ def test_linear_full_stacks(dev, which):
             else:
                 rows = np.sort(gen.choice(OL.d_out, 64, replace=False))
                 for b in range(B):
-                    rtf = oracle.lora_down(OL, x[b])
+                    _, rtf = oracle.lora_down(OL, rq[b], rs[b])
                     ry, racc = oracle.linear_rows(OL, rq[b], rs[b], rtf, rows)
                     assert np.array_equal(acc[b, rows], racc), (which, B, c, b)
                     assert assert_tol(y[b, rows], ry, f"{which} B{B} copy{c}") == 0
@@ -278,12 +279,12 @@ def test_device_wait_timeout_is_reported(dev):
 
 def _prefill_compare(dev, lin_host, x, rows):
     """Prefill through the C ABI vs the oracle: int8 codes and scales of every token exact; scaffold
-    accumulators exact and the LoRA intermediate / outputs within tolerance on the listed rows."""
+    accumulators and LoRA-down accumulators exact and the outputs within tolerance on the listed rows."""
     from bit_quantized_mamba_b200 import dfssm
     L = dfssm.Linear.from_host(lin_host, dev)
     M = x.shape[0]
     dbg = dict(acc=torch.zeros((M, L.d_out), dtype=torch.int32, device=dev),
-               lora_tf=torch.zeros((M, L.rank), dtype=torch.float32, device=dev),
+               lora_t=torch.zeros((M, L.rank), dtype=torch.int32, device=dev),
                xq=torch.zeros((M, L.d_in), dtype=torch.int8, device=dev),
                xscale=torch.zeros(M, dtype=torch.float32, device=dev))
     y = dfssm.linear_prefill(L, to_dev(x, dev), debug=dbg)
@@ -292,10 +293,10 @@ def _prefill_compare(dev, lin_host, x, rows):
     rq, rs = oracle.quantize(x)
     assert np.array_equal(dbg["xq"].cpu().numpy(), rq), "prefill int8 codes differ"
     assert np.array_equal(dbg["xscale"].cpu().numpy(), rs), "prefill scales differ"
-    yg, accg, tfg = y.cpu().numpy(), dbg["acc"].cpu().numpy(), dbg["lora_tf"].cpu().numpy()
+    yg, accg, tg = y.cpu().numpy(), dbg["acc"].cpu().numpy(), dbg["lora_t"].cpu().numpy()
     for m in rows:
-        tf = oracle.lora_down(OL, x[m])
-        assert_tol(tfg[m], tf, f"prefill tf row {m}")
+        t, tf = oracle.lora_down(OL, rq[m], rs[m])
+        assert np.array_equal(tg[m], t), f"prefill LoRA-down accumulators differ at row {m}"
         yr, accr = oracle.linear_core(OL, rq[m], rs[m], tf)
         assert np.array_equal(accg[m], accr), f"prefill scaffold accumulators differ at row {m}"
         assert_tol(yg[m], yr, f"prefill y row {m}")

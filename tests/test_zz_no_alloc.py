@@ -27,7 +27,7 @@ def dev():
 
 def _taps(B, L, dev):
     return dict(acc=torch.zeros((B, L.d_out), dtype=torch.int32, device=dev),
-                lora_tf=torch.zeros((B, L.rank), dtype=torch.float32, device=dev),
+                lora_t=torch.zeros((B, L.rank), dtype=torch.int32, device=dev),
                 xq=torch.zeros((B, L.d_in), dtype=torch.int8, device=dev),
                 xscale=torch.zeros(B, dtype=torch.float32, device=dev))
 
@@ -43,7 +43,7 @@ def test_noalloc_matches_workspace_entry_point_on_two_calls(dev):
         y_ref = dfssm.linear_decode(L, x, debug=ref_taps)
         y = dfssm.linear_decode_noalloc(L, x, debug=got_taps)
         torch.cuda.synchronize()
-        for k in ("acc", "lora_tf", "xq", "xscale"):
+        for k in ("acc", "lora_t", "xq", "xscale"):
             assert torch.equal(got_taps[k], ref_taps[k]), (seed, k)
         yr, yg = y_ref.cpu().numpy().astype(np.float64), y.cpu().numpy().astype(np.float64)
         assert np.all(np.abs(yg - yr) <= RTOL * (1 + np.abs(yr))), seed
