@@ -329,6 +329,32 @@ def run_ours(args, rank, world, local_rank):
                 gbs = nbytes / (us_per_call * 1e-6) / 1e9
                 gemv[f"{which}_B{B}"] = {"us_per_call": round(us_per_call, 3), "GB_s": round(gbs, 1),
                                          "frac_of_measured_hbm": round(gbs / hbm, 3)}
+                if B > 4:
+                    continue
+                # the same 48 copies in one dfssm_linear_decode_multi launch (shared input x)
+                ys = [torch.empty((B, L.d_out), dtype=torch.float32, device=dev) for L in lins]
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.stream(stream):
+                    dfssm.linear_decode_multi(lins, xb, ys, stream=torch.cuda.current_stream())
+                    torch.cuda.synchronize()
+                    with torch.cuda.graph(g, stream=stream):
+                        dfssm.linear_decode_multi(lins, xb, ys, stream=torch.cuda.current_stream())
+                tot, reps = 0.0, 10
+                with torch.cuda.stream(stream):
+                    for r in range(reps + 2):
+                        flush.fill_(r & 0xFF)
+                        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                        a.record()
+                        g.replay()
+                        b.record()
+                        b.synchronize()
+                        if r >= 2:
+                            tot += a.elapsed_time(b)
+                del g, ys
+                us_all = tot / reps * 1e3
+                gbs = nbytes * len(lins) / (us_all * 1e-6) / 1e9
+                gemv[f"{which}_B{B}_multi"] = {"us_per_48_copies": round(us_all, 3), "GB_s": round(gbs, 1),
+                                               "frac_of_measured_hbm": round(gbs / hbm, 3)}
             del lins
 
     # ---- prefill (2048 tokens) on tcgen05 int8, and the int8 LM head on the last token

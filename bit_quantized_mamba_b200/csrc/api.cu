@@ -174,6 +174,7 @@ int dfssm_linear_decode(const dfssm_linear_t* lin, const float* x, int B, float*
     return DFSSM_EWORKSPACE;
   if (!device_ok()) return DFSSM_EDEVICE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (dfssm::stream_supported(lin->d_in, B)) return dfssm::launch_linear_stream(lin, 1, x, B, &y, dbg, s);
   dfssm::QuantScratch qs = dfssm::carve_quant_scratch(workspace, B, lin->d_in);
   dfssm::QuantArgs qa{};
   qa.x = x;
@@ -200,6 +201,23 @@ int dfssm_linear_decode(const dfssm_linear_t* lin, const float* x, int B, float*
   e = dfssm::launch_gemv(ga, s);
   if (e != cudaSuccess) return cuda_fail(e);
   return DFSSM_OK;
+}
+
+int dfssm_linear_decode_multi(const dfssm_linear_t* lins, int n, const float* x, int B, float* const* ys,
+                              void* stream) {
+  if (!lins || !ys || !x || n < 1 || B < 1) return DFSSM_EINVAL;
+  if (n > DFSSM_MAX_LAYERS) return DFSSM_EUNSUPPORTED;
+  for (int j = 0; j < n; ++j) {
+    const int st = check_linear(&lins[j]);
+    if (st) return st;
+    if (lins[j].d_in != lins[0].d_in) return DFSSM_EINVAL;
+    if (!ys[j]) return DFSSM_EINVAL;
+    if (!aligned(ys[j], 4)) return DFSSM_EALIGN;
+  }
+  if (!dfssm::stream_supported(lins[0].d_in, B)) return DFSSM_EUNSUPPORTED;
+  if (!aligned(x, 16)) return DFSSM_EALIGN;
+  if (!device_ok()) return DFSSM_EDEVICE;
+  return dfssm::launch_linear_stream(lins, n, x, B, ys, nullptr, static_cast<cudaStream_t>(stream));
 }
 
 int dfssm_conv_step(float* conv_state, const float* w, const float* b, const float* x_in, float* x_out,
@@ -354,12 +372,25 @@ int dfssm_layer_decode(const dfssm_layer_t* layers, int n_layers, const dfssm_di
 }
 
 int dfssm_device_status(void* workspace, void* stream) {
-  if (!workspace || !aligned(workspace, 256)) return DFSSM_EWORKSPACE;
+  if (workspace && !aligned(workspace, 256)) return DFSSM_EWORKSPACE;
   if (!device_ok()) return DFSSM_EDEVICE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
   int code = 0;
-  const int e = dfssm::read_device_error(workspace, static_cast<cudaStream_t>(stream), &code);
-  if (e) return cuda_fail(static_cast<cudaError_t>(e));
-  return code ? DFSSM_ETIMEOUT : DFSSM_OK;
+  if (workspace) {
+    const int e = dfssm::read_device_error(workspace, s, &code);
+    if (e) return cuda_fail(static_cast<cudaError_t>(e));
+  }
+  // the streaming linear kernels' module status word
+  int* word = nullptr;
+  const int st = dfssm::stream_status_word(&word);
+  if (st) return st;
+  int h = 0;
+  cudaError_t e = cudaMemcpyAsync(&h, word, sizeof(int), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(word, 0, sizeof(int), s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e);
+  return (code || h) ? DFSSM_ETIMEOUT : DFSSM_OK;
 }
 
 int dfssm_selftest_timeout(void* workspace, size_t ws_bytes, void* stream) {

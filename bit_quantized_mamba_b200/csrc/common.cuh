@@ -110,24 +110,102 @@ __device__ __forceinline__ int perm_index(int i) {
   return (i & ~31) + ((j & 7) << 2) + (j >> 3);
 }
 
+// ---------------------------------------------------------------- scaffold GEMV inner loop
+
+// Shared-memory position of natural activation index i: the dp4a-permuted codes of 128-input segment
+// `seg` occupy eight 16-byte chunks, and chunk v of every segment is stored contiguously across the
+// NSEG segments (byte (v * NSEG + seg) * 16 + pos % 16), so the lanes that each own one segment read
+// consecutive chunks without bank conflicts.
+template <int NSEG>
+__device__ __forceinline__ int seg_index(int i) {
+  const int seg = i >> 7;
+  const int pos = perm_index(i) & 127;
+  return ((pos >> 4) * NSEG + seg) * 16 + (pos & 15);
+}
+
+// Sum over bit=1 positions of q for 128 weights (one uint4 of sign bits) against the permuted codes of
+// their segment; chunk v of the segment is qp4[v * NSEG].
+template <int NSEG>
+__device__ __forceinline__ int bits_dot(uint4 w, const uint4* qp4) {
+  int acc8[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) acc8[k] = 0;
+  const uint32_t w4[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const uint4 qa = qp4[(2 * j) * NSEG], qb = qp4[(2 * j + 1) * NSEG];
+    const uint32_t qp[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
+#pragma unroll
+    for (int k = 0; k < 8; ++k) acc8[k] = dp4a_us(w4[j] & (0x01010101u << k), qp[k], acc8[k]);
+  }
+  int S = 0;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) S += acc8[k] >> k;
+  return S;
+}
+
 // ---------------------------------------------------------------- the method's arithmetic
 // These few functions fix the rounding sequence of every fp32 value the decode path stores; all
 // kernels (the per-op kernels and the fused decode kernel) use them, so both paths agree bit for bit.
-
-// Linear output for one (token, row): fl32(acc*s*sW + sA * sum_r W_A[r]*tf[r]), fp64 in this order.
-__device__ __forceinline__ float linear_out(int acc, float s, float sW, float sA, const int8_t* wa,
-                                            const float* tf, int rank) {
-  double lora = 0.0;
-  for (int r = 0; r < rank; ++r) lora = dadd(lora, dmul((double)wa[r], (double)tf[r]));
-  const double scaffold = dmul(dmul((double)acc, (double)s), (double)sW);
-  const double corr = rank > 0 ? dmul((double)sA, lora) : 0.0;
-  return __double2float_rn(dadd(scaffold, corr));
-}
 
 // Exact fp64 value of a 32-bit integer without the (slow) integer-to-double conversion unit:
 // 2^52 + 2^31 + w read as a double, minus 2^52 + 2^31.
 __device__ __forceinline__ double int_to_f64(int w) {
   return __hiloint2double(0x43300000, w ^ (int)0x80000000) - 4503601774854144.0;
+}
+
+// Linear output for one (token, row): fl32(acc*s*sW + sA * sum_r W_A[r]*tf[r]), fp64 in this order.
+// Operands already in fp64 (exact images of the fp32 values); wa holds W_A[row][0..15] as 16 bytes
+// (entries >= rank ignored).  Integers reach fp64 through int_to_f64, not the conversion unit.
+// N independent (token, row) outputs are evaluated with their dependency chains interleaved; RK is the
+// rank when known at compile time, or -1 (then `rank` is used).
+template <int N, int RK>
+__device__ __forceinline__ void linear_out_n(const int (&acc)[N], const double (&s)[N], const double (&sW)[N],
+                                             const double (&sA)[N], const uint4 (&wa)[N],
+                                             const double* const (&tf)[N], int rank, float (&out)[N]) {
+  const int rk = RK >= 0 ? RK : rank;
+  double lora[N];
+#pragma unroll
+  for (int n = 0; n < N; ++n) lora[n] = 0.0;
+#pragma unroll
+  for (int r = 0; r < DFSSM_MAX_RANK; ++r) {
+    if (r < rk) {
+#pragma unroll
+      for (int n = 0; n < N; ++n) {
+        const uint32_t w = r < 4 ? wa[n].x : r < 8 ? wa[n].y : r < 12 ? wa[n].z : wa[n].w;
+        lora[n] = dadd(lora[n], dmul(int_to_f64((int)(int8_t)(w >> (8 * (r & 3)))), tf[n][r]));
+      }
+    }
+  }
+#pragma unroll
+  for (int n = 0; n < N; ++n) {
+    const double scaffold = dmul(dmul(int_to_f64(acc[n]), s[n]), sW[n]);
+    const double corr = rk > 0 ? dmul(sA[n], lora[n]) : 0.0;
+    out[n] = __double2float_rn(dadd(scaffold, corr));
+  }
+}
+__device__ __forceinline__ float linear_out_d(int acc, double s, double sW, double sA, uint4 wa,
+                                              const double* tf, int rank) {
+  const int a[1] = {acc};
+  const double sv[1] = {s}, w[1] = {sW}, av[1] = {sA};
+  const uint4 wv[1] = {wa};
+  const double* const t[1] = {tf};
+  float o[1];
+  linear_out_n<1, -1>(a, sv, w, av, wv, t, rank, o);
+  return o[0];
+}
+// Same with fp32 operands.
+__device__ __forceinline__ float linear_out(int acc, float s, float sW, float sA, uint4 wa, const float* tf,
+                                            int rank) {
+  double tfd[DFSSM_MAX_RANK];
+#pragma unroll
+  for (int r = 0; r < DFSSM_MAX_RANK; ++r) tfd[r] = r < rank ? (double)tf[r] : 0.0;
+  return linear_out_d(acc, (double)s, (double)sW, (double)sA, wa, tfd, rank);
+}
+// Same, W_A row in 16-byte-aligned memory (shared memory or registers).
+__device__ __forceinline__ float linear_out(int acc, float s, float sW, float sA, const int8_t* wa,
+                                            const float* tf, int rank) {
+  return linear_out(acc, s, sW, sA, *reinterpret_cast<const uint4*>(wa), tf, rank);
 }
 
 // LoRA intermediate tf = fl32(t * sB * s) (fp64, this order): t = sum_i W_B[r,i] q_i is the exact int32

@@ -165,40 +165,6 @@ __device__ __forceinline__ void cp_async_wait_all() {
   asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
 }
 
-// ------------------------------------------------------------------------------ GEMV inner loop
-
-// Shared-memory position of natural activation index i: the dp4a-permuted codes of 128-input segment
-// `seg` occupy eight 16-byte chunks, and chunk v of every segment is stored contiguously across the
-// NSEG segments (byte (v * NSEG + seg) * 16 + pos % 16), so the lanes that each own one segment read
-// consecutive chunks without bank conflicts.
-template <int NSEG>
-__device__ __forceinline__ int seg_index(int i) {
-  const int seg = i >> 7;
-  const int pos = perm_index(i) & 127;
-  return ((pos >> 4) * NSEG + seg) * 16 + (pos & 15);
-}
-
-// Sum over bit=1 positions of q for 128 weights (one uint4 of sign bits) against the permuted codes of
-// their segment; chunk v of the segment is qp4[v * NSEG].
-template <int NSEG>
-__device__ __forceinline__ int bits_dot(uint4 w, const uint4* qp4) {
-  int acc8[8];
-#pragma unroll
-  for (int k = 0; k < 8; ++k) acc8[k] = 0;
-  const uint32_t w4[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    const uint4 qa = qp4[(2 * j) * NSEG], qb = qp4[(2 * j + 1) * NSEG];
-    const uint32_t qp[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
-#pragma unroll
-    for (int k = 0; k < 8; ++k) acc8[k] = dp4a_us(w4[j] & (0x01010101u << k), qp[k], acc8[k]);
-  }
-  int S = 0;
-#pragma unroll
-  for (int k = 0; k < 8; ++k) S += acc8[k] >> k;
-  return S;
-}
-
 // LoRA down-projection row r = warp: t[r] = sum_i W_B[r,i] q_i over NCH 16-byte chunks, lane taking
 // chunks lane, lane + 32, ... of the natural-order codes and of W_B row r (conflict-free in shared memory).
 template <int NCH>

@@ -110,6 +110,12 @@ cudaError_t launch_fused_decode(const dfssm_layer_t* layers, int n_layers, float
 cudaError_t launch_timeout_selftest(void* ws, cudaStream_t st, long long spin_limit);
 // Reads and clears the device error word of a fused-decode workspace region (synchronises st).
 int read_device_error(void* ws, cudaStream_t st, int* code);
+// Streaming decode of n linears that share x (B <= 4, d_in = 128 * 2^k <= 8192): one persistent launch.
+bool stream_supported(int d_in, int B);
+int launch_linear_stream(const dfssm_linear_t* lins, int n, const float* x, int B, float* const* ys,
+                         const dfssm_debug_t* dbg, cudaStream_t st);
+// Device address of the streaming kernels' status word on the current device.
+int stream_status_word(int** out);
 // Records e as the text returned by dfssm_last_cuda_error (this thread) and returns DFSSM_ECUDA.
 int record_cuda_failure(cudaError_t e);
 }  // namespace dfssm

@@ -344,7 +344,7 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_generic_kernel(GemvArgs a) 
   if (valid && lane == 0) {
     float sW = a.w_scale[row];
     float sA = a.rank > 0 ? a.lora_a_scale[row] : 0.0f;
-    int8_t wa[DFSSM_MAX_RANK];
+    alignas(16) int8_t wa[DFSSM_MAX_RANK] = {};
     for (int r = 0; r < a.rank; ++r) wa[r] = a.lora_a[(size_t)row * a.rank + r];
 #pragma unroll
     for (int b = 0; b < BT; ++b)

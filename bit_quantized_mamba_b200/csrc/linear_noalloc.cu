@@ -91,11 +91,13 @@ extern "C" int dfssm_linear_decode_noalloc(const dfssm_linear_t* lin, const floa
       cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
       major != 10)
     return DFSSM_EDEVICE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // B <= 4 at d_in in {1024, ..., 8192}: the single streaming kernel needs no scratch at all
+  if (dfssm::stream_supported(lin->d_in, B)) return dfssm::launch_linear_stream(lin, 1, x, B, &y, dbg, s);
   void* scratch = nullptr;
   st = scratch_address(&scratch);
   if (st) return st;
 
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
   const dfssm::QuantScratch qs = dfssm::carve_quant_scratch(scratch, B, lin->d_in);
   dfssm::QuantArgs qa{};
   qa.x = x;

@@ -1,0 +1,767 @@
+// Streaming decode of DF-SSM linears that share one input (gist.science technical summary of DF-SSM,
+// §2.B "Frozen Scaffold with LoRA Correction" and §2.C "Optimized Inference Pipeline": the scaffold
+// matmul on 1-bit packed weights with int8 activations and int32 accumulation, plus the int8 LoRA).
+//
+// At batch <= 4 the scaffold product is a matrix-vector product bound by the HBM stream of sign bits, so
+// one persistent, warp-specialised kernel does everything for any number of linears that read the same x:
+//   * the rows of all linears are cut into 16 KB tiles of packed bits; each CTA takes a contiguous range
+//     of tiles.  A producer warp streams every tile into a ring of shared-memory stages and its rows' W_A
+//     and scales into a second ring, with bulk asynchronous copies (cp.async.bulk, completion counted on
+//     mbarriers), several tiles ahead, and copies each linear's W_B ahead of that linear's first tile;
+//     a bits stage is refilled as soon as the GEMV warps have read it, a parameter stage once its
+//     epilogue is done;
+//   * sixteen GEMV warps quantize x (per-token absmax int8, codes in the dp4a-permuted,
+//     bank-conflict-free segment layout and in natural order; at batch 1 each lane keeps its segment's
+//     codes in registers), compute each linear's LoRA-down t = W_B q (exact int32, dp4a) and
+//     tf = fl32(t sB s), and turn every stage into int32 accumulators
+//     acc = 2 sum_{bit=1} q - sum q (one AND and one dp4a per four weights);
+//   * six epilogue warps turn each stage's accumulators into y = fl32(acc s sW + sA sum_r W_A tf) (the
+//     fp64 epilogue shared by every path) while the GEMV warps already work on the next stages, and
+//     release the stage to the producer.
+// The linear descriptors are copied into shared memory at the start, so the hot loops never index the
+// kernel's parameter block with a run-time index.
+// The sign bits are immutable weights, so the producer starts streaming before the kernel waits on the
+// preceding kernel of the stream (programmatic dependent launch).
+//
+// Every mbarrier wait is bounded.  A wait that runs out of budget stores a timeout code in the module's
+// status word (read and cleared by dfssm_device_status); the CTA then stops computing, still waits
+// (bounded) for every copy it issued, and returns.
+
+#include <mutex>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace dfssm {
+namespace stream {
+
+constexpr int NCW = 16;                  // GEMV warps
+constexpr int NEW = 6;                   // epilogue warps
+constexpr int PROD_WARP = NCW + NEW;     // producer warp
+constexpr int NT = (NCW + NEW + 1) * 32;
+constexpr int TILE_BYTES = 16384;        // packed bits per tile
+constexpr int MAX_TR = 128;              // rows per tile (d_in >= 1024)
+constexpr int MAX_B = 4;
+constexpr int R = DFSSM_MAX_RANK;
+constexpr int MAX_NS = 8;                // stages per ring (bits ring and parameter ring alike)
+// parameter stage: W_A rows (16 B), sW, sA (4 B each) by bulk copy, then the int32 accumulators and the
+// LoRA intermediates (fp64) written by the GEMV warps
+constexpr int P_WA = 0, P_SW = MAX_TR * 16, P_SA = P_SW + MAX_TR * 4, P_ACC = P_SA + MAX_TR * 4,
+              P_TF = P_ACC + MAX_TR * MAX_B * 4, P_BYTES = P_TF + MAX_B * R * 8;
+constexpr int MAX_LIN = DFSSM_MAX_LAYERS;
+constexpr long long kWaitBudget = 2000000000LL;  // clock cycles per wait (~1 s)
+constexpr int kTimeoutCode = 0x5EA0715E;
+
+struct Lin {
+  const uint32_t* bits;
+  const float* w_scale;
+  const int8_t* lora_b;
+  const float* lora_b_scale;
+  const int8_t* lora_a;
+  const float* lora_a_scale;
+  float* y;        // [B][d_out]
+  int d_out;
+  int rank;
+  int tile0;       // index of this linear's first tile in the global tile list
+  int ntiles;
+  int ptma;        // set on the device: the per-row parameters may travel with the bits (bulk copy)
+};
+
+struct Params {
+  Lin lin[MAX_LIN];
+  int n_lin;
+  int d_in;
+  int B;
+  const float* x;  // [B][d_in]
+  int total_tiles;
+  int tile_rows;
+  // optional taps (single linear only): codes, scales, LoRA-down t, scaffold accumulators
+  int8_t* dbg_xq;
+  float* dbg_s;
+  int32_t* dbg_t;
+  int32_t* dbg_acc;
+  int* status;
+};
+
+// ------------------------------------------------------------------------------ mbarrier / bulk copy
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait for the completion of the phase with the given parity.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity))
+    if (clock64() - t0 > kWaitBudget) return false;
+  return true;
+}
+// Bulk copy of `bytes` (multiple of 16; both addresses 16-byte aligned) from global to shared memory,
+// completion counted on `bar`.
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+// Named barrier over the GEMV warps only.
+__device__ __forceinline__ void consumer_sync() {
+  asm volatile("bar.sync 1, %0;" ::"n"(NCW * 32) : "memory");
+}
+
+// Bounded wait that also gives up once another role has aborted.
+__device__ __forceinline__ bool mbar_wait_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity)) {
+    if (*abort_flag) return false;
+    if (clock64() - t0 > kWaitBudget) return false;
+  }
+  return true;
+}
+
+// One L2 prefetch per 128-byte line of [p, p + bytes), spread over n threads (this one is idx).
+__device__ __forceinline__ void prefetch_range(const void* p, size_t bytes, int idx, int n) {
+  const uintptr_t a0 = reinterpret_cast<uintptr_t>(p) & ~uintptr_t(127);
+  const uintptr_t e = reinterpret_cast<uintptr_t>(p) + bytes;
+  for (uintptr_t a = a0 + (uintptr_t)idx * 128; a < e; a += (uintptr_t)n * 128)
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(a) : "memory");
+}
+
+// Dynamic shared memory: the bits ring, the parameter ring (ns stages each), W_B of the current linear
+// when it fits, and the codes in both layouts.  ns is the largest stage count (<= 8) that fits.
+constexpr size_t kSmemBudget = 215 * 1024;
+__host__ __device__ constexpr size_t base_smem(int din, int bt, int ns) {
+  return (size_t)ns * (TILE_BYTES + P_BYTES) + 2 * (size_t)bt * din;
+}
+__host__ __device__ constexpr int n_stages(int din, int bt) {
+  return base_smem(din, bt, 8) <= kSmemBudget ? 8 : base_smem(din, bt, 7) <= kSmemBudget ? 7
+         : base_smem(din, bt, 6) <= kSmemBudget ? 6 : 5;
+}
+__host__ __device__ constexpr bool wb_in_smem(int din, int bt) {
+  return base_smem(din, bt, n_stages(din, bt)) + (size_t)R * din <= kSmemBudget;
+}
+__host__ __device__ constexpr size_t smem_bytes(int din, int bt) {
+  return base_smem(din, bt, n_stages(din, bt)) + (wb_in_smem(din, bt) ? (size_t)R * din : 0);
+}
+
+// Position in the CTA's contiguous tile range: linear j, tile t of that linear.
+struct Cursor {
+  int j, t;
+  __device__ __forceinline__ void start(const Lin* L, int n, int k) {
+    j = 0;
+    while (j + 1 < n && L[j + 1].tile0 <= k) ++j;
+    t = k - L[j].tile0;
+  }
+  __device__ __forceinline__ void next(const Lin* L) {
+    if (++t == L[j].ntiles) {
+      ++j;
+      t = 0;
+    }
+  }
+};
+
+// W_A row of one output row as 16 bytes (zero beyond rank).
+__device__ __forceinline__ uint4 load_wa(const Lin& L, int row) {
+  if (L.rank == R) return __ldg(reinterpret_cast<const uint4*>(L.lora_a + (size_t)row * R));
+  uint32_t w[4] = {0u, 0u, 0u, 0u};
+  for (int r = 0; r < L.rank; ++r)
+    w[r >> 2] |= (uint32_t)(uint8_t)L.lora_a[(size_t)row * L.rank + r] << (8 * (r & 3));
+  return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+// 128 x (sum over bit=1 positions of q) for 128 weights against BT tokens' permuted codes of one segment:
+// token b's chunk v is q0[b * DIN / 16 + v * SEGS].
+template <int SEGS, int BT>
+__device__ __forceinline__ void bits_dot_tokens(uint4 w, const uint4* q0, int B, int (&S)[BT]) {
+  constexpr int DIN16 = SEGS * 8;  // 16-byte chunks per token
+  const uint32_t w4[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+  for (int b = 0; b < BT; ++b) {
+    if (b < B) {
+      const uint4* qp4 = q0 + b * DIN16;
+      int acc8[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) acc8[k] = 0;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const uint4 qa = qp4[(2 * j) * SEGS], qb = qp4[(2 * j + 1) * SEGS];
+        const uint32_t qp[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
+#pragma unroll
+        for (int k = 0; k < 8; ++k) acc8[k] = dp4a_us(w4[j] & (0x01010101u << k), qp[k], acc8[k]);
+      }
+      // acc8[k] = 2^k X_k exactly; sum_k acc8[k] 2^(7-k) = 128 sum_k X_k (multiply-adds, no shifts)
+#pragma unroll
+      for (int k = 0; k < 8; ++k) S[b] += acc8[k] * (1 << (7 - k));
+    }
+  }
+}
+
+// Same (128 x the sum) for one token whose eight code chunks of the segment are held in registers.
+__device__ __forceinline__ int bits_dot_regs(uint4 w, const uint4 (&q)[8]) {
+  const uint32_t w4[4] = {w.x, w.y, w.z, w.w};
+  int acc8[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) acc8[k] = 0;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const uint4 qa = q[2 * j], qb = q[2 * j + 1];
+    const uint32_t qp[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
+#pragma unroll
+    for (int k = 0; k < 8; ++k) acc8[k] = dp4a_us(w4[j] & (0x01010101u << k), qp[k], acc8[k]);
+  }
+  int S = 0;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) S += acc8[k] * (1 << (7 - k));
+  return S;
+}
+
+// LPR lanes per row, NSEG 16-byte segments per lane (d_in = 128 LPR NSEG >= 1024), BT token slots.
+// Warps 0..15 quantize x, compute the LoRA-down at each linear and accumulate the scaffold rows of every
+// stage into the accumulator ring; warps 16..21 turn accumulators into outputs (fp64 epilogue); warp 22
+// streams the stages.
+template <int LPR, int NSEG, int BT>
+__global__ void __launch_bounds__(NT, 1) stream_kernel(const __grid_constant__ Params p) {
+  constexpr int SEGS = LPR * NSEG;
+  constexpr int DIN = 128 * SEGS;
+  constexpr int ROW16 = DIN / 128;             // 16-byte chunks of packed bits per row
+  constexpr int RPW = 32 / LPR;                // rows per warp per pass
+  constexpr int RPP = NCW * RPW;               // rows per pass
+  constexpr int TR = TILE_BYTES / (DIN / 8);   // rows per tile
+  constexpr int PASSES = TR / RPP;
+  static_assert(PASSES >= 1 && PASSES * RPP == TR && TR <= MAX_TR, "tile shape");
+  static_assert(LPR >= BT, "one lane per token in a row group");
+  constexpr bool WB_SMEM = wb_in_smem(DIN, BT);
+  constexpr int NS = n_stages(DIN, BT);
+  constexpr int XPT = DIN / (NCW * 32);                    // x values per GEMV thread per token
+  constexpr bool XREG = BT * XPT <= 16;                    // keep x in registers between the two passes
+  constexpr bool REGQ = BT == 1 && NSEG == 1;              // one token: the lane's codes live in registers
+
+  extern __shared__ __align__(128) unsigned char smem[];
+  unsigned char* pring = smem + (size_t)NS * TILE_BYTES;                            // [NS][P_BYTES]
+  int8_t* wb_sm = reinterpret_cast<int8_t*>(pring + (size_t)NS * P_BYTES);          // [R][DIN] if WB_SMEM
+  int8_t* q_perm = wb_sm + (WB_SMEM ? R * DIN : 0);                                 // [BT][DIN]
+  int8_t* q_nat = q_perm + BT * DIN;                                                // [BT][DIN]
+  __shared__ Lin lin_sm[MAX_LIN];
+  __shared__ uint64_t bfull[MAX_NS], bempty[MAX_NS], pfull[MAX_NS], pacc[MAX_NS], pempty[MAX_NS], wb_full,
+      wb_empty;
+  __shared__ float s_tok[MAX_B];
+  __shared__ double s_tokd[MAX_B];
+  __shared__ double tf_cur[MAX_B][R];
+  __shared__ int t_sm[MAX_B][R];
+  __shared__ float red_f[NCW][MAX_B];
+  __shared__ int red_i[NCW][MAX_B];
+  __shared__ volatile int abort_flag;
+  __shared__ int wb_ok;
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int G = gridDim.x, c = blockIdx.x;
+  const int k0 = (int)((long long)c * p.total_tiles / G);
+  const int k1 = (int)((long long)(c + 1) * p.total_tiles / G);
+  const int ntiles = k1 - k0;
+  const int B = p.B;
+
+  if (tid < p.n_lin) {
+    Lin L = p.lin[tid];
+    const auto al16 = [](const void* q) { return (reinterpret_cast<uintptr_t>(q) & 15) == 0; };
+    L.ptma = L.rank == R && al16(L.lora_a) && al16(L.w_scale) && al16(L.lora_a_scale);
+    lin_sm[tid] = L;
+  }
+  if (tid == 0) {
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(&bfull[s], 1);
+      mbar_init(&bempty[s], NCW);
+      mbar_init(&pfull[s], 1);
+      mbar_init(&pacc[s], NCW);
+      mbar_init(&pempty[s], 1);
+    }
+    mbar_init(&wb_full, 1);
+    mbar_init(&wb_empty, 1);
+    abort_flag = 0;
+    int ok = WB_SMEM ? 1 : 0;
+    for (int j = 0; j < p.n_lin; ++j)
+      if (p.lin[j].rank > 0 && (reinterpret_cast<uintptr_t>(p.lin[j].lora_b) & 15)) ok = 0;
+    wb_ok = ok;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+  pdl_launch_dependents();
+  const bool use_wb = wb_ok != 0;
+  if (ntiles <= 0) return;
+
+  // ------------------------------------------------------------------ producer warp
+  // lane l < NS owns stage l of both rings and issues tiles l, l + NS, ... of the range (one warp
+  // instruction issues the copies of several stages); lane 31 streams the linears' W_B; the remaining
+  // lanes warm L2 with the parameters that do not travel by bulk copy.
+  if (warp == PROD_WARP) {
+    if (lane < NS) {
+      const int sl = lane;
+      Cursor cu;
+      cu.start(lin_sm, p.n_lin, min(k0 + sl, k1 - 1));
+      int i = sl;
+      bool ok = true;
+      for (; i < ntiles; i += NS) {
+        if (i > sl)
+          for (int q = 0; q < NS; ++q) cu.next(lin_sm);
+        const Lin& L = lin_sm[cu.j];
+        const uint32_t par = ((i / NS) & 1) ^ 1;
+        if ((i >= NS && (!mbar_wait_or_abort(&bempty[sl], par, &abort_flag) ||
+                         !mbar_wait_or_abort(&pempty[sl], par, &abort_flag))) || abort_flag) {
+          ok = false;
+          break;
+        }
+        const int r0 = cu.t * TR, nr = min(TR, L.d_out - r0), n4 = nr & ~3;
+        const uint32_t bits_bytes = (uint32_t)nr * (DIN / 8);
+        mbar_expect_tx(&bfull[sl], bits_bytes);
+        bulk_g2s(smem + (size_t)sl * TILE_BYTES, L.bits + (size_t)r0 * (DIN / 32), bits_bytes, &bfull[sl]);
+        unsigned char* ps = pring + (size_t)sl * P_BYTES;
+        mbar_expect_tx(&pfull[sl], L.ptma ? (uint32_t)(nr * 16 + 2 * n4 * 4) : 0u);
+        if (L.ptma) {
+          bulk_g2s(ps + P_WA, L.lora_a + (size_t)r0 * R, (uint32_t)(nr * 16), &pfull[sl]);
+          if (n4 > 0) {
+            bulk_g2s(ps + P_SW, L.w_scale + r0, (uint32_t)(n4 * 4), &pfull[sl]);
+            bulk_g2s(ps + P_SA, L.lora_a_scale + r0, (uint32_t)(n4 * 4), &pfull[sl]);
+          }
+        }
+      }
+      if (!ok) {
+        // stop: record the failure and wait (bounded) for this stage's copies still in flight
+        atomicExch(p.status, kTimeoutCode);
+        abort_flag = 1;
+        if (i - NS >= 0) {
+          mbar_wait(&bfull[sl], ((i - NS) / NS) & 1);
+          mbar_wait(&pfull[sl], ((i - NS) / NS) & 1);
+        }
+      }
+    } else if (lane == 31) {
+      if (!use_wb) return;
+      // W_B of each linear of the range that has a LoRA, in order; the GEMV warps release the buffer
+      // after computing t of the previous one
+      Cursor a, b;
+      a.start(lin_sm, p.n_lin, k0);
+      b.start(lin_sm, p.n_lin, k1 - 1);
+      int m = 0;
+      bool ok = true;
+      for (int j = a.j; j <= b.j; ++j) {
+        const Lin& L = lin_sm[j];
+        if (L.rank == 0) continue;
+        if ((m > 0 && !mbar_wait_or_abort(&wb_empty, (m - 1) & 1, &abort_flag)) || abort_flag) {
+          ok = false;
+          break;
+        }
+        mbar_expect_tx(&wb_full, (uint32_t)(L.rank * DIN));
+        bulk_g2s(wb_sm, L.lora_b, (uint32_t)(L.rank * DIN), &wb_full);
+        ++m;
+      }
+      if (!ok) {
+        atomicExch(p.status, kTimeoutCode);
+        abort_flag = 1;
+        if (m > 0) mbar_wait(&wb_full, (m - 1) & 1);
+      }
+    } else {
+      Cursor a, b;
+      a.start(lin_sm, p.n_lin, k0);
+      b.start(lin_sm, p.n_lin, k1 - 1);
+      const int idx = lane - NS, nl = 31 - NS;
+      for (int j = a.j; j <= b.j; ++j) {
+        const Lin& L = lin_sm[j];
+        const int ra = j == a.j ? a.t * TR : 0;
+        const int rb = j == b.j ? min(L.d_out, (b.t + 1) * TR) : L.d_out;
+        if (L.rank > 0) prefetch_range(L.lora_b_scale, (size_t)L.rank * 4, idx, nl);
+        if (!use_wb && L.rank > 0) prefetch_range(L.lora_b, (size_t)L.rank * DIN, idx, nl);
+        if (rb > ra && !L.ptma) {
+          prefetch_range(L.w_scale + ra, (size_t)(rb - ra) * 4, idx, nl);
+          if (L.rank > 0) {
+            prefetch_range(L.lora_a_scale + ra, (size_t)(rb - ra) * 4, idx, nl);
+            prefetch_range(L.lora_a + (size_t)ra * L.rank, (size_t)(rb - ra) * L.rank, idx, nl);
+          }
+        }
+      }
+    }
+    return;
+  }
+
+  // ------------------------------------------------------------------ epilogue warps
+  // epilogue warp e takes the tiles i = e, e + NEW, ... of the range, whole, so several tiles' fp64
+  // epilogues are in flight at once
+  if (warp >= NCW) {
+    pdl_wait();  // the outputs may still be read or written by the preceding kernel of the stream
+    const int e = warp - NCW;
+    Cursor cu;
+    cu.start(lin_sm, p.n_lin, k0);
+    bool dead = false;
+    for (int i = 0; i < ntiles; ++i, cu.next(lin_sm)) {
+      if (i % NEW != e) continue;
+      const Lin& L = lin_sm[cu.j];
+      const int sp = i % NS;
+      const uint32_t par = (i / NS) & 1;
+      if (!dead && (!mbar_wait_or_abort(&pacc[sp], par, &abort_flag) ||
+                    !mbar_wait_or_abort(&pfull[sp], par, &abort_flag))) {
+        dead = true;
+        atomicExch(p.status, kTimeoutCode);
+        abort_flag = 1;
+      }
+      if (!dead) {
+        const int r0 = cu.t * TR, nr = min(TR, L.d_out - r0), n4 = nr & ~3;
+        const unsigned char* ps = pring + (size_t)sp * P_BYTES;
+        const uint4* wa_st = reinterpret_cast<const uint4*>(ps + P_WA);
+        const float* sw_st = reinterpret_cast<const float*>(ps + P_SW);
+        const float* sa_st = reinterpret_cast<const float*>(ps + P_SA);
+        const int* acc = reinterpret_cast<const int*>(ps + P_ACC);
+        const double* tf = reinterpret_cast<const double*>(ps + P_TF);
+        // two (row, token) jobs per lane per step, their fp64 chains interleaved
+        const auto fetch = [&](int job, int& a, double& sw, double& sa, uint4& wa, int& row, int& b) {
+          const int rr = job / B;
+          b = job - rr * B;
+          row = r0 + rr;
+          float fw, fa = 0.0f;
+          wa = make_uint4(0u, 0u, 0u, 0u);
+          if (L.ptma) {
+            wa = wa_st[rr];
+            if (rr < n4) {
+              fw = sw_st[rr];
+              fa = sa_st[rr];
+            } else {
+              fw = __ldg(L.w_scale + row);
+              fa = __ldg(L.lora_a_scale + row);
+            }
+          } else {
+            fw = __ldg(L.w_scale + row);
+            if (L.rank > 0) {
+              fa = __ldg(L.lora_a_scale + row);
+              wa = load_wa(L, row);
+            }
+          }
+          sw = (double)fw;
+          sa = (double)fa;
+          a = acc[rr * MAX_B + b];
+        };
+        for (int job = lane; job < nr * B; job += 64) {
+          int a[2], row[2], b[2];
+          double sd[2], sw[2], sa[2];
+          uint4 wa[2];
+          const bool two = job + 32 < nr * B;
+          fetch(job, a[0], sw[0], sa[0], wa[0], row[0], b[0]);
+          fetch(two ? job + 32 : job, a[1], sw[1], sa[1], wa[1], row[1], b[1]);
+          sd[0] = s_tokd[b[0]];
+          sd[1] = s_tokd[b[1]];
+          const double* const t2[2] = {tf + b[0] * R, tf + b[1] * R};
+          float out[2];
+          if (L.rank == R) linear_out_n<2, R>(a, sd, sw, sa, wa, t2, R, out);
+          else linear_out_n<2, -1>(a, sd, sw, sa, wa, t2, L.rank, out);
+#pragma unroll
+          for (int n = 0; n < 2; ++n) {
+            if (n == 0 || two) {
+              L.y[(size_t)b[n] * L.d_out + row[n]] = out[n];
+              if (p.dbg_acc) p.dbg_acc[(size_t)b[n] * L.d_out + row[n]] = a[n];
+            }
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&pempty[sp]);
+    }
+    return;
+  }
+
+  // ------------------------------------------------------------------ GEMV warps
+  pdl_wait();  // x may come from the preceding kernel of the stream
+  int sumq[BT];
+  {
+    float xr[XREG ? BT * XPT : 1];
+#pragma unroll
+    for (int b = 0; b < BT; ++b) {
+      float m = 0.0f;
+#pragma unroll
+      for (int k = 0; k < XPT; ++k) {
+        const int i = tid + k * NCW * 32;
+        const float v = b < B ? p.x[(size_t)b * DIN + i] : 0.0f;
+        if (XREG) xr[b * XPT + k] = v;
+        m = fmaxf(m, fabsf(v));
+      }
+      m = warp_max(m);
+      if (lane == 0) red_f[warp][b] = m;
+    }
+    consumer_sync();
+#pragma unroll
+    for (int b = 0; b < BT; ++b) {
+      float m = 0.0f;
+#pragma unroll
+      for (int w = 0; w < NCW; ++w) m = fmaxf(m, red_f[w][b]);
+      const float s0 = m == 0.0f ? 0.0f : __fdiv_rn(m, 127.0f);
+      const float inv_s0 = m == 0.0f ? 0.0f : __frcp_rn(s0);
+      int sq = 0;
+      if (b < B) {
+#pragma unroll
+        for (int k = 0; k < XPT; ++k) {
+          const int i = tid + k * NCW * 32;
+          const float v = XREG ? xr[b * XPT + k] : p.x[(size_t)b * DIN + i];
+          const int code = m == 0.0f ? 0 : quant_code_fast(v, s0, inv_s0);
+          q_perm[b * DIN + seg_index<SEGS>(i)] = (int8_t)code;
+          q_nat[b * DIN + i] = (int8_t)code;
+          sq += code;
+          if (p.dbg_xq && c == 0) p.dbg_xq[(size_t)b * DIN + i] = (int8_t)code;
+        }
+      }
+      sq = warp_sum(sq);
+      if (lane == 0) red_i[warp][b] = sq;
+      if (tid == b && b < B) {
+        s_tok[b] = s0;
+        s_tokd[b] = (double)s0;
+        if (p.dbg_s && c == 0) p.dbg_s[b] = s0;
+      }
+    }
+    consumer_sync();
+#pragma unroll
+    for (int b = 0; b < BT; ++b) {
+      int sq = 0;
+#pragma unroll
+      for (int w = 0; w < NCW; ++w) sq += red_i[w][b];
+      sumq[b] = sq;
+    }
+  }
+
+  const int li = lane % LPR, rsub = lane / LPR;
+  uint4 qreg[REGQ ? 8 : 1];
+  if (REGQ) {
+    const uint4* q0 = reinterpret_cast<const uint4*>(q_perm) + li;
+#pragma unroll
+    for (int v = 0; v < 8; ++v) qreg[v] = q0[v * SEGS];
+  }
+  Cursor cu;
+  cu.start(lin_sm, p.n_lin, k0);
+  int cur_j = -1, m_wb = 0;
+  bool dead = false;
+  for (int i = 0; i < ntiles; ++i, cu.next(lin_sm)) {
+    const Lin& L = lin_sm[cu.j];
+    if (cu.j != cur_j) {
+      // LoRA down-projection of this linear for every token: warp r computes t[.][r]
+      const float sB = (tid < BT * R && tid % R < L.rank) ? __ldg(L.lora_b_scale + tid % R) : 0.0f;
+      if (L.rank > 0 && use_wb && !dead && !mbar_wait_or_abort(&wb_full, m_wb & 1, &abort_flag)) {
+        dead = true;
+        atomicExch(p.status, kTimeoutCode);
+        abort_flag = 1;
+      }
+      consumer_sync();
+      if (!dead) {
+        for (int r = warp; r < L.rank; r += NCW) {
+          int part[BT];
+#pragma unroll
+          for (int b = 0; b < BT; ++b) part[b] = 0;
+          if (use_wb) {
+            const uint4* w4 = reinterpret_cast<const uint4*>(wb_sm + r * DIN);
+#pragma unroll
+            for (int ch = lane; ch < DIN / 16; ch += 32) {
+              const uint4 w = w4[ch];
+#pragma unroll
+              for (int b = 0; b < BT; ++b) {
+                if (b < B) {
+                  const uint4 q = reinterpret_cast<const uint4*>(q_nat + b * DIN)[ch];
+                  part[b] = dp4a_ss(w.x, q.x, part[b]);
+                  part[b] = dp4a_ss(w.y, q.y, part[b]);
+                  part[b] = dp4a_ss(w.z, q.z, part[b]);
+                  part[b] = dp4a_ss(w.w, q.w, part[b]);
+                }
+              }
+            }
+          } else {
+            const uint32_t* wb = reinterpret_cast<const uint32_t*>(L.lora_b + (size_t)r * DIN);
+#pragma unroll 8
+            for (int w = lane; w < DIN / 4; w += 32) {
+              const uint32_t wv = __ldg(wb + w);
+#pragma unroll
+              for (int b = 0; b < BT; ++b)
+                if (b < B) part[b] = dp4a_ss(wv, reinterpret_cast<const uint32_t*>(q_nat + b * DIN)[w], part[b]);
+            }
+          }
+#pragma unroll
+          for (int b = 0; b < BT; ++b) {
+            part[b] = __reduce_add_sync(0xffffffffu, part[b]);
+            if (lane == 0 && b < B) t_sm[b][r] = part[b];
+          }
+        }
+      }
+      consumer_sync();
+      if (L.rank > 0 && use_wb) {
+        if (tid == 0) mbar_arrive(&wb_empty);  // W_B buffer free for the next linear
+        ++m_wb;
+      }
+      if (tid < BT * R) {
+        const int b = tid / R, r = tid % R;
+        float tf = 0.0f;
+        if (b < B && r < L.rank) {
+          tf = lora_tf(t_sm[b][r], sB, s_tok[b]);
+          if (p.dbg_t && c == 0) p.dbg_t[b * L.rank + r] = t_sm[b][r];
+        }
+        tf_cur[b][r] = (double)tf;
+      }
+      consumer_sync();
+      cur_j = cu.j;
+    }
+    const int sb = i % NS, sp = sb;
+    if (!dead && !mbar_wait_or_abort(&bfull[sb], (i / NS) & 1, &abort_flag)) {
+      dead = true;
+      atomicExch(p.status, kTimeoutCode);
+      abort_flag = 1;
+    }
+    if (!dead) {
+      const uint4* tile = reinterpret_cast<const uint4*>(smem + (size_t)sb * TILE_BYTES);
+      int* acc = reinterpret_cast<int*>(pring + (size_t)sp * P_BYTES + P_ACC);
+      const int nr = min(TR, L.d_out - cu.t * TR);
+#pragma unroll
+      for (int ps = 0; ps < PASSES; ++ps) {
+        const int rr = ps * RPP + warp * RPW + rsub;
+        const bool valid = rr < nr;
+        int S[BT];
+#pragma unroll
+        for (int b = 0; b < BT; ++b) S[b] = 0;
+#pragma unroll
+        for (int sg = 0; sg < NSEG; ++sg) {
+          const int seg = sg * LPR + li;
+          const uint4 w = valid ? tile[rr * ROW16 + seg] : make_uint4(0u, 0u, 0u, 0u);
+          if constexpr (REGQ) S[0] += bits_dot_regs(w, qreg);
+          else bits_dot_tokens<SEGS, BT>(w, reinterpret_cast<const uint4*>(q_perm) + seg, B, S);
+        }
+#pragma unroll
+        for (int b = 0; b < BT; ++b) {
+#pragma unroll
+          for (int o = LPR / 2; o > 0; o >>= 1) S[b] += __shfl_xor_sync(0xffffffffu, S[b], o);
+        }
+        // lane b of the row group stores token b's accumulator
+#pragma unroll
+        for (int b = 0; b < BT; ++b)
+          if (valid && b < B && li == b) acc[rr * MAX_B + b] = (S[b] >> 6) - sumq[b];  // 2 sum - sum q
+      }
+      if (tid < BT * R)
+        reinterpret_cast<double*>(pring + (size_t)sp * P_BYTES + P_TF)[tid] = tf_cur[tid / R][tid % R];
+    }
+    __syncwarp();
+    if (lane == 0) {
+      mbar_arrive(&bempty[sb]);  // the bits stage may be refilled
+      mbar_arrive(&pacc[sp]);    // accumulators and tf of this tile are ready
+    }
+  }
+}
+
+// Module status word: kTimeoutCode after a wait ran out of budget (sticky until read).
+static __device__ int g_stream_status;
+
+template <int LPR, int NSEG, int BT>
+cudaError_t launch_t(const Params& p, int grid, cudaStream_t st) {
+  constexpr int DIN = 128 * LPR * NSEG;
+  constexpr size_t smem = smem_bytes(DIN, BT);
+  auto k = stream_kernel<LPR, NSEG, BT>;
+  // once per instantiation, not per launch, so that launches can be captured in a CUDA graph
+  static const cudaError_t set = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (set != cudaSuccess) return set;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(NT);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, k, p);
+}
+
+template <int BT>
+cudaError_t dispatch(const Params& p, int grid, cudaStream_t st) {
+  switch (p.d_in / 128) {
+    case 8: return launch_t<8, 1, BT>(p, grid, st);
+    case 16: return launch_t<16, 1, BT>(p, grid, st);
+    case 32: return launch_t<32, 1, BT>(p, grid, st);
+    case 64: return launch_t<32, 2, BT>(p, grid, st);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace stream
+
+bool stream_supported(int d_in, int B) {
+  return B >= 1 && B <= stream::MAX_B && (d_in == 1024 || d_in == 2048 || d_in == 4096 || d_in == 8192);
+}
+
+int stream_status_word(int** out) {
+  static std::mutex mu;
+  static int* addr[64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return record_cuda_failure(e);
+  if (dev < 0 || dev >= 64) return DFSSM_EUNSUPPORTED;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
+    void* a = nullptr;
+    e = cudaGetSymbolAddress(&a, stream::g_stream_status);
+    if (e != cudaSuccess) return record_cuda_failure(e);
+    addr[dev] = static_cast<int*>(a);
+  }
+  *out = addr[dev];
+  return DFSSM_OK;
+}
+
+int launch_linear_stream(const dfssm_linear_t* lins, int n, const float* x, int B, float* const* ys,
+                         const dfssm_debug_t* dbg, cudaStream_t st) {
+  stream::Params p;
+  const int d_in = lins[0].d_in;
+  const int tile_rows = stream::TILE_BYTES / (d_in / 8);
+  int tiles = 0;
+  for (int j = 0; j < n; ++j) {
+    const dfssm_linear_t& L = lins[j];
+    stream::Lin& q = p.lin[j];
+    q.bits = L.bits;
+    q.w_scale = L.w_scale;
+    q.lora_b = L.lora_b;
+    q.lora_b_scale = L.lora_b_scale;
+    q.lora_a = L.lora_a;
+    q.lora_a_scale = L.lora_a_scale;
+    q.y = ys[j];
+    q.d_out = L.d_out;
+    q.rank = L.rank;
+    q.tile0 = tiles;
+    q.ntiles = (L.d_out + tile_rows - 1) / tile_rows;
+    tiles += q.ntiles;
+  }
+  p.n_lin = n;
+  p.d_in = d_in;
+  p.B = B;
+  p.x = x;
+  p.total_tiles = tiles;
+  p.tile_rows = tile_rows;
+  p.dbg_xq = dbg ? dbg->xq : nullptr;
+  p.dbg_s = dbg ? dbg->xscale : nullptr;
+  p.dbg_t = dbg ? dbg->lora_t : nullptr;
+  p.dbg_acc = dbg ? dbg->acc : nullptr;
+  int st_rc = stream_status_word(&p.status);
+  if (st_rc) return st_rc;
+  const int grid = tiles < num_sms() ? tiles : num_sms();
+  const cudaError_t e = B == 1 ? stream::dispatch<1>(p, grid, st) : stream::dispatch<4>(p, grid, st);
+  if (e != cudaSuccess) return record_cuda_failure(e);
+  return DFSSM_OK;
+}
+
+}  // namespace dfssm

@@ -66,6 +66,7 @@ SIGNATURES = {
     "dfssm_linear_decode": (_I, [_P, _P, _I, _P, _P, _Z, _P, _P]),
     "dfssm_linear_prefill": (_I, [_P, _P, _I, _P, _P, _Z, _P, _P]),
     "dfssm_linear_decode_noalloc": (_I, [_P, _P, _I, _P, _P, _P]),
+    "dfssm_linear_decode_multi": (_I, [_P, _I, _P, _I, _P, _P]),
     "dfssm_conv_step": (_I, [_P, _P, _P, _P, _P, _I, _I, _P]),
     "dfssm_ssm_step": (_I, [_P] * 9 + [_I] * 5 + [_P]),
     "dfssm_layer_decode": (_I, [_P, _I, _P, _P, _P, _P, _I, _P, _Z, _P]),
@@ -184,6 +185,18 @@ def linear_decode_noalloc(lin: Linear, x: torch.Tensor, y: torch.Tensor | None =
     return y
 
 
+def linear_decode_multi(lins, x: torch.Tensor, ys=None, stream=None):
+    """n linears that share x in one launch (dfssm_linear_decode_multi); returns the list of outputs."""
+    B = x.shape[0]
+    if ys is None:
+        ys = [torch.empty((B, L.d_out), dtype=torch.float32, device=x.device) for L in lins]
+    arr = (LinearT * len(lins))(*[L.cstruct() for L in lins])
+    ptrs = (C.c_void_p * len(lins))(*[_ptr(y) for y in ys])
+    _check("dfssm_linear_decode_multi", lib().dfssm_linear_decode_multi(
+        arr, len(lins), _ptr(x), B, ptrs, _stream(stream)))
+    return ys
+
+
 def linear_prefill(lin: Linear, x: torch.Tensor, y: torch.Tensor | None = None, ws=None,
                    debug: dict | None = None, stream=None) -> torch.Tensor:
     M = x.shape[0]
@@ -269,8 +282,9 @@ def layer_decode(stack: LayerStack, hidden: torch.Tensor, ws=None, stream=None) 
     return hidden
 
 
-def device_status(ws, stream=None) -> int:
-    """Synchronise the stream, read and clear the fused-decode error word: 0 (DFSSM_OK) or -5."""
+def device_status(ws=None, stream=None) -> int:
+    """Synchronise the stream, read and clear the device error words (the workspace's, if given, and
+    the library's own): 0 (DFSSM_OK) or -5 (DFSSM_ETIMEOUT)."""
     return int(lib().dfssm_device_status(_ptr(ws), _stream(stream)))
 
 

@@ -82,7 +82,8 @@ def _rand_linear(seed, d_out, d_in, rank):
 @pytest.mark.parametrize("d_out,d_in,rank,B", [
     (1, 32, 0, 1), (33, 64, 1, 2), (127, 96, 7, 3), (129, 160, 16, 5), (512, 256, 16, 16),
     (300, 384, 16, 4), (257, 1024, 16, 1), (1000, 8192, 16, 2), (8512, 2048, 16, 3),
-    (2048, 4096, 16, 16), (77, 512, 16, 1)])
+    (2048, 4096, 16, 16), (77, 512, 16, 1), (1, 128, 0, 1), (640, 256, 5, 4), (8512, 2048, 16, 1),
+    (2048, 4096, 16, 4), (1100, 1024, 1, 2)])
 def test_linear_shapes(dev, d_out, d_in, rank, B):
     lin = _rand_linear(d_out * 7 + d_in + rank + B, d_out, d_in, rank)
     gen = np.random.default_rng(B)
@@ -130,6 +131,61 @@ def test_linear_full_stacks(dev, which):
                     ry, racc = oracle.linear_rows(OL, rq[b], rs[b], rtf, rows)
                     assert np.array_equal(acc[b, rows], racc), (which, B, c, b)
                     assert assert_tol(y[b, rows], ry, f"{which} B{B} copy{c}") == 0
+
+
+@pytest.mark.parametrize("B", [1, 4])
+def test_linear_multi_matches_per_call(dev, B):
+    """dfssm_linear_decode_multi over the 48 in_proj copies equals 48 dfssm_linear_decode calls bit for
+    bit; copy 0 is checked in full and copy 47 on sampled rows against the oracle."""
+    from bit_quantized_mamba_b200 import dfssm
+    data = inputs.in_proj_stack()
+    lins = [dfssm.Linear.from_host(l, dev) for l in data["linears"]]
+    x = data["x"][:B]
+    xd = to_dev(x, dev)
+    ys = dfssm.linear_decode_multi(lins, xd)
+    ref = [dfssm.linear_decode(L, xd) for L in lins]
+    torch.cuda.synchronize()
+    for c in range(len(lins)):
+        assert torch.equal(ys[c], ref[c]), c
+    r = oracle.linear_decode(oracle.Linear.from_dict(data["linears"][0]), x)
+    assert assert_tol(ys[0].cpu().numpy(), r["y"], "multi copy 0") == 0
+    OL = oracle.Linear.from_dict(data["linears"][47])
+    rq, rs = oracle.quantize(x)
+    rows = np.arange(0, OL.d_out, 97)
+    y47 = ys[47].cpu().numpy()
+    for b in range(B):
+        _, rtf = oracle.lora_down(OL, rq[b], rs[b])
+        ry, _ = oracle.linear_rows(OL, rq[b], rs[b], rtf, rows)
+        assert assert_tol(y47[b, rows], ry, f"multi copy 47 token {b}") == 0
+
+
+def test_linear_multi_mixed_shapes(dev):
+    """Linears of different d_out (ragged tiles, rank 0 and rank < 16) sharing one input."""
+    from bit_quantized_mamba_b200 import dfssm
+    hosts = [_rand_linear(70 + j, d_out, 1024, rank) for j, (d_out, rank) in
+             enumerate([(1, 16), (4353, 16), (129, 0), (300, 3), (2048, 16)])]
+    lins = [dfssm.Linear.from_host(h, dev) for h in hosts]
+    gen = np.random.default_rng(3)
+    x = inputs.normal(gen, (3, 1024))
+    x[2] = 0.0
+    ys = dfssm.linear_decode_multi(lins, to_dev(x, dev))
+    torch.cuda.synchronize()
+    for j, h in enumerate(hosts):
+        r = oracle.linear_decode(oracle.Linear.from_dict(h), x)
+        assert assert_tol(ys[j].cpu().numpy(), r["y"], f"mixed linear {j}") == 0
+
+
+def test_linear_multi_rejects_unsupported(dev):
+    from bit_quantized_mamba_b200 import dfssm
+    g = np.random.default_rng(8)
+    lins = [dfssm.Linear.from_host(inputs.linear(g, 64, 384), dev)]
+    with pytest.raises(dfssm.DfssmError) as e:
+        dfssm.linear_decode_multi(lins, torch.zeros((1, 384), device=dev))
+    assert e.value.status == -3  # d_in outside {1024, 2048, 4096, 8192}
+    lins = [dfssm.Linear.from_host(inputs.linear(g, 64, 256), dev)]
+    with pytest.raises(dfssm.DfssmError) as e:
+        dfssm.linear_decode_multi(lins, torch.zeros((5, 256), device=dev))
+    assert e.value.status == -3  # B > 4
 
 
 def test_conv_step(dev):
