@@ -295,7 +295,7 @@ int dfssm_layer_decode(const dfssm_layer_t* layers, int n_layers, const dfssm_di
     return DFSSM_EWORKSPACE;
   if (!device_ok()) return DFSSM_EDEVICE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (dfssm::fused_decode_supported(*dims, B, layers, n_layers)) {
+  if (dfssm::fused_decode_supported(*dims, B, layers, n_layers, conv_states)) {
     const cudaError_t fe = dfssm::launch_fused_decode(layers, n_layers, hidden, conv_states, ssm_states,
                                                       workspace, s, kSpinLimitCycles);
     return fe == cudaSuccess ? DFSSM_OK : cuda_fail(fe);

@@ -152,7 +152,8 @@ __device__ __forceinline__ void prefetch_lines(const void* p, unsigned bytes) {
   for (; a < e; a += 128) asm volatile("prefetch.global.L2 [%0];" ::"l"(a) : "memory");
 }
 
-// Asynchronous global -> shared copies (completion awaited with cp_async_wait_all before a barrier).
+// Asynchronous global -> shared copies, committed in groups; a thread waits for its own groups
+// (cp_async_wait<N>: all but the N most recent are complete), and a CTA barrier then publishes them.
 __device__ __forceinline__ void cp_async4(void* dst, const void* src) {
   const unsigned d = (unsigned)__cvta_generic_to_shared(dst);
   asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(d), "l"(src) : "memory");
@@ -161,8 +162,46 @@ __device__ __forceinline__ void cp_async16(void* dst, const void* src) {
   const unsigned d = (unsigned)__cvta_generic_to_shared(dst);
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(src) : "memory");
 }
-__device__ __forceinline__ void cp_async_wait_all() {
-  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// Bulk asynchronous copies (one instruction per contiguous range) with mbarrier completion.
+__device__ __forceinline__ uint32_t smem_u32(const void* q) { return (uint32_t)__cvta_generic_to_shared(q); }
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred q;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 q, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait for the phase with the given parity; false when the clock budget ran out.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, long long limit) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity))
+    if (clock64() - t0 > limit) return false;
+  return true;
+}
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
 }
 
 // LoRA down-projection row r = warp: t[r] = sum_i W_B[r,i] q_i over NCH 16-byte chunks, lane taking
@@ -196,6 +235,8 @@ __device__ __forceinline__ int lora_row(const int8_t* wb_row, const int8_t* qn, 
 
 __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ Params p) {
   extern __shared__ __align__(16) int8_t wb_sm[];  // W_B of in_proj [R][DM], then of out_proj [R][E]
+  // every layer's pointers, copied once: the layer loop never indexes the parameter block at run time
+  __shared__ LayerPtrs lsm[DFSSM_MAX_LAYERS];
   int8_t* const wb_in = wb_sm;
   int8_t* const wb_out = wb_sm + R * DM;
   __shared__ __align__(16) int8_t q_perm[E];
@@ -212,11 +253,14 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ P
   __shared__ float in_sw[MAX_IN], in_sa[MAX_IN];
   __shared__ __align__(16) int8_t in_wa[MAX_IN][R];
   // the 320 rows every CTA needs
-  __shared__ float sh_sw[NSH], sh_sa[NSH];
+  __shared__ __align__(16) float sh_sw[NSH];
+  __shared__ __align__(16) float sh_sa[NSH];
   __shared__ __align__(16) int8_t sh_wa[NSH][R];
   __shared__ __align__(16) float4 bc_w[2 * N];
-  __shared__ float bc_b[2 * N];
-  __shared__ float bc_st[2 * N][3];
+  __shared__ __align__(16) float bc_b[2 * N];
+  __shared__ __align__(16) float bc_st[2 * N][3];
+  // bulk-copy completion: [0] the rows every CTA needs + in_proj W_B, [1] out_proj W_B (once per layer)
+  __shared__ uint64_t ldbar[2];
   __shared__ float bc_new[2 * N];
   __shared__ __align__(16) float Bsm[N];
   __shared__ __align__(16) double Cd[N];
@@ -250,15 +294,29 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ P
   const int dt_head = tid - 2 * N;  // threads [256, 320) own the dt rows
   const bool dt_own = tid >= 2 * N && tid < NSH && (dt_head == hA || dt_head == hA + 1);
 
+  {
+    // LayerPtrs is 21 pointers: thread t copies pointer t % 21 of layer t / 21
+    constexpr int NPTR = sizeof(LayerPtrs) / sizeof(void*);
+    static_assert(sizeof(LayerPtrs) == NPTR * sizeof(void*), "LayerPtrs holds pointers only");
+    const void* const* src = reinterpret_cast<const void* const*>(p.L);
+    const void** dst = reinterpret_cast<const void**>(lsm);
+    for (int k = tid; k < p.n_layers * NPTR; k += NT) dst[k] = src[k];
+    if (tid == 0) {
+      mbar_init(&ldbar[0], 1);
+      mbar_init(&ldbar[1], 1);
+      asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+  }
   for (int l = 0; l < p.n_layers; ++l) {
-    const LayerPtrs& Lp = p.L[l];
+    const LayerPtrs& Lp = lsm[l];
     const bool has_next = l + 1 < p.n_layers;
 
     // ---------------------------------------------------------------- loads for the whole layer
     if ((tid == kPrefetchThread || tid == kPrefetchThread + 1) && has_next) {
       // this CTA's slice of the next layer, and (spread over CTAs 0..4) the parts every CTA reads.
       // Issued by warp 1: a bulk prefetch stalls its thread, and thread 0 polls the counters.
-      const LayerPtrs& Nx = p.L[l + 1];
+      const LayerPtrs& Nx = lsm[l + 1];
       if (tid == kPrefetchThread) {
         prefetch_l2(Nx.in_bits + (size_t)(SH0 + sh0) * (DM / 32), n_sh * (DM / 8));
         prefetch_l2(Nx.in_bits + (size_t)rs0 * (DM / 32), n_ssm * (DM / 8));
@@ -354,19 +412,20 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ P
       cp_async4(&in_sa[tid], Lp.in_las + row);
       cp_async16(in_wa[tid], Lp.in_la + (size_t)row * R);
     }
-    if (tid < NSH) {
-      const int row = SH0 + tid;
-      cp_async4(&sh_sw[tid], Lp.in_ws + row);
-      cp_async4(&sh_sa[tid], Lp.in_las + row);
-      cp_async16(sh_wa[tid], Lp.in_la + (size_t)row * R);
-    }
-    if (tid < 2 * N) {
-      const int ch = E + tid;
-      cp_async16(&bc_w[tid], Lp.conv_w + (size_t)ch * 4);
-      cp_async4(&bc_b[tid], Lp.conv_b + ch);
-      cp_async4(&bc_st[tid][0], Lp.conv_state + (size_t)ch * 3 + 0);
-      cp_async4(&bc_st[tid][1], Lp.conv_state + (size_t)ch * 3 + 1);
-      cp_async4(&bc_st[tid][2], Lp.conv_state + (size_t)ch * 3 + 2);
+    if (tid == 0) {
+      // the contiguous ranges every CTA needs, one bulk copy each; every generic access of the previous
+      // layer to these buffers is ordered before them by the barrier that ended that layer
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      mbar_expect_tx(&ldbar[0], NSH * 4 * 2 + NSH * R + 2 * N * (16 + 4 + 12) + R * DM);
+      bulk_g2s(sh_sw, Lp.in_ws + SH0, NSH * 4, &ldbar[0]);
+      bulk_g2s(sh_sa, Lp.in_las + SH0, NSH * 4, &ldbar[0]);
+      bulk_g2s(sh_wa, Lp.in_la + (size_t)SH0 * R, NSH * R, &ldbar[0]);
+      bulk_g2s(bc_w, Lp.conv_w + (size_t)E * 4, 2 * N * 16, &ldbar[0]);
+      bulk_g2s(bc_b, Lp.conv_b + E, 2 * N * 4, &ldbar[0]);
+      bulk_g2s(bc_st, Lp.conv_state + (size_t)E * 3, 2 * N * 12, &ldbar[0]);
+      bulk_g2s(wb_in, Lp.in_lb, R * DM, &ldbar[0]);
+      mbar_expect_tx(&ldbar[1], R * E);
+      bulk_g2s(wb_out, Lp.out_lb, R * E, &ldbar[1]);
     }
     if (tid < n_out) {
       const int row = ro0 + tid;
@@ -375,14 +434,22 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ P
       cp_async16(o_wa[tid], Lp.out_la + (size_t)row * R);
     }
     if (tid < 2 && hA + tid < H) cp_async4(&Dv[tid], Lp.D + hA + tid);
-    // W_B of both linears (every CTA computes t = W_B q itself)
-    for (int k = tid; k < R * DM / 16; k += NT) cp_async16(wb_in + 16 * k, Lp.in_lb + 16 * (size_t)k);
-    for (int k = tid; k < R * E / 16; k += NT) cp_async16(wb_out + 16 * k, Lp.out_lb + 16 * (size_t)k);
-    cp_async_wait_all();
+    cp_async_commit();  // this thread's row parameters (awaited after the h wait)
 
     // ---------------------------------------------------------------- phase A: h -> in_proj
-    if (l > 0 && !block_wait(p.ctr + CTR_H * CTR_STRIDE, NC * l, p.err, p.status, p.spin_limit, &sflag))
+    if (l > 0 && !block_wait(p.ctr + CTR_H * CTR_STRIDE, NC * l, p.err, p.status, p.spin_limit, &sflag)) {
+      cp_async_wait<0>();  // nothing of this CTA may still be landing in its shared memory
+      mbar_wait(&ldbar[0], l & 1, p.spin_limit);
+      mbar_wait(&ldbar[1], l & 1, p.spin_limit);
       return;
+    }
+    cp_async_wait<0>();  // this thread's row parameters; the quantizer's barriers publish them
+    if (!mbar_wait(&ldbar[0], l & 1, p.spin_limit)) {  // shared rows and in_proj W_B
+      atomicExch(p.err, 1);
+      atomicExch(p.status, kTimeoutMagic);
+      mbar_wait(&ldbar[1], l & 1, p.spin_limit);
+      return;
+    }
     double ssA;
     float s0A;
     {
@@ -456,8 +523,11 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ P
     if (tid >= kChainBase && tid < kChainBase + R) tf[tid - kChainBase] = lora_tf(t_sm[tid - kChainBase], lbs_in, s_scale);
 
     // ---------------------------------------------------------------- phase B: epilogues + SSM
-    if (!block_wait(p.ctr + CTR_BC * CTR_STRIDE, NC * (l + 1), p.err, p.status, p.spin_limit, &sflag))
+    if (!block_wait(p.ctr + CTR_BC * CTR_STRIDE, NC * (l + 1), p.err, p.status, p.spin_limit, &sflag)) {
+      cp_async_wait<0>();  // nothing of this CTA may still be landing in its shared memory
+      mbar_wait(&ldbar[1], l & 1, p.spin_limit);
       return;
+    }
     const float s_in = s_scale;
     if (tid < NSH) {
       // rows every CTA needs: B, C (conv + SiLU) and dt of this CTA's heads
@@ -523,8 +593,16 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ P
       if (ssm_slot[ps] < n_ssm) st_f4(Lp.ssm_state + (size_t)(rs0 + ssm_slot[ps]) * N + lane * 4, snew[ps]);
 
     // ---------------------------------------------------------------- phase C: gated norm -> out_proj
-    if (!block_wait(p.ctr + CTR_G * CTR_STRIDE, NC * (l + 1), p.err, p.status, p.spin_limit, &sflag))
+    if (!block_wait(p.ctr + CTR_G * CTR_STRIDE, NC * (l + 1), p.err, p.status, p.spin_limit, &sflag)) {
+      cp_async_wait<0>();  // nothing of this CTA may still be landing in its shared memory
+      mbar_wait(&ldbar[1], l & 1, p.spin_limit);
       return;
+    }
+    if (!mbar_wait(&ldbar[1], l & 1, p.spin_limit)) {  // out_proj W_B
+      atomicExch(p.err, 1);
+      atomicExch(p.status, kTimeoutMagic);
+      return;
+    }
     // every CTA has now read the old B/C conv state: the owners of those rows shift it
     for (int j = tid; j < n_sh; j += NT) {
       const int k = sh0 + j;
@@ -611,12 +689,21 @@ __global__ void timeout_selftest_kernel(int* ctr, int* err, int* status, long lo
 
 size_t fused_decode_workspace_bytes() { return fused::WS_BYTES; }
 
-bool fused_decode_supported(const dfssm_dims_t& d, int B, const dfssm_layer_t* layers, int n) {
+bool fused_decode_supported(const dfssm_dims_t& d, int B, const dfssm_layer_t* layers, int n,
+                            float* const* conv_states) {
   if (B != 1 || d.d_model != fused::DM || d.nheads != fused::H || d.headdim != fused::P ||
       d.d_state != fused::N || d.ngroups != 1)
     return false;
-  for (int l = 0; l < n; ++l)
-    if (layers[l].in_proj.rank != fused::R || layers[l].out_proj.rank != fused::R) return false;
+  // the ranges fetched by bulk copy must start on 16-byte boundaries
+  const auto a16 = [](const void* q) { return (reinterpret_cast<uintptr_t>(q) & 15) == 0; };
+  for (int l = 0; l < n; ++l) {
+    const dfssm_layer_t& L = layers[l];
+    if (L.in_proj.rank != fused::R || L.out_proj.rank != fused::R) return false;
+    if (!a16(L.in_proj.w_scale) || !a16(L.in_proj.lora_a_scale) || !a16(L.in_proj.lora_a) ||
+        !a16(L.in_proj.lora_b) || !a16(L.out_proj.lora_b) || !a16(L.conv_w) || !a16(L.conv_b) ||
+        !a16(conv_states[l]))
+      return false;
+  }
   const int nc = num_sms();
   // ownership limits: in_proj rows per CTA <= 64, out_proj rows <= 16, SSM rows <= 32; partial-sum
   // buffers sized for MAX_CTAS

@@ -102,7 +102,8 @@ size_t prefill_workspace_bytes(int M, int d_in, int d_out);
 
 // Fused persistent decode (one cooperative launch per token through all layers).
 size_t fused_decode_workspace_bytes();
-bool fused_decode_supported(const dfssm_dims_t& d, int B, const dfssm_layer_t* layers, int n);
+bool fused_decode_supported(const dfssm_dims_t& d, int B, const dfssm_layer_t* layers, int n,
+                            float* const* conv_states);
 cudaError_t launch_fused_decode(const dfssm_layer_t* layers, int n_layers, float* hidden,
                                 float* const* conv_states, float* const* ssm_states, void* ws,
                                 cudaStream_t st, long long spin_limit);

@@ -151,17 +151,19 @@ __device__ __forceinline__ void prefetch_range(const void* p, size_t bytes, int 
 }
 
 // Dynamic shared memory: the bits ring, the parameter ring (ns stages each), W_B of the current linear
-// when it fits, and the codes in both layouts.  ns is the largest stage count (<= 8) that fits.
+// when it fits, and the codes in both layouts.  W_B in shared memory is preferred (it takes the LoRA-down
+// off global-memory latency) as long as at least 6 stages remain; then the largest stage count <= 8.
 constexpr size_t kSmemBudget = 215 * 1024;
 __host__ __device__ constexpr size_t base_smem(int din, int bt, int ns) {
   return (size_t)ns * (TILE_BYTES + P_BYTES) + 2 * (size_t)bt * din;
 }
-__host__ __device__ constexpr int n_stages(int din, int bt) {
-  return base_smem(din, bt, 8) <= kSmemBudget ? 8 : base_smem(din, bt, 7) <= kSmemBudget ? 7
-         : base_smem(din, bt, 6) <= kSmemBudget ? 6 : 5;
+__host__ __device__ constexpr bool fits(int din, int bt, int ns, bool wb) {
+  return base_smem(din, bt, ns) + (wb ? (size_t)R * din : 0) <= kSmemBudget;
 }
-__host__ __device__ constexpr bool wb_in_smem(int din, int bt) {
-  return base_smem(din, bt, n_stages(din, bt)) + (size_t)R * din <= kSmemBudget;
+__host__ __device__ constexpr bool wb_in_smem(int din, int bt) { return fits(din, bt, 6, true); }
+__host__ __device__ constexpr int n_stages(int din, int bt) {
+  return fits(din, bt, 8, wb_in_smem(din, bt)) ? 8 : fits(din, bt, 7, wb_in_smem(din, bt)) ? 7
+         : fits(din, bt, 6, wb_in_smem(din, bt)) ? 6 : 5;
 }
 __host__ __device__ constexpr size_t smem_bytes(int din, int bt) {
   return base_smem(din, bt, n_stages(din, bt)) + (wb_in_smem(din, bt) ? (size_t)R * din : 0);
@@ -316,6 +318,28 @@ __global__ void __launch_bounds__(NT, 1) stream_kernel(const __grid_constant__ P
   // instruction issues the copies of several stages); lane 31 streams the linears' W_B; the remaining
   // lanes warm L2 with the parameters that do not travel by bulk copy.
   if (warp == PROD_WARP) {
+    // the W_B copies (lane 31): the first one goes into the copy queue ahead of every tile
+    Cursor wa, wz;
+    wa.start(lin_sm, p.n_lin, k0);
+    wz.start(lin_sm, p.n_lin, k1 - 1);
+    int wj = wa.j, wm = 0;
+    bool wok = true;
+    const auto issue_wb = [&]() {  // next linear of the range with a LoRA; false when none is left
+      while (wj <= wz.j && lin_sm[wj].rank == 0) ++wj;
+      if (wj > wz.j) return false;
+      if (wm > 0 && !mbar_wait_or_abort(&wb_empty, (wm - 1) & 1, &abort_flag)) {
+        wok = false;
+        return false;
+      }
+      const Lin& L = lin_sm[wj];
+      mbar_expect_tx(&wb_full, (uint32_t)(L.rank * DIN));
+      bulk_g2s(wb_sm, L.lora_b, (uint32_t)(L.rank * DIN), &wb_full);
+      ++wm;
+      ++wj;
+      return true;
+    };
+    if (use_wb && lane == 31) issue_wb();
+    __syncwarp();
     if (lane < NS) {
       const int sl = lane;
       Cursor cu;
@@ -357,29 +381,16 @@ __global__ void __launch_bounds__(NT, 1) stream_kernel(const __grid_constant__ P
       }
     } else if (lane == 31) {
       if (!use_wb) return;
-      // W_B of each linear of the range that has a LoRA, in order; the GEMV warps release the buffer
-      // after computing t of the previous one
-      Cursor a, b;
-      a.start(lin_sm, p.n_lin, k0);
-      b.start(lin_sm, p.n_lin, k1 - 1);
-      int m = 0;
-      bool ok = true;
-      for (int j = a.j; j <= b.j; ++j) {
-        const Lin& L = lin_sm[j];
-        if (L.rank == 0) continue;
-        if ((m > 0 && !mbar_wait_or_abort(&wb_empty, (m - 1) & 1, &abort_flag)) || abort_flag) {
-          ok = false;
-          break;
-        }
-        mbar_expect_tx(&wb_full, (uint32_t)(L.rank * DIN));
-        bulk_g2s(wb_sm, L.lora_b, (uint32_t)(L.rank * DIN), &wb_full);
-        ++m;
+      // the following linears' W_B, in order; the GEMV warps release the buffer after computing t of
+      // the previous one
+      while (wok && !abort_flag && issue_wb()) {
       }
-      if (!ok) {
+      if (!wok) {
         atomicExch(p.status, kTimeoutCode);
         abort_flag = 1;
-        if (m > 0) mbar_wait(&wb_full, (m - 1) & 1);
       }
+      if (!wok || abort_flag)
+        if (wm > 0) mbar_wait(&wb_full, (wm - 1) & 1);
     } else {
       Cursor a, b;
       a.start(lin_sm, p.n_lin, k0);
