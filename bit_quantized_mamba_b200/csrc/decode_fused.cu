@@ -89,6 +89,9 @@ constexpr size_t OFF_GBUF = OFF_SACC + ((NSH * 4 + 255) / 256) * 256;
 constexpr size_t WS_BYTES = OFF_GBUF + E * 4;
 // dynamic shared memory: W_B of in_proj [R][DM] and of out_proj [R][E]
 constexpr int WB_BYTES = R * (DM + E);
+// dynamic shared memory: W_B of both linears, then the CTA's SSM state rows of two consecutive layers
+constexpr int ST_BYTES = MAX_SSM * N * 4;
+constexpr int DYN_BYTES = WB_BYTES + 2 * ST_BYTES;
 
 // ------------------------------------------------------------------------------ synchronisation
 
@@ -222,6 +225,31 @@ __device__ __forceinline__ int lora_row(const int8_t* wb_row, const int8_t* qn, 
   return __reduce_add_sync(0xffffffffu, t);
 }
 
+// Block-wide absmax of the threads' non-negative m (one redux per warp; the bit patterns of non-negative
+// floats order like the floats).  Contains one CTA barrier.
+__device__ __forceinline__ float block_absmax(float m, int lane, int warp, unsigned* red_u) {
+  const unsigned mw = __reduce_max_sync(0xffffffffu, __float_as_uint(m));
+  if (lane == 0) red_u[warp] = mw;
+  __syncthreads();
+  unsigned mb = 0u;
+#pragma unroll
+  for (int q = 0; q < NW / 4; ++q) {
+    const uint4 u = reinterpret_cast<const uint4*>(red_u)[q];
+    mb = max(max(mb, u.x), max(u.y, max(u.z, u.w)));
+  }
+  return __uint_as_float(mb);
+}
+// Sum of the sixteen per-warp partial sums.
+__device__ __forceinline__ int block_sum16(const int* red_i) {
+  int t = 0;
+#pragma unroll
+  for (int q = 0; q < NW / 4; ++q) {
+    const int4 u = reinterpret_cast<const int4*>(red_i)[q];
+    t += (u.x + u.y) + (u.z + u.w);
+  }
+  return t;
+}
+
 // ------------------------------------------------------------------------------ the kernel
 //
 // Per layer (three hand-offs):
@@ -239,11 +267,13 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ P
   __shared__ LayerPtrs lsm[DFSSM_MAX_LAYERS];
   int8_t* const wb_in = wb_sm;
   int8_t* const wb_out = wb_sm + R * DM;
+  float* const st_sm = reinterpret_cast<float*>(wb_sm + WB_BYTES);  // [2][MAX_SSM][N], layer l in l & 1
   __shared__ __align__(16) int8_t q_perm[E];
   __shared__ __align__(16) int8_t q_nat[E];
-  __shared__ double red_d[NW];
-  __shared__ float red_f[NW];
-  __shared__ int red_i[NW];
+  __shared__ double ss_sm[NT];                 // per-thread sums of squares (summed by the chain warp)
+  __shared__ __align__(16) unsigned red_u[NW];  // per-warp absmax (bit pattern of a non-negative float)
+  __shared__ __align__(16) int red_i[NW];       // per-warp code sums
+  __shared__ float lbs_o[R];                    // out_proj W_B row scales
   __shared__ int t_sm[R];
   __shared__ int sflag;
   __shared__ float tf[R];
@@ -261,6 +291,8 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ P
   __shared__ __align__(16) float bc_st[2 * N][3];
   // bulk-copy completion: [0] the rows every CTA needs + in_proj W_B, [1] out_proj W_B (once per layer)
   __shared__ uint64_t ldbar[2];
+  // SSM state rows of layer l arrive in buffer l & 1, one layer ahead (completes once per two layers)
+  __shared__ uint64_t stbar[2];
   __shared__ float bc_new[2 * N];
   __shared__ __align__(16) float Bsm[N];
   __shared__ __align__(16) double Cd[N];
@@ -304,10 +336,26 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ P
     if (tid == 0) {
       mbar_init(&ldbar[0], 1);
       mbar_init(&ldbar[1], 1);
+      mbar_init(&stbar[0], 1);
+      mbar_init(&stbar[1], 1);
       asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+      // layer 0's SSM state rows of this CTA
+      mbar_expect_tx(&stbar[0], n_ssm * N * 4);
+      bulk_g2s(st_sm, p.L[0].ssm_state + (size_t)rs0 * N, n_ssm * N * 4, &stbar[0]);
     }
     __syncthreads();
   }
+  // An aborting CTA first waits (bounded) for everything it may still have landing in its shared memory:
+  // its own cp.async copies and the bulk copies of layer l (and of layer l + 1's state rows).
+  const auto drain = [&](int l, bool has_next) {
+    cp_async_wait<0>();
+    if (tid == 0) {
+      mbar_wait(&ldbar[0], l & 1, p.spin_limit);
+      mbar_wait(&ldbar[1], l & 1, p.spin_limit);
+      mbar_wait(&stbar[l & 1], (l >> 1) & 1, p.spin_limit);
+      if (has_next) mbar_wait(&stbar[(l + 1) & 1], ((l + 1) >> 1) & 1, p.spin_limit);
+    }
+  };
   for (int l = 0; l < p.n_layers; ++l) {
     const LayerPtrs& Lp = lsm[l];
     const bool has_next = l + 1 < p.n_layers;
@@ -372,23 +420,13 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ P
     }
     w_out = slot_out < n_out ? ld_stream_u4(Lp.out_bits + (size_t)(ro0 + slot_out) * (E / 32) + lane * 4)
                              : make_uint4(0, 0, 0, 0);
-    float4 sv[2];
-#pragma unroll
-    for (int ps = 0; ps < 2; ++ps) {
-      const int rr = ssm_slot[ps];
-      sv[ps] = rr < n_ssm ? ld_evict_first_f4(Lp.ssm_state + (size_t)(rs0 + rr) * N + lane * 4)
-                          : make_float4(0.f, 0.f, 0.f, 0.f);
-    }
     float nw[4], gw[8];
 #pragma unroll
     for (int k = 0; k < 4; ++k) nw[k] = __ldg(Lp.norm_w + tid + k * NT);
 #pragma unroll
     for (int k = 0; k < 8; ++k) gw[k] = __ldg(Lp.gnorm_w + tid + k * NT);
-    float lbs_in = 0.f, lbs_out = 0.f;
-    if (tid >= kChainBase && tid < kChainBase + R) {
-      lbs_in = __ldg(Lp.in_lbs + tid - kChainBase);
-      lbs_out = __ldg(Lp.out_lbs + tid - kChainBase);
-    }
+    float lbs_in = 0.f;
+    if (tid >= kChainBase && tid < kChainBase + R) lbs_in = __ldg(Lp.in_lbs + tid - kChainBase);
     // own x channels: conv taps, bias, state (thread NSH + j handles channel rs0 + j)
     float4 cw = make_float4(0.f, 0.f, 0.f, 0.f);
     float cb = 0.f, cs0 = 0.f, cs1 = 0.f, cs2 = 0.f;
@@ -416,6 +454,13 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ P
       // the contiguous ranges every CTA needs, one bulk copy each; every generic access of the previous
       // layer to these buffers is ordered before them by the barrier that ended that layer
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      // first in the copy queue: the next layer's SSM state rows of this CTA (their buffer was last
+      // read in layer l - 1)
+      if (has_next) {
+        const int nb = (l + 1) & 1;
+        mbar_expect_tx(&stbar[nb], n_ssm * N * 4);
+        bulk_g2s(st_sm + nb * MAX_SSM * N, lsm[l + 1].ssm_state + (size_t)rs0 * N, n_ssm * N * 4, &stbar[nb]);
+      }
       mbar_expect_tx(&ldbar[0], NSH * 4 * 2 + NSH * R + 2 * N * (16 + 4 + 12) + R * DM);
       bulk_g2s(sh_sw, Lp.in_ws + SH0, NSH * 4, &ldbar[0]);
       bulk_g2s(sh_sa, Lp.in_las + SH0, NSH * 4, &ldbar[0]);
@@ -434,23 +479,23 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ P
       cp_async16(o_wa[tid], Lp.out_la + (size_t)row * R);
     }
     if (tid < 2 && hA + tid < H) cp_async4(&Dv[tid], Lp.D + hA + tid);
+    if (tid < R) cp_async4(&lbs_o[tid], Lp.out_lbs + tid);
     cp_async_commit();  // this thread's row parameters (awaited after the h wait)
 
     // ---------------------------------------------------------------- phase A: h -> in_proj
     if (l > 0 && !block_wait(p.ctr + CTR_H * CTR_STRIDE, NC * l, p.err, p.status, p.spin_limit, &sflag)) {
-      cp_async_wait<0>();  // nothing of this CTA may still be landing in its shared memory
-      mbar_wait(&ldbar[0], l & 1, p.spin_limit);
-      mbar_wait(&ldbar[1], l & 1, p.spin_limit);
+      drain(l, has_next);
       return;
     }
     cp_async_wait<0>();  // this thread's row parameters; the quantizer's barriers publish them
     if (!mbar_wait(&ldbar[0], l & 1, p.spin_limit)) {  // shared rows and in_proj W_B
       atomicExch(p.err, 1);
       atomicExch(p.status, kTimeoutMagic);
-      mbar_wait(&ldbar[1], l & 1, p.spin_limit);
+      drain(l, has_next);
       return;
     }
-    double ssA;
+    // RMSNorm folded into the quantizer: codes from the absmax alone; the sum of squares (for the scale)
+    // is parked per thread and reduced by the chain warp off the critical path
     float s0A;
     {
       float v[4];
@@ -464,20 +509,8 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ P
         m = fmaxf(m, fabsf(v[k]));
       }
       if (tid < n_out) h_old[tid] = __ldcg(p.hidden + ro0 + tid);
-      ss = warp_sum(ss);
-      m = warp_max(m);
-      if (lane == 0) {
-        red_d[warp] = ss;
-        red_f[warp] = m;
-      }
-      __syncthreads();
-      ss = 0.0;
-      m = 0.0f;
-#pragma unroll
-      for (int w = 0; w < NW; ++w) {
-        ss += red_d[w];
-        m = fmaxf(m, red_f[w]);
-      }
+      ss_sm[tid] = ss;
+      m = block_absmax(m, lane, warp, red_u);
       const float s0 = m == 0.0f ? 0.0f : __fdiv_rn(m, 127.0f);
       const float inv_s0 = m == 0.0f ? 0.0f : __frcp_rn(s0);
       int sq = 0;
@@ -488,15 +521,12 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ P
         q_nat[tid + k * NT] = (int8_t)code;
         sq += code;
       }
-      sq = warp_sum(sq);
+      sq = __reduce_add_sync(0xffffffffu, sq);
       if (lane == 0) red_i[warp] = sq;
       __syncthreads();
-      ssA = ss;
       s0A = s0;
     }
-    int sumq = 0;
-#pragma unroll
-    for (int w = 0; w < NW; ++w) sumq += red_i[w];
+    const int sumq = block_sum16(red_i);
     // scaffold GEMV over the owned rows; pass 0 holds the rows every CTA needs
     {
       const uint4* qp4 = reinterpret_cast<const uint4*>(q_perm) + li_in;
@@ -505,11 +535,12 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ P
         int S = bits_dot<DM / 128>(w_in[ps], qp4);
 #pragma unroll
         for (int o = 8; o > 0; o >>= 1) S += __shfl_xor_sync(0xffffffffu, S, o);
-        if (li_in == 0 && slot_in[ps] < n_in) acc_in[slot_in[ps]] = 2 * S - sumq;
+        if (li_in == 0 && slot_in[ps] < n_in) {
+          acc_in[slot_in[ps]] = 2 * S - sumq;
+          if (ps == 0 && slot_in[0] < n_sh) p.sacc[sh0 + slot_in[0]] = 2 * S - sumq;
+        }
         if (ps == 0) {
-          __syncthreads();
-          if (tid < n_sh) p.sacc[sh0 + tid] = acc_in[tid];
-          block_arrive(p.ctr + CTR_BC * CTR_STRIDE);
+          block_arrive(p.ctr + CTR_BC * CTR_STRIDE);  // its barrier orders the accumulators above
           // LoRA down of the codes: warp r computes t[r]
           const int t = lora_row<DM / 16>(wb_in + warp * DM, q_nat, lane);
           if (lane == 0) t_sm[warp] = t;
@@ -518,14 +549,19 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ P
     }
     // the fp64 scale chain (RMS, quantizer scale, LoRA intermediate), off the GEMV's critical path: the
     // chain warp has no pass-1 rows, and the epilogue needs the results only after the B/C wait
-    if (tid == kChainBase + R) s_scale = rms_scale(s0A, rms_of(ssA, DM));
+    if (warp == kChainWarp) {
+      double ss = 0.0;
+#pragma unroll
+      for (int k = 0; k < NT / 32; ++k) ss += ss_sm[lane + 32 * k];
+      ss = warp_sum(ss);
+      if (lane == R) s_scale = rms_scale(s0A, rms_of(ss, DM));
+    }
     __syncthreads();
     if (tid >= kChainBase && tid < kChainBase + R) tf[tid - kChainBase] = lora_tf(t_sm[tid - kChainBase], lbs_in, s_scale);
 
     // ---------------------------------------------------------------- phase B: epilogues + SSM
     if (!block_wait(p.ctr + CTR_BC * CTR_STRIDE, NC * (l + 1), p.err, p.status, p.spin_limit, &sflag)) {
-      cp_async_wait<0>();  // nothing of this CTA may still be landing in its shared memory
-      mbar_wait(&ldbar[1], l & 1, p.spin_limit);
+      drain(l, has_next);
       return;
     }
     const float s_in = s_scale;
@@ -555,11 +591,17 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ P
       st[2] = xr;
     }
     __syncthreads();
+    if (!mbar_wait(&stbar[l & 1], (l >> 1) & 1, p.spin_limit)) {  // this layer's SSM state rows
+      atomicExch(p.err, 1);
+      atomicExch(p.status, kTimeoutMagic);
+      drain(l, has_next);
+      return;
+    }
     float4 snew[2];
 #pragma unroll
     for (int ps = 0; ps < 2; ++ps) {
       const int rr = ssm_slot[ps];
-      snew[ps] = sv[ps];
+      snew[ps] = make_float4(0.f, 0.f, 0.f, 0.f);
       if (rr < n_ssm) {
         const int hp = rs0 + rr;
         const int hi = hp / P - hA;
@@ -569,7 +611,7 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ P
         const float4 b4 = reinterpret_cast<const float4*>(Bsm)[lane];
         const double2 c01 = reinterpret_cast<const double2*>(Cd)[2 * lane];
         const double2 c23 = reinterpret_cast<const double2*>(Cd)[2 * lane + 1];
-        float4 s4 = sv[ps];
+        float4 s4 = reinterpret_cast<const float4*>(st_sm + ((l & 1) * MAX_SSM + rr) * N)[lane];
         s4.x = ssm_state(dA, s4.x, dtx, b4.x);
         s4.y = ssm_state(dA, s4.y, dtx, b4.y);
         s4.z = ssm_state(dA, s4.z, dtx, b4.z);
@@ -594,13 +636,13 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ P
 
     // ---------------------------------------------------------------- phase C: gated norm -> out_proj
     if (!block_wait(p.ctr + CTR_G * CTR_STRIDE, NC * (l + 1), p.err, p.status, p.spin_limit, &sflag)) {
-      cp_async_wait<0>();  // nothing of this CTA may still be landing in its shared memory
-      mbar_wait(&ldbar[1], l & 1, p.spin_limit);
+      drain(l, has_next);
       return;
     }
     if (!mbar_wait(&ldbar[1], l & 1, p.spin_limit)) {  // out_proj W_B
       atomicExch(p.err, 1);
       atomicExch(p.status, kTimeoutMagic);
+      drain(l, has_next);
       return;
     }
     // every CTA has now read the old B/C conv state: the owners of those rows shift it
@@ -624,20 +666,8 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ P
         v[k] = fmul(g, gw[k]);
         m = fmaxf(m, fabsf(v[k]));
       }
-      ss = warp_sum(ss);
-      m = warp_max(m);
-      if (lane == 0) {
-        red_d[warp] = ss;
-        red_f[warp] = m;
-      }
-      __syncthreads();
-      ss = 0.0;
-      m = 0.0f;
-#pragma unroll
-      for (int w = 0; w < NW; ++w) {
-        ss += red_d[w];
-        m = fmaxf(m, red_f[w]);
-      }
+      ss_sm[tid] = ss;
+      m = block_absmax(m, lane, warp, red_u);
       const float s0 = m == 0.0f ? 0.0f : __fdiv_rn(m, 127.0f);
       const float inv_s0 = m == 0.0f ? 0.0f : __frcp_rn(s0);
       int sq = 0;
@@ -648,7 +678,7 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ P
         q_nat[tid + k * NT] = (int8_t)code;
         sq += code;
       }
-      sq = warp_sum(sq);
+      sq = __reduce_add_sync(0xffffffffu, sq);
       if (lane == 0) red_i[warp] = sq;
       __syncthreads();
       // LoRA down of the codes (warp r: t[r]); the GEMV warps then take one out_proj row each, and the
@@ -656,11 +686,13 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ P
       const int t = lora_row<E / 16>(wb_out + warp * E, q_nat, lane);
       if (lane == 0) t_sm[warp] = t;
       if (warp == kChainWarp) {
-        if (lane == 0) s_scale = rms_scale(s0, rms_of(ss, E));
-      } else {
-        int sumq_c = 0;
+        double sst = 0.0;
 #pragma unroll
-        for (int w = 0; w < NW; ++w) sumq_c += red_i[w];
+        for (int k = 0; k < NT / 32; ++k) sst += ss_sm[lane + 32 * k];
+        sst = warp_sum(sst);
+        if (lane == 0) s_scale = rms_scale(s0, rms_of(sst, E));
+      } else {
+        const int sumq_c = block_sum16(red_i);
         const uint4* qp4 = reinterpret_cast<const uint4*>(q_perm) + lane;
         int S = bits_dot<E / 128>(w_out, qp4);
         S = warp_sum(S);
@@ -668,12 +700,14 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ P
       }
     }
     __syncthreads();
-    if (tid >= kChainBase && tid < kChainBase + R) tf[tid - kChainBase] = lora_tf(t_sm[tid - kChainBase], lbs_out, s_scale);
-    __syncthreads();
     if (tid < n_out) {
-      const float y = linear_out(acc_out[tid], s_scale, o_sw[tid], o_sa[tid], o_wa[tid], tf, R);
-      const float hn = fadd(h_old[tid], y);
-      p.hidden[ro0 + tid] = hn;
+      // each epilogue thread forms the sixteen LoRA intermediates itself (no further barrier)
+      double tfd[R];
+#pragma unroll
+      for (int r = 0; r < R; ++r) tfd[r] = (double)lora_tf(t_sm[r], lbs_o[r], s_scale);
+      const float y = linear_out_d(acc_out[tid], (double)s_scale, (double)o_sw[tid], (double)o_sa[tid],
+                                   *reinterpret_cast<const uint4*>(o_wa[tid]), tfd, R);
+      p.hidden[ro0 + tid] = fadd(h_old[tid], y);
     }
     block_arrive(p.ctr + CTR_H * CTR_STRIDE);
   }
@@ -760,9 +794,9 @@ cudaError_t launch_fused_decode(const dfssm_layer_t* layers, int n_layers, float
   cfg.blockDim = dim3(fused::NT);
   // set once (not per launch, so that launches can be captured in a CUDA graph)
   static const cudaError_t attr_set = cudaFuncSetAttribute(
-      fused::decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, fused::WB_BYTES);
+      fused::decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, fused::DYN_BYTES);
   if (attr_set != cudaSuccess) return attr_set;
-  cfg.dynamicSmemBytes = fused::WB_BYTES;
+  cfg.dynamicSmemBytes = fused::DYN_BYTES;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeCooperative;
