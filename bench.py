@@ -163,6 +163,12 @@ def run_reference(args, rank):
 
 # ---------------------------------------------------------------------------------- our arm
 
+# DRAM traffic of one decode_kernel launch (dram__bytes_read.sum + dram__bytes_write.sum, one ncu capture
+# of the fourth launch of `bench.py --ncu --warmup 3`: 280.90 MB + 57.09 MB), valid only for the kernel
+# source it was measured on; reported as null once that source changes.
+TRAFFIC_MEASURED = {"sha": "9ded017b15d8", "bytes": 337_984_000}
+
+
 def src_sha(*names):
     h = hashlib.sha1()
     for n in names:
@@ -419,7 +425,9 @@ def run_ours(args, rank, world, local_rank):
     us_tok = ms_per_step * 1e3 / N_TOKENS
     achieved = BYTES_TOKEN / (us_tok * 1e-6) / 1e9
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
-                "frac": round(achieved / hbm, 4), "traffic": None,
+                "frac": round(achieved / hbm, 4),
+                "traffic": (TRAFFIC_MEASURED["bytes"]
+                            if src_sha("decode_fused.cu", "common.cuh") == TRAFFIC_MEASURED["sha"] else None),
                 "kernel": "dfssm::fused::decode_kernel (one cooperative launch per token, 48 layers)",
                 "bytes_per_launch": BYTES_TOKEN, "peak_kind": peak_kind}
     line = {
@@ -467,6 +475,21 @@ def run_prefill_profile(args):
     torch.cuda.synchronize()
 
 
+def run_gemv_profile(args):
+    """Eager dfssm_linear_decode_multi calls over the 48 in_proj copies at batch 1, for ncu."""
+    import torch
+    from bit_quantized_mamba_b200 import build, dfssm, inputs
+    build.build()
+    dev = torch.device("cuda", 0)
+    data = inputs.in_proj_stack()
+    lins = [dfssm.Linear.from_host(l, dev) for l in data["linears"]]
+    x = torch.from_numpy(data["x"][:1].copy()).to(dev)
+    ys = [torch.empty((1, L.d_out), dtype=torch.float32, device=dev) for L in lins]
+    for _ in range(args.warmup + 1):
+        dfssm.linear_decode_multi(lins, x, ys)
+    torch.cuda.synchronize()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -479,10 +502,12 @@ def main():
                     help="skip the GEMV sweep, prefill and LM-head measurements")
     ap.add_argument("--ncu-prefill", action="store_true",
                     help="profiling mode: run the 2048-token in_proj prefill --warmup + 1 times and exit")
+    ap.add_argument("--ncu-gemv", action="store_true",
+                    help="profiling mode: the 48-copy in_proj multi-linear decode --warmup + 1 times and exit")
     ap.add_argument("--ncu", action="store_true",
                     help="profiling mode: decode --warmup tokens then one more token, eagerly, and exit")
     args = ap.parse_args()
-    if args.warmup < 3 and not args.ncu:
+    if args.warmup < 3 and not (args.ncu or args.ncu_gemv or args.ncu_prefill):
         args.warmup = 3
     rank = int(os.environ.get("RANK", 0))
     world = int(os.environ.get("WORLD_SIZE", 1))
@@ -492,6 +517,9 @@ def main():
         return
     if args.ncu_prefill:
         run_prefill_profile(args)
+        return
+    if args.ncu_gemv:
+        run_gemv_profile(args)
         return
     if world > 1:
         import datetime
