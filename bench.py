@@ -335,8 +335,6 @@ def run_ours(args, rank, world, local_rank):
                 gbs = nbytes / (us_per_call * 1e-6) / 1e9
                 gemv[f"{which}_B{B}"] = {"us_per_call": round(us_per_call, 3), "GB_s": round(gbs, 1),
                                          "frac_of_measured_hbm": round(gbs / hbm, 3)}
-                if B > 4:
-                    continue
                 # the same 48 copies in one dfssm_linear_decode_multi launch (shared input x)
                 ys = [torch.empty((B, L.d_out), dtype=torch.float32, device=dev) for L in lins]
                 g = torch.cuda.CUDAGraph()

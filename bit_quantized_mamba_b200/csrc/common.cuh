@@ -101,6 +101,25 @@ __device__ __forceinline__ int quant_code_fast(float v, float s0, float inv_s0) 
   if (fabsf(t - k) < 0.499f) return (int)fminf(fmaxf(k, -127.0f), 127.0f);
   return quant_code(v, s0);
 }
+// The codes of N values at once, the same as quant_code_fast for each: the product path for all of them
+// without branches, then (rarely) the IEEE division for those close to a rounding boundary, behind one
+// branch.  inv_s0 = 0 (an all-zero token) gives code 0 everywhere.
+template <int N>
+__device__ __forceinline__ void quant_codes(const float (&v)[N], float s0, float inv_s0, int (&code)[N]) {
+  uint32_t near = 0u;
+#pragma unroll
+  for (int e = 0; e < N; ++e) {
+    const float t = v[e] * inv_s0;
+    const float k = rintf(t);
+    code[e] = (int)fminf(fmaxf(k, -127.0f), 127.0f);
+    near |= (fabsf(t - k) < 0.499f ? 0u : 1u) << e;
+  }
+  if (near) {
+#pragma unroll
+    for (int e = 0; e < N; ++e)
+      if ((near >> e) & 1u) code[e] = quant_code(v[e], s0);
+  }
+}
 
 // Position of natural-order activation index i inside the dp4a-friendly permuted layout: within each
 // 32-element block, word k (k = 0..7) holds elements k, k+8, k+16, k+24 in its four bytes.  With that

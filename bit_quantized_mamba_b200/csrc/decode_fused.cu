@@ -514,12 +514,13 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ P
       const float s0 = m == 0.0f ? 0.0f : __fdiv_rn(m, 127.0f);
       const float inv_s0 = m == 0.0f ? 0.0f : __frcp_rn(s0);
       int sq = 0;
+      int cd[4];
+      quant_codes<4>(v, s0, inv_s0, cd);
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
-        const int code = m == 0.0f ? 0 : quant_code_fast(v[k], s0, inv_s0);
-        q_perm[seg_index<DM / 128>(tid + k * NT)] = (int8_t)code;
-        q_nat[tid + k * NT] = (int8_t)code;
-        sq += code;
+        q_perm[seg_index<DM / 128>(tid + k * NT)] = (int8_t)cd[k];
+        q_nat[tid + k * NT] = (int8_t)cd[k];
+        sq += cd[k];
       }
       sq = __reduce_add_sync(0xffffffffu, sq);
       if (lane == 0) red_i[warp] = sq;
@@ -671,12 +672,13 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ P
       const float s0 = m == 0.0f ? 0.0f : __fdiv_rn(m, 127.0f);
       const float inv_s0 = m == 0.0f ? 0.0f : __frcp_rn(s0);
       int sq = 0;
+      int cd[8];
+      quant_codes<8>(v, s0, inv_s0, cd);
 #pragma unroll
       for (int k = 0; k < 8; ++k) {
-        const int code = m == 0.0f ? 0 : quant_code_fast(v[k], s0, inv_s0);
-        q_perm[seg_index<E / 128>(tid + k * NT)] = (int8_t)code;
-        q_nat[tid + k * NT] = (int8_t)code;
-        sq += code;
+        q_perm[seg_index<E / 128>(tid + k * NT)] = (int8_t)cd[k];
+        q_nat[tid + k * NT] = (int8_t)cd[k];
+        sq += cd[k];
       }
       sq = __reduce_add_sync(0xffffffffu, sq);
       if (lane == 0) red_i[warp] = sq;

@@ -92,7 +92,7 @@ extern "C" int dfssm_linear_decode_noalloc(const dfssm_linear_t* lin, const floa
       major != 10)
     return DFSSM_EDEVICE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  // B <= 4 at d_in in {1024, ..., 8192}: the single streaming kernel needs no scratch at all
+  // in the streaming kernel's range the single kernel needs no scratch at all
   if (dfssm::stream_supported(lin->d_in, B)) return dfssm::launch_linear_stream(lin, 1, x, B, &y, dbg, s);
   void* scratch = nullptr;
   st = scratch_address(&scratch);

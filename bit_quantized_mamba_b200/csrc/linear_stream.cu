@@ -2,7 +2,7 @@
 // §2.B "Frozen Scaffold with LoRA Correction" and §2.C "Optimized Inference Pipeline": the scaffold
 // matmul on 1-bit packed weights with int8 activations and int32 accumulation, plus the int8 LoRA).
 //
-// At batch <= 4 the scaffold product is a matrix-vector product bound by the HBM stream of sign bits, so
+// At batch <= 16 the scaffold product is a matrix-vector product (ALU-bound beyond a few tokens), so
 // one persistent, warp-specialised kernel does everything for any number of linears that read the same x:
 //   * the rows of all linears are cut into 16 KB tiles of packed bits; each CTA takes a contiguous range
 //     of tiles.  A producer warp streams every tile into a ring of shared-memory stages and its rows' W_A
@@ -41,13 +41,35 @@ constexpr int PROD_WARP = NCW + NEW;     // producer warp
 constexpr int NT = (NCW + NEW + 1) * 32;
 constexpr int TILE_BYTES = 16384;        // packed bits per tile
 constexpr int MAX_TR = 128;              // rows per tile (d_in >= 1024)
-constexpr int MAX_B = 4;
+constexpr int MAX_B = 16;
 constexpr int R = DFSSM_MAX_RANK;
 constexpr int MAX_NS = 8;                // stages per ring (bits ring and parameter ring alike)
-// parameter stage: W_A rows (16 B), sW, sA (4 B each) by bulk copy, then the int32 accumulators and the
-// LoRA intermediates (fp64) written by the GEMV warps
-constexpr int P_WA = 0, P_SW = MAX_TR * 16, P_SA = P_SW + MAX_TR * 4, P_ACC = P_SA + MAX_TR * 4,
-              P_TF = P_ACC + MAX_TR * MAX_B * 4, P_BYTES = P_TF + MAX_B * R * 8;
+// Permuted codes of one token in shared memory: eight rows of 16-byte chunks (row v holds chunk v of every
+// 128-input segment, in segment order) plus one pad chunk per row.  A GEMV lane that owns segment seg reads
+// row v at chunk seg (consecutive lanes, consecutive chunks); the pad puts the eight chunks of one segment
+// (written together by the quantizer) in eight different bank groups.
+__host__ __device__ constexpr int q_row(int segs) { return segs + 1; }        // chunks per row
+__host__ __device__ constexpr int q_tok(int segs) { return 8 * q_row(segs); }  // chunks per token
+__host__ __device__ constexpr int q_tok_bytes(int din) { return 16 * q_tok(din / 128); }
+// Byte offset, within a token, of natural input index i.
+template <int SEGS>
+__device__ __forceinline__ int q_index(int i) {
+  const int seg = i >> 7;
+  const int pos = perm_index(i) & 127;
+  return ((pos >> 4) * q_row(SEGS) + seg) * 16 + (pos & 15);
+}
+// Parameter stage of a tile of tr rows for bt token slots: W_A rows (16 B each), sW and sA (4 B each) by
+// bulk copy, then the int32 accumulators [bt][tr] and the LoRA intermediates [bt][16] (fp64) written by the
+// GEMV warps.  Every offset is a multiple of 16 bytes for tr >= 16.
+struct PLayout {
+  int sw, sa, acc, tf, bytes;
+};
+__host__ __device__ constexpr int rows_per_tile(int din) { return TILE_BYTES / (din / 8); }
+__host__ __device__ constexpr PLayout p_layout(int din, int bt) {
+  return PLayout{rows_per_tile(din) * 16, rows_per_tile(din) * 20, rows_per_tile(din) * 24,
+                 rows_per_tile(din) * 24 + rows_per_tile(din) * bt * 4,
+                 rows_per_tile(din) * 24 + rows_per_tile(din) * bt * 4 + bt * R * 8};
+}
 constexpr int MAX_LIN = DFSSM_MAX_LAYERS;
 constexpr long long kWaitBudget = 2000000000LL;  // clock cycles per wait (~1 s)
 constexpr int kTimeoutCode = 0x5EA0715E;
@@ -155,7 +177,7 @@ __device__ __forceinline__ void prefetch_range(const void* p, size_t bytes, int 
 // off global-memory latency) as long as at least 6 stages remain; then the largest stage count <= 8.
 constexpr size_t kSmemBudget = 215 * 1024;
 __host__ __device__ constexpr size_t base_smem(int din, int bt, int ns) {
-  return (size_t)ns * (TILE_BYTES + P_BYTES) + 2 * (size_t)bt * din;
+  return (size_t)ns * (TILE_BYTES + p_layout(din, bt).bytes) + (size_t)bt * (q_tok_bytes(din) + din);
 }
 __host__ __device__ constexpr bool fits(int din, int bt, int ns, bool wb) {
   return base_smem(din, bt, ns) + (wb ? (size_t)R * din : 0) <= kSmemBudget;
@@ -163,7 +185,7 @@ __host__ __device__ constexpr bool fits(int din, int bt, int ns, bool wb) {
 __host__ __device__ constexpr bool wb_in_smem(int din, int bt) { return fits(din, bt, 6, true); }
 __host__ __device__ constexpr int n_stages(int din, int bt) {
   return fits(din, bt, 8, wb_in_smem(din, bt)) ? 8 : fits(din, bt, 7, wb_in_smem(din, bt)) ? 7
-         : fits(din, bt, 6, wb_in_smem(din, bt)) ? 6 : 5;
+         : fits(din, bt, 6, wb_in_smem(din, bt)) ? 6 : fits(din, bt, 5, wb_in_smem(din, bt)) ? 5 : 4;
 }
 __host__ __device__ constexpr size_t smem_bytes(int din, int bt) {
   return base_smem(din, bt, n_stages(din, bt)) + (wb_in_smem(din, bt) ? (size_t)R * din : 0);
@@ -195,10 +217,10 @@ __device__ __forceinline__ uint4 load_wa(const Lin& L, int row) {
 }
 
 // 128 x (sum over bit=1 positions of q) for 128 weights against BT tokens' permuted codes of one segment:
-// token b's chunk v is q0[b * DIN / 16 + v * SEGS].
+// token b's chunk v is q0[b * q_tok(SEGS) + v * q_row(SEGS)].
 template <int SEGS, int BT>
 __device__ __forceinline__ void bits_dot_tokens(uint4 w, const uint4* q0, int B, int (&S)[BT]) {
-  constexpr int DIN16 = SEGS * 8;  // 16-byte chunks per token
+  constexpr int DIN16 = q_tok(SEGS);  // 16-byte chunks per token, pads included
   const uint32_t w4[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
   for (int b = 0; b < BT; ++b) {
@@ -209,7 +231,7 @@ __device__ __forceinline__ void bits_dot_tokens(uint4 w, const uint4* q0, int B,
       for (int k = 0; k < 8; ++k) acc8[k] = 0;
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        const uint4 qa = qp4[(2 * j) * SEGS], qb = qp4[(2 * j + 1) * SEGS];
+        const uint4 qa = qp4[(2 * j) * q_row(SEGS)], qb = qp4[(2 * j + 1) * q_row(SEGS)];
         const uint32_t qp[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
 #pragma unroll
         for (int k = 0; k < 8; ++k) acc8[k] = dp4a_us(w4[j] & (0x01010101u << k), qp[k], acc8[k]);
@@ -251,21 +273,29 @@ __global__ void __launch_bounds__(NT, 1) stream_kernel(const __grid_constant__ P
   constexpr int ROW16 = DIN / 128;             // 16-byte chunks of packed bits per row
   constexpr int RPW = 32 / LPR;                // rows per warp per pass
   constexpr int RPP = NCW * RPW;               // rows per pass
-  constexpr int TR = TILE_BYTES / (DIN / 8);   // rows per tile
+  constexpr int TR = rows_per_tile(DIN);      // rows per tile
+  constexpr PLayout PL = p_layout(DIN, BT);
   constexpr int PASSES = TR / RPP;
   static_assert(PASSES >= 1 && PASSES * RPP == TR && TR <= MAX_TR, "tile shape");
-  static_assert(LPR >= BT, "one lane per token in a row group");
   constexpr bool WB_SMEM = wb_in_smem(DIN, BT);
   constexpr int NS = n_stages(DIN, BT);
   constexpr int XPT = DIN / (NCW * 32);                    // x values per GEMV thread per token
   constexpr bool XREG = BT * XPT <= 16;                    // keep x in registers between the two passes
   constexpr bool REGQ = BT == 1 && NSEG == 1;              // one token: the lane's codes live in registers
+  // many tokens: a run-time token loop against the lane's weight masks held in registers
+  constexpr bool TOKLOOP = BT > 4;
+  static_assert(!TOKLOOP || NSEG == 1, "token loop needs one segment per lane");
+  // Epilogue warps in use.  Warp e takes every NEP-th tile, so it waits on a stage's barriers at most one
+  // phase ahead of the last completed one only if NEP <= NS (an mbarrier parity wait cannot tell phase n
+  // from phase n - 2).
+  constexpr int NEP = NEW < NS ? NEW : NS;
 
   extern __shared__ __align__(128) unsigned char smem[];
-  unsigned char* pring = smem + (size_t)NS * TILE_BYTES;                            // [NS][P_BYTES]
-  int8_t* wb_sm = reinterpret_cast<int8_t*>(pring + (size_t)NS * P_BYTES);          // [R][DIN] if WB_SMEM
-  int8_t* q_perm = wb_sm + (WB_SMEM ? R * DIN : 0);                                 // [BT][DIN]
-  int8_t* q_nat = q_perm + BT * DIN;                                                // [BT][DIN]
+  unsigned char* pring = smem + (size_t)NS * TILE_BYTES;                            // [NS][PL.bytes]
+  int8_t* wb_sm = reinterpret_cast<int8_t*>(pring + (size_t)NS * PL.bytes);         // [R][DIN] if WB_SMEM
+  constexpr int QTB = q_tok_bytes(DIN);                                             // permuted token bytes
+  int8_t* q_perm = wb_sm + (WB_SMEM ? R * DIN : 0);                                 // [BT][QTB]
+  int8_t* q_nat = q_perm + BT * QTB;                                                // [BT][DIN]
   __shared__ Lin lin_sm[MAX_LIN];
   __shared__ uint64_t bfull[MAX_NS], bempty[MAX_NS], pfull[MAX_NS], pacc[MAX_NS], pempty[MAX_NS], wb_full,
       wb_empty;
@@ -275,6 +305,7 @@ __global__ void __launch_bounds__(NT, 1) stream_kernel(const __grid_constant__ P
   __shared__ int t_sm[MAX_B][R];
   __shared__ float red_f[NCW][MAX_B];
   __shared__ int red_i[NCW][MAX_B];
+  __shared__ int s_sumq[MAX_B];
   __shared__ volatile int abort_flag;
   __shared__ int wb_ok;
 
@@ -284,6 +315,8 @@ __global__ void __launch_bounds__(NT, 1) stream_kernel(const __grid_constant__ P
   const int k1 = (int)((long long)(c + 1) * p.total_tiles / G);
   const int ntiles = k1 - k0;
   const int B = p.B;
+  // fewer tiles than epilogue warps: every epilogue warp takes a share of every tile instead of whole tiles
+  const bool epi_split = ntiles < NEP;
 
   if (tid < p.n_lin) {
     Lin L = p.lin[tid];
@@ -297,7 +330,7 @@ __global__ void __launch_bounds__(NT, 1) stream_kernel(const __grid_constant__ P
       mbar_init(&bempty[s], NCW);
       mbar_init(&pfull[s], 1);
       mbar_init(&pacc[s], NCW);
-      mbar_init(&pempty[s], 1);
+      mbar_init(&pempty[s], epi_split ? NEP : 1);
     }
     mbar_init(&wb_full, 1);
     mbar_init(&wb_empty, 1);
@@ -360,13 +393,13 @@ __global__ void __launch_bounds__(NT, 1) stream_kernel(const __grid_constant__ P
         const uint32_t bits_bytes = (uint32_t)nr * (DIN / 8);
         mbar_expect_tx(&bfull[sl], bits_bytes);
         bulk_g2s(smem + (size_t)sl * TILE_BYTES, L.bits + (size_t)r0 * (DIN / 32), bits_bytes, &bfull[sl]);
-        unsigned char* ps = pring + (size_t)sl * P_BYTES;
+        unsigned char* ps = pring + (size_t)sl * PL.bytes;
         mbar_expect_tx(&pfull[sl], L.ptma ? (uint32_t)(nr * 16 + 2 * n4 * 4) : 0u);
         if (L.ptma) {
-          bulk_g2s(ps + P_WA, L.lora_a + (size_t)r0 * R, (uint32_t)(nr * 16), &pfull[sl]);
+          bulk_g2s(ps, L.lora_a + (size_t)r0 * R, (uint32_t)(nr * 16), &pfull[sl]);
           if (n4 > 0) {
-            bulk_g2s(ps + P_SW, L.w_scale + r0, (uint32_t)(n4 * 4), &pfull[sl]);
-            bulk_g2s(ps + P_SA, L.lora_a_scale + r0, (uint32_t)(n4 * 4), &pfull[sl]);
+            bulk_g2s(ps + PL.sw, L.w_scale + r0, (uint32_t)(n4 * 4), &pfull[sl]);
+            bulk_g2s(ps + PL.sa, L.lora_a_scale + r0, (uint32_t)(n4 * 4), &pfull[sl]);
           }
         }
       }
@@ -415,16 +448,17 @@ __global__ void __launch_bounds__(NT, 1) stream_kernel(const __grid_constant__ P
   }
 
   // ------------------------------------------------------------------ epilogue warps
-  // epilogue warp e takes the tiles i = e, e + NEW, ... of the range, whole, so several tiles' fp64
-  // epilogues are in flight at once
+  // epilogue warp e takes the tiles i = e, e + NEP, ... of the range, whole, so several tiles' fp64
+  // epilogues are in flight at once; with fewer tiles than warps each warp takes a share of every tile
   if (warp >= NCW) {
-    pdl_wait();  // the outputs may still be read or written by the preceding kernel of the stream
     const int e = warp - NCW;
+    if (e >= NEP) return;
+    pdl_wait();  // the outputs may still be read or written by the preceding kernel of the stream
     Cursor cu;
     cu.start(lin_sm, p.n_lin, k0);
     bool dead = false;
     for (int i = 0; i < ntiles; ++i, cu.next(lin_sm)) {
-      if (i % NEW != e) continue;
+      if (!epi_split && i % NEP != e) continue;
       const Lin& L = lin_sm[cu.j];
       const int sp = i % NS;
       const uint32_t par = (i / NS) & 1;
@@ -436,16 +470,17 @@ __global__ void __launch_bounds__(NT, 1) stream_kernel(const __grid_constant__ P
       }
       if (!dead) {
         const int r0 = cu.t * TR, nr = min(TR, L.d_out - r0), n4 = nr & ~3;
-        const unsigned char* ps = pring + (size_t)sp * P_BYTES;
-        const uint4* wa_st = reinterpret_cast<const uint4*>(ps + P_WA);
-        const float* sw_st = reinterpret_cast<const float*>(ps + P_SW);
-        const float* sa_st = reinterpret_cast<const float*>(ps + P_SA);
-        const int* acc = reinterpret_cast<const int*>(ps + P_ACC);
-        const double* tf = reinterpret_cast<const double*>(ps + P_TF);
-        // two (row, token) jobs per lane per step, their fp64 chains interleaved
+        const unsigned char* ps = pring + (size_t)sp * PL.bytes;
+        const uint4* wa_st = reinterpret_cast<const uint4*>(ps);
+        const float* sw_st = reinterpret_cast<const float*>(ps + PL.sw);
+        const float* sa_st = reinterpret_cast<const float*>(ps + PL.sa);
+        const int* acc = reinterpret_cast<const int*>(ps + PL.acc);
+        const double* tf = reinterpret_cast<const double*>(ps + PL.tf);
+        // two (token, row) jobs per lane per step, their fp64 chains interleaved; consecutive lanes take
+        // consecutive rows of one token (coalesced outputs, one broadcast tf row)
         const auto fetch = [&](int job, int& a, double& sw, double& sa, uint4& wa, int& row, int& b) {
-          const int rr = job / B;
-          b = job - rr * B;
+          b = job / nr;
+          const int rr = job - b * nr;
           row = r0 + rr;
           float fw, fa = 0.0f;
           wa = make_uint4(0u, 0u, 0u, 0u);
@@ -467,15 +502,16 @@ __global__ void __launch_bounds__(NT, 1) stream_kernel(const __grid_constant__ P
           }
           sw = (double)fw;
           sa = (double)fa;
-          a = acc[rr * MAX_B + b];
+          a = acc[b * TR + rr];
         };
-        for (int job = lane; job < nr * B; job += 64) {
+        const int jstride = epi_split ? NEP * 32 : 32;
+        for (int job = (epi_split ? e * 32 : 0) + lane; job < nr * B; job += 2 * jstride) {
           int a[2], row[2], b[2];
           double sd[2], sw[2], sa[2];
           uint4 wa[2];
-          const bool two = job + 32 < nr * B;
+          const bool two = job + jstride < nr * B;
           fetch(job, a[0], sw[0], sa[0], wa[0], row[0], b[0]);
-          fetch(two ? job + 32 : job, a[1], sw[1], sa[1], wa[1], row[1], b[1]);
+          fetch(two ? job + jstride : job, a[1], sw[1], sa[1], wa[1], row[1], b[1]);
           sd[0] = s_tokd[b[0]];
           sd[1] = s_tokd[b[1]];
           const double* const t2[2] = {tf + b[0] * R, tf + b[1] * R};
@@ -500,7 +536,94 @@ __global__ void __launch_bounds__(NT, 1) stream_kernel(const __grid_constant__ P
   // ------------------------------------------------------------------ GEMV warps
   pdl_wait();  // x may come from the preceding kernel of the stream
   int sumq[BT];
-  {
+  if constexpr (BT > 1) {
+    // WPT warps per token slot, each over a contiguous slice of the token, 16-byte loads issued in
+    // batches before any use: every CTA asks for all of x at once with many loads in flight, instead of
+    // token by token.  The token of each slot is rotated by the CTA index, so that the CTAs do not all
+    // ask for the same lines of x at the same moment.
+    constexpr int WPT = NCW / BT;               // warps per token slot
+    constexpr int CH = DIN / 4 / WPT;           // float4 per warp slice
+    constexpr int U = CH / 32 < 8 ? CH / 32 : 8;  // loads in flight per lane
+    static_assert(CH % (32 * U) == 0, "quantizer slice");
+    const int slot = warp / WPT, part = warp % WPT;
+    const bool active = slot < B;
+    const int b = active ? (slot + c) % B : 0;
+    const float4* xs = reinterpret_cast<const float4*>(p.x + (size_t)b * DIN) + part * CH;
+    float m = 0.0f;
+    if (active) {
+#pragma unroll 1
+      for (int v0 = lane; v0 < CH; v0 += 32 * U) {
+        float4 t[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) t[u] = __ldg(xs + v0 + 32 * u);
+#pragma unroll
+        for (int u = 0; u < U; ++u)
+          m = fmaxf(m, fmaxf(fmaxf(fabsf(t[u].x), fabsf(t[u].y)), fmaxf(fabsf(t[u].z), fabsf(t[u].w))));
+      }
+    }
+    m = warp_max(m);
+    if (lane == 0) red_f[warp][0] = m;
+    consumer_sync();
+    m = 0.0f;
+#pragma unroll
+    for (int j = 0; j < WPT; ++j) m = fmaxf(m, red_f[slot * WPT + j][0]);
+    const float s0 = m == 0.0f ? 0.0f : __fdiv_rn(m, 127.0f);
+    const float inv_s0 = m == 0.0f ? 0.0f : __frcp_rn(s0);
+    int sq = 0;
+    if (active) {
+#pragma unroll 1
+      for (int v0 = lane; v0 < CH; v0 += 32 * U) {
+        float4 t[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) t[u] = __ldg(xs + v0 + 32 * u);
+        // codes two float4 at a time (one rarely taken branch per eight values)
+#pragma unroll
+        for (int u2 = 0; u2 < U; u2 += 2) {
+          constexpr int G = U < 2 ? U : 2;
+          float tv[4 * G];
+#pragma unroll
+          for (int g = 0; g < G; ++g) {
+            tv[4 * g] = t[u2 + g].x;
+            tv[4 * g + 1] = t[u2 + g].y;
+            tv[4 * g + 2] = t[u2 + g].z;
+            tv[4 * g + 3] = t[u2 + g].w;
+          }
+          int cd[4 * G];
+          quant_codes<4 * G>(tv, s0, inv_s0, cd);
+#pragma unroll
+          for (int g = 0; g < G; ++g) {
+            const int v = part * CH + v0 + 32 * (u2 + g);  // float4 index within the token
+            uint32_t packed = 0u;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              q_perm[b * QTB + q_index<SEGS>(4 * v + e)] = (int8_t)cd[4 * g + e];
+              packed |= (uint32_t)(cd[4 * g + e] & 0xFF) << (8 * e);
+              sq += cd[4 * g + e];
+            }
+            reinterpret_cast<uint32_t*>(q_nat + b * DIN)[v] = packed;
+          }
+        }
+      }
+    }
+    sq = warp_sum(sq);
+    if (lane == 0) red_i[warp][0] = sq;
+    if (active && part == 0 && lane == 0) {
+      s_tok[b] = s0;
+      s_tokd[b] = (double)s0;
+      if (p.dbg_s && c == 0) p.dbg_s[b] = s0;
+    }
+    consumer_sync();
+    if (tid < B) {
+      const int sl = ((tid - c) % B + B) % B;  // the slot that quantized token tid
+      int t = 0;
+#pragma unroll
+      for (int j = 0; j < WPT; ++j) t += red_i[sl * WPT + j][0];
+      s_sumq[tid] = t;
+    }
+    consumer_sync();
+#pragma unroll
+    for (int bb = 0; bb < BT; ++bb) sumq[bb] = bb < B ? s_sumq[bb] : 0;
+  } else {
     float xr[XREG ? BT * XPT : 1];
 #pragma unroll
     for (int b = 0; b < BT; ++b) {
@@ -508,7 +631,7 @@ __global__ void __launch_bounds__(NT, 1) stream_kernel(const __grid_constant__ P
 #pragma unroll
       for (int k = 0; k < XPT; ++k) {
         const int i = tid + k * NCW * 32;
-        const float v = b < B ? p.x[(size_t)b * DIN + i] : 0.0f;
+        const float v = b < B ? __ldg(p.x + (size_t)b * DIN + i) : 0.0f;
         if (XREG) xr[b * XPT + k] = v;
         m = fmaxf(m, fabsf(v));
       }
@@ -525,15 +648,18 @@ __global__ void __launch_bounds__(NT, 1) stream_kernel(const __grid_constant__ P
       const float inv_s0 = m == 0.0f ? 0.0f : __frcp_rn(s0);
       int sq = 0;
       if (b < B) {
+        float v[XPT];
+#pragma unroll
+        for (int k = 0; k < XPT; ++k)
+          v[k] = XREG ? xr[b * XPT + k] : __ldg(p.x + (size_t)b * DIN + tid + k * NCW * 32);
+        int cd[XPT];
+        quant_codes<XPT>(v, s0, inv_s0, cd);
 #pragma unroll
         for (int k = 0; k < XPT; ++k) {
           const int i = tid + k * NCW * 32;
-          const float v = XREG ? xr[b * XPT + k] : p.x[(size_t)b * DIN + i];
-          const int code = m == 0.0f ? 0 : quant_code_fast(v, s0, inv_s0);
-          q_perm[b * DIN + seg_index<SEGS>(i)] = (int8_t)code;
-          q_nat[b * DIN + i] = (int8_t)code;
-          sq += code;
-          if (p.dbg_xq && c == 0) p.dbg_xq[(size_t)b * DIN + i] = (int8_t)code;
+          q_perm[b * QTB + q_index<SEGS>(i)] = (int8_t)cd[k];
+          q_nat[b * DIN + i] = (int8_t)cd[k];
+          sq += cd[k];
         }
       }
       sq = warp_sum(sq);
@@ -551,15 +677,18 @@ __global__ void __launch_bounds__(NT, 1) stream_kernel(const __grid_constant__ P
 #pragma unroll
       for (int w = 0; w < NCW; ++w) sq += red_i[w][b];
       sumq[b] = sq;
+      if (tid == b) s_sumq[b] = sq;
     }
   }
 
+  if (p.dbg_xq && c == 0)  // debug tap: the natural-order codes (published by the last consumer_sync)
+    for (int i = tid; i < B * DIN; i += NCW * 32) p.dbg_xq[i] = q_nat[i];
   const int li = lane % LPR, rsub = lane / LPR;
   uint4 qreg[REGQ ? 8 : 1];
   if (REGQ) {
     const uint4* q0 = reinterpret_cast<const uint4*>(q_perm) + li;
 #pragma unroll
-    for (int v = 0; v < 8; ++v) qreg[v] = q0[v * SEGS];
+    for (int v = 0; v < 8; ++v) qreg[v] = q0[v * q_row(SEGS)];
   }
   Cursor cu;
   cu.start(lin_sm, p.n_lin, k0);
@@ -577,7 +706,8 @@ __global__ void __launch_bounds__(NT, 1) stream_kernel(const __grid_constant__ P
       }
       consumer_sync();
       if (!dead) {
-        for (int r = warp; r < L.rank; r += NCW) {
+        for (int rw = warp; rw < L.rank; rw += NCW) {
+          const int r = (rw + c) % L.rank;  // rotated by CTA: the CTAs read different W_B rows at a time
           int part[BT];
 #pragma unroll
           for (int b = 0; b < BT; ++b) part[b] = 0;
@@ -586,25 +716,30 @@ __global__ void __launch_bounds__(NT, 1) stream_kernel(const __grid_constant__ P
 #pragma unroll
             for (int ch = lane; ch < DIN / 16; ch += 32) {
               const uint4 w = w4[ch];
+              // every token slot, used or not (slots >= B read stale codes and are never stored): no
+              // per-token branches in the unrolled loop
 #pragma unroll
               for (int b = 0; b < BT; ++b) {
-                if (b < B) {
-                  const uint4 q = reinterpret_cast<const uint4*>(q_nat + b * DIN)[ch];
-                  part[b] = dp4a_ss(w.x, q.x, part[b]);
-                  part[b] = dp4a_ss(w.y, q.y, part[b]);
-                  part[b] = dp4a_ss(w.z, q.z, part[b]);
-                  part[b] = dp4a_ss(w.w, q.w, part[b]);
-                }
+                const uint4 q = reinterpret_cast<const uint4*>(q_nat + b * DIN)[ch];
+                part[b] = dp4a_ss(w.x, q.x, part[b]);
+                part[b] = dp4a_ss(w.y, q.y, part[b]);
+                part[b] = dp4a_ss(w.z, q.z, part[b]);
+                part[b] = dp4a_ss(w.w, q.w, part[b]);
               }
             }
           } else {
+            // eight words of the W_B row in flight per lane before they are used
             const uint32_t* wb = reinterpret_cast<const uint32_t*>(L.lora_b + (size_t)r * DIN);
-#pragma unroll 8
-            for (int w = lane; w < DIN / 4; w += 32) {
-              const uint32_t wv = __ldg(wb + w);
+#pragma unroll 1
+            for (int w0 = lane; w0 < DIN / 4; w0 += 32 * 8) {  // DIN / 4 is a multiple of 256
+              uint32_t wv[8];
 #pragma unroll
-              for (int b = 0; b < BT; ++b)
-                if (b < B) part[b] = dp4a_ss(wv, reinterpret_cast<const uint32_t*>(q_nat + b * DIN)[w], part[b]);
+              for (int u = 0; u < 8; ++u) wv[u] = __ldg(wb + w0 + 32 * u);
+#pragma unroll
+              for (int u = 0; u < 8; ++u)
+#pragma unroll
+                for (int b = 0; b < BT; ++b)  // every slot, as above
+                  part[b] = dp4a_ss(wv[u], reinterpret_cast<const uint32_t*>(q_nat + b * DIN)[w0 + 32 * u], part[b]);
             }
           }
 #pragma unroll
@@ -639,8 +774,43 @@ __global__ void __launch_bounds__(NT, 1) stream_kernel(const __grid_constant__ P
     }
     if (!dead) {
       const uint4* tile = reinterpret_cast<const uint4*>(smem + (size_t)sb * TILE_BYTES);
-      int* acc = reinterpret_cast<int*>(pring + (size_t)sp * P_BYTES + P_ACC);
+      int* acc = reinterpret_cast<int*>(pring + (size_t)sp * PL.bytes + PL.acc);
       const int nr = min(TR, L.d_out - cu.t * TR);
+      if constexpr (TOKLOOP) {
+#pragma unroll 1
+        for (int ps = 0; ps < PASSES; ++ps) {
+          const int rr = ps * RPP + warp * RPW + rsub;
+          const bool valid = rr < nr;
+          const uint4 w = valid ? tile[rr * ROW16 + li] : make_uint4(0u, 0u, 0u, 0u);
+          const uint32_t w4[4] = {w.x, w.y, w.z, w.w};
+          uint32_t mw[32];  // bit k of every byte of word j, in place: the dp4a masks for all tokens
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+#pragma unroll
+            for (int k = 0; k < 8; ++k) mw[j * 8 + k] = w4[j] & (0x01010101u << k);
+          const uint4* q0 = reinterpret_cast<const uint4*>(q_perm) + li;
+#pragma unroll 2
+          for (int b = 0; b < B; ++b) {
+            const uint4* qp4 = q0 + b * q_tok(SEGS);
+            int acc8[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) acc8[k] = 0;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const uint4 qa = qp4[(2 * j) * q_row(SEGS)], qb = qp4[(2 * j + 1) * q_row(SEGS)];
+              const uint32_t qp[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
+#pragma unroll
+              for (int k = 0; k < 8; ++k) acc8[k] = dp4a_us(mw[j * 8 + k], qp[k], acc8[k]);
+            }
+            int S = 0;
+#pragma unroll
+            for (int k = 0; k < 8; ++k) S += acc8[k] * (1 << (7 - k));
+#pragma unroll
+            for (int o = LPR / 2; o > 0; o >>= 1) S += __shfl_xor_sync(0xffffffffu, S, o);
+            if (valid && (b % LPR) == li) acc[b * TR + rr] = (S >> 6) - s_sumq[b];  // 2 sum - sum q
+          }
+        }
+      } else {
 #pragma unroll
       for (int ps = 0; ps < PASSES; ++ps) {
         const int rr = ps * RPP + warp * RPW + rsub;
@@ -660,13 +830,14 @@ __global__ void __launch_bounds__(NT, 1) stream_kernel(const __grid_constant__ P
 #pragma unroll
           for (int o = LPR / 2; o > 0; o >>= 1) S[b] += __shfl_xor_sync(0xffffffffu, S[b], o);
         }
-        // lane b of the row group stores token b's accumulator
+        // lane b % LPR of the row group stores token b's accumulator
 #pragma unroll
         for (int b = 0; b < BT; ++b)
-          if (valid && b < B && li == b) acc[rr * MAX_B + b] = (S[b] >> 6) - sumq[b];  // 2 sum - sum q
+          if (valid && b < B && (b % LPR) == li) acc[b * TR + rr] = (S[b] >> 6) - sumq[b];  // 2 sum - sum q
+      }
       }
       if (tid < BT * R)
-        reinterpret_cast<double*>(pring + (size_t)sp * P_BYTES + P_TF)[tid] = tf_cur[tid / R][tid % R];
+        reinterpret_cast<double*>(pring + (size_t)sp * PL.bytes + PL.tf)[tid] = tf_cur[tid / R][tid % R];
     }
     __syncwarp();
     if (lane == 0) {
@@ -706,7 +877,9 @@ cudaError_t dispatch(const Params& p, int grid, cudaStream_t st) {
     case 8: return launch_t<8, 1, BT>(p, grid, st);
     case 16: return launch_t<16, 1, BT>(p, grid, st);
     case 32: return launch_t<32, 1, BT>(p, grid, st);
-    case 64: return launch_t<32, 2, BT>(p, grid, st);
+    case 64:
+      if constexpr (BT <= 4) return launch_t<32, 2, BT>(p, grid, st);
+      return cudaErrorInvalidValue;
     default: return cudaErrorInvalidValue;
   }
 }
@@ -714,7 +887,9 @@ cudaError_t dispatch(const Params& p, int grid, cudaStream_t st) {
 }  // namespace stream
 
 bool stream_supported(int d_in, int B) {
-  return B >= 1 && B <= stream::MAX_B && (d_in == 1024 || d_in == 2048 || d_in == 4096 || d_in == 8192);
+  if (B < 1 || B > stream::MAX_B) return false;
+  if (B <= 4) return d_in == 1024 || d_in == 2048 || d_in == 4096 || d_in == 8192;
+  return d_in == 1024 || d_in == 2048 || d_in == 4096;  // 16 token slots of codes must fit beside the rings
 }
 
 int stream_status_word(int** out) {
@@ -770,7 +945,9 @@ int launch_linear_stream(const dfssm_linear_t* lins, int n, const float* x, int 
   int st_rc = stream_status_word(&p.status);
   if (st_rc) return st_rc;
   const int grid = tiles < num_sms() ? tiles : num_sms();
-  const cudaError_t e = B == 1 ? stream::dispatch<1>(p, grid, st) : stream::dispatch<4>(p, grid, st);
+  const cudaError_t e = B == 1   ? stream::dispatch<1>(p, grid, st)
+                        : B <= 4 ? stream::dispatch<4>(p, grid, st)
+                                 : stream::dispatch<16>(p, grid, st);
   if (e != cudaSuccess) return record_cuda_failure(e);
   return DFSSM_OK;
 }

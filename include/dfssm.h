@@ -100,8 +100,9 @@ size_t dfssm_workspace_size(int op, int a, int b, int c);
  * Batch-B decode of one linear (scaffold GEMV + fused int8 LoRA), technical summary §2.B–C.
  *   x   device f32 [B][d_in] (16-byte aligned),  y device f32 [B][d_out]
  *   1 <= B <= 16.  dbg may be NULL.  workspace: dfssm_workspace_size(DFSSM_OP_LINEAR_DECODE, B, d_in, d_out).
- * For B <= 4 and d_in in {1024, 2048, 4096, 8192} the call is one kernel that quantizes x in every CTA
- * and streams the sign bits through shared memory; the workspace is then left untouched.  Otherwise a
+ * For d_in in {1024, 2048, 4096} (any B <= 16) and d_in = 8192 with B <= 4 the call is one kernel that
+ * quantizes x in every CTA and streams the sign bits through shared memory; the workspace is then left
+ * untouched.  Otherwise a
  * quantize kernel writes the codes into the workspace and a GEMV kernel reads them.
  */
 int dfssm_linear_decode(const dfssm_linear_t* lin, const float* x, int B, float* y, void* workspace,
@@ -113,7 +114,8 @@ int dfssm_linear_decode(const dfssm_linear_t* lin, const float* x, int B, float*
  * projections of one activation, or a stack of layer copies, stream their sign bits back to back).
  *   lins  host array of n descriptors (device pointers inside), all with the same d_in
  *   x     device f32 [B][d_in] (16-byte aligned);  ys host array of n device pointers, ys[j] f32 [B][d_out_j]
- *   1 <= n <= 64, 1 <= B <= 4, d_in in {1024, 2048, 4096, 8192}; other sizes return DFSSM_EUNSUPPORTED.
+ *   1 <= n <= 64; d_in in {1024, 2048, 4096} with 1 <= B <= 16, or d_in = 8192 with 1 <= B <= 4; other
+ *   sizes return DFSSM_EUNSUPPORTED.
  * No workspace.  The outputs must not overlap each other or x.
  */
 int dfssm_linear_decode_multi(const dfssm_linear_t* lins, int n, const float* x, int B, float* const* ys,
@@ -127,9 +129,9 @@ int dfssm_linear_decode_multi(const dfssm_linear_t* lins, int n, const float* x,
  * can block and synchronise the device.
  *   Limits: 1 <= B <= 16 and d_in <= 8192; larger sizes return DFSSM_EUNSUPPORTED before anything runs.
  *   Scratch: a fixed 132,608-byte array in the library's own device memory, held by every device that
- *   loads the library until the process exits.  The call allocates and frees nothing.  Calls with B <= 4
- *   and d_in in {1024, 2048, 4096, 8192} run the single streaming kernel of dfssm_linear_decode and use no
- *   scratch.
+ *   loads the library until the process exits.  The call allocates and frees nothing.  Calls in the
+ *   streaming kernel's range (d_in in {1024, 2048, 4096}, or d_in = 8192 with B <= 4) run that kernel and
+ *   use no scratch.
  *   Set-up: the first call on a device looks up that array's device address (cudaGetSymbolAddress, with
  *   that device current) and caches it; make that first call before any stream capture.
  *   Sharing: all calls on a device use the same array.  Each call writes everything it reads there, so
@@ -218,7 +220,7 @@ int dfssm_lm_head(const int8_t* W, const float* s_row, int V, int d, const float
  * shape) hands data between its CTAs through counters in the workspace; every wait has a clock budget
  * (about one second).  A wait that runs out makes every CTA of that launch return early (its outputs are
  * then incomplete) and records a sticky status word in the workspace; each new launch starts with fresh
- * counters.  The streaming linear kernels (dfssm_linear_decode at B <= 4, dfssm_linear_decode_multi)
+ * counters.  The streaming linear kernel (dfssm_linear_decode in its range, dfssm_linear_decode_multi)
  * bound their shared-memory pipeline waits the same way and record a timeout in a status word of the
  * library's own device memory (one per device).  dfssm_device_status synchronises `stream`, reads and
  * clears the workspace status word (workspace may be NULL: then only the library's word) and the

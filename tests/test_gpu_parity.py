@@ -83,7 +83,8 @@ def _rand_linear(seed, d_out, d_in, rank):
     (1, 32, 0, 1), (33, 64, 1, 2), (127, 96, 7, 3), (129, 160, 16, 5), (512, 256, 16, 16),
     (300, 384, 16, 4), (257, 1024, 16, 1), (1000, 8192, 16, 2), (8512, 2048, 16, 3),
     (2048, 4096, 16, 16), (77, 512, 16, 1), (1, 128, 0, 1), (640, 256, 5, 4), (8512, 2048, 16, 1),
-    (2048, 4096, 16, 4), (1100, 1024, 1, 2)])
+    (2048, 4096, 16, 4), (1100, 1024, 1, 2), (8512, 2048, 16, 5), (1030, 1024, 3, 9),
+    (8512, 2048, 16, 16), (4097, 4096, 16, 13), (300, 1024, 0, 16)])
 def test_linear_shapes(dev, d_out, d_in, rank, B):
     lin = _rand_linear(d_out * 7 + d_in + rank + B, d_out, d_in, rank)
     gen = np.random.default_rng(B)
@@ -133,18 +134,21 @@ def test_linear_full_stacks(dev, which):
                     assert assert_tol(y[b, rows], ry, f"{which} B{B} copy{c}") == 0
 
 
-@pytest.mark.parametrize("B", [1, 4])
-def test_linear_multi_matches_per_call(dev, B):
-    """dfssm_linear_decode_multi over the 48 in_proj copies equals 48 dfssm_linear_decode calls bit for
-    bit; copy 0 is checked in full and copy 47 on sampled rows against the oracle."""
+@pytest.mark.parametrize("which", ["in_proj", "out_proj"])
+@pytest.mark.parametrize("B", [1, 4, 16])
+def test_linear_multi_matches_per_call(dev, which, B):
+    """dfssm_linear_decode_multi over the 48 in_proj (or out_proj) copies equals 48 dfssm_linear_decode
+    calls bit for bit; copy 0 is checked in full and copy 47 on sampled rows against the oracle.  Each
+    CTA of the multi launch runs through many tiles, so every ring stage is reused several times."""
     from bit_quantized_mamba_b200 import dfssm
-    data = inputs.in_proj_stack()
+    data = (inputs.in_proj_stack if which == "in_proj" else inputs.out_proj_stack)()
     lins = [dfssm.Linear.from_host(l, dev) for l in data["linears"]]
     x = data["x"][:B]
     xd = to_dev(x, dev)
     ys = dfssm.linear_decode_multi(lins, xd)
     ref = [dfssm.linear_decode(L, xd) for L in lins]
     torch.cuda.synchronize()
+    assert dfssm.device_status() == 0  # no wait ran out of budget
     for c in range(len(lins)):
         assert torch.equal(ys[c], ref[c]), c
     r = oracle.linear_decode(oracle.Linear.from_dict(data["linears"][0]), x)
@@ -182,10 +186,10 @@ def test_linear_multi_rejects_unsupported(dev):
     with pytest.raises(dfssm.DfssmError) as e:
         dfssm.linear_decode_multi(lins, torch.zeros((1, 384), device=dev))
     assert e.value.status == -3  # d_in outside {1024, 2048, 4096, 8192}
-    lins = [dfssm.Linear.from_host(inputs.linear(g, 64, 256), dev)]
+    lins = [dfssm.Linear.from_host(inputs.linear(g, 64, 8192), dev)]
     with pytest.raises(dfssm.DfssmError) as e:
-        dfssm.linear_decode_multi(lins, torch.zeros((5, 256), device=dev))
-    assert e.value.status == -3  # B > 4
+        dfssm.linear_decode_multi(lins, torch.zeros((5, 8192), device=dev))
+    assert e.value.status == -3  # d_in 8192 takes at most 4 tokens
 
 
 def test_conv_step(dev):

@@ -34,9 +34,9 @@ def _taps(B, L, dev):
 
 def test_noalloc_matches_workspace_entry_point_on_two_calls(dev):
     from bit_quantized_mamba_b200 import dfssm
-    # calls in a row: an in_proj-shaped token (streaming kernel, no scratch), then eight out_proj tokens
-    # and three tokens of a d_in = 384 linear (both through the shared scratch array)
-    for seed, (d_out, d_in, B) in enumerate([(8512, 2048, 1), (2048, 4096, 8), (1000, 384, 3)]):
+    # calls in a row: an in_proj-shaped token (streaming kernel, no scratch), then eight tokens of a
+    # d_in = 8192 linear and three of a d_in = 384 linear (both through the shared scratch array)
+    for seed, (d_out, d_in, B) in enumerate([(8512, 2048, 1), (1000, 8192, 8), (1000, 384, 3)]):
         g = np.random.default_rng(100 + seed)
         L = dfssm.Linear.from_host(inputs.linear(g, d_out, d_in), dev)
         x = torch.from_numpy(inputs.normal(g, (B, d_in)) * np.float32(1.5)).to(dev)
