@@ -155,8 +155,11 @@ __global__ void expand_bits_kernel(const uint32_t* __restrict__ bits, int8_t* __
 
 // Quantization for the prefill: one warp per token.  Codes (natural order) and scale exactly as the
 // decode quantizer; the LoRA down-projection t = W_B q on the codes (int32, dp4a) with W_B staged in
-// shared memory, and tf = fl32(t sB s) rounded as in the decode path.
+// shared memory (zero rows beyond the rank, so every lane runs all sixteen rows without branches), and
+// tf = fl32(t sB s) rounded as in the decode path.  Each lane keeps eight 16-byte loads of its token in
+// flight.
 constexpr int QW = 8;  // tokens (warps) per CTA
+constexpr int QU = 8;  // float4 loads in flight per lane
 __global__ void __launch_bounds__(QW * 32) prefill_quant_kernel(const float* __restrict__ x, int M, int K,
                                                                const int8_t* __restrict__ lora_b,
                                                                const float* __restrict__ lora_b_scale,
@@ -165,18 +168,36 @@ __global__ void __launch_bounds__(QW * 32) prefill_quant_kernel(const float* __r
                                                                float* __restrict__ tf_out,
                                                                int8_t* dbg_xq, float* dbg_s, int32_t* dbg_t) {
   extern __shared__ __align__(16) unsigned char sm[];
-  int8_t* wb = reinterpret_cast<int8_t*>(sm);  // [rank][K]
+  int8_t* wb = reinterpret_cast<int8_t*>(sm);  // [16][K]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int i = threadIdx.x * 4; i < rank * K; i += blockDim.x * 4)
-    *reinterpret_cast<uint32_t*>(wb + i) = __ldg(reinterpret_cast<const uint32_t*>(lora_b + i));
+  // W_B into shared memory, eight 4-byte loads in flight per thread
+  for (int i0 = threadIdx.x * 4; i0 < DFSSM_MAX_RANK * K; i0 += 8 * QW * 32 * 4) {
+    uint32_t w[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int i = i0 + u * QW * 32 * 4;
+      w[u] = i < rank * K ? __ldg(reinterpret_cast<const uint32_t*>(lora_b + i)) : 0u;
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int i = i0 + u * QW * 32 * 4;
+      if (i < DFSSM_MAX_RANK * K) *reinterpret_cast<uint32_t*>(wb + i) = w[u];
+    }
+  }
   __syncthreads();
   const int m = blockIdx.x * QW + warp;
   if (m >= M) return;
-  const float* xr = x + (size_t)m * K;
+  const float4* xr = reinterpret_cast<const float4*>(x + (size_t)m * K);
+  const int K4 = K / 4;  // a multiple of 32: the bounds tests below are uniform over the warp
   float m_abs = 0.0f;
-  for (int i = lane * 4; i < K; i += 128) {
-    const float4 v = __ldg(reinterpret_cast<const float4*>(xr + i));
-    m_abs = fmaxf(m_abs, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
+  for (int i0 = lane; i0 < K4; i0 += 32 * QU) {
+    float4 v[QU];
+#pragma unroll
+    for (int u = 0; u < QU; ++u)
+      v[u] = i0 + 32 * u < K4 ? __ldg(xr + i0 + 32 * u) : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int u = 0; u < QU; ++u)
+      m_abs = fmaxf(m_abs, fmaxf(fmaxf(fabsf(v[u].x), fabsf(v[u].y)), fmaxf(fabsf(v[u].z), fabsf(v[u].w))));
   }
   m_abs = warp_max(m_abs);
   const float s0 = m_abs == 0.0f ? 0.0f : __fdiv_rn(m_abs, 127.0f);
@@ -184,20 +205,28 @@ __global__ void __launch_bounds__(QW * 32) prefill_quant_kernel(const float* __r
   int u[DFSSM_MAX_RANK];
 #pragma unroll
   for (int r = 0; r < DFSSM_MAX_RANK; ++r) u[r] = 0;
-  for (int i = lane * 4; i < K; i += 128) {
-    const float4 v = __ldg(reinterpret_cast<const float4*>(xr + i));
-    const float vv[4] = {v.x, v.y, v.z, v.w};
-    uint32_t packed = 0;
+  for (int i0 = lane; i0 < K4; i0 += 32 * QU) {
+    float4 v[QU];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int c = m_abs == 0.0f ? 0 : quant_code_fast(vv[j], s0, inv_s0);
-      packed |= (uint32_t)(uint8_t)(int8_t)c << (8 * j);
+    for (int q = 0; q < QU; ++q)
+      v[q] = i0 + 32 * q < K4 ? __ldg(xr + i0 + 32 * q) : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int q = 0; q < QU; ++q) {
+      const int i = i0 + 32 * q;
+      if (i < K4) {
+        const float vv[4] = {v[q].x, v[q].y, v[q].z, v[q].w};
+        int cd[4];
+        quant_codes<4>(vv, s0, inv_s0, cd);
+        uint32_t packed = 0;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) packed |= ((uint32_t)cd[j] & 0xFFu) << (8 * j);
+        reinterpret_cast<uint32_t*>(xq + (size_t)m * K)[i] = packed;
+        if (dbg_xq) reinterpret_cast<uint32_t*>(dbg_xq + (size_t)m * K)[i] = packed;
+#pragma unroll
+        for (int r = 0; r < DFSSM_MAX_RANK; ++r)
+          u[r] = dp4a_ss(reinterpret_cast<const uint32_t*>(wb + (size_t)r * K)[i], packed, u[r]);
+      }
     }
-    *reinterpret_cast<uint32_t*>(xq + (size_t)m * K + i) = packed;
-    if (dbg_xq) *reinterpret_cast<uint32_t*>(dbg_xq + (size_t)m * K + i) = packed;
-#pragma unroll
-    for (int r = 0; r < DFSSM_MAX_RANK; ++r)
-      if (r < rank) u[r] = dp4a_ss(*reinterpret_cast<const uint32_t*>(wb + (size_t)r * K + i), packed, u[r]);
   }
 #pragma unroll
   for (int r = 0; r < DFSSM_MAX_RANK; ++r) u[r] = __reduce_add_sync(0xffffffffu, u[r]);
@@ -223,7 +252,9 @@ __global__ void __launch_bounds__(QW * 32) prefill_quant_kernel(const float* __r
 constexpr int EPI_WARPS = 8;
 constexpr int PNT = 64 + EPI_WARPS * 32;   // 320 threads
 constexpr int PTMEM_COLS = 2 * BN;         // two 256-column accumulators
-constexpr size_t PSMEM_BYTES = (size_t)STAGES * STAGE_BYTES + 1024 + 512 + 2 * BN * (16 * 4 + 8);
+constexpr int STG_LD = 17;                 // staging row stride (floats): conflict-free both ways
+constexpr size_t PSMEM_BYTES =
+    (size_t)STAGES * STAGE_BYTES + 1024 + 512 + 2 * BN * (8 * 4 + 8) + EPI_WARPS * 32 * STG_LD * 4;
 
 __global__ void __launch_bounds__(PNT, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
@@ -236,10 +267,12 @@ __global__ void __launch_bounds__(PNT, 1)
   uint64_t* acc_full = empty + STAGES;     // [2] MMA -> epilogue
   uint64_t* acc_empty = acc_full + 2;      // [2] epilogue -> MMA
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(acc_empty + 2);
-  // per-accumulator column parameters of the tile being drained: W_A rows (as fp32), sW, sA
-  float* col_wa = reinterpret_cast<float*>(smem + STAGES * STAGE_BYTES + 512);      // [2][BN][16]
-  float* col_sw = col_wa + 2 * BN * 16;                                             // [2][BN]
+  // per-accumulator column parameters of the tile being drained: W_A rows as bf16 pairs (int8 values
+  // are exact in bf16; half the shared-memory reads of fp32), sW, sA
+  uint32_t* col_wa = reinterpret_cast<uint32_t*>(smem + STAGES * STAGE_BYTES + 512);  // [2][BN][8]
+  float* col_sw = reinterpret_cast<float*>(col_wa + 2 * BN * 8);                     // [2][BN]
   float* col_sa = col_sw + 2 * BN;                                                  // [2][BN]
+  float* stg_all = col_sa + 2 * BN;  // [EPI_WARPS][32][STG_LD]: a warp's 32 x 16 output chunk
   __shared__ int abort_flag;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -329,6 +362,7 @@ __global__ void __launch_bounds__(PNT, 1)
     const int q = warp & 3;
     const int half = e >> 2;
     const int etid = threadIdx.x - 64;  // 0..255
+    float* stg = stg_all + (size_t)e * 32 * STG_LD;
     int local = 0;
     for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++local) {
       const int buf = local & 1;
@@ -336,16 +370,25 @@ __global__ void __launch_bounds__(PNT, 1)
       // column parameters of this tile, staged once per tile by the 256 epilogue threads
       {
         const int n = n0 + etid;
-        float* wa_dst = col_wa + (size_t)(buf * BN + etid) * 16;
+        float wf[16];
         if (n < ep.N && ep.rank == DFSSM_MAX_RANK) {
           const uint4 w4 = __ldg(reinterpret_cast<const uint4*>(ep.la) + n);
           const uint32_t wv[4] = {w4.x, w4.y, w4.z, w4.w};
 #pragma unroll
-          for (int r = 0; r < 16; ++r) wa_dst[r] = int8_to_f32((int)(int8_t)(wv[r >> 2] >> (8 * (r & 3))));
+          for (int r = 0; r < 16; ++r) wf[r] = int8_to_f32((int)(int8_t)(wv[r >> 2] >> (8 * (r & 3))));
         } else {
+#pragma unroll
           for (int r = 0; r < 16; ++r)
-            wa_dst[r] = (n < ep.N && r < ep.rank) ? (float)ep.la[(size_t)n * ep.rank + r] : 0.0f;
+            wf[r] = (n < ep.N && r < ep.rank) ? (float)ep.la[(size_t)n * ep.rank + r] : 0.0f;
         }
+        // bf16 of a small integer: the upper half of its fp32 pattern (exact)
+        uint32_t pk[8];
+#pragma unroll
+        for (int r2 = 0; r2 < 8; ++r2)
+          pk[r2] = (__float_as_uint(wf[2 * r2]) >> 16) | (__float_as_uint(wf[2 * r2 + 1]) & 0xFFFF0000u);
+        uint4* wa_dst = reinterpret_cast<uint4*>(col_wa + (size_t)(buf * BN + etid) * 8);
+        wa_dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        wa_dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
         col_sw[buf * BN + etid] = n < ep.N ? __ldg(ep.w_scale + n) : 0.0f;
         col_sa[buf * BN + etid] = (n < ep.N && ep.rank > 0) ? __ldg(ep.la_scale + n) : 0.0f;
       }
@@ -380,33 +423,39 @@ __global__ void __launch_bounds__(PNT, 1)
         const int c0 = half * (BN / 2) + cc;
         uint32_t v[16];
         tmem_ld16(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * BN + c0), v);
-        if (m >= ep.M) continue;
         float out[16];
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
           const int cidx = buf * BN + c0 + j;
-          const float4* wa4 = reinterpret_cast<const float4*>(col_wa + (size_t)cidx * 16);
+          const uint4* wa4 = reinterpret_cast<const uint4*>(col_wa + (size_t)cidx * 8);
           float lora = 0.f;
 #pragma unroll
-          for (int r4 = 0; r4 < 4; ++r4) {
-            const float4 w = wa4[r4];
-            lora = fmaf(w.x, tfm[4 * r4], lora);
-            lora = fmaf(w.y, tfm[4 * r4 + 1], lora);
-            lora = fmaf(w.z, tfm[4 * r4 + 2], lora);
-            lora = fmaf(w.w, tfm[4 * r4 + 3], lora);
+          for (int h2 = 0; h2 < 2; ++h2) {
+            const uint4 w = wa4[h2];
+            const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              lora = fmaf(__uint_as_float(wv[k] << 16), tfm[8 * h2 + 2 * k], lora);
+              lora = fmaf(__uint_as_float(wv[k] & 0xFFFF0000u), tfm[8 * h2 + 2 * k + 1], lora);
+            }
           }
           const int acc = (int)v[j];
           out[j] = fmaf((float)acc, sm * col_sw[cidx], col_sa[cidx] * lora);
-          if (ep.acc && n0 + c0 + j < ep.N) ep.acc[(size_t)m * ep.N + n0 + c0 + j] = acc;
+          if (ep.acc && m < ep.M && n0 + c0 + j < ep.N) ep.acc[(size_t)m * ep.N + n0 + c0 + j] = acc;
         }
-        float* yrow = ep.y + (size_t)m * ep.N + n0 + c0;
-        if (n0 + c0 + 16 <= ep.N && (ep.N % 4) == 0) {
+        // through shared memory: lane l holds row l of the chunk; the stores then write two 64-byte row
+        // segments per instruction (lanes 0-15 one row, 16-31 the next)
 #pragma unroll
-          for (int j = 0; j < 16; j += 4)
-            *reinterpret_cast<float4*>(yrow + j) = make_float4(out[j], out[j + 1], out[j + 2], out[j + 3]);
-        } else {
-          for (int j = 0; j < 16 && n0 + c0 + j < ep.N; ++j) yrow[j] = out[j];
+        for (int j = 0; j < 16; ++j) stg[lane * STG_LD + j] = out[j];
+        __syncwarp();
+        const int cj = lane & 15, n = n0 + c0 + cj;
+#pragma unroll 4
+        for (int k = 0; k < 16; ++k) {
+          const int r = 2 * k + (lane >> 4);
+          const int mr = m0 + q * 32 + r;
+          if (mr < ep.M && n < ep.N) ep.y[(size_t)mr * ep.N + n] = stg[r * STG_LD + cj];
         }
+        __syncwarp();
       }
       // this warp's reads of the accumulator are complete: release it to the MMA warp
       asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
@@ -521,7 +570,7 @@ extern "C" int dfssm_linear_prefill(const dfssm_linear_t* lin, const float* x, i
   prefill::Ws w = prefill::carve(workspace, M, K, N);
 
   // 1. per-token quantization and LoRA down-projection (one warp per token)
-  const size_t qsmem = (size_t)lin->rank * K;
+  const size_t qsmem = (size_t)DFSSM_MAX_RANK * K;  // W_B padded to sixteen rows
   static bool qattr = false;
   if (!qattr) {
     const cudaError_t ea = cudaFuncSetAttribute(prefill::prefill_quant_kernel,
