@@ -5,17 +5,19 @@
 //   1. quantize every token (per-token absmax int8 codes, natural order, exactly as in decode) and its
 //      LoRA down-projection (fp32, one warp per token);
 //   2. expand the packed sign bits once to +-1 int8 rows in the workspace;
-//   3. acc[m][n] = sum_k q[m][k] w[n][k] on tcgen05.mma kind::i8 (128x256 tiles, K steps of 128 bytes,
-//      TMA loads with 128-byte swizzle into a 4-stage shared-memory ring, two TMEM accumulators in a
-//      persistent kernel), then the epilogue reads TMEM and writes
-//      y[m][n] = acc s[m] sW[n] + sA[n] sum_r W_A[n][r] tf[m][r] while the next tile accumulates.
-// The integer accumulators are exact; the epilogue is fp32 with fused multiply-add.
+//   3. acc[m][n] = sum_k q[m][k] w[n][k] on tcgen05.mma kind::i8 (128x128 tiles, K steps of 128 bytes,
+//      TMA loads with 128-byte swizzle into a 4-stage shared-memory ring, a persistent kernel), and
+//      the LoRA-up sum_r W_A[n][r] tf[m][r] on the tensor core as well (bf16 operands, fp32
+//      accumulation, tf split into two bf16 halves), then the epilogue reads both accumulators and writes
+//      y[m][n] = acc s[m] sW[n] + sA[n] lora[m][n] while the next tile accumulates.
+// The integer accumulators are exact; the LoRA-up and the epilogue are fp32.
 //
 // Every wait on an mbarrier is bounded: a wait that runs out of budget sets the workspace error word,
 // the CTA stops issuing work, waits (bounded) for its copies in flight, frees its tensor memory and
 // returns.
 
 #include <cuda.h>
+#include <cuda_bf16.h>
 #include <cudaTypedefs.h>
 
 #include <cstdio>
@@ -27,18 +29,22 @@
 namespace dfssm {
 namespace prefill {
 
-constexpr int BM = 128, BN = 256, BK = 128;  // tile; BK bytes = BK int8 elements
-constexpr int STAGES = 3;
-constexpr int UMMA_K = 32;                   // K of one kind::i8 MMA
+constexpr int BM = 128, BN = 128, BK = 128;  // tile; BK bytes = BK int8 elements
+constexpr int STAGES = 4;
+constexpr int UMMA_K = 32;                   // K of one kind::i8 MMA (bytes)
 constexpr int A_BYTES = BM * BK, B_BYTES = BN * BK, STAGE_BYTES = A_BYTES + B_BYTES;
+// LoRA-up on the tensor core: per tile, A_l = [tf_hi | tf_lo] of the tile's rows and B_l = [W_A | W_A] of
+// its columns, bf16, each row padded to 128 bytes (the 128-byte swizzle of the main operands); two
+// kind::f16 MMAs (K = 16 each) give sum_r W_A tf_hi + sum_r W_A tf_lo in an fp32 accumulator.
+constexpr int LROW = 128;                    // bytes per LoRA operand row (64 bf16, 32 used)
+constexpr int LA_BYTES = BM * LROW, LB_BYTES = BN * LROW, LSTAGE_BYTES = LA_BYTES + LB_BYTES;
+constexpr int UMMA_K16 = 32;                 // K of one kind::f16 MMA: 16 bf16 = 32 bytes
 constexpr long long kWaitBudget = 4000000000LL;  // clock cycles per wait (~2 s)
 
 struct EpiArgs {
   const float* s;       // [M] per-token scale
-  const float* tf;      // [M][16] LoRA intermediate
   const float* w_scale; // [N]
   const float* la_scale;// [N]
-  const int8_t* la;     // [N][rank]
   int rank;
   float* y;             // [M][N]
   int32_t* acc;         // [M][N] or null
@@ -100,6 +106,9 @@ __device__ __forceinline__ uint64_t umma_desc_k_sw128(uint32_t smem_addr) {
 // kind::i8 instruction descriptor: D s32, A s8, B s8, both K-major, M = BM, N = BN.
 constexpr uint32_t kIdesc = (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
                             ((uint32_t)(BM >> 4) << 24);
+// kind::f16 instruction descriptor: D f32, A bf16, B bf16, both K-major, M = BM, N = BN.
+constexpr uint32_t kIdescBf16 = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
+                                ((uint32_t)(BM >> 4) << 24);
 
 __device__ __forceinline__ void umma_i8(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t accum) {
   asm volatile(
@@ -107,6 +116,14 @@ __device__ __forceinline__ void umma_i8(uint32_t tmem_d, uint64_t adesc, uint64_
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
       "l"(adesc), "l"(bdesc), "r"(kIdesc), "r"(accum)
+      : "memory");
+}
+__device__ __forceinline__ void umma_bf16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t accum) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(kIdescBf16), "r"(accum)
       : "memory");
 }
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
@@ -166,6 +183,7 @@ __global__ void __launch_bounds__(QW * 32) prefill_quant_kernel(const float* __r
                                                                int rank, int8_t* __restrict__ xq,
                                                                float* __restrict__ s_out,
                                                                float* __restrict__ tf_out,
+                                                               uint16_t* __restrict__ tfhl,
                                                                int8_t* dbg_xq, float* dbg_s, int32_t* dbg_t) {
   extern __shared__ __align__(16) unsigned char sm[];
   int8_t* wb = reinterpret_cast<int8_t*>(sm);  // [16][K]
@@ -230,14 +248,25 @@ __global__ void __launch_bounds__(QW * 32) prefill_quant_kernel(const float* __r
   }
 #pragma unroll
   for (int r = 0; r < DFSSM_MAX_RANK; ++r) u[r] = __reduce_add_sync(0xffffffffu, u[r]);
+  float tf = 0.0f;
   if (lane < DFSSM_MAX_RANK) {
     int tv = 0;
 #pragma unroll
     for (int r = 0; r < DFSSM_MAX_RANK; ++r)
       if (r == lane) tv = u[r];
-    const float tf = lane < rank ? lora_tf(tv, __ldg(lora_b_scale + lane), s0) : 0.0f;
+    tf = lane < rank ? lora_tf(tv, __ldg(lora_b_scale + lane), s0) : 0.0f;
     tf_out[(size_t)m * DFSSM_MAX_RANK + lane] = tf;
     if (dbg_t && lane < rank) dbg_t[(size_t)m * rank + lane] = tv;
+  }
+  // the LoRA-up operand row of this token: [bf16(tf) | bf16(tf - bf16(tf)) | 0 ...] (64 bf16): the two
+  // halves sum to tf within 2^-16 relative; lane l < 16 writes hi[l], lane 16 + r writes lo[r]
+  {
+    const float tr = __shfl_sync(0xffffffffu, tf, lane & 15);
+    const __nv_bfloat16 hi = __float2bfloat16_rn(tr);
+    const __nv_bfloat16 lo = __float2bfloat16_rn(tr - __bfloat162float(hi));
+    uint16_t* row = tfhl + (size_t)m * (LROW / 2);
+    row[lane] = __bfloat16_as_ushort(lane < 16 ? hi : lo);
+    row[32 + lane] = 0;
   }
   if (lane == 0) {
     s_out[m] = s0;
@@ -245,34 +274,82 @@ __global__ void __launch_bounds__(QW * 32) prefill_quant_kernel(const float* __r
   }
 }
 
-// Persistent tcgen05 GEMM: one CTA per SM walks the output tiles; warp 0 streams A/B stages with TMA,
-// warp 1 issues the MMAs into one of two TMEM accumulators, warps 2..9 drain the other accumulator (two
-// warps per 32-lane TMEM quadrant, each taking half of the 256 columns), so a tile's epilogue overlaps
-// the next tile's main loop.
+// The LoRA-up operand row of output column n: [W_A[n] | W_A[n] | 0 ...] as 64 bf16 (int8 values are
+// exact in bf16; zero beyond the rank).  One thread per column.
+__global__ void lora_a_bf16_kernel(const int8_t* __restrict__ la, int rank, int N, uint4* __restrict__ out) {
+  const int n = blockIdx.x * blockDim.x + threadIdx.x;
+  if (n >= N) return;
+  int wv[16];
+  if (rank == 16) {  // one 16-byte row (16-byte aligned at rank 16)
+    const uint4 q = __ldg(reinterpret_cast<const uint4*>(la) + n);
+    const uint32_t qw[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+    for (int r = 0; r < 16; ++r) wv[r] = (int)(int8_t)(qw[r >> 2] >> (8 * (r & 3)));
+  } else {
+#pragma unroll
+    for (int r = 0; r < 16; ++r) wv[r] = r < rank ? (int)la[(size_t)n * rank + r] : 0;
+  }
+  uint32_t pk[8];
+#pragma unroll
+  for (int r2 = 0; r2 < 8; ++r2)
+    pk[r2] = (__float_as_uint(int8_to_f32(wv[2 * r2])) >> 16) |
+             (__float_as_uint(int8_to_f32(wv[2 * r2 + 1])) & 0xFFFF0000u);
+  uint4* dst = out + (size_t)n * (LROW / 16);
+  const uint4 a = make_uint4(pk[0], pk[1], pk[2], pk[3]), b = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+  const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+  dst[0] = a;
+  dst[1] = b;
+  dst[2] = a;
+  dst[3] = b;
+  dst[4] = z;
+  dst[5] = z;
+  dst[6] = z;
+  dst[7] = z;
+}
+
+// Persistent tcgen05 GEMM: one CTA per SM walks the 128 x 128 output tiles; warp 0 streams A/B stages
+// (and each tile's LoRA operands) with TMA, warp 1 issues the MMAs (the int8 scaffold product into one
+// of two int32 accumulators, then the LoRA-up into the matching fp32 accumulator), warps 2..9 drain the
+// other pair (two warps per 32-lane TMEM quadrant, each taking half of the 128 columns), so a tile's
+// epilogue overlaps the next tile's main loop.  TMEM columns: [0, 256) int32 accumulators, [256, 512)
+// fp32 LoRA accumulators.
 constexpr int EPI_WARPS = 8;
 constexpr int PNT = 64 + EPI_WARPS * 32;   // 320 threads
-constexpr int PTMEM_COLS = 2 * BN;         // two 256-column accumulators
+constexpr int PTMEM_COLS = 4 * BN;         // two (int32, fp32) accumulator pairs of BN columns
 constexpr int STG_LD = 17;                 // staging row stride (floats): conflict-free both ways
-constexpr size_t PSMEM_BYTES =
-    (size_t)STAGES * STAGE_BYTES + 1024 + 512 + 2 * BN * (8 * 4 + 8) + EPI_WARPS * 32 * STG_LD * 4;
+constexpr size_t OFF_LORA = (size_t)STAGES * STAGE_BYTES;
+constexpr size_t OFF_BARS = OFF_LORA + 2 * (size_t)LSTAGE_BYTES;
+constexpr size_t OFF_COLS = OFF_BARS + 512;
+constexpr size_t OFF_STG = OFF_COLS + 2 * BN * 8;
+constexpr size_t PSMEM_BYTES = 1024 + OFF_STG + EPI_WARPS * 32 * STG_LD * 4;
+
+// Bounded wait that ignores the abort flag (used to drain work already issued).
+__device__ __forceinline__ void mbar_wait_drain(uint64_t* bar, uint32_t parity) {
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity))
+    if (clock64() - t0 > kWaitBudget) return;
+}
 
 __global__ void __launch_bounds__(PNT, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
+                const __grid_constant__ CUtensorMap map_la, const __grid_constant__ CUtensorMap map_lb,
                 const EpiArgs ep) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+  unsigned char* lbase = smem + OFF_LORA;  // [2][LSTAGE_BYTES]
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + OFF_BARS);
   uint64_t* empty = full + STAGES;
   uint64_t* acc_full = empty + STAGES;     // [2] MMA -> epilogue
   uint64_t* acc_empty = acc_full + 2;      // [2] epilogue -> MMA
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(acc_empty + 2);
-  // per-accumulator column parameters of the tile being drained: W_A rows as bf16 pairs (int8 values
-  // are exact in bf16; half the shared-memory reads of fp32), sW, sA
-  uint32_t* col_wa = reinterpret_cast<uint32_t*>(smem + STAGES * STAGE_BYTES + 512);  // [2][BN][8]
-  float* col_sw = reinterpret_cast<float*>(col_wa + 2 * BN * 8);                     // [2][BN]
-  float* col_sa = col_sw + 2 * BN;                                                  // [2][BN]
-  float* stg_all = col_sa + 2 * BN;  // [EPI_WARPS][32][STG_LD]: a warp's 32 x 16 output chunk
+  uint64_t* lfull = acc_empty + 2;         // [2] LoRA operands landed
+  uint64_t* lempty = lfull + 2;            // [2] LoRA operands consumed by the MMAs
+  uint64_t* mma_done = lempty + 2;         // every MMA of this CTA complete
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(mma_done + 1);
+  // per-accumulator column parameters of the tile being drained: sW, sA
+  float* col_sw = reinterpret_cast<float*>(smem + OFF_COLS);  // [2][BN]
+  float* col_sa = col_sw + 2 * BN;                            // [2][BN]
+  float* stg_all = reinterpret_cast<float*>(smem + OFF_STG);  // [EPI_WARPS][32][STG_LD]
   __shared__ int abort_flag;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -289,7 +366,10 @@ __global__ void __launch_bounds__(PNT, 1)
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
       mbar_init(&acc_empty[b], EPI_WARPS);
+      mbar_init(&lfull[b], 1);
+      mbar_init(&lempty[b], 1);
     }
+    mbar_init(mma_done, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 1) {
@@ -305,11 +385,20 @@ __global__ void __launch_bounds__(PNT, 1)
   const uint32_t tmem_base = *tmem_holder;
 
   if (warp == 0 && lane == 0) {
-    // ---- TMA producer: k-blocks of every tile of this CTA, through the stage ring
-    int it = 0;
+    // ---- TMA producer: per tile its LoRA operands, then its k-blocks through the stage ring
+    int it = 0, lt = 0;
     bool ok = true;
-    for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
+    for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x, ++lt) {
       const int n0 = (t % tiles_n) * BN, m0 = (t / tiles_n) * BM;
+      const int lb = lt & 1;
+      if (lt >= 2 && !mbar_wait(&lempty[lb], ((lt >> 1) - 1) & 1, &abort_flag)) {
+        abort_flag = 1;
+        break;
+      }
+      unsigned char* ldst = lbase + lb * LSTAGE_BYTES;
+      mbar_expect_tx(&lfull[lb], LSTAGE_BYTES);
+      tma_load_2d(ldst, &map_la, 0, m0, &lfull[lb]);
+      tma_load_2d(ldst + LA_BYTES, &map_lb, 0, n0, &lfull[lb]);
       for (int kb = 0; kb < kblocks; ++kb, ++it) {
         const int s = it % STAGES;
         if (it >= STAGES && !mbar_wait(&empty[s], ((it / STAGES) - 1) & 1, &abort_flag)) {
@@ -323,13 +412,13 @@ __global__ void __launch_bounds__(PNT, 1)
         tma_load_2d(a_dst + A_BYTES, &map_b, kb * BK, n0, &full[s]);
       }
     }
-    // the last stages' copies land before this CTA may exit
-    for (int j = (it > STAGES ? it - STAGES : 0); j < it; ++j)
-      mbar_wait(&full[j % STAGES], (j / STAGES) & 1, &abort_flag);
+    // the last copies land before this CTA may exit
+    for (int j = (it > STAGES ? it - STAGES : 0); j < it; ++j) mbar_wait_drain(&full[j % STAGES], (j / STAGES) & 1);
+    for (int j = (lt > 2 ? lt - 2 : 0); j < lt; ++j) mbar_wait_drain(&lfull[j & 1], (j >> 1) & 1);
   } else if (warp == 1 && lane == 0) {
     // ---- MMA issuer
     int it = 0, local = 0;
-    bool ok = true;
+    bool ok = true, issued = false;
     for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x, ++local) {
       const int buf = local & 1;
       if (local >= 2 && !mbar_wait(&acc_empty[buf], ((local >> 1) - 1) & 1, &abort_flag)) {
@@ -338,6 +427,7 @@ __global__ void __launch_bounds__(PNT, 1)
       }
       asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
       const uint32_t d_tmem = tmem_base + (uint32_t)(buf * BN);
+      const uint32_t l_tmem = tmem_base + (uint32_t)(2 * BN + buf * BN);
       for (int kb = 0; kb < kblocks; ++kb, ++it) {
         const int s = it % STAGES;
         if (!mbar_wait(&full[s], (it / STAGES) & 1, &abort_flag)) {
@@ -353,8 +443,28 @@ __global__ void __launch_bounds__(PNT, 1)
           umma_i8(d_tmem, umma_desc_k_sw128(a_addr + kk * UMMA_K), umma_desc_k_sw128(b_addr + kk * UMMA_K),
                   (kb > 0 || kk > 0) ? 1u : 0u);
         umma_commit(&empty[s]);
+        issued = true;
       }
+      if (!ok) break;
+      // LoRA-up of the tile: [tf_hi | tf_lo] x [W_A | W_A]^T, fp32 accumulation
+      if (!mbar_wait(&lfull[buf], (local >> 1) & 1, &abort_flag)) {
+        abort_flag = 1;
+        break;
+      }
+      asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+      const uint32_t la_addr = smem_u32(lbase + buf * LSTAGE_BYTES);
+      const uint32_t lb_addr = la_addr + LA_BYTES;
+#pragma unroll
+      for (int kk = 0; kk < 2; ++kk)
+        umma_bf16(l_tmem, umma_desc_k_sw128(la_addr + kk * UMMA_K16), umma_desc_k_sw128(lb_addr + kk * UMMA_K16),
+                  kk > 0 ? 1u : 0u);
+      umma_commit(&lempty[buf]);
       umma_commit(&acc_full[buf]);
+    }
+    // every MMA this thread issued completes before the tensor memory is released
+    if (issued) {
+      umma_commit(mma_done);
+      mbar_wait_drain(mma_done, 0);
     }
   } else if (warp >= 2) {
     // ---- epilogue: warp e = warp - 2 drains TMEM lanes [32 (warp % 4), +32) and column half e / 4
@@ -367,52 +477,18 @@ __global__ void __launch_bounds__(PNT, 1)
     for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++local) {
       const int buf = local & 1;
       const int n0 = (t % tiles_n) * BN, m0 = (t / tiles_n) * BM;
-      // column parameters of this tile, staged once per tile by the 256 epilogue threads
-      {
+      // column scales of this tile, staged once per tile
+      if (etid < BN) {
         const int n = n0 + etid;
-        float wf[16];
-        if (n < ep.N && ep.rank == DFSSM_MAX_RANK) {
-          const uint4 w4 = __ldg(reinterpret_cast<const uint4*>(ep.la) + n);
-          const uint32_t wv[4] = {w4.x, w4.y, w4.z, w4.w};
-#pragma unroll
-          for (int r = 0; r < 16; ++r) wf[r] = int8_to_f32((int)(int8_t)(wv[r >> 2] >> (8 * (r & 3))));
-        } else {
-#pragma unroll
-          for (int r = 0; r < 16; ++r)
-            wf[r] = (n < ep.N && r < ep.rank) ? (float)ep.la[(size_t)n * ep.rank + r] : 0.0f;
-        }
-        // bf16 of a small integer: the upper half of its fp32 pattern (exact)
-        uint32_t pk[8];
-#pragma unroll
-        for (int r2 = 0; r2 < 8; ++r2)
-          pk[r2] = (__float_as_uint(wf[2 * r2]) >> 16) | (__float_as_uint(wf[2 * r2 + 1]) & 0xFFFF0000u);
-        uint4* wa_dst = reinterpret_cast<uint4*>(col_wa + (size_t)(buf * BN + etid) * 8);
-        wa_dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-        wa_dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
         col_sw[buf * BN + etid] = n < ep.N ? __ldg(ep.w_scale + n) : 0.0f;
         col_sa[buf * BN + etid] = (n < ep.N && ep.rank > 0) ? __ldg(ep.la_scale + n) : 0.0f;
       }
       asm volatile("bar.sync 1, %0;" ::"n"(EPI_WARPS * 32) : "memory");
       const int row = q * 32 + lane;
       const int m = m0 + row;
-      float sm = 0.f;
-      float tfm[DFSSM_MAX_RANK];
-#pragma unroll
-      for (int r = 0; r < DFSSM_MAX_RANK; ++r) tfm[r] = 0.f;
-      if (m < ep.M) {
-        sm = __ldg(ep.s + m);
-        const float4* tp = reinterpret_cast<const float4*>(ep.tf + (size_t)m * DFSSM_MAX_RANK);
-#pragma unroll
-        for (int r4 = 0; r4 < 4; ++r4) {
-          const float4 v = __ldg(tp + r4);
-          tfm[4 * r4] = v.x;
-          tfm[4 * r4 + 1] = v.y;
-          tfm[4 * r4 + 2] = v.z;
-          tfm[4 * r4 + 3] = v.w;
-        }
-      }
+      const float sm = m < ep.M ? __ldg(ep.s + m) : 0.f;
       // every epilogue warp runs every tile iteration (the named barrier above counts on it); after an
-      // abort the accumulator is simply not read
+      // abort the accumulators are simply not read
       const bool ok = !abort_flag && mbar_wait(&acc_full[buf], (local >> 1) & 1, &abort_flag);
       asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
       if (!ok) {
@@ -421,26 +497,15 @@ __global__ void __launch_bounds__(PNT, 1)
       }
       for (int cc = 0; ok && cc < BN / 2; cc += 16) {
         const int c0 = half * (BN / 2) + cc;
-        uint32_t v[16];
+        uint32_t v[16], lv[16];
         tmem_ld16(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * BN + c0), v);
+        tmem_ld16(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(2 * BN + buf * BN + c0), lv);
         float out[16];
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
           const int cidx = buf * BN + c0 + j;
-          const uint4* wa4 = reinterpret_cast<const uint4*>(col_wa + (size_t)cidx * 8);
-          float lora = 0.f;
-#pragma unroll
-          for (int h2 = 0; h2 < 2; ++h2) {
-            const uint4 w = wa4[h2];
-            const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              lora = fmaf(__uint_as_float(wv[k] << 16), tfm[8 * h2 + 2 * k], lora);
-              lora = fmaf(__uint_as_float(wv[k] & 0xFFFF0000u), tfm[8 * h2 + 2 * k + 1], lora);
-            }
-          }
           const int acc = (int)v[j];
-          out[j] = fmaf((float)acc, sm * col_sw[cidx], col_sa[cidx] * lora);
+          out[j] = fmaf((float)acc, sm * col_sw[cidx], col_sa[cidx] * __uint_as_float(lv[j]));
           if (ep.acc && m < ep.M && n0 + c0 + j < ep.N) ep.acc[(size_t)m * ep.N + n0 + c0 + j] = acc;
         }
         // through shared memory: lane l holds row l of the chunk; the stores then write two 64-byte row
@@ -457,7 +522,7 @@ __global__ void __launch_bounds__(PNT, 1)
         }
         __syncwarp();
       }
-      // this warp's reads of the accumulator are complete: release it to the MMA warp
+      // this warp's reads of the accumulators are complete: release them to the MMA warp
       asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
       __syncwarp();
       if (lane == 0)
@@ -512,12 +577,14 @@ struct Ws {
   int32_t* sumq;
   float* tf;
   int8_t* w8;
+  uint16_t* tfhl;  // [M][64] bf16 LoRA-up operand rows
+  uint4* la2;      // [N][64] bf16 LoRA-up operand rows
   int* err;
 };
 
 size_t ws_bytes(int M, int K, int N) {
   return al256((size_t)M * K) + al256((size_t)M * 4) * 2 + al256((size_t)M * 16 * 4) +
-         al256((size_t)N * K) + 256;
+         al256((size_t)N * K) + al256((size_t)M * LROW) + al256((size_t)N * LROW) + 256;
 }
 
 Ws carve(void* base, int M, int K, int N) {
@@ -533,6 +600,10 @@ Ws carve(void* base, int M, int K, int N) {
   p += al256((size_t)M * 16 * 4);
   w.w8 = reinterpret_cast<int8_t*>(p);
   p += al256((size_t)N * K);
+  w.tfhl = reinterpret_cast<uint16_t*>(p);
+  p += al256((size_t)M * LROW);
+  w.la2 = reinterpret_cast<uint4*>(p);
+  p += al256((size_t)N * LROW);
   w.err = reinterpret_cast<int*>(p);
   return w;
 }
@@ -579,27 +650,30 @@ extern "C" int dfssm_linear_prefill(const dfssm_linear_t* lin, const float* x, i
     qattr = true;
   }
   prefill::prefill_quant_kernel<<<(M + prefill::QW - 1) / prefill::QW, prefill::QW * 32, qsmem, st>>>(
-      x, M, K, lin->lora_b, lin->lora_b_scale, lin->rank, w.xq, w.s, w.tf, dbg ? dbg->xq : nullptr,
+      x, M, K, lin->lora_b, lin->lora_b_scale, lin->rank, w.xq, w.s, w.tf, w.tfhl, dbg ? dbg->xq : nullptr,
       dbg ? dbg->xscale : nullptr, dbg ? dbg->lora_t : nullptr);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return record_cuda_failure(e);
-  // 2. +-1 int8 weights
+  // 2. +-1 int8 weights, and W_A rows as the bf16 LoRA-up operand
   const long long words = (long long)N * (K / 32);
   prefill::expand_bits_kernel<<<(unsigned)((words + 255) / 256), 256, 0, st>>>(lin->bits, w.w8, words);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return record_cuda_failure(e);
+  prefill::lora_a_bf16_kernel<<<(N + 255) / 256, 256, 0, st>>>(lin->lora_a, lin->rank, N, w.la2);
   e = cudaGetLastError();
   if (e != cudaSuccess) return record_cuda_failure(e);
   e = cudaMemsetAsync(w.err, 0, sizeof(int), st);
   if (e != cudaSuccess) return record_cuda_failure(e);
   // 3. tcgen05 GEMM + epilogue
-  CUtensorMap map_a, map_b;
-  if (!prefill::make_map(&map_a, w.xq, M, K, prefill::BM) || !prefill::make_map(&map_b, w.w8, N, K, prefill::BN))
+  CUtensorMap map_a, map_b, map_la, map_lb;
+  if (!prefill::make_map(&map_a, w.xq, M, K, prefill::BM) || !prefill::make_map(&map_b, w.w8, N, K, prefill::BN) ||
+      !prefill::make_map(&map_la, w.tfhl, M, prefill::LROW, prefill::BM) ||
+      !prefill::make_map(&map_lb, w.la2, N, prefill::LROW, prefill::BN))
     return DFSSM_EUNSUPPORTED;
   prefill::EpiArgs ep{};
   ep.s = w.s;
-  ep.tf = w.tf;
   ep.w_scale = lin->w_scale;
   ep.la_scale = lin->lora_a_scale;
-  ep.la = lin->lora_a;
   ep.rank = lin->rank;
   ep.y = y;
   ep.acc = dbg ? dbg->acc : nullptr;
@@ -616,7 +690,7 @@ extern "C" int dfssm_linear_prefill(const dfssm_linear_t* lin, const float* x, i
   }
   const int tiles = ((N + prefill::BN - 1) / prefill::BN) * ((M + prefill::BM - 1) / prefill::BM);
   const int grid = tiles < num_sms() ? tiles : num_sms();
-  prefill::gemm_kernel<<<grid, prefill::PNT, prefill::PSMEM_BYTES, st>>>(map_a, map_b, ep);
+  prefill::gemm_kernel<<<grid, prefill::PNT, prefill::PSMEM_BYTES, st>>>(map_a, map_b, map_la, map_lb, ep);
   e = cudaGetLastError();
   if (e != cudaSuccess) return record_cuda_failure(e);
   return DFSSM_OK;
