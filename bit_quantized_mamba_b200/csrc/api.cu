@@ -407,23 +407,12 @@ int dfssm_lm_head(const int8_t* W, const float* s_row, int V, int d, const float
   if (!W || !s_row || !x || !logits || V < 1 || d < 16 || d % 16) return DFSSM_EINVAL;
   if (d > 8192) return DFSSM_EUNSUPPORTED;
   if (!aligned(W, 16) || !aligned(x, 4)) return DFSSM_EALIGN;
-  if (!workspace || !aligned(workspace, 256) || ws_bytes < dfssm::quant_scratch_bytes(1, d))
-    return DFSSM_EWORKSPACE;
+  (void)workspace;  // the kernel quantizes the token itself; the workspace is no longer used
+  (void)ws_bytes;
   if (!device_ok()) return DFSSM_EDEVICE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  dfssm::QuantScratch qs = dfssm::carve_quant_scratch(workspace, 1, d);
-  dfssm::QuantArgs qa{};
-  qa.x = x;
-  qa.ldx = d;
-  qa.n = d;
-  qa.B = 1;
-  qa.rank = 0;
-  qa.permute = false;
-  qa.out = qs;
-  cudaError_t e = dfssm::launch_quant(qa, s);
-  if (e != cudaSuccess) return cuda_fail(e);
-  dfssm::Int8GemvArgs ia{W, s_row, V, d, qs, logits, acc};
-  e = dfssm::launch_int8_gemv(ia, s);
+  dfssm::Int8GemvArgs ia{W, s_row, V, d, x, logits, acc};
+  const cudaError_t e = dfssm::launch_int8_gemv(ia, s);
   return e == cudaSuccess ? DFSSM_OK : cuda_fail(e);
 }
 

@@ -86,7 +86,7 @@ struct Int8GemvArgs {
   const int8_t* W;
   const float* s_row;
   int V, d;
-  QuantScratch in;          // natural-order codes of one token
+  const float* x;           // the token, fp32 [d] (quantized by every CTA of the kernel)
   float* logits;
   int32_t* acc;
 };

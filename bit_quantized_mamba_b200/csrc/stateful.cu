@@ -122,43 +122,107 @@ cudaError_t launch_ssm(const SsmArgs& a, cudaStream_t st) {
 
 // ------------------------------------------------------------------------------ int8 LM-head GEMV
 // logits[v] = fl32(acc[v] * s * s_row[v]) (fp64, this order), acc[v] = sum_i W[v,i] q_i (int32 exact).
-// One warp per row; each lane streams 16-byte chunks of the row and accumulates 4 dp4a per chunk.
+// Every CTA quantizes the token itself (per-token absmax int8, the decode quantizer: no separate launch
+// and no hand-off).  Each warp owns a contiguous, balanced range of rows and streams it as units of 2 KB
+// (four 16-byte chunks per lane of one row), always with the next unit's loads in flight while the current
+// one is summed; the first unit is requested before the quantizer runs, so its latency is hidden.  The
+// stream rate is set by the number of resident threads (1024 per SM), not by the loads per thread.
 
-__global__ void __launch_bounds__(256) int8_gemv_kernel(Int8GemvArgs a) {
+constexpr int LMH_U = 4;  // chunks per lane per unit (a unit is 32 x 4 x 16 B = 2 KB of one row)
+constexpr int LMH_CTAS_PER_SM = 4;  // 1024 streaming threads per SM
+__global__ void __launch_bounds__(256, LMH_CTAS_PER_SM) int8_gemv_kernel(Int8GemvArgs a) {
   extern __shared__ __align__(16) unsigned char smem[];
   uint4* qsm = reinterpret_cast<uint4*>(smem);
+  __shared__ float red[8];
   const int lane = threadIdx.x & 31;
   const int warps_total = gridDim.x * (blockDim.x >> 5);
   const int warp_g = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int chunks = a.d >> 4;
+  const int G = (chunks + 32 * LMH_U - 1) / (32 * LMH_U);  // units per row
+  const int r0 = (int)((long long)warp_g * a.V / warps_total);
+  const int r1 = (int)((long long)(warp_g + 1) * a.V / warps_total);
+  const int n_units = (r1 - r0) * G;
+  // unit j: row r0 + j / G, chunks g * 128 + lane + 32 u (g = j % G)
+  const auto load_unit = [&](int j, uint4 (&x)[LMH_U]) {
+    const int row = r0 + j / G, g = j - (j / G) * G;
+    const uint4* w = reinterpret_cast<const uint4*>(a.W + (size_t)row * a.d);
+#pragma unroll
+    for (int u = 0; u < LMH_U; ++u) {
+      const int c = g * 32 * LMH_U + lane + 32 * u;
+      x[u] = (j < n_units && c < chunks) ? ld_stream_u4(w + c) : make_uint4(0u, 0u, 0u, 0u);
+    }
+  };
+  uint4 cur[LMH_U];
+  load_unit(0, cur);  // weights do not depend on the token: in flight during the quantizer
   pdl_launch_dependents();
   pdl_wait();
-  const uint4* qsrc = reinterpret_cast<const uint4*>(a.in.q);
-  for (int i = threadIdx.x; i < chunks; i += blockDim.x) qsm[i] = qsrc[i];
+  // quantize the token (two passes over x, 8 KB for d = 2048): thread t takes inputs t + 256 k
+  float m = 0.0f;
+  for (int k0 = 0; k0 * 256 < a.d; k0 += 8) {
+    float v[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const int i = threadIdx.x + 256 * (k0 + k);
+      v[k] = i < a.d ? __ldg(a.x + i) : 0.0f;
+    }
+#pragma unroll
+    for (int k = 0; k < 8; ++k) m = fmaxf(m, fabsf(v[k]));
+  }
+  m = warp_max(m);
+  if (lane == 0) red[threadIdx.x >> 5] = m;
   __syncthreads();
-  const float s = a.in.s[0];
-  for (int row = warp_g; row < a.V; row += warps_total) {
-    const uint4* wrow = reinterpret_cast<const uint4*>(a.W + (size_t)row * a.d);
-    int acc = 0;
-    for (int c = lane; c < chunks; c += 32) {
-      const uint4 w = ld_stream_u4(wrow + c);
-      const uint4 q = qsm[c];
-      acc = dp4a_ss(w.x, q.x, acc);
-      acc = dp4a_ss(w.y, q.y, acc);
-      acc = dp4a_ss(w.z, q.z, acc);
-      acc = dp4a_ss(w.w, q.w, acc);
+  m = 0.0f;
+#pragma unroll
+  for (int w = 0; w < 8; ++w) m = fmaxf(m, red[w]);
+  const float s = m == 0.0f ? 0.0f : __fdiv_rn(m, 127.0f);
+  const float inv_s = m == 0.0f ? 0.0f : __frcp_rn(s);
+  int8_t* qb = reinterpret_cast<int8_t*>(smem);
+  for (int k0 = 0; k0 * 256 < a.d; k0 += 8) {
+    float vv[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const int i = threadIdx.x + 256 * (k0 + k);
+      vv[k] = i < a.d ? __ldg(a.x + i) : 0.0f;
     }
-    acc = warp_sum(acc);
-    if (lane == 0) {
-      a.logits[row] =
-          __double2float_rn(dmul(dmul((double)acc, (double)s), (double)a.s_row[row]));
-      if (a.acc) a.acc[row] = acc;
+    int cd[8];
+    quant_codes<8>(vv, s, inv_s, cd);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const int i = threadIdx.x + 256 * (k0 + k);
+      if (i < a.d) qb[i] = (int8_t)cd[k];
     }
+  }
+  __syncthreads();
+  int acc = 0;
+  for (int j = 0; j < n_units; ++j) {
+    uint4 nxt[LMH_U];
+    load_unit(j + 1, nxt);
+    const int g = j % G;
+#pragma unroll
+    for (int u = 0; u < LMH_U; ++u) {
+      const int c = g * 32 * LMH_U + lane + 32 * u;
+      const uint4 q = c < chunks ? qsm[c] : make_uint4(0u, 0u, 0u, 0u);
+      acc = dp4a_ss(cur[u].x, q.x, acc);
+      acc = dp4a_ss(cur[u].y, q.y, acc);
+      acc = dp4a_ss(cur[u].z, q.z, acc);
+      acc = dp4a_ss(cur[u].w, q.w, acc);
+    }
+    if (g == G - 1) {
+      const int row = r0 + j / G;
+      acc = warp_sum(acc);
+      if (lane == 0) {
+        a.logits[row] = __double2float_rn(dmul(dmul((double)acc, (double)s), (double)a.s_row[row]));
+        if (a.acc) a.acc[row] = acc;
+      }
+      acc = 0;
+    }
+#pragma unroll
+    for (int u = 0; u < LMH_U; ++u) cur[u] = nxt[u];
   }
 }
 
 cudaError_t launch_int8_gemv(const Int8GemvArgs& a, cudaStream_t st) {
-  const int blocks = num_sms() * 8;
+  const int blocks = num_sms() * LMH_CTAS_PER_SM;  // all resident: each CTA quantizes x once
   return launch_pdl(int8_gemv_kernel, dim3(blocks), dim3(256), (size_t)a.d, st, a);
 }
 

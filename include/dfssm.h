@@ -209,8 +209,11 @@ int dfssm_layer_decode(const dfssm_layer_t* layers, int n_layers, const dfssm_di
 /*
  * Int8 LM head on one token (technical summary §2.B: int8 LM head with per-row scaling).
  *   W device i8 [V][d] (16-byte aligned, d % 16 == 0), s_row device f32 [V], x device f32 [d],
- *   logits device f32 [V].   logits[v] = fl32(acc[v] s s_row[v]), acc[v] = sum_i W[v,i] q[i].
- *   acc (device i32 [V]) may be NULL.  workspace: dfssm_workspace_size(DFSSM_OP_LM_HEAD, 1, d, V).
+ *   logits device f32 [V].   logits[v] = fl32(acc[v] s s_row[v]), acc[v] = sum_i W[v,i] q[i], with
+ *   (q, s) the per-token absmax int8 quantization of x (as in dfssm_linear_decode).  d <= 8192.
+ *   acc (device i32 [V]) may be NULL.  One kernel: every CTA quantizes x itself, so the call needs no
+ *   scratch; workspace and ws_bytes are not read (may be NULL / 0; dfssm_workspace_size still reports the
+ *   size earlier versions used).
  */
 int dfssm_lm_head(const int8_t* W, const float* s_row, int V, int d, const float* x, float* logits,
                   int32_t* acc, void* workspace, size_t ws_bytes, void* stream);
