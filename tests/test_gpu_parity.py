@@ -303,6 +303,25 @@ def test_lm_head(dev):
     assert assert_tol(logits, rl, "lm head") == 0
 
 
+@pytest.mark.parametrize("V,d,zero", [(1, 16, False), (37, 4096, False), (5003, 8192, False), (300, 2048, True),
+                                       (70001, 512, False)])
+def test_lm_head_shapes(dev, V, d, zero):
+    """Other widths (the in-kernel quantizer's loop edges), row counts below and above one row pair per
+    warp, and an all-zero token (s = 0, every code 0, logits 0)."""
+    from bit_quantized_mamba_b200 import dfssm
+    g = np.random.default_rng(V * 31 + d)
+    W = g.integers(-127, 128, size=(V, d), dtype=np.int8)
+    s_row = g.uniform(1e-4, 1e-3, size=V).astype(np.float32)
+    x = np.zeros(d, np.float32) if zero else inputs.normal(g, (d,))
+    acc = torch.zeros(V, dtype=torch.int32, device=dev)
+    logits = dfssm.lm_head(to_dev(W, dev), to_dev(s_row, dev), to_dev(x, dev), acc=acc).cpu().numpy()
+    rl, racc = oracle.lm_head(W, s_row, x)
+    assert np.array_equal(acc.cpu().numpy(), racc)
+    assert assert_tol(logits, rl, f"lm head {V}x{d}") == 0
+    if zero:
+        assert not logits.any()
+
+
 FULL = dict(d_model=2048, nheads=64, headdim=64, d_state=128, ngroups=1)
 
 
