@@ -39,8 +39,9 @@ constexpr int NCW = 16;                  // GEMV warps
 constexpr int NEW = 6;                   // epilogue warps
 constexpr int PROD_WARP = NCW + NEW;     // producer warp
 constexpr int NT = (NCW + NEW + 1) * 32;
-constexpr int TILE_BYTES = 16384;        // packed bits per tile
-constexpr int MAX_TR = 128;              // rows per tile (d_in >= 1024)
+// Packed bits per tile (tb): 16 KB, or 32 KB with one token slot when a launch has more tiles than SMs
+// (half the per-tile hand-offs per byte; more token slots need the shared memory for their codes).
+constexpr int MAX_TR = 256;              // rows per tile (d_in >= 1024)
 constexpr int MAX_B = 16;
 constexpr int R = DFSSM_MAX_RANK;
 constexpr int MAX_NS = 8;                // stages per ring (bits ring and parameter ring alike)
@@ -64,11 +65,11 @@ __device__ __forceinline__ int q_index(int i) {
 struct PLayout {
   int sw, sa, acc, tf, bytes;
 };
-__host__ __device__ constexpr int rows_per_tile(int din) { return TILE_BYTES / (din / 8); }
-__host__ __device__ constexpr PLayout p_layout(int din, int bt) {
-  return PLayout{rows_per_tile(din) * 16, rows_per_tile(din) * 20, rows_per_tile(din) * 24,
-                 rows_per_tile(din) * 24 + rows_per_tile(din) * bt * 4,
-                 rows_per_tile(din) * 24 + rows_per_tile(din) * bt * 4 + bt * R * 8};
+__host__ __device__ constexpr int rows_per_tile(int din, int tb) { return tb / (din / 8); }
+__host__ __device__ constexpr PLayout p_layout(int din, int bt, int tb) {
+  return PLayout{rows_per_tile(din, tb) * 16, rows_per_tile(din, tb) * 20, rows_per_tile(din, tb) * 24,
+                 rows_per_tile(din, tb) * 24 + rows_per_tile(din, tb) * bt * 4,
+                 rows_per_tile(din, tb) * 24 + rows_per_tile(din, tb) * bt * 4 + bt * R * 8};
 }
 constexpr int MAX_LIN = DFSSM_MAX_LAYERS;
 constexpr long long kWaitBudget = 2000000000LL;  // clock cycles per wait (~1 s)
@@ -174,21 +175,27 @@ __device__ __forceinline__ void prefetch_range(const void* p, size_t bytes, int 
 
 // Dynamic shared memory: the bits ring, the parameter ring (ns stages each), W_B of the current linear
 // when it fits, and the codes in both layouts.  W_B in shared memory is preferred (it takes the LoRA-down
-// off global-memory latency) as long as at least 6 stages remain; then the largest stage count <= 8.
+// off global-memory latency) as long as ~96 KB of bits stay in flight; then the largest stage count <= 8.
 constexpr size_t kSmemBudget = 215 * 1024;
-__host__ __device__ constexpr size_t base_smem(int din, int bt, int ns) {
-  return (size_t)ns * (TILE_BYTES + p_layout(din, bt).bytes) + (size_t)bt * (q_tok_bytes(din) + din);
+__host__ __device__ constexpr size_t base_smem(int din, int bt, int ns, int tb) {
+  return (size_t)ns * (tb + p_layout(din, bt, tb).bytes) + (size_t)bt * (q_tok_bytes(din) + din);
 }
-__host__ __device__ constexpr bool fits(int din, int bt, int ns, bool wb) {
-  return base_smem(din, bt, ns) + (wb ? (size_t)R * din : 0) <= kSmemBudget;
+__host__ __device__ constexpr bool fits(int din, int bt, int ns, bool wb, int tb) {
+  return base_smem(din, bt, ns, tb) + (wb ? (size_t)R * din : 0) <= kSmemBudget;
 }
-__host__ __device__ constexpr bool wb_in_smem(int din, int bt) { return fits(din, bt, 6, true); }
-__host__ __device__ constexpr int n_stages(int din, int bt) {
-  return fits(din, bt, 8, wb_in_smem(din, bt)) ? 8 : fits(din, bt, 7, wb_in_smem(din, bt)) ? 7
-         : fits(din, bt, 6, wb_in_smem(din, bt)) ? 6 : fits(din, bt, 5, wb_in_smem(din, bt)) ? 5 : 4;
+// W_B stays in shared memory if at least ~96 KB of sign bits remain in flight beside it
+__host__ __device__ constexpr bool wb_in_smem(int din, int bt, int tb) {
+  return fits(din, bt, tb >= 32768 ? 4 : 6, true, tb);
 }
-__host__ __device__ constexpr size_t smem_bytes(int din, int bt) {
-  return base_smem(din, bt, n_stages(din, bt)) + (wb_in_smem(din, bt) ? (size_t)R * din : 0);
+__host__ __device__ constexpr int n_stages(int din, int bt, int tb) {
+  return fits(din, bt, 8, wb_in_smem(din, bt, tb), tb)   ? 8
+         : fits(din, bt, 7, wb_in_smem(din, bt, tb), tb) ? 7
+         : fits(din, bt, 6, wb_in_smem(din, bt, tb), tb) ? 6
+         : fits(din, bt, 5, wb_in_smem(din, bt, tb), tb) ? 5
+                                                         : 4;
+}
+__host__ __device__ constexpr size_t smem_bytes(int din, int bt, int tb) {
+  return base_smem(din, bt, n_stages(din, bt, tb), tb) + (wb_in_smem(din, bt, tb) ? (size_t)R * din : 0);
 }
 
 // Position in the CTA's contiguous tile range: linear j, tile t of that linear.
@@ -266,19 +273,20 @@ __device__ __forceinline__ int bits_dot_regs(uint4 w, const uint4 (&q)[8]) {
 // Warps 0..15 quantize x, compute the LoRA-down at each linear and accumulate the scaffold rows of every
 // stage into the accumulator ring; warps 16..21 turn accumulators into outputs (fp64 epilogue); warp 22
 // streams the stages.
-template <int LPR, int NSEG, int BT>
+template <int LPR, int NSEG, int BT, int TB>
 __global__ void __launch_bounds__(NT, 1) stream_kernel(const __grid_constant__ Params p) {
   constexpr int SEGS = LPR * NSEG;
   constexpr int DIN = 128 * SEGS;
   constexpr int ROW16 = DIN / 128;             // 16-byte chunks of packed bits per row
   constexpr int RPW = 32 / LPR;                // rows per warp per pass
   constexpr int RPP = NCW * RPW;               // rows per pass
-  constexpr int TR = rows_per_tile(DIN);      // rows per tile
-  constexpr PLayout PL = p_layout(DIN, BT);
+  constexpr int TILE_BYTES = TB;
+  constexpr int TR = rows_per_tile(DIN, TB);  // rows per tile
+  constexpr PLayout PL = p_layout(DIN, BT, TB);
   constexpr int PASSES = TR / RPP;
   static_assert(PASSES >= 1 && PASSES * RPP == TR && TR <= MAX_TR, "tile shape");
-  constexpr bool WB_SMEM = wb_in_smem(DIN, BT);
-  constexpr int NS = n_stages(DIN, BT);
+  constexpr bool WB_SMEM = wb_in_smem(DIN, BT, TB);
+  constexpr int NS = n_stages(DIN, BT, TB);
   constexpr int XPT = DIN / (NCW * 32);                    // x values per GEMV thread per token
   constexpr bool XREG = BT * XPT <= 16;                    // keep x in registers between the two passes
   constexpr bool REGQ = BT == 1 && NSEG == 1;              // one token: the lane's codes live in registers
@@ -850,11 +858,11 @@ __global__ void __launch_bounds__(NT, 1) stream_kernel(const __grid_constant__ P
 // Module status word: kTimeoutCode after a wait ran out of budget (sticky until read).
 static __device__ int g_stream_status;
 
-template <int LPR, int NSEG, int BT>
+template <int LPR, int NSEG, int BT, int TB>
 cudaError_t launch_t(const Params& p, int grid, cudaStream_t st) {
   constexpr int DIN = 128 * LPR * NSEG;
-  constexpr size_t smem = smem_bytes(DIN, BT);
-  auto k = stream_kernel<LPR, NSEG, BT>;
+  constexpr size_t smem = smem_bytes(DIN, BT, TB);
+  auto k = stream_kernel<LPR, NSEG, BT, TB>;
   // once per instantiation, not per launch, so that launches can be captured in a CUDA graph
   static const cudaError_t set = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (set != cudaSuccess) return set;
@@ -871,14 +879,14 @@ cudaError_t launch_t(const Params& p, int grid, cudaStream_t st) {
   return cudaLaunchKernelEx(&cfg, k, p);
 }
 
-template <int BT>
+template <int BT, int TB>
 cudaError_t dispatch(const Params& p, int grid, cudaStream_t st) {
   switch (p.d_in / 128) {
-    case 8: return launch_t<8, 1, BT>(p, grid, st);
-    case 16: return launch_t<16, 1, BT>(p, grid, st);
-    case 32: return launch_t<32, 1, BT>(p, grid, st);
+    case 8: return launch_t<8, 1, BT, TB>(p, grid, st);
+    case 16: return launch_t<16, 1, BT, TB>(p, grid, st);
+    case 32: return launch_t<32, 1, BT, TB>(p, grid, st);
     case 64:
-      if constexpr (BT <= 4) return launch_t<32, 2, BT>(p, grid, st);
+      if constexpr (BT <= 4) return launch_t<32, 2, BT, TB>(p, grid, st);
       return cudaErrorInvalidValue;
     default: return cudaErrorInvalidValue;
   }
@@ -914,7 +922,12 @@ int launch_linear_stream(const dfssm_linear_t* lins, int n, const float* x, int 
                          const dfssm_debug_t* dbg, cudaStream_t st) {
   stream::Params p;
   const int d_in = lins[0].d_in;
-  const int tile_rows = stream::TILE_BYTES / (d_in / 8);
+  // tile size: 32 KB with one token slot when 16 KB tiles would outnumber the SMs, else 16 KB
+  int tiles16 = 0;
+  for (int j = 0; j < n; ++j) tiles16 += (lins[j].d_out + stream::rows_per_tile(d_in, 16384) - 1) /
+                                         stream::rows_per_tile(d_in, 16384);
+  const int tb = (B == 1 && tiles16 > num_sms()) ? 32768 : 16384;
+  const int tile_rows = stream::rows_per_tile(d_in, tb);
   int tiles = 0;
   for (int j = 0; j < n; ++j) {
     const dfssm_linear_t& L = lins[j];
@@ -945,9 +958,10 @@ int launch_linear_stream(const dfssm_linear_t* lins, int n, const float* x, int 
   int st_rc = stream_status_word(&p.status);
   if (st_rc) return st_rc;
   const int grid = tiles < num_sms() ? tiles : num_sms();
-  const cudaError_t e = B == 1   ? stream::dispatch<1>(p, grid, st)
-                        : B <= 4 ? stream::dispatch<4>(p, grid, st)
-                                 : stream::dispatch<16>(p, grid, st);
+  const cudaError_t e = B == 1   ? (tb == 32768 ? stream::dispatch<1, 32768>(p, grid, st)
+                                                : stream::dispatch<1, 16384>(p, grid, st))
+                        : B <= 4 ? stream::dispatch<4, 16384>(p, grid, st)
+                                 : stream::dispatch<16, 16384>(p, grid, st);
   if (e != cudaSuccess) return record_cuda_failure(e);
   return DFSSM_OK;
 }
