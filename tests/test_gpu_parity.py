@@ -179,6 +179,28 @@ def test_linear_multi_mixed_shapes(dev):
         assert assert_tol(ys[j].cpu().numpy(), r["y"], f"mixed linear {j}") == 0
 
 
+@pytest.mark.parametrize("d_in,shapes", [
+    (1024, [(12000, 16), (8000, 16), (129, 0), (300, 3)]),
+    (8192, [(2000, 16), (1000, 5), (17, 16)])])
+def test_linear_multi_large_tiles(dev, d_in, shapes):
+    """Batch 1 with more 16 KB tiles than SMs: the launch streams 32 KB tiles (256 rows at d_in 1024, 32 at
+    8192).  Every output equals the single call's (16 KB tiles) bit for bit and the oracle within
+    tolerance."""
+    from bit_quantized_mamba_b200 import dfssm
+    hosts = [_rand_linear(90 + j, d_out, d_in, rank) for j, (d_out, rank) in enumerate(shapes)]
+    lins = [dfssm.Linear.from_host(h, dev) for h in hosts]
+    x = inputs.normal(np.random.default_rng(d_in), (1, d_in))
+    xd = to_dev(x, dev)
+    ys = dfssm.linear_decode_multi(lins, xd)
+    ref = [dfssm.linear_decode(L, xd) for L in lins]
+    torch.cuda.synchronize()
+    assert dfssm.device_status() == 0
+    for j, h in enumerate(hosts):
+        assert torch.equal(ys[j], ref[j]), j
+        r = oracle.linear_decode(oracle.Linear.from_dict(h), x)
+        assert assert_tol(ys[j].cpu().numpy(), r["y"], f"large-tile linear {j}") == 0
+
+
 def test_linear_multi_rejects_unsupported(dev):
     from bit_quantized_mamba_b200 import dfssm
     g = np.random.default_rng(8)
