@@ -269,6 +269,37 @@ __device__ __forceinline__ int bits_dot_regs(uint4 w, const uint4 (&q)[8]) {
   return S;
 }
 
+// Row sums of P passes held by the LPR lanes of a row group (each lane one partial per pass): after the
+// call, lane li holds the full sum of pass pass_of(li).  Each butterfly stage sends the half of the
+// passes that the partner keeps, so P passes cost log2(P) extra values instead of P full reductions.
+template <int P, int LPR>
+__device__ __forceinline__ int pass_of(int li) {
+  if constexpr (P == 1) return 0;
+  else if constexpr (P == 2) return (li & (LPR / 2)) ? 1 : 0;
+  else return ((li & (LPR / 2)) ? 2 : 0) + ((li & (LPR / 4)) ? 1 : 0);
+}
+template <int P, int LPR>
+__device__ __forceinline__ int reduce_passes(const int (&S)[P], int li) {
+  static_assert(P == 1 || P == 2 || P == 4, "one, two or four passes");
+  static_assert(LPR >= 2 * P, "row group too small");
+  int v;
+  if constexpr (P == 1) {
+    v = S[0];
+  } else if constexpr (P == 2) {
+    const bool hi = (li & (LPR / 2)) != 0;
+    v = (hi ? S[1] : S[0]) + __shfl_xor_sync(0xffffffffu, hi ? S[0] : S[1], LPR / 2);
+  } else {
+    const bool hi = (li & (LPR / 2)) != 0;
+    const int t0 = (hi ? S[2] : S[0]) + __shfl_xor_sync(0xffffffffu, hi ? S[0] : S[2], LPR / 2);
+    const int t1 = (hi ? S[3] : S[1]) + __shfl_xor_sync(0xffffffffu, hi ? S[1] : S[3], LPR / 2);
+    const bool hi2 = (li & (LPR / 4)) != 0;
+    v = (hi2 ? t1 : t0) + __shfl_xor_sync(0xffffffffu, hi2 ? t0 : t1, LPR / 4);
+  }
+#pragma unroll
+  for (int o = LPR / (2 * P); o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
 // LPR lanes per row, NSEG 16-byte segments per lane (d_in = 128 LPR NSEG >= 1024), BT token slots.
 // Warps 0..15 quantize x, compute the LoRA-down at each linear and accumulate the scaffold rows of every
 // stage into the accumulator ring; warps 16..21 turn accumulators into outputs (fp64 epilogue); warp 22
@@ -818,6 +849,32 @@ __global__ void __launch_bounds__(NT, 1) stream_kernel(const __grid_constant__ P
             if (valid && (b % LPR) == li) acc[b * TR + rr] = (S >> 6) - s_sumq[b];  // 2 sum - sum q
           }
         }
+      } else if constexpr (BT == 1) {
+        // one token: every pass's partial sum first, then one transposed reduction over the row group
+        // (a few shuffles for all passes instead of a full reduction per pass)
+        int Sp[PASSES];
+#pragma unroll
+        for (int ps = 0; ps < PASSES; ++ps) {
+          const int rr = ps * RPP + warp * RPW + rsub;
+          const bool valid = rr < nr;
+          int Sv = 0;
+#pragma unroll
+          for (int sg = 0; sg < NSEG; ++sg) {
+            const int seg = sg * LPR + li;
+            const uint4 w = valid ? tile[rr * ROW16 + seg] : make_uint4(0u, 0u, 0u, 0u);
+            if constexpr (REGQ) {
+              Sv += bits_dot_regs(w, qreg);
+            } else {
+              int St[1] = {0};
+              bits_dot_tokens<SEGS, 1>(w, reinterpret_cast<const uint4*>(q_perm) + seg, 1, St);
+              Sv += St[0];
+            }
+          }
+          Sp[ps] = Sv;
+        }
+        const int Sr = reduce_passes<PASSES, LPR>(Sp, li);
+        const int rr = pass_of<PASSES, LPR>(li) * RPP + warp * RPW + rsub;
+        if ((li & (LPR / PASSES - 1)) == 0 && rr < nr) acc[rr] = (Sr >> 6) - sumq[0];  // 2 sum - sum q
       } else {
 #pragma unroll
       for (int ps = 0; ps < PASSES; ++ps) {
