@@ -188,7 +188,23 @@ __global__ void __launch_bounds__(QW * 32) prefill_quant_kernel(const float* __r
   extern __shared__ __align__(16) unsigned char sm[];
   int8_t* wb = reinterpret_cast<int8_t*>(sm);  // [16][K]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // W_B into shared memory, eight 4-byte loads in flight per thread
+  // W_B into shared memory: 16-byte loads when W_B is 16-byte aligned (rank K is a multiple of 16),
+  // else eight 4-byte loads in flight per thread
+  if ((reinterpret_cast<uintptr_t>(lora_b) & 15) == 0) {
+    for (int i0 = threadIdx.x * 16; i0 < DFSSM_MAX_RANK * K; i0 += 8 * QW * 32 * 16) {
+      uint4 w[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int i = i0 + u * QW * 32 * 16;
+        w[u] = i < rank * K ? __ldg(reinterpret_cast<const uint4*>(lora_b + i)) : make_uint4(0u, 0u, 0u, 0u);
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int i = i0 + u * QW * 32 * 16;
+        if (i < DFSSM_MAX_RANK * K) *reinterpret_cast<uint4*>(wb + i) = w[u];
+      }
+    }
+  } else
   for (int i0 = threadIdx.x * 4; i0 < DFSSM_MAX_RANK * K; i0 += 8 * QW * 32 * 4) {
     uint32_t w[8];
 #pragma unroll
@@ -207,14 +223,15 @@ __global__ void __launch_bounds__(QW * 32) prefill_quant_kernel(const float* __r
   if (m >= M) return;
   const float4* xr = reinterpret_cast<const float4*>(x + (size_t)m * K);
   const int K4 = K / 4;  // a multiple of 32: the bounds tests below are uniform over the warp
+  constexpr int UB = QU;  // float4 per lane per batch
   float m_abs = 0.0f;
-  for (int i0 = lane; i0 < K4; i0 += 32 * QU) {
-    float4 v[QU];
+  for (int i0 = lane; i0 < K4; i0 += 32 * UB) {
+    float4 v[UB];
 #pragma unroll
-    for (int u = 0; u < QU; ++u)
+    for (int u = 0; u < UB; ++u)
       v[u] = i0 + 32 * u < K4 ? __ldg(xr + i0 + 32 * u) : make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-    for (int u = 0; u < QU; ++u)
+    for (int u = 0; u < UB; ++u)
       m_abs = fmaxf(m_abs, fmaxf(fmaxf(fabsf(v[u].x), fabsf(v[u].y)), fmaxf(fabsf(v[u].z), fabsf(v[u].w))));
   }
   m_abs = warp_max(m_abs);
@@ -223,13 +240,13 @@ __global__ void __launch_bounds__(QW * 32) prefill_quant_kernel(const float* __r
   int u[DFSSM_MAX_RANK];
 #pragma unroll
   for (int r = 0; r < DFSSM_MAX_RANK; ++r) u[r] = 0;
-  for (int i0 = lane; i0 < K4; i0 += 32 * QU) {
-    float4 v[QU];
+  for (int i0 = lane; i0 < K4; i0 += 32 * UB) {
+    float4 v[UB];
 #pragma unroll
-    for (int q = 0; q < QU; ++q)
+    for (int q = 0; q < UB; ++q)
       v[q] = i0 + 32 * q < K4 ? __ldg(xr + i0 + 32 * q) : make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-    for (int q = 0; q < QU; ++q) {
+    for (int q = 0; q < UB; ++q) {
       const int i = i0 + 32 * q;
       if (i < K4) {
         const float vv[4] = {v[q].x, v[q].y, v[q].z, v[q].w};
@@ -275,36 +292,33 @@ __global__ void __launch_bounds__(QW * 32) prefill_quant_kernel(const float* __r
 }
 
 // The LoRA-up operand row of output column n: [W_A[n] | W_A[n] | 0 ...] as 64 bf16 (int8 values are
-// exact in bf16; zero beyond the rank).  One thread per column.
+// exact in bf16; zero beyond the rank).  One thread per 16-byte chunk of a row (eight per row): chunks 0/1
+// and 2/3 hold W_A[n][0..7] / W_A[n][8..15], chunks 4..7 are zero.
 __global__ void lora_a_bf16_kernel(const int8_t* __restrict__ la, int rank, int N, uint4* __restrict__ out) {
-  const int n = blockIdx.x * blockDim.x + threadIdx.x;
-  if (n >= N) return;
-  int wv[16];
-  if (rank == 16) {  // one 16-byte row (16-byte aligned at rank 16)
-    const uint4 q = __ldg(reinterpret_cast<const uint4*>(la) + n);
-    const uint32_t qw[4] = {q.x, q.y, q.z, q.w};
+  const long long t = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (t >= 8LL * N) return;
+  const int n = (int)(t >> 3), ch = (int)(t & 7);
+  uint4 o = make_uint4(0u, 0u, 0u, 0u);
+  if (ch < 4) {
+    const int r0 = 8 * (ch & 1);
+    int wv[8];
+    if (rank == 16) {  // 16-byte aligned rows at rank 16
+      const uint2 q = __ldg(reinterpret_cast<const uint2*>(la + (size_t)n * 16 + r0));
+      const uint32_t qw[2] = {q.x, q.y};
 #pragma unroll
-    for (int r = 0; r < 16; ++r) wv[r] = (int)(int8_t)(qw[r >> 2] >> (8 * (r & 3)));
-  } else {
+      for (int r = 0; r < 8; ++r) wv[r] = (int)(int8_t)(qw[r >> 2] >> (8 * (r & 3)));
+    } else {
 #pragma unroll
-    for (int r = 0; r < 16; ++r) wv[r] = r < rank ? (int)la[(size_t)n * rank + r] : 0;
+      for (int r = 0; r < 8; ++r) wv[r] = r0 + r < rank ? (int)la[(size_t)n * rank + r0 + r] : 0;
+    }
+    uint32_t pk[4];
+#pragma unroll
+    for (int r2 = 0; r2 < 4; ++r2)
+      pk[r2] = (__float_as_uint(int8_to_f32(wv[2 * r2])) >> 16) |
+               (__float_as_uint(int8_to_f32(wv[2 * r2 + 1])) & 0xFFFF0000u);
+    o = make_uint4(pk[0], pk[1], pk[2], pk[3]);
   }
-  uint32_t pk[8];
-#pragma unroll
-  for (int r2 = 0; r2 < 8; ++r2)
-    pk[r2] = (__float_as_uint(int8_to_f32(wv[2 * r2])) >> 16) |
-             (__float_as_uint(int8_to_f32(wv[2 * r2 + 1])) & 0xFFFF0000u);
-  uint4* dst = out + (size_t)n * (LROW / 16);
-  const uint4 a = make_uint4(pk[0], pk[1], pk[2], pk[3]), b = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-  const uint4 z = make_uint4(0u, 0u, 0u, 0u);
-  dst[0] = a;
-  dst[1] = b;
-  dst[2] = a;
-  dst[3] = b;
-  dst[4] = z;
-  dst[5] = z;
-  dst[6] = z;
-  dst[7] = z;
+  out[(size_t)n * (LROW / 16) + ch] = o;
 }
 
 // Persistent tcgen05 GEMM: one CTA per SM walks the 128 x 128 output tiles; warp 0 streams A/B stages
@@ -659,7 +673,7 @@ extern "C" int dfssm_linear_prefill(const dfssm_linear_t* lin, const float* x, i
   prefill::expand_bits_kernel<<<(unsigned)((words + 255) / 256), 256, 0, st>>>(lin->bits, w.w8, words);
   e = cudaGetLastError();
   if (e != cudaSuccess) return record_cuda_failure(e);
-  prefill::lora_a_bf16_kernel<<<(N + 255) / 256, 256, 0, st>>>(lin->lora_a, lin->rank, N, w.la2);
+  prefill::lora_a_bf16_kernel<<<(unsigned)((8LL * N + 255) / 256), 256, 0, st>>>(lin->lora_a, lin->rank, N, w.la2);
   e = cudaGetLastError();
   if (e != cudaSuccess) return record_cuda_failure(e);
   e = cudaMemsetAsync(w.err, 0, sizeof(int), st);
