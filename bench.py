@@ -181,7 +181,7 @@ def run_ours(args, rank, world, local_rank):
     import numpy as np
     import torch
     import torch.distributed as dist
-    from bit_quantized_mamba_b200 import build, dfssm, inputs
+    from bit_quantized_mamba_b200 import build, dfssm, inputs, replicas
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
@@ -191,15 +191,10 @@ def run_ours(args, rank, world, local_rank):
         dist.barrier()
 
     def barrier():
-        if world > 1:
-            dist.barrier()
+        replicas.barrier(world)
 
     def max_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return replicas.max_over_ranks(x, world, dev)
 
     # ---- model, states, embeddings (seeded; identical replica on every rank)
     model = inputs.decode_model(seed=3)
@@ -269,7 +264,7 @@ def run_ours(args, rank, world, local_rank):
     ms = start.elapsed_time(end)
     ms = max_over_ranks(ms)
     ms_per_step = ms / args.steps
-    value = world * N_TOKENS * args.steps / (ms / 1e3)
+    value = replicas.whole_job_rate(N_TOKENS * args.steps, world, ms / 1e3)
 
     # ---- end to end through the public API: pinned host embeddings in, final hidden state out
     out_host = torch.empty((1, 2048), dtype=torch.float32).pin_memory()
@@ -293,7 +288,7 @@ def run_ours(args, rank, world, local_rank):
         e1.record()
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1))
-    e2e_value = world * N_TOKENS * e2e_steps / (e2e_ms / 1e3)
+    e2e_value = replicas.whole_job_rate(N_TOKENS * e2e_steps, world, e2e_ms / 1e3)
 
     # ---- scaffold GEMV sweep: 48 in_proj / out_proj copies through dfssm_linear_decode, captured in
     # a CUDA graph (48 calls = 96 kernels, PDL-chained); L2 flushed before each timed replay
