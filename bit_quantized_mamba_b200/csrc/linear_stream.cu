@@ -4,8 +4,9 @@
 //
 // At batch <= 16 the scaffold product is a matrix-vector product (ALU-bound beyond a few tokens), so
 // one persistent, warp-specialised kernel does everything for any number of linears that read the same x:
-//   * the rows of all linears are cut into 16 KB tiles of packed bits; each CTA takes a contiguous range
-//     of tiles.  A producer warp streams every tile into a ring of shared-memory stages and its rows' W_A
+//   * the rows of all linears are cut into tiles of packed bits (16 KB; 32 KB at one token slot when the
+//     launch has more 16 KB tiles than SMs); each CTA takes a contiguous range of tiles.  A producer warp
+//     streams every tile into a ring of shared-memory stages and its rows' W_A
 //     and scales into a second ring, with bulk asynchronous copies (cp.async.bulk, completion counted on
 //     mbarriers), several tiles ahead, and copies each linear's W_B ahead of that linear's first tile;
 //     a bits stage is refilled as soon as the GEMV warps have read it, a parameter stage once its
@@ -15,9 +16,11 @@
 //     codes in registers), compute each linear's LoRA-down t = W_B q (exact int32, dp4a) and
 //     tf = fl32(t sB s), and turn every stage into int32 accumulators
 //     acc = 2 sum_{bit=1} q - sum q (one AND and one dp4a per four weights);
-//   * six epilogue warps turn each stage's accumulators into y = fl32(acc s sW + sA sum_r W_A tf) (the
-//     fp64 epilogue shared by every path) while the GEMV warps already work on the next stages, and
-//     release the stage to the producer.
+//   * up to six epilogue warps (never more than ring stages) turn each stage's accumulators into
+//     y = fl32(acc s sW + sA sum_r W_A tf) (the fp64 epilogue shared by every path) while the GEMV warps
+//     already work on the next stages, and release the stage to the producer.
+// Template parameters: LPR lanes per row and NSEG 16-byte segments per lane (d_in = 128 LPR NSEG), BT
+// token slots (1, 4 or 16), TB tile bytes.
 // The linear descriptors are copied into shared memory at the start, so the hot loops never index the
 // kernel's parameter block with a run-time index.
 // The sign bits are immutable weights, so the producer starts streaming before the kernel waits on the
@@ -300,10 +303,10 @@ __device__ __forceinline__ int reduce_passes(const int (&S)[P], int li) {
   return v;
 }
 
-// LPR lanes per row, NSEG 16-byte segments per lane (d_in = 128 LPR NSEG >= 1024), BT token slots.
-// Warps 0..15 quantize x, compute the LoRA-down at each linear and accumulate the scaffold rows of every
-// stage into the accumulator ring; warps 16..21 turn accumulators into outputs (fp64 epilogue); warp 22
-// streams the stages.
+// LPR lanes per row, NSEG 16-byte segments per lane (d_in = 128 LPR NSEG >= 1024), BT token slots, TB
+// bytes of sign bits per tile.  Warps 0..15 quantize x, compute the LoRA-down at each linear and accumulate
+// the scaffold rows of every stage into the accumulator ring; warps 16..21 (the first NEP of them) turn
+// accumulators into outputs (fp64 epilogue); warp 22 streams the stages.
 template <int LPR, int NSEG, int BT, int TB>
 __global__ void __launch_bounds__(NT, 1) stream_kernel(const __grid_constant__ Params p) {
   constexpr int SEGS = LPR * NSEG;
