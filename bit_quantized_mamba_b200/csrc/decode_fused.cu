@@ -34,6 +34,7 @@ constexpr int MAX_IN = 64, MAX_OUT = 16, MAX_SSM = 32;
 constexpr int MIN_CTAS = 137, MAX_CTAS = 256;  // >= 137: at most 15 out_proj rows per CTA
 static_assert(NW == R, "one warp per LoRA row");
 constexpr int kPrefetchThread = 32;     // warp 1 issues the next layer's L2 prefetches
+constexpr int kCopyThread = 64;         // warp 2 issues the layer's bulk copies (thread 0 polls)
 constexpr int kChainWarp = NW - 1;      // warp 15 computes the fp64 scale chain (no out_proj row)
 constexpr int kChainBase = kChainWarp * 32;
 
@@ -450,9 +451,10 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ P
       cp_async4(&in_sa[tid], Lp.in_las + row);
       cp_async16(in_wa[tid], Lp.in_la + (size_t)row * R);
     }
-    if (tid == 0) {
+    if (tid == kCopyThread) {
       // the contiguous ranges every CTA needs, one bulk copy each; every generic access of the previous
-      // layer to these buffers is ordered before them by the barrier that ended that layer
+      // layer to these buffers is ordered before them by the barrier that ended that layer.  Issued by a
+      // thread other than the poller of the h hand-off, so that polling starts at once.
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       // first in the copy queue: the next layer's SSM state rows of this CTA (their buffer was last
       // read in layer l - 1)
