@@ -164,9 +164,9 @@ def run_reference(args, rank):
 # ---------------------------------------------------------------------------------- our arm
 
 # DRAM traffic of one decode_kernel launch (dram__bytes_read.sum + dram__bytes_write.sum, one ncu capture
-# of the fourth launch of `bench.py --ncu --warmup 3`: 280.90 MB + 57.09 MB), valid only for the kernel
+# of the fourth launch of `bench.py --ncu --warmup 3`: 280.58 MB + 57.18 MB), valid only for the kernel
 # source it was measured on; reported as null once that source changes.
-TRAFFIC_MEASURED = {"sha": "e6412b781a11", "bytes": 340_589_056}
+TRAFFIC_MEASURED = {"sha": "941fff55c4bb", "bytes": 337_766_912}
 
 
 def src_sha(*names):
