@@ -16,6 +16,8 @@ no distribution is given):
   A_log                          U(0, 2.7);   dt_bias U(-4, -1)
   D skip*                        U(0.5, 1.5); RMSNorm weights* U(0.5, 1.5)
   LM head W                      int8 uniform on [-127, 127];  row scales* U(1e-4, 1e-3)
+  tied embedding / LM head*      one int8 matrix as the LM head;  final RMSNorm weight* U(0.5, 1.5)
+  first token of a generation*   uniform on [0, vocab)
 """
 from __future__ import annotations
 
@@ -124,6 +126,20 @@ def prefill(seed: int = 4, m: int = 2048, vocab: int = VOCAB) -> dict:
     lm_w = g.integers(-127, 128, size=(vocab, D_MODEL), dtype=np.int8)
     lm_s = g.uniform(1e-4, 1e-3, size=vocab).astype(np.float32)
     return dict(x_in=x_in, x_out=x_out, in_proj=in_proj, out_proj=out_proj, lm_w=lm_w, lm_s=lm_s)
+
+
+def generation_model(seed: int = 5, n_layers: int = N_LAYERS, vocab: int = VOCAB, **dims) -> dict:
+    """A stack of layers plus the tied int8 embedding / LM head [vocab x d_model] with its row scales,
+    the final RMSNorm weight and a first token, for greedy generation."""
+    g = rng(seed)
+    layers = [layer(g, **dims) for _ in range(n_layers)]
+    d_model = dims.get("d_model", D_MODEL)
+    emb_w = g.integers(-127, 128, size=(vocab, d_model), dtype=np.int8)
+    emb_s = g.uniform(1e-4, 1e-3, size=vocab).astype(np.float32)
+    final_norm_w = g.uniform(0.5, 1.5, size=d_model).astype(np.float32)
+    first_token = int(g.integers(0, vocab))
+    return dict(layers=layers, emb_w=emb_w, emb_s=emb_s, final_norm_w=final_norm_w,
+                first_token=first_token)
 
 
 def zero_states(batch: int = 1, n_layers: int = N_LAYERS, nheads: int = N_HEADS,

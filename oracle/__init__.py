@@ -44,6 +44,9 @@ def _declare(L):
     L.oracle_gate.argtypes = [_P, _P, _P, _I]
     L.oracle_layer_decode.argtypes = [_I] * 7 + [_P] * 12 + [_P] * 7 + [_P] * 3 + [_P, _P]
     L.oracle_lm_head.argtypes = [_P, _P, _I, _I, _P, _P, _I, _P, _P]
+    L.oracle_embed.argtypes = [_P, _P, _I, _I, _I, _P]
+    L.oracle_embed.restype = _I
+    L.oracle_final_head.argtypes = [_P, _P, _I, _I, _P, _P, _P, _I, _P, _P]
 
 
 def _p(a):
@@ -245,3 +248,56 @@ def lm_head(W, s_row, x, rows=None):
     acc = np.zeros(n, np.int32)
     lib().oracle_lm_head(_p(W), _p(s_row), V, d, _p(x), _p(rp), n, _p(logits), _p(acc))
     return logits, acc
+
+
+def embed(W, s_row, token: int):
+    """Row `token` of the tied int8 embedding, dequantized: fl32(W[token] * s_row[token])."""
+    W = _c(W, np.int8)
+    V, d = W.shape
+    s_row = _c(s_row, np.float32)
+    e = np.zeros(d, np.float32)
+    if lib().oracle_embed(_p(W), _p(s_row), V, d, int(token), _p(e)) != 0:
+        raise IndexError(f"token {token} outside [0, {V})")
+    return e
+
+
+def final_head(W, s_row, h, norm_w=None, rows=None):
+    """Final RMSNorm (folded into the quantizer; None: no norm) + int8 LM head on one token h [d].
+    Returns (logits, acc) for all rows or the listed rows."""
+    W = _c(W, np.int8)
+    V, d = W.shape
+    s_row = _c(s_row, np.float32)
+    h = _c(h, np.float32).reshape(d)
+    nw = None if norm_w is None else _c(norm_w, np.float32).reshape(d)
+    rp = None if rows is None else _c(rows, np.int32)
+    n = V if rows is None else len(rp)
+    logits = np.zeros(n, np.float32)
+    acc = np.zeros(n, np.int32)
+    lib().oracle_final_head(_p(W), _p(s_row), V, d, _p(h), _p(nw), _p(rp), n, _p(logits), _p(acc))
+    return logits, acc
+
+
+def greedy(logits) -> int:
+    """Greedy choice: the index of the largest logit, the smallest such index on ties."""
+    return int(np.argmax(np.asarray(logits)))
+
+
+def generate(layers, W, s_row, final_norm_w, first_token: int, n_tokens: int, conv_states,
+             ssm_states, forced_tokens=None):
+    """Greedy generation, batch 1: each step embeds the current token, runs every layer (states
+    updated in place), applies the final head and takes the greedy choice as the next token.
+    forced_tokens (optional, length n_tokens + 1) feeds those tokens instead of the oracle's own
+    choices (teacher forcing).  Returns (tokens [n_tokens + 1], hidden [n_tokens][d] after the last
+    layer, logits [n_tokens][V])."""
+    tokens = [int(first_token)]
+    hid, lg = [], []
+    for t in range(n_tokens):
+        cur = tokens[-1] if forced_tokens is None else int(forced_tokens[t])
+        h = embed(W, s_row, cur)[None, :].copy()
+        for L, cs, ss in zip(layers, conv_states, ssm_states):
+            layer_decode(L, h, cs, ss)
+        hid.append(h[0].copy())
+        logits, _ = final_head(W, s_row, h[0], final_norm_w)
+        lg.append(logits)
+        tokens.append(greedy(logits))
+    return tokens, np.stack(hid), np.stack(lg)

@@ -129,7 +129,7 @@ inline double silu64(double v) { return v / (1.0 + std::exp(-v)); }
 
 extern "C" {
 
-int oracle_abi_version(void) { return 3; }
+int oracle_abi_version(void) { return 4; }
 
 // Pinned by: exhaustive byte-pattern round trip against an independent packer, brute force.
 int oracle_sign(const uint32_t* bits, int d_in, int o, int i) { return unpack_sign(bits, d_in, o, i); }
@@ -351,6 +351,51 @@ void oracle_lm_head(const int8_t* W, const float* s_row, int V, int d, const flo
   std::vector<int8_t> q((size_t)d);
   float s = 0.0f;
   quantize_row(x, d, q.data(), &s);
+  const int count = rows ? n_rows : V;
+#pragma omp parallel for schedule(static)
+  for (int k = 0; k < count; ++k) {
+    const int vrow = rows ? rows[k] : k;
+    int64_t a = 0;
+    for (int i = 0; i < d; ++i) a += (int64_t)W[(size_t)vrow * d + i] * (int64_t)q[i];
+    if (acc_out) acc_out[k] = (int32_t)a;
+    logits[k] = r32((double)a * (double)s * (double)s_row[vrow]);
+  }
+}
+
+
+// Token embedding from the int8 embedding matrix ([TS-2B]: "embedding/LM head matrices are quantized
+// to int8 with per-channel/row scaling").  Reading: the embedding and the LM head are ONE tied matrix
+// W [V][d] with one scale per row ([TS-3]: the embedding/LM-head share is 37% of 278 MB, i.e. a single
+// 50288 x 2048 int8 matrix), so
+//   e[i] = fl32(W[tok, i] * s_row[tok]).
+// Returns 0, or -1 (e left untouched) when tok is outside [0, V).
+// Pinned by: power-of-two row scales give the exact products; agreement with an IEEE fp32 multiply;
+// the row index selects the row.
+int oracle_embed(const int8_t* W, const float* s_row, int V, int d, int tok, float* e) {
+  if (tok < 0 || tok >= V) return -1;
+  for (int i = 0; i < d; ++i) e[i] = r32((double)W[(size_t)tok * d + i] * (double)s_row[tok]);
+  return 0;
+}
+
+// Final RMSNorm + int8 LM head on one token (reading: the Mamba-2 language model [MAP] applies an
+// RMSNorm with its own weight, eps 1e-5, to the last layer's residual stream before the LM head).
+// The norm is folded into the quantizer exactly as for the pre-mixer norm (rmsnorm_quantize):
+//   (q, s) = rmsnorm_quantize(h, norm_w);  logits[v] = fl32(acc[v] * s * s_row[v]),
+//   acc[v] = sum_i W[v,i] * q[i].
+// norm_w == NULL gives the plain LM head (oracle_lm_head).  Only rows listed in `rows` are computed
+// when rows != NULL.
+// Pinned by: brute-force int64 matmul of the pinned codes; agreement with the plain LM head on the
+// explicitly normalized row away from rounding ties.
+void oracle_final_head(const int8_t* W, const float* s_row, int V, int d, const float* h,
+                       const float* norm_w, const int* rows, int n_rows, float* logits,
+                       int32_t* acc_out) {
+  std::vector<int8_t> q((size_t)d);
+  std::vector<float> v((size_t)d);
+  float s = 0.0f;
+  if (norm_w)
+    rmsnorm_quantize(h, norm_w, d, 1e-5, q.data(), &s, v.data());
+  else
+    quantize_row(h, d, q.data(), &s);
   const int count = rows ? n_rows : V;
 #pragma omp parallel for schedule(static)
   for (int k = 0; k < count; ++k) {

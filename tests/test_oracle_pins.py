@@ -465,6 +465,118 @@ def test_lm_head_brute_force():
     assert np.array_equal(a2, acc[rows]) and np.array_equal(l2, logits[rows])
 
 
+# --------------------------------------------------------------------- embedding, final head, greedy
+
+def test_embed_power_of_two_scales_are_exact():
+    """Row scales 2^-k make every dequantized value exact: catches a wrong row, a dropped scale or a
+    transposed matrix."""
+    g = np.random.default_rng(51)
+    W = g.integers(-127, 128, (40, 96), dtype=np.int8)
+    k = g.integers(4, 16, 40)
+    sr = np.ldexp(1.0, -k).astype(np.float32)
+    for tok in (0, 17, 39):
+        e = oracle.embed(W, sr, tok)
+        assert np.array_equal(e.astype(np.float64), W[tok].astype(np.float64) * 2.0 ** -int(k[tok]))
+
+
+def test_embed_matches_ieee_fp32_multiply_and_rejects_bad_tokens():
+    g = np.random.default_rng(52)
+    W = g.integers(-127, 128, (50, 64), dtype=np.int8)
+    sr = g.uniform(1e-4, 1e-3, 50).astype(np.float32)
+    for tok in (0, 1, 49):
+        assert np.array_equal(oracle.embed(W, sr, tok), W[tok].astype(np.float32) * sr[tok])
+    for bad in (-1, 50):
+        with pytest.raises(IndexError):
+            oracle.embed(W, sr, bad)
+
+
+def test_final_head_constant_row_closed_form():
+    """h = c (all equal), unit norm weight: every code is 127 sign(c), so
+    logits[v] = sign(c) * sum_i W[v,i] * s_row[v] / sqrt(1 + eps / c^2).  Catches a missing RMS factor,
+    a wrong epsilon, a sign error or the norm weight left out."""
+    g = np.random.default_rng(53)
+    W = g.integers(-127, 128, (64, 128), dtype=np.int8)
+    sr = g.uniform(1e-4, 1e-3, 64).astype(np.float32)
+    ones = np.ones(128, np.float32)
+    for c in (-2.5, 0.01, 7.0):
+        logits, acc = oracle.final_head(W, sr, np.full(128, c, np.float32), ones)
+        rowsum = W.astype(np.int64).sum(axis=1)
+        assert np.array_equal(acc, 127 * int(np.sign(c)) * rowsum)
+        want = np.sign(c) * rowsum * sr.astype(np.float64) / np.sqrt(1 + 1e-5 / c ** 2)
+        assert np.allclose(logits, want, rtol=1e-6, atol=0)
+
+
+def test_final_head_norm_weight_enters_the_codes():
+    """A norm weight that is zero on half the inputs zeroes their codes (the weight multiplies before
+    the quantizer, not after)."""
+    g = np.random.default_rng(54)
+    W = g.integers(-127, 128, (32, 64), dtype=np.int8)
+    sr = g.uniform(1e-4, 1e-3, 32).astype(np.float32)
+    h = g.standard_normal(64).astype(np.float32)
+    w = np.ones(64, np.float32)
+    w[32:] = 0
+    _, acc = oracle.final_head(W, sr, h, w)
+    _, acc_half = oracle.final_head(W[:, :32].copy(), sr, h[:32].copy(), w[:32].copy())
+    assert np.array_equal(acc, acc_half)
+
+
+def test_final_head_fold_matches_explicit_normalization():
+    """The folded norm equals the plain LM head on the explicitly normalized row: same integer sums
+    (no code is near a rounding tie for this input) and logits to fp32 precision."""
+    g = np.random.default_rng(55)
+    V, d = 500, 256
+    W = g.integers(-127, 128, (V, d), dtype=np.int8)
+    sr = g.uniform(1e-4, 1e-3, V).astype(np.float32)
+    h = (g.standard_normal(d) * 2).astype(np.float32)
+    w = g.uniform(0.5, 1.5, d).astype(np.float32)
+    logits, acc = oracle.final_head(W, sr, h, w)
+    h64 = h.astype(np.float64)
+    u = h64 / np.sqrt(np.mean(h64 ** 2) + 1e-5) * w
+    r = u / (np.abs(u).max() / 127)
+    assert np.all(np.abs(np.abs(r - np.floor(r)) - 0.5) > 1e-4)  # no near-tie code for this seed
+    q = np.rint(r).astype(np.int64)
+    assert np.array_equal(acc, W.astype(np.int64) @ q)
+    l2, a2 = oracle.lm_head(W, sr, u.astype(np.float32))
+    assert np.array_equal(a2, acc)
+    assert np.allclose(logits, l2, rtol=2e-7, atol=0)
+    # the plain head is the final head without a norm
+    l3, a3 = oracle.final_head(W, sr, h)
+    l4, a4 = oracle.lm_head(W, sr, h)
+    assert np.array_equal(l3, l4) and np.array_equal(a3, a4)
+    rows = np.array([499, 3, 250])
+    l5, a5 = oracle.final_head(W, sr, h, w, rows)
+    assert np.array_equal(l5, logits[rows]) and np.array_equal(a5, acc[rows])
+
+
+def test_greedy_takes_first_index_on_ties():
+    assert oracle.greedy(np.array([0.5, 2.0, -1.0, 2.0], np.float32)) == 1
+    assert oracle.greedy(np.array([-3.0, -3.0], np.float32)) == 0
+
+
+def test_generate_with_identity_layers_follows_the_head():
+    """With every out_proj scaled to zero the layers leave the residual stream unchanged, so each
+    step's hidden state is the embedding itself and the next token is the greedy choice of the head
+    on it, computed here by brute force from the pinned quantizer codes."""
+    dims = dict(SMALL)
+    m = inputs.generation_model(seed=56, n_layers=2, vocab=300, **dims)
+    for ld in m["layers"]:
+        ld["out_proj"]["w_scale"][:] = 0
+        ld["out_proj"]["lora_a_scale"][:] = 0
+    layers = [_oracle_layer(ld) for ld in m["layers"]]
+    conv, ssm = inputs.zero_states(1, 2, 4, 16, 16, 1)
+    W, sr, fw = m["emb_w"], m["emb_s"], m["final_norm_w"]
+    toks, hid, _ = oracle.generate(layers, W, sr, fw, m["first_token"], 5, conv, ssm)
+    assert toks[0] == m["first_token"] and len(toks) == 6
+    assert np.any(ssm != 0)
+    for t in range(5):
+        e = W[toks[t]].astype(np.float32) * sr[toks[t]]
+        assert np.array_equal(hid[t], e)
+        q, s, _, _ = oracle.rmsnorm_quantize(e[None], fw)
+        acc = W.astype(np.int64) @ q[0].astype(np.int64)
+        logits = (acc.astype(np.float64) * float(s[0]) * sr.astype(np.float64)).astype(np.float32)
+        assert toks[t + 1] == int(np.argmax(logits))
+
+
 # ------------------------------------------------------------------------------------- shape pins
 
 def test_model_size_and_composition_pin():
