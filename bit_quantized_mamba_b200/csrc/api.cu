@@ -70,6 +70,52 @@ LayerWs carve_layer_ws(void* base, int B, int d_model, int E, int C, int d_ip) {
   return w;
 }
 
+// Greedy-choice scratch of the head kernel: the 64-bit argmax key and the finished-CTA count.
+constexpr size_t kGreedyBytes = 256;
+
+// Generation workspace: [layer-decode region (B = 1, sized as dfssm_workspace_size reports)]
+// [hidden f32 d_model][logits f32 V][greedy scratch].
+struct GenerateWs {
+  size_t layer, hidden, logits, greedy, total;
+};
+GenerateWs generate_ws(int V, int d_model, int d_inner) {
+  GenerateWs g;
+  const int C = d_inner + 2048, d_ip = 2 * d_inner + 2048 + 1024;
+  g.layer = 0;
+  g.hidden = align256(layer_ws_bytes(1, d_model, d_inner, C, d_ip));
+  g.logits = g.hidden + align256(sizeof(float) * (size_t)d_model);
+  g.greedy = g.logits + align256(sizeof(float) * (size_t)V);
+  g.total = g.greedy + kGreedyBytes;
+  return g;
+}
+
+int check_head(const int8_t* W, const float* s_row, int V, int d) {
+  if (!W || !s_row || V < 1 || d < 16 || d % 16) return DFSSM_EINVAL;
+  if (d > 8192) return DFSSM_EUNSUPPORTED;
+  if (!aligned(W, 16) || !aligned(s_row, 4)) return DFSSM_EALIGN;
+  return DFSSM_OK;
+}
+
+int enqueue_embed(const int8_t* W, const float* s_row, int V, int d, const int32_t* token, float* h,
+                  cudaStream_t s) {
+  int* status = nullptr;
+  const int st = dfssm::stream_status_word(&status);
+  if (st) return st;
+  dfssm::EmbedArgs ea{W, s_row, V, d, token, h, status};
+  const cudaError_t e = dfssm::launch_embed(ea, s);
+  return e == cudaSuccess ? DFSSM_OK : cuda_fail(e);
+}
+
+int enqueue_head(const int8_t* W, const float* s_row, int V, int d, const float* h, const float* norm_w,
+                 float* logits, int32_t* acc, int32_t* token, void* greedy, cudaStream_t s) {
+  dfssm::Int8GemvArgs ia{W, s_row, V, d, h, logits, acc};
+  ia.norm_w = norm_w;
+  ia.greedy = static_cast<unsigned long long*>(greedy);
+  ia.token = token;
+  const cudaError_t e = dfssm::launch_int8_gemv(ia, s);
+  return e == cudaSuccess ? DFSSM_OK : cuda_fail(e);
+}
+
 // Clock budget of one device-side wait of the fused decode kernel (about 1 s at 2 GHz).
 constexpr long long kSpinLimitCycles = 2000000000LL;
 
@@ -101,6 +147,117 @@ dfssm::GemvArgs gemv_args(const dfssm_linear_t* L, int B, const dfssm::QuantScra
   g.B = B;
   g.in = qs;
   return g;
+}
+
+// dfssm_layer_decode; with launch == false only the arguments are checked.
+int layer_decode_impl(const dfssm_layer_t* layers, int n_layers, const dfssm_dims_t* dims, float* hidden,
+                      float* const* conv_states, float* const* ssm_states, int B, void* workspace,
+                      size_t ws_bytes, void* stream, bool launch) {
+  if (!layers || !dims || !hidden || !conv_states || !ssm_states) return DFSSM_EINVAL;
+  if (n_layers < 1 || B < 1) return DFSSM_EINVAL;
+  if (n_layers > DFSSM_MAX_LAYERS || B > DFSSM_MAX_BATCH) return DFSSM_EUNSUPPORTED;
+  const int Dm = dims->d_model, H = dims->nheads, P = dims->headdim, N = dims->d_state,
+            G = dims->ngroups;
+  if (Dm < 32 || Dm % 32 || H < 1 || P < 1 || N < 4 || G < 1 || H % G) return DFSSM_EINVAL;
+  const int E = H * P;
+  const int C = E + 2 * G * N;
+  const int d_ip = 2 * E + 2 * G * N + H;
+  if (E % 32 || N % 4 || N > 512 || Dm > 8192 || E > 8192 || 2 * G * N > 2048 || H > 1024)
+    return DFSSM_EUNSUPPORTED;
+  if (!aligned(hidden, 16)) return DFSSM_EALIGN;
+  for (int l = 0; l < n_layers; ++l) {
+    const dfssm_layer_t& Ly = layers[l];
+    int st = check_linear(&Ly.in_proj);
+    if (st) return st;
+    st = check_linear(&Ly.out_proj);
+    if (st) return st;
+    if (Ly.in_proj.d_out != d_ip || Ly.in_proj.d_in != Dm || Ly.out_proj.d_out != Dm ||
+        Ly.out_proj.d_in != E)
+      return DFSSM_EINVAL;
+    if (!Ly.conv_w || !Ly.conv_b || !Ly.A_log || !Ly.dt_bias || !Ly.D || !Ly.norm_w || !Ly.gnorm_w)
+      return DFSSM_EINVAL;
+    if (!conv_states[l] || !ssm_states[l]) return DFSSM_EINVAL;
+    if (!aligned(Ly.conv_w, 16) || !aligned(ssm_states[l], 16)) return DFSSM_EALIGN;
+  }
+  if (!workspace || !aligned(workspace, 256) || ws_bytes < layer_ws_bytes(B, Dm, E, C, d_ip))
+    return DFSSM_EWORKSPACE;
+  if (!device_ok()) return DFSSM_EDEVICE;
+  if (!launch) return DFSSM_OK;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (dfssm::fused_decode_supported(*dims, B, layers, n_layers, conv_states)) {
+    const cudaError_t fe = dfssm::launch_fused_decode(layers, n_layers, hidden, conv_states, ssm_states,
+                                                      workspace, s, kSpinLimitCycles);
+    return fe == cudaSuccess ? DFSSM_OK : cuda_fail(fe);
+  }
+  LayerWs w = carve_layer_ws(workspace, B, Dm, E, C, d_ip);
+  cudaError_t e = cudaSuccess;
+  for (int l = 0; l < n_layers && e == cudaSuccess; ++l) {
+    const dfssm_layer_t& Ly = layers[l];
+    // pre-norm + quantize + LoRA-down
+    dfssm::QuantArgs qa{};
+    qa.x = hidden;
+    qa.ldx = Dm;
+    qa.norm_w = Ly.norm_w;
+    qa.n = Dm;
+    qa.B = B;
+    qa.lora_b = Ly.in_proj.lora_b;
+    qa.lora_b_scale = Ly.in_proj.lora_b_scale;
+    qa.rank = Ly.in_proj.rank;
+    qa.permute = true;
+    qa.out = w.qs;
+    e = dfssm::launch_quant(qa, s);
+    if (e != cudaSuccess) break;
+    // in_proj
+    dfssm::GemvArgs ga = gemv_args(&Ly.in_proj, B, w.qs);
+    ga.y = w.zxbcdt;
+    ga.ldy = d_ip;
+    e = dfssm::launch_gemv(ga, s);
+    if (e != cudaSuccess) break;
+    // conv over x|B|C
+    dfssm::ConvArgs ca{conv_states[l], Ly.conv_w, Ly.conv_b, w.zxbcdt + E, d_ip, w.xc, C, B, C};
+    e = dfssm::launch_conv(ca, s);
+    if (e != cudaSuccess) break;
+    // SSM + gate
+    dfssm::SsmArgs sa{};
+    sa.state = ssm_states[l];
+    sa.x = w.xc;
+    sa.ldx = C;
+    sa.dt_raw = w.zxbcdt + E + C;
+    sa.lddt = d_ip;
+    sa.A_log = Ly.A_log;
+    sa.dt_bias = Ly.dt_bias;
+    sa.D = Ly.D;
+    sa.Bm = w.xc + E;
+    sa.Cm = w.xc + E + G * N;
+    sa.ldbc = C;
+    sa.y = w.g;
+    sa.ldy = E;
+    sa.z = w.zxbcdt;
+    sa.ldz = d_ip;
+    sa.B = B;
+    sa.H = H;
+    sa.P = P;
+    sa.N = N;
+    sa.G = G;
+    e = dfssm::launch_ssm(sa, s);
+    if (e != cudaSuccess) break;
+    // gated norm + quantize + LoRA-down
+    qa.x = w.g;
+    qa.ldx = E;
+    qa.norm_w = Ly.gnorm_w;
+    qa.n = E;
+    qa.lora_b = Ly.out_proj.lora_b;
+    qa.lora_b_scale = Ly.out_proj.lora_b_scale;
+    qa.rank = Ly.out_proj.rank;
+    e = dfssm::launch_quant(qa, s);
+    if (e != cudaSuccess) break;
+    // out_proj + residual
+    ga = gemv_args(&Ly.out_proj, B, w.qs);
+    ga.resid = hidden;
+    ga.ldr = Dm;
+    e = dfssm::launch_gemv(ga, s);
+  }
+  return e == cudaSuccess ? DFSSM_OK : cuda_fail(e);
 }
 
 }  // namespace
@@ -145,6 +302,12 @@ size_t dfssm_workspace_size(int op, int a, int b, int c) {
     case DFSSM_OP_LM_HEAD:
       if (b < 16 || b % 16 || b > 8192 || c < 1) return 0;
       return dfssm::quant_scratch_bytes(1, b);
+    case DFSSM_OP_HEAD_GREEDY:
+      if (b < 16 || b % 16 || b > 8192 || c < 1) return 0;
+      return kGreedyBytes;
+    case DFSSM_OP_GENERATE:
+      if (a < 1 || b < 32 || b % 32 || b > 8192 || c < 32) return 0;
+      return generate_ws(a, b, c).total;
     default: return 0;
   }
 }
@@ -265,110 +428,8 @@ int dfssm_ssm_step(float* ssm_state, const float* x, const float* dt_raw, const 
 int dfssm_layer_decode(const dfssm_layer_t* layers, int n_layers, const dfssm_dims_t* dims,
                        float* hidden, float* const* conv_states, float* const* ssm_states, int B,
                        void* workspace, size_t ws_bytes, void* stream) {
-  if (!layers || !dims || !hidden || !conv_states || !ssm_states) return DFSSM_EINVAL;
-  if (n_layers < 1 || B < 1) return DFSSM_EINVAL;
-  if (n_layers > DFSSM_MAX_LAYERS || B > DFSSM_MAX_BATCH) return DFSSM_EUNSUPPORTED;
-  const int Dm = dims->d_model, H = dims->nheads, P = dims->headdim, N = dims->d_state,
-            G = dims->ngroups;
-  if (Dm < 32 || Dm % 32 || H < 1 || P < 1 || N < 4 || G < 1 || H % G) return DFSSM_EINVAL;
-  const int E = H * P;
-  const int C = E + 2 * G * N;
-  const int d_ip = 2 * E + 2 * G * N + H;
-  if (E % 32 || N % 4 || N > 512 || Dm > 8192 || E > 8192 || 2 * G * N > 2048 || H > 1024)
-    return DFSSM_EUNSUPPORTED;
-  if (!aligned(hidden, 16)) return DFSSM_EALIGN;
-  for (int l = 0; l < n_layers; ++l) {
-    const dfssm_layer_t& Ly = layers[l];
-    int st = check_linear(&Ly.in_proj);
-    if (st) return st;
-    st = check_linear(&Ly.out_proj);
-    if (st) return st;
-    if (Ly.in_proj.d_out != d_ip || Ly.in_proj.d_in != Dm || Ly.out_proj.d_out != Dm ||
-        Ly.out_proj.d_in != E)
-      return DFSSM_EINVAL;
-    if (!Ly.conv_w || !Ly.conv_b || !Ly.A_log || !Ly.dt_bias || !Ly.D || !Ly.norm_w || !Ly.gnorm_w)
-      return DFSSM_EINVAL;
-    if (!conv_states[l] || !ssm_states[l]) return DFSSM_EINVAL;
-    if (!aligned(Ly.conv_w, 16) || !aligned(ssm_states[l], 16)) return DFSSM_EALIGN;
-  }
-  if (!workspace || !aligned(workspace, 256) || ws_bytes < layer_ws_bytes(B, Dm, E, C, d_ip))
-    return DFSSM_EWORKSPACE;
-  if (!device_ok()) return DFSSM_EDEVICE;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (dfssm::fused_decode_supported(*dims, B, layers, n_layers, conv_states)) {
-    const cudaError_t fe = dfssm::launch_fused_decode(layers, n_layers, hidden, conv_states, ssm_states,
-                                                      workspace, s, kSpinLimitCycles);
-    return fe == cudaSuccess ? DFSSM_OK : cuda_fail(fe);
-  }
-  LayerWs w = carve_layer_ws(workspace, B, Dm, E, C, d_ip);
-  cudaError_t e = cudaSuccess;
-  for (int l = 0; l < n_layers && e == cudaSuccess; ++l) {
-    const dfssm_layer_t& Ly = layers[l];
-    // pre-norm + quantize + LoRA-down
-    dfssm::QuantArgs qa{};
-    qa.x = hidden;
-    qa.ldx = Dm;
-    qa.norm_w = Ly.norm_w;
-    qa.n = Dm;
-    qa.B = B;
-    qa.lora_b = Ly.in_proj.lora_b;
-    qa.lora_b_scale = Ly.in_proj.lora_b_scale;
-    qa.rank = Ly.in_proj.rank;
-    qa.permute = true;
-    qa.out = w.qs;
-    e = dfssm::launch_quant(qa, s);
-    if (e != cudaSuccess) break;
-    // in_proj
-    dfssm::GemvArgs ga = gemv_args(&Ly.in_proj, B, w.qs);
-    ga.y = w.zxbcdt;
-    ga.ldy = d_ip;
-    e = dfssm::launch_gemv(ga, s);
-    if (e != cudaSuccess) break;
-    // conv over x|B|C
-    dfssm::ConvArgs ca{conv_states[l], Ly.conv_w, Ly.conv_b, w.zxbcdt + E, d_ip, w.xc, C, B, C};
-    e = dfssm::launch_conv(ca, s);
-    if (e != cudaSuccess) break;
-    // SSM + gate
-    dfssm::SsmArgs sa{};
-    sa.state = ssm_states[l];
-    sa.x = w.xc;
-    sa.ldx = C;
-    sa.dt_raw = w.zxbcdt + E + C;
-    sa.lddt = d_ip;
-    sa.A_log = Ly.A_log;
-    sa.dt_bias = Ly.dt_bias;
-    sa.D = Ly.D;
-    sa.Bm = w.xc + E;
-    sa.Cm = w.xc + E + G * N;
-    sa.ldbc = C;
-    sa.y = w.g;
-    sa.ldy = E;
-    sa.z = w.zxbcdt;
-    sa.ldz = d_ip;
-    sa.B = B;
-    sa.H = H;
-    sa.P = P;
-    sa.N = N;
-    sa.G = G;
-    e = dfssm::launch_ssm(sa, s);
-    if (e != cudaSuccess) break;
-    // gated norm + quantize + LoRA-down
-    qa.x = w.g;
-    qa.ldx = E;
-    qa.norm_w = Ly.gnorm_w;
-    qa.n = E;
-    qa.lora_b = Ly.out_proj.lora_b;
-    qa.lora_b_scale = Ly.out_proj.lora_b_scale;
-    qa.rank = Ly.out_proj.rank;
-    e = dfssm::launch_quant(qa, s);
-    if (e != cudaSuccess) break;
-    // out_proj + residual
-    ga = gemv_args(&Ly.out_proj, B, w.qs);
-    ga.resid = hidden;
-    ga.ldr = Dm;
-    e = dfssm::launch_gemv(ga, s);
-  }
-  return e == cudaSuccess ? DFSSM_OK : cuda_fail(e);
+  return layer_decode_impl(layers, n_layers, dims, hidden, conv_states, ssm_states, B, workspace,
+                           ws_bytes, stream, true);
 }
 
 int dfssm_device_status(void* workspace, void* stream) {
@@ -390,6 +451,7 @@ int dfssm_device_status(void* workspace, void* stream) {
   if (e == cudaSuccess) e = cudaMemsetAsync(word, 0, sizeof(int), s);
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);
   if (e != cudaSuccess) return cuda_fail(e);
+  if (code == 0 && h == dfssm::kBadTokenCode) return DFSSM_EINVAL;
   return (code || h) ? DFSSM_ETIMEOUT : DFSSM_OK;
 }
 
@@ -414,6 +476,73 @@ int dfssm_lm_head(const int8_t* W, const float* s_row, int V, int d, const float
   dfssm::Int8GemvArgs ia{W, s_row, V, d, x, logits, acc};
   const cudaError_t e = dfssm::launch_int8_gemv(ia, s);
   return e == cudaSuccess ? DFSSM_OK : cuda_fail(e);
+}
+
+int dfssm_embed(const int8_t* W, const float* s_row, int V, int d, const int32_t* token, float* h,
+                void* stream) {
+  int st = check_head(W, s_row, V, d);
+  if (st) return st;
+  if (!token || !h) return DFSSM_EINVAL;
+  if (!aligned(token, 4) || !aligned(h, 16)) return DFSSM_EALIGN;
+  if (!device_ok()) return DFSSM_EDEVICE;
+  return enqueue_embed(W, s_row, V, d, token, h, static_cast<cudaStream_t>(stream));
+}
+
+int dfssm_head_greedy(const int8_t* W, const float* s_row, int V, int d, const float* h,
+                      const float* norm_w, float* logits, int32_t* acc, int32_t* token, void* workspace,
+                      size_t ws_bytes, void* stream) {
+  int st = check_head(W, s_row, V, d);
+  if (st) return st;
+  if (!h || !logits || !token) return DFSSM_EINVAL;
+  if (!aligned(h, 4) || !aligned(token, 4) || (norm_w && !aligned(norm_w, 4))) return DFSSM_EALIGN;
+  if (!workspace || !aligned(workspace, 256) || ws_bytes < kGreedyBytes) return DFSSM_EWORKSPACE;
+  if (!device_ok()) return DFSSM_EDEVICE;
+  return enqueue_head(W, s_row, V, d, h, norm_w, logits, acc, token, workspace,
+                      static_cast<cudaStream_t>(stream));
+}
+
+int dfssm_generate(const dfssm_layer_t* layers, int n_layers, const dfssm_dims_t* dims,
+                   const int8_t* W, const float* s_row, int V, const float* final_norm_w,
+                   int32_t* tokens, int n_tokens, float* const* conv_states, float* const* ssm_states,
+                   float* hidden_taps, float* logits, void* workspace, size_t ws_bytes, void* stream) {
+  if (!dims || !tokens || !final_norm_w || n_tokens < 1) return DFSSM_EINVAL;
+  const int Dm = dims->d_model, E = dims->nheads * dims->headdim;
+  int st = check_head(W, s_row, V, Dm);
+  if (st) return st;
+  if (!aligned(tokens, 4) || !aligned(final_norm_w, 4) || (hidden_taps && !aligned(hidden_taps, 4)) ||
+      (logits && !aligned(logits, 4)))
+    return DFSSM_EALIGN;
+  if (Dm < 32 || Dm % 32 || E < 32) return DFSSM_EINVAL;
+  const GenerateWs g = generate_ws(V, Dm, E);
+  if (!workspace || !aligned(workspace, 256) || ws_bytes < g.total) return DFSSM_EWORKSPACE;
+  char* base = static_cast<char*>(workspace);
+  float* hidden = reinterpret_cast<float*>(base + g.hidden);
+  float* lg = reinterpret_cast<float*>(base + g.logits);
+  void* greedy = base + g.greedy;
+  st = layer_decode_impl(layers, n_layers, dims, hidden, conv_states, ssm_states, 1, base + g.layer,
+                         g.hidden, stream, false);
+  if (st) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  for (int t = 0; t < n_tokens; ++t) {
+    st = enqueue_embed(W, s_row, V, Dm, tokens + t, hidden, s);
+    if (st) return st;
+    st = layer_decode_impl(layers, n_layers, dims, hidden, conv_states, ssm_states, 1, base + g.layer,
+                           g.hidden, stream, true);
+    if (st) return st;
+    if (hidden_taps) {
+      const cudaError_t e = cudaMemcpyAsync(hidden_taps + (size_t)t * Dm, hidden, sizeof(float) * Dm,
+                                            cudaMemcpyDeviceToDevice, s);
+      if (e != cudaSuccess) return cuda_fail(e);
+    }
+    st = enqueue_head(W, s_row, V, Dm, hidden, final_norm_w, lg, nullptr, tokens + t + 1, greedy, s);
+    if (st) return st;
+  }
+  if (logits) {
+    const cudaError_t e =
+        cudaMemcpyAsync(logits, lg, sizeof(float) * (size_t)V, cudaMemcpyDeviceToDevice, s);
+    if (e != cudaSuccess) return cuda_fail(e);
+  }
+  return DFSSM_OK;
 }
 
 }  // extern "C"

@@ -89,8 +89,26 @@ struct Int8GemvArgs {
   const float* x;           // the token, fp32 [d] (quantized by every CTA of the kernel)
   float* logits;
   int32_t* acc;
+  const float* norm_w = nullptr;     // final RMSNorm weight [d], folded into the quantizer (optional)
+  // greedy choice (optional): the argmax key and the CTA count live in `greedy` (2 x u64, zero
+  // before the launch, left zero after it); the last CTA writes the index to *token
+  unsigned long long* greedy = nullptr;
+  int32_t* token = nullptr;
 };
 cudaError_t launch_int8_gemv(const Int8GemvArgs& a, cudaStream_t st);
+
+// Embedding row lookup from the tied int8 matrix: h[i] = fl32(W[tok, i] * s_row[tok]), tok = *token.
+// An id outside [0, V) writes zeros and sets *status to kBadTokenCode.
+constexpr int kBadTokenCode = 0x70CE1D;
+struct EmbedArgs {
+  const int8_t* W;
+  const float* s_row;
+  int V, d;
+  const int32_t* token;
+  float* h;
+  int* status;
+};
+cudaError_t launch_embed(const EmbedArgs& a, cudaStream_t st);
 
 int num_sms();
 

@@ -123,17 +123,33 @@ cudaError_t launch_ssm(const SsmArgs& a, cudaStream_t st) {
 // ------------------------------------------------------------------------------ int8 LM-head GEMV
 // logits[v] = fl32(acc[v] * s * s_row[v]) (fp64, this order), acc[v] = sum_i W[v,i] q_i (int32 exact).
 // Every CTA quantizes the token itself (per-token absmax int8, the decode quantizer: no separate launch
-// and no hand-off).  Each warp owns a contiguous, balanced range of rows and streams it as units of 2 KB
-// (four 16-byte chunks per lane of one row), always with the next unit's loads in flight while the current
-// one is summed; the first unit is requested before the quantizer runs, so its latency is hidden.  The
-// stream rate is set by the number of resident threads (1024 per SM), not by the loads per thread.
+// and no hand-off); with a final RMSNorm weight the norm is folded in as for the layers' pre-norm:
+// codes of v = fl32(x w), s = fl32(s0 / rms), rms = sqrt(sum x^2 / d + 1e-5).  Each warp owns a
+// contiguous, balanced range of rows and streams it as units of 2 KB (four 16-byte chunks per lane of
+// one row), always with the next unit's loads in flight while the current one is summed; the first unit
+// is requested before the quantizer runs, so its latency is hidden.  The stream rate is set by the
+// number of resident threads (1024 per SM), not by the loads per thread.
+//
+// Greedy choice: every warp keeps the largest (logit, -row) key of its rows and merges it into one
+// 64-bit word with atomicMax; the CTA that finishes last (counted with a second word, release/acquire
+// through the fences around the count) turns the key into the row index and clears both words.
 
 constexpr int LMH_U = 4;  // chunks per lane per unit (a unit is 32 x 4 x 16 B = 2 KB of one row)
 constexpr int LMH_CTAS_PER_SM = 4;  // 1024 streaming threads per SM
+
+// Order-preserving map of a finite fp32 value to u32 (larger value, larger key); -0 maps as +0, so
+// equal logits tie and the smaller row wins.
+__device__ __forceinline__ unsigned long long greedy_key(float v, int row) {
+  unsigned u = __float_as_uint(v == 0.0f ? 0.0f : v);
+  u = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+  return ((unsigned long long)u << 32) | (unsigned long long)(0xFFFFFFFFu - (unsigned)row);
+}
+
 __global__ void __launch_bounds__(256, LMH_CTAS_PER_SM) int8_gemv_kernel(Int8GemvArgs a) {
   extern __shared__ __align__(16) unsigned char smem[];
   uint4* qsm = reinterpret_cast<uint4*>(smem);
   __shared__ float red[8];
+  __shared__ double red_ss[8];
   const int lane = threadIdx.x & 31;
   const int warps_total = gridDim.x * (blockDim.x >> 5);
   const int warp_g = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
@@ -156,8 +172,10 @@ __global__ void __launch_bounds__(256, LMH_CTAS_PER_SM) int8_gemv_kernel(Int8Gem
   load_unit(0, cur);  // weights do not depend on the token: in flight during the quantizer
   pdl_launch_dependents();
   pdl_wait();
+  const bool norm = a.norm_w != nullptr;
   // quantize the token (two passes over x, 8 KB for d = 2048): thread t takes inputs t + 256 k
   float m = 0.0f;
+  double ss = 0.0;
   for (int k0 = 0; k0 * 256 < a.d; k0 += 8) {
     float v[8];
 #pragma unroll
@@ -165,17 +183,34 @@ __global__ void __launch_bounds__(256, LMH_CTAS_PER_SM) int8_gemv_kernel(Int8Gem
       const int i = threadIdx.x + 256 * (k0 + k);
       v[k] = i < a.d ? __ldg(a.x + i) : 0.0f;
     }
+    if (norm) {
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const int i = threadIdx.x + 256 * (k0 + k);
+        ss = fma((double)v[k], (double)v[k], ss);  // the square of an fp32 value is exact in fp64
+        v[k] = i < a.d ? fmul(v[k], __ldg(a.norm_w + i)) : 0.0f;
+      }
+    }
 #pragma unroll
     for (int k = 0; k < 8; ++k) m = fmaxf(m, fabsf(v[k]));
   }
   m = warp_max(m);
-  if (lane == 0) red[threadIdx.x >> 5] = m;
+  if (norm) ss = warp_sum(ss);
+  if (lane == 0) {
+    red[threadIdx.x >> 5] = m;
+    red_ss[threadIdx.x >> 5] = ss;
+  }
   __syncthreads();
   m = 0.0f;
+  ss = 0.0;
 #pragma unroll
-  for (int w = 0; w < 8; ++w) m = fmaxf(m, red[w]);
-  const float s = m == 0.0f ? 0.0f : __fdiv_rn(m, 127.0f);
-  const float inv_s = m == 0.0f ? 0.0f : __frcp_rn(s);
+  for (int w = 0; w < 8; ++w) {
+    m = fmaxf(m, red[w]);
+    ss += red_ss[w];
+  }
+  const float s0 = m == 0.0f ? 0.0f : __fdiv_rn(m, 127.0f);
+  const float inv_s0 = m == 0.0f ? 0.0f : __frcp_rn(s0);
+  const float s = norm ? rms_scale(s0, rms_of(ss, a.d)) : s0;
   int8_t* qb = reinterpret_cast<int8_t*>(smem);
   for (int k0 = 0; k0 * 256 < a.d; k0 += 8) {
     float vv[8];
@@ -183,9 +218,10 @@ __global__ void __launch_bounds__(256, LMH_CTAS_PER_SM) int8_gemv_kernel(Int8Gem
     for (int k = 0; k < 8; ++k) {
       const int i = threadIdx.x + 256 * (k0 + k);
       vv[k] = i < a.d ? __ldg(a.x + i) : 0.0f;
+      if (norm) vv[k] = i < a.d ? fmul(vv[k], __ldg(a.norm_w + i)) : 0.0f;
     }
     int cd[8];
-    quant_codes<8>(vv, s, inv_s, cd);
+    quant_codes<8>(vv, s0, inv_s0, cd);
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
       const int i = threadIdx.x + 256 * (k0 + k);
@@ -194,6 +230,7 @@ __global__ void __launch_bounds__(256, LMH_CTAS_PER_SM) int8_gemv_kernel(Int8Gem
   }
   __syncthreads();
   int acc = 0;
+  unsigned long long best = 0ull;
   for (int j = 0; j < n_units; ++j) {
     uint4 nxt[LMH_U];
     load_unit(j + 1, nxt);
@@ -211,19 +248,68 @@ __global__ void __launch_bounds__(256, LMH_CTAS_PER_SM) int8_gemv_kernel(Int8Gem
       const int row = r0 + j / G;
       acc = warp_sum(acc);
       if (lane == 0) {
-        a.logits[row] = __double2float_rn(dmul(dmul((double)acc, (double)s), (double)a.s_row[row]));
+        const float lg = __double2float_rn(dmul(dmul((double)acc, (double)s), (double)a.s_row[row]));
+        a.logits[row] = lg;
         if (a.acc) a.acc[row] = acc;
+        const unsigned long long key = greedy_key(lg, row);
+        best = key > best ? key : best;
       }
       acc = 0;
     }
 #pragma unroll
     for (int u = 0; u < LMH_U; ++u) cur[u] = nxt[u];
   }
+  if (a.greedy) {
+    if (lane == 0 && n_units > 0) atomicMax(a.greedy, best);
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      __threadfence();
+      const unsigned long long done = atomicAdd(a.greedy + 1, 1ull);
+      if (done == (unsigned long long)gridDim.x - 1) {
+        __threadfence();
+        const unsigned long long key = atomicOr(a.greedy, 0ull);
+        *a.token = (int32_t)(0xFFFFFFFFu - (unsigned)(key & 0xFFFFFFFFull));
+        a.greedy[0] = 0ull;
+        a.greedy[1] = 0ull;
+      }
+    }
+  }
 }
 
 cudaError_t launch_int8_gemv(const Int8GemvArgs& a, cudaStream_t st) {
   const int blocks = num_sms() * LMH_CTAS_PER_SM;  // all resident: each CTA quantizes x once
   return launch_pdl(int8_gemv_kernel, dim3(blocks), dim3(256), (size_t)a.d, st, a);
+}
+
+// ------------------------------------------------------------------------------ embedding lookup
+// One CTA; thread t converts 16 consecutive int8 values of the row (d % 16 == 0, rows 16-byte aligned).
+__global__ void __launch_bounds__(512) embed_kernel(EmbedArgs a) {
+  pdl_launch_dependents();
+  pdl_wait();
+  const int tok = *a.token;
+  const bool ok = tok >= 0 && tok < a.V;
+  if (!ok && threadIdx.x == 0) atomicExch(a.status, kBadTokenCode);
+  const float sc = ok ? a.s_row[tok] : 0.0f;
+  const uint4* row = reinterpret_cast<const uint4*>(a.W + (size_t)(ok ? tok : 0) * a.d);
+  float4* h4 = reinterpret_cast<float4*>(a.h);
+  for (int c = threadIdx.x; c < (a.d >> 4); c += blockDim.x) {
+    const uint4 w = ok ? __ldg(row + c) : make_uint4(0u, 0u, 0u, 0u);
+    const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      float4 o;
+      o.x = fmul((float)(int8_t)(wv[k] & 0xFFu), sc);
+      o.y = fmul((float)(int8_t)((wv[k] >> 8) & 0xFFu), sc);
+      o.z = fmul((float)(int8_t)((wv[k] >> 16) & 0xFFu), sc);
+      o.w = fmul((float)(int8_t)(wv[k] >> 24), sc);
+      h4[4 * c + k] = o;
+    }
+  }
+}
+
+cudaError_t launch_embed(const EmbedArgs& a, cudaStream_t st) {
+  const int threads = (a.d >> 4) < 512 ? (((a.d >> 4) + 31) & ~31) : 512;
+  return launch_pdl(embed_kernel, dim3(1), dim3(threads), 0, st, a);
 }
 
 }  // namespace dfssm

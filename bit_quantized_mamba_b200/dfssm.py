@@ -18,6 +18,8 @@ OP_LINEAR_DECODE = 1
 OP_LINEAR_PREFILL = 2
 OP_LAYER_DECODE = 3
 OP_LM_HEAD = 4
+OP_HEAD_GREEDY = 5
+OP_GENERATE = 6
 MAX_RANK = 16
 MAX_BATCH = 16
 MAX_LAYERS = 64
@@ -71,6 +73,9 @@ SIGNATURES = {
     "dfssm_ssm_step": (_I, [_P] * 9 + [_I] * 5 + [_P]),
     "dfssm_layer_decode": (_I, [_P, _I, _P, _P, _P, _P, _I, _P, _Z, _P]),
     "dfssm_lm_head": (_I, [_P, _P, _I, _I, _P, _P, _P, _P, _Z, _P]),
+    "dfssm_embed": (_I, [_P, _P, _I, _I, _P, _P, _P]),
+    "dfssm_head_greedy": (_I, [_P, _P, _I, _I, _P, _P, _P, _P, _P, _P, _Z, _P]),
+    "dfssm_generate": (_I, [_P, _I, _P, _P, _P, _I, _P, _P, _I, _P, _P, _P, _P, _P, _Z, _P]),
     "dfssm_pack_signs": (_I, [_P, _I, _I, _P]),
     "dfssm_device_status": (_I, [_P, _P]),
     "dfssm_selftest_timeout": (_I, [_P, _Z, _P]),
@@ -284,7 +289,7 @@ def layer_decode(stack: LayerStack, hidden: torch.Tensor, ws=None, stream=None) 
 
 def device_status(ws=None, stream=None) -> int:
     """Synchronise the stream, read and clear the device error words (the workspace's, if given, and
-    the library's own): 0 (DFSSM_OK) or -5 (DFSSM_ETIMEOUT)."""
+    the library's own): 0 (DFSSM_OK), -5 (DFSSM_ETIMEOUT) or -1 (DFSSM_EINVAL: a bad token id)."""
     return int(lib().dfssm_device_status(_ptr(ws), _stream(stream)))
 
 
@@ -302,6 +307,47 @@ def lm_head(W, s_row, x, logits=None, acc=None, ws=None, stream=None):
     _check("dfssm_lm_head", lib().dfssm_lm_head(_ptr(W), _ptr(s_row), V, d, _ptr(x), _ptr(logits),
                                                 _ptr(acc), _ptr(ws), ws.numel(), _stream(stream)))
     return logits
+
+
+def embed(W, s_row, token, h=None, stream=None):
+    """Row token[0] of the tied int8 embedding, dequantized (token: device int32 [1])."""
+    V, d = W.shape
+    if h is None:
+        h = torch.empty(d, dtype=torch.float32, device=W.device)
+    _check("dfssm_embed", lib().dfssm_embed(_ptr(W), _ptr(s_row), V, d, _ptr(token), _ptr(h),
+                                            _stream(stream)))
+    return h
+
+
+def head_greedy(W, s_row, h, norm_w=None, logits=None, acc=None, token=None, ws=None, stream=None):
+    """Final RMSNorm (norm_w; None = no norm) + int8 LM head + greedy choice on one token.
+    Returns (token device int32 [1], logits)."""
+    V, d = W.shape
+    if logits is None:
+        logits = torch.empty(V, dtype=torch.float32, device=h.device)
+    if token is None:
+        token = torch.empty(1, dtype=torch.int32, device=h.device)
+    if ws is None:
+        ws = workspace(workspace_size(OP_HEAD_GREEDY, 1, d, V), h.device)
+    _check("dfssm_head_greedy", lib().dfssm_head_greedy(
+        _ptr(W), _ptr(s_row), V, d, _ptr(h), _ptr(norm_w), _ptr(logits), _ptr(acc), _ptr(token),
+        _ptr(ws), ws.numel(), _stream(stream)))
+    return token, logits
+
+
+def generate(stack: "LayerStack", W, s_row, final_norm_w, tokens, hidden_taps=None, logits=None,
+             ws=None, stream=None):
+    """Greedy generation at batch 1: tokens (device int32 [n + 1]) holds the first token in [0];
+    entries 1..n are written.  The stack's states advance by n steps."""
+    V, d = W.shape
+    n = tokens.numel() - 1
+    if ws is None:
+        ws = workspace(workspace_size(OP_GENERATE, V, stack.d_model, stack.d_inner), W.device)
+    _check("dfssm_generate", lib().dfssm_generate(
+        stack._layers, stack.n, C.byref(stack.dims), _ptr(W), _ptr(s_row), V, _ptr(final_norm_w),
+        _ptr(tokens), n, stack._conv, stack._ssm, _ptr(hidden_taps), _ptr(logits), _ptr(ws),
+        ws.numel(), _stream(stream)))
+    return tokens
 
 
 def pack_signs(signs: np.ndarray) -> np.ndarray:

@@ -35,7 +35,7 @@
 extern "C" {
 #endif
 
-#define DFSSM_ABI_VERSION 2
+#define DFSSM_ABI_VERSION 3
 #define DFSSM_MAX_RANK 16
 #define DFSSM_MAX_BATCH 16
 #define DFSSM_MAX_LAYERS 64
@@ -92,7 +92,9 @@ enum {
   DFSSM_OP_LINEAR_DECODE = 1,  /* a = B,  b = d_in,  c = d_out                         */
   DFSSM_OP_LINEAR_PREFILL = 2, /* a = M,  b = d_in,  c = d_out                         */
   DFSSM_OP_LAYER_DECODE = 3,   /* a = B,  b = d_model, c = d_inner (nheads*headdim)     */
-  DFSSM_OP_LM_HEAD = 4         /* a = 1,  b = d,     c = V                             */
+  DFSSM_OP_LM_HEAD = 4,        /* a = 1,  b = d,     c = V                             */
+  DFSSM_OP_HEAD_GREEDY = 5,    /* a = 1,  b = d,     c = V                             */
+  DFSSM_OP_GENERATE = 6        /* a = V,  b = d_model, c = d_inner                     */
 };
 size_t dfssm_workspace_size(int op, int a, int b, int c);
 
@@ -219,6 +221,53 @@ int dfssm_lm_head(const int8_t* W, const float* s_row, int V, int d, const float
                   int32_t* acc, void* workspace, size_t ws_bytes, void* stream);
 
 /*
+ * Token embedding from the tied int8 embedding / LM-head matrix (technical summary §2.B: the embedding
+ * and LM head are int8 with per-row scaling; §3: together they are 37% of the 278 MB model, i.e. one
+ * V x d_model matrix, read here as shared by both).
+ *   W device i8 [V][d] (16-byte aligned, d % 16 == 0, d <= 8192), s_row device f32 [V],
+ *   token device i32 [1] (read on the device when the stream reaches the call), h device f32 [d]
+ *   (16-byte aligned).   h[i] = fl32(W[tok, i] * s_row[tok]).
+ * A token outside [0, V) writes h = 0 and records a sticky code in the library's status word:
+ * dfssm_device_status then returns DFSSM_EINVAL.  One single-CTA kernel.
+ */
+int dfssm_embed(const int8_t* W, const float* s_row, int V, int d, const int32_t* token, float* h,
+                void* stream);
+
+/*
+ * Final RMSNorm + int8 LM head + greedy choice on one token (the Mamba-2 language model's final norm
+ * before its LM head, a reading of the cited architecture; the head as in dfssm_lm_head).
+ *   h device f32 [d] (the residual stream after the last layer); norm_w device f32 [d] or NULL (then no
+ *   norm: the logits are exactly dfssm_lm_head's).  With norm_w the RMS factor is folded into the
+ *   quantizer scale: (q, s0) = quant(fl32(h w)), s = fl32(s0 / sqrt(sum h^2 / d + 1e-5)) (fp64), and
+ *   logits[v] = fl32(acc[v] s s_row[v]), acc[v] = sum_i W[v,i] q[i].
+ *   token device i32 [1] receives the index of the largest logit (the smallest index on ties; -0 and +0
+ *   are equal).  logits device f32 [V] (required), acc device i32 [V] or NULL.
+ *   workspace: dfssm_workspace_size(DFSSM_OP_HEAD_GREEDY, 1, d, V) bytes, zero-filled before its first
+ *   use; each call leaves it zero again.  One kernel.
+ */
+int dfssm_head_greedy(const int8_t* W, const float* s_row, int V, int d, const float* h,
+                      const float* norm_w, float* logits, int32_t* acc, int32_t* token, void* workspace,
+                      size_t ws_bytes, void* stream);
+
+/*
+ * Greedy generation at batch 1 (technical summary §2.C: the 48-layer decode step, with the int8
+ * embedding and LM head of §2.B): for t = 0 .. n_tokens-1
+ *   h = embed(tokens[t]);  dfssm_layer_decode(layers, h);  tokens[t+1] = greedy(final_head(h)).
+ *   tokens device i32 [n_tokens + 1]: tokens[0] is the first token (set by the caller), the rest are
+ *   written.  W, s_row, V as for dfssm_embed; final_norm_w device f32 [d_model].  Layers, dims and
+ *   states as for dfssm_layer_decode with B = 1 (the states advance by n_tokens steps).
+ *   hidden_taps device f32 [n_tokens][d_model] or NULL: the residual stream after the last layer at each
+ *   step.  logits (device f32 [V] or NULL) receives the last step's logits.
+ *   workspace: dfssm_workspace_size(DFSSM_OP_GENERATE, V, d_model, d_inner), zero-filled before its first
+ *   use.  Three kernels per token (embedding, the layers, the head); the calls are stream-ordered and
+ *   can be captured in a CUDA graph.
+ */
+int dfssm_generate(const dfssm_layer_t* layers, int n_layers, const dfssm_dims_t* dims,
+                   const int8_t* W, const float* s_row, int V, const float* final_norm_w,
+                   int32_t* tokens, int n_tokens, float* const* conv_states, float* const* ssm_states,
+                   float* hidden_taps, float* logits, void* workspace, size_t ws_bytes, void* stream);
+
+/*
  * Device-side failure detection of dfssm_layer_decode.  The fused decode kernel (batch 1, Mamba-2-1.3B
  * shape) hands data between its CTAs through counters in the workspace; every wait has a clock budget
  * (about one second).  A wait that runs out makes every CTA of that launch return early (its outputs are
@@ -227,7 +276,8 @@ int dfssm_lm_head(const int8_t* W, const float* s_row, int V, int d, const float
  * bound their shared-memory pipeline waits the same way and record a timeout in a status word of the
  * library's own device memory (one per device).  dfssm_device_status synchronises `stream`, reads and
  * clears the workspace status word (workspace may be NULL: then only the library's word) and the
- * library's word, and returns DFSSM_OK or DFSSM_ETIMEOUT.  No device trap or fault is ever raised.
+ * library's word, and returns DFSSM_OK, DFSSM_ETIMEOUT, or DFSSM_EINVAL when the only recorded event is
+ * an out-of-range token given to dfssm_embed.  No device trap or fault is ever raised.
  */
 int dfssm_device_status(void* workspace, void* stream);
 

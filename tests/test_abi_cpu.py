@@ -37,7 +37,7 @@ def test_library_exports_every_declared_symbol(L):
     for n in names:
         assert hasattr(L, n), f"{n} declared in dfssm.h but not exported"
     assert set(names) == set(dfssm.SIGNATURES), "binding and header disagree"
-    assert L.dfssm_abi_version() == 2
+    assert L.dfssm_abi_version() == 3
 
 
 def test_status_strings(L):
@@ -52,6 +52,10 @@ def test_workspace_sizes(L):
     assert dfssm.workspace_size(dfssm.OP_LINEAR_DECODE, 1, 100, 8512) == 0
     assert dfssm.workspace_size(dfssm.OP_LAYER_DECODE, 1, 2048, 4096) > 8512 * 4
     assert dfssm.workspace_size(dfssm.OP_LM_HEAD, 1, 2048, 50288) >= 2048
+    assert dfssm.workspace_size(dfssm.OP_HEAD_GREEDY, 1, 2048, 50288) >= 16
+    gen = dfssm.workspace_size(dfssm.OP_GENERATE, 50288, 2048, 4096)
+    assert gen >= dfssm.workspace_size(dfssm.OP_LAYER_DECODE, 1, 2048, 4096) + 4 * (2048 + 50288) + 16
+    assert dfssm.workspace_size(dfssm.OP_GENERATE, 0, 2048, 4096) == 0
 
 
 def test_argument_validation_precedes_device_use(L):
@@ -72,6 +76,19 @@ def test_argument_validation_precedes_device_use(L):
     assert L.dfssm_ssm_step(16, 16, 16, 16, 16, 16, 16, 16, 16, 1, 4, 4, 6, 1, None) == -3  # N % 4
     assert L.dfssm_conv_step(None, 16, 16, 16, 16, 1, 8, None) == -1
     assert L.dfssm_lm_head(16, 16, 10, 24, 16, 16, None, 256, 1 << 20, None) == -1  # d % 16
+    assert L.dfssm_embed(16, 16, 10, 24, 16, 16, None) == -1                         # d % 16
+    assert L.dfssm_embed(16, 16, 10, 32, 16, 8, None) == -2                          # h misaligned
+    assert L.dfssm_embed(16, 16, 10, 32, None, 16, None) == -1                       # no token
+    assert L.dfssm_head_greedy(16, 16, 10, 32, 16, None, 16, None, 16, None, 256, None) == -7
+    assert L.dfssm_head_greedy(16, 16, 10, 32, 16, None, None, None, 16, 256, 256, None) == -1
+    assert L.dfssm_head_greedy(16, 16, 10, 16384, 16, None, 16, None, 16, 256, 256, None) == -3
+    dims = dfssm.DimsT(2048, 64, 64, 128, 1)
+    assert L.dfssm_generate(None, 48, C.byref(dims), 16, 16, 10, 16, 16, 0, None, None, None, None,
+                            256, 1 << 30, None) == -1                                 # n_tokens 0
+    assert L.dfssm_generate(None, 48, C.byref(dims), 16, 16, 10, 16, 16, 4, None, None, None, None,
+                            256, 1024, None) == -7                                    # workspace
+    assert L.dfssm_generate(None, 48, C.byref(dims), 16, 16, 10, 16, 16, 4, None, None, None, None,
+                            256, 1 << 30, None) == -1                                 # no layers
 
 
 def test_pack_signs_matches_oracle_bit_layout(L):
