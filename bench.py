@@ -410,6 +410,64 @@ def run_ours(args, rank, world, local_rank):
         prefill["int8_peak_TOPS"] = round(int8_peak, 1)
         prefill["int8_peak_kind"] = "measured bf16 burst x 2 (nominal int8/bf16 ratio)"
         del W
+    # ---- greedy generation: embedding + the 48 layers + final RMSNorm / int8 LM head / argmax per token,
+    # 64 tokens captured in one CUDA graph (the bench's stack, the tied 50288 x 2048 matrix of seed 5)
+    generate = {}
+    if not args.no_extras:
+        gm = inputs.generation_model(seed=5, n_layers=0)
+        GW = torch.from_numpy(gm["emb_w"]).to(dev)
+        Gs = torch.from_numpy(gm["emb_s"]).to(dev)
+        Gn = torch.from_numpy(gm["final_norm_w"]).to(dev)
+        V = GW.shape[0]
+        toks = torch.zeros(N_TOKENS + 1, dtype=torch.int32, device=dev)
+        toks[0] = gm["first_token"]
+        gws = dfssm.workspace(dfssm.workspace_size(dfssm.OP_GENERATE, V, 2048, 4096), dev)
+        with torch.cuda.stream(stream):
+            dfssm.generate(stack, GW, Gs, Gn, toks, ws=gws, stream=torch.cuda.current_stream())
+        torch.cuda.synchronize()
+        ggraph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(ggraph, stream=stream):
+            dfssm.generate(stack, GW, Gs, Gn, toks, ws=gws, stream=torch.cuda.current_stream())
+        torch.cuda.synchronize()
+        with torch.cuda.stream(stream):
+            for _ in range(2):
+                ggraph.replay()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            reps = 3
+            a.record()
+            for _ in range(reps):
+                ggraph.replay()
+            b.record()
+        torch.cuda.synchronize()
+        g_us = a.elapsed_time(b) * 1e3 / (reps * N_TOKENS)
+        # the head alone (final norm + LM head + greedy choice), L2 flushed before each call
+        hidden = torch.from_numpy(inputs.normal(np.random.default_rng(9), (2048,))).to(dev)
+        hws = dfssm.workspace(dfssm.workspace_size(dfssm.OP_HEAD_GREEDY, 1, 2048, V), dev)
+        lg = torch.empty(V, dtype=torch.float32, device=dev)
+        tk = torch.empty(1, dtype=torch.int32, device=dev)
+        with torch.cuda.stream(stream):
+            for _ in range(3):
+                dfssm.head_greedy(GW, Gs, hidden, Gn, lg, token=tk, ws=hws, stream=torch.cuda.current_stream())
+            torch.cuda.synchronize()
+            tot = 0.0
+            for r in range(10):
+                flush.fill_(r & 0xFF)
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record()
+                dfssm.head_greedy(GW, Gs, hidden, Gn, lg, token=tk, ws=hws, stream=torch.cuda.current_stream())
+                b.record()
+                b.synchronize()
+                tot += a.elapsed_time(b)
+        head_us = tot * 1e3 / 10
+        head_bytes = GW.numel() + 4 * V + 2 * 4 * 2048
+        generate = {"tokens_per_s": round(1e6 / g_us, 1), "us_per_token": round(g_us, 2),
+                    "kernels_per_token": 3, "engine": "CUDA graph of 64 dfssm_generate steps",
+                    "head_us_per_call": round(head_us, 2),
+                    "head_GB_s": round(head_bytes / (head_us * 1e-6) / 1e9, 1),
+                    "head_frac_of_measured_hbm": round(head_bytes / (head_us * 1e-6) / 1e9 / hbm, 3),
+                    "last_token": int(toks[-1].item())}
+        ggraph = None
+        del GW
     del flush
     torch.cuda.synchronize()
 
@@ -435,6 +493,7 @@ def run_ours(args, rank, world, local_rank):
         "roofline": roofline,
         "scaffold_gemv": gemv,
         "prefill": prefill,
+        "generate": generate,
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": N_TOKENS * 2048 * 4,
                 "d2h_bytes_per_step": 2048 * 4},
         "gpu_launches": args.steps * N_TOKENS,
