@@ -89,6 +89,24 @@ GenerateWs generate_ws(int V, int d_model, int d_inner) {
   return g;
 }
 
+// Layer-prefill workspace: [zxbcdt f32 M x d_ip][xc f32 M x C][g f32 M x E][linear-prefill region], with
+// C and d_ip at their largest supported values (2 ngroups d_state <= 2048, nheads <= 1024).
+struct PrefillLayerWs {
+  size_t zx, xc, g, lin, total;
+};
+PrefillLayerWs prefill_layer_ws(int M, int d_model, int E) {
+  PrefillLayerWs w;
+  const size_t C = (size_t)E + 2048, d_ip = 2 * (size_t)E + 2048 + 1024;
+  w.zx = 0;
+  w.xc = w.zx + align256(sizeof(float) * (size_t)M * d_ip);
+  w.g = w.xc + align256(sizeof(float) * (size_t)M * C);
+  w.lin = w.g + align256(sizeof(float) * (size_t)M * E);
+  const size_t a = dfssm::prefill_workspace_bytes(M, d_model, (int)d_ip);
+  const size_t b = dfssm::prefill_workspace_bytes(M, E, d_model);
+  w.total = w.lin + align256(a > b ? a : b);
+  return w;
+}
+
 int check_head(const int8_t* W, const float* s_row, int V, int d) {
   if (!W || !s_row || V < 1 || d < 16 || d % 16) return DFSSM_EINVAL;
   if (d > 8192) return DFSSM_EUNSUPPORTED;
@@ -308,6 +326,9 @@ size_t dfssm_workspace_size(int op, int a, int b, int c) {
     case DFSSM_OP_GENERATE:
       if (a < 1 || b < 32 || b % 32 || b > 8192 || c < 32) return 0;
       return generate_ws(a, b, c).total;
+    case DFSSM_OP_LAYER_PREFILL:
+      if (a < 1 || b < 128 || b % 128 || b > 8192 || c < 128 || c % 128 || c > 8192) return 0;
+      return prefill_layer_ws(a, b, c).total;
     default: return 0;
   }
 }
@@ -541,6 +562,82 @@ int dfssm_generate(const dfssm_layer_t* layers, int n_layers, const dfssm_dims_t
     const cudaError_t e =
         cudaMemcpyAsync(logits, lg, sizeof(float) * (size_t)V, cudaMemcpyDeviceToDevice, s);
     if (e != cudaSuccess) return cuda_fail(e);
+  }
+  return DFSSM_OK;
+}
+
+int dfssm_layer_prefill(const dfssm_layer_t* layers, int n_layers, const dfssm_dims_t* dims,
+                        float* hidden, float* const* conv_states, float* const* ssm_states, int M,
+                        void* workspace, size_t ws_bytes, void* stream) {
+  if (!layers || !dims || !hidden || !conv_states || !ssm_states || n_layers < 1 || M < 1)
+    return DFSSM_EINVAL;
+  if (n_layers > DFSSM_MAX_LAYERS) return DFSSM_EUNSUPPORTED;
+  const int Dm = dims->d_model, H = dims->nheads, P = dims->headdim, N = dims->d_state, G = dims->ngroups;
+  if (Dm < 32 || H < 1 || P < 1 || N < 4 || G < 1 || H % G) return DFSSM_EINVAL;
+  const int E = H * P;
+  const int C = E + 2 * G * N;
+  const int d_ip = 2 * E + 2 * G * N + H;
+  if (Dm % 128 || E % 128 || Dm > 8192 || E > 8192 || 2 * G * N > 2048 || H > 1024 ||
+      !dfssm::scan_supported(H, P, N, G))
+    return DFSSM_EUNSUPPORTED;
+  if (!aligned(hidden, 16)) return DFSSM_EALIGN;
+  for (int l = 0; l < n_layers; ++l) {
+    const dfssm_layer_t& Ly = layers[l];
+    int st = check_linear(&Ly.in_proj);
+    if (st) return st;
+    st = check_linear(&Ly.out_proj);
+    if (st) return st;
+    if (Ly.in_proj.d_out != d_ip || Ly.in_proj.d_in != Dm || Ly.out_proj.d_out != Dm ||
+        Ly.out_proj.d_in != E)
+      return DFSSM_EINVAL;
+    if (!Ly.conv_w || !Ly.conv_b || !Ly.A_log || !Ly.dt_bias || !Ly.D || !Ly.norm_w || !Ly.gnorm_w)
+      return DFSSM_EINVAL;
+    if (!conv_states[l] || !ssm_states[l]) return DFSSM_EINVAL;
+    if (!aligned(Ly.conv_w, 16) || !aligned(ssm_states[l], 16) || !aligned(Ly.norm_w, 16) ||
+        !aligned(Ly.gnorm_w, 16))
+      return DFSSM_EALIGN;
+  }
+  const PrefillLayerWs w = prefill_layer_ws(M, Dm, E);
+  if (!workspace || !aligned(workspace, 256) || ws_bytes < w.total) return DFSSM_EWORKSPACE;
+  if (!device_ok()) return DFSSM_EDEVICE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  char* base = static_cast<char*>(workspace);
+  float* zx = reinterpret_cast<float*>(base + w.zx);
+  float* xc = reinterpret_cast<float*>(base + w.xc);
+  float* g = reinterpret_cast<float*>(base + w.g);
+  void* lin_ws = base + w.lin;
+  const size_t lin_bytes = ws_bytes - w.lin;
+  for (int l = 0; l < n_layers; ++l) {
+    const dfssm_layer_t& Ly = layers[l];
+    int st = dfssm::linear_prefill_impl(&Ly.in_proj, hidden, M, zx, Ly.norm_w, false, lin_ws, lin_bytes,
+                                        nullptr, stream);
+    if (st) return st;
+    dfssm::ConvSeqArgs ca{zx, d_ip, E, conv_states[l], Ly.conv_w, Ly.conv_b, xc, M, C};
+    cudaError_t e = dfssm::launch_conv_seq(ca, s);
+    if (e != cudaSuccess) return cuda_fail(e);
+    dfssm::ScanArgs sa{};
+    sa.zx = zx;
+    sa.ld_zx = d_ip;
+    sa.dt_off = E + C;
+    sa.xc = xc;
+    sa.ld_xc = C;
+    sa.b_off = E;
+    sa.c_off = E + G * N;
+    sa.A_log = Ly.A_log;
+    sa.dt_bias = Ly.dt_bias;
+    sa.D = Ly.D;
+    sa.state = ssm_states[l];
+    sa.g = g;
+    sa.M = M;
+    sa.H = H;
+    sa.P = P;
+    sa.N = N;
+    sa.G = G;
+    e = dfssm::launch_ssm_scan(sa, s);
+    if (e != cudaSuccess) return cuda_fail(e);
+    st = dfssm::linear_prefill_impl(&Ly.out_proj, g, M, hidden, Ly.gnorm_w, true, lin_ws, lin_bytes,
+                                    nullptr, stream);
+    if (st) return st;
   }
   return DFSSM_OK;
 }

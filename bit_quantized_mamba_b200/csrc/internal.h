@@ -82,6 +82,37 @@ struct SsmArgs {
 };
 cudaError_t launch_ssm(const SsmArgs& a, cudaStream_t st);
 
+// Sequence conv of a prompt (B = 1): xc[t][c] for t < M from the in_proj output rows zx[t][x_off + c]
+// and the incoming shift-register state [C][3] (oldest first), then the state is advanced by M tokens.
+struct ConvSeqArgs {
+  const float* zx;
+  int ld_zx, x_off;
+  float* state;
+  const float* w;  // [C][4], 16-byte aligned
+  const float* b;
+  float* xc;       // [M][C]
+  int M, C;
+};
+cudaError_t launch_conv_seq(const ConvSeqArgs& a, cudaStream_t st);
+
+// Sequence SSM scan of a prompt (B = 1) with the gate: g[t][h*P+p] for t < M; the state [H][P][N]
+// advances by M tokens.  z at column 0 and dt_raw at column dt_off of zx rows; x at column 0, B at b_off
+// and C at c_off (group g at + g*N) of xc rows.
+struct ScanArgs {
+  const float* zx;
+  int ld_zx, dt_off;
+  const float* xc;
+  int ld_xc, b_off, c_off;
+  const float* A_log;
+  const float* dt_bias;
+  const float* D;
+  float* state;
+  float* g;        // [M][H*P]
+  int M, H, P, N, G;
+};
+cudaError_t launch_ssm_scan(const ScanArgs& a, cudaStream_t st);
+bool scan_supported(int H, int P, int N, int G);
+
 struct Int8GemvArgs {
   const int8_t* W;
   const float* s_row;
@@ -120,6 +151,12 @@ size_t prefill_workspace_bytes(int M, int d_in, int d_out);
 
 // Fused persistent decode (one cooperative launch per token through all layers).
 size_t fused_decode_workspace_bytes();
+
+// dfssm_linear_prefill with two options for the layer prefill: a norm weight folded into the per-token
+// quantizer (norm_w, may be NULL), and a residual epilogue (y[m][n] = fl32(y[m][n] + out)).
+int linear_prefill_impl(const dfssm_linear_t* lin, const float* x, int M, float* y, const float* norm_w,
+                        bool resid, void* workspace, size_t ws_bytes, const dfssm_debug_t* dbg,
+                        void* stream);
 bool fused_decode_supported(const dfssm_dims_t& d, int B, const dfssm_layer_t* layers, int n,
                             float* const* conv_states);
 cudaError_t launch_fused_decode(const dfssm_layer_t* layers, int n_layers, float* hidden,

@@ -6,18 +6,17 @@
 //      LoRA down-projection (fp32, one warp per token);
 //   2. expand the packed sign bits once to +-1 int8 rows in the workspace;
 //   3. acc[m][n] = sum_k q[m][k] w[n][k] on tcgen05.mma kind::i8 (128x128 tiles, K steps of 128 bytes,
-//      TMA loads with 128-byte swizzle into a 4-stage shared-memory ring, a persistent kernel), and
-//      the LoRA-up sum_r W_A[n][r] tf[m][r] on the tensor core as well (bf16 operands, fp32
-//      accumulation, tf split into two bf16 halves), then the epilogue reads both accumulators and writes
-//      y[m][n] = acc s[m] sW[n] + sA[n] lora[m][n] while the next tile accumulates.
-// The integer accumulators are exact; the LoRA-up and the epilogue are fp32.
+//      TMA loads with 128-byte swizzle into a 4-stage shared-memory ring, a persistent kernel); the
+//      epilogue reads the accumulator from tensor memory while the next tile accumulates and forms
+//      y[m][n] = fl32(acc s[m] sW[n] + sA[n] sum_r W_A[n][r] tf[m][r]) in fp64 with the decode path's
+//      rounding sequence (the rank-16 LoRA-up is 16 multiply-adds per output, far below the scaffold's K).
+// The integer accumulators are exact and every output equals the decode definition bit for bit.
 //
 // Every wait on an mbarrier is bounded: a wait that runs out of budget sets the workspace error word,
 // the CTA stops issuing work, waits (bounded) for its copies in flight, frees its tensor memory and
 // returns.
 
 #include <cuda.h>
-#include <cuda_bf16.h>
 #include <cudaTypedefs.h>
 
 #include <cstdio>
@@ -33,12 +32,6 @@ constexpr int BM = 128, BN = 128, BK = 128;  // tile; BK bytes = BK int8 element
 constexpr int STAGES = 4;
 constexpr int UMMA_K = 32;                   // K of one kind::i8 MMA (bytes)
 constexpr int A_BYTES = BM * BK, B_BYTES = BN * BK, STAGE_BYTES = A_BYTES + B_BYTES;
-// LoRA-up on the tensor core: per tile, A_l = [tf_hi | tf_lo] of the tile's rows and B_l = [W_A | W_A] of
-// its columns, bf16, each row padded to 128 bytes (the 128-byte swizzle of the main operands); two
-// kind::f16 MMAs (K = 16 each) give sum_r W_A tf_hi + sum_r W_A tf_lo in an fp32 accumulator.
-constexpr int LROW = 128;                    // bytes per LoRA operand row (64 bf16, 32 used)
-constexpr int LA_BYTES = BM * LROW, LB_BYTES = BN * LROW, LSTAGE_BYTES = LA_BYTES + LB_BYTES;
-constexpr int UMMA_K16 = 32;                 // K of one kind::f16 MMA: 16 bf16 = 32 bytes
 constexpr long long kWaitBudget = 4000000000LL;  // clock cycles per wait (~2 s)
 
 struct EpiArgs {
@@ -48,8 +41,11 @@ struct EpiArgs {
   int rank;
   float* y;             // [M][N]
   int32_t* acc;         // [M][N] or null
+  const float* tf;      // [M][16] LoRA intermediates (zero beyond the rank)
+  const int8_t* lora_a; // [N][rank]
   int M, N, K;
   int* err;
+  int resid;            // 1: y[m][n] = fl32(y[m][n] + out) (residual add in place), 0: y = out
 };
 
 // ------------------------------------------------------------------------------ PTX helpers
@@ -106,9 +102,6 @@ __device__ __forceinline__ uint64_t umma_desc_k_sw128(uint32_t smem_addr) {
 // kind::i8 instruction descriptor: D s32, A s8, B s8, both K-major, M = BM, N = BN.
 constexpr uint32_t kIdesc = (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
                             ((uint32_t)(BM >> 4) << 24);
-// kind::f16 instruction descriptor: D f32, A bf16, B bf16, both K-major, M = BM, N = BN.
-constexpr uint32_t kIdescBf16 = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
-                                ((uint32_t)(BM >> 4) << 24);
 
 __device__ __forceinline__ void umma_i8(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t accum) {
   asm volatile(
@@ -116,14 +109,6 @@ __device__ __forceinline__ void umma_i8(uint32_t tmem_d, uint64_t adesc, uint64_
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
       "l"(adesc), "l"(bdesc), "r"(kIdesc), "r"(accum)
-      : "memory");
-}
-__device__ __forceinline__ void umma_bf16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t accum) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
-      "l"(adesc), "l"(bdesc), "r"(kIdescBf16), "r"(accum)
       : "memory");
 }
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
@@ -140,12 +125,6 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
         "=r"(r[15])
       : "r"(taddr));
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-}
-
-// Exact fp32 value of a small integer (|w| < 2^22) without the conversion unit: the bit pattern of
-// 1.5 * 2^23 plus w is the float 1.5 * 2^23 + w.
-__device__ __forceinline__ float int8_to_f32(int w) {
-  return __int_as_float(0x4B400000 + w) - 12582912.0f;
 }
 
 // ------------------------------------------------------------------------------ kernels
@@ -174,16 +153,17 @@ __global__ void expand_bits_kernel(const uint32_t* __restrict__ bits, int8_t* __
 // decode quantizer; the LoRA down-projection t = W_B q on the codes (int32, dp4a) with W_B staged in
 // shared memory (zero rows beyond the rank, so every lane runs all sixteen rows without branches), and
 // tf = fl32(t sB s) rounded as in the decode path.  Each lane keeps eight 16-byte loads of its token in
-// flight.
+// flight.  With a norm weight (a layer's pre-norm or gated norm) the RMSNorm is folded in as in decode:
+// the codes are those of v = fl32(x w), and s = fl32(s0 / rms), rms = sqrt(sum x^2 / K + 1e-5) (fp64).
 constexpr int QW = 8;  // tokens (warps) per CTA
 constexpr int QU = 8;  // float4 loads in flight per lane
 __global__ void __launch_bounds__(QW * 32) prefill_quant_kernel(const float* __restrict__ x, int M, int K,
                                                                const int8_t* __restrict__ lora_b,
                                                                const float* __restrict__ lora_b_scale,
-                                                               int rank, int8_t* __restrict__ xq,
+                                                               int rank, const float* __restrict__ norm_w,
+                                                               int8_t* __restrict__ xq,
                                                                float* __restrict__ s_out,
                                                                float* __restrict__ tf_out,
-                                                               uint16_t* __restrict__ tfhl,
                                                                int8_t* dbg_xq, float* dbg_s, int32_t* dbg_t) {
   extern __shared__ __align__(16) unsigned char sm[];
   int8_t* wb = reinterpret_cast<int8_t*>(sm);  // [16][K]
@@ -222,14 +202,33 @@ __global__ void __launch_bounds__(QW * 32) prefill_quant_kernel(const float* __r
   const int m = blockIdx.x * QW + warp;
   if (m >= M) return;
   const float4* xr = reinterpret_cast<const float4*>(x + (size_t)m * K);
+  const float4* wr = reinterpret_cast<const float4*>(norm_w);
   const int K4 = K / 4;  // a multiple of 32: the bounds tests below are uniform over the warp
   constexpr int UB = QU;  // float4 per lane per batch
+  // v = fl32(x w) with a norm weight, else x
+  const auto scale4 = [&](float4 a, int i) {
+    if (!wr) return a;
+    const float4 w = __ldg(wr + i);
+    return make_float4(fmul(a.x, w.x), fmul(a.y, w.y), fmul(a.z, w.z), fmul(a.w, w.w));
+  };
   float m_abs = 0.0f;
+  double ss = 0.0;
   for (int i0 = lane; i0 < K4; i0 += 32 * UB) {
     float4 v[UB];
 #pragma unroll
     for (int u = 0; u < UB; ++u)
       v[u] = i0 + 32 * u < K4 ? __ldg(xr + i0 + 32 * u) : make_float4(0.f, 0.f, 0.f, 0.f);
+    if (wr) {
+#pragma unroll
+      for (int u = 0; u < UB; ++u) {
+        // squares of fp32 values are exact in fp64
+        ss = fma((double)v[u].x, (double)v[u].x, ss);
+        ss = fma((double)v[u].y, (double)v[u].y, ss);
+        ss = fma((double)v[u].z, (double)v[u].z, ss);
+        ss = fma((double)v[u].w, (double)v[u].w, ss);
+        if (i0 + 32 * u < K4) v[u] = scale4(v[u], i0 + 32 * u);
+      }
+    }
 #pragma unroll
     for (int u = 0; u < UB; ++u)
       m_abs = fmaxf(m_abs, fmaxf(fmaxf(fabsf(v[u].x), fabsf(v[u].y)), fmaxf(fabsf(v[u].z), fabsf(v[u].w))));
@@ -237,6 +236,7 @@ __global__ void __launch_bounds__(QW * 32) prefill_quant_kernel(const float* __r
   m_abs = warp_max(m_abs);
   const float s0 = m_abs == 0.0f ? 0.0f : __fdiv_rn(m_abs, 127.0f);
   const float inv_s0 = m_abs == 0.0f ? 0.0f : __frcp_rn(s0);
+  const float s_tok = wr ? rms_scale(s0, rms_of(warp_sum(ss), K)) : s0;
   int u[DFSSM_MAX_RANK];
 #pragma unroll
   for (int r = 0; r < DFSSM_MAX_RANK; ++r) u[r] = 0;
@@ -249,7 +249,8 @@ __global__ void __launch_bounds__(QW * 32) prefill_quant_kernel(const float* __r
     for (int q = 0; q < UB; ++q) {
       const int i = i0 + 32 * q;
       if (i < K4) {
-        const float vv[4] = {v[q].x, v[q].y, v[q].z, v[q].w};
+        const float4 vs = scale4(v[q], i);
+        const float vv[4] = {vs.x, vs.y, vs.z, vs.w};
         int cd[4];
         quant_codes<4>(vv, s0, inv_s0, cd);
         uint32_t packed = 0;
@@ -271,70 +272,28 @@ __global__ void __launch_bounds__(QW * 32) prefill_quant_kernel(const float* __r
 #pragma unroll
     for (int r = 0; r < DFSSM_MAX_RANK; ++r)
       if (r == lane) tv = u[r];
-    tf = lane < rank ? lora_tf(tv, __ldg(lora_b_scale + lane), s0) : 0.0f;
+    tf = lane < rank ? lora_tf(tv, __ldg(lora_b_scale + lane), s_tok) : 0.0f;
     tf_out[(size_t)m * DFSSM_MAX_RANK + lane] = tf;
     if (dbg_t && lane < rank) dbg_t[(size_t)m * rank + lane] = tv;
   }
-  // the LoRA-up operand row of this token: [bf16(tf) | bf16(tf - bf16(tf)) | 0 ...] (64 bf16): the two
-  // halves sum to tf within 2^-16 relative; lane l < 16 writes hi[l], lane 16 + r writes lo[r]
-  {
-    const float tr = __shfl_sync(0xffffffffu, tf, lane & 15);
-    const __nv_bfloat16 hi = __float2bfloat16_rn(tr);
-    const __nv_bfloat16 lo = __float2bfloat16_rn(tr - __bfloat162float(hi));
-    uint16_t* row = tfhl + (size_t)m * (LROW / 2);
-    row[lane] = __bfloat16_as_ushort(lane < 16 ? hi : lo);
-    row[32 + lane] = 0;
-  }
   if (lane == 0) {
-    s_out[m] = s0;
-    if (dbg_s) dbg_s[m] = s0;
+    s_out[m] = s_tok;
+    if (dbg_s) dbg_s[m] = s_tok;
   }
-}
-
-// The LoRA-up operand row of output column n: [W_A[n] | W_A[n] | 0 ...] as 64 bf16 (int8 values are
-// exact in bf16; zero beyond the rank).  One thread per 16-byte chunk of a row (eight per row): chunks 0/1
-// and 2/3 hold W_A[n][0..7] / W_A[n][8..15], chunks 4..7 are zero.
-__global__ void lora_a_bf16_kernel(const int8_t* __restrict__ la, int rank, int N, uint4* __restrict__ out) {
-  const long long t = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-  if (t >= 8LL * N) return;
-  const int n = (int)(t >> 3), ch = (int)(t & 7);
-  uint4 o = make_uint4(0u, 0u, 0u, 0u);
-  if (ch < 4) {
-    const int r0 = 8 * (ch & 1);
-    int wv[8];
-    if (rank == 16) {  // 16-byte aligned rows at rank 16
-      const uint2 q = __ldg(reinterpret_cast<const uint2*>(la + (size_t)n * 16 + r0));
-      const uint32_t qw[2] = {q.x, q.y};
-#pragma unroll
-      for (int r = 0; r < 8; ++r) wv[r] = (int)(int8_t)(qw[r >> 2] >> (8 * (r & 3)));
-    } else {
-#pragma unroll
-      for (int r = 0; r < 8; ++r) wv[r] = r0 + r < rank ? (int)la[(size_t)n * rank + r0 + r] : 0;
-    }
-    uint32_t pk[4];
-#pragma unroll
-    for (int r2 = 0; r2 < 4; ++r2)
-      pk[r2] = (__float_as_uint(int8_to_f32(wv[2 * r2])) >> 16) |
-               (__float_as_uint(int8_to_f32(wv[2 * r2 + 1])) & 0xFFFF0000u);
-    o = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-  }
-  out[(size_t)n * (LROW / 16) + ch] = o;
 }
 
 // Persistent tcgen05 GEMM: one CTA per SM walks the 128 x 128 output tiles; warp 0 streams A/B stages
-// (and each tile's LoRA operands) with TMA, warp 1 issues the MMAs (the int8 scaffold product into one
-// of two int32 accumulators, then the LoRA-up into the matching fp32 accumulator), warps 2..9 drain the
-// other pair (two warps per 32-lane TMEM quadrant, each taking half of the 128 columns), so a tile's
-// epilogue overlaps the next tile's main loop.  TMEM columns: [0, 256) int32 accumulators, [256, 512)
-// fp32 LoRA accumulators.
+// with TMA, warp 1 issues the int8 MMAs into one of two int32 accumulators, warps 2..9 drain the other
+// one (two warps per 32-lane TMEM quadrant, each taking half of the 128 columns) and evaluate the fp64
+// epilogue, so a tile's epilogue overlaps the next tile's main loop.  TMEM columns: [0, 256).
 constexpr int EPI_WARPS = 8;
 constexpr int PNT = 64 + EPI_WARPS * 32;   // 320 threads
-constexpr int PTMEM_COLS = 4 * BN;         // two (int32, fp32) accumulator pairs of BN columns
+constexpr int PTMEM_COLS = 2 * BN;         // two int32 accumulators of BN columns
 constexpr int STG_LD = 17;                 // staging row stride (floats): conflict-free both ways
-constexpr size_t OFF_LORA = (size_t)STAGES * STAGE_BYTES;
-constexpr size_t OFF_BARS = OFF_LORA + 2 * (size_t)LSTAGE_BYTES;
+constexpr size_t OFF_BARS = (size_t)STAGES * STAGE_BYTES;
 constexpr size_t OFF_COLS = OFF_BARS + 512;
-constexpr size_t OFF_STG = OFF_COLS + 2 * BN * 8;
+constexpr size_t OFF_WA = OFF_COLS + 2 * BN * 8;   // [2][BN] W_A rows (16 bytes each)
+constexpr size_t OFF_STG = OFF_WA + 2 * BN * 16;
 constexpr size_t PSMEM_BYTES = 1024 + OFF_STG + EPI_WARPS * 32 * STG_LD * 4;
 
 // Bounded wait that ignores the abort flag (used to drain work already issued).
@@ -346,23 +305,20 @@ __device__ __forceinline__ void mbar_wait_drain(uint64_t* bar, uint32_t parity) 
 
 __global__ void __launch_bounds__(PNT, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
-                const __grid_constant__ CUtensorMap map_la, const __grid_constant__ CUtensorMap map_lb,
                 const EpiArgs ep) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  unsigned char* lbase = smem + OFF_LORA;  // [2][LSTAGE_BYTES]
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + OFF_BARS);
   uint64_t* empty = full + STAGES;
   uint64_t* acc_full = empty + STAGES;     // [2] MMA -> epilogue
   uint64_t* acc_empty = acc_full + 2;      // [2] epilogue -> MMA
-  uint64_t* lfull = acc_empty + 2;         // [2] LoRA operands landed
-  uint64_t* lempty = lfull + 2;            // [2] LoRA operands consumed by the MMAs
-  uint64_t* mma_done = lempty + 2;         // every MMA of this CTA complete
+  uint64_t* mma_done = acc_empty + 2;      // every MMA of this CTA complete
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(mma_done + 1);
-  // per-accumulator column parameters of the tile being drained: sW, sA
+  // per-accumulator column parameters of the tile being drained: sW, sA, W_A row
   float* col_sw = reinterpret_cast<float*>(smem + OFF_COLS);  // [2][BN]
   float* col_sa = col_sw + 2 * BN;                            // [2][BN]
+  uint4* col_wa = reinterpret_cast<uint4*>(smem + OFF_WA);    // [2][BN]
   float* stg_all = reinterpret_cast<float*>(smem + OFF_STG);  // [EPI_WARPS][32][STG_LD]
   __shared__ int abort_flag;
 
@@ -380,8 +336,6 @@ __global__ void __launch_bounds__(PNT, 1)
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
       mbar_init(&acc_empty[b], EPI_WARPS);
-      mbar_init(&lfull[b], 1);
-      mbar_init(&lempty[b], 1);
     }
     mbar_init(mma_done, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -399,20 +353,11 @@ __global__ void __launch_bounds__(PNT, 1)
   const uint32_t tmem_base = *tmem_holder;
 
   if (warp == 0 && lane == 0) {
-    // ---- TMA producer: per tile its LoRA operands, then its k-blocks through the stage ring
-    int it = 0, lt = 0;
+    // ---- TMA producer: each tile's k-blocks through the stage ring
+    int it = 0;
     bool ok = true;
-    for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x, ++lt) {
+    for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
       const int n0 = (t % tiles_n) * BN, m0 = (t / tiles_n) * BM;
-      const int lb = lt & 1;
-      if (lt >= 2 && !mbar_wait(&lempty[lb], ((lt >> 1) - 1) & 1, &abort_flag)) {
-        abort_flag = 1;
-        break;
-      }
-      unsigned char* ldst = lbase + lb * LSTAGE_BYTES;
-      mbar_expect_tx(&lfull[lb], LSTAGE_BYTES);
-      tma_load_2d(ldst, &map_la, 0, m0, &lfull[lb]);
-      tma_load_2d(ldst + LA_BYTES, &map_lb, 0, n0, &lfull[lb]);
       for (int kb = 0; kb < kblocks; ++kb, ++it) {
         const int s = it % STAGES;
         if (it >= STAGES && !mbar_wait(&empty[s], ((it / STAGES) - 1) & 1, &abort_flag)) {
@@ -428,7 +373,6 @@ __global__ void __launch_bounds__(PNT, 1)
     }
     // the last copies land before this CTA may exit
     for (int j = (it > STAGES ? it - STAGES : 0); j < it; ++j) mbar_wait_drain(&full[j % STAGES], (j / STAGES) & 1);
-    for (int j = (lt > 2 ? lt - 2 : 0); j < lt; ++j) mbar_wait_drain(&lfull[j & 1], (j >> 1) & 1);
   } else if (warp == 1 && lane == 0) {
     // ---- MMA issuer
     int it = 0, local = 0;
@@ -441,7 +385,6 @@ __global__ void __launch_bounds__(PNT, 1)
       }
       asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
       const uint32_t d_tmem = tmem_base + (uint32_t)(buf * BN);
-      const uint32_t l_tmem = tmem_base + (uint32_t)(2 * BN + buf * BN);
       for (int kb = 0; kb < kblocks; ++kb, ++it) {
         const int s = it % STAGES;
         if (!mbar_wait(&full[s], (it / STAGES) & 1, &abort_flag)) {
@@ -460,19 +403,6 @@ __global__ void __launch_bounds__(PNT, 1)
         issued = true;
       }
       if (!ok) break;
-      // LoRA-up of the tile: [tf_hi | tf_lo] x [W_A | W_A]^T, fp32 accumulation
-      if (!mbar_wait(&lfull[buf], (local >> 1) & 1, &abort_flag)) {
-        abort_flag = 1;
-        break;
-      }
-      asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-      const uint32_t la_addr = smem_u32(lbase + buf * LSTAGE_BYTES);
-      const uint32_t lb_addr = la_addr + LA_BYTES;
-#pragma unroll
-      for (int kk = 0; kk < 2; ++kk)
-        umma_bf16(l_tmem, umma_desc_k_sw128(la_addr + kk * UMMA_K16), umma_desc_k_sw128(lb_addr + kk * UMMA_K16),
-                  kk > 0 ? 1u : 0u);
-      umma_commit(&lempty[buf]);
       umma_commit(&acc_full[buf]);
     }
     // every MMA this thread issued completes before the tensor memory is released
@@ -491,16 +421,32 @@ __global__ void __launch_bounds__(PNT, 1)
     for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++local) {
       const int buf = local & 1;
       const int n0 = (t % tiles_n) * BN, m0 = (t / tiles_n) * BM;
-      // column scales of this tile, staged once per tile
+      // column parameters of this tile, staged once per tile: sW, sA and the W_A row (zero beyond the
+      // rank)
       if (etid < BN) {
         const int n = n0 + etid;
         col_sw[buf * BN + etid] = n < ep.N ? __ldg(ep.w_scale + n) : 0.0f;
         col_sa[buf * BN + etid] = (n < ep.N && ep.rank > 0) ? __ldg(ep.la_scale + n) : 0.0f;
+        uint4 wa = make_uint4(0u, 0u, 0u, 0u);
+        if (n < ep.N && ep.rank == DFSSM_MAX_RANK) {
+          wa = __ldg(reinterpret_cast<const uint4*>(ep.lora_a) + n);  // 16-byte rows at rank 16
+        } else if (n < ep.N) {
+          uint32_t w[4] = {0u, 0u, 0u, 0u};
+          for (int r = 0; r < ep.rank; ++r)
+            w[r >> 2] |= ((uint32_t)(uint8_t)ep.lora_a[(size_t)n * ep.rank + r]) << (8 * (r & 3));
+          wa = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+        col_wa[buf * BN + etid] = wa;
       }
       asm volatile("bar.sync 1, %0;" ::"n"(EPI_WARPS * 32) : "memory");
       const int row = q * 32 + lane;
       const int m = m0 + row;
-      const float sm = m < ep.M ? __ldg(ep.s + m) : 0.f;
+      const double sm = m < ep.M ? (double)__ldg(ep.s + m) : 0.0;
+      // this row's LoRA intermediates in fp64 (exact images of the fp32 values)
+      double tfd[DFSSM_MAX_RANK];
+#pragma unroll
+      for (int r = 0; r < DFSSM_MAX_RANK; ++r)
+        tfd[r] = (m < ep.M && r < ep.rank) ? (double)__ldg(ep.tf + (size_t)m * DFSSM_MAX_RANK + r) : 0.0;
       // every epilogue warp runs every tile iteration (the named barrier above counts on it); after an
       // abort the accumulators are simply not read
       const bool ok = !abort_flag && mbar_wait(&acc_full[buf], (local >> 1) & 1, &abort_flag);
@@ -511,16 +457,34 @@ __global__ void __launch_bounds__(PNT, 1)
       }
       for (int cc = 0; ok && cc < BN / 2; cc += 16) {
         const int c0 = half * (BN / 2) + cc;
-        uint32_t v[16], lv[16];
+        uint32_t v[16];
         tmem_ld16(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * BN + c0), v);
-        tmem_ld16(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(2 * BN + buf * BN + c0), lv);
         float out[16];
+        // y = fl32(acc s sW + sA sum_r W_A tf): the decode path's definition, four outputs interleaved
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const int cidx = buf * BN + c0 + j;
-          const int acc = (int)v[j];
-          out[j] = fmaf((float)acc, sm * col_sw[cidx], col_sa[cidx] * __uint_as_float(lv[j]));
-          if (ep.acc && m < ep.M && n0 + c0 + j < ep.N) ep.acc[(size_t)m * ep.N + n0 + c0 + j] = acc;
+        for (int j0 = 0; j0 < 16; j0 += 4) {
+          int a4[4];
+          double s4[4], w4[4], sa4[4];
+          uint4 wa4[4];
+          const double* tf4[4] = {tfd, tfd, tfd, tfd};
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int cidx = buf * BN + c0 + j0 + j;
+            a4[j] = (int)v[j0 + j];
+            s4[j] = sm;
+            w4[j] = (double)col_sw[cidx];
+            sa4[j] = (double)col_sa[cidx];
+            wa4[j] = col_wa[cidx];
+          }
+          float o4[4];
+          linear_out_n<4, -1>(a4, s4, w4, sa4, wa4, tf4, ep.rank, o4);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) out[j0 + j] = o4[j];
+        }
+        if (ep.acc && m < ep.M) {
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            if (n0 + c0 + j < ep.N) ep.acc[(size_t)m * ep.N + n0 + c0 + j] = (int)v[j];
         }
         // through shared memory: lane l holds row l of the chunk; the stores then write two 64-byte row
         // segments per instruction (lanes 0-15 one row, 16-31 the next)
@@ -532,7 +496,10 @@ __global__ void __launch_bounds__(PNT, 1)
         for (int k = 0; k < 16; ++k) {
           const int r = 2 * k + (lane >> 4);
           const int mr = m0 + q * 32 + r;
-          if (mr < ep.M && n < ep.N) ep.y[(size_t)mr * ep.N + n] = stg[r * STG_LD + cj];
+          if (mr < ep.M && n < ep.N) {
+            float* dst = ep.y + (size_t)mr * ep.N + n;
+            *dst = ep.resid ? fadd(*dst, stg[r * STG_LD + cj]) : stg[r * STG_LD + cj];
+          }
         }
         __syncwarp();
       }
@@ -591,14 +558,12 @@ struct Ws {
   int32_t* sumq;
   float* tf;
   int8_t* w8;
-  uint16_t* tfhl;  // [M][64] bf16 LoRA-up operand rows
-  uint4* la2;      // [N][64] bf16 LoRA-up operand rows
   int* err;
 };
 
 size_t ws_bytes(int M, int K, int N) {
   return al256((size_t)M * K) + al256((size_t)M * 4) * 2 + al256((size_t)M * 16 * 4) +
-         al256((size_t)N * K) + al256((size_t)M * LROW) + al256((size_t)N * LROW) + 256;
+         al256((size_t)N * K) + 256;
 }
 
 Ws carve(void* base, int M, int K, int N) {
@@ -614,10 +579,6 @@ Ws carve(void* base, int M, int K, int N) {
   p += al256((size_t)M * 16 * 4);
   w.w8 = reinterpret_cast<int8_t*>(p);
   p += al256((size_t)N * K);
-  w.tfhl = reinterpret_cast<uint16_t*>(p);
-  p += al256((size_t)M * LROW);
-  w.la2 = reinterpret_cast<uint4*>(p);
-  p += al256((size_t)N * LROW);
   w.err = reinterpret_cast<int*>(p);
   return w;
 }
@@ -631,6 +592,12 @@ size_t prefill_workspace_bytes(int M, int d_in, int d_out) { return prefill::ws_
 extern "C" int dfssm_linear_prefill(const dfssm_linear_t* lin, const float* x, int M, float* y,
                                     void* workspace, size_t ws_bytes, const dfssm_debug_t* dbg,
                                     void* stream) {
+  return dfssm::linear_prefill_impl(lin, x, M, y, nullptr, false, workspace, ws_bytes, dbg, stream);
+}
+
+int dfssm::linear_prefill_impl(const dfssm_linear_t* lin, const float* x, int M, float* y,
+                               const float* norm_w, bool resid, void* workspace, size_t ws_bytes,
+                               const dfssm_debug_t* dbg, void* stream) {
   using namespace dfssm;
   if (!lin || !x || !y || M < 1) return DFSSM_EINVAL;
   if (lin->d_out < 1 || lin->d_in < 128 || lin->d_in % 128 || lin->d_in > 8192) return DFSSM_EINVAL;
@@ -642,6 +609,7 @@ extern "C" int dfssm_linear_prefill(const dfssm_linear_t* lin, const float* x, i
       (reinterpret_cast<uintptr_t>(y) & 15))
     return DFSSM_EALIGN;
   if (lin->rank == DFSSM_MAX_RANK && (reinterpret_cast<uintptr_t>(lin->lora_a) & 15)) return DFSSM_EALIGN;
+  if (norm_w && (reinterpret_cast<uintptr_t>(norm_w) & 15)) return DFSSM_EALIGN;
   if (lin->rank > 0 && (reinterpret_cast<uintptr_t>(lin->lora_b) & 3)) return DFSSM_EALIGN;
   const int K = lin->d_in, N = lin->d_out;
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255) ||
@@ -664,37 +632,35 @@ extern "C" int dfssm_linear_prefill(const dfssm_linear_t* lin, const float* x, i
     qattr = true;
   }
   prefill::prefill_quant_kernel<<<(M + prefill::QW - 1) / prefill::QW, prefill::QW * 32, qsmem, st>>>(
-      x, M, K, lin->lora_b, lin->lora_b_scale, lin->rank, w.xq, w.s, w.tf, w.tfhl, dbg ? dbg->xq : nullptr,
+      x, M, K, lin->lora_b, lin->lora_b_scale, lin->rank, norm_w, w.xq, w.s, w.tf, dbg ? dbg->xq : nullptr,
       dbg ? dbg->xscale : nullptr, dbg ? dbg->lora_t : nullptr);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return record_cuda_failure(e);
-  // 2. +-1 int8 weights, and W_A rows as the bf16 LoRA-up operand
+  // 2. +-1 int8 weights
   const long long words = (long long)N * (K / 32);
   prefill::expand_bits_kernel<<<(unsigned)((words + 255) / 256), 256, 0, st>>>(lin->bits, w.w8, words);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return record_cuda_failure(e);
-  prefill::lora_a_bf16_kernel<<<(unsigned)((8LL * N + 255) / 256), 256, 0, st>>>(lin->lora_a, lin->rank, N, w.la2);
   e = cudaGetLastError();
   if (e != cudaSuccess) return record_cuda_failure(e);
   e = cudaMemsetAsync(w.err, 0, sizeof(int), st);
   if (e != cudaSuccess) return record_cuda_failure(e);
   // 3. tcgen05 GEMM + epilogue
-  CUtensorMap map_a, map_b, map_la, map_lb;
-  if (!prefill::make_map(&map_a, w.xq, M, K, prefill::BM) || !prefill::make_map(&map_b, w.w8, N, K, prefill::BN) ||
-      !prefill::make_map(&map_la, w.tfhl, M, prefill::LROW, prefill::BM) ||
-      !prefill::make_map(&map_lb, w.la2, N, prefill::LROW, prefill::BN))
+  CUtensorMap map_a, map_b;
+  if (!prefill::make_map(&map_a, w.xq, M, K, prefill::BM) || !prefill::make_map(&map_b, w.w8, N, K, prefill::BN))
     return DFSSM_EUNSUPPORTED;
   prefill::EpiArgs ep{};
   ep.s = w.s;
   ep.w_scale = lin->w_scale;
   ep.la_scale = lin->lora_a_scale;
   ep.rank = lin->rank;
+  ep.tf = w.tf;
+  ep.lora_a = lin->lora_a;
   ep.y = y;
   ep.acc = dbg ? dbg->acc : nullptr;
   ep.M = M;
   ep.N = N;
   ep.K = K;
   ep.err = w.err;
+  ep.resid = resid ? 1 : 0;
   static bool attr_done = false;
   if (!attr_done) {
     e = cudaFuncSetAttribute(prefill::gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -704,7 +670,7 @@ extern "C" int dfssm_linear_prefill(const dfssm_linear_t* lin, const float* x, i
   }
   const int tiles = ((N + prefill::BN - 1) / prefill::BN) * ((M + prefill::BM - 1) / prefill::BM);
   const int grid = tiles < num_sms() ? tiles : num_sms();
-  prefill::gemm_kernel<<<grid, prefill::PNT, prefill::PSMEM_BYTES, st>>>(map_a, map_b, map_la, map_lb, ep);
+  prefill::gemm_kernel<<<grid, prefill::PNT, prefill::PSMEM_BYTES, st>>>(map_a, map_b, ep);
   e = cudaGetLastError();
   if (e != cudaSuccess) return record_cuda_failure(e);
   return DFSSM_OK;

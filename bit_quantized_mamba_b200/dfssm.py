@@ -20,6 +20,7 @@ OP_LAYER_DECODE = 3
 OP_LM_HEAD = 4
 OP_HEAD_GREEDY = 5
 OP_GENERATE = 6
+OP_LAYER_PREFILL = 7
 MAX_RANK = 16
 MAX_BATCH = 16
 MAX_LAYERS = 64
@@ -73,6 +74,7 @@ SIGNATURES = {
     "dfssm_ssm_step": (_I, [_P] * 9 + [_I] * 5 + [_P]),
     "dfssm_layer_decode": (_I, [_P, _I, _P, _P, _P, _P, _I, _P, _Z, _P]),
     "dfssm_lm_head": (_I, [_P, _P, _I, _I, _P, _P, _P, _P, _Z, _P]),
+    "dfssm_layer_prefill": (_I, [_P, _I, _P, _P, _P, _P, _I, _P, _Z, _P]),
     "dfssm_embed": (_I, [_P, _P, _I, _I, _P, _P, _P]),
     "dfssm_head_greedy": (_I, [_P, _P, _I, _I, _P, _P, _P, _P, _P, _P, _Z, _P]),
     "dfssm_generate": (_I, [_P, _I, _P, _P, _P, _I, _P, _P, _I, _P, _P, _P, _P, _P, _Z, _P]),
@@ -283,6 +285,18 @@ def layer_decode(stack: LayerStack, hidden: torch.Tensor, ws=None, stream=None) 
                        hidden.device)
     _check("dfssm_layer_decode", lib().dfssm_layer_decode(
         stack._layers, stack.n, C.byref(stack.dims), _ptr(hidden), stack._conv, stack._ssm, B,
+        _ptr(ws), ws.numel(), _stream(stream)))
+    return hidden
+
+
+def layer_prefill(stack: LayerStack, hidden: torch.Tensor, ws=None, stream=None) -> torch.Tensor:
+    """Prefill of an M-token prompt (hidden [M][d_model], batch 1) through every layer of the stack;
+    hidden is updated in place and the stack's states advance by M tokens."""
+    M = hidden.shape[0]
+    if ws is None:
+        ws = workspace(workspace_size(OP_LAYER_PREFILL, M, stack.d_model, stack.d_inner), hidden.device)
+    _check("dfssm_layer_prefill", lib().dfssm_layer_prefill(
+        stack._layers, stack.n, C.byref(stack.dims), _ptr(hidden), stack._conv, stack._ssm, M,
         _ptr(ws), ws.numel(), _stream(stream)))
     return hidden
 

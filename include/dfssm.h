@@ -94,7 +94,8 @@ enum {
   DFSSM_OP_LAYER_DECODE = 3,   /* a = B,  b = d_model, c = d_inner (nheads*headdim)     */
   DFSSM_OP_LM_HEAD = 4,        /* a = 1,  b = d,     c = V                             */
   DFSSM_OP_HEAD_GREEDY = 5,    /* a = 1,  b = d,     c = V                             */
-  DFSSM_OP_GENERATE = 6        /* a = V,  b = d_model, c = d_inner                     */
+  DFSSM_OP_GENERATE = 6,       /* a = V,  b = d_model, c = d_inner                     */
+  DFSSM_OP_LAYER_PREFILL = 7   /* a = M,  b = d_model, c = d_inner                     */
 };
 size_t dfssm_workspace_size(int op, int a, int b, int c);
 
@@ -200,13 +201,34 @@ typedef struct {
  *   ssm_states   HOST array [n_layers] of device f32 [B][nheads][headdim][d_state]
  * Per layer: (q,s) = quant(RMSNorm(h)); zxbcdt = in_proj (LoRA on RMSNorm(h)); x|B|C = SiLU(conv(xBC));
  * y = SSM(x, dt, B, C); g = y*SiLU(z); (q',s') = quant(RMSNorm(g)); h += out_proj.  The RMS factor is
- * folded into the quantizer scale and the LoRA intermediate: s = fl32(s0/rms), tf = fl32(u sB / rms)
- * with v = fl32(h w) quantized and u = W_B v.   1 <= B <= 16, n_layers <= 64.
+ * folded into the quantizer scale: the codes q are those of v = fl32(h w), s = fl32(s0/rms) with s0 the
+ * absmax scale of v, and the LoRA intermediate is tf = fl32(t sB s) with t = W_B q (int32).
+ * 1 <= B <= 16, n_layers <= 64.
  * workspace: dfssm_workspace_size(DFSSM_OP_LAYER_DECODE, B, d_model, d_inner).
  */
 int dfssm_layer_decode(const dfssm_layer_t* layers, int n_layers, const dfssm_dims_t* dims,
                        float* hidden, float* const* conv_states, float* const* ssm_states, int B,
                        void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * Prefill of an M-token prompt (batch 1) through n_layers layers: for each layer, in order,
+ *   (q, s) = quant(RMSNorm(h_t)) and zxbcdt = in_proj for all t  (tcgen05 int8 GEMM, as dfssm_linear_prefill
+ *   with the pre-norm folded into the quantizer);  xBC = conv over the sequence, continuing conv_state;
+ *   y = the SSM recurrence stepped through t = 0 .. M-1, continuing ssm_state;  g = y SiLU(z);
+ *   h_t += out_proj(quant(RMSNorm(g_t)))  (tcgen05 GEMM with the gated norm folded in, residual add in
+ *   its epilogue).
+ * The conv and SSM steps follow, token after token, exactly the decode step's arithmetic (technical
+ * summary §2.C "Stateful Ops"), so afterwards conv_states / ssm_states hold what M calls of
+ * dfssm_layer_decode would leave and decoding continues from them; the linears carry the prefill GEMM's
+ * precision (int32 accumulators exact, LoRA-up and epilogue in fp32).
+ *   hidden device f32 [M][d_model] (16-byte aligned), updated in place: the residual stream after the last
+ *   layer.  Layers, dims and states as for dfssm_layer_decode with B = 1.  Requires d_model and d_inner
+ *   multiples of 128 (<= 8192), headdim a multiple of 16, d_state a multiple of 4 (<= 512).
+ *   workspace: dfssm_workspace_size(DFSSM_OP_LAYER_PREFILL, M, d_model, d_inner).
+ */
+int dfssm_layer_prefill(const dfssm_layer_t* layers, int n_layers, const dfssm_dims_t* dims,
+                        float* hidden, float* const* conv_states, float* const* ssm_states, int M,
+                        void* workspace, size_t ws_bytes, void* stream);
 
 /*
  * Int8 LM head on one token (technical summary §2.B: int8 LM head with per-row scaling).

@@ -301,3 +301,15 @@ def generate(layers, W, s_row, final_norm_w, first_token: int, n_tokens: int, co
         lg.append(logits)
         tokens.append(greedy(logits))
     return tokens, np.stack(hid), np.stack(lg)
+
+
+def layer_prefill(layers, h, conv_states, ssm_states):
+    """Prefill of a prompt h [M][d_model] (batch 1) through the layers, layer after layer: each layer
+    runs its decode step on tokens 0 .. M-1 in order (the definition of the recurrent model on a
+    sequence), h and the per-layer states conv_states[l] [1][C][3], ssm_states[l] [1][H][P][N] are
+    updated in place."""
+    assert h.dtype == np.float32 and h.flags["C_CONTIGUOUS"]
+    for L, cs, ss in zip(layers, conv_states, ssm_states):
+        for t in range(h.shape[0]):
+            layer_decode(L, h[t:t + 1], cs, ss)
+    return h

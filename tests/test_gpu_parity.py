@@ -380,7 +380,8 @@ def test_device_wait_timeout_is_reported(dev):
 
 def _prefill_compare(dev, lin_host, x, rows):
     """Prefill through the C ABI vs the oracle: int8 codes and scales of every token exact; scaffold
-    accumulators and LoRA-down accumulators exact and the outputs within tolerance on the listed rows."""
+    accumulators, LoRA-down accumulators and outputs (the decode definition, fp64 epilogue) exact on the
+    listed rows."""
     from bit_quantized_mamba_b200 import dfssm
     L = dfssm.Linear.from_host(lin_host, dev)
     M = x.shape[0]
@@ -401,6 +402,7 @@ def _prefill_compare(dev, lin_host, x, rows):
         yr, accr = oracle.linear_core(OL, rq[m], rs[m], tf)
         assert np.array_equal(accg[m], accr), f"prefill scaffold accumulators differ at row {m}"
         assert_tol(yg[m], yr, f"prefill y row {m}")
+        assert np.array_equal(yg[m], yr), f"prefill y row {m}: {(yg[m] != yr).sum()} values differ"
 
 
 def test_prefill_ragged_small(dev):

@@ -465,6 +465,23 @@ def test_lm_head_brute_force():
     assert np.array_equal(a2, acc[rows]) and np.array_equal(l2, logits[rows])
 
 
+def test_prefill_layer_major_equals_token_major():
+    """A prompt through the stack layer after layer (each layer over the whole prompt) equals feeding the
+    tokens one at a time through every layer: the same recurrence, states carried per layer."""
+    m = inputs.decode_model(seed=42, n_layers=3, n_tokens=5, **SMALL)
+    layers = [_oracle_layer(ld) for ld in m["layers"]]
+    conv_a, ssm_a = inputs.zero_states(1, 3, 4, 16, 16, 1)
+    conv_b, ssm_b = conv_a.copy(), ssm_a.copy()
+    prompt = np.ascontiguousarray(m["emb"][:, 0, :])
+    h_a = oracle.layer_prefill(layers, prompt.copy(), conv_a, ssm_a)
+    for t in range(5):
+        h_t = np.ascontiguousarray(m["emb"][t])
+        for l in range(3):
+            oracle.layer_decode(layers[l], h_t, conv_b[l], ssm_b[l])
+        assert np.array_equal(h_a[t], h_t[0])
+    assert np.array_equal(ssm_a, ssm_b) and np.array_equal(conv_a, conv_b)
+
+
 # --------------------------------------------------------------------- embedding, final head, greedy
 
 def test_embed_power_of_two_scales_are_exact():
