@@ -89,10 +89,11 @@ GenerateWs generate_ws(int V, int d_model, int d_inner) {
   return g;
 }
 
-// Layer-prefill workspace: [zxbcdt f32 M x d_ip][xc f32 M x C][g f32 M x E][linear-prefill region], with
-// C and d_ip at their largest supported values (2 ngroups d_state <= 2048, nheads <= 1024).
+// Layer-prefill workspace: [zxbcdt f32 M x d_ip][xc f32 M x C][g f32 M x E][SiLU(z) f32 M x E]
+// [dt, dA f32 M x nheads x 2][linear-prefill region], with C, d_ip and nheads at their largest supported
+// values (2 ngroups d_state <= 2048, nheads <= 1024).
 struct PrefillLayerWs {
-  size_t zx, xc, g, lin, total;
+  size_t zx, xc, g, sz, dtdA, lin, total;
 };
 PrefillLayerWs prefill_layer_ws(int M, int d_model, int E) {
   PrefillLayerWs w;
@@ -100,7 +101,9 @@ PrefillLayerWs prefill_layer_ws(int M, int d_model, int E) {
   w.zx = 0;
   w.xc = w.zx + align256(sizeof(float) * (size_t)M * d_ip);
   w.g = w.xc + align256(sizeof(float) * (size_t)M * C);
-  w.lin = w.g + align256(sizeof(float) * (size_t)M * E);
+  w.sz = w.g + align256(sizeof(float) * (size_t)M * E);
+  w.dtdA = w.sz + align256(sizeof(float) * (size_t)M * E);
+  w.lin = w.dtdA + align256(sizeof(float) * (size_t)M * 1024 * 2);
   const size_t a = dfssm::prefill_workspace_bytes(M, d_model, (int)d_ip);
   const size_t b = dfssm::prefill_workspace_bytes(M, E, d_model);
   w.total = w.lin + align256(a > b ? a : b);
@@ -628,6 +631,8 @@ int dfssm_layer_prefill(const dfssm_layer_t* layers, int n_layers, const dfssm_d
     sa.D = Ly.D;
     sa.state = ssm_states[l];
     sa.g = g;
+    sa.sz = reinterpret_cast<float*>(base + w.sz);
+    sa.dtdA = reinterpret_cast<float*>(base + w.dtdA);
     sa.M = M;
     sa.H = H;
     sa.P = P;

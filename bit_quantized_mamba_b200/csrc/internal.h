@@ -108,6 +108,8 @@ struct ScanArgs {
   const float* D;
   float* state;
   float* g;        // [M][H*P]
+  float* sz;       // scratch [M][H*P]: fl32(SiLU(z)), written by the scan's first kernel
+  float* dtdA;     // scratch [M][H][2]: dt and dA
   int M, H, P, N, G;
 };
 cudaError_t launch_ssm_scan(const ScanArgs& a, cudaStream_t st);

@@ -292,7 +292,7 @@ constexpr int PTMEM_COLS = 2 * BN;         // two int32 accumulators of BN colum
 constexpr int STG_LD = 17;                 // staging row stride (floats): conflict-free both ways
 constexpr size_t OFF_BARS = (size_t)STAGES * STAGE_BYTES;
 constexpr size_t OFF_COLS = OFF_BARS + 512;
-constexpr size_t OFF_WA = OFF_COLS + 2 * BN * 8;   // [2][BN] W_A rows (16 bytes each)
+constexpr size_t OFF_WA = OFF_COLS + 2 * BN * 16;  // [2][BN] W_A rows (16 bytes each)
 constexpr size_t OFF_STG = OFF_WA + 2 * BN * 16;
 constexpr size_t PSMEM_BYTES = 1024 + OFF_STG + EPI_WARPS * 32 * STG_LD * 4;
 
@@ -315,9 +315,9 @@ __global__ void __launch_bounds__(PNT, 1)
   uint64_t* acc_empty = acc_full + 2;      // [2] epilogue -> MMA
   uint64_t* mma_done = acc_empty + 2;      // every MMA of this CTA complete
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(mma_done + 1);
-  // per-accumulator column parameters of the tile being drained: sW, sA, W_A row
-  float* col_sw = reinterpret_cast<float*>(smem + OFF_COLS);  // [2][BN]
-  float* col_sa = col_sw + 2 * BN;                            // [2][BN]
+  // per-accumulator column parameters of the tile being drained: sW, sA (fp64 images), W_A row
+  double* col_sw = reinterpret_cast<double*>(smem + OFF_COLS);  // [2][BN]
+  double* col_sa = col_sw + 2 * BN;                             // [2][BN]
   uint4* col_wa = reinterpret_cast<uint4*>(smem + OFF_WA);    // [2][BN]
   float* stg_all = reinterpret_cast<float*>(smem + OFF_STG);  // [EPI_WARPS][32][STG_LD]
   __shared__ int abort_flag;
@@ -425,8 +425,8 @@ __global__ void __launch_bounds__(PNT, 1)
       // rank)
       if (etid < BN) {
         const int n = n0 + etid;
-        col_sw[buf * BN + etid] = n < ep.N ? __ldg(ep.w_scale + n) : 0.0f;
-        col_sa[buf * BN + etid] = (n < ep.N && ep.rank > 0) ? __ldg(ep.la_scale + n) : 0.0f;
+        col_sw[buf * BN + etid] = n < ep.N ? (double)__ldg(ep.w_scale + n) : 0.0;
+        col_sa[buf * BN + etid] = (n < ep.N && ep.rank > 0) ? (double)__ldg(ep.la_scale + n) : 0.0;
         uint4 wa = make_uint4(0u, 0u, 0u, 0u);
         if (n < ep.N && ep.rank == DFSSM_MAX_RANK) {
           wa = __ldg(reinterpret_cast<const uint4*>(ep.lora_a) + n);  // 16-byte rows at rank 16
@@ -472,8 +472,8 @@ __global__ void __launch_bounds__(PNT, 1)
             const int cidx = buf * BN + c0 + j0 + j;
             a4[j] = (int)v[j0 + j];
             s4[j] = sm;
-            w4[j] = (double)col_sw[cidx];
-            sa4[j] = (double)col_sa[cidx];
+            w4[j] = col_sw[cidx];
+            sa4[j] = col_sa[cidx];
             wa4[j] = col_wa[cidx];
           }
           float o4[4];

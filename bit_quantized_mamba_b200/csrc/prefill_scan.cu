@@ -10,8 +10,8 @@
 // The scan is the stepped recurrence, not the chunked (SSD dual) reordering of it: every state element
 // follows the same rounding sequence as in decode.  Parallelism comes from the 262,144 independent
 // (h, p, n) recurrences of the 1.3B shape: one warp per (h, p) row (four state elements per lane), sixteen
-// rows of one head per CTA, the tokens' B, C, dt, x and z staged through shared memory sixteen tokens at
-// a time, the next chunk's loads in flight while the current one is stepped.
+// rows of one head per CTA, the tokens' B, C, dt, x and z staged through shared memory eight tokens at a
+// time, the next chunk's loads in flight while the current one is stepped.
 
 #include "common.cuh"
 #include "internal.h"
@@ -20,7 +20,8 @@ namespace dfssm {
 namespace scan {
 
 constexpr int SW = 16;  // rows (warps) per CTA
-constexpr int ST = 16;  // tokens per staged chunk
+constexpr int ST = 8;   // tokens per staged chunk
+static_assert(ST == 8, "the scan's token butterfly maps 8 tokens onto lane bits 4..2");
 
 // ------------------------------------------------------------------------------ causal conv
 __global__ void __launch_bounds__(256) conv_seq_kernel(ConvSeqArgs a) {
@@ -52,14 +53,59 @@ __global__ void __launch_bounds__(256) conv_state_kernel(ConvSeqArgs a) {
 }
 
 // ------------------------------------------------------------------------------ SSM scan
+// Per-token scalars of the scan, all tokens in parallel ahead of the sequential kernel: the gate
+// fl32(SiLU(z)) of every (t, h, p) and dt, dA of every (t, h) (fp64 transcendental functions, rounded as
+// in decode).  Thread j < E of token t takes z[t][j]; thread E + h takes head h's dt.
+__global__ void __launch_bounds__(256) scan_prep_kernel(ScanArgs a) {
+  const int E = a.H * a.P;
+  const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= (long long)a.M * (E + a.H)) return;
+  const int t = (int)(idx / (E + a.H)), j = (int)(idx - (long long)t * (E + a.H));
+  if (j < E) {
+    a.sz[(size_t)t * E + j] = silu_f64(__ldg(a.zx + (size_t)t * a.ld_zx + j));
+  } else {
+    const int h = j - E;
+    const float dt = ssm_dt(__ldg(a.zx + (size_t)t * a.ld_zx + a.dt_off + h), __ldg(a.dt_bias + h));
+    reinterpret_cast<float2*>(a.dtdA)[(size_t)t * a.H + h] = make_float2(dt, ssm_dA(dt, __ldg(a.A_log + h)));
+  }
+}
+
 // NJ float4 chunks of the state row per lane (N <= 128 NJ).  Shared memory per buffer: B and C of ST
-// tokens (2 ST N floats), x and z of the CTA's rows (2 ST SW), dt and dA (2 ST); plus two ST x SW
+// tokens (2 ST N), x and fl32(SiLU(z)) of the CTA's rows (2 ST SW), dt and dA (2 ST); plus two ST x SW
 // buffers of gated outputs.
-template <int NJ>
+//
+// Per token a lane advances its state elements (the fp32 recurrence) and adds their readout products to
+// its partial sum.  Each product S C of two fp32 values is split exactly into fl32(S C) + error (one fma)
+// and accumulated as an unevaluated pair of fp32 values (hi + lo, with the exact two-sum error of every
+// addition folded into lo): about 48 significant bits, like an fp64 accumulation far below the fp32
+// rounding of the result, but on the fp32 pipes (converting every state element to fp64 each step would
+// saturate the conversion unit).  The ST partial pairs of a chunk are reduced across the warp together by
+// a transposed butterfly (ST/2 + ST/4 + ... exchanges instead of five per token), converted to fp64 once
+// per token, and the token outputs are finished by ST lane groups in parallel.
+__host__ __device__ constexpr int SCAN_BUF_FLOATS(int N) { return 2 * ST * N + 2 * ST * SW + 2 * ST; }
+
+// (hi, lo) += a: the two-sum of hi and a (exact: hi + a = t + e) with e folded into lo.
+__device__ __forceinline__ void df_add(float& hi, float& lo, float a) {
+  const float t = __fadd_rn(hi, a);
+  const float bp = __fsub_rn(t, hi);
+  const float e = __fadd_rn(__fsub_rn(hi, __fsub_rn(t, bp)), __fsub_rn(a, bp));
+  hi = t;
+  lo = __fadd_rn(lo, e);
+}
+// (hi, lo) += s c with the product split exactly: s c = p + fma(s, c, -p).
+__device__ __forceinline__ void df_add_prod(float& hi, float& lo, float s, float c) {
+  const float p = __fmul_rn(s, c);
+  lo = __fadd_rn(lo, __fmaf_rn(s, c, -p));
+  df_add(hi, lo, p);
+}
+
+// NFIX > 0 fixes d_state at compile time (then NJ = NFIX / 128 and every index is a constant shift);
+// NFIX = 0 reads it from the arguments.
+template <int NJ, int NFIX>
 __global__ void __launch_bounds__(SW * 32, NJ == 1 ? 2 : 1) ssm_scan_kernel(ScanArgs a) {
   extern __shared__ __align__(16) float smf[];
-  const int N = a.N, n4 = N / 4;
-  const int buf_floats = 2 * ST * N + 2 * ST * SW + 2 * ST;
+  const int N = NFIX > 0 ? NFIX : a.N, n4 = N / 4;
+  const int buf_floats = SCAN_BUF_FLOATS(N);
   float* gs = smf + 2 * buf_floats;  // [2][ST][SW]
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int row0 = blockIdx.x * SW;  // SW consecutive (h, p) rows of one head (P % SW == 0)
@@ -67,7 +113,7 @@ __global__ void __launch_bounds__(SW * 32, NJ == 1 ? 2 : 1) ssm_scan_kernel(Scan
   const int grp = h / (a.H / a.G);
   const int E = a.H * a.P;
   const int row = row0 + warp;
-  const float Dh = __ldg(a.D + h), dtb = __ldg(a.dt_bias + h), Al = __ldg(a.A_log + h);
+  const float Dh = __ldg(a.D + h);
   const float* Bsrc = a.xc + a.b_off + (size_t)grp * N;
   const float* Csrc = a.xc + a.c_off + (size_t)grp * N;
 
@@ -81,7 +127,8 @@ __global__ void __launch_bounds__(SW * 32, NJ == 1 ? 2 : 1) ssm_scan_kernel(Scan
   // staging of chunk k into registers, then into buffer k & 1
   constexpr int PF = (2 * ST * 32 * NJ + SW * 32 - 1) / (SW * 32);  // B/C float4 per thread (max)
   float4 pbc[PF];
-  float px = 0.f, pz = 0.f, pdt = 0.f;
+  float px = 0.f, pz = 0.f;
+  float2 pdt = make_float2(0.f, 0.f);
   const auto load_chunk = [&](int t0) {
     const int nT = min(ST, a.M - t0);
 #pragma unroll
@@ -99,20 +146,20 @@ __global__ void __launch_bounds__(SW * 32, NJ == 1 ? 2 : 1) ssm_scan_kernel(Scan
       const int tt = tid / SW, w = tid - tt * SW;
       if (tt < nT) {
         px = __ldg(a.xc + (size_t)(t0 + tt) * a.ld_xc + row0 + w);
-        pz = __ldg(a.zx + (size_t)(t0 + tt) * a.ld_zx + row0 + w);
+        pz = __ldg(a.sz + (size_t)(t0 + tt) * E + row0 + w);
       }
     }
-    if (tid < nT) pdt = __ldg(a.zx + (size_t)(t0 + tid) * a.ld_zx + a.dt_off + h);
+    if (tid < nT) pdt = __ldg(reinterpret_cast<const float2*>(a.dtdA) + (size_t)(t0 + tid) * a.H + h);
   };
   const auto store_chunk = [&](int t0, int b) {
     const int nT = min(ST, a.M - t0);
     float* base = smf + b * buf_floats;
-    float* Bs = base;               // [ST][N]
-    float* Cs = base + ST * N;      // [ST][N]
-    float* xs = base + 2 * ST * N;  // [ST][SW]
-    float* zs = xs + ST * SW;       // [ST][SW]
-    float* dts = zs + ST * SW;      // [ST]
-    float* dAs = dts + ST;          // [ST]
+    float* Bs = base;                                     // [ST][N]
+    float* Cs = base + ST * N;                            // [ST][N]
+    float* xs = base + 2 * ST * N;                        // [ST][SW]
+    float* szs = xs + ST * SW;                            // [ST][SW] fl32(SiLU(z))
+    float* dts = szs + ST * SW;                           // [ST]
+    float* dAs = dts + ST;                                // [ST]
 #pragma unroll
     for (int k = 0; k < PF; ++k) {
       const int i = tid + k * SW * 32;
@@ -124,12 +171,11 @@ __global__ void __launch_bounds__(SW * 32, NJ == 1 ? 2 : 1) ssm_scan_kernel(Scan
     }
     if (tid < ST * SW) {
       xs[tid] = px;
-      zs[tid] = pz;
+      szs[tid] = pz;
     }
     if (tid < nT) {
-      const float dt = ssm_dt(pdt, dtb);
-      dts[tid] = dt;
-      dAs[tid] = ssm_dA(dt, Al);
+      dts[tid] = pdt.x;
+      dAs[tid] = pdt.y;
     }
   };
 
@@ -149,34 +195,67 @@ __global__ void __launch_bounds__(SW * 32, NJ == 1 ? 2 : 1) ssm_scan_kernel(Scan
     const float* Bs = base;
     const float* Cs = base + ST * N;
     const float* xs = base + 2 * ST * N;
-    const float* zs = xs + ST * SW;
-    const float* dts = zs + ST * SW;
+    const float* szs = xs + ST * SW;
+    const float* dts = szs + ST * SW;
     const float* dAs = dts + ST;
-    float* gout = gs + (k & 1) * ST * SW;
-    for (int tt = 0; tt < nT; ++tt) {
-      const float dt = dts[tt], dA = dAs[tt], xv = xs[tt * SW + warp];
-      const float dtx = fmul(dt, xv);
-      double acc = 0.0;
+    // 1. the recurrence through the chunk; (ph[tt], pl[tt]) = this lane's share of token tt's readout
+    float ph[ST], pl[ST];
 #pragma unroll
-      for (int j = 0; j < NJ; ++j) {
-        const int c = lane + 32 * j;
-        if (c < n4) {
-          const float4 b4 = reinterpret_cast<const float4*>(Bs + (size_t)tt * N)[c];
-          const float4 c4 = reinterpret_cast<const float4*>(Cs + (size_t)tt * N)[c];
-          S[j].x = ssm_state(dA, S[j].x, dtx, b4.x);
-          S[j].y = ssm_state(dA, S[j].y, dtx, b4.y);
-          S[j].z = ssm_state(dA, S[j].z, dtx, b4.z);
-          S[j].w = ssm_state(dA, S[j].w, dtx, b4.w);
-          acc = fma((double)S[j].x, (double)c4.x, acc);  // products of two fp32 are exact in fp64
-          acc = fma((double)S[j].y, (double)c4.y, acc);
-          acc = fma((double)S[j].z, (double)c4.z, acc);
-          acc = fma((double)S[j].w, (double)c4.w, acc);
+    for (int tt = 0; tt < ST; ++tt) {
+      ph[tt] = 0.0f;
+      pl[tt] = 0.0f;
+      if (tt < nT) {
+        const float dA = dAs[tt];
+        const float dtx = fmul(dts[tt], xs[tt * SW + warp]);
+#pragma unroll
+        for (int j = 0; j < NJ; ++j) {
+          const int c = lane + 32 * j;
+          if (c < n4) {
+            const float4 b4 = reinterpret_cast<const float4*>(Bs + (size_t)tt * N)[c];
+            const float4 c4 = reinterpret_cast<const float4*>(Cs + (size_t)tt * N)[c];
+            S[j].x = ssm_state(dA, S[j].x, dtx, b4.x);
+            S[j].y = ssm_state(dA, S[j].y, dtx, b4.y);
+            S[j].z = ssm_state(dA, S[j].z, dtx, b4.z);
+            S[j].w = ssm_state(dA, S[j].w, dtx, b4.w);
+            df_add_prod(ph[tt], pl[tt], S[j].x, c4.x);
+            df_add_prod(ph[tt], pl[tt], S[j].y, c4.y);
+            df_add_prod(ph[tt], pl[tt], S[j].z, c4.z);
+            df_add_prod(ph[tt], pl[tt], S[j].w, c4.w);
+          }
         }
       }
-      acc = warp_sum(acc);
-      if (lane == 0) {
-        const float y = __double2float_rn(dadd(acc, dmul((double)Dh, (double)xv)));
-        gout[tt * SW + warp] = fmul(y, silu_f64(zs[tt * SW + warp]));
+    }
+    // 2. transposed butterfly: after the exchanges over lane bits 4, 3, 2 each lane holds one token's
+    //    partial pair (token = lane bits 4..2), summed over lane bits 1, 0 at the end
+#pragma unroll
+    for (int half = ST / 2, off = 16; half >= 1; half >>= 1, off >>= 1) {
+      const bool upper = (lane & off) != 0;
+#pragma unroll
+      for (int i = 0; i < half; ++i) {
+        const float send_h = upper ? ph[i] : ph[i + half], send_l = upper ? pl[i] : pl[i + half];
+        const float keep_h = upper ? ph[i + half] : ph[i], keep_l = upper ? pl[i + half] : pl[i];
+        const float oh = __shfl_xor_sync(0xffffffffu, send_h, off);
+        const float ol = __shfl_xor_sync(0xffffffffu, send_l, off);
+        ph[i] = keep_h;
+        pl[i] = __fadd_rn(keep_l, ol);
+        df_add(ph[i], pl[i], oh);
+      }
+    }
+#pragma unroll
+    for (int off = 2; off >= 1; off >>= 1) {
+      const float oh = __shfl_xor_sync(0xffffffffu, ph[0], off);
+      const float ol = __shfl_xor_sync(0xffffffffu, pl[0], off);
+      pl[0] = __fadd_rn(pl[0], ol);
+      df_add(ph[0], pl[0], oh);
+    }
+    const double tot = dadd((double)ph[0], (double)pl[0]);
+    // 3. token outputs: lane group g = lane / 4 finishes token g
+    {
+      const int tt = ((lane >> 4) & 1) * 4 + ((lane >> 3) & 1) * 2 + ((lane >> 2) & 1);
+      if ((lane & 3) == 0 && tt < nT) {
+        const float xv = xs[tt * SW + warp];
+        const float y = __double2float_rn(dadd(tot, dmul((double)Dh, (double)xv)));
+        gs[(k & 1) * ST * SW + tt * SW + warp] = fmul(y, szs[tt * SW + warp]);
       }
     }
     if (k + 1 < n_chunks) store_chunk(t0 + ST, (k + 1) & 1);  // buffer (k+1)&1 was last read in chunk k-1
@@ -197,18 +276,21 @@ __global__ void __launch_bounds__(SW * 32, NJ == 1 ? 2 : 1) ssm_scan_kernel(Scan
   }
 }
 
-template <int NJ>
+template <int NJ, int NFIX>
 cudaError_t launch_scan_nj(const ScanArgs& a, cudaStream_t st) {
-  const size_t smem = sizeof(float) * (2 * (2 * ST * a.N + 2 * ST * SW + 2 * ST) + 2 * ST * SW);
+  const size_t smem = sizeof(float) * (2 * SCAN_BUF_FLOATS(a.N) + 2 * ST * SW);
   static bool attr = false;
   if (!attr) {
-    const cudaError_t e = cudaFuncSetAttribute(ssm_scan_kernel<NJ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                               (int)(sizeof(float) * (2 * (2 * ST * 512 + 2 * ST * SW + 2 * ST) +
-                                                                      2 * ST * SW)));
+    const cudaError_t e = cudaFuncSetAttribute(ssm_scan_kernel<NJ, NFIX>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               (int)(sizeof(float) * (2 * SCAN_BUF_FLOATS(512) + 2 * ST * SW)));
     if (e != cudaSuccess) return e;
     attr = true;
   }
-  ssm_scan_kernel<NJ><<<(a.H * a.P) / SW, SW * 32, smem, st>>>(a);
+  const long long n_prep = (long long)a.M * (a.H * a.P + a.H);
+  scan_prep_kernel<<<(unsigned)((n_prep + 255) / 256), 256, 0, st>>>(a);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  ssm_scan_kernel<NJ, NFIX><<<(a.H * a.P) / SW, SW * 32, smem, st>>>(a);
   return cudaGetLastError();
 }
 
@@ -224,9 +306,10 @@ cudaError_t launch_conv_seq(const ConvSeqArgs& a, cudaStream_t st) {
 }
 
 cudaError_t launch_ssm_scan(const ScanArgs& a, cudaStream_t st) {
-  if (a.N <= 128) return scan::launch_scan_nj<1>(a, st);
-  if (a.N <= 256) return scan::launch_scan_nj<2>(a, st);
-  return scan::launch_scan_nj<4>(a, st);
+  if (a.N == 128) return scan::launch_scan_nj<1, 128>(a, st);
+  if (a.N <= 128) return scan::launch_scan_nj<1, 0>(a, st);
+  if (a.N <= 256) return scan::launch_scan_nj<2, 0>(a, st);
+  return scan::launch_scan_nj<4, 0>(a, st);
 }
 
 bool scan_supported(int H, int P, int N, int G) {
