@@ -292,8 +292,8 @@ constexpr int PTMEM_COLS = 2 * BN;         // two int32 accumulators of BN colum
 constexpr int STG_LD = 17;                 // staging row stride (floats): conflict-free both ways
 constexpr size_t OFF_BARS = (size_t)STAGES * STAGE_BYTES;
 constexpr size_t OFF_COLS = OFF_BARS + 512;
-constexpr size_t OFF_WA = OFF_COLS + 2 * BN * 16;  // [2][BN] W_A rows (16 bytes each)
-constexpr size_t OFF_STG = OFF_WA + 2 * BN * 16;
+constexpr size_t OFF_WA = OFF_COLS + 2 * BN * 16;  // [2][BN][16] W_A rows as fp64 (zero beyond the rank)
+constexpr size_t OFF_STG = OFF_WA + 2 * BN * DFSSM_MAX_RANK * 8;
 constexpr size_t PSMEM_BYTES = 1024 + OFF_STG + EPI_WARPS * 32 * STG_LD * 4;
 
 // Bounded wait that ignores the abort flag (used to drain work already issued).
@@ -318,7 +318,7 @@ __global__ void __launch_bounds__(PNT, 1)
   // per-accumulator column parameters of the tile being drained: sW, sA (fp64 images), W_A row
   double* col_sw = reinterpret_cast<double*>(smem + OFF_COLS);  // [2][BN]
   double* col_sa = col_sw + 2 * BN;                             // [2][BN]
-  uint4* col_wa = reinterpret_cast<uint4*>(smem + OFF_WA);    // [2][BN]
+  double* col_wa = reinterpret_cast<double*>(smem + OFF_WA);  // [2][BN][16]
   float* stg_all = reinterpret_cast<float*>(smem + OFF_STG);  // [EPI_WARPS][32][STG_LD]
   __shared__ int abort_flag;
 
@@ -427,16 +427,10 @@ __global__ void __launch_bounds__(PNT, 1)
         const int n = n0 + etid;
         col_sw[buf * BN + etid] = n < ep.N ? (double)__ldg(ep.w_scale + n) : 0.0;
         col_sa[buf * BN + etid] = (n < ep.N && ep.rank > 0) ? (double)__ldg(ep.la_scale + n) : 0.0;
-        uint4 wa = make_uint4(0u, 0u, 0u, 0u);
-        if (n < ep.N && ep.rank == DFSSM_MAX_RANK) {
-          wa = __ldg(reinterpret_cast<const uint4*>(ep.lora_a) + n);  // 16-byte rows at rank 16
-        } else if (n < ep.N) {
-          uint32_t w[4] = {0u, 0u, 0u, 0u};
-          for (int r = 0; r < ep.rank; ++r)
-            w[r >> 2] |= ((uint32_t)(uint8_t)ep.lora_a[(size_t)n * ep.rank + r]) << (8 * (r & 3));
-          wa = make_uint4(w[0], w[1], w[2], w[3]);
-        }
-        col_wa[buf * BN + etid] = wa;
+        double* wd = col_wa + (size_t)(buf * BN + etid) * DFSSM_MAX_RANK;
+#pragma unroll
+        for (int r = 0; r < DFSSM_MAX_RANK; ++r)
+          wd[r] = (n < ep.N && r < ep.rank) ? (double)ep.lora_a[(size_t)n * ep.rank + r] : 0.0;
       }
       asm volatile("bar.sync 1, %0;" ::"n"(EPI_WARPS * 32) : "memory");
       const int row = q * 32 + lane;
@@ -460,26 +454,24 @@ __global__ void __launch_bounds__(PNT, 1)
         uint32_t v[16];
         tmem_ld16(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * BN + c0), v);
         float out[16];
-        // y = fl32(acc s sW + sA sum_r W_A tf): the decode path's definition, four outputs interleaved
+        // y = fl32(acc s sW + sA sum_r W_A tf), fp64, the decode path's rounding sequence (linear_out_n):
+        // the LoRA sum runs over r = 0..15 in order; fma(w, tf, lora) equals lora + w tf rounded once
+        // because the product of an int8 and an fp32 value is exact in fp64, and the zero weights beyond
+        // the rank leave the sum unchanged (it is never -0).
 #pragma unroll
-        for (int j0 = 0; j0 < 16; j0 += 4) {
-          int a4[4];
-          double s4[4], w4[4], sa4[4];
-          uint4 wa4[4];
-          const double* tf4[4] = {tfd, tfd, tfd, tfd};
+        for (int j = 0; j < 16; ++j) {
+          const int cidx = buf * BN + c0 + j;
+          const double2* w2 = reinterpret_cast<const double2*>(col_wa + (size_t)cidx * DFSSM_MAX_RANK);
+          double lora = 0.0;
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const int cidx = buf * BN + c0 + j0 + j;
-            a4[j] = (int)v[j0 + j];
-            s4[j] = sm;
-            w4[j] = col_sw[cidx];
-            sa4[j] = col_sa[cidx];
-            wa4[j] = col_wa[cidx];
+          for (int r2 = 0; r2 < DFSSM_MAX_RANK / 2; ++r2) {
+            const double2 w = w2[r2];
+            lora = fma(w.x, tfd[2 * r2], lora);
+            lora = fma(w.y, tfd[2 * r2 + 1], lora);
           }
-          float o4[4];
-          linear_out_n<4, -1>(a4, s4, w4, sa4, wa4, tf4, ep.rank, o4);
-#pragma unroll
-          for (int j = 0; j < 4; ++j) out[j0 + j] = o4[j];
+          const double scaffold = dmul(dmul(int_to_f64((int)v[j]), sm), col_sw[cidx]);
+          const double corr = ep.rank > 0 ? dmul(col_sa[cidx], lora) : 0.0;
+          out[j] = __double2float_rn(dadd(scaffold, corr));
         }
         if (ep.acc && m < ep.M) {
 #pragma unroll
