@@ -410,6 +410,33 @@ def run_ours(args, rank, world, local_rank):
         prefill["int8_peak_TOPS"] = round(int8_peak, 1)
         prefill["int8_peak_kind"] = "measured bf16 burst x 2 (nominal int8/bf16 ratio)"
         del W
+    # ---- layer prefill: a 2048-token prompt through the 48 layers (in_proj GEMM, conv and SSM over the
+    # prompt, out_proj GEMM), states continuing from the bench's decode
+    prefill_layers = {}
+    if not args.no_extras:
+        Mp = 2048
+        hp0 = torch.from_numpy(inputs.normal(np.random.default_rng(11), (Mp, 2048))).to(dev)
+        hp = hp0.clone()
+        pws_l = dfssm.workspace(dfssm.workspace_size(dfssm.OP_LAYER_PREFILL, Mp, 2048, 4096), dev)
+        with torch.cuda.stream(stream):
+            dfssm.layer_prefill(stack, hp, pws_l, stream=torch.cuda.current_stream())
+            torch.cuda.synchronize()
+            tot = 0.0
+            reps = 2
+            for r in range(reps):
+                hp.copy_(hp0)
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record()
+                dfssm.layer_prefill(stack, hp, pws_l, stream=torch.cuda.current_stream())
+                b.record()
+                b.synchronize()
+                tot += a.elapsed_time(b)
+        pms = tot / reps
+        prefill_layers = {"prompt_tokens": Mp, "layers": 48, "ms_per_prompt": round(pms, 3),
+                          "tokens_per_s": round(Mp / (pms * 1e-3), 1),
+                          "kernels_per_layer": 10}
+        del pws_l, hp, hp0
+
     # ---- greedy generation: embedding + the 48 layers + final RMSNorm / int8 LM head / argmax per token,
     # 64 tokens captured in one CUDA graph (the bench's stack, the tied 50288 x 2048 matrix of seed 5)
     generate = {}
@@ -493,6 +520,7 @@ def run_ours(args, rank, world, local_rank):
         "roofline": roofline,
         "scaffold_gemv": gemv,
         "prefill": prefill,
+        "prefill_layers": prefill_layers,
         "generate": generate,
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": N_TOKENS * 2048 * 4,
                 "d2h_bytes_per_step": 2048 * 4},
