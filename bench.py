@@ -570,6 +570,44 @@ def run_gemv_profile(args):
     torch.cuda.synchronize()
 
 
+def run_layer_prefill_profile(args):
+    """Eager 2048-token prompts through one layer of the 1.3B shape (dfssm_layer_prefill), for ncu."""
+    import numpy as np
+    import torch
+    from bit_quantized_mamba_b200 import build, dfssm, inputs
+    build.build()
+    dev = torch.device("cuda", 0)
+    m = inputs.decode_model(seed=3, n_layers=1, n_tokens=1)
+    dims = dict(d_model=2048, nheads=64, headdim=64, d_state=128, ngroups=1)
+    conv, ssm = inputs.zero_states(1, 1)
+    stack = dfssm.LayerStack([dfssm.Layer.from_host(m["layers"][0], dev)], dims,
+                             [torch.from_numpy(conv[0]).to(dev)], [torch.from_numpy(ssm[0]).to(dev)])
+    h0 = torch.from_numpy(inputs.normal(np.random.default_rng(11), (2048, 2048))).to(dev)
+    ws = dfssm.workspace(dfssm.workspace_size(dfssm.OP_LAYER_PREFILL, 2048, 2048, 4096), dev)
+    for _ in range(args.warmup + 1):
+        h = h0.clone()
+        dfssm.layer_prefill(stack, h, ws)
+    torch.cuda.synchronize()
+
+
+def run_head_profile(args):
+    """Eager final-norm + LM-head + greedy calls over the 50288 x 2048 tied matrix, for ncu."""
+    import numpy as np
+    import torch
+    from bit_quantized_mamba_b200 import build, dfssm, inputs
+    build.build()
+    dev = torch.device("cuda", 0)
+    gm = inputs.generation_model(seed=5, n_layers=0)
+    W = torch.from_numpy(gm["emb_w"]).to(dev)
+    s_row = torch.from_numpy(gm["emb_s"]).to(dev)
+    nw = torch.from_numpy(gm["final_norm_w"]).to(dev)
+    h = torch.from_numpy(inputs.normal(np.random.default_rng(9), (2048,))).to(dev)
+    ws = dfssm.workspace(dfssm.workspace_size(dfssm.OP_HEAD_GREEDY, 1, 2048, W.shape[0]), dev)
+    for _ in range(args.warmup + 1):
+        dfssm.head_greedy(W, s_row, h, nw, ws=ws)
+    torch.cuda.synchronize()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -584,10 +622,15 @@ def main():
                     help="profiling mode: run the 2048-token in_proj prefill --warmup + 1 times and exit")
     ap.add_argument("--ncu-gemv", action="store_true",
                     help="profiling mode: the 48-copy in_proj multi-linear decode --warmup + 1 times and exit")
+    ap.add_argument("--ncu-layer-prefill", action="store_true",
+                    help="profiling mode: a 2048-token prompt through one layer --warmup + 1 times and exit")
+    ap.add_argument("--ncu-head", action="store_true",
+                    help="profiling mode: the final norm + LM head + greedy choice --warmup + 1 times and exit")
     ap.add_argument("--ncu", action="store_true",
                     help="profiling mode: decode --warmup tokens then one more token, eagerly, and exit")
     args = ap.parse_args()
-    if args.warmup < 3 and not (args.ncu or args.ncu_gemv or args.ncu_prefill):
+    profiling = args.ncu or args.ncu_gemv or args.ncu_prefill or args.ncu_layer_prefill or args.ncu_head
+    if args.warmup < 3 and not profiling:
         args.warmup = 3
     rank = int(os.environ.get("RANK", 0))
     world = int(os.environ.get("WORLD_SIZE", 1))
@@ -600,6 +643,12 @@ def main():
         return
     if args.ncu_gemv:
         run_gemv_profile(args)
+        return
+    if args.ncu_layer_prefill:
+        run_layer_prefill_profile(args)
+        return
+    if args.ncu_head:
+        run_head_profile(args)
         return
     if world > 1:
         import datetime
