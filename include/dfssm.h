@@ -147,8 +147,8 @@ int dfssm_linear_decode_noalloc(const dfssm_linear_t* lin, const float* x, int B
  * M-token prefill of one linear on int8 tcgen05 tensor cores (technical summary §2.C: the scaffold
  * matmul on INT8 tensor cores).  Same math as dfssm_linear_decode, per row of x.
  *   x device f32 [M][d_in], y device f32 [M][d_out], M >= 1.  d_in % 128 == 0 required.
- *   dbg->acc, dbg->xq and dbg->xscale are exact; tf and y are fp32 to within 1e-6 relative of the fp64
- *   definition (the prefill epilogue uses fp32 fused multiply-add).
+ *   dbg->acc, dbg->xq, dbg->xscale and dbg->lora_t are exact, and y is bit-identical to the decode path
+ *   (the epilogue evaluates the definition in fp64 with the decode rounding sequence).
  */
 int dfssm_linear_prefill(const dfssm_linear_t* lin, const float* x, int M, float* y, void* workspace,
                          size_t ws_bytes, const dfssm_debug_t* dbg, void* stream);
@@ -219,8 +219,9 @@ int dfssm_layer_decode(const dfssm_layer_t* layers, int n_layers, const dfssm_di
  *   its epilogue).
  * The conv and SSM steps follow, token after token, exactly the decode step's arithmetic (technical
  * summary §2.C "Stateful Ops"), so afterwards conv_states / ssm_states hold what M calls of
- * dfssm_layer_decode would leave and decoding continues from them; the linears carry the prefill GEMM's
- * precision (int32 accumulators exact, LoRA-up and epilogue in fp32).
+ * dfssm_layer_decode would leave and decoding continues from them; the linears are exact as in decode.
+ * The SSM readout sum_n S C is accumulated in about 48 bits (a pair of fp32 values) instead of fp64, so
+ * the outputs agree with the decode definition to that precision, not bit for bit.
  *   hidden device f32 [M][d_model] (16-byte aligned), updated in place: the residual stream after the last
  *   layer.  Layers, dims and states as for dfssm_layer_decode with B = 1.  Requires d_model and d_inner
  *   multiples of 128 (<= 8192), headdim a multiple of 16, d_state a multiple of 4 (<= 512).
