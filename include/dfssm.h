@@ -44,7 +44,7 @@ typedef enum {
   DFSSM_OK = 0,
   DFSSM_EINVAL = -1,       /* bad size, NULL pointer or inconsistent arguments                      */
   DFSSM_EALIGN = -2,       /* a pointer is not aligned as documented                                */
-  DFSSM_EUNSUPPORTED = -3, /* valid, but outside what this build implements (e.g. B > 16)           */
+  DFSSM_EUNSUPPORTED = -3, /* valid, but outside what the library implements (e.g. B > 16)         */
   DFSSM_ECUDA = -4,        /* a CUDA runtime call failed; see dfssm_last_cuda_error()                */
   DFSSM_ETIMEOUT = -5,     /* a device-side wait ran out of its iteration budget                    */
   DFSSM_EDEVICE = -6,      /* no usable sm_100 device                                               */
