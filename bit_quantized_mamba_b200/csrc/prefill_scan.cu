@@ -276,6 +276,160 @@ __global__ void __launch_bounds__(SW * 32, NJ == 1 ? 2 : 1) ssm_scan_kernel(Scan
   }
 }
 
+// d_state 128 (the model shape): each lane owns eight state elements (two float4 chunks: c and c + 16),
+// a warp two (h, p) rows (lanes 0-15 and 16-31), a CTA of eight warps the same sixteen rows of one head
+// as above.  Twice the state elements per lane spread the per-token loads, the butterfly and the output
+// step over twice the work; the butterfly runs within each half-warp (token = lane bits 3..1).
+constexpr int W128 = SW / 2;  // warps per CTA
+__global__ void __launch_bounds__(W128 * 32, 2) ssm_scan128_kernel(ScanArgs a) {
+  constexpr int N = 128, n4 = 32;
+  constexpr int NT = W128 * 32;
+  extern __shared__ __align__(16) float smf[];
+  constexpr int buf_floats = SCAN_BUF_FLOATS(N);
+  float* gs = smf + 2 * buf_floats;  // [2][ST][SW]
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int hl = lane & 15;                // lane within the half-warp
+  const int rloc = 2 * warp + (lane >> 4);  // this half-warp's row within the CTA
+  const int row0 = blockIdx.x * SW;
+  const int h = row0 / a.P;
+  const int grp = h / (a.H / a.G);
+  const int E = a.H * a.P;
+  const int row = row0 + rloc;
+  const float Dh = __ldg(a.D + h);
+  const float* Bsrc = a.xc + a.b_off + (size_t)grp * N;
+  const float* Csrc = a.xc + a.c_off + (size_t)grp * N;
+
+  float4 S[2];
+#pragma unroll
+  for (int j = 0; j < 2; ++j) S[j] = reinterpret_cast<const float4*>(a.state + (size_t)row * N)[hl + 16 * j];
+
+  constexpr int PF = 2 * ST * n4 / NT;  // B/C float4 per thread per chunk (2)
+  float4 pbc[PF];
+  float px = 0.f, pz = 0.f;
+  float2 pdt = make_float2(0.f, 0.f);
+  const auto load_chunk = [&](int t0) {
+    const int nT = min(ST, a.M - t0);
+#pragma unroll
+    for (int k = 0; k < PF; ++k) {
+      const int i = tid + k * NT;  // < 2 ST n4
+      const int tt = i >> 6, which = (i >> 5) & 1, c = i & 31;
+      pbc[k] = tt < nT ? __ldg(reinterpret_cast<const float4*>((which ? Csrc : Bsrc) + (size_t)(t0 + tt) * a.ld_xc) + c)
+                       : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    if (tid < ST * SW) {
+      const int tt = tid / SW, w = tid - tt * SW;
+      if (tt < nT) {
+        px = __ldg(a.xc + (size_t)(t0 + tt) * a.ld_xc + row0 + w);
+        pz = __ldg(a.sz + (size_t)(t0 + tt) * E + row0 + w);
+      }
+    }
+    if (tid < nT) pdt = __ldg(reinterpret_cast<const float2*>(a.dtdA) + (size_t)(t0 + tid) * a.H + h);
+  };
+  const auto store_chunk = [&](int t0, int b) {
+    const int nT = min(ST, a.M - t0);
+    float* base = smf + b * buf_floats;
+#pragma unroll
+    for (int k = 0; k < PF; ++k) {
+      const int i = tid + k * NT;
+      const int tt = i >> 6, which = (i >> 5) & 1, c = i & 31;
+      reinterpret_cast<float4*>(base + which * ST * N + tt * N)[c] = pbc[k];
+    }
+    float* xs = base + 2 * ST * N;
+    if (tid < ST * SW) {
+      xs[tid] = px;
+      xs[ST * SW + tid] = pz;
+    }
+    if (tid < nT) {
+      xs[2 * ST * SW + tid] = pdt.x;
+      xs[2 * ST * SW + ST + tid] = pdt.y;
+    }
+  };
+
+  const int n_chunks = (a.M + ST - 1) / ST;
+  load_chunk(0);
+  store_chunk(0, 0);
+  __syncthreads();
+  for (int k = 0; k < n_chunks; ++k) {
+    const int t0 = k * ST, nT = min(ST, a.M - t0);
+    if (k + 1 < n_chunks) load_chunk(t0 + ST);
+    if (k > 0 && tid < ST * SW) {
+      const int tt = tid / SW, w = tid - tt * SW;
+      a.g[(size_t)(t0 - ST + tt) * E + row0 + w] = gs[((k - 1) & 1) * ST * SW + tid];
+    }
+    const float* base = smf + (k & 1) * buf_floats;
+    const float* Bs = base;
+    const float* Cs = base + ST * N;
+    const float* xs = base + 2 * ST * N;
+    const float* szs = xs + ST * SW;
+    const float* dts = szs + ST * SW;
+    const float* dAs = dts + ST;
+    float ph[ST], pl[ST];
+#pragma unroll
+    for (int tt = 0; tt < ST; ++tt) {
+      ph[tt] = 0.0f;
+      pl[tt] = 0.0f;
+      if (tt < nT) {
+        const float dA = dAs[tt];
+        const float dtx = fmul(dts[tt], xs[tt * SW + rloc]);
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          const float4 b4 = reinterpret_cast<const float4*>(Bs + tt * N)[hl + 16 * j];
+          const float4 c4 = reinterpret_cast<const float4*>(Cs + tt * N)[hl + 16 * j];
+          S[j].x = ssm_state(dA, S[j].x, dtx, b4.x);
+          S[j].y = ssm_state(dA, S[j].y, dtx, b4.y);
+          S[j].z = ssm_state(dA, S[j].z, dtx, b4.z);
+          S[j].w = ssm_state(dA, S[j].w, dtx, b4.w);
+          df_add_prod(ph[tt], pl[tt], S[j].x, c4.x);
+          df_add_prod(ph[tt], pl[tt], S[j].y, c4.y);
+          df_add_prod(ph[tt], pl[tt], S[j].z, c4.z);
+          df_add_prod(ph[tt], pl[tt], S[j].w, c4.w);
+        }
+      }
+    }
+    // transposed butterfly within each half-warp over lane bits 3, 2, 1, then the pair over bit 0
+#pragma unroll
+    for (int half = ST / 2, off = 8; half >= 1; half >>= 1, off >>= 1) {
+      const bool upper = (lane & off) != 0;
+#pragma unroll
+      for (int i = 0; i < half; ++i) {
+        const float send_h = upper ? ph[i] : ph[i + half], send_l = upper ? pl[i] : pl[i + half];
+        const float keep_h = upper ? ph[i + half] : ph[i], keep_l = upper ? pl[i + half] : pl[i];
+        const float oh = __shfl_xor_sync(0xffffffffu, send_h, off);
+        const float ol = __shfl_xor_sync(0xffffffffu, send_l, off);
+        ph[i] = keep_h;
+        pl[i] = __fadd_rn(keep_l, ol);
+        df_add(ph[i], pl[i], oh);
+      }
+    }
+    {
+      const float oh = __shfl_xor_sync(0xffffffffu, ph[0], 1);
+      const float ol = __shfl_xor_sync(0xffffffffu, pl[0], 1);
+      pl[0] = __fadd_rn(pl[0], ol);
+      df_add(ph[0], pl[0], oh);
+    }
+    {
+      const int tt = ((lane >> 3) & 1) * 4 + ((lane >> 2) & 1) * 2 + ((lane >> 1) & 1);
+      if ((lane & 1) == 0 && tt < nT) {
+        const double tot = dadd((double)ph[0], (double)pl[0]);
+        const float xv = xs[tt * SW + rloc];
+        const float y = __double2float_rn(dadd(tot, dmul((double)Dh, (double)xv)));
+        gs[(k & 1) * ST * SW + tt * SW + rloc] = fmul(y, szs[tt * SW + rloc]);
+      }
+    }
+    if (k + 1 < n_chunks) store_chunk(t0 + ST, (k + 1) & 1);
+    __syncthreads();
+  }
+  {
+    const int k = n_chunks - 1, t0 = k * ST, nT = min(ST, a.M - t0);
+    if (tid < ST * SW) {
+      const int tt = tid / SW, w = tid - tt * SW;
+      if (tt < nT) a.g[(size_t)(t0 + tt) * E + row0 + w] = gs[(k & 1) * ST * SW + tid];
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < 2; ++j) reinterpret_cast<float4*>(a.state + (size_t)row * N)[hl + 16 * j] = S[j];
+}
+
 template <int NJ, int NFIX>
 cudaError_t launch_scan_nj(const ScanArgs& a, cudaStream_t st) {
   const size_t smem = sizeof(float) * (2 * SCAN_BUF_FLOATS(a.N) + 2 * ST * SW);
@@ -306,7 +460,15 @@ cudaError_t launch_conv_seq(const ConvSeqArgs& a, cudaStream_t st) {
 }
 
 cudaError_t launch_ssm_scan(const ScanArgs& a, cudaStream_t st) {
-  if (a.N == 128) return scan::launch_scan_nj<1, 128>(a, st);
+  if (a.N == 128) {
+    const size_t smem = sizeof(float) * (2 * scan::SCAN_BUF_FLOATS(128) + 2 * scan::ST * scan::SW);
+    const long long n_prep = (long long)a.M * (a.H * a.P + a.H);
+    scan::scan_prep_kernel<<<(unsigned)((n_prep + 255) / 256), 256, 0, st>>>(a);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    scan::ssm_scan128_kernel<<<(a.H * a.P) / scan::SW, scan::W128 * 32, smem, st>>>(a);
+    return cudaGetLastError();
+  }
   if (a.N <= 128) return scan::launch_scan_nj<1, 0>(a, st);
   if (a.N <= 256) return scan::launch_scan_nj<2, 0>(a, st);
   return scan::launch_scan_nj<4, 0>(a, st);
