@@ -3,6 +3,8 @@ oracle's own formulas retyped.  CPU only.
 
 Each test names the plausible mistake it would catch.
 """
+import os
+
 import numpy as np
 import pytest
 from scipy.special import expit
@@ -596,10 +598,23 @@ def test_generate_with_identity_layers_follows_the_head():
 
 # ------------------------------------------------------------------------------------- shape pins
 
+def _golden(name):
+    vals = {}
+    with open(os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden", name)) as f:
+        for line in f:
+            line = line.split("#", 1)[0].strip()
+            if line:
+                k, v = line.split()
+                vals[k] = float(v)
+    return vals
+
+
 def test_model_size_and_composition_pin():
-    """The 1.3B shapes reproduce the printed size split of the 278 MB model (56% scaffold, 37%
-    embedding/LM head, 4% LoRA, rest other) and 1 bit per scaffold weight (8x less than int8)."""
-    total = 278e6
+    """The 1.3B shapes reproduce the printed sizes (tests/golden/model_size.txt): the split of the 278 MB
+    model (scaffold, embedding/LM head, LoRA, other), the 2.7 GB FP16 teacher (every weight in fp16) and
+    its 9.7x reduction, and 1 bit per scaffold weight (8x less than int8)."""
+    g = _golden("model_size.txt")
+    total = g["compressed_model_mb"] * 1e6
     L, Dm, E, Nst, H = inputs.N_LAYERS, inputs.D_MODEL, inputs.D_INNER, inputs.D_STATE, inputs.N_HEADS
     d_ip = inputs.D_IN_PROJ
     assert d_ip == 2 * E + 2 * Nst + H == 8512
@@ -607,9 +622,13 @@ def test_model_size_and_composition_pin():
     scaffold_bytes = scaffold_weights / 8
     lm_bytes = inputs.VOCAB * Dm
     lora_bytes = L * (inputs.RANK * Dm + d_ip * inputs.RANK + inputs.RANK * E + Dm * inputs.RANK)
-    assert round(100 * scaffold_bytes / total) == 56
-    assert round(100 * lm_bytes / total) == 37
-    assert 4 <= 100 * lora_bytes / total < 5
+    assert round(100 * scaffold_bytes / total) == g["share_scaffold_pct"]
+    assert round(100 * lm_bytes / total) == g["share_embedding_lm_head_pct"]
+    assert g["share_lora_pct"] <= 100 * lora_bytes / total < g["share_lora_pct"] + 1
     other = total - scaffold_bytes - lm_bytes - lora_bytes
-    assert 2 <= 100 * other / total < 3.5
-    assert scaffold_weights / scaffold_bytes == 8
+    assert abs(100 * other / total - g["share_other_pct"]) < 1
+    assert scaffold_weights / scaffold_bytes == g["scaffold_memory_reduction_x"]
+    # the FP16 teacher: the scaffold's weights and the embedding/LM-head matrix at 2 bytes each
+    teacher_bytes = 2 * (scaffold_weights + inputs.VOCAB * Dm)
+    assert round(teacher_bytes / 1e9, 1) == g["fp16_teacher_gb"]
+    assert round(g["fp16_teacher_gb"] * 1e9 / total, 1) == g["reduction_x"]
