@@ -185,16 +185,17 @@ def ssm_step(ssm_state, x, dt_raw, A_log, dt_bias, D, Bm, Cm):
 
 
 def rmsnorm_quantize(h, w):
-    """RMSNorm folded into the quantizer. Returns (q [B][n], s [B], v [B][n], rms [B])."""
+    """RMSNorm then the per-token quantizer. Returns (q [B][n], s [B], u [B][n], r [B]): u the normalized
+    rows fl32(fl32(h r) w), r = fl32(1 / sqrt(mean(h^2) + 1e-5))."""
     h = _c(np.atleast_2d(h), np.float32)
     B, n = h.shape
     w = _c(w, np.float32)
     q = np.zeros((B, n), np.int8)
     s = np.zeros(B, np.float32)
-    v = np.zeros((B, n), np.float32)
-    rms = np.zeros(B, np.float64)
-    lib().oracle_rmsnorm_quantize(_p(h), _p(w), B, n, _p(q), _p(s), _p(v), _p(rms))
-    return q, s, v, rms
+    u = np.zeros((B, n), np.float32)
+    r = np.zeros(B, np.float32)
+    lib().oracle_rmsnorm_quantize(_p(h), _p(w), B, n, _p(q), _p(s), _p(u), _p(r))
+    return q, s, u, r
 
 
 def gate(y, z):
@@ -262,7 +263,7 @@ def embed(W, s_row, token: int):
 
 
 def final_head(W, s_row, h, norm_w=None, rows=None):
-    """Final RMSNorm (folded into the quantizer; None: no norm) + int8 LM head on one token h [d].
+    """Final RMSNorm (then the quantizer; None: no norm) + int8 LM head on one token h [d].
     Returns (logits, acc) for all rows or the listed rows."""
     W = _c(W, np.int8)
     V, d = W.shape
@@ -307,7 +308,8 @@ def layer_prefill(layers, h, conv_states, ssm_states):
     """Prefill of a prompt h [M][d_model] (batch 1) through the layers, layer after layer: each layer
     runs its decode step on tokens 0 .. M-1 in order (the definition of the recurrent model on a
     sequence), h and the per-layer states conv_states[l] [1][C][3], ssm_states[l] [1][H][P][N] are
-    updated in place."""
+    updated in place.  Pinned by a hand-written float64 layer applied token by token through two layers
+    (one head, d_state 1)."""
     assert h.dtype == np.float32 and h.flags["C_CONTIGUOUS"]
     for L, cs, ss in zip(layers, conv_states, ssm_states):
         for t in range(h.shape[0]):

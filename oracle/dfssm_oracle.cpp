@@ -106,21 +106,20 @@ void linear_core(int d_out, int d_in, int rank, const uint32_t* bits, const floa
   }
 }
 
-// Mamba-2 pre-mixer RMSNorm followed by the per-token quantizer (reading: eps = 1e-5, weight per
-// channel).  The quantizer is invariant to a positive scalar factor of its input — q(c*v) = q(v) and
-// s(c*v) = c*s(v) in exact arithmetic — so the RMS factor is folded into the scale:
-//   v_i = fl32(h_i * w_i);  (q, s0) = quantize(v);  rms = sqrt(sum_i h_i^2 / n + eps);  s = fl32(s0 / rms).
-// Returns rms (fp64) and leaves v = fl32(h*w) in v_out.
-double rmsnorm_quantize(const float* h, const float* w, int n, double eps, int8_t* q, float* s_out,
-                        float* v_out) {
+// Mamba-2 RMSNorm (reading: eps = 1e-5, one weight per channel) followed by the per-token quantizer,
+// each exactly as defined, one after the other:
+//   r   = fl32(1 / sqrt(sum_i h_i^2 / n + eps))     (fp64; the sum in index order, the squares exact)
+//   u_i = fl32(fl32(h_i * r) * w_i)                  (the normalized, weighted row, stored fp32)
+//   (q, s) = quantize(u)                             (quantize_row above)
+// Writes u to u_out and returns r.
+float rmsnorm_quantize(const float* h, const float* w, int n, double eps, int8_t* q, float* s_out,
+                       float* u_out) {
   double ss = 0.0;
   for (int i = 0; i < n; ++i) ss += (double)h[i] * (double)h[i];
-  for (int i = 0; i < n; ++i) v_out[i] = r32((double)h[i] * (double)w[i]);
-  float s0 = 0.0f;
-  quantize_row(v_out, n, q, &s0);
-  const double rms = std::sqrt(ss / (double)n + eps);
-  *s_out = r32((double)s0 / rms);
-  return rms;
+  const float r = r32(1.0 / std::sqrt(ss / (double)n + eps));
+  for (int i = 0; i < n; ++i) u_out[i] = r32((double)r32((double)h[i] * (double)r) * (double)w[i]);
+  quantize_row(u_out, n, q, s_out);
+  return r;
 }
 
 inline double silu64(double v) { return v / (1.0 + std::exp(-v)); }
@@ -129,7 +128,7 @@ inline double silu64(double v) { return v / (1.0 + std::exp(-v)); }
 
 extern "C" {
 
-int oracle_abi_version(void) { return 4; }
+int oracle_abi_version(void) { return 5; }
 
 // Pinned by: exhaustive byte-pattern round trip against an independent packer, brute force.
 int oracle_sign(const uint32_t* bits, int d_in, int o, int i) { return unpack_sign(bits, d_in, o, i); }
@@ -267,16 +266,17 @@ void oracle_ssm_step(float* ssm_state, const float* x, const float* dt_raw, cons
   }
 }
 
-// Pre-mixer RMSNorm + per-token quantization of B rows (the RMS factor folded into the scale); also
-// returns v = fl32(h*w) [B][n] and rms [B].
-// Pinned by: a constant row reconstructs w*sign(c); codes agree with quantizing the explicitly
-// normalized row away from rounding ties; scale relation.
+// RMSNorm + per-token quantization of B rows (rmsnorm_quantize); also returns the normalized rows
+// u [B][n] and the factors r [B].
+// Pinned by: r against the correctly rounded fp32 of the real-number factor (exact decimal arithmetic);
+// u against the real-number normalization to fp32 accuracy; the codes and scale are the pinned
+// quantizer's on u; a constant row gives w*sign(c)/sqrt(1 + eps/c^2); a zero weight zeroes a code.
 void oracle_rmsnorm_quantize(const float* h, const float* w, int B, int n, int8_t* q, float* s,
-                             float* v, double* rms) {
+                             float* u, float* r) {
   for (int b = 0; b < B; ++b) {
-    const double r = rmsnorm_quantize(h + (size_t)b * n, w, n, 1e-5, q + (size_t)b * n, s + b,
-                                      v + (size_t)b * n);
-    if (rms) rms[b] = r;
+    const float rb = rmsnorm_quantize(h + (size_t)b * n, w, n, 1e-5, q + (size_t)b * n, s + b,
+                                      u + (size_t)b * n);
+    if (r) r[b] = rb;
   }
 }
 
@@ -298,8 +298,9 @@ void oracle_gate(const float* y, const float* z, float* g, int n) {
 //   g       = gate(y, z);  (q', s') = rmsnorm_quantize(g, gnorm_w);  tf' = lora_down(q', s')
 //   h       = fl32(h + out_proj(q', s', tf'))
 // Shapes: D = d_model, E = d_inner = H*P, C = E + 2*G*N conv channels, in_proj rows 2E + 2GN + H.
-// Pinned by: composition of the separately pinned steps in this order; a zero out_proj scale leaves
-// h unchanged.
+// Pinned by: the whole step written out by hand in float64 from the definitions for one head of 32
+// channels with d_state 1 over four tokens (and over a five-token prompt through two layers); a zero
+// out_proj scale leaves h unchanged.
 void oracle_layer_decode(int B, int Dm, int H, int P, int N, int G, int rank,
                          // in_proj
                          const uint32_t* in_bits, const float* in_ws, const int8_t* in_lb,
@@ -378,14 +379,14 @@ int oracle_embed(const int8_t* W, const float* s_row, int V, int d, int tok, flo
 }
 
 // Final RMSNorm + int8 LM head on one token (reading: the Mamba-2 language model [MAP] applies an
-// RMSNorm with its own weight, eps 1e-5, to the last layer's residual stream before the LM head).
-// The norm is folded into the quantizer exactly as for the pre-mixer norm (rmsnorm_quantize):
+// RMSNorm with its own weight, eps 1e-5, to the last layer's residual stream before the LM head), the
+// same norm-then-quantize as the pre-mixer norm (rmsnorm_quantize):
 //   (q, s) = rmsnorm_quantize(h, norm_w);  logits[v] = fl32(acc[v] * s * s_row[v]),
 //   acc[v] = sum_i W[v,i] * q[i].
 // norm_w == NULL gives the plain LM head (oracle_lm_head).  Only rows listed in `rows` are computed
 // when rows != NULL.
-// Pinned by: brute-force int64 matmul of the pinned codes; agreement with the plain LM head on the
-// explicitly normalized row away from rounding ties.
+// Pinned by: brute-force int64 matmul of the pinned codes; equality with the plain LM head applied to the
+// pinned normalized row; a constant row's closed form; a zero norm weight zeroes its codes.
 void oracle_final_head(const int8_t* W, const float* s_row, int V, int d, const float* h,
                        const float* norm_w, const int* rows, int n_rows, float* logits,
                        int32_t* acc_out) {

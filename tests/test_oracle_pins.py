@@ -5,6 +5,8 @@ Each test names the plausible mistake it would catch.
 """
 import os
 
+from decimal import Decimal, getcontext
+
 import numpy as np
 import pytest
 from scipy.special import expit
@@ -359,34 +361,83 @@ def test_ssm_dA_to_zero_is_memoryless():
 
 # --------------------------------------------------------------------------------- norms and gate
 
-def test_rmsnorm_constant_row_reconstructs_weight():
-    g = np.random.default_rng(30)
-    w = g.uniform(0.5, 1.5, 256).astype(np.float32)
-    for c in (-3.0, 0.25, 40.0):
-        h = np.full((1, 256), c, np.float32)
-        q, s, _, rms = oracle.rmsnorm_quantize(h, w)
-        assert abs(rms[0] - np.sqrt(c * c + 1e-5)) <= 1e-12 * abs(c)
-        u = np.sign(c) * w.astype(np.float64) / np.sqrt(1 + 1e-5 / c ** 2)
-        assert np.all(np.abs(s[0] * q[0] - u) <= s[0] / 2 * 1.0001)
+def _f32_correctly_rounded(d: Decimal):
+    """The fp32 value nearest the exact decimal d, and the relative distance of d from the nearest fp32
+    rounding boundary (a midpoint between two fp32 neighbours)."""
+    f = np.float32(float(d))
+    cands = [np.nextafter(f, np.float32(-np.inf)), f, np.nextafter(f, np.float32(np.inf))]
+    best = min(cands, key=lambda c: abs(Decimal(float(c)) - d))
+    lo, hi = np.nextafter(best, np.float32(-np.inf)), np.nextafter(best, np.float32(np.inf))
+    mids = [(Decimal(float(best)) + Decimal(float(lo))) / 2, (Decimal(float(best)) + Decimal(float(hi))) / 2]
+    margin = min(abs(d - m) for m in mids) / abs(d)
+    return best, margin
 
 
-def test_rmsnorm_fold_matches_explicit_normalization_away_from_ties():
-    """Quantizing the explicitly normalized row gives the same codes except within 1e-4 of a rounding
-    tie, and the scale is the explicit one to fp32 precision."""
+def test_rmsnorm_factor_is_the_correctly_rounded_real_number():
+    """r = 1/sqrt(mean(h^2) + eps), evaluated exactly in 60-digit decimal arithmetic from the fp32 inputs
+    and rounded once to fp32.  Catches a wrong epsilon, n - 1 for n, a missing square root, or the sum
+    of |h| instead of h^2.  Rows near a rounding boundary (relative margin below 2^-45, where the fp64
+    evaluation may legitimately round the other way) are skipped and counted."""
+    getcontext().prec = 60
+    g = np.random.default_rng(33)
+    rows = [g.standard_normal(256) * 3, g.standard_normal(2048), g.standard_normal(64) * 1e-3,
+            np.full(32, 2.0 ** -9), g.uniform(-1, 1, 4096) * 50, np.zeros(128)]
+    checked = 0
+    for h in rows:
+        h = h.astype(np.float32)
+        w = np.ones(h.size, np.float32)
+        _, _, _, r = oracle.rmsnorm_quantize(h[None], w)
+        ss = sum(Decimal(float(v)) ** 2 for v in h)
+        exact = 1 / (ss / h.size + Decimal(1e-5)).sqrt()
+        want, margin = _f32_correctly_rounded(exact)
+        if margin < Decimal(2) ** -45:
+            continue
+        assert r[0] == want, (h.size, r[0], want)
+        checked += 1
+    assert checked >= 5
+
+
+def test_rmsnorm_normalized_row_and_codes():
+    """u = h w / sqrt(mean(h^2) + eps) to fp32 accuracy (two fp32 roundings and r's), and the codes and
+    scale are exactly those of the pinned quantizer applied to u: catches a missing weight, a quantizer
+    that runs before the norm, or the RMS factor applied to the scale instead of the values."""
     g = np.random.default_rng(31)
     h = (g.standard_normal((8, 2048)) * 3).astype(np.float32)
     w = g.uniform(0.5, 1.5, 2048).astype(np.float32)
-    q, s, v, rms = oracle.rmsnorm_quantize(h, w)
-    assert np.array_equal(v, (h.astype(np.float64) * w).astype(np.float32))
-    for b in range(8):
-        hb = h[b].astype(np.float64)
-        u = hb / np.sqrt(np.mean(hb ** 2) + 1e-5) * w
-        m = np.abs(u).max()
-        r = u / (m / 127)
-        near_tie = np.abs(np.abs(r - np.floor(r)) - 0.5) < 1e-4
-        exact = np.rint(r).astype(np.int64)
-        assert np.all((exact == q[b]) | near_tie)
-        assert abs(s[b] - m / 127) <= 1e-6 * m / 127
+    q, s, u, r = oracle.rmsnorm_quantize(h, w)
+    h64 = h.astype(np.float64)
+    exact = h64 / np.sqrt(np.mean(h64 ** 2, axis=1, keepdims=True) + 1e-5) * w
+    assert np.all(np.abs(u - exact) <= 4 * 2.0 ** -24 * np.abs(exact))
+    q2, s2 = oracle.quantize(u)
+    assert np.array_equal(q, q2) and np.array_equal(s, s2)
+
+
+def test_rmsnorm_constant_row_closed_form():
+    """h = c everywhere: mean(h^2) = c^2, so u_i = w_i sign(c) / sqrt(1 + eps/c^2), and the largest
+    weight's code is 127 sign(c)."""
+    g = np.random.default_rng(30)
+    w = g.uniform(0.5, 1.5, 256).astype(np.float32)
+    for c in (-3.0, 0.25, 40.0, 1e-3):
+        q, s, u, r = oracle.rmsnorm_quantize(np.full((1, 256), c, np.float32), w)
+        want = np.sign(c) * w.astype(np.float64) / np.sqrt(1 + 1e-5 / c ** 2)
+        assert np.all(np.abs(u[0] - want) <= 3 * 2.0 ** -24 * np.abs(want))
+        assert q[0, np.argmax(w)] == 127 * np.sign(c)
+        assert np.all(np.abs(s[0] * q[0] - want) <= s[0] / 2 * 1.0001)
+
+
+def test_rmsnorm_zero_weight_and_zero_row():
+    """A zero weight zeroes its code (the weight multiplies before the quantizer); an all-zero row gives
+    r = fl32(1/sqrt(eps)), u = 0, s = 0 and all codes 0."""
+    g = np.random.default_rng(34)
+    h = g.standard_normal((1, 64)).astype(np.float32)
+    w = np.ones(64, np.float32)
+    w[::2] = 0
+    q, s, u, _ = oracle.rmsnorm_quantize(h, w)
+    assert np.all(q[0, ::2] == 0) and np.all(u[0, ::2] == 0)
+    assert np.any(q[0, 1::2] != 0)
+    q, s, u, r = oracle.rmsnorm_quantize(np.zeros((1, 64), np.float32), np.ones(64, np.float32))
+    assert r[0] == np.float32(1 / np.sqrt(1e-5))
+    assert np.all(u == 0) and np.all(q == 0) and s[0] == 0
 
 
 def test_gate_silu_against_logistic():
@@ -423,32 +474,89 @@ def test_layer_zero_out_proj_keeps_residual():
     assert np.any(ssm[0] != 0) and np.any(taps["y"] != 0)
 
 
-def test_layer_composition_of_pinned_steps():
-    """The layer equals the pinned steps wired as: norm+quant (+ LoRA down on the codes) ->
-    in_proj -> split z|x|B|C|dt -> conv -> SSM -> gate -> norm+quant -> out_proj -> residual."""
-    m = inputs.decode_model(seed=41, n_layers=1, n_tokens=3, **SMALL)
-    lay = _oracle_layer(m["layers"][0])
-    E, N = 64, 16
-    conv_a, ssm_a = inputs.zero_states(1, 1, 4, 16, 16, 1)
-    conv_b, ssm_b = conv_a.copy(), ssm_a.copy()
-    for t in range(3):
-        h_a = m["emb"][t].copy()
-        oracle.layer_decode(lay, h_a, conv_a[0], ssm_a[0])
-        h_b = m["emb"][t].copy()
-        q, s, v, rms = oracle.rmsnorm_quantize(h_b, lay["norm_w"])
-        _, tf = oracle.lora_down(lay["in_proj"], q[0], s[0])
-        zx, _ = oracle.linear_core(lay["in_proj"], q[0], s[0], tf)
-        z, xbc, dt = zx[:E], zx[E:E + E + 2 * N], zx[E + E + 2 * N:]
-        xc = oracle.conv_step(conv_b[0], lay["conv_w"], lay["conv_b"], xbc[None])[0]
-        y = oracle.ssm_step(ssm_b[0], xc[None, :E], dt[None], lay["A_log"], lay["dt_bias"], lay["D"],
-                            xc[None, E:E + N], xc[None, E + N:])[0]
-        gg = oracle.gate(y, z)
-        q2, s2, v2, rms2 = oracle.rmsnorm_quantize(gg[None], lay["gnorm_w"])
-        _, tf2 = oracle.lora_down(lay["out_proj"], q2[0], s2[0])
-        out, _ = oracle.linear_core(lay["out_proj"], q2[0], s2[0], tf2)
-        h_b = (h_b[0] + out).astype(np.float32)
-        assert np.array_equal(h_a[0], h_b)
-        assert np.array_equal(ssm_a, ssm_b) and np.array_equal(conv_a, conv_b)
+def _hand_layer(P, h, conv, S):
+    """One decode step of a Mamba-2 layer with one head, d_state 1 and ngroups 1, written out from the
+    definitions in float64 numpy (no oracle call): RMSNorm, per-token absmax int8 codes, the +-1
+    scaffold and the int8 LoRA on the codes, the split z | x | B | C | dt, the width-4 causal conv with
+    SiLU, softplus dt, the scalar-state recurrence S <- exp(dt A) S + dt x B, y = S C + D x, the gate
+    y SiLU(z), the gated RMSNorm, out_proj and the residual.  conv [C][3] and S [E] are updated in
+    place; returns the new h and the codes' distances from a rounding tie (to check the margin)."""
+    silu = lambda v: v / (1 + np.exp(-v))
+
+    def norm_codes(v, w):
+        u = v / np.sqrt(np.mean(v * v) + 1e-5) * w
+        s = np.abs(u).max() / 127
+        t = u / s
+        return np.rint(t), s, np.abs(np.abs(t - np.floor(t)) - 0.5)
+
+    def linear(L, q, s):
+        sign = unpack_pm1(L["bits"]).astype(np.float64)
+        t = L["lora_b"].astype(np.float64) @ q
+        tf = t * L["lora_b_scale"] * s
+        return (sign @ q) * s * L["w_scale"] + L["lora_a_scale"] * (L["lora_a"].astype(np.float64) @ tf)
+
+    E = P["gnorm_w"].size
+    q, s, gap1 = norm_codes(h, P["norm_w"])
+    zx = linear(P["in_proj"], q, s)
+    z, xbc, dt_raw = zx[:E], zx[E:2 * E + 2], zx[2 * E + 2]
+    w = P["conv_w"].astype(np.float64)
+    pre = P["conv_b"] + w[:, 0] * conv[:, 0] + w[:, 1] * conv[:, 1] + w[:, 2] * conv[:, 2] + w[:, 3] * xbc
+    conv[:, :2] = conv[:, 1:]
+    conv[:, 2] = xbc
+    xc = silu(pre)
+    x, Bv, Cv = xc[:E], xc[E], xc[E + 1]
+    dt = np.log1p(np.exp(dt_raw + P["dt_bias"][0]))
+    a = np.exp(dt * -np.exp(float(P["A_log"][0])))
+    S[:] = a * S + dt * x * Bv
+    y = S * Cv + P["D"][0] * x
+    g = y * silu(z)
+    q2, s2, gap2 = norm_codes(g, P["gnorm_w"])
+    return h + linear(P["out_proj"], q2, s2), min(gap1.min(), gap2.min())
+
+
+WIRE = dict(d_model=32, nheads=1, headdim=32, d_state=1, ngroups=1, rank=3)
+
+
+def test_layer_wiring_against_hand_computed_closed_form():
+    """The oracle's layer decode over four tokens equals the whole step written out in float64 from the
+    definitions (one head of 32 channels, d_state 1, rank 3): catches a wrong split order, the gate after
+    the norm, a missing D skip or residual, a conv state shifted the wrong way, or dt from the wrong row.
+    The test's own codes stay at least 1e-3 away from a rounding tie, so both sides pick the same codes
+    and agree to fp32 rounding."""
+    m = inputs.decode_model(seed=43, n_layers=1, n_tokens=4, **WIRE)
+    P = m["layers"][0]
+    lay = _oracle_layer(P)
+    conv, ssm = inputs.zero_states(1, 1, 1, 32, 1, 1)
+    conv_h = np.zeros((34, 3))
+    S_h = np.zeros(32)
+    for t in range(4):
+        h = m["emb"][t].copy()
+        oracle.layer_decode(lay, h, conv[0], ssm[0])
+        want, gap = _hand_layer(P, m["emb"][t][0].astype(np.float64), conv_h, S_h)
+        assert gap > 1e-3
+        assert np.allclose(h[0], want, rtol=2e-6, atol=1e-6), t
+        assert np.allclose(ssm[0, 0, 0, :, 0], S_h, rtol=2e-6, atol=1e-7)
+        assert np.allclose(conv[0, 0], conv_h, rtol=1e-6, atol=1e-7)
+
+
+def test_layer_prefill_against_hand_computed_closed_form():
+    """A 5-token prompt through two such layers: the oracle's layer-major prefill equals the hand-written
+    step applied token by token through both layers, and so does the token-major decode."""
+    m = inputs.decode_model(seed=44, n_layers=2, n_tokens=5, **WIRE)
+    layers = [_oracle_layer(ld) for ld in m["layers"]]
+    conv, ssm = inputs.zero_states(1, 2, 1, 32, 1, 1)
+    prompt = np.ascontiguousarray(m["emb"][:, 0, :])
+    h = oracle.layer_prefill(layers, prompt.copy(), conv, ssm)
+    conv_h = [np.zeros((34, 3)) for _ in range(2)]
+    S_h = [np.zeros(32) for _ in range(2)]
+    for t in range(5):
+        v = prompt[t].astype(np.float64)
+        for l in range(2):
+            v, gap = _hand_layer(m["layers"][l], v, conv_h[l], S_h[l])
+            assert gap > 1e-3
+        assert np.allclose(h[t], v, rtol=5e-6, atol=2e-6), t
+    for l in range(2):
+        assert np.allclose(ssm[l, 0, 0, :, 0], S_h[l], rtol=5e-6, atol=1e-7)
 
 
 # ------------------------------------------------------------------------------------------ LM head
@@ -539,9 +647,9 @@ def test_final_head_norm_weight_enters_the_codes():
     assert np.array_equal(acc, acc_half)
 
 
-def test_final_head_fold_matches_explicit_normalization():
-    """The folded norm equals the plain LM head on the explicitly normalized row: same integer sums
-    (no code is near a rounding tie for this input) and logits to fp32 precision."""
+def test_final_head_is_the_lm_head_of_the_normalized_row():
+    """The final head equals the plain LM head applied to the pinned normalized row u (same integer sums,
+    same logits), and its integer sums are the brute-force product with the codes of u."""
     g = np.random.default_rng(55)
     V, d = 500, 256
     W = g.integers(-127, 128, (V, d), dtype=np.int8)
@@ -549,15 +657,10 @@ def test_final_head_fold_matches_explicit_normalization():
     h = (g.standard_normal(d) * 2).astype(np.float32)
     w = g.uniform(0.5, 1.5, d).astype(np.float32)
     logits, acc = oracle.final_head(W, sr, h, w)
-    h64 = h.astype(np.float64)
-    u = h64 / np.sqrt(np.mean(h64 ** 2) + 1e-5) * w
-    r = u / (np.abs(u).max() / 127)
-    assert np.all(np.abs(np.abs(r - np.floor(r)) - 0.5) > 1e-4)  # no near-tie code for this seed
-    q = np.rint(r).astype(np.int64)
-    assert np.array_equal(acc, W.astype(np.int64) @ q)
-    l2, a2 = oracle.lm_head(W, sr, u.astype(np.float32))
-    assert np.array_equal(a2, acc)
-    assert np.allclose(logits, l2, rtol=2e-7, atol=0)
+    q, s, u, _ = oracle.rmsnorm_quantize(h[None], w)
+    assert np.array_equal(acc, W.astype(np.int64) @ q[0].astype(np.int64))
+    l2, a2 = oracle.lm_head(W, sr, u[0])
+    assert np.array_equal(a2, acc) and np.array_equal(l2, logits)
     # the plain head is the final head without a norm
     l3, a3 = oracle.final_head(W, sr, h)
     l4, a4 = oracle.lm_head(W, sr, h)
