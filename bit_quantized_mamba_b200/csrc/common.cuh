@@ -233,14 +233,13 @@ __device__ __forceinline__ float lora_tf(int t, float sB, float s) {
   return __double2float_rn(dmul(dmul(int_to_f64(t), (double)sB), (double)s));
 }
 
-// RMS of a row with sum of squares ss: sqrt(ss/n + 1e-5) (fp64); the quantizer scale of the normalized
-// row is fl32(s0 / rms).
-__device__ __forceinline__ double rms_of(double ss, int n) {
-  return __dsqrt_rn(__dadd_rn(__ddiv_rn(ss, (double)n), 1e-5));
+// RMSNorm (eps 1e-5, a weight per channel), then the quantizer on the normalized row:
+//   r = fl32(1 / sqrt(ss / n + 1e-5))   (fp64; ss the fp64 sum of the exact squares of the row)
+//   u = fl32(fl32(h * r) * w)
+__device__ __forceinline__ float rms_factor(double ss, int n) {
+  return __double2float_rn(__ddiv_rn(1.0, __dsqrt_rn(__dadd_rn(__ddiv_rn(ss, (double)n), 1e-5))));
 }
-__device__ __forceinline__ float rms_scale(float s0, double rms) {
-  return __double2float_rn(__ddiv_rn((double)s0, rms));
-}
+__device__ __forceinline__ float norm_value(float h, float r, float w) { return fmul(fmul(h, r), w); }
 
 // Conv pre-activation fl32(b + w0*s0 + w1*s1 + w2*s2 + w3*x) (fp64, this order), then SiLU.
 __device__ __forceinline__ float conv_out(float4 w, float bias, float s0, float s1, float s2, float x) {

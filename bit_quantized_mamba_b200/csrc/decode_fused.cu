@@ -35,7 +35,7 @@ constexpr int MIN_CTAS = 137, MAX_CTAS = 256;  // >= 137: at most 15 out_proj ro
 static_assert(NW == R, "one warp per LoRA row");
 constexpr int kPrefetchThread = 32;     // warp 1 issues the next layer's L2 prefetches
 constexpr int kCopyThread = 64;         // warp 2 issues the layer's bulk copies (thread 0 polls)
-constexpr int kChainWarp = NW - 1;      // warp 15 computes the fp64 scale chain (no out_proj row)
+constexpr int kChainWarp = NW - 1;      // warp 15 forms the LoRA intermediate (no out_proj row)
 constexpr int kChainBase = kChainWarp * 32;
 
 enum { CTR_H = 0, CTR_BC, CTR_G, N_CTR };
@@ -240,6 +240,17 @@ __device__ __forceinline__ float block_absmax(float m, int lane, int warp, unsig
   }
   return __uint_as_float(mb);
 }
+// Block-wide fp64 sum of the threads' v (every thread gets the same value: the per-warp sums are added
+// in warp order).  Contains one CTA barrier.
+__device__ __forceinline__ double block_sum_d(double v, int lane, int warp, double* red_d) {
+  v = warp_sum(v);
+  if (lane == 0) red_d[warp] = v;
+  __syncthreads();
+  double t = 0.0;
+#pragma unroll
+  for (int q = 0; q < NW; ++q) t += red_d[q];
+  return t;
+}
 // Sum of the sixteen per-warp partial sums.
 __device__ __forceinline__ int block_sum16(const int* red_i) {
   int t = 0;
@@ -271,7 +282,7 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ P
   float* const st_sm = reinterpret_cast<float*>(wb_sm + WB_BYTES);  // [2][MAX_SSM][N], layer l in l & 1
   __shared__ __align__(16) int8_t q_perm[E];
   __shared__ __align__(16) int8_t q_nat[E];
-  __shared__ double ss_sm[NT];                 // per-thread sums of squares (summed by the chain warp)
+  __shared__ __align__(16) double red_d[NW];   // per-warp sums of squares
   __shared__ __align__(16) unsigned red_u[NW];  // per-warp absmax (bit pattern of a non-negative float)
   __shared__ __align__(16) int red_i[NW];       // per-warp code sums
   __shared__ float lbs_o[R];                    // out_proj W_B row scales
@@ -496,22 +507,25 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ P
       drain(l, has_next);
       return;
     }
-    // RMSNorm folded into the quantizer: codes from the absmax alone; the sum of squares (for the scale)
-    // is parked per thread and reduced by the chain warp off the critical path
+    // RMSNorm, then the quantizer on the normalized row: r from the block sum of squares, then the
+    // absmax of u = fl32(fl32(h r) w)
     float s0A;
     {
-      float v[4];
+      float hv[4], v[4];
       double ss = 0.0;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        hv[k] = __ldcg(p.hidden + tid + k * NT);
+        ss += (double)hv[k] * (double)hv[k];
+      }
+      if (tid < n_out) h_old[tid] = __ldcg(p.hidden + ro0 + tid);
+      const float rn = rms_factor(block_sum_d(ss, lane, warp, red_d), DM);
       float m = 0.0f;
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
-        const float hv = __ldcg(p.hidden + tid + k * NT);
-        ss += (double)hv * (double)hv;
-        v[k] = fmul(hv, nw[k]);
+        v[k] = norm_value(hv[k], rn, nw[k]);
         m = fmaxf(m, fabsf(v[k]));
       }
-      if (tid < n_out) h_old[tid] = __ldcg(p.hidden + ro0 + tid);
-      ss_sm[tid] = ss;
       m = block_absmax(m, lane, warp, red_u);
       const float s0 = m == 0.0f ? 0.0f : __fdiv_rn(m, 127.0f);
       const float inv_s0 = m == 0.0f ? 0.0f : __frcp_rn(s0);
@@ -550,17 +564,10 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ P
         }
       }
     }
-    // the fp64 scale chain (RMS, quantizer scale, LoRA intermediate), off the GEMV's critical path: the
-    // chain warp has no pass-1 rows, and the epilogue needs the results only after the B/C wait
-    if (warp == kChainWarp) {
-      double ss = 0.0;
-#pragma unroll
-      for (int k = 0; k < NT / 32; ++k) ss += ss_sm[lane + 32 * k];
-      ss = warp_sum(ss);
-      if (lane == R) s_scale = rms_scale(s0A, rms_of(ss, DM));
-    }
+    // the LoRA intermediate (off the GEMV's critical path: the epilogue needs it only after the B/C wait)
     __syncthreads();
-    if (tid >= kChainBase && tid < kChainBase + R) tf[tid - kChainBase] = lora_tf(t_sm[tid - kChainBase], lbs_in, s_scale);
+    if (tid >= kChainBase && tid < kChainBase + R) tf[tid - kChainBase] = lora_tf(t_sm[tid - kChainBase], lbs_in, s0A);
+    if (tid == kChainBase + R) s_scale = s0A;
 
     // ---------------------------------------------------------------- phase B: epilogues + SSM
     if (!block_wait(p.ctr + CTR_BC * CTR_STRIDE, NC * (l + 1), p.err, p.status, p.spin_limit, &sflag)) {
@@ -659,17 +666,20 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ P
       }
     }
     {
-      float v[8];
+      float gv[8], v[8];
       double ss = 0.0;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        gv[k] = __ldcg(p.gbuf + tid + k * NT);
+        ss += (double)gv[k] * (double)gv[k];
+      }
+      const float rn = rms_factor(block_sum_d(ss, lane, warp, red_d), E);
       float m = 0.0f;
 #pragma unroll
       for (int k = 0; k < 8; ++k) {
-        const float g = __ldcg(p.gbuf + tid + k * NT);
-        ss += (double)g * (double)g;
-        v[k] = fmul(g, gw[k]);
+        v[k] = norm_value(gv[k], rn, gw[k]);
         m = fmaxf(m, fabsf(v[k]));
       }
-      ss_sm[tid] = ss;
       m = block_absmax(m, lane, warp, red_u);
       const float s0 = m == 0.0f ? 0.0f : __fdiv_rn(m, 127.0f);
       const float inv_s0 = m == 0.0f ? 0.0f : __frcp_rn(s0);
@@ -684,18 +694,12 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ P
       }
       sq = __reduce_add_sync(0xffffffffu, sq);
       if (lane == 0) red_i[warp] = sq;
+      if (tid == 0) s_scale = s0;
       __syncthreads();
-      // LoRA down of the codes (warp r: t[r]); the GEMV warps then take one out_proj row each, and the
-      // chain warp (no out_proj row) computes the quantizer scale
+      // LoRA down of the codes (warp r: t[r]); every warp with an out_proj row then takes it
       const int t = lora_row<E / 16>(wb_out + warp * E, q_nat, lane);
       if (lane == 0) t_sm[warp] = t;
-      if (warp == kChainWarp) {
-        double sst = 0.0;
-#pragma unroll
-        for (int k = 0; k < NT / 32; ++k) sst += ss_sm[lane + 32 * k];
-        sst = warp_sum(sst);
-        if (lane == 0) s_scale = rms_scale(s0, rms_of(sst, E));
-      } else {
+      if (warp != kChainWarp) {
         const int sumq_c = block_sum16(red_i);
         const uint4* qp4 = reinterpret_cast<const uint4*>(q_perm) + lane;
         int S = bits_dot<E / 128>(w_out, qp4);

@@ -66,8 +66,8 @@ static cudaError_t launch_pdl(Kern k, dim3 grid, dim3 block, size_t smem, cudaSt
 }
 
 // ------------------------------------------------------------------------------- quantize kernel
-// One CTA per token.  v = x (or fl32(x*norm_w) when the RMSNorm is folded in); s0 = fl32(absmax/127);
-// q = clamp(rint(fl32(v/s0)), +-127); rms = 1 (or sqrt(sum x^2 / n + 1e-5) in fp64); s = fl32(s0/rms).
+// One CTA per token.  v = x, or with a norm weight the RMSNorm of x: r = fl32(1/sqrt(sum x^2/n + 1e-5))
+// (fp64) and v = fl32(fl32(x r) w); then s = fl32(absmax(v)/127), q = clamp(rint(fl32(v/s)), +-127).
 // LoRA down on the codes: t[r] = sum_i W_B[r,i] q_i (int32, dp4a), tf[r] = fl32(t[r] sB[r] s).
 
 constexpr int kQuantThreads = 512;
@@ -87,31 +87,32 @@ __global__ void __launch_bounds__(kQuantThreads) quant_kernel(QuantArgs a) {
   constexpr int NW = kQuantThreads / 32;
   const float* x = a.x + (size_t)b * a.ldx;
 
-  double ss = 0.0;
+  float r = 1.0f;
+  if (a.norm_w) {
+    double ss = 0.0;
+    for (int i = tid; i < a.n; i += kQuantThreads) {
+      const float xv = x[i];
+      ss += (double)xv * (double)xv;  // the square of an fp32 value is exact in fp64
+    }
+    ss = warp_sum(ss);
+    if (lane == 0) red_d[wid] = ss;
+    __syncthreads();
+    ss = 0.0;
+    for (int w = 0; w < NW; ++w) ss += red_d[w];
+    r = rms_factor(ss, a.n);
+  }
   float m = 0.0f;
   for (int i = tid; i < a.n; i += kQuantThreads) {
     const float xv = x[i];
-    float vv = xv;
-    if (a.norm_w) {
-      ss += (double)xv * (double)xv;
-      vv = fmul(xv, a.norm_w[i]);
-    }
+    const float vv = a.norm_w ? norm_value(xv, r, a.norm_w[i]) : xv;
     v[i] = vv;
     m = fmaxf(m, fabsf(vv));
   }
   m = warp_max(m);
-  ss = warp_sum(ss);
-  if (lane == 0) {
-    red_f[wid] = m;
-    red_d[wid] = ss;
-  }
+  if (lane == 0) red_f[wid] = m;
   __syncthreads();
   m = 0.0f;
-  ss = 0.0;
-  for (int w = 0; w < NW; ++w) {
-    m = fmaxf(m, red_f[w]);
-    ss += red_d[w];
-  }
+  for (int w = 0; w < NW; ++w) m = fmaxf(m, red_f[w]);
   const float s0 = (m == 0.0f) ? 0.0f : __fdiv_rn(m, 127.0f);
   const float inv_s0 = (m == 0.0f) ? 0.0f : __frcp_rn(s0);
 
@@ -137,8 +138,7 @@ __global__ void __launch_bounds__(kQuantThreads) quant_kernel(QuantArgs a) {
     if (lane == 0) t_sm[r] = part;
   }
   __syncthreads();
-  const double rms = a.norm_w ? rms_of(ss, a.n) : 1.0;
-  const float s = a.norm_w ? rms_scale(s0, rms) : s0;
+  const float s = s0;
   if (tid < DFSSM_MAX_RANK) {
     float tf = 0.0f;
     if (tid < a.rank) {

@@ -153,8 +153,8 @@ __global__ void expand_bits_kernel(const uint32_t* __restrict__ bits, int8_t* __
 // decode quantizer; the LoRA down-projection t = W_B q on the codes (int32, dp4a) with W_B staged in
 // shared memory (zero rows beyond the rank, so every lane runs all sixteen rows without branches), and
 // tf = fl32(t sB s) rounded as in the decode path.  Each lane keeps eight 16-byte loads of its token in
-// flight.  With a norm weight (a layer's pre-norm or gated norm) the RMSNorm is folded in as in decode:
-// the codes are those of v = fl32(x w), and s = fl32(s0 / rms), rms = sqrt(sum x^2 / K + 1e-5) (fp64).
+// flight.  With a norm weight (a layer's pre-norm or gated norm) the token is first normalized as in
+// decode: r = fl32(1/sqrt(sum x^2 / K + 1e-5)) (fp64) and v = fl32(fl32(x r) w) is quantized.
 constexpr int QW = 8;  // tokens (warps) per CTA
 constexpr int QU = 8;  // float4 loads in flight per lane
 __global__ void __launch_bounds__(QW * 32) prefill_quant_kernel(const float* __restrict__ x, int M, int K,
@@ -205,14 +205,33 @@ __global__ void __launch_bounds__(QW * 32) prefill_quant_kernel(const float* __r
   const float4* wr = reinterpret_cast<const float4*>(norm_w);
   const int K4 = K / 4;  // a multiple of 32: the bounds tests below are uniform over the warp
   constexpr int UB = QU;  // float4 per lane per batch
-  // v = fl32(x w) with a norm weight, else x
+  // RMSNorm factor (with a norm weight): a first pass for the sum of squares (exact squares in fp64)
+  float rn = 1.0f;
+  if (wr) {
+    double ss = 0.0;
+    for (int i0 = lane; i0 < K4; i0 += 32 * UB) {
+      float4 v[UB];
+#pragma unroll
+      for (int u = 0; u < UB; ++u)
+        v[u] = i0 + 32 * u < K4 ? __ldg(xr + i0 + 32 * u) : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int u = 0; u < UB; ++u) {
+        ss = fma((double)v[u].x, (double)v[u].x, ss);
+        ss = fma((double)v[u].y, (double)v[u].y, ss);
+        ss = fma((double)v[u].z, (double)v[u].z, ss);
+        ss = fma((double)v[u].w, (double)v[u].w, ss);
+      }
+    }
+    rn = rms_factor(warp_sum(ss), K);
+  }
+  // v = fl32(fl32(x r) w) with a norm weight, else x
   const auto scale4 = [&](float4 a, int i) {
     if (!wr) return a;
     const float4 w = __ldg(wr + i);
-    return make_float4(fmul(a.x, w.x), fmul(a.y, w.y), fmul(a.z, w.z), fmul(a.w, w.w));
+    return make_float4(norm_value(a.x, rn, w.x), norm_value(a.y, rn, w.y), norm_value(a.z, rn, w.z),
+                       norm_value(a.w, rn, w.w));
   };
   float m_abs = 0.0f;
-  double ss = 0.0;
   for (int i0 = lane; i0 < K4; i0 += 32 * UB) {
     float4 v[UB];
 #pragma unroll
@@ -220,14 +239,8 @@ __global__ void __launch_bounds__(QW * 32) prefill_quant_kernel(const float* __r
       v[u] = i0 + 32 * u < K4 ? __ldg(xr + i0 + 32 * u) : make_float4(0.f, 0.f, 0.f, 0.f);
     if (wr) {
 #pragma unroll
-      for (int u = 0; u < UB; ++u) {
-        // squares of fp32 values are exact in fp64
-        ss = fma((double)v[u].x, (double)v[u].x, ss);
-        ss = fma((double)v[u].y, (double)v[u].y, ss);
-        ss = fma((double)v[u].z, (double)v[u].z, ss);
-        ss = fma((double)v[u].w, (double)v[u].w, ss);
+      for (int u = 0; u < UB; ++u)
         if (i0 + 32 * u < K4) v[u] = scale4(v[u], i0 + 32 * u);
-      }
     }
 #pragma unroll
     for (int u = 0; u < UB; ++u)
@@ -236,7 +249,7 @@ __global__ void __launch_bounds__(QW * 32) prefill_quant_kernel(const float* __r
   m_abs = warp_max(m_abs);
   const float s0 = m_abs == 0.0f ? 0.0f : __fdiv_rn(m_abs, 127.0f);
   const float inv_s0 = m_abs == 0.0f ? 0.0f : __frcp_rn(s0);
-  const float s_tok = wr ? rms_scale(s0, rms_of(warp_sum(ss), K)) : s0;
+  const float s_tok = s0;
   int u[DFSSM_MAX_RANK];
 #pragma unroll
   for (int r = 0; r < DFSSM_MAX_RANK; ++r) u[r] = 0;

@@ -123,8 +123,8 @@ cudaError_t launch_ssm(const SsmArgs& a, cudaStream_t st) {
 // ------------------------------------------------------------------------------ int8 LM-head GEMV
 // logits[v] = fl32(acc[v] * s * s_row[v]) (fp64, this order), acc[v] = sum_i W[v,i] q_i (int32 exact).
 // Every CTA quantizes the token itself (per-token absmax int8, the decode quantizer: no separate launch
-// and no hand-off); with a final RMSNorm weight the norm is folded in as for the layers' pre-norm:
-// codes of v = fl32(x w), s = fl32(s0 / rms), rms = sqrt(sum x^2 / d + 1e-5).  Each warp owns a
+// and no hand-off); with a final RMSNorm weight the token is first normalized as for the layers'
+// pre-norm: r = fl32(1/sqrt(sum x^2 / d + 1e-5)) (fp64) and v = fl32(fl32(x r) w) is quantized.  Each warp owns a
 // contiguous, balanced range of rows and streams it as units of 2 KB (four 16-byte chunks per lane of
 // one row), always with the next unit's loads in flight while the current one is summed; the first unit
 // is requested before the quantizer runs, so its latency is hidden.  The stream rate is set by the
@@ -173,53 +173,56 @@ __global__ void __launch_bounds__(256, LMH_CTAS_PER_SM) int8_gemv_kernel(Int8Gem
   pdl_launch_dependents();
   pdl_wait();
   const bool norm = a.norm_w != nullptr;
-  // quantize the token (two passes over x, 8 KB for d = 2048): thread t takes inputs t + 256 k
-  float m = 0.0f;
-  double ss = 0.0;
-  for (int k0 = 0; k0 * 256 < a.d; k0 += 8) {
-    float v[8];
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const int i = threadIdx.x + 256 * (k0 + k);
-      v[k] = i < a.d ? __ldg(a.x + i) : 0.0f;
-    }
-    if (norm) {
+  // quantize the token (8 KB for d = 2048; with a norm weight a first pass sums the squares):
+  // thread t takes inputs t + 256 k
+  float rn = 1.0f;
+  if (norm) {
+    double ss = 0.0;
+    for (int k0 = 0; k0 * 256 < a.d; k0 += 8) {
+      float v[8];
 #pragma unroll
       for (int k = 0; k < 8; ++k) {
         const int i = threadIdx.x + 256 * (k0 + k);
-        ss = fma((double)v[k], (double)v[k], ss);  // the square of an fp32 value is exact in fp64
-        v[k] = i < a.d ? fmul(v[k], __ldg(a.norm_w + i)) : 0.0f;
+        v[k] = i < a.d ? __ldg(a.x + i) : 0.0f;
       }
+#pragma unroll
+      for (int k = 0; k < 8; ++k) ss = fma((double)v[k], (double)v[k], ss);  // exact squares in fp64
     }
+    ss = warp_sum(ss);
+    if (lane == 0) red_ss[threadIdx.x >> 5] = ss;
+    __syncthreads();
+    ss = 0.0;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) ss += red_ss[w];
+    rn = rms_factor(ss, a.d);
+  }
+  const auto value = [&](int i) {
+    if (i >= a.d) return 0.0f;
+    const float xv = __ldg(a.x + i);
+    return norm ? norm_value(xv, rn, __ldg(a.norm_w + i)) : xv;
+  };
+  float m = 0.0f;
+  for (int k0 = 0; k0 * 256 < a.d; k0 += 8) {
+    float v[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) v[k] = value(threadIdx.x + 256 * (k0 + k));
 #pragma unroll
     for (int k = 0; k < 8; ++k) m = fmaxf(m, fabsf(v[k]));
   }
   m = warp_max(m);
-  if (norm) ss = warp_sum(ss);
-  if (lane == 0) {
-    red[threadIdx.x >> 5] = m;
-    red_ss[threadIdx.x >> 5] = ss;
-  }
+  if (lane == 0) red[threadIdx.x >> 5] = m;
   __syncthreads();
   m = 0.0f;
-  ss = 0.0;
 #pragma unroll
-  for (int w = 0; w < 8; ++w) {
-    m = fmaxf(m, red[w]);
-    ss += red_ss[w];
-  }
+  for (int w = 0; w < 8; ++w) m = fmaxf(m, red[w]);
   const float s0 = m == 0.0f ? 0.0f : __fdiv_rn(m, 127.0f);
   const float inv_s0 = m == 0.0f ? 0.0f : __frcp_rn(s0);
-  const float s = norm ? rms_scale(s0, rms_of(ss, a.d)) : s0;
+  const float s = s0;
   int8_t* qb = reinterpret_cast<int8_t*>(smem);
   for (int k0 = 0; k0 * 256 < a.d; k0 += 8) {
     float vv[8];
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const int i = threadIdx.x + 256 * (k0 + k);
-      vv[k] = i < a.d ? __ldg(a.x + i) : 0.0f;
-      if (norm) vv[k] = i < a.d ? fmul(vv[k], __ldg(a.norm_w + i)) : 0.0f;
-    }
+    for (int k = 0; k < 8; ++k) vv[k] = value(threadIdx.x + 256 * (k0 + k));
     int cd[8];
     quant_codes<8>(vv, s0, inv_s0, cd);
 #pragma unroll
