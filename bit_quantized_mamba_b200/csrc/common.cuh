@@ -86,33 +86,61 @@ __device__ __forceinline__ float silu_f64(float v) {
   return __double2float_rn(__ddiv_rn(d, __dadd_rn(1.0, exp(-d))));
 }
 
-// Per-token quantization code of v for scale s0 > 0: clamp(rint(fl32(v / s0)), -127, 127).
-__device__ __forceinline__ int quant_code(float v, float s0) {
-  float r = rintf(__fdiv_rn(v, s0));
-  r = fminf(fmaxf(r, -127.0f), 127.0f);
-  return (int)r;
+// Per-token quantizer scale s0 = fl32(m / 127) of a row with absmax m, and the reciprocal the code fast
+// path multiplies by.  s0 is the fp32 rounding of the fp64 product m * fl64(1/127): its relative error is
+// below 2^-51, and m / 127 is never within 2^-32 (relative) of an fp32 rounding midpoint (m has a 24-bit
+// significand, so 127 times a midpoint would need an odd multiple of 127 to equal an even integer), so the
+// result is always the IEEE quotient.  The reciprocal is approximate (relative error ~2^-23), which the
+// code fast path tolerates (see quant_codes); m == 0 gives s0 = 0 and a zero reciprocal.
+__device__ __forceinline__ float quant_scale(float m) {
+  return __double2float_rn(__dmul_rn((double)m, 1.0 / 127.0));
 }
-// Same code, computed as rint(v * fl32(1/s0)) unless that product lies within 1e-3 of a rounding
-// boundary: |v/s0| <= 127, and both v*fl32(1/s0) and fl32(v/s0) are within 2e-5 of v/s0, so away from a
-// boundary they round to the same integer; near one, the IEEE division decides.
+__device__ __forceinline__ float quant_inv(float s0) {
+  if (s0 == 0.0f) return 0.0f;
+  if (s0 < 1e-30f) return __frcp_rn(s0);  // subnormal range: no flush to zero
+  float r;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(s0));
+  return r;
+}
+
+// Round-half-to-even of |t| < 2^22 on the fp32 adder: t + 1.5*2^23 rounds t to an integer (ties to even)
+// and leaves that integer in the low significand bits.  kf is the rounded value as a float.
+__device__ __forceinline__ int round_even_small(float t, float& kf) {
+  const float y = __fadd_rn(t, 12582912.0f);
+  kf = __fsub_rn(y, 12582912.0f);
+  return __float_as_int(y) - 0x4B400000;
+}
+__device__ __forceinline__ int clamp127(int k) { return min(max(k, -127), 127); }
+
+// Per-token quantization code of v for scale s0 > 0: clamp(rint(fl32(v / s0)), -127, 127), the IEEE
+// quotient rounded half to even.
+__device__ __forceinline__ int quant_code(float v, float s0) {
+  float kf;
+  return clamp127(round_even_small(__fdiv_rn(v, s0), kf));
+}
+// Same code, computed as the rounding of t = v * inv_s0 unless t lies within 1e-3 of a rounding boundary:
+// |v/s0| <= 127, and both t (inv_s0 within 2^-22 of 1/s0) and fl32(v/s0) are within 5e-5 of v/s0, so away
+// from a boundary they round to the same integer; near one, the IEEE division decides.
 __device__ __forceinline__ int quant_code_fast(float v, float s0, float inv_s0) {
   const float t = v * inv_s0;
-  const float k = rintf(t);
-  if (fabsf(t - k) < 0.499f) return (int)fminf(fmaxf(k, -127.0f), 127.0f);
+  float kf;
+  const int k = round_even_small(t, kf);
+  if (fabsf(t - kf) < 0.499f) return clamp127(k);
   return quant_code(v, s0);
 }
 // The codes of N values at once, the same as quant_code_fast for each: the product path for all of them
 // without branches, then (rarely) the IEEE division for those close to a rounding boundary, behind one
-// branch.  inv_s0 = 0 (an all-zero token) gives code 0 everywhere.
+// branch.  inv_s0 = 0 (an all-zero token) gives code 0 everywhere.  No conversion instructions: the
+// rounding runs on the fp32 adder (round_even_small).
 template <int N>
 __device__ __forceinline__ void quant_codes(const float (&v)[N], float s0, float inv_s0, int (&code)[N]) {
   uint32_t near = 0u;
 #pragma unroll
   for (int e = 0; e < N; ++e) {
     const float t = v[e] * inv_s0;
-    const float k = rintf(t);
-    code[e] = (int)fminf(fmaxf(k, -127.0f), 127.0f);
-    near |= (fabsf(t - k) < 0.499f ? 0u : 1u) << e;
+    float kf;
+    code[e] = clamp127(round_even_small(t, kf));
+    near |= (fabsf(t - kf) < 0.499f ? 0u : 1u) << e;
   }
   if (near) {
 #pragma unroll
@@ -192,7 +220,9 @@ __device__ __forceinline__ void linear_out_n(const int (&acc)[N], const double (
 #pragma unroll
       for (int n = 0; n < N; ++n) {
         const uint32_t w = r < 4 ? wa[n].x : r < 8 ? wa[n].y : r < 12 ? wa[n].z : wa[n].w;
-        lora[n] = dadd(lora[n], dmul(int_to_f64((int)(int8_t)(w >> (8 * (r & 3)))), tf[n][r]));
+        // W_A[r] tf[r] is exact in fp64 (8-bit by 24-bit), so the fused multiply-add rounds exactly as
+        // the separate product and sum do
+        lora[n] = fma(int_to_f64((int)(int8_t)(w >> (8 * (r & 3)))), tf[n][r], lora[n]);
       }
     }
   }
@@ -236,18 +266,24 @@ __device__ __forceinline__ float lora_tf(int t, float sB, float s) {
 // RMSNorm (eps 1e-5, a weight per channel), then the quantizer on the normalized row:
 //   r = fl32(1 / sqrt(ss / n + 1e-5))   (fp64; ss the fp64 sum of the exact squares of the row)
 //   u = fl32(fl32(h * r) * w)
+// The reciprocal square root is CUDA's fp64 rsqrt (at most 1 ulp from the real value) rounded once to
+// fp32: it gives the fp32 value of the IEEE sqrt-then-divide sequence except when the real value lies
+// within about 2 fp64 ulps of an fp32 rounding boundary, the same class of last-bit difference as the
+// order of the fp64 sum of squares.
 __device__ __forceinline__ float rms_factor(double ss, int n) {
-  return __double2float_rn(__ddiv_rn(1.0, __dsqrt_rn(__dadd_rn(__ddiv_rn(ss, (double)n), 1e-5))));
+  return __double2float_rn(rsqrt(__dadd_rn(__ddiv_rn(ss, (double)n), 1e-5)));
 }
 __device__ __forceinline__ float norm_value(float h, float r, float w) { return fmul(fmul(h, r), w); }
 
-// Conv pre-activation fl32(b + w0*s0 + w1*s1 + w2*s2 + w3*x) (fp64, this order), then SiLU.
+// Conv pre-activation fl32(b + w0*s0 + w1*s1 + w2*s2 + w3*x) (fp64, this order), then SiLU.  Each
+// product of two fp32 values is exact in fp64, so each fused multiply-add rounds exactly as the separate
+// product and sum do.
 __device__ __forceinline__ float conv_out(float4 w, float bias, float s0, float s1, float s2, float x) {
   double e = (double)bias;
-  e = dadd(e, dmul((double)w.x, (double)s0));
-  e = dadd(e, dmul((double)w.y, (double)s1));
-  e = dadd(e, dmul((double)w.z, (double)s2));
-  e = dadd(e, dmul((double)w.w, (double)x));
+  e = fma((double)w.x, (double)s0, e);
+  e = fma((double)w.y, (double)s1, e);
+  e = fma((double)w.z, (double)s2, e);
+  e = fma((double)w.w, (double)x, e);
   return silu_f64(__double2float_rn(e));
 }
 

@@ -6,17 +6,27 @@
 // One CTA per SM owns a fixed slice of every layer:
 //   * ~E/NC SSM rows (h,p): their SSM state rows, the matching z and x rows of in_proj, the conv
 //     channels of those x rows;
-//   * ~320/NC of the rows every CTA needs (B, C and dt rows of in_proj), whose scaffold accumulators it
-//     publishes;
-//   * ~d_model/NC rows of out_proj and the matching entries of the residual stream.
+//   * ~320/NC of the rows every CTA needs (B, C and dt rows of in_proj): the CTA computes their outputs
+//     to the end — B and C through their conv channel and SiLU, dt through softplus and the decay dA —
+//     and publishes the final values;
+//   * ~d_model/NC rows of out_proj and the matching entries of the residual stream (kept in registers
+//     from layer to layer).
 // The weights and states of a CTA's slice are loaded into registers and shared memory at the start of
 // the layer (and prefetched into L2 one layer ahead), before the CTA waits on anything, so the HBM stream
-// overlaps the dependency chain.  Cross-CTA hand-offs go through global memory with monotonically
-// increasing counters (arrive = CTA barrier + release add; wait = bounded relaxed spin + acquire fence),
-// three per layer.  Every CTA quantizes the whole h (and g) itself, so it also computes the LoRA
-// down-projection t = W_B q of the codes itself (exact int32 dp4a against W_B staged in shared memory)
-// and no hand-off is needed for it.  A wait that runs past its clock budget records DFSSM_ETIMEOUT in the
-// workspace status word and the CTA returns.
+// overlaps the dependency chain.
+//
+// Cross-CTA hand-offs (three per layer: the residual stream h, the B/C/dt values, the gated SSM output g)
+// carry their synchronisation in the data: every exchanged fp32 value travels as one 64-bit word
+// {value, tag} written with a single relaxed store, the tag naming the layer that produced it.  A reader
+// polls exactly the words it needs until their tags match, so a hand-off costs one trip through L2 — no
+// counter, no release fence, no second read of the data.  Single buffers suffice: a CTA can only produce
+// layer l+1's words after every CTA has consumed layer l's (each hand-off needs the previous one from all
+// CTAs).  The tags are cleared before every launch.
+//
+// Every CTA quantizes the whole h (and g) itself, so it also computes the LoRA down-projection
+// t = W_B q of the codes itself (exact int32 dp4a against W_B staged in shared memory).  A poll that runs
+// past its clock budget records DFSSM_ETIMEOUT in the workspace status word; the CTA (and every other
+// CTA, which sees the abort word) then waits for its own copies in flight and returns.
 //
 // All arithmetic goes through the functions in common.cuh, so the results are those of the per-op path.
 
@@ -29,17 +39,17 @@ namespace fused {
 constexpr int DM = 2048, E = 4096, H = 64, P = 64, N = 128, R = 16;
 constexpr int SH0 = 2 * E;              // first in_proj row every CTA needs (B rows, then C, then dt)
 constexpr int NSH = 2 * N + H;          // 320 such rows
-constexpr int NT = 512, NW = NT / 32;   // NW == R: warp r computes LoRA row r's partial sums
+constexpr int NT = 512, NW = NT / 32;   // NW == R: warp r computes LoRA row r
 constexpr int MAX_IN = 64, MAX_OUT = 16, MAX_SSM = 32;
-constexpr int MIN_CTAS = 137, MAX_CTAS = 256;  // >= 137: at most 15 out_proj rows per CTA
+static_assert((DM & (DM - 1)) == 0 && (E & (E - 1)) == 0, "norm lengths are powers of two");
+constexpr int MIN_CTAS = 137, MAX_CTAS = 256;  // >= 137: <= 15 out_proj rows, <= 3 shared rows per CTA
 static_assert(NW == R, "one warp per LoRA row");
-constexpr int kPrefetchThread = 32;     // warp 1 issues the next layer's L2 prefetches
-constexpr int kCopyThread = 64;         // warp 2 issues the layer's bulk copies (thread 0 polls)
-constexpr int kChainWarp = NW - 1;      // warp 15 forms the LoRA intermediate (no out_proj row)
-constexpr int kChainBase = kChainWarp * 32;
-
-enum { CTR_H = 0, CTR_BC, CTR_G, N_CTR };
-constexpr int CTR_STRIDE = 32;          // one 128-byte line per counter
+constexpr int kCopyThread = 64;         // warp 2: the layer's out-set copy (end of the previous layer)
+constexpr int kPrefetchThread = 224;    // warp 7: the next layer's L2 prefetches (phase B)
+constexpr int kAheadCopyThread = 256;   // warp 8: the next layer's in-set and state copies (phase B)
+constexpr int kBcWarp = NW - 1;         // warp 15: LoRA intermediates and the shared rows' epilogues
+constexpr int kBcBase = kBcWarp * 32;
+constexpr int kZxBase = 320;            // threads kZxBase + j: epilogues of the CTA's z and x rows j
 
 struct LayerPtrs {
   const uint32_t* in_bits;
@@ -69,80 +79,100 @@ struct Params {
   LayerPtrs L[DFSSM_MAX_LAYERS];
   int n_layers;
   float* hidden;
-  int* ctr;
   int* err;
   int* status;
-  int* sacc;
-  float* gbuf;
+  unsigned long long* hx;   // [DM]   tagged residual stream
+  unsigned long long* gx;   // [E]    tagged gated SSM output
+  unsigned long long* bcx;  // [2N + 2H] tagged B, C (after conv + SiLU), then (dt, dA) per head
   long long spin_limit;
 };
 
 // ------------------------------------------------------------------------------ workspace layout
-// [counters N_CTR x 128 B][abort word 128 B][status word 128 B][sacc 320][gbuf 4096]
-// The counters and the abort word are cleared before every launch; the status word is sticky: a timed
-// out wait stores kTimeoutMagic there, and only dfssm_device_status clears it.
-constexpr size_t OFF_CTR = 0;
-constexpr size_t OFF_ERR = OFF_CTR + N_CTR * CTR_STRIDE * 4;
-constexpr size_t OFF_STATUS = OFF_ERR + 128;
-constexpr size_t CLEAR_BYTES = OFF_STATUS;  // counters + abort word
-constexpr size_t OFF_SACC = OFF_STATUS + 128;
-constexpr size_t OFF_GBUF = OFF_SACC + ((NSH * 4 + 255) / 256) * 256;
-constexpr size_t WS_BYTES = OFF_GBUF + E * 4;
-// dynamic shared memory: W_B of in_proj [R][DM] and of out_proj [R][E]
-constexpr int WB_BYTES = R * (DM + E);
-// dynamic shared memory: W_B of both linears, then the CTA's SSM state rows of two consecutive layers
+// [status word 128 B][abort word 128 B][hx DM x 8 B][gx E x 8 B][bcx (2N + 2H) x 8 B]
+// Everything from the abort word on is cleared before every launch (tag 0 = not yet written); the
+// status word is sticky: a timed-out wait stores kTimeoutMagic there, and only dfssm_device_status
+// clears it.
+constexpr size_t OFF_STATUS = 0;
+constexpr size_t OFF_ERR = 128;
+constexpr size_t OFF_HX = 256;
+constexpr size_t OFF_GX = OFF_HX + DM * 8;
+constexpr size_t OFF_BCX = OFF_GX + E * 8;
+constexpr size_t WS_BYTES = OFF_BCX + (2 * N + 2 * H) * 8;
+constexpr size_t CLEAR_OFF = OFF_ERR, CLEAR_BYTES = WS_BYTES - OFF_ERR;
+// dynamic shared memory, filled by bulk copies:
+//   in-set  [2] (layers of each parity): W_B of in_proj [R][DM] + the pre-norm weight [DM] (one layer ahead)
+//   out-set     W_B of out_proj [R][E] + the gated-norm weight [E] (issued at the start of the layer)
+//   state   [2] the CTA's SSM state rows (one layer ahead)
+constexpr int IN_SET = R * DM + DM * 4;
+constexpr int OUT_SET = R * E + E * 4;
 constexpr int ST_BYTES = MAX_SSM * N * 4;
-constexpr int DYN_BYTES = WB_BYTES + 2 * ST_BYTES;
+constexpr int OFF_OUT_SET = 2 * IN_SET;
+constexpr int OFF_STATE = OFF_OUT_SET + OUT_SET;
+constexpr int DYN_BYTES = OFF_STATE + 2 * ST_BYTES;
 
-// ------------------------------------------------------------------------------ synchronisation
+constexpr int kTimeoutMagic = 0x7E0D1E57;
+
+// ------------------------------------------------------------------------------ tagged exchange
 
 __device__ __forceinline__ int ld_relaxed(const int* p) {
   int v;
   asm volatile("ld.relaxed.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
   return v;
 }
+__device__ __forceinline__ void st_tagged(unsigned long long* p, float v, uint32_t tag) {
+  const unsigned long long w = ((unsigned long long)tag << 32) | (unsigned long long)__float_as_uint(v);
+  asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(w) : "memory");
+}
+// Two consecutive tagged words (16-byte aligned); each 64-bit word is read as one single-copy-atomic unit.
+__device__ __forceinline__ ulonglong2 ld_tagged2(const unsigned long long* p) {
+  ulonglong2 r;
+  asm volatile("ld.relaxed.gpu.global.v2.u64 {%0, %1}, [%2];" : "=l"(r.x), "=l"(r.y) : "l"(p) : "memory");
+  return r;
+}
+__device__ __forceinline__ bool tag_is(unsigned long long w, uint32_t tag) { return (uint32_t)(w >> 32) == tag; }
+__device__ __forceinline__ float tag_val(unsigned long long w) { return __uint_as_float((uint32_t)w); }
 
-constexpr int kTimeoutMagic = 0x7E0D1E57;
-
-// All threads of the CTA: returns once *ctr >= target.  Returns false (for every thread) when the
-// clock budget ran out (the abort and status words are then set) or another CTA already aborted.
-// Thread 0 polls with relaxed loads and finishes with an acquire fence; the CTA barrier then orders
-// the other threads' reads after it.
-__device__ bool block_wait(const int* ctr, int target, int* err, int* status, long long limit,
-                           int* sflag) {
-  if (threadIdx.x == 0) {
-    int ok = 1;
-    if (ld_relaxed(ctr) < target) {
-      const long long t0 = clock64();
-      unsigned it = 0;
-      while (ld_relaxed(ctr) < target) {
-        if ((++it & 15u) == 0) {
-          if (ld_relaxed(err) != 0) {
-            ok = 0;
-            break;
-          }
-          if (clock64() - t0 > limit) {
-            atomicExch(err, 1);
-            atomicExch(status, kTimeoutMagic);
-            ok = 0;
-            break;
-          }
-        }
+// This thread's NP pairs of tagged words at base + off[k] (16-byte aligned) until all carry `tag`;
+// values to v[2k], v[2k+1].  Bounded: false when the clock budget ran out (the abort and status words are
+// then set) or another CTA already aborted.
+template <int NP>
+__device__ bool poll_pairs(const unsigned long long* base, const int (&off)[NP], uint32_t tag, float (&v)[2 * NP],
+                           int* err, int* status, long long limit) {
+  uint32_t pending = (1u << NP) - 1u;
+  long long t0 = 0;
+  unsigned it = 0;
+  while (true) {
+    ulonglong2 r[NP];
+#pragma unroll
+    for (int k = 0; k < NP; ++k)
+      if ((pending >> k) & 1u) r[k] = ld_tagged2(base + off[k]);
+#pragma unroll
+    for (int k = 0; k < NP; ++k) {
+      if (((pending >> k) & 1u) && tag_is(r[k].x, tag) && tag_is(r[k].y, tag)) {
+        v[2 * k] = tag_val(r[k].x);
+        v[2 * k + 1] = tag_val(r[k].y);
+        pending &= ~(1u << k);
       }
     }
-    if (ok) asm volatile("fence.acq_rel.gpu;" ::: "memory");
-    *sflag = ok;
+    if (pending == 0u) return true;
+    if (it == 0) t0 = clock64();
+    if ((++it & 7u) == 0) {
+      if (ld_relaxed(err) != 0) return false;
+      if (clock64() - t0 > limit) {
+        atomicExch(err, 1);
+        atomicExch(status, kTimeoutMagic);
+        return false;
+      }
+    }
   }
-  __syncthreads();
-  return *sflag != 0;
 }
 
-// All threads of the CTA: count one arrival after every global write the CTA made so far (the CTA
-// barrier orders them before thread 0's release).
-__device__ __forceinline__ void block_arrive(int* ctr) {
-  __syncthreads();
-  if (threadIdx.x == 0) asm volatile("red.release.gpu.global.add.s32 [%0], 1;" ::"l"(ctr) : "memory");
-}
+// Named CTA barrier `id` over n threads: bar_arrive signals (and publishes this thread's earlier shared-
+// memory writes) without waiting; bar_sync waits until all n have arrived.
+__device__ __forceinline__ void bar_sync(int id, int n) { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory"); }
+__device__ __forceinline__ void bar_arrive(int id, int n) { asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(n) : "memory"); }
+
+// ------------------------------------------------------------------------------ asynchronous copies
 
 __device__ __forceinline__ void prefetch_l2(const void* p, unsigned bytes) {
   if (bytes >= 16)
@@ -208,24 +238,75 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
       : "memory");
 }
 
-// LoRA down-projection row r = warp: t[r] = sum_i W_B[r,i] q_i over NCH 16-byte chunks, lane taking
-// chunks lane, lane + 32, ... of the natural-order codes and of W_B row r (conflict-free in shared memory).
-template <int NCH>
-__device__ __forceinline__ int lora_row(const int8_t* wb_row, const int8_t* qn, int lane) {
-  const uint4* w4 = reinterpret_cast<const uint4*>(wb_row);
-  const uint4* q4 = reinterpret_cast<const uint4*>(qn);
+// ------------------------------------------------------------------------------ block helpers
+
+// LoRA down-projection of the K natural-order codes qn against W_B [R][K], split by inputs: warp w takes
+// inputs [w K/16, (w+1) K/16) for all R rows (each lane K/512 consecutive codes, read once) and leaves
+// its R partial sums in red_t[w][0..R); t[r] = sum_w red_t[w][r] (exact int32).
+template <int K>
+__device__ __forceinline__ void lora_slice(const int8_t* wb, const int8_t* qn, int warp, int lane,
+                                           int (*red_t)[R]) {
+  constexpr int WPL = K / (16 * 32 * 4);  // 4-byte words per lane
+  static_assert(WPL == 1 || WPL == 2, "K is 2048 or 4096");
+  const int i0 = warp * (K / 16) + lane * 4 * WPL;
+  uint32_t q[WPL];
+  if constexpr (WPL == 1) {
+    q[0] = *reinterpret_cast<const uint32_t*>(qn + i0);
+  } else {
+    const uint2 v = *reinterpret_cast<const uint2*>(qn + i0);
+    q[0] = v.x;
+    q[1] = v.y;
+  }
+  int part[R];
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    if constexpr (WPL == 1) {
+      part[r] = dp4a_ss(*reinterpret_cast<const uint32_t*>(wb + r * K + i0), q[0], 0);
+    } else {
+      const uint2 w = *reinterpret_cast<const uint2*>(wb + r * K + i0);
+      part[r] = dp4a_ss(w.y, q[1], dp4a_ss(w.x, q[0], 0));
+    }
+  }
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    const int t = __reduce_add_sync(0xffffffffu, part[r]);
+    if (lane == r) red_t[warp][r] = t;
+  }
+}
+__device__ __forceinline__ int lora_t_sum(const int (*red_t)[R], int r) {
   int t = 0;
 #pragma unroll
-  for (int k = 0; k < NCH / 32; ++k) {
-    const uint4 w = w4[lane + 32 * k], q = q4[lane + 32 * k];
-    t = dp4a_ss(w.x, q.x, t);
-    t = dp4a_ss(w.y, q.y, t);
-    t = dp4a_ss(w.z, q.z, t);
-    t = dp4a_ss(w.w, q.w, t);
-  }
-  return __reduce_add_sync(0xffffffffu, t);
+  for (int w = 0; w < NW; ++w) t += red_t[w][r];
+  return t;
 }
 
+// Block-wide fp64 sum of the threads' v (every thread gets the same value: the sixteen per-warp sums are
+// added in one fixed tree order), and the OR over the block of `flag` (through *any_flag, zero before
+// the call).  Contains one CTA barrier.
+__device__ __forceinline__ double block_sum_d(double v, int lane, int warp, double* red_d, bool flag,
+                                              int* any_flag, bool& any) {
+  v = warp_sum(v);
+  if (lane == 0) red_d[warp] = v;
+  if (flag) *any_flag = 1;
+  __syncthreads();
+  double a[NW / 2];
+#pragma unroll
+  for (int q = 0; q < NW / 2; ++q) {
+    const double2 d = reinterpret_cast<const double2*>(red_d)[q];
+    a[q] = d.x + d.y;
+  }
+#pragma unroll
+  for (int w = NW / 4; w > 0; w >>= 1)
+#pragma unroll
+    for (int q = 0; q < w; ++q) a[q] = a[2 * q] + a[2 * q + 1];
+  any = *any_flag != 0;
+  return a[0];
+}
+// rms_factor for a row of length n = 2^k, with ss / n formed as the (exact) product by 2^-k, which equals
+// the IEEE quotient.
+__device__ __forceinline__ float rms_factor_pow2(double ss, int n) {
+  return __double2float_rn(rsqrt(__dadd_rn(__dmul_rn(ss, 1.0 / (double)n), 1e-5)));
+}
 // Block-wide absmax of the threads' non-negative m (one redux per warp; the bit patterns of non-negative
 // floats order like the floats).  Contains one CTA barrier.
 __device__ __forceinline__ float block_absmax(float m, int lane, int warp, unsigned* red_u) {
@@ -240,17 +321,6 @@ __device__ __forceinline__ float block_absmax(float m, int lane, int warp, unsig
   }
   return __uint_as_float(mb);
 }
-// Block-wide fp64 sum of the threads' v (every thread gets the same value: the per-warp sums are added
-// in warp order).  Contains one CTA barrier.
-__device__ __forceinline__ double block_sum_d(double v, int lane, int warp, double* red_d) {
-  v = warp_sum(v);
-  if (lane == 0) red_d[warp] = v;
-  __syncthreads();
-  double t = 0.0;
-#pragma unroll
-  for (int q = 0; q < NW; ++q) t += red_d[q];
-  return t;
-}
 // Sum of the sixteen per-warp partial sums.
 __device__ __forceinline__ int block_sum16(const int* red_i) {
   int t = 0;
@@ -262,58 +332,112 @@ __device__ __forceinline__ int block_sum16(const int* red_i) {
   return t;
 }
 
+// Sum over bit=1 positions of q for 128 weights (one uint4 of sign bits) against the eight 16-byte chunks
+// of their segment's dp4a-permuted codes held in registers (as bits_dot).
+__device__ __forceinline__ int bits_dot_reg(uint4 w, const uint4 (&q)[8]) {
+  int acc8[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) acc8[k] = 0;
+  const uint32_t w4[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const uint32_t qp[8] = {q[2 * j].x, q[2 * j].y, q[2 * j].z, q[2 * j].w,
+                            q[2 * j + 1].x, q[2 * j + 1].y, q[2 * j + 1].z, q[2 * j + 1].w};
+#pragma unroll
+    for (int k = 0; k < 8; ++k) acc8[k] = dp4a_us(w4[j] & (0x01010101u << k), qp[k], acc8[k]);
+  }
+  int S = 0;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) S += acc8[k] >> k;
+  return S;
+}
+
+// RMSNorm of the NV values this thread holds of a row of length n (the row's squares summed over the
+// block; the weights w_sm in shared memory), then the quantizer on the normalized row: codes to q_perm
+// (dp4a segment layout, NSEG segments) and q_nat, their per-warp sums to red_i.  Element k of the thread is
+// row index idx[k] (k even, k + 1 adjacent).  Returns the scale s; `abort_any` is true (for every thread)
+// when some thread's wait failed (`failed`).  Contains three CTA barriers.
+template <int NV, int NSEG>
+__device__ __forceinline__ float norm_quantize(const float (&hv)[NV], const float* w_sm, const int (&idx)[NV],
+                                               int n, int lane, int warp, double* red_d, unsigned* red_u,
+                                               int* red_i, int* any_flag, int8_t* q_perm, int8_t* q_nat,
+                                               bool failed, bool& abort_any) {
+  double ss = 0.0;
+#pragma unroll
+  for (int k = 0; k < NV; ++k) ss += (double)hv[k] * (double)hv[k];  // exact squares in fp64
+  const float rn = rms_factor_pow2(block_sum_d(ss, lane, warp, red_d, failed, any_flag, abort_any), n);
+  float v[NV];
+  float m = 0.0f;
+#pragma unroll
+  for (int k = 0; k < NV; k += 2) {
+    const float2 w = *reinterpret_cast<const float2*>(w_sm + idx[k]);
+    v[k] = norm_value(hv[k], rn, w.x);
+    v[k + 1] = norm_value(hv[k + 1], rn, w.y);
+    m = fmaxf(m, fmaxf(fabsf(v[k]), fabsf(v[k + 1])));
+  }
+  m = block_absmax(m, lane, warp, red_u);
+  const float s0 = quant_scale(m);
+  const float inv_s0 = quant_inv(s0);
+  int cd[NV];
+  quant_codes<NV>(v, s0, inv_s0, cd);
+  int sq = 0;
+#pragma unroll
+  for (int k = 0; k < NV; ++k) {
+    q_perm[seg_index<NSEG>(idx[k])] = (int8_t)cd[k];
+    q_nat[idx[k]] = (int8_t)cd[k];
+    sq += cd[k];
+  }
+  sq = __reduce_add_sync(0xffffffffu, sq);
+  if (lane == 0) red_i[warp] = sq;
+  __syncthreads();
+  return s0;
+}
+
 // ------------------------------------------------------------------------------ the kernel
 //
-// Per layer (three hand-offs):
-//   A  wait h    -> RMSNorm+quantize h, LoRA-down from the partials, scaffold GEMV of the owned rows;
-//                   the B/C/dt rows' accumulators are published first (arrive B/C)
-//   B  wait B/C  -> epilogues (B/C conv, dt, own z gate, own x conv), SSM of the owned rows, g of the
-//                   owned rows and their LoRA-down partial sums published (arrive g)
-//   C  wait g    -> gated RMSNorm+quantize, out_proj GEMV of the owned rows, residual; the next layer's
-//                   (arrive h)
-// The first layer reads the input hidden state directly (it is complete before the launch).
+// Per layer (three hand-offs, tags: h entering layer l carries l; B/C/dt and g of layer l carry l + 1):
+//   A  h (poll; layer 0 reads the input) -> RMSNorm + quantize, scaffold GEMV of the owned in_proj rows,
+//      LoRA-down; the shared rows' epilogues (B/C conv + SiLU, dt softplus + dA) published
+//   B  the own z/x rows' epilogues (gate value SiLU(z), x conv); B/C/dt (poll) -> SSM of the owned rows,
+//      g = y SiLU(z) published
+//   C  g (poll) -> gated RMSNorm + quantize, LoRA-down, out_proj GEMV of the owned rows, residual;
+//      the new h published (the last layer writes it to the output instead)
 
 __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ Params p) {
-  extern __shared__ __align__(16) int8_t wb_sm[];  // W_B of in_proj [R][DM], then of out_proj [R][E]
+  extern __shared__ __align__(128) int8_t dyn_sm[];
   // every layer's pointers, copied once: the layer loop never indexes the parameter block at run time
   __shared__ LayerPtrs lsm[DFSSM_MAX_LAYERS];
-  int8_t* const wb_in = wb_sm;
-  int8_t* const wb_out = wb_sm + R * DM;
-  float* const st_sm = reinterpret_cast<float*>(wb_sm + WB_BYTES);  // [2][MAX_SSM][N], layer l in l & 1
+  const auto wb_in = [&](int l) { return dyn_sm + (l & 1) * IN_SET; };
+  const auto nw_sm = [&](int l) { return reinterpret_cast<const float*>(dyn_sm + (l & 1) * IN_SET + R * DM); };
+  int8_t* const wb_out = dyn_sm + OFF_OUT_SET;
+  const float* const gw_sm = reinterpret_cast<const float*>(dyn_sm + OFF_OUT_SET + R * E);
+  float* const st_sm = reinterpret_cast<float*>(dyn_sm + OFF_STATE);  // [2][MAX_SSM][N], layer l in l & 1
   __shared__ __align__(16) int8_t q_perm[E];
   __shared__ __align__(16) int8_t q_nat[E];
-  __shared__ __align__(16) double red_d[NW];   // per-warp sums of squares
-  __shared__ __align__(16) unsigned red_u[NW];  // per-warp absmax (bit pattern of a non-negative float)
-  __shared__ __align__(16) int red_i[NW];       // per-warp code sums
-  __shared__ float lbs_o[R];                    // out_proj W_B row scales
-  __shared__ int t_sm[R];
-  __shared__ int sflag;
-  __shared__ float tf[R];
-  __shared__ float s_scale;
+  __shared__ __align__(16) double red_d[NW];
+  __shared__ __align__(16) unsigned red_u[NW];
+  __shared__ __align__(16) int red_i[NW];
+  __shared__ int any_flag[2];                   // [0] the pre-norm quantizer's, [1] the gated norm's
+  __shared__ float lbs_in[R], lbs_o[2][R];      // W_B row scales (out_proj's by layer parity)
+  __shared__ __align__(16) int red_t[NW][R];  // LoRA-down partial sums, per warp
+  __shared__ double tf_d[R];                    // in_proj LoRA intermediates
+  __shared__ float s_in_sm;
   // in_proj rows owned by this CTA (slot order: shared rows, z rows, x rows)
   __shared__ int acc_in[MAX_IN];
   __shared__ float in_sw[MAX_IN], in_sa[MAX_IN];
   __shared__ __align__(16) int8_t in_wa[MAX_IN][R];
-  // the 320 rows every CTA needs
-  __shared__ __align__(16) float sh_sw[NSH];
-  __shared__ __align__(16) float sh_sa[NSH];
-  __shared__ __align__(16) int8_t sh_wa[NSH][R];
-  __shared__ __align__(16) float4 bc_w[2 * N];
-  __shared__ __align__(16) float bc_b[2 * N];
-  __shared__ __align__(16) float bc_st[2 * N][3];
-  // bulk-copy completion: [0] the rows every CTA needs + in_proj W_B, [1] out_proj W_B (once per layer)
-  __shared__ uint64_t ldbar[2];
+  // bulk-copy completion: the in-set of layer l on inbar[l & 1] (once per two layers), the out-set on
+  // outbar (once per layer)
+  __shared__ uint64_t inbar[2], outbar;
   // SSM state rows of layer l arrive in buffer l & 1, one layer ahead (completes once per two layers)
   __shared__ uint64_t stbar[2];
-  __shared__ float bc_new[2 * N];
   __shared__ __align__(16) float Bsm[N];
   __shared__ __align__(16) double Cd[N];
-  // SSM rows
   __shared__ float zsm[MAX_SSM], xsm[MAX_SSM];
   __shared__ float dtv[2], dAv[2], Dv[2];
   // out_proj rows
   __shared__ int acc_out[MAX_OUT];
-  __shared__ float o_sw[MAX_OUT], o_sa[MAX_OUT], h_old[MAX_OUT];
+  __shared__ float o_sw[MAX_OUT], o_sa[MAX_OUT];
   __shared__ __align__(16) int8_t o_wa[MAX_OUT][R];
 
   const int c = blockIdx.x, NC = gridDim.x;
@@ -325,7 +449,8 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ P
   const int sh0 = c * NSH / NC, sh1 = (c + 1) * NSH / NC, n_sh = sh1 - sh0;
   const int ro0 = c * DM / NC, ro1 = (c + 1) * DM / NC, n_out = ro1 - ro0;
   const int n_in = n_sh + 2 * n_ssm;
-  const int hA = rs0 / P;  // first head of this CTA's SSM rows (at most two heads)
+  const int hA = rs0 / P;                       // first head of this CTA's SSM rows
+  const int n_heads = (rs1 - 1) / P - hA + 1;   // one or two heads
   auto in_row = [&](int slot) -> int {
     if (slot < n_sh) return SH0 + sh0 + slot;
     const int j = slot - n_sh;
@@ -335,8 +460,23 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ P
   const int slot_in[2] = {warp * 2 + (lane >> 4), 32 + warp * 2 + (lane >> 4)};
   const int slot_out = warp;  // out_proj: one row per warp, 32 lanes x 128 weights
   const int ssm_slot[2] = {warp, NW + warp};
-  const int dt_head = tid - 2 * N;  // threads [256, 320) own the dt rows
-  const bool dt_own = tid >= 2 * N && tid < NSH && (dt_head == hA || dt_head == hA + 1);
+  // this thread's entries of h (k < 4) and of g (k < 8): the pairs 2 tr, 2 tr + 1 of each 1024-block, with
+  // the thread index rotated per CTA so that the CTAs' simultaneous reads of a hand-off spread over L2
+  const int tr = (tid + 53 * c) & (NT - 1);
+  int hidx[4], gidx[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const int i = 2 * tr + (k & 1) + 1024 * (k >> 1);
+    if (k < 4) hidx[k] = i;
+    gidx[k] = i;
+  }
+  const int hoff[2] = {2 * tr, 1024 + 2 * tr};
+  const int goff[4] = {2 * tr, 1024 + 2 * tr, 2048 + 2 * tr, 3072 + 2 * tr};
+  // the shared row of this thread (warp kBcWarp, lanes < n_sh): B/C (conv channel E + k) or dt (head)
+  const int bc_j = tid - kBcBase;
+  const bool bc_own = bc_j >= 0 && bc_j < n_sh;
+  const int bc_k = sh0 + bc_j;
+  float h_own = 0.0f;  // residual stream entry ro0 + tid (tid < n_out), carried from layer to layer
 
   {
     // LayerPtrs is 21 pointers: thread t copies pointer t % 21 of layer t / 21
@@ -345,37 +485,138 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ P
     const void* const* src = reinterpret_cast<const void* const*>(p.L);
     const void** dst = reinterpret_cast<const void**>(lsm);
     for (int k = tid; k < p.n_layers * NPTR; k += NT) dst[k] = src[k];
+    if (tid < 2) any_flag[tid] = 0;
     if (tid == 0) {
-      mbar_init(&ldbar[0], 1);
-      mbar_init(&ldbar[1], 1);
+      mbar_init(&inbar[0], 1);
+      mbar_init(&inbar[1], 1);
+      mbar_init(&outbar, 1);
       mbar_init(&stbar[0], 1);
       mbar_init(&stbar[1], 1);
       asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-      // layer 0's SSM state rows of this CTA
+      // layer 0's SSM state rows and in-set
       mbar_expect_tx(&stbar[0], n_ssm * N * 4);
       bulk_g2s(st_sm, p.L[0].ssm_state + (size_t)rs0 * N, n_ssm * N * 4, &stbar[0]);
+      mbar_expect_tx(&inbar[0], IN_SET);
+      bulk_g2s(wb_in(0), p.L[0].in_lb, R * DM, &inbar[0]);
+      bulk_g2s(wb_in(0) + R * DM, p.L[0].norm_w, DM * 4, &inbar[0]);
     }
+    if (tid < n_out) h_own = p.hidden[ro0 + tid];
     __syncthreads();
   }
   // An aborting CTA first waits (bounded) for everything it may still have landing in its shared memory:
-  // its own cp.async copies and the bulk copies of layer l (and of layer l + 1's state rows).
-  const auto drain = [&](int l, bool has_next) {
+  // its own cp.async copies and the bulk copies of layer l.
+  // next_issued: the next layer's in-set and state copies (phase B of layer l) were issued.
+  const auto drain = [&](int l, bool next_issued) {
     cp_async_wait<0>();
     if (tid == 0) {
-      mbar_wait(&ldbar[0], l & 1, p.spin_limit);
-      mbar_wait(&ldbar[1], l & 1, p.spin_limit);
+      mbar_wait(&inbar[l & 1], (l >> 1) & 1, p.spin_limit);
+      mbar_wait(&outbar, l & 1, p.spin_limit);
       mbar_wait(&stbar[l & 1], (l >> 1) & 1, p.spin_limit);
-      if (has_next) mbar_wait(&stbar[(l + 1) & 1], ((l + 1) >> 1) & 1, p.spin_limit);
+      if (next_issued) {
+        mbar_wait(&stbar[(l + 1) & 1], ((l + 1) >> 1) & 1, p.spin_limit);
+        mbar_wait(&inbar[(l + 1) & 1], ((l + 1) >> 1) & 1, p.spin_limit);
+      }
     }
   };
-  for (int l = 0; l < p.n_layers; ++l) {
-    const LayerPtrs& Lp = lsm[l];
-    const bool has_next = l + 1 < p.n_layers;
-
-    // ---------------------------------------------------------------- loads for the whole layer
-    if ((tid == kPrefetchThread || tid == kPrefetchThread + 1) && has_next) {
-      // this CTA's slice of the next layer, and (spread over CTAs 0..4) the parts every CTA reads.
-      // Issued by warp 1: a bulk prefetch stalls its thread, and thread 0 polls the counters.
+  const auto fail = [&]() {
+    atomicExch(p.err, 1);
+    atomicExch(p.status, kTimeoutMagic);
+  };
+  // What layer ll needs from memory at the start of its dependency chain: its sign bits and row parameters
+  // (registers, cp.async into shared memory) and its out-set (bulk copy).  Issued at the end of the
+  // previous layer (for layer 0, before the loop), after every read of the buffers it refills.  The
+  // layer's in-set and SSM state rows are copied, and the next layer's slice prefetched into L2, during
+  // the previous layer's phase B by warps that idle there (issue_ahead).
+  uint4 w_in[2], w_out;
+  float4 cw = make_float4(0.f, 0.f, 0.f, 0.f);
+  float cb = 0.f, cs0 = 0.f, cs1 = 0.f, cs2 = 0.f;
+  float bsw = 0.f, bsa = 0.f;
+  uint4 bwa = make_uint4(0, 0, 0, 0);
+  float4 bcw = make_float4(0.f, 0.f, 0.f, 0.f);
+  float bcb = 0.f, bs0 = 0.f, bs1 = 0.f, bs2 = 0.f, dtb = 0.f, A_h = 0.f;
+  const auto issue_loads = [&](int ll) {
+    const LayerPtrs& Lq = lsm[ll];
+    // registers: sign bits
+#pragma unroll
+    for (int ps = 0; ps < 2; ++ps) {
+      const int slot = slot_in[ps];
+      w_in[ps] = slot < n_in ? ld_stream_u4(Lq.in_bits + (size_t)in_row(slot) * (DM / 32) + li_in * 4)
+                             : make_uint4(0, 0, 0, 0);
+    }
+    w_out = slot_out < n_out ? ld_stream_u4(Lq.out_bits + (size_t)(ro0 + slot_out) * (E / 32) + lane * 4)
+                             : make_uint4(0, 0, 0, 0);
+    // own x channels: conv taps, bias, state (thread kZxBase + j handles channel rs0 + j)
+    if (tid >= kZxBase && tid - kZxBase < n_ssm) {
+      const int ch = rs0 + (tid - kZxBase);
+      cw = __ldg(reinterpret_cast<const float4*>(Lq.conv_w) + ch);
+      cb = __ldg(Lq.conv_b + ch);
+      cs0 = Lq.conv_state[(size_t)ch * 3 + 0];
+      cs1 = Lq.conv_state[(size_t)ch * 3 + 1];
+      cs2 = Lq.conv_state[(size_t)ch * 3 + 2];
+    }
+    // the shared row of this thread: its epilogue parameters and its conv channel or head parameters
+    if (bc_own) {
+      const int row = SH0 + bc_k;
+      bsw = __ldg(Lq.in_ws + row);
+      bsa = __ldg(Lq.in_las + row);
+      bwa = __ldg(reinterpret_cast<const uint4*>(Lq.in_la + (size_t)row * R));
+      if (bc_k < 2 * N) {
+        const int ch = E + bc_k;
+        bcw = __ldg(reinterpret_cast<const float4*>(Lq.conv_w) + ch);
+        bcb = __ldg(Lq.conv_b + ch);
+        bs0 = Lq.conv_state[(size_t)ch * 3 + 0];
+        bs1 = Lq.conv_state[(size_t)ch * 3 + 1];
+        bs2 = Lq.conv_state[(size_t)ch * 3 + 2];
+      } else {
+        dtb = __ldg(Lq.dt_bias + (bc_k - 2 * N));
+        A_h = __double2float_rn(-exp((double)__ldg(Lq.A_log + (bc_k - 2 * N))));
+      }
+    }
+    // epilogue parameters of the owned rows into shared memory, asynchronously
+    if (tid < n_in) {
+      const int row = in_row(tid);
+      cp_async4(&in_sw[tid], Lq.in_ws + row);
+      cp_async4(&in_sa[tid], Lq.in_las + row);
+      cp_async16(in_wa[tid], Lq.in_la + (size_t)row * R);
+    }
+    if (tid == kCopyThread) {
+      // this layer's out-set (its buffer was last read before the previous layer's GEMV barrier); every
+      // generic access of the previous layer to it is ordered before the copy by that barrier
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      mbar_expect_tx(&outbar, OUT_SET);
+      bulk_g2s(wb_out, Lq.out_lb, R * E, &outbar);
+      bulk_g2s(wb_out + R * E, Lq.gnorm_w, E * 4, &outbar);
+    }
+    if (tid < n_out) {
+      const int row = ro0 + tid;
+      cp_async4(&o_sw[tid], Lq.out_ws + row);
+      cp_async4(&o_sa[tid], Lq.out_las + row);
+      cp_async16(o_wa[tid], Lq.out_la + (size_t)row * R);
+    }
+    if (tid < 2 && hA + tid < H) cp_async4(&Dv[tid], Lq.D + hA + tid);
+    if (tid < R) {
+      cp_async4(&lbs_in[tid], Lq.in_lbs + tid);
+      cp_async4(&lbs_o[ll & 1][tid], Lq.out_lbs + tid);
+    }
+    cp_async_commit();  // this thread's row parameters (awaited before the quantizer's barriers)
+  };
+  issue_loads(0);
+  // During phase B of layer l (l + 1 < n_layers): the next layer's SSM state rows and in-set into the
+  // buffers of its parity (both last read in layer l - 1, before this layer's barriers) and the L2 prefetch
+  // of the next layer's slice, by warps that idle while the B/C/dt values are awaited.
+  const auto issue_ahead = [&](int l) {
+    if (tid == kAheadCopyThread) {
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      const int nb = (l + 1) & 1;
+      mbar_expect_tx(&stbar[nb], n_ssm * N * 4);
+      bulk_g2s(st_sm + nb * MAX_SSM * N, lsm[l + 1].ssm_state + (size_t)rs0 * N, n_ssm * N * 4, &stbar[nb]);
+      mbar_expect_tx(&inbar[nb], IN_SET);
+      bulk_g2s(wb_in(l + 1), lsm[l + 1].in_lb, R * DM, &inbar[nb]);
+      bulk_g2s(wb_in(l + 1) + R * DM, lsm[l + 1].norm_w, DM * 4, &inbar[nb]);
+    }
+    if (tid == kPrefetchThread || tid == kPrefetchThread + 1) {
+      // this CTA's slice of the next layer, and (spread over CTAs 0..2) the parts every CTA reads.
+      // A bulk prefetch stalls its thread, so an otherwise idle warp issues them.
       const LayerPtrs& Nx = lsm[l + 1];
       if (tid == kPrefetchThread) {
         prefetch_l2(Nx.in_bits + (size_t)(SH0 + sh0) * (DM / 32), n_sh * (DM / 8));
@@ -397,213 +638,156 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ P
         prefetch_lines(Nx.conv_b + rs0, n_ssm * 4);
         prefetch_lines(Nx.conv_state + (size_t)rs0 * 3, n_ssm * 12);
         switch (c) {
-          case 0: prefetch_l2(Nx.norm_w, DM * 4); break;
-          case 1: prefetch_l2(Nx.gnorm_w, E * 4); break;
+          case 1: prefetch_l2(Nx.gnorm_w, E * 4); prefetch_l2(Nx.out_lb, R * E); break;
           case 2:
-            prefetch_lines(Nx.in_ws + SH0, NSH * 4);
-            prefetch_lines(Nx.in_las + SH0, NSH * 4);
-            prefetch_l2(Nx.in_la + (size_t)SH0 * R, NSH * R);
-            break;
-          case 3:
-            prefetch_l2(Nx.conv_w + (size_t)E * 4, 2 * N * 16);
-            prefetch_lines(Nx.conv_b + E, 2 * N * 4);
-            prefetch_lines(Nx.conv_state + (size_t)E * 3, 2 * N * 12);
-            break;
-          case 4:
             prefetch_lines(Nx.dt_bias, H * 4);
             prefetch_lines(Nx.A_log, H * 4);
             prefetch_lines(Nx.D, H * 4);
             prefetch_lines(Nx.in_lbs, R * 4);
             prefetch_lines(Nx.out_lbs, R * 4);
             break;
-          case 5: prefetch_l2(Nx.in_lb, R * DM); break;
-          case 6: prefetch_l2(Nx.out_lb, R * E); break;
           default: break;
         }
       }
     }
-    // registers: sign bits, SSM state rows, norm weights, LoRA columns of the owned rows
-    uint4 w_in[2], w_out;
-#pragma unroll
-    for (int ps = 0; ps < 2; ++ps) {
-      const int slot = slot_in[ps];
-      w_in[ps] = slot < n_in ? ld_stream_u4(Lp.in_bits + (size_t)in_row(slot) * (DM / 32) + li_in * 4)
-                             : make_uint4(0, 0, 0, 0);
-    }
-    w_out = slot_out < n_out ? ld_stream_u4(Lp.out_bits + (size_t)(ro0 + slot_out) * (E / 32) + lane * 4)
-                             : make_uint4(0, 0, 0, 0);
-    float nw[4], gw[8];
-#pragma unroll
-    for (int k = 0; k < 4; ++k) nw[k] = __ldg(Lp.norm_w + tid + k * NT);
-#pragma unroll
-    for (int k = 0; k < 8; ++k) gw[k] = __ldg(Lp.gnorm_w + tid + k * NT);
-    float lbs_in = 0.f;
-    if (tid >= kChainBase && tid < kChainBase + R) lbs_in = __ldg(Lp.in_lbs + tid - kChainBase);
-    // own x channels: conv taps, bias, state (thread NSH + j handles channel rs0 + j)
-    float4 cw = make_float4(0.f, 0.f, 0.f, 0.f);
-    float cb = 0.f, cs0 = 0.f, cs1 = 0.f, cs2 = 0.f;
-    if (tid >= NSH && tid - NSH < n_ssm) {
-      const int ch = rs0 + (tid - NSH);
-      cw = __ldg(reinterpret_cast<const float4*>(Lp.conv_w) + ch);
-      cb = __ldg(Lp.conv_b + ch);
-      cs0 = Lp.conv_state[(size_t)ch * 3 + 0];
-      cs1 = Lp.conv_state[(size_t)ch * 3 + 1];
-      cs2 = Lp.conv_state[(size_t)ch * 3 + 2];
-    }
-    float dtb = 0.f, A_h = 0.f;
-    if (dt_own) {
-      dtb = __ldg(Lp.dt_bias + dt_head);
-      A_h = __double2float_rn(-exp((double)__ldg(Lp.A_log + dt_head)));
-    }
-    // epilogue parameters into shared memory, asynchronously
-    if (tid < n_in) {
-      const int row = in_row(tid);
-      cp_async4(&in_sw[tid], Lp.in_ws + row);
-      cp_async4(&in_sa[tid], Lp.in_las + row);
-      cp_async16(in_wa[tid], Lp.in_la + (size_t)row * R);
-    }
-    if (tid == kCopyThread) {
-      // the contiguous ranges every CTA needs, one bulk copy each; every generic access of the previous
-      // layer to these buffers is ordered before them by the barrier that ended that layer.  Issued by a
-      // thread other than the poller of the h hand-off, so that polling starts at once.
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      // first in the copy queue: the next layer's SSM state rows of this CTA (their buffer was last
-      // read in layer l - 1)
-      if (has_next) {
-        const int nb = (l + 1) & 1;
-        mbar_expect_tx(&stbar[nb], n_ssm * N * 4);
-        bulk_g2s(st_sm + nb * MAX_SSM * N, lsm[l + 1].ssm_state + (size_t)rs0 * N, n_ssm * N * 4, &stbar[nb]);
-      }
-      mbar_expect_tx(&ldbar[0], NSH * 4 * 2 + NSH * R + 2 * N * (16 + 4 + 12) + R * DM);
-      bulk_g2s(sh_sw, Lp.in_ws + SH0, NSH * 4, &ldbar[0]);
-      bulk_g2s(sh_sa, Lp.in_las + SH0, NSH * 4, &ldbar[0]);
-      bulk_g2s(sh_wa, Lp.in_la + (size_t)SH0 * R, NSH * R, &ldbar[0]);
-      bulk_g2s(bc_w, Lp.conv_w + (size_t)E * 4, 2 * N * 16, &ldbar[0]);
-      bulk_g2s(bc_b, Lp.conv_b + E, 2 * N * 4, &ldbar[0]);
-      bulk_g2s(bc_st, Lp.conv_state + (size_t)E * 3, 2 * N * 12, &ldbar[0]);
-      bulk_g2s(wb_in, Lp.in_lb, R * DM, &ldbar[0]);
-      mbar_expect_tx(&ldbar[1], R * E);
-      bulk_g2s(wb_out, Lp.out_lb, R * E, &ldbar[1]);
-    }
-    if (tid < n_out) {
-      const int row = ro0 + tid;
-      cp_async4(&o_sw[tid], Lp.out_ws + row);
-      cp_async4(&o_sa[tid], Lp.out_las + row);
-      cp_async16(o_wa[tid], Lp.out_la + (size_t)row * R);
-    }
-    if (tid < 2 && hA + tid < H) cp_async4(&Dv[tid], Lp.D + hA + tid);
-    if (tid < R) cp_async4(&lbs_o[tid], Lp.out_lbs + tid);
-    cp_async_commit();  // this thread's row parameters (awaited after the h wait)
+  };
+  for (int l = 0; l < p.n_layers; ++l) {
+    const LayerPtrs& Lp = lsm[l];
+    const bool has_next = l + 1 < p.n_layers;
+    const uint32_t tag_h = (uint32_t)l, tag_l = (uint32_t)(l + 1);
 
     // ---------------------------------------------------------------- phase A: h -> in_proj
-    if (l > 0 && !block_wait(p.ctr + CTR_H * CTR_STRIDE, NC * l, p.err, p.status, p.spin_limit, &sflag)) {
-      drain(l, has_next);
-      return;
+    float hv[4];
+    bool ok = true;
+    if (l == 0) {
+#pragma unroll
+      for (int k = 0; k < 4; k += 2) {
+        const float2 v = *reinterpret_cast<const float2*>(p.hidden + hidx[k]);
+        hv[k] = v.x;
+        hv[k + 1] = v.y;
+      }
+    } else {
+      // every warp has finished the previous layer (the out_proj epilogue and the loads for this layer)
+      // before any thread starts polling: spinning loads would otherwise slow those warps down
+      __syncthreads();
+      ok = poll_pairs<2>(p.hx, hoff, tag_h, hv, p.err, p.status, p.spin_limit);
     }
     cp_async_wait<0>();  // this thread's row parameters; the quantizer's barriers publish them
-    if (!mbar_wait(&ldbar[0], l & 1, p.spin_limit)) {  // shared rows and in_proj W_B
-      atomicExch(p.err, 1);
-      atomicExch(p.status, kTimeoutMagic);
-      drain(l, has_next);
+    if (ok && !mbar_wait(&inbar[l & 1], (l >> 1) & 1, p.spin_limit)) {  // in_proj W_B and the norm weight
+      fail();
+      ok = false;
+    }
+    bool abort_any = false;
+    const float s_in = norm_quantize<4, DM / 128>(hv, nw_sm(l), hidx, DM, lane, warp, red_d, red_u, red_i,
+                                                  &any_flag[0], q_perm, q_nat, !ok, abort_any);
+    if (abort_any) {
+      drain(l, false);
       return;
     }
-    // RMSNorm, then the quantizer on the normalized row: r from the block sum of squares, then the
-    // absmax of u = fl32(fl32(h r) w)
-    float s0A;
-    {
-      float hv[4], v[4];
-      double ss = 0.0;
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        hv[k] = __ldcg(p.hidden + tid + k * NT);
-        ss += (double)hv[k] * (double)hv[k];
-      }
-      if (tid < n_out) h_old[tid] = __ldcg(p.hidden + ro0 + tid);
-      const float rn = rms_factor(block_sum_d(ss, lane, warp, red_d), DM);
-      float m = 0.0f;
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        v[k] = norm_value(hv[k], rn, nw[k]);
-        m = fmaxf(m, fabsf(v[k]));
-      }
-      m = block_absmax(m, lane, warp, red_u);
-      const float s0 = m == 0.0f ? 0.0f : __fdiv_rn(m, 127.0f);
-      const float inv_s0 = m == 0.0f ? 0.0f : __frcp_rn(s0);
-      int sq = 0;
-      int cd[4];
-      quant_codes<4>(v, s0, inv_s0, cd);
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        q_perm[seg_index<DM / 128>(tid + k * NT)] = (int8_t)cd[k];
-        q_nat[tid + k * NT] = (int8_t)cd[k];
-        sq += cd[k];
-      }
-      sq = __reduce_add_sync(0xffffffffu, sq);
-      if (lane == 0) red_i[warp] = sq;
-      __syncthreads();
-      s0A = s0;
-    }
+    if (tid == 0) any_flag[1] = 0;  // the gated norm's flag (last read in the previous layer)
     const int sumq = block_sum16(red_i);
-    // scaffold GEMV over the owned rows; pass 0 holds the rows every CTA needs
+    // scaffold GEMV over the owned rows, pass 0 (the shared rows first), then LoRA-down row `warp`
+    uint4 qreg[8];  // this lane's segment of the codes, for both passes
+#pragma unroll
+    for (int v = 0; v < 8; ++v) qreg[v] = reinterpret_cast<const uint4*>(q_perm)[li_in + v * (DM / 128)];
     {
-      const uint4* qp4 = reinterpret_cast<const uint4*>(q_perm) + li_in;
+      int S = bits_dot_reg(w_in[0], qreg);
 #pragma unroll
-      for (int ps = 0; ps < 2; ++ps) {
-        int S = bits_dot<DM / 128>(w_in[ps], qp4);
-#pragma unroll
-        for (int o = 8; o > 0; o >>= 1) S += __shfl_xor_sync(0xffffffffu, S, o);
-        if (li_in == 0 && slot_in[ps] < n_in) {
-          acc_in[slot_in[ps]] = 2 * S - sumq;
-          if (ps == 0 && slot_in[0] < n_sh) p.sacc[sh0 + slot_in[0]] = 2 * S - sumq;
-        }
-        if (ps == 0) {
-          block_arrive(p.ctr + CTR_BC * CTR_STRIDE);  // its barrier orders the accumulators above
-          // LoRA down of the codes: warp r computes t[r]
-          const int t = lora_row<DM / 16>(wb_in + warp * DM, q_nat, lane);
-          if (lane == 0) t_sm[warp] = t;
-        }
-      }
+      for (int o = 8; o > 0; o >>= 1) S += __shfl_xor_sync(0xffffffffu, S, o);
+      if (li_in == 0 && slot_in[0] < n_in) acc_in[slot_in[0]] = 2 * S - sumq;
+      lora_slice<DM>(wb_in(l), q_nat, warp, lane, red_t);
     }
-    // the LoRA intermediate (off the GEMV's critical path: the epilogue needs it only after the B/C wait)
     __syncthreads();
-    if (tid >= kChainBase && tid < kChainBase + R) tf[tid - kChainBase] = lora_tf(t_sm[tid - kChainBase], lbs_in, s0A);
-    if (tid == kChainBase + R) s_scale = s0A;
-
-    // ---------------------------------------------------------------- phase B: epilogues + SSM
-    if (!block_wait(p.ctr + CTR_BC * CTR_STRIDE, NC * (l + 1), p.err, p.status, p.spin_limit, &sflag)) {
-      drain(l, has_next);
-      return;
-    }
-    const float s_in = s_scale;
-    if (tid < NSH) {
-      // rows every CTA needs: B, C (conv + SiLU) and dt of this CTA's heads
-      const float y = linear_out(__ldcg(p.sacc + tid), s_in, sh_sw[tid], sh_sa[tid], sh_wa[tid], tf, R);
-      if (tid < 2 * N) {
-        bc_new[tid] = y;
-        const float xc = conv_out(bc_w[tid], bc_b[tid], bc_st[tid][0], bc_st[tid][1], bc_st[tid][2], y);
-        if (tid < N) Bsm[tid] = xc;
-        else Cd[tid - N] = (double)xc;
-      } else if (dt_own) {
-        const float dt = ssm_dt(y, dtb);
-        dtv[dt_head - hA] = dt;
-        dAv[dt_head - hA] = __double2float_rn(exp((double)fmul(dt, A_h)));
+    const auto pass1 = [&]() {
+      int S = bits_dot_reg(w_in[1], qreg);
+#pragma unroll
+      for (int o = 8; o > 0; o >>= 1) S += __shfl_xor_sync(0xffffffffu, S, o);
+      if (li_in == 0 && slot_in[1] < n_in) acc_in[slot_in[1]] = 2 * S - sumq;
+    };
+    if (warp == kBcWarp) {
+      // LoRA intermediates (published to the z/x epilogues through barrier 1 without waiting there),
+      // then the shared rows' epilogues, published to every CTA as final values
+      if (lane < R) tf_d[lane] = (double)lora_tf(lora_t_sum(red_t, lane), lbs_in[lane], s_in);
+      if (lane == R) s_in_sm = s_in;
+      if (32 + warp * 2 < n_in) pass1();  // only when a CTA owns more than 62 in_proj rows
+      bar_arrive(1, NT);
+      __syncwarp();
+      if (bc_own) {
+        double tfl[R];
+#pragma unroll
+        for (int r = 0; r < R; ++r) tfl[r] = tf_d[r];
+        const float y = linear_out_d(acc_in[bc_j], (double)s_in, (double)bsw, (double)bsa, bwa, tfl, R);
+        if (bc_k < 2 * N) {
+          st_tagged(p.bcx + bc_k, conv_out(bcw, bcb, bs0, bs1, bs2, y), tag_l);
+          float* st = Lp.conv_state + (size_t)(E + bc_k) * 3;
+          st[0] = bs1;
+          st[1] = bs2;
+          st[2] = y;
+        } else {
+          const float dt = ssm_dt(y, dtb);
+          const float dA = __double2float_rn(exp((double)fmul(dt, A_h)));
+          const int hh = bc_k - 2 * N;
+          st_tagged(p.bcx + 2 * N + 2 * hh, dt, tag_l);
+          st_tagged(p.bcx + 2 * N + 2 * hh + 1, dA, tag_l);
+        }
       }
-    } else if (tid - NSH < n_ssm) {
+    } else {
+      // pass 1: the remaining z/x rows
+      if (32 + warp * 2 < n_in) pass1();
+      bar_sync(1, NT);
+    }
+
+    // ---------------------------------------------------------------- phase B: z/x epilogues + SSM
+    if (tid >= kZxBase && tid - kZxBase < n_ssm) {
       // the owned z rows (gate value SiLU(z) kept) and x rows (conv of the owned x channels)
-      const int j = tid - NSH;
+      const int j = tid - kZxBase;
       const int sz = n_sh + j, sx = n_sh + n_ssm + j;
-      zsm[j] = silu_f64(linear_out(acc_in[sz], s_in, in_sw[sz], in_sa[sz], in_wa[sz], tf, R));
-      const float xr = linear_out(acc_in[sx], s_in, in_sw[sx], in_sa[sx], in_wa[sx], tf, R);
+      double tfl[R];
+#pragma unroll
+      for (int r = 0; r < R; ++r) tfl[r] = tf_d[r];
+      const double sd = (double)s_in_sm;
+      const float zr = linear_out_d(acc_in[sz], sd, (double)in_sw[sz], (double)in_sa[sz],
+                                    *reinterpret_cast<const uint4*>(in_wa[sz]), tfl, R);
+      const float xr = linear_out_d(acc_in[sx], sd, (double)in_sw[sx], (double)in_sa[sx],
+                                    *reinterpret_cast<const uint4*>(in_wa[sx]), tfl, R);
+      zsm[j] = silu_f64(zr);
       xsm[j] = conv_out(cw, cb, cs0, cs1, cs2, xr);
       float* st = Lp.conv_state + (size_t)(rs0 + j) * 3;
       st[0] = cs1;
       st[1] = cs2;
       st[2] = xr;
     }
-    __syncthreads();
-    if (!mbar_wait(&stbar[l & 1], (l >> 1) & 1, p.spin_limit)) {  // this layer's SSM state rows
-      atomicExch(p.err, 1);
-      atomicExch(p.status, kTimeoutMagic);
+    if (has_next) issue_ahead(l);
+    // B and C (threads 0..127: one pair each), dt and dA of the CTA's heads (threads 128, 129)
+    ok = true;
+    if (tid < N) {
+      float v[2];
+      const int off[1] = {2 * tid};
+      ok = poll_pairs<1>(p.bcx, off, tag_l, v, p.err, p.status, p.spin_limit);
+      if (ok) {
+        const int i = 2 * tid;
+        if (i < N) {
+          Bsm[i] = v[0];
+          Bsm[i + 1] = v[1];
+        } else {
+          Cd[i - N] = (double)v[0];
+          Cd[i + 1 - N] = (double)v[1];
+        }
+      }
+    } else if (tid - N < n_heads) {
+      float v[2];
+      const int off[1] = {2 * N + 2 * (hA + tid - N)};
+      ok = poll_pairs<1>(p.bcx, off, tag_l, v, p.err, p.status, p.spin_limit);
+      if (ok) {
+        dtv[tid - N] = v[0];
+        dAv[tid - N] = v[1];
+      }
+    }
+    if (ok && !mbar_wait(&stbar[l & 1], (l >> 1) & 1, p.spin_limit)) {  // this layer's SSM state rows
+      fail();
+      ok = false;
+    }
+    if (__syncthreads_or(!ok)) {
       drain(l, has_next);
       return;
     }
@@ -634,97 +818,63 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ P
         acc = warp_sum(acc);
         if (lane == 0) {
           const float y = __double2float_rn(dadd(acc, dmul((double)Dv[hi], (double)xv)));
-          const float g = fmul(y, zsm[rr]);
-          p.gbuf[hp] = g;
+          st_tagged(p.gx + hp, fmul(y, zsm[rr]), tag_l);
         }
       }
     }
-    block_arrive(p.ctr + CTR_G * CTR_STRIDE);
 #pragma unroll
     for (int ps = 0; ps < 2; ++ps)
       if (ssm_slot[ps] < n_ssm) st_f4(Lp.ssm_state + (size_t)(rs0 + ssm_slot[ps]) * N + lane * 4, snew[ps]);
 
     // ---------------------------------------------------------------- phase C: gated norm -> out_proj
-    if (!block_wait(p.ctr + CTR_G * CTR_STRIDE, NC * (l + 1), p.err, p.status, p.spin_limit, &sflag)) {
+    float gv[8];
+    __syncthreads();  // as before the h poll: no thread spins while others still work on this phase
+    ok = poll_pairs<4>(p.gx, goff, tag_l, gv, p.err, p.status, p.spin_limit);
+    if (ok && !mbar_wait(&outbar, l & 1, p.spin_limit)) {  // out_proj W_B and the gated-norm weight
+      fail();
+      ok = false;
+    }
+    const float s_out = norm_quantize<8, E / 128>(gv, gw_sm, gidx, E, lane, warp, red_d, red_u, red_i,
+                                                  &any_flag[1], q_perm, q_nat, !ok, abort_any);
+    if (abort_any) {
       drain(l, has_next);
       return;
     }
-    if (!mbar_wait(&ldbar[1], l & 1, p.spin_limit)) {  // out_proj W_B
-      atomicExch(p.err, 1);
-      atomicExch(p.status, kTimeoutMagic);
-      drain(l, has_next);
-      return;
-    }
-    // every CTA has now read the old B/C conv state: the owners of those rows shift it
-    for (int j = tid; j < n_sh; j += NT) {
-      const int k = sh0 + j;
-      if (k < 2 * N) {
-        float* st = Lp.conv_state + (size_t)(E + k) * 3;
-        st[0] = bc_st[k][1];
-        st[1] = bc_st[k][2];
-        st[2] = bc_new[k];
-      }
-    }
+    if (tid == 0) any_flag[0] = 0;  // the next layer's pre-norm flag
     {
-      float gv[8], v[8];
-      double ss = 0.0;
-#pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        gv[k] = __ldcg(p.gbuf + tid + k * NT);
-        ss += (double)gv[k] * (double)gv[k];
-      }
-      const float rn = rms_factor(block_sum_d(ss, lane, warp, red_d), E);
-      float m = 0.0f;
-#pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        v[k] = norm_value(gv[k], rn, gw[k]);
-        m = fmaxf(m, fabsf(v[k]));
-      }
-      m = block_absmax(m, lane, warp, red_u);
-      const float s0 = m == 0.0f ? 0.0f : __fdiv_rn(m, 127.0f);
-      const float inv_s0 = m == 0.0f ? 0.0f : __frcp_rn(s0);
-      int sq = 0;
-      int cd[8];
-      quant_codes<8>(v, s0, inv_s0, cd);
-#pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        q_perm[seg_index<E / 128>(tid + k * NT)] = (int8_t)cd[k];
-        q_nat[tid + k * NT] = (int8_t)cd[k];
-        sq += cd[k];
-      }
-      sq = __reduce_add_sync(0xffffffffu, sq);
-      if (lane == 0) red_i[warp] = sq;
-      if (tid == 0) s_scale = s0;
-      __syncthreads();
-      // LoRA down of the codes (warp r: t[r]); every warp with an out_proj row then takes it
-      const int t = lora_row<E / 16>(wb_out + warp * E, q_nat, lane);
-      if (lane == 0) t_sm[warp] = t;
-      if (warp != kChainWarp) {
+      // LoRA down of the codes (by input slices); every warp with an out_proj row then takes it
+      lora_slice<E>(wb_out, q_nat, warp, lane, red_t);
+      if (slot_out < n_out) {
         const int sumq_c = block_sum16(red_i);
-        const uint4* qp4 = reinterpret_cast<const uint4*>(q_perm) + lane;
-        int S = bits_dot<E / 128>(w_out, qp4);
+        int S = bits_dot<E / 128>(w_out, reinterpret_cast<const uint4*>(q_perm) + lane);
         S = warp_sum(S);
-        if (lane == 0 && slot_out < n_out) acc_out[slot_out] = 2 * S - sumq_c;
+        if (lane == 0) acc_out[slot_out] = 2 * S - sumq_c;
       }
     }
     __syncthreads();
-    if (tid < n_out) {
-      // each epilogue thread forms the sixteen LoRA intermediates itself (no further barrier)
+    if (warp == 0) {
+      // lanes r < R form the LoRA intermediate tf[r]; every epilogue lane takes all sixteen by shuffle
+      const double tf_r = lane < R ? (double)lora_tf(lora_t_sum(red_t, lane), lbs_o[l & 1][lane], s_out) : 0.0;
       double tfd[R];
 #pragma unroll
-      for (int r = 0; r < R; ++r) tfd[r] = (double)lora_tf(t_sm[r], lbs_o[r], s_scale);
-      const float y = linear_out_d(acc_out[tid], (double)s_scale, (double)o_sw[tid], (double)o_sa[tid],
-                                   *reinterpret_cast<const uint4*>(o_wa[tid]), tfd, R);
-      p.hidden[ro0 + tid] = fadd(h_old[tid], y);
+      for (int r = 0; r < R; ++r) tfd[r] = __shfl_sync(0xffffffffu, tf_r, r);
+      if (tid < n_out) {
+        const float y = linear_out_d(acc_out[tid], (double)s_out, (double)o_sw[tid], (double)o_sa[tid],
+                                     *reinterpret_cast<const uint4*>(o_wa[tid]), tfd, R);
+        h_own = fadd(h_own, y);
+        if (has_next) st_tagged(p.hx + ro0 + tid, h_own, tag_l);
+        else p.hidden[ro0 + tid] = h_own;
+      }
     }
-    block_arrive(p.ctr + CTR_H * CTR_STRIDE);
+    if (has_next) issue_loads(l + 1);
   }
 }
 
-// Waits on a counter that nothing increments, with a short budget: exercises the timeout path.
-__global__ void timeout_selftest_kernel(int* ctr, int* err, int* status, long long limit) {
-  __shared__ int sflag;
-  block_wait(ctr, 1, err, status, limit, &sflag);
+// Polls a tagged word that nothing writes, with a short budget: exercises the timeout path.
+__global__ void timeout_selftest_kernel(const unsigned long long* word, int* err, int* status, long long limit) {
+  float v[2];
+  const int off[1] = {0};
+  poll_pairs<1>(word, off, 1u, v, err, status, limit);
 }
 
 }  // namespace fused
@@ -736,19 +886,19 @@ bool fused_decode_supported(const dfssm_dims_t& d, int B, const dfssm_layer_t* l
   if (B != 1 || d.d_model != fused::DM || d.nheads != fused::H || d.headdim != fused::P ||
       d.d_state != fused::N || d.ngroups != 1)
     return false;
-  // the ranges fetched by bulk copy must start on 16-byte boundaries
+  // vector loads (16 bytes: W_A rows, conv taps; 8 bytes: norm weights) and the bulk copies of W_B
   const auto a16 = [](const void* q) { return (reinterpret_cast<uintptr_t>(q) & 15) == 0; };
+  const auto a8 = [](const void* q) { return (reinterpret_cast<uintptr_t>(q) & 7) == 0; };
   for (int l = 0; l < n; ++l) {
     const dfssm_layer_t& L = layers[l];
     if (L.in_proj.rank != fused::R || L.out_proj.rank != fused::R) return false;
-    if (!a16(L.in_proj.w_scale) || !a16(L.in_proj.lora_a_scale) || !a16(L.in_proj.lora_a) ||
-        !a16(L.in_proj.lora_b) || !a16(L.out_proj.lora_b) || !a16(L.conv_w) || !a16(L.conv_b) ||
+    if (!a16(L.in_proj.lora_a) || !a16(L.out_proj.lora_a) || !a16(L.in_proj.lora_b) ||
+        !a16(L.out_proj.lora_b) || !a16(L.conv_w) || !a8(L.norm_w) || !a8(L.gnorm_w) ||
         !a16(conv_states[l]))
       return false;
   }
   const int nc = num_sms();
-  // ownership limits: in_proj rows per CTA <= 64, out_proj rows <= 16, SSM rows <= 32; partial-sum
-  // buffers sized for MAX_CTAS
+  // ownership limits: in_proj rows per CTA <= 64, out_proj rows <= 16, SSM rows <= 32
   if (nc < fused::MIN_CTAS || nc > fused::MAX_CTAS) return false;
   int coop = 0, dev = 0;
   cudaGetDevice(&dev);
@@ -789,21 +939,19 @@ cudaError_t launch_fused_decode(const dfssm_layer_t* layers, int n_layers, float
   char* base = static_cast<char*>(ws);
   p.n_layers = n_layers;
   p.hidden = hidden;
-  p.ctr = reinterpret_cast<int*>(base + fused::OFF_CTR);
-  p.err = reinterpret_cast<int*>(base + fused::OFF_ERR);
   p.status = reinterpret_cast<int*>(base + fused::OFF_STATUS);
-  p.sacc = reinterpret_cast<int*>(base + fused::OFF_SACC);
-  p.gbuf = reinterpret_cast<float*>(base + fused::OFF_GBUF);
+  p.err = reinterpret_cast<int*>(base + fused::OFF_ERR);
+  p.hx = reinterpret_cast<unsigned long long*>(base + fused::OFF_HX);
+  p.gx = reinterpret_cast<unsigned long long*>(base + fused::OFF_GX);
+  p.bcx = reinterpret_cast<unsigned long long*>(base + fused::OFF_BCX);
   p.spin_limit = spin_limit;
-  cudaError_t e = cudaMemsetAsync(p.ctr, 0, fused::CLEAR_BYTES, st);
+  cudaError_t e = cudaMemsetAsync(base + fused::CLEAR_OFF, 0, fused::CLEAR_BYTES, st);
+  if (e != cudaSuccess) return e;
+  e = set_max_dynamic_smem(reinterpret_cast<const void*>(fused::decode_kernel), fused::DYN_BYTES);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(num_sms());
   cfg.blockDim = dim3(fused::NT);
-  // set once (not per launch, so that launches can be captured in a CUDA graph)
-  static const cudaError_t attr_set = cudaFuncSetAttribute(
-      fused::decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, fused::DYN_BYTES);
-  if (attr_set != cudaSuccess) return attr_set;
   cfg.dynamicSmemBytes = fused::DYN_BYTES;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
@@ -816,12 +964,12 @@ cudaError_t launch_fused_decode(const dfssm_layer_t* layers, int n_layers, float
 
 cudaError_t launch_timeout_selftest(void* ws, cudaStream_t st, long long spin_limit) {
   char* base = static_cast<char*>(ws);
-  int* ctr = reinterpret_cast<int*>(base + fused::OFF_CTR);
   int* err = reinterpret_cast<int*>(base + fused::OFF_ERR);
   int* status = reinterpret_cast<int*>(base + fused::OFF_STATUS);
-  cudaError_t e = cudaMemsetAsync(ctr, 0, fused::CLEAR_BYTES, st);
+  const unsigned long long* word = reinterpret_cast<const unsigned long long*>(base + fused::OFF_HX);
+  cudaError_t e = cudaMemsetAsync(base + fused::CLEAR_OFF, 0, fused::CLEAR_BYTES, st);
   if (e != cudaSuccess) return e;
-  fused::timeout_selftest_kernel<<<1, 32, 0, st>>>(ctr, err, status, spin_limit);
+  fused::timeout_selftest_kernel<<<1, 32, 0, st>>>(word, err, status, spin_limit);
   return cudaGetLastError();
 }
 

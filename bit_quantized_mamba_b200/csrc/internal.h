@@ -143,7 +143,12 @@ struct EmbedArgs {
 };
 cudaError_t launch_embed(const EmbedArgs& a, cudaStream_t st);
 
+// Streaming multiprocessors of the current device.
 int num_sms();
+// Sets the dynamic shared-memory limit of a kernel on the current device, once per (kernel, device): the
+// attribute is per device, and setting it once (not per launch) keeps launches capturable in a CUDA
+// graph.  Thread-safe.  The record is per process: after cudaDeviceReset the library must not be used.
+cudaError_t set_max_dynamic_smem(const void* func, int bytes);
 
 }  // namespace dfssm
 

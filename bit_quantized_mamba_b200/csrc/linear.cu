@@ -11,6 +11,10 @@
 //     acc                =  2 * sum_{i: bit=1} q_i - sum_i q_i
 // which is 2 integer instructions per 4 weights, exact in int32.
 
+#include <atomic>
+#include <mutex>
+#include <vector>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -39,14 +43,35 @@ QuantScratch carve_quant_scratch(void* base, int B, int n) {
 }
 
 int num_sms() {
-  static int sms = 0;
+  constexpr int kMaxDevices = 64;
+  static std::atomic<int> cache[kMaxDevices];  // 0 = not yet queried
+  int dev = 0;
+  cudaGetDevice(&dev);
+  int sms = (dev >= 0 && dev < kMaxDevices) ? cache[dev].load(std::memory_order_relaxed) : 0;
   if (sms == 0) {
-    int dev = 0;
-    cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (sms <= 0) sms = 148;
+    if (dev >= 0 && dev < kMaxDevices) cache[dev].store(sms, std::memory_order_relaxed);
   }
   return sms;
+}
+
+cudaError_t set_max_dynamic_smem(const void* func, int bytes) {
+  struct Done {
+    const void* func;
+    int dev, bytes;
+  };
+  static std::mutex mu;
+  static std::vector<Done> done;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(mu);
+  for (const Done& d : done)
+    if (d.func == func && d.dev == dev && d.bytes >= bytes) return cudaSuccess;
+  e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) done.push_back(Done{func, dev, bytes});
+  return e;
 }
 
 template <typename Kern, typename... Args>
@@ -113,8 +138,8 @@ __global__ void __launch_bounds__(kQuantThreads) quant_kernel(QuantArgs a) {
   __syncthreads();
   m = 0.0f;
   for (int w = 0; w < NW; ++w) m = fmaxf(m, red_f[w]);
-  const float s0 = (m == 0.0f) ? 0.0f : __fdiv_rn(m, 127.0f);
-  const float inv_s0 = (m == 0.0f) ? 0.0f : __frcp_rn(s0);
+  const float s0 = quant_scale(m);
+  const float inv_s0 = quant_inv(s0);
 
   int8_t* qout = a.out.q + (size_t)b * a.n;
   int sq = 0;
@@ -358,10 +383,8 @@ static cudaError_t launch_fast(const GemvArgs& a, cudaStream_t st) {
   const size_t smem = (size_t)a.B * a.d_in;
   auto k = gemv_kernel<LPR, NSEG, BT>;
   if (smem > 48 * 1024) {
-    // once per instantiation (the largest size any call can need), not per launch, so that launches
-    // can be captured in a CUDA graph
-    static const cudaError_t set = cudaFuncSetAttribute(
-        k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)(DFSSM_MAX_BATCH * 8192));
+    // the largest size any call can need, once per device
+    const cudaError_t set = set_max_dynamic_smem(reinterpret_cast<const void*>(k), DFSSM_MAX_BATCH * 8192);
     if (set != cudaSuccess) return set;
   }
   return launch_pdl(k, dim3((a.d_out + RPC - 1) / RPC), dim3(kGemvThreads), smem, st, a);
@@ -373,8 +396,7 @@ static cudaError_t launch_generic(const GemvArgs& a, cudaStream_t st) {
   const size_t smem = (size_t)a.B * a.d_in;
   auto k = gemv_generic_kernel<BT>;
   if (smem > 48 * 1024) {
-    static const cudaError_t set = cudaFuncSetAttribute(
-        k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)(DFSSM_MAX_BATCH * 8192));
+    const cudaError_t set = set_max_dynamic_smem(reinterpret_cast<const void*>(k), DFSSM_MAX_BATCH * 8192);
     if (set != cudaSuccess) return set;
   }
   return launch_pdl(k, dim3((a.d_out + RPC - 1) / RPC), dim3(kGemvThreads), smem, st, a);

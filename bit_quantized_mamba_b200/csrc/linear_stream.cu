@@ -609,8 +609,8 @@ __global__ void __launch_bounds__(NT, 1) stream_kernel(const __grid_constant__ P
     m = 0.0f;
 #pragma unroll
     for (int j = 0; j < WPT; ++j) m = fmaxf(m, red_f[slot * WPT + j][0]);
-    const float s0 = m == 0.0f ? 0.0f : __fdiv_rn(m, 127.0f);
-    const float inv_s0 = m == 0.0f ? 0.0f : __frcp_rn(s0);
+    const float s0 = quant_scale(m);
+    const float inv_s0 = quant_inv(s0);
     int sq = 0;
     if (active) {
 #pragma unroll 1
@@ -686,8 +686,8 @@ __global__ void __launch_bounds__(NT, 1) stream_kernel(const __grid_constant__ P
       float m = 0.0f;
 #pragma unroll
       for (int w = 0; w < NCW; ++w) m = fmaxf(m, red_f[w][b]);
-      const float s0 = m == 0.0f ? 0.0f : __fdiv_rn(m, 127.0f);
-      const float inv_s0 = m == 0.0f ? 0.0f : __frcp_rn(s0);
+      const float s0 = quant_scale(m);
+      const float inv_s0 = quant_inv(s0);
       int sq = 0;
       if (b < B) {
         float v[XPT];
@@ -923,8 +923,7 @@ cudaError_t launch_t(const Params& p, int grid, cudaStream_t st) {
   constexpr int DIN = 128 * LPR * NSEG;
   constexpr size_t smem = smem_bytes(DIN, BT, TB);
   auto k = stream_kernel<LPR, NSEG, BT, TB>;
-  // once per instantiation, not per launch, so that launches can be captured in a CUDA graph
-  static const cudaError_t set = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  const cudaError_t set = set_max_dynamic_smem(reinterpret_cast<const void*>(k), (int)smem);
   if (set != cudaSuccess) return set;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);

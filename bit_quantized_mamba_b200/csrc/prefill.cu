@@ -247,8 +247,8 @@ __global__ void __launch_bounds__(QW * 32) prefill_quant_kernel(const float* __r
       m_abs = fmaxf(m_abs, fmaxf(fmaxf(fabsf(v[u].x), fabsf(v[u].y)), fmaxf(fabsf(v[u].z), fabsf(v[u].w))));
   }
   m_abs = warp_max(m_abs);
-  const float s0 = m_abs == 0.0f ? 0.0f : __fdiv_rn(m_abs, 127.0f);
-  const float inv_s0 = m_abs == 0.0f ? 0.0f : __frcp_rn(s0);
+  const float s0 = quant_scale(m_abs);
+  const float inv_s0 = quant_inv(s0);
   const float s_tok = s0;
   int u[DFSSM_MAX_RANK];
 #pragma unroll
@@ -629,13 +629,8 @@ int dfssm::linear_prefill_impl(const dfssm_linear_t* lin, const float* x, int M,
 
   // 1. per-token quantization and LoRA down-projection (one warp per token)
   const size_t qsmem = (size_t)DFSSM_MAX_RANK * K;  // W_B padded to sixteen rows
-  static bool qattr = false;
-  if (!qattr) {
-    const cudaError_t ea = cudaFuncSetAttribute(prefill::prefill_quant_kernel,
-                                                cudaFuncAttributeMaxDynamicSharedMemorySize, 16 * 8192);
-    if (ea != cudaSuccess) return record_cuda_failure(ea);
-    qattr = true;
-  }
+  const cudaError_t ea = set_max_dynamic_smem(reinterpret_cast<const void*>(prefill::prefill_quant_kernel), 16 * 8192);
+  if (ea != cudaSuccess) return record_cuda_failure(ea);
   prefill::prefill_quant_kernel<<<(M + prefill::QW - 1) / prefill::QW, prefill::QW * 32, qsmem, st>>>(
       x, M, K, lin->lora_b, lin->lora_b_scale, lin->rank, norm_w, w.xq, w.s, w.tf, dbg ? dbg->xq : nullptr,
       dbg ? dbg->xscale : nullptr, dbg ? dbg->lora_t : nullptr);
@@ -666,13 +661,8 @@ int dfssm::linear_prefill_impl(const dfssm_linear_t* lin, const float* x, int M,
   ep.K = K;
   ep.err = w.err;
   ep.resid = resid ? 1 : 0;
-  static bool attr_done = false;
-  if (!attr_done) {
-    e = cudaFuncSetAttribute(prefill::gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)prefill::PSMEM_BYTES);
-    if (e != cudaSuccess) return record_cuda_failure(e);
-    attr_done = true;
-  }
+  e = set_max_dynamic_smem(reinterpret_cast<const void*>(prefill::gemm_kernel), (int)prefill::PSMEM_BYTES);
+  if (e != cudaSuccess) return record_cuda_failure(e);
   const int tiles = ((N + prefill::BN - 1) / prefill::BN) * ((M + prefill::BM - 1) / prefill::BM);
   const int grid = tiles < num_sms() ? tiles : num_sms();
   prefill::gemm_kernel<<<grid, prefill::PNT, prefill::PSMEM_BYTES, st>>>(map_a, map_b, ep);

@@ -433,12 +433,10 @@ __global__ void __launch_bounds__(W128 * 32, 2) ssm_scan128_kernel(ScanArgs a) {
 template <int NJ, int NFIX>
 cudaError_t launch_scan_nj(const ScanArgs& a, cudaStream_t st) {
   const size_t smem = sizeof(float) * (2 * SCAN_BUF_FLOATS(a.N) + 2 * ST * SW);
-  static bool attr = false;
-  if (!attr) {
-    const cudaError_t e = cudaFuncSetAttribute(ssm_scan_kernel<NJ, NFIX>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  {
+    const cudaError_t e = set_max_dynamic_smem(reinterpret_cast<const void*>(ssm_scan_kernel<NJ, NFIX>),
                                                (int)(sizeof(float) * (2 * SCAN_BUF_FLOATS(512) + 2 * ST * SW)));
     if (e != cudaSuccess) return e;
-    attr = true;
   }
   const long long n_prep = (long long)a.M * (a.H * a.P + a.H);
   scan_prep_kernel<<<(unsigned)((n_prep + 255) / 256), 256, 0, st>>>(a);

@@ -215,8 +215,8 @@ __global__ void __launch_bounds__(256, LMH_CTAS_PER_SM) int8_gemv_kernel(Int8Gem
   m = 0.0f;
 #pragma unroll
   for (int w = 0; w < 8; ++w) m = fmaxf(m, red[w]);
-  const float s0 = m == 0.0f ? 0.0f : __fdiv_rn(m, 127.0f);
-  const float inv_s0 = m == 0.0f ? 0.0f : __frcp_rn(s0);
+  const float s0 = quant_scale(m);
+  const float inv_s0 = quant_inv(s0);
   const float s = s0;
   int8_t* qb = reinterpret_cast<int8_t*>(smem);
   for (int k0 = 0; k0 * 256 < a.d; k0 += 8) {
