@@ -29,6 +29,9 @@ N_TOKENS = 64
 WORKLOAD = ("DF-SSM Mamba-2-1.3B-shape decode: 48 layers, d_model 2048, d_inner 4096, 64 heads x 64, "
             "d_state 128, batch 1, 64 tokens per step")
 
+# B200 HBM3e nominal bandwidth (GB/s), reported beside the measured copy bandwidth.
+NOMINAL_HBM_GBS = 8000.0
+
 # Algorithmic bytes (weights + state read/write) per layer per token at batch 1.
 BYTES_IN_PROJ = 8512 * 2048 // 8 + 8512 * 4 + (16 * 2048 + 8512 * 16) + (16 * 4 + 8512 * 4)
 BYTES_OUT_PROJ = 2048 * 4096 // 8 + 2048 * 4 + (16 * 4096 + 2048 * 16) + (16 * 4 + 2048 * 4)
@@ -109,53 +112,80 @@ class ClockSampler:
 
 # ------------------------------------------------------------------------------ reference arm
 
-def time_oracle_decode(n_tokens: int, budget_s: float | None = None):
-    """Run the CPU oracle on the first n_tokens of the decode workload; returns (tokens, seconds)."""
-    import numpy as np
-    import oracle
-    from bit_quantized_mamba_b200 import inputs
-    model = inputs.decode_model(seed=3)
-    olayers = []
-    for l in model["layers"]:
-        olayers.append(dict(l, in_proj=oracle.Linear.from_dict(l["in_proj"]),
-                            out_proj=oracle.Linear.from_dict(l["out_proj"])))
-    conv, ssm = inputs.zero_states(1, 48)
-    done = 0
-    t0 = time.perf_counter()
-    for t in range(n_tokens):
-        h = np.ascontiguousarray(model["emb"][t])
-        for i, ol in enumerate(olayers):
-            oracle.layer_decode(ol, h, conv[i], ssm[i])
-        done += 1
-        if budget_s is not None and time.perf_counter() - t0 > budget_s:
-            break
-    return done, time.perf_counter() - t0
+class OracleDecode:
+    """The CPU oracle running the decode workload's 64-token stream (48 layers, batch 1) from the same
+    zero starting state as the GPU arm; each call advances it by whole tokens."""
+
+    def __init__(self):
+        import oracle
+        from bit_quantized_mamba_b200 import inputs
+        self.model = inputs.decode_model(seed=3)
+        self.layers = [dict(l, in_proj=oracle.Linear.from_dict(l["in_proj"]),
+                            out_proj=oracle.Linear.from_dict(l["out_proj"])) for l in self.model["layers"]]
+        self.conv, self.ssm = inputs.zero_states(1, 48)
+        self.t = 0
+
+    def run(self, n_tokens: int, budget_s: float | None = None):
+        """Decode up to n_tokens next tokens of the stream (stopping after budget_s seconds, at least one
+        token); returns (tokens, seconds)."""
+        import numpy as np
+        import oracle
+        done = 0
+        t0 = time.perf_counter()
+        while done < n_tokens:
+            h = np.ascontiguousarray(self.model["emb"][self.t % N_TOKENS])
+            for i, ol in enumerate(self.layers):
+                oracle.layer_decode(ol, h, self.conv[i], self.ssm[i])
+            self.t += 1
+            done += 1
+            if budget_s is not None and time.perf_counter() - t0 > budget_s:
+                break
+        return done, time.perf_counter() - t0
 
 
-def omp_threads():
-    return int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+def host_cores():
+    return os.cpu_count() or 1
+
+
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
 
 
 def run_reference(args, rank):
+    """The reference arm: the CPU oracle on the same 64-token stream from the same zero starting state
+    (states carried from step to step as on the GPU), one token per step so that the run stays within a
+    few minutes, on all host cores."""
     if rank != 0:
         return
-    import numpy as np  # noqa: F401
+    import oracle
+    threads = host_cores()
+    oracle.set_threads(threads)
+    dec = OracleDecode()
     tokens_per_step = 1
     per = []
     for i in range(args.warmup + args.steps):
-        n, dt = time_oracle_decode(tokens_per_step)
+        n, dt = dec.run(tokens_per_step)
         if i >= args.warmup:
             per.append(dt / n)
     sec_per_token = sum(per) / len(per)
     value = 1.0 / sec_per_token
+    sample = (f"tokens {args.warmup}..{args.warmup + args.steps - 1} of the 64-token stream (tokens "
+              f"0..{args.warmup - 1} untimed), one token x 48 layers per step, states carried from zero")
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec_per_token * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8",
         "data": "synthetic", "config": {"workload": WORKLOAD, "batch": 1,
                                         "tokens_per_step": tokens_per_step},
-        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": omp_threads(), "kind": "oracle",
-                         "sample": f"{tokens_per_step} token(s) x 48 layers per step"},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                         "cpu_model": cpu_model(), "sample": sample},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -268,7 +298,7 @@ def run_ours(args, rank, world, local_rank):
 
     # ---- end to end through the public API: pinned host embeddings in, final hidden state out
     out_host = torch.empty((1, 2048), dtype=torch.float32).pin_memory()
-    e2e_steps = max(2, min(args.steps, 5))
+    e2e_steps = args.steps
 
     def e2e_step():
         emb.copy_(emb_host, non_blocking=True)
@@ -294,6 +324,7 @@ def run_ours(args, rank, world, local_rank):
     # a CUDA graph (48 calls = 96 kernels, PDL-chained); L2 flushed before each timed replay
     hbm, peak_kind = peaks()
     flush = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    mws = dfssm.workspace(dfssm.workspace_size(dfssm.OP_LINEAR_MULTI, 0, 0, 0), dev)
     gemv = {}
     if not args.no_extras:
         for which, data_fn, nbytes in (("in_proj", inputs.in_proj_stack, BYTES_IN_PROJ),
@@ -334,10 +365,10 @@ def run_ours(args, rank, world, local_rank):
                 ys = [torch.empty((B, L.d_out), dtype=torch.float32, device=dev) for L in lins]
                 g = torch.cuda.CUDAGraph()
                 with torch.cuda.stream(stream):
-                    dfssm.linear_decode_multi(lins, xb, ys, stream=torch.cuda.current_stream())
+                    dfssm.linear_decode_multi(lins, xb, ys, ws=mws, stream=torch.cuda.current_stream())
                     torch.cuda.synchronize()
                     with torch.cuda.graph(g, stream=stream):
-                        dfssm.linear_decode_multi(lins, xb, ys, stream=torch.cuda.current_stream())
+                        dfssm.linear_decode_multi(lins, xb, ys, ws=mws, stream=torch.cuda.current_stream())
                 tot, reps = 0.0, 10
                 with torch.cuda.stream(stream):
                     for r in range(reps + 2):
@@ -504,6 +535,7 @@ def run_ours(args, rank, world, local_rank):
     achieved = BYTES_TOKEN / (us_tok * 1e-6) / 1e9
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
                 "frac": round(achieved / hbm, 4),
+                "frac_of_nominal_8TBs": round(achieved / NOMINAL_HBM_GBS, 4),
                 "traffic": (TRAFFIC_MEASURED["bytes"]
                             if src_sha("decode_fused.cu", "common.cuh") == TRAFFIC_MEASURED["sha"] else None),
                 "kernel": "dfssm::fused::decode_kernel (one cooperative launch per token, 48 layers)",
@@ -528,12 +560,22 @@ def run_ours(args, rank, world, local_rank):
         "clocks": clocks,
     }
 
-    # CPU baseline: the oracle on a bounded sample of the same workload (rank 0, N = 1 only)
+    # CPU baseline: the oracle on a bounded sample of the same workload (rank 0, N = 1 only), on all host
+    # cores and on one
     if world == 1 and not args.no_cpu_baseline:
-        n, dt = time_oracle_decode(N_TOKENS, budget_s=args.cpu_budget)
-        line["cpu_baseline"] = {"value": n / dt, "unit": "tokens/s", "cores": omp_threads(),
-                                "kind": "oracle",
-                                "sample": f"first {n} token(s) of the 64-token decode, 48 layers"}
+        import oracle
+        cores = host_cores()
+        oracle.set_threads(cores)
+        n, dt = OracleDecode().run(N_TOKENS, budget_s=args.cpu_budget)
+        oracle.set_threads(1)
+        n1, dt1 = OracleDecode().run(N_TOKENS, budget_s=args.cpu_budget)
+        oracle.set_threads(cores)
+        line["cpu_baseline"] = {"value": n / dt, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                                "cpu_model": cpu_model(),
+                                "sample": f"first {n} token(s) of the 64-token decode, 48 layers, from the "
+                                          f"zero state, on {cores} threads",
+                                "single_thread": {"value": n1 / dt1, "unit": "tokens/s", "cores": 1,
+                                                  "sample": f"first {n1} token(s), 1 thread"}}
     if rank == 0:
         print(json.dumps(line), flush=True)
     graph = None
@@ -565,8 +607,9 @@ def run_gemv_profile(args):
     lins = [dfssm.Linear.from_host(l, dev) for l in data["linears"]]
     x = torch.from_numpy(data["x"][:1].copy()).to(dev)
     ys = [torch.empty((1, L.d_out), dtype=torch.float32, device=dev) for L in lins]
+    ws = dfssm.workspace(dfssm.workspace_size(dfssm.OP_LINEAR_MULTI, 0, 0, 0), dev)
     for _ in range(args.warmup + 1):
-        dfssm.linear_decode_multi(lins, x, ys)
+        dfssm.linear_decode_multi(lins, x, ys, ws=ws)
     torch.cuda.synchronize()
 
 
@@ -614,7 +657,8 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--cpu-budget", type=float, default=10.0,
+                    help="seconds of oracle decode per CPU-baseline leg (all cores, then one core)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the GEMV sweep, prefill and LM-head measurements")

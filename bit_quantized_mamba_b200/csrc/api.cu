@@ -19,23 +19,8 @@ int cuda_fail(cudaError_t e) {
 inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-int check_linear(const dfssm_linear_t* L) {
-  if (!L) return DFSSM_EINVAL;
-  if (L->d_out < 1 || L->d_in < 32 || L->d_in % 32 != 0 || L->d_in > 8192) return DFSSM_EINVAL;
-  if (L->rank < 0 || L->rank > DFSSM_MAX_RANK) return DFSSM_EINVAL;
-  if (!L->bits || !L->w_scale) return DFSSM_EINVAL;
-  if (L->rank > 0 && (!L->lora_b || !L->lora_b_scale || !L->lora_a || !L->lora_a_scale))
-    return DFSSM_EINVAL;
-  if (!aligned(L->bits, 16) || !aligned(L->w_scale, 4)) return DFSSM_EALIGN;
-  if (L->rank > 0) {
-    if (!aligned(L->lora_b, 4) || !aligned(L->lora_b_scale, 4) || !aligned(L->lora_a_scale, 4))
-      return DFSSM_EALIGN;
-    if (L->rank == DFSSM_MAX_RANK && !aligned(L->lora_a, 16)) return DFSSM_EALIGN;
-  }
-  return DFSSM_OK;
-}
-
-size_t linear_decode_ws(int B, int d_in) { return dfssm::quant_scratch_bytes(B, d_in); }
+// Linear-decode workspace: [status word, kStatusBytes][quantize -> GEMV hand-off (quant scratch)].
+size_t linear_decode_ws(int B, int d_in) { return dfssm::kStatusBytes + dfssm::quant_scratch_bytes(B, d_in); }
 
 struct LayerWs {
   float* zxbcdt;  // [B][d_ip]
@@ -118,10 +103,7 @@ int check_head(const int8_t* W, const float* s_row, int V, int d) {
 }
 
 int enqueue_embed(const int8_t* W, const float* s_row, int V, int d, const int32_t* token, float* h,
-                  cudaStream_t s) {
-  int* status = nullptr;
-  const int st = dfssm::stream_status_word(&status);
-  if (st) return st;
+                  int* status, cudaStream_t s) {
   dfssm::EmbedArgs ea{W, s_row, V, d, token, h, status};
   const cudaError_t e = dfssm::launch_embed(ea, s);
   return e == cudaSuccess ? DFSSM_OK : cuda_fail(e);
@@ -188,9 +170,9 @@ int layer_decode_impl(const dfssm_layer_t* layers, int n_layers, const dfssm_dim
   if (!aligned(hidden, 16)) return DFSSM_EALIGN;
   for (int l = 0; l < n_layers; ++l) {
     const dfssm_layer_t& Ly = layers[l];
-    int st = check_linear(&Ly.in_proj);
+    int st = dfssm::check_linear(&Ly.in_proj);
     if (st) return st;
-    st = check_linear(&Ly.out_proj);
+    st = dfssm::check_linear(&Ly.out_proj);
     if (st) return st;
     if (Ly.in_proj.d_out != d_ip || Ly.in_proj.d_in != Dm || Ly.out_proj.d_out != Dm ||
         Ly.out_proj.d_in != E)
@@ -283,6 +265,35 @@ int layer_decode_impl(const dfssm_layer_t* layers, int n_layers, const dfssm_dim
 
 }  // namespace
 
+// Argument checks of one linear descriptor: d_in a multiple of 32 (above 8192: unsupported), rank 0..16,
+// the pointers present and aligned as the header states.
+int dfssm::check_linear(const dfssm_linear_t* L) {
+  if (!L) return DFSSM_EINVAL;
+  if (L->d_out < 1 || L->d_in < 32 || L->d_in % 32 != 0) return DFSSM_EINVAL;
+  if (L->d_in > 8192) return DFSSM_EUNSUPPORTED;
+  if (L->rank < 0 || L->rank > DFSSM_MAX_RANK) return DFSSM_EINVAL;
+  if (!L->bits || !L->w_scale) return DFSSM_EINVAL;
+  if (L->rank > 0 && (!L->lora_b || !L->lora_b_scale || !L->lora_a || !L->lora_a_scale))
+    return DFSSM_EINVAL;
+  if (!aligned(L->bits, 16) || !aligned(L->w_scale, 4)) return DFSSM_EALIGN;
+  if (L->rank > 0) {
+    if (!aligned(L->lora_b, 4) || !aligned(L->lora_b_scale, 4) || !aligned(L->lora_a_scale, 4))
+      return DFSSM_EALIGN;
+    if (L->rank == DFSSM_MAX_RANK && !aligned(L->lora_a, 16)) return DFSSM_EALIGN;
+  }
+  return DFSSM_OK;
+}
+
+int dfssm::read_status_word(int* word, cudaStream_t st, int* code) {
+  int h = 0;
+  cudaError_t e = cudaMemcpyAsync(&h, word, sizeof(int), cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e == cudaSuccess) e = cudaMemsetAsync(word, 0, sizeof(int), st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  *code = h;
+  return e == cudaSuccess ? 0 : (int)e;
+}
+
 int dfssm::record_cuda_failure(cudaError_t e) { return cuda_fail(e); }
 
 extern "C" {
@@ -332,6 +343,9 @@ size_t dfssm_workspace_size(int op, int a, int b, int c) {
     case DFSSM_OP_LAYER_PREFILL:
       if (a < 1 || b < 128 || b % 128 || b > 8192 || c < 128 || c % 128 || c > 8192) return 0;
       return prefill_layer_ws(a, b, c).total;
+    case DFSSM_OP_LINEAR_MULTI:
+    case DFSSM_OP_EMBED:
+      return dfssm::kStatusBytes;
     default: return 0;
   }
 }
@@ -352,7 +366,7 @@ int dfssm_pack_signs(const int8_t* signs, int d_out, int d_in, uint32_t* bits) {
 
 int dfssm_linear_decode(const dfssm_linear_t* lin, const float* x, int B, float* y, void* workspace,
                         size_t ws_bytes, const dfssm_debug_t* dbg, void* stream) {
-  int st = check_linear(lin);
+  int st = dfssm::check_linear(lin);
   if (st) return st;
   if (!x || !y || B < 1) return DFSSM_EINVAL;
   if (B > DFSSM_MAX_BATCH) return DFSSM_EUNSUPPORTED;
@@ -361,8 +375,10 @@ int dfssm_linear_decode(const dfssm_linear_t* lin, const float* x, int B, float*
     return DFSSM_EWORKSPACE;
   if (!device_ok()) return DFSSM_EDEVICE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (dfssm::stream_supported(lin->d_in, B)) return dfssm::launch_linear_stream(lin, 1, x, B, &y, dbg, s);
-  dfssm::QuantScratch qs = dfssm::carve_quant_scratch(workspace, B, lin->d_in);
+  if (dfssm::stream_supported(lin->d_in, B))
+    return dfssm::launch_linear_stream(lin, 1, x, B, &y, dbg, static_cast<int*>(workspace), s);
+  dfssm::QuantScratch qs =
+      dfssm::carve_quant_scratch(static_cast<char*>(workspace) + dfssm::kStatusBytes, B, lin->d_in);
   dfssm::QuantArgs qa{};
   qa.x = x;
   qa.ldx = lin->d_in;
@@ -391,11 +407,11 @@ int dfssm_linear_decode(const dfssm_linear_t* lin, const float* x, int B, float*
 }
 
 int dfssm_linear_decode_multi(const dfssm_linear_t* lins, int n, const float* x, int B, float* const* ys,
-                              void* stream) {
+                              void* workspace, size_t ws_bytes, void* stream) {
   if (!lins || !ys || !x || n < 1 || B < 1) return DFSSM_EINVAL;
   if (n > DFSSM_MAX_LAYERS) return DFSSM_EUNSUPPORTED;
   for (int j = 0; j < n; ++j) {
-    const int st = check_linear(&lins[j]);
+    const int st = dfssm::check_linear(&lins[j]);
     if (st) return st;
     if (lins[j].d_in != lins[0].d_in) return DFSSM_EINVAL;
     if (!ys[j]) return DFSSM_EINVAL;
@@ -403,8 +419,10 @@ int dfssm_linear_decode_multi(const dfssm_linear_t* lins, int n, const float* x,
   }
   if (!dfssm::stream_supported(lins[0].d_in, B)) return DFSSM_EUNSUPPORTED;
   if (!aligned(x, 16)) return DFSSM_EALIGN;
+  if (!workspace || !aligned(workspace, 256) || ws_bytes < dfssm::kStatusBytes) return DFSSM_EWORKSPACE;
   if (!device_ok()) return DFSSM_EDEVICE;
-  return dfssm::launch_linear_stream(lins, n, x, B, ys, nullptr, static_cast<cudaStream_t>(stream));
+  return dfssm::launch_linear_stream(lins, n, x, B, ys, nullptr, static_cast<int*>(workspace),
+                                     static_cast<cudaStream_t>(stream));
 }
 
 int dfssm_conv_step(float* conv_state, const float* w, const float* b, const float* x_in, float* x_out,
@@ -460,23 +478,16 @@ int dfssm_device_status(void* workspace, void* stream) {
   if (workspace && !aligned(workspace, 256)) return DFSSM_EWORKSPACE;
   if (!device_ok()) return DFSSM_EDEVICE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  int code = 0;
-  if (workspace) {
-    const int e = dfssm::read_device_error(workspace, s, &code);
-    if (e) return cuda_fail(static_cast<cudaError_t>(e));
+  int* word = static_cast<int*>(workspace);
+  if (!word) {
+    const int st = dfssm::noalloc_status_word(&word);
+    if (st) return st;
   }
-  // the streaming linear kernels' module status word
-  int* word = nullptr;
-  const int st = dfssm::stream_status_word(&word);
-  if (st) return st;
-  int h = 0;
-  cudaError_t e = cudaMemcpyAsync(&h, word, sizeof(int), cudaMemcpyDeviceToHost, s);
-  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
-  if (e == cudaSuccess) e = cudaMemsetAsync(word, 0, sizeof(int), s);
-  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
-  if (e != cudaSuccess) return cuda_fail(e);
-  if (code == 0 && h == dfssm::kBadTokenCode) return DFSSM_EINVAL;
-  return (code || h) ? DFSSM_ETIMEOUT : DFSSM_OK;
+  int code = 0;
+  const int e = dfssm::read_status_word(word, s, &code);
+  if (e) return cuda_fail(static_cast<cudaError_t>(e));
+  if (code == dfssm::kBadTokenCode) return DFSSM_EINVAL;
+  return code ? DFSSM_ETIMEOUT : DFSSM_OK;
 }
 
 int dfssm_selftest_timeout(void* workspace, size_t ws_bytes, void* stream) {
@@ -503,13 +514,15 @@ int dfssm_lm_head(const int8_t* W, const float* s_row, int V, int d, const float
 }
 
 int dfssm_embed(const int8_t* W, const float* s_row, int V, int d, const int32_t* token, float* h,
-                void* stream) {
+                void* workspace, size_t ws_bytes, void* stream) {
   int st = check_head(W, s_row, V, d);
   if (st) return st;
   if (!token || !h) return DFSSM_EINVAL;
   if (!aligned(token, 4) || !aligned(h, 16)) return DFSSM_EALIGN;
+  if (!workspace || !aligned(workspace, 256) || ws_bytes < dfssm::kStatusBytes) return DFSSM_EWORKSPACE;
   if (!device_ok()) return DFSSM_EDEVICE;
-  return enqueue_embed(W, s_row, V, d, token, h, static_cast<cudaStream_t>(stream));
+  return enqueue_embed(W, s_row, V, d, token, h, static_cast<int*>(workspace),
+                       static_cast<cudaStream_t>(stream));
 }
 
 int dfssm_head_greedy(const int8_t* W, const float* s_row, int V, int d, const float* h,
@@ -548,7 +561,7 @@ int dfssm_generate(const dfssm_layer_t* layers, int n_layers, const dfssm_dims_t
   if (st) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   for (int t = 0; t < n_tokens; ++t) {
-    st = enqueue_embed(W, s_row, V, Dm, tokens + t, hidden, s);
+    st = enqueue_embed(W, s_row, V, Dm, tokens + t, hidden, reinterpret_cast<int*>(base + g.layer), s);
     if (st) return st;
     st = layer_decode_impl(layers, n_layers, dims, hidden, conv_states, ssm_states, 1, base + g.layer,
                            g.hidden, stream, true);
@@ -586,9 +599,9 @@ int dfssm_layer_prefill(const dfssm_layer_t* layers, int n_layers, const dfssm_d
   if (!aligned(hidden, 16)) return DFSSM_EALIGN;
   for (int l = 0; l < n_layers; ++l) {
     const dfssm_layer_t& Ly = layers[l];
-    int st = check_linear(&Ly.in_proj);
+    int st = dfssm::check_linear(&Ly.in_proj);
     if (st) return st;
-    st = check_linear(&Ly.out_proj);
+    st = dfssm::check_linear(&Ly.out_proj);
     if (st) return st;
     if (Ly.in_proj.d_out != d_ip || Ly.in_proj.d_in != Dm || Ly.out_proj.d_out != Dm ||
         Ly.out_proj.d_in != E)

@@ -110,7 +110,7 @@ constexpr int OFF_OUT_SET = 2 * IN_SET;
 constexpr int OFF_STATE = OFF_OUT_SET + OUT_SET;
 constexpr int DYN_BYTES = OFF_STATE + 2 * ST_BYTES;
 
-constexpr int kTimeoutMagic = 0x7E0D1E57;
+constexpr int kTimeoutMagic = kDeviceTimeout;
 
 // ------------------------------------------------------------------------------ tagged exchange
 
@@ -971,18 +971,6 @@ cudaError_t launch_timeout_selftest(void* ws, cudaStream_t st, long long spin_li
   if (e != cudaSuccess) return e;
   fused::timeout_selftest_kernel<<<1, 32, 0, st>>>(word, err, status, spin_limit);
   return cudaGetLastError();
-}
-
-int read_device_error(void* ws, cudaStream_t st, int* code) {
-  char* base = static_cast<char*>(ws);
-  int* status = reinterpret_cast<int*>(base + fused::OFF_STATUS);
-  int h = 0;
-  cudaError_t e = cudaMemcpyAsync(&h, status, sizeof(int), cudaMemcpyDeviceToHost, st);
-  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
-  if (e == cudaSuccess) e = cudaMemsetAsync(status, 0, sizeof(int), st);
-  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
-  *code = (h == fused::kTimeoutMagic) ? 1 : 0;
-  return e == cudaSuccess ? 0 : (int)e;
 }
 
 }  // namespace dfssm

@@ -130,9 +130,15 @@ struct Int8GemvArgs {
 };
 cudaError_t launch_int8_gemv(const Int8GemvArgs& a, cudaStream_t st);
 
+// Codes a kernel leaves in a device status word (the first word of a call's workspace, or the no-alloc
+// entry point's module word): a bounded wait ran out of its budget, or an embedding id was out of range.
+constexpr int kDeviceTimeout = 0x7E0D1E57;
+constexpr int kBadTokenCode = 0x70CE1D;
+// Every workspace that carries a status word keeps it in its first kStatusBytes.
+constexpr size_t kStatusBytes = 256;
+
 // Embedding row lookup from the tied int8 matrix: h[i] = fl32(W[tok, i] * s_row[tok]), tok = *token.
 // An id outside [0, V) writes zeros and sets *status to kBadTokenCode.
-constexpr int kBadTokenCode = 0x70CE1D;
 struct EmbedArgs {
   const int8_t* W;
   const float* s_row;
@@ -171,14 +177,17 @@ cudaError_t launch_fused_decode(const dfssm_layer_t* layers, int n_layers, float
                                 cudaStream_t st, long long spin_limit);
 // Launches a kernel that waits on a counter nothing increments, with the given clock budget.
 cudaError_t launch_timeout_selftest(void* ws, cudaStream_t st, long long spin_limit);
-// Reads and clears the device error word of a fused-decode workspace region (synchronises st).
-int read_device_error(void* ws, cudaStream_t st, int* code);
-// Streaming decode of n linears that share x (B <= 4, d_in = 128 * 2^k <= 8192): one persistent launch.
+// Streaming decode of n linears that share x (B <= 16 at d_in 1024/2048/4096, B <= 4 at 8192): one
+// persistent launch; a wait that runs out of budget stores kDeviceTimeout in *status.
 bool stream_supported(int d_in, int B);
 int launch_linear_stream(const dfssm_linear_t* lins, int n, const float* x, int B, float* const* ys,
-                         const dfssm_debug_t* dbg, cudaStream_t st);
-// Device address of the streaming kernels' status word on the current device.
-int stream_status_word(int** out);
+                         const dfssm_debug_t* dbg, int* status, cudaStream_t st);
+// Reads and clears a device status word (synchronises st); *code = the word's value.
+int read_status_word(int* word, cudaStream_t st, int* code);
+// The no-alloc entry point's module status word on the current device.
+int noalloc_status_word(int** out);
+// Argument checks shared by the linear entry points (DFSSM_OK or the status to return).
+int check_linear(const dfssm_linear_t* L);
 // Records e as the text returned by dfssm_last_cuda_error (this thread) and returns DFSSM_ECUDA.
 int record_cuda_failure(cudaError_t e);
 }  // namespace dfssm

@@ -17,7 +17,9 @@
 // In host code the array's name is only a host-side stand-in, not a device address.  The device address
 // is looked up with cudaGetSymbolAddress the first time this entry point runs on a device (with that
 // device current) and cached; that first call on each device should therefore come before any stream
-// capture.
+// capture, and the library must not be used across a cudaDeviceReset of that device.  A timed-out wait
+// of the streaming kernel on this path is recorded in a module status word beside the array (read by
+// dfssm_device_status with a NULL workspace).
 
 #include <cstdio>
 #include <mutex>
@@ -34,6 +36,9 @@ constexpr int kMaxDin = 8192;
 constexpr size_t kScratchBytes = (size_t)kMaxTokens * kMaxDin + 256 + 256 + 1024;
 
 static __device__ __align__(256) unsigned char g_linear_scratch[kScratchBytes];
+// This entry point's status word (a timed-out wait of the streaming kernel; read and cleared by
+// dfssm_device_status with a NULL workspace).
+static __device__ int g_noalloc_status;
 
 constexpr int kMaxDevices = 64;
 void* g_scratch_addr[kMaxDevices] = {};
@@ -41,8 +46,11 @@ std::mutex g_scratch_mu;
 
 bool aligned_to(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
-// Device address of g_linear_scratch on the current device (looked up once per device).
-int scratch_address(void** out) {
+void* g_status_addr[kMaxDevices] = {};
+
+// Device addresses of g_linear_scratch and g_noalloc_status on the current device (looked up once per
+// device; the cache assumes the device's context lives as long as the process: no cudaDeviceReset).
+int module_addresses(void** scratch, int** status) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return dfssm::record_cuda_failure(e);
@@ -50,37 +58,25 @@ int scratch_address(void** out) {
   std::lock_guard<std::mutex> lock(g_scratch_mu);
   if (g_scratch_addr[dev] == nullptr) {
     void* p = nullptr;
+    void* q = nullptr;
     e = cudaGetSymbolAddress(&p, g_linear_scratch);
+    if (e == cudaSuccess) e = cudaGetSymbolAddress(&q, g_noalloc_status);
     if (e != cudaSuccess) return dfssm::record_cuda_failure(e);
     g_scratch_addr[dev] = p;
+    g_status_addr[dev] = q;
   }
-  *out = g_scratch_addr[dev];
-  return DFSSM_OK;
-}
-
-int check_linear_args(const dfssm_linear_t* L) {
-  if (!L) return DFSSM_EINVAL;
-  if (L->d_out < 1 || L->d_in < 32 || L->d_in % 32 != 0) return DFSSM_EINVAL;
-  if (L->d_in > kMaxDin) return DFSSM_EUNSUPPORTED;
-  if (L->rank < 0 || L->rank > DFSSM_MAX_RANK) return DFSSM_EINVAL;
-  if (!L->bits || !L->w_scale) return DFSSM_EINVAL;
-  if (L->rank > 0 && (!L->lora_b || !L->lora_b_scale || !L->lora_a || !L->lora_a_scale))
-    return DFSSM_EINVAL;
-  if (!aligned_to(L->bits, 16) || !aligned_to(L->w_scale, 4)) return DFSSM_EALIGN;
-  if (L->rank > 0) {
-    if (!aligned_to(L->lora_b, 4) || !aligned_to(L->lora_b_scale, 4) ||
-        !aligned_to(L->lora_a_scale, 4))
-      return DFSSM_EALIGN;
-    if (L->rank == DFSSM_MAX_RANK && !aligned_to(L->lora_a, 16)) return DFSSM_EALIGN;
-  }
+  if (scratch) *scratch = g_scratch_addr[dev];
+  if (status) *status = static_cast<int*>(g_status_addr[dev]);
   return DFSSM_OK;
 }
 
 }  // namespace
 
+int dfssm::noalloc_status_word(int** out) { return module_addresses(nullptr, out); }
+
 extern "C" int dfssm_linear_decode_noalloc(const dfssm_linear_t* lin, const float* x, int B, float* y,
                                            const dfssm_debug_t* dbg, void* stream) {
-  int st = check_linear_args(lin);
+  int st = dfssm::check_linear(lin);
   if (st) return st;
   if (!x || !y || B < 1) return DFSSM_EINVAL;
   if (B > kMaxTokens) return DFSSM_EUNSUPPORTED;
@@ -92,11 +88,13 @@ extern "C" int dfssm_linear_decode_noalloc(const dfssm_linear_t* lin, const floa
       major != 10)
     return DFSSM_EDEVICE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  // in the streaming kernel's range the single kernel needs no scratch at all
-  if (dfssm::stream_supported(lin->d_in, B)) return dfssm::launch_linear_stream(lin, 1, x, B, &y, dbg, s);
   void* scratch = nullptr;
-  st = scratch_address(&scratch);
+  int* status = nullptr;
+  st = module_addresses(&scratch, &status);
   if (st) return st;
+  // in the streaming kernel's range the single kernel needs no scratch (only the status word)
+  if (dfssm::stream_supported(lin->d_in, B))
+    return dfssm::launch_linear_stream(lin, 1, x, B, &y, dbg, status, s);
 
   const dfssm::QuantScratch qs = dfssm::carve_quant_scratch(scratch, B, lin->d_in);
   dfssm::QuantArgs qa{};

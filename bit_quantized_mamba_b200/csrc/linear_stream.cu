@@ -26,11 +26,9 @@
 // The sign bits are immutable weights, so the producer starts streaming before the kernel waits on the
 // preceding kernel of the stream (programmatic dependent launch).
 //
-// Every mbarrier wait is bounded.  A wait that runs out of budget stores a timeout code in the module's
-// status word (read and cleared by dfssm_device_status); the CTA then stops computing, still waits
-// (bounded) for every copy it issued, and returns.
-
-#include <mutex>
+// Every mbarrier wait is bounded.  A wait that runs out of budget stores a timeout code in the call's
+// status word (the first word of its workspace; read and cleared by dfssm_device_status); the CTA then
+// stops computing, still waits (bounded) for every copy it issued, and returns.
 
 #include "common.cuh"
 #include "internal.h"
@@ -76,7 +74,7 @@ __host__ __device__ constexpr PLayout p_layout(int din, int bt, int tb) {
 }
 constexpr int MAX_LIN = DFSSM_MAX_LAYERS;
 constexpr long long kWaitBudget = 2000000000LL;  // clock cycles per wait (~1 s)
-constexpr int kTimeoutCode = 0x5EA0715E;
+constexpr int kTimeoutCode = kDeviceTimeout;
 
 struct Lin {
   const uint32_t* bits;
@@ -915,8 +913,6 @@ __global__ void __launch_bounds__(NT, 1) stream_kernel(const __grid_constant__ P
   }
 }
 
-// Module status word: kTimeoutCode after a wait ran out of budget (sticky until read).
-static __device__ int g_stream_status;
 
 template <int LPR, int NSEG, int BT, int TB>
 cudaError_t launch_t(const Params& p, int grid, cudaStream_t st) {
@@ -959,26 +955,8 @@ bool stream_supported(int d_in, int B) {
   return d_in == 1024 || d_in == 2048 || d_in == 4096;  // 16 token slots of codes must fit beside the rings
 }
 
-int stream_status_word(int** out) {
-  static std::mutex mu;
-  static int* addr[64] = {};
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return record_cuda_failure(e);
-  if (dev < 0 || dev >= 64) return DFSSM_EUNSUPPORTED;
-  std::lock_guard<std::mutex> lock(mu);
-  if (!addr[dev]) {
-    void* a = nullptr;
-    e = cudaGetSymbolAddress(&a, stream::g_stream_status);
-    if (e != cudaSuccess) return record_cuda_failure(e);
-    addr[dev] = static_cast<int*>(a);
-  }
-  *out = addr[dev];
-  return DFSSM_OK;
-}
-
 int launch_linear_stream(const dfssm_linear_t* lins, int n, const float* x, int B, float* const* ys,
-                         const dfssm_debug_t* dbg, cudaStream_t st) {
+                         const dfssm_debug_t* dbg, int* status, cudaStream_t st) {
   stream::Params p;
   const int d_in = lins[0].d_in;
   // tile size: 32 KB with one token slot when 16 KB tiles would outnumber the SMs, else 16 KB
@@ -1014,8 +992,7 @@ int launch_linear_stream(const dfssm_linear_t* lins, int n, const float* x, int 
   p.dbg_s = dbg ? dbg->xscale : nullptr;
   p.dbg_t = dbg ? dbg->lora_t : nullptr;
   p.dbg_acc = dbg ? dbg->acc : nullptr;
-  int st_rc = stream_status_word(&p.status);
-  if (st_rc) return st_rc;
+  p.status = status;
   const int grid = tiles < num_sms() ? tiles : num_sms();
   const cudaError_t e = B == 1   ? (tb == 32768 ? stream::dispatch<1, 32768>(p, grid, st)
                                                 : stream::dispatch<1, 16384>(p, grid, st))

@@ -21,6 +21,8 @@ OP_LM_HEAD = 4
 OP_HEAD_GREEDY = 5
 OP_GENERATE = 6
 OP_LAYER_PREFILL = 7
+OP_LINEAR_MULTI = 8
+OP_EMBED = 9
 MAX_RANK = 16
 MAX_BATCH = 16
 MAX_LAYERS = 64
@@ -69,13 +71,13 @@ SIGNATURES = {
     "dfssm_linear_decode": (_I, [_P, _P, _I, _P, _P, _Z, _P, _P]),
     "dfssm_linear_prefill": (_I, [_P, _P, _I, _P, _P, _Z, _P, _P]),
     "dfssm_linear_decode_noalloc": (_I, [_P, _P, _I, _P, _P, _P]),
-    "dfssm_linear_decode_multi": (_I, [_P, _I, _P, _I, _P, _P]),
+    "dfssm_linear_decode_multi": (_I, [_P, _I, _P, _I, _P, _P, C.c_size_t, _P]),
     "dfssm_conv_step": (_I, [_P, _P, _P, _P, _P, _I, _I, _P]),
     "dfssm_ssm_step": (_I, [_P] * 9 + [_I] * 5 + [_P]),
     "dfssm_layer_decode": (_I, [_P, _I, _P, _P, _P, _P, _I, _P, _Z, _P]),
     "dfssm_lm_head": (_I, [_P, _P, _I, _I, _P, _P, _P, _P, _Z, _P]),
     "dfssm_layer_prefill": (_I, [_P, _I, _P, _P, _P, _P, _I, _P, _Z, _P]),
-    "dfssm_embed": (_I, [_P, _P, _I, _I, _P, _P, _P]),
+    "dfssm_embed": (_I, [_P, _P, _I, _I, _P, _P, _P, C.c_size_t, _P]),
     "dfssm_head_greedy": (_I, [_P, _P, _I, _I, _P, _P, _P, _P, _P, _P, _Z, _P]),
     "dfssm_generate": (_I, [_P, _I, _P, _P, _P, _I, _P, _P, _I, _P, _P, _P, _P, _P, _Z, _P]),
     "dfssm_pack_signs": (_I, [_P, _I, _I, _P]),
@@ -192,15 +194,18 @@ def linear_decode_noalloc(lin: Linear, x: torch.Tensor, y: torch.Tensor | None =
     return y
 
 
-def linear_decode_multi(lins, x: torch.Tensor, ys=None, stream=None):
-    """n linears that share x in one launch (dfssm_linear_decode_multi); returns the list of outputs."""
+def linear_decode_multi(lins, x: torch.Tensor, ys=None, ws=None, stream=None):
+    """n linears that share x in one launch (dfssm_linear_decode_multi); returns the list of outputs.
+    ws (optional) holds the call's status word."""
     B = x.shape[0]
     if ys is None:
         ys = [torch.empty((B, L.d_out), dtype=torch.float32, device=x.device) for L in lins]
+    if ws is None:
+        ws = workspace(workspace_size(OP_LINEAR_MULTI, 0, 0, 0), x.device)
     arr = (LinearT * len(lins))(*[L.cstruct() for L in lins])
     ptrs = (C.c_void_p * len(lins))(*[_ptr(y) for y in ys])
     _check("dfssm_linear_decode_multi", lib().dfssm_linear_decode_multi(
-        arr, len(lins), _ptr(x), B, ptrs, _stream(stream)))
+        arr, len(lins), _ptr(x), B, ptrs, _ptr(ws), ws.numel(), _stream(stream)))
     return ys
 
 
@@ -302,8 +307,9 @@ def layer_prefill(stack: LayerStack, hidden: torch.Tensor, ws=None, stream=None)
 
 
 def device_status(ws=None, stream=None) -> int:
-    """Synchronise the stream, read and clear the device error words (the workspace's, if given, and
-    the library's own): 0 (DFSSM_OK), -5 (DFSSM_ETIMEOUT) or -1 (DFSSM_EINVAL: a bad token id)."""
+    """Synchronise the stream, read and clear the status word at the start of the workspace (None: the
+    no-alloc entry point's module word): 0 (DFSSM_OK), -5 (DFSSM_ETIMEOUT) or -1 (DFSSM_EINVAL: a bad
+    token id)."""
     return int(lib().dfssm_device_status(_ptr(ws), _stream(stream)))
 
 
@@ -323,13 +329,16 @@ def lm_head(W, s_row, x, logits=None, acc=None, ws=None, stream=None):
     return logits
 
 
-def embed(W, s_row, token, h=None, stream=None):
-    """Row token[0] of the tied int8 embedding, dequantized (token: device int32 [1])."""
+def embed(W, s_row, token, h=None, ws=None, stream=None):
+    """Row token[0] of the tied int8 embedding, dequantized (token: device int32 [1]).  ws (optional)
+    holds the call's status word (an out-of-range id is reported there)."""
     V, d = W.shape
     if h is None:
         h = torch.empty(d, dtype=torch.float32, device=W.device)
-    _check("dfssm_embed", lib().dfssm_embed(_ptr(W), _ptr(s_row), V, d, _ptr(token), _ptr(h),
-                                            _stream(stream)))
+    if ws is None:
+        ws = workspace(workspace_size(OP_EMBED, 0, 0, 0), W.device)
+    _check("dfssm_embed", lib().dfssm_embed(_ptr(W), _ptr(s_row), V, d, _ptr(token), _ptr(h), _ptr(ws),
+                                            ws.numel(), _stream(stream)))
     return h
 
 

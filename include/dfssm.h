@@ -11,16 +11,24 @@
  *
  * Conventions for every entry point:
  *   - Pointers documented as "device" must point to memory of the current CUDA device.  The caller owns
- *     every buffer; the library allocates no device memory.  Scratch comes from a caller-provided
- *     workspace of at least dfssm_workspace_size(...) bytes, 256-byte aligned.
+ *     every buffer, and the library calls no allocating routine.  Scratch comes from a caller-provided
+ *     workspace of at least dfssm_workspace_size(...) bytes, 256-byte aligned, zero-filled before its
+ *     first use.  The one exception is dfssm_linear_decode_noalloc, which keeps its scratch and status
+ *     word in fixed arrays of the library's own device memory.
+ *   - Device-side errors (a wait that ran out of its clock budget, an embedding id out of range) are
+ *     recorded in a status word at the start of the call's workspace (for dfssm_linear_decode,
+ *     dfssm_linear_decode_multi, dfssm_embed, dfssm_layer_decode and dfssm_generate), read and cleared
+ *     by dfssm_device_status.
  *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy default stream).  Inputs
  *     must not be modified, and outputs not read, until the stream reaches the call.  Weights and
  *     parameters must be fully written before the call is enqueued (kernels may read them before they
  *     wait on the preceding kernel of the stream).
  *   - Arguments are validated before anything is launched; on a negative status nothing was enqueued.
- *   - Calls that share a workspace must not overlap on the GPU.  The library keeps no global state
- *     beyond cached device attributes, so calls on different streams with different workspaces may run
- *     concurrently.
+ *   - Concurrency: calls that share a workspace must not overlap on the GPU.  The library's only state
+ *     outside the caller's buffers is per-device and set once (the kernels' shared-memory attribute and
+ *     the SM count, guarded by a mutex) plus the no-alloc entry point's module arrays; so calls on
+ *     different streams with different workspaces may run concurrently, from any host threads.  A
+ *     cudaDeviceReset invalidates those per-device records: do not use the library after one.
  *   - fp32 values that feed an int8 quantizer are computed as single correctly rounded fp32 operations,
  *     with sums and transcendental functions evaluated in fp64 and rounded once, so that quantization
  *     codes are reproducible by a plain CPU evaluation of the same definitions.
@@ -35,7 +43,7 @@
 extern "C" {
 #endif
 
-#define DFSSM_ABI_VERSION 3
+#define DFSSM_ABI_VERSION 4
 #define DFSSM_MAX_RANK 16
 #define DFSSM_MAX_BATCH 16
 #define DFSSM_MAX_LAYERS 64
@@ -60,7 +68,8 @@ typedef enum {
  *   lora_b_scale  device f32 [rank]    per-row scale of W_B
  *   lora_a        device i8  [d_out][rank]  W_A, row-major
  *   lora_a_scale  device f32 [d_out]   per-row scale of W_A
- * Constraints: d_in % 32 == 0, d_in <= 8192, d_out >= 1, 0 <= rank <= 16.  rank == 0 means no LoRA
+ * Constraints: d_in % 32 == 0, d_out >= 1, 0 <= rank <= 16 (otherwise DFSSM_EINVAL); d_in <= 8192
+ * (otherwise DFSSM_EUNSUPPORTED).  rank == 0 means no LoRA
  * (lora_* may then be NULL).
  * Computes, for each token b with input x and (q, s) its per-token int8 quantization:
  *   acc[o] = sum_i sign(o,i) q[i]  (int32, exact)
@@ -95,7 +104,9 @@ enum {
   DFSSM_OP_LM_HEAD = 4,        /* a = 1,  b = d,     c = V                             */
   DFSSM_OP_HEAD_GREEDY = 5,    /* a = 1,  b = d,     c = V                             */
   DFSSM_OP_GENERATE = 6,       /* a = V,  b = d_model, c = d_inner                     */
-  DFSSM_OP_LAYER_PREFILL = 7   /* a = M,  b = d_model, c = d_inner                     */
+  DFSSM_OP_LAYER_PREFILL = 7,  /* a = M,  b = d_model, c = d_inner                     */
+  DFSSM_OP_LINEAR_MULTI = 8,   /* (no size arguments): the status word only             */
+  DFSSM_OP_EMBED = 9           /* (no size arguments): the status word only             */
 };
 size_t dfssm_workspace_size(int op, int a, int b, int c);
 
@@ -104,9 +115,9 @@ size_t dfssm_workspace_size(int op, int a, int b, int c);
  *   x   device f32 [B][d_in] (16-byte aligned),  y device f32 [B][d_out]
  *   1 <= B <= 16.  dbg may be NULL.  workspace: dfssm_workspace_size(DFSSM_OP_LINEAR_DECODE, B, d_in, d_out).
  * For d_in in {1024, 2048, 4096} (any B <= 16) and d_in = 8192 with B <= 4 the call is one kernel that
- * quantizes x in every CTA and streams the sign bits through shared memory; the workspace is then left
- * untouched.  Otherwise a
- * quantize kernel writes the codes into the workspace and a GEMV kernel reads them.
+ * quantizes x in every CTA and streams the sign bits through shared memory; only the workspace's status
+ * word is used then.  Otherwise a quantize kernel writes the codes into the workspace and a GEMV kernel
+ * reads them.
  */
 int dfssm_linear_decode(const dfssm_linear_t* lin, const float* x, int B, float* y, void* workspace,
                         size_t ws_bytes, const dfssm_debug_t* dbg, void* stream);
@@ -119,10 +130,11 @@ int dfssm_linear_decode(const dfssm_linear_t* lin, const float* x, int B, float*
  *   x     device f32 [B][d_in] (16-byte aligned);  ys host array of n device pointers, ys[j] f32 [B][d_out_j]
  *   1 <= n <= 64; d_in in {1024, 2048, 4096} with 1 <= B <= 16, or d_in = 8192 with 1 <= B <= 4; other
  *   sizes return DFSSM_EUNSUPPORTED.
- * No workspace.  The outputs must not overlap each other or x.
+ *   workspace: dfssm_workspace_size(DFSSM_OP_LINEAR_MULTI, 0, 0, 0) bytes (the status word).
+ * The outputs must not overlap each other or x.
  */
 int dfssm_linear_decode_multi(const dfssm_linear_t* lins, int n, const float* x, int B, float* const* ys,
-                              void* stream);
+                              void* workspace, size_t ws_bytes, void* stream);
 
 /*
  * dfssm_linear_decode for callers that cannot allocate device memory.  The paper has no counterpart: this
@@ -136,9 +148,12 @@ int dfssm_linear_decode_multi(const dfssm_linear_t* lins, int n, const float* x,
  *   streaming kernel's range (d_in in {1024, 2048, 4096}, or d_in = 8192 with B <= 4) run that kernel and
  *   use no scratch.
  *   Set-up: the first call on a device looks up that array's device address (cudaGetSymbolAddress, with
- *   that device current) and caches it; make that first call before any stream capture.
+ *   that device current) and caches it; make that first call before any stream capture, and do not use
+ *   the library across a cudaDeviceReset of that device.
  *   Sharing: all calls on a device use the same array.  Each call writes everything it reads there, so
  *   nothing needs clearing, but calls that overlap on the GPU (unordered streams) race: order them.
+ *   Status: a timed-out wait is recorded in a module status word beside the array, read and cleared by
+ *   dfssm_device_status(NULL, stream).
  */
 int dfssm_linear_decode_noalloc(const dfssm_linear_t* lin, const float* x, int B, float* y,
                                 const dfssm_debug_t* dbg, void* stream);
@@ -250,18 +265,19 @@ int dfssm_lm_head(const int8_t* W, const float* s_row, int V, int d, const float
  *   W device i8 [V][d] (16-byte aligned, d % 16 == 0, d <= 8192), s_row device f32 [V],
  *   token device i32 [1] (read on the device when the stream reaches the call), h device f32 [d]
  *   (16-byte aligned).   h[i] = fl32(W[tok, i] * s_row[tok]).
- * A token outside [0, V) writes h = 0 and records a sticky code in the library's status word:
- * dfssm_device_status then returns DFSSM_EINVAL.  One single-CTA kernel.
+ * A token outside [0, V) writes h = 0 and records a sticky code in the workspace's status word:
+ * dfssm_device_status(workspace) then returns DFSSM_EINVAL.  One single-CTA kernel.
+ *   workspace: dfssm_workspace_size(DFSSM_OP_EMBED, 0, 0, 0) bytes (the status word).
  */
 int dfssm_embed(const int8_t* W, const float* s_row, int V, int d, const int32_t* token, float* h,
-                void* stream);
+                void* workspace, size_t ws_bytes, void* stream);
 
 /*
  * Final RMSNorm + int8 LM head + greedy choice on one token (the Mamba-2 language model's final norm
  * before its LM head, a reading of the cited architecture; the head as in dfssm_lm_head).
  *   h device f32 [d] (the residual stream after the last layer); norm_w device f32 [d] or NULL (then no
- *   norm: the logits are exactly dfssm_lm_head's).  With norm_w the RMS factor is folded into the
- *   quantizer scale: (q, s0) = quant(fl32(h w)), s = fl32(s0 / sqrt(sum h^2 / d + 1e-5)) (fp64), and
+ *   norm: the logits are exactly dfssm_lm_head's).  With norm_w the token is normalized first:
+ *   r = fl32(1 / sqrt(sum h^2 / d + 1e-5)) (fp64), u = fl32(fl32(h r) w), (q, s) = quant(u), and
  *   logits[v] = fl32(acc[v] s s_row[v]), acc[v] = sum_i W[v,i] q[i].
  *   token device i32 [1] receives the index of the largest logit (the smallest index on ties; -0 and +0
  *   are equal).  logits device f32 [V] (required), acc device i32 [V] or NULL.
@@ -291,21 +307,22 @@ int dfssm_generate(const dfssm_layer_t* layers, int n_layers, const dfssm_dims_t
                    float* hidden_taps, float* logits, void* workspace, size_t ws_bytes, void* stream);
 
 /*
- * Device-side failure detection of dfssm_layer_decode.  The fused decode kernel (batch 1, Mamba-2-1.3B
- * shape) hands data between its CTAs through counters in the workspace; every wait has a clock budget
- * (about one second).  A wait that runs out makes every CTA of that launch return early (its outputs are
- * then incomplete) and records a sticky status word in the workspace; each new launch starts with fresh
- * counters.  The streaming linear kernel (dfssm_linear_decode in its range, dfssm_linear_decode_multi)
- * bound their shared-memory pipeline waits the same way and record a timeout in a status word of the
- * library's own device memory (one per device).  dfssm_device_status synchronises `stream`, reads and
- * clears the workspace status word (workspace may be NULL: then only the library's word) and the
- * library's word, and returns DFSSM_OK, DFSSM_ETIMEOUT, or DFSSM_EINVAL when the only recorded event is
- * an out-of-range token given to dfssm_embed.  No device trap or fault is ever raised.
+ * Device-side failure detection.  The fused decode kernel of dfssm_layer_decode (batch 1, Mamba-2-1.3B
+ * shape) hands data between its CTAs through tagged words in the workspace; every wait has a clock
+ * budget (about one second).  A wait that runs out makes every CTA of that launch return early (its
+ * outputs are then incomplete) and records a sticky code in the workspace's status word; each new launch
+ * starts with fresh tags.  The streaming linear kernel (dfssm_linear_decode in its range,
+ * dfssm_linear_decode_multi) bounds its shared-memory pipeline waits the same way and records a timeout
+ * in the status word of the call's workspace; dfssm_embed records an out-of-range token there.
+ * dfssm_device_status synchronises `stream`, reads and clears the status word at the start of
+ * `workspace` (NULL: the module status word of dfssm_linear_decode_noalloc), and returns DFSSM_OK,
+ * DFSSM_ETIMEOUT, or DFSSM_EINVAL for an out-of-range embedding id.  No device trap or fault is ever
+ * raised.
  */
 int dfssm_device_status(void* workspace, void* stream);
 
-/* Diagnostic: launch a one-warp kernel that waits, with a budget of about 1 ms, on a workspace counter
- * that nothing increments, so that the next dfssm_device_status returns DFSSM_ETIMEOUT.  workspace as
+/* Diagnostic: launch a one-warp kernel that waits, with a budget of about 1 ms, on a workspace word that
+ * nothing writes, so that the next dfssm_device_status returns DFSSM_ETIMEOUT.  workspace as
  * for dfssm_layer_decode. */
 int dfssm_selftest_timeout(void* workspace, size_t ws_bytes, void* stream);
 

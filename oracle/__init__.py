@@ -31,6 +31,8 @@ _I = C.c_int
 
 def _declare(L):
     L.oracle_abi_version.restype = _I
+    L.oracle_set_threads.argtypes = [_I]
+    L.oracle_set_threads.restype = _I
     L.oracle_sign.argtypes = [_P, _I, _I, _I]
     L.oracle_sign.restype = _I
     L.oracle_quantize.argtypes = [_P, _I, _I, _P, _P]
@@ -58,6 +60,12 @@ def _p(a):
 
 def _c(a, dtype):
     return np.ascontiguousarray(a, dtype=dtype)
+
+
+def set_threads(n: int) -> int:
+    """Host threads of the oracle's OpenMP loops (for the CPU-baseline timing); returns the previous
+    maximum.  n <= 0 leaves it unchanged."""
+    return lib().oracle_set_threads(int(n))
 
 
 def sign(bits: np.ndarray, d_in: int, o: int, i: int) -> int:

@@ -28,6 +28,8 @@
 //
 // Parity status per function is stated in each header comment ("pinned by" / "parity unpinned").
 
+#include <omp.h>
+
 #include <cmath>
 #include <cstdint>
 #include <cstdlib>
@@ -129,6 +131,14 @@ inline double silu64(double v) { return v / (1.0 + std::exp(-v)); }
 extern "C" {
 
 int oracle_abi_version(void) { return 5; }
+
+// Host threads the OpenMP loops of this library use (timing of the CPU baseline); returns the previous
+// maximum.  No arithmetic.
+int oracle_set_threads(int n) {
+  const int prev = omp_get_max_threads();
+  if (n > 0) omp_set_num_threads(n);
+  return prev;
+}
 
 // Pinned by: exhaustive byte-pattern round trip against an independent packer, brute force.
 int oracle_sign(const uint32_t* bits, int d_in, int o, int i) { return unpack_sign(bits, d_in, o, i); }

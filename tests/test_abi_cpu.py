@@ -37,7 +37,7 @@ def test_library_exports_every_declared_symbol(L):
     for n in names:
         assert hasattr(L, n), f"{n} declared in dfssm.h but not exported"
     assert set(names) == set(dfssm.SIGNATURES), "binding and header disagree"
-    assert L.dfssm_abi_version() == 3
+    assert L.dfssm_abi_version() == 4
 
 
 def test_status_strings(L):
@@ -56,6 +56,11 @@ def test_workspace_sizes(L):
     gen = dfssm.workspace_size(dfssm.OP_GENERATE, 50288, 2048, 4096)
     assert gen >= dfssm.workspace_size(dfssm.OP_LAYER_DECODE, 1, 2048, 4096) + 4 * (2048 + 50288) + 16
     assert dfssm.workspace_size(dfssm.OP_GENERATE, 0, 2048, 4096) == 0
+    # the status word every workspace starts with
+    assert dfssm.workspace_size(dfssm.OP_LINEAR_MULTI, 0, 0, 0) == 256
+    assert dfssm.workspace_size(dfssm.OP_EMBED, 0, 0, 0) == 256
+    assert (dfssm.workspace_size(dfssm.OP_LINEAR_DECODE, 1, 2048, 8512)
+            >= 256 + 2048 + 16 * 16 * 4)
 
 
 def test_argument_validation_precedes_device_use(L):
@@ -76,9 +81,11 @@ def test_argument_validation_precedes_device_use(L):
     assert L.dfssm_ssm_step(16, 16, 16, 16, 16, 16, 16, 16, 16, 1, 4, 4, 6, 1, None) == -3  # N % 4
     assert L.dfssm_conv_step(None, 16, 16, 16, 16, 1, 8, None) == -1
     assert L.dfssm_lm_head(16, 16, 10, 24, 16, 16, None, 256, 1 << 20, None) == -1  # d % 16
-    assert L.dfssm_embed(16, 16, 10, 24, 16, 16, None) == -1                         # d % 16
-    assert L.dfssm_embed(16, 16, 10, 32, 16, 8, None) == -2                          # h misaligned
-    assert L.dfssm_embed(16, 16, 10, 32, None, 16, None) == -1                       # no token
+    assert L.dfssm_embed(16, 16, 10, 24, 16, 16, 256, 256, None) == -1              # d % 16
+    assert L.dfssm_embed(16, 16, 10, 32, 16, 8, 256, 256, None) == -2               # h misaligned
+    assert L.dfssm_embed(16, 16, 10, 32, None, 16, 256, 256, None) == -1            # no token
+    assert L.dfssm_embed(16, 16, 10, 32, 16, 16, None, 256, None) == -7             # no workspace
+    assert L.dfssm_embed(16, 16, 10, 32, 16, 16, 256, 64, None) == -7               # workspace too small
     assert L.dfssm_head_greedy(16, 16, 10, 32, 16, None, 16, None, 16, None, 256, None) == -7
     assert L.dfssm_head_greedy(16, 16, 10, 32, 16, None, None, None, 16, 256, 256, None) == -1
     assert L.dfssm_head_greedy(16, 16, 10, 16384, 16, None, 16, None, 16, 256, 256, None) == -3
@@ -89,6 +96,42 @@ def test_argument_validation_precedes_device_use(L):
                             256, 1024, None) == -7                                    # workspace
     assert L.dfssm_generate(None, 48, C.byref(dims), 16, 16, 10, 16, 16, 4, None, None, None, None,
                             256, 1 << 30, None) == -1                                 # no layers
+
+
+def _linears(dfssm, *descs):
+    arr = (dfssm.LinearT * len(descs))(*descs)
+    return arr
+
+
+def test_multi_and_noalloc_validate_like_the_single_call(L):
+    """dfssm_linear_decode_multi and dfssm_linear_decode_noalloc reject the same malformed descriptors as
+    dfssm_linear_decode (one shared check), and their own size limits, before touching a device."""
+    from bit_quantized_mamba_b200 import dfssm
+    ys = (C.c_void_p * 2)(16, 16)
+    good = dfssm.LinearT(512, 2048, 16, 16, 16, 16, 16, 16, 16)
+    cases = [
+        (dfssm.LinearT(512, 100, 16, 16, 16, 16, 16, 16, 16), -1),   # d_in not a multiple of 32
+        (dfssm.LinearT(512, 256, 17, 16, 16, 16, 16, 16, 16), -1),   # rank > 16
+        (dfssm.LinearT(512, 256, 16, 8, 16, 16, 16, 16, 16), -2),    # bits misaligned
+        (dfssm.LinearT(512, 256, 16, 16, 16, 16, 16, 8, 16), -2),    # W_A misaligned at rank 16
+        (dfssm.LinearT(512, 256, 16, None, 16, 16, 16, 16, 16), -1), # no bits
+        (dfssm.LinearT(512, 8224, 16, 16, 16, 16, 16, 16, 16), -3),  # d_in above 8192
+    ]
+    for desc, want in cases:
+        assert L.dfssm_linear_decode(C.byref(desc), 16, 1, 16, 256, 1 << 20, None, None) == want
+        assert L.dfssm_linear_decode_noalloc(C.byref(desc), 16, 1, 16, None, None) == want
+        arr = _linears(dfssm, good, desc)
+        assert L.dfssm_linear_decode_multi(arr, 2, 16, 1, ys, 256, 256, None) == want
+    assert L.dfssm_linear_decode_noalloc(None, 16, 1, 16, None, None) == -1
+    assert L.dfssm_linear_decode_noalloc(C.byref(good), 16, 17, 16, None, None) == -3   # B > 16
+    assert L.dfssm_linear_decode_noalloc(C.byref(good), 8, 1, 16, None, None) == -2     # x misaligned
+    assert L.dfssm_linear_decode_noalloc(C.byref(good), None, 1, 16, None, None) == -1  # no x
+    arr = _linears(dfssm, good, good)
+    assert L.dfssm_linear_decode_multi(arr, 2, 16, 1, ys, None, 256, None) == -7        # no workspace
+    assert L.dfssm_linear_decode_multi(arr, 2, 16, 1, ys, 256, 16, None) == -7          # too small
+    odd = dfssm.LinearT(512, 384, 16, 16, 16, 16, 16, 16, 16)
+    arr = _linears(dfssm, odd, odd)
+    assert L.dfssm_linear_decode_multi(arr, 2, 16, 1, ys, 256, 256, None) == -3         # d_in 384
 
 
 def test_pack_signs_matches_oracle_bit_layout(L):

@@ -55,11 +55,12 @@ def test_embed_bit_exact(dev, vocab):
     m, W, sr, _ = vocab
     V = m["emb_w"].shape[0]
     tok = torch.zeros(1, dtype=torch.int32, device=dev)
+    ws = dfssm.workspace(dfssm.workspace_size(dfssm.OP_EMBED, 0, 0, 0), dev)
     for t in (0, 1, V - 1, m["first_token"], 31337):
         tok.fill_(t)
-        h = dfssm.embed(W, sr, tok).cpu().numpy()
+        h = dfssm.embed(W, sr, tok, ws=ws).cpu().numpy()
         assert np.array_equal(h, oracle.embed(m["emb_w"], m["emb_s"], t)), t
-    assert dfssm.device_status() == 0
+    assert dfssm.device_status(ws) == 0
 
 
 def test_embed_rejects_out_of_range_token(dev, vocab):
@@ -67,12 +68,13 @@ def test_embed_rejects_out_of_range_token(dev, vocab):
     from bit_quantized_mamba_b200 import dfssm
     m, W, sr, _ = vocab
     V = m["emb_w"].shape[0]
+    ws = dfssm.workspace(dfssm.workspace_size(dfssm.OP_EMBED, 0, 0, 0), dev)
     for bad in (V, -1):
         h = torch.full((2048,), 7.0, device=dev)
-        dfssm.embed(W, sr, torch.tensor([bad], dtype=torch.int32, device=dev), h)
-        assert dfssm.device_status() == -1
+        dfssm.embed(W, sr, torch.tensor([bad], dtype=torch.int32, device=dev), h, ws=ws)
+        assert dfssm.device_status(ws) == -1
         assert not h.any()
-    assert dfssm.device_status() == 0  # the status word was cleared by the read
+    assert dfssm.device_status(ws) == 0  # the status word was cleared by the read
 
 
 @pytest.mark.parametrize("norm", [True, False])
@@ -143,8 +145,10 @@ def _generate_compare(dev, m, dims, n_tokens):
     tokens[0] = m["first_token"]
     taps = torch.zeros((n_tokens, dims["d_model"]), dtype=torch.float32, device=dev)
     last = torch.zeros(V, dtype=torch.float32, device=dev)
-    dfssm.generate(stack, W, sr, fw, tokens, hidden_taps=taps, logits=last)
-    assert dfssm.device_status() == 0
+    gws = dfssm.workspace(dfssm.workspace_size(dfssm.OP_GENERATE, V, dims["d_model"],
+                                               dims["nheads"] * dims["headdim"]), dev)
+    dfssm.generate(stack, W, sr, fw, tokens, hidden_taps=taps, logits=last, ws=gws)
+    assert dfssm.device_status(gws) == 0
     gt = [int(t) for t in tokens.cpu().numpy()]
     taps = taps.cpu().numpy()
     olayers = []

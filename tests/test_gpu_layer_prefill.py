@@ -62,7 +62,6 @@ def _prefill_compare(dev, dims, n_layers, M, seed, decode_after=2):
     dfssm.layer_prefill(stack, h)
     ref = oracle.layer_prefill(olayers, prompt.copy(), conv, ssm)
     torch.cuda.synchronize()
-    assert dfssm.device_status() == 0
     assert_tol(h.cpu().numpy(), ref, f"hidden after prefill of {M}")
     for l in range(n_layers):
         assert_tol(stack.ssm_states[l].cpu().numpy(), ssm[l], f"ssm state layer {l}")

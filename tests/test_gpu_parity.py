@@ -145,10 +145,11 @@ def test_linear_multi_matches_per_call(dev, which, B):
     lins = [dfssm.Linear.from_host(l, dev) for l in data["linears"]]
     x = data["x"][:B]
     xd = to_dev(x, dev)
-    ys = dfssm.linear_decode_multi(lins, xd)
+    ws = dfssm.workspace(dfssm.workspace_size(dfssm.OP_LINEAR_MULTI, 0, 0, 0), dev)
+    ys = dfssm.linear_decode_multi(lins, xd, ws=ws)
     ref = [dfssm.linear_decode(L, xd) for L in lins]
     torch.cuda.synchronize()
-    assert dfssm.device_status() == 0  # no wait ran out of budget
+    assert dfssm.device_status(ws) == 0  # no wait ran out of budget
     for c in range(len(lins)):
         assert torch.equal(ys[c], ref[c]), c
     r = oracle.linear_decode(oracle.Linear.from_dict(data["linears"][0]), x)
@@ -191,10 +192,11 @@ def test_linear_multi_large_tiles(dev, d_in, shapes):
     lins = [dfssm.Linear.from_host(h, dev) for h in hosts]
     x = inputs.normal(np.random.default_rng(d_in), (1, d_in))
     xd = to_dev(x, dev)
-    ys = dfssm.linear_decode_multi(lins, xd)
+    ws = dfssm.workspace(dfssm.workspace_size(dfssm.OP_LINEAR_MULTI, 0, 0, 0), dev)
+    ys = dfssm.linear_decode_multi(lins, xd, ws=ws)
     ref = [dfssm.linear_decode(L, xd) for L in lins]
     torch.cuda.synchronize()
-    assert dfssm.device_status() == 0
+    assert dfssm.device_status(ws) == 0
     for j, h in enumerate(hosts):
         assert torch.equal(ys[j], ref[j]), j
         r = oracle.linear_decode(oracle.Linear.from_dict(h), x)
