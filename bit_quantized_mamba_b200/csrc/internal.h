@@ -3,6 +3,7 @@
 
 #include <cstddef>
 #include <cstdint>
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 namespace dfssm {
@@ -186,6 +187,9 @@ int launch_linear_stream(const dfssm_linear_t* lins, int n, const float* x, int 
 int read_status_word(int* word, cudaStream_t st, int* code);
 // The no-alloc entry point's module status word on the current device.
 int noalloc_status_word(int** out);
+// A row-major u8 matrix [rows][row_bytes] (row_bytes a multiple of 128) as a TMA tensor map with boxes of
+// 128 bytes x box_rows rows and the 128-byte swizzle (16-byte chunk c of row r lands at chunk c ^ (r & 7)).
+bool encode_u8_map_sw128(CUtensorMap* map, const void* base, int rows, int row_bytes, int box_rows);
 // Argument checks shared by the linear entry points (DFSSM_OK or the status to return).
 int check_linear(const dfssm_linear_t* L);
 // Records e as the text returned by dfssm_last_cuda_error (this thread) and returns DFSSM_ECUDA.

@@ -92,6 +92,9 @@ struct Lin {
 };
 
 struct Params {
+  // per linear, for the tensor-core path (several token slots): the sign bits as a 2-D tensor
+  // [d_out][d_in / 8 bytes], loaded as boxes of 128 bytes x TR rows with the 128-byte swizzle
+  CUtensorMap tmap[MAX_LIN];
   Lin lin[MAX_LIN];
   int n_lin;
   int d_in;
@@ -109,6 +112,15 @@ struct Params {
 
 // ------------------------------------------------------------------------------ mbarrier / bulk copy
 
+// acc += A(16 x 32, u8, row-major) * B(32 x 8, s8, column-major), int32 (the warp-wide legacy MMA).
+__device__ __forceinline__ void mma_u8s8(int (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return (uint32_t)__cvta_generic_to_shared(p);
 }
@@ -121,6 +133,14 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
 __device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
                : "memory");
+}
+// One 2-D TMA box (coordinates: byte column c0, row c1) into shared memory, completion on bar.
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int c0, int c1, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
+      "[%4];" ::"r"(smem_u32(dst)),
+      "l"(map), "r"(c0), "r"(c1), "r"(smem_u32(bar))
+      : "memory");
 }
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
@@ -177,9 +197,12 @@ __device__ __forceinline__ void prefetch_range(const void* p, size_t bytes, int 
 // Dynamic shared memory: the bits ring, the parameter ring (ns stages each), W_B of the current linear
 // when it fits, and the codes in both layouts.  W_B in shared memory is preferred (it takes the LoRA-down
 // off global-memory latency) as long as ~96 KB of bits stay in flight; then the largest stage count <= 8.
-constexpr size_t kSmemBudget = 215 * 1024;
+constexpr size_t kSmemBudget = 214 * 1024;  // 1 KB is kept for aligning the tile ring to 1 KB
+// Token stride of the permuted codes: with several token slots (tensor-core path) each token is padded by
+// 16 bytes, so that the eight tokens of an MMA column block fall into different shared-memory banks.
+__host__ __device__ constexpr int q_tok_stride(int din, int bt) { return q_tok_bytes(din) + (bt > 1 ? 16 : 0); }
 __host__ __device__ constexpr size_t base_smem(int din, int bt, int ns, int tb) {
-  return (size_t)ns * (tb + p_layout(din, bt, tb).bytes) + (size_t)bt * (q_tok_bytes(din) + din);
+  return (size_t)ns * (tb + p_layout(din, bt, tb).bytes) + (size_t)bt * (q_tok_stride(din, bt) + din);
 }
 __host__ __device__ constexpr bool fits(int din, int bt, int ns, bool wb, int tb) {
   return base_smem(din, bt, ns, tb) + (wb ? (size_t)R * din : 0) <= kSmemBudget;
@@ -196,7 +219,8 @@ __host__ __device__ constexpr int n_stages(int din, int bt, int tb) {
                                                          : 4;
 }
 __host__ __device__ constexpr size_t smem_bytes(int din, int bt, int tb) {
-  return base_smem(din, bt, n_stages(din, bt, tb), tb) + (wb_in_smem(din, bt, tb) ? (size_t)R * din : 0);
+  return base_smem(din, bt, n_stages(din, bt, tb), tb) + (wb_in_smem(din, bt, tb) ? (size_t)R * din : 0) +
+         1024;
 }
 
 // Position in the CTA's contiguous tile range: linear j, tile t of that linear.
@@ -322,20 +346,26 @@ __global__ void __launch_bounds__(NT, 1) stream_kernel(const __grid_constant__ P
   constexpr int XPT = DIN / (NCW * 32);                    // x values per GEMV thread per token
   constexpr bool XREG = BT * XPT <= 16;                    // keep x in registers between the two passes
   constexpr bool REGQ = BT == 1 && NSEG == 1;              // one token: the lane's codes live in registers
-  // many tokens: a run-time token loop against the lane's weight masks held in registers
-  constexpr bool TOKLOOP = BT > 4;
-  static_assert(!TOKLOOP || NSEG == 1, "token loop needs one segment per lane");
+  // several token slots: the scaffold product on the int8 MMA (0/1 sign masks x codes), the tiles loaded by
+  // TMA with the 128-byte swizzle; warp w takes rows [16 (w / KS), +16) x segments [SEGW (w % KS), +SEGW)
+  constexpr bool MMA = BT > 1;
+  constexpr int MB = TR / 16, KS = MMA ? NCW / MB : 1, SEGW = SEGS / KS, NB = (BT + 7) / 8;
+  static_assert(!MMA || (MB * KS == NCW && KS * SEGW == SEGS && DIN % 1024 == 0), "MMA tile split");
+  constexpr int QTS = q_tok_stride(DIN, BT);
   // Epilogue warps in use.  Warp e takes every NEP-th tile, so it waits on a stage's barriers at most one
   // phase ahead of the last completed one only if NEP <= NS (an mbarrier parity wait cannot tell phase n
   // from phase n - 2).
   constexpr int NEP = NEW < NS ? NEW : NS;
 
-  extern __shared__ __align__(128) unsigned char smem[];
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  // the tile ring starts on a 1 KB boundary (the 128-byte swizzle of the TMA path repeats every 1 KB)
+  unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                         ~uintptr_t(1023));
   unsigned char* pring = smem + (size_t)NS * TILE_BYTES;                            // [NS][PL.bytes]
   int8_t* wb_sm = reinterpret_cast<int8_t*>(pring + (size_t)NS * PL.bytes);         // [R][DIN] if WB_SMEM
   constexpr int QTB = q_tok_bytes(DIN);                                             // permuted token bytes
   int8_t* q_perm = wb_sm + (WB_SMEM ? R * DIN : 0);                                 // [BT][QTB]
-  int8_t* q_nat = q_perm + BT * QTB;                                                // [BT][DIN]
+  int8_t* q_nat = q_perm + BT * QTS;                                                // [BT][DIN]
   __shared__ Lin lin_sm[MAX_LIN];
   __shared__ uint64_t bfull[MAX_NS], bempty[MAX_NS], pfull[MAX_NS], pacc[MAX_NS], pempty[MAX_NS], wb_full,
       wb_empty;
@@ -380,6 +410,12 @@ __global__ void __launch_bounds__(NT, 1) stream_kernel(const __grid_constant__ P
       if (p.lin[j].rank > 0 && (reinterpret_cast<uintptr_t>(p.lin[j].lora_b) & 15)) ok = 0;
     wb_ok = ok;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if constexpr (MMA) {
+    for (int s2 = 0; s2 < NS; ++s2) {
+      int* acc0 = reinterpret_cast<int*>(pring + (size_t)s2 * PL.bytes + PL.acc);
+      for (int k = tid; k < TR * BT; k += NT) acc0[k] = 0;
+    }
   }
   __syncthreads();
   pdl_launch_dependents();
@@ -430,9 +466,17 @@ __global__ void __launch_bounds__(NT, 1) stream_kernel(const __grid_constant__ P
           break;
         }
         const int r0 = cu.t * TR, nr = min(TR, L.d_out - r0), n4 = nr & ~3;
-        const uint32_t bits_bytes = (uint32_t)nr * (DIN / 8);
-        mbar_expect_tx(&bfull[sl], bits_bytes);
-        bulk_g2s(smem + (size_t)sl * TILE_BYTES, L.bits + (size_t)r0 * (DIN / 32), bits_bytes, &bfull[sl]);
+        if constexpr (MMA) {
+          // DIN / 1024 boxes of TR rows x 128 bytes (rows past d_out arrive as zeros)
+          mbar_expect_tx(&bfull[sl], (uint32_t)(TR * (DIN / 8)));
+#pragma unroll
+          for (int h = 0; h < DIN / 1024; ++h)
+            tma_load_2d(smem + (size_t)sl * TILE_BYTES + h * TR * 128, &p.tmap[cu.j], h * 128, r0, &bfull[sl]);
+        } else {
+          const uint32_t bits_bytes = (uint32_t)nr * (DIN / 8);
+          mbar_expect_tx(&bfull[sl], bits_bytes);
+          bulk_g2s(smem + (size_t)sl * TILE_BYTES, L.bits + (size_t)r0 * (DIN / 32), bits_bytes, &bfull[sl]);
+        }
         unsigned char* ps = pring + (size_t)sl * PL.bytes;
         mbar_expect_tx(&pfull[sl], L.ptma ? (uint32_t)(nr * 16 + 2 * n4 * 4) : 0u);
         if (L.ptma) {
@@ -514,7 +558,7 @@ __global__ void __launch_bounds__(NT, 1) stream_kernel(const __grid_constant__ P
         const uint4* wa_st = reinterpret_cast<const uint4*>(ps);
         const float* sw_st = reinterpret_cast<const float*>(ps + PL.sw);
         const float* sa_st = reinterpret_cast<const float*>(ps + PL.sa);
-        const int* acc = reinterpret_cast<const int*>(ps + PL.acc);
+        int* acc = reinterpret_cast<int*>(const_cast<unsigned char*>(ps) + PL.acc);
         const double* tf = reinterpret_cast<const double*>(ps + PL.tf);
         // two (token, row) jobs per lane per step, their fp64 chains interleaved; consecutive lanes take
         // consecutive rows of one token (coalesced outputs, one broadcast tf row)
@@ -543,6 +587,7 @@ __global__ void __launch_bounds__(NT, 1) stream_kernel(const __grid_constant__ P
           sw = (double)fw;
           sa = (double)fa;
           a = acc[b * TR + rr];
+          if constexpr (MMA) acc[b * TR + rr] = 0;  // the next tile of this stage adds into zero
         };
         const int jstride = epi_split ? NEP * 32 : 32;
         for (int job = (epi_split ? e * 32 : 0) + lane; job < nr * B; job += 2 * jstride) {
@@ -636,7 +681,7 @@ __global__ void __launch_bounds__(NT, 1) stream_kernel(const __grid_constant__ P
             uint32_t packed = 0u;
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-              q_perm[b * QTB + q_index<SEGS>(4 * v + e)] = (int8_t)cd[4 * g + e];
+              q_perm[b * QTS + q_index<SEGS>(4 * v + e)] = (int8_t)cd[4 * g + e];
               packed |= (uint32_t)(cd[4 * g + e] & 0xFF) << (8 * e);
               sq += cd[4 * g + e];
             }
@@ -697,7 +742,7 @@ __global__ void __launch_bounds__(NT, 1) stream_kernel(const __grid_constant__ P
 #pragma unroll
         for (int k = 0; k < XPT; ++k) {
           const int i = tid + k * NCW * 32;
-          q_perm[b * QTB + q_index<SEGS>(i)] = (int8_t)cd[k];
+          q_perm[b * QTS + q_index<SEGS>(i)] = (int8_t)cd[k];
           q_nat[b * DIN + i] = (int8_t)cd[k];
           sq += cd[k];
         }
@@ -816,41 +861,52 @@ __global__ void __launch_bounds__(NT, 1) stream_kernel(const __grid_constant__ P
       const uint4* tile = reinterpret_cast<const uint4*>(smem + (size_t)sb * TILE_BYTES);
       int* acc = reinterpret_cast<int*>(pring + (size_t)sp * PL.bytes + PL.acc);
       const int nr = min(TR, L.d_out - cu.t * TR);
-      if constexpr (TOKLOOP) {
-#pragma unroll 1
-        for (int ps = 0; ps < PASSES; ++ps) {
-          const int rr = ps * RPP + warp * RPW + rsub;
-          const bool valid = rr < nr;
-          const uint4 w = valid ? tile[rr * ROW16 + li] : make_uint4(0u, 0u, 0u, 0u);
-          const uint32_t w4[4] = {w.x, w.y, w.z, w.w};
-          uint32_t mw[32];  // bit k of every byte of word j, in place: the dp4a masks for all tokens
+      if constexpr (MMA) {
+        // rows ra = 16 mb + g and ra + 8 of the tile, segments seg of this warp's k-slice; A = the 0/1 sign
+        // masks of 32 inputs, k-ordered as the permuted codes (k = 4j + b <-> input 8b + j of the 32-input
+        // block, so that mask word j is (w >> j) & 0x01010101 and code word j is word j of the block)
+        const int mb = warp / KS, ks = warp % KS;
+        const int g = lane >> 2, t = lane & 3;
+        const int ra = mb * 16 + g, rb = ra + 8;
+        const unsigned char* tl = reinterpret_cast<const unsigned char*>(tile);
+        int cf[NB][4];
 #pragma unroll
-          for (int j = 0; j < 4; ++j)
+        for (int nb = 0; nb < NB; ++nb)
 #pragma unroll
-            for (int k = 0; k < 8; ++k) mw[j * 8 + k] = w4[j] & (0x01010101u << k);
-          const uint4* q0 = reinterpret_cast<const uint4*>(q_perm) + li;
-#pragma unroll 2
-          for (int b = 0; b < B; ++b) {
-            const uint4* qp4 = q0 + b * q_tok(SEGS);
-            int acc8[8];
+          for (int q = 0; q < 4; ++q) cf[nb][q] = 0;
+        // this lane's token of each column block (slots past BT read the last slot: in bounds, not stored)
+        const int8_t* qtok[NB];
 #pragma unroll
-            for (int k = 0; k < 8; ++k) acc8[k] = 0;
+        for (int nb = 0; nb < NB; ++nb) qtok[nb] = q_perm + min(nb * 8 + g, BT - 1) * QTS + 4 * t;
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              const uint4 qa = qp4[(2 * j) * q_row(SEGS)], qb = qp4[(2 * j + 1) * q_row(SEGS)];
-              const uint32_t qp[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
+        for (int sgi = 0; sgi < SEGW; ++sgi) {
+          const int seg = ks * SEGW + sgi;
+          const int hb = (seg >> 3) * TR * 128, ch = seg & 7;
+          const uint4 wa = *reinterpret_cast<const uint4*>(tl + hb + ra * 128 + ((ch ^ (ra & 7)) << 4));
+          const uint4 wb = *reinterpret_cast<const uint4*>(tl + hb + rb * 128 + ((ch ^ (rb & 7)) << 4));
+          const uint32_t w_a[4] = {wa.x, wa.y, wa.z, wa.w}, w_b[4] = {wb.x, wb.y, wb.z, wb.w};
 #pragma unroll
-              for (int k = 0; k < 8; ++k) acc8[k] = dp4a_us(mw[j * 8 + k], qp[k], acc8[k]);
-            }
-            int S = 0;
+          for (int kb = 0; kb < 4; ++kb) {
+            const uint32_t af[4] = {(w_a[kb] >> t) & 0x01010101u, (w_b[kb] >> t) & 0x01010101u,
+                                    (w_a[kb] >> (t + 4)) & 0x01010101u, (w_b[kb] >> (t + 4)) & 0x01010101u};
+            const int o0 = ((2 * kb) * q_row(SEGS) + seg) * 16, o1 = o0 + q_row(SEGS) * 16;
 #pragma unroll
-            for (int k = 0; k < 8; ++k) S += acc8[k] * (1 << (7 - k));
-#pragma unroll
-            for (int o = LPR / 2; o > 0; o >>= 1) S += __shfl_xor_sync(0xffffffffu, S, o);
-            if (valid && (b % LPR) == li) acc[b * TR + rr] = (S >> 6) - s_sumq[b];  // 2 sum - sum q
+            for (int nb = 0; nb < NB; ++nb)
+              mma_u8s8(cf[nb], af, *reinterpret_cast<const uint32_t*>(qtok[nb] + o0),
+                       *reinterpret_cast<const uint32_t*>(qtok[nb] + o1));
           }
         }
-      } else if constexpr (BT == 1) {
+        // acc = 2 sum_{bit=1} q - sum q, summed over the KS k-slices in shared memory
+#pragma unroll
+        for (int nb = 0; nb < NB; ++nb) {
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int row = q < 2 ? ra : rb, tok = nb * 8 + 2 * t + (q & 1);
+            if (row < nr && tok < B)
+              atomicAdd(acc + tok * TR + row, 2 * cf[nb][q] - (ks == 0 ? s_sumq[tok] : 0));
+          }
+        }
+      } else {
         // one token: every pass's partial sum first, then one transposed reduction over the row group
         // (a few shuffles for all passes instead of a full reduction per pass)
         int Sp[PASSES];
@@ -876,31 +932,6 @@ __global__ void __launch_bounds__(NT, 1) stream_kernel(const __grid_constant__ P
         const int Sr = reduce_passes<PASSES, LPR>(Sp, li);
         const int rr = pass_of<PASSES, LPR>(li) * RPP + warp * RPW + rsub;
         if ((li & (LPR / PASSES - 1)) == 0 && rr < nr) acc[rr] = (Sr >> 6) - sumq[0];  // 2 sum - sum q
-      } else {
-#pragma unroll
-      for (int ps = 0; ps < PASSES; ++ps) {
-        const int rr = ps * RPP + warp * RPW + rsub;
-        const bool valid = rr < nr;
-        int S[BT];
-#pragma unroll
-        for (int b = 0; b < BT; ++b) S[b] = 0;
-#pragma unroll
-        for (int sg = 0; sg < NSEG; ++sg) {
-          const int seg = sg * LPR + li;
-          const uint4 w = valid ? tile[rr * ROW16 + seg] : make_uint4(0u, 0u, 0u, 0u);
-          if constexpr (REGQ) S[0] += bits_dot_regs(w, qreg);
-          else bits_dot_tokens<SEGS, BT>(w, reinterpret_cast<const uint4*>(q_perm) + seg, B, S);
-        }
-#pragma unroll
-        for (int b = 0; b < BT; ++b) {
-#pragma unroll
-          for (int o = LPR / 2; o > 0; o >>= 1) S[b] += __shfl_xor_sync(0xffffffffu, S[b], o);
-        }
-        // lane b % LPR of the row group stores token b's accumulator
-#pragma unroll
-        for (int b = 0; b < BT; ++b)
-          if (valid && b < B && (b % LPR) == li) acc[b * TR + rr] = (S[b] >> 6) - sumq[b];  // 2 sum - sum q
-      }
       }
       if (tid < BT * R)
         reinterpret_cast<double*>(pring + (size_t)sp * PL.bytes + PL.tf)[tid] = tf_cur[tid / R][tid % R];
@@ -981,6 +1012,9 @@ int launch_linear_stream(const dfssm_linear_t* lins, int n, const float* x, int 
     q.tile0 = tiles;
     q.ntiles = (L.d_out + tile_rows - 1) / tile_rows;
     tiles += q.ntiles;
+    // the tensor-core path (several token slots) loads the sign bits as swizzled 2-D boxes
+    if (B > 1 && !encode_u8_map_sw128(&p.tmap[j], L.bits, L.d_out, d_in / 8, tile_rows))
+      return DFSSM_EUNSUPPORTED;
   }
   p.n_lin = n;
   p.d_in = d_in;

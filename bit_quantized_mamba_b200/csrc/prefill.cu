@@ -590,6 +590,19 @@ Ws carve(void* base, int M, int K, int N) {
 
 }  // namespace prefill
 
+bool encode_u8_map_sw128(CUtensorMap* map, const void* base, int rows, int row_bytes, int box_rows) {
+  auto fn = prefill::encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)row_bytes, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)row_bytes};
+  cuuint32_t box[2] = {128u, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box,
+                        estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 size_t prefill_workspace_bytes(int M, int d_in, int d_out) { return prefill::ws_bytes(M, d_in, d_out); }
 
 }  // namespace dfssm
