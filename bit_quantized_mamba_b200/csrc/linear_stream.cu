@@ -358,9 +358,9 @@ __global__ void __launch_bounds__(NT, 1) stream_kernel(const __grid_constant__ P
   constexpr int NEP = NEW < NS ? NEW : NS;
 
   extern __shared__ __align__(1024) unsigned char smem_raw[];
-  // the tile ring starts on a 1 KB boundary (the 128-byte swizzle of the TMA path repeats every 1 KB)
-  unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                                         ~uintptr_t(1023));
+  // the tile ring starts on a 1 KB boundary (the 128-byte swizzle of the TMA path repeats every 1 KB),
+  // reached by an offset from the array itself so that every access stays a shared-memory access
+  unsigned char* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   unsigned char* pring = smem + (size_t)NS * TILE_BYTES;                            // [NS][PL.bytes]
   int8_t* wb_sm = reinterpret_cast<int8_t*>(pring + (size_t)NS * PL.bytes);         // [R][DIN] if WB_SMEM
   constexpr int QTB = q_tok_bytes(DIN);                                             // permuted token bytes
@@ -560,13 +560,10 @@ __global__ void __launch_bounds__(NT, 1) stream_kernel(const __grid_constant__ P
         const float* sa_st = reinterpret_cast<const float*>(ps + PL.sa);
         int* acc = reinterpret_cast<int*>(const_cast<unsigned char*>(ps) + PL.acc);
         const double* tf = reinterpret_cast<const double*>(ps + PL.tf);
-        // two (token, row) jobs per lane per step, their fp64 chains interleaved; consecutive lanes take
-        // consecutive rows of one token (coalesced outputs, one broadcast tf row)
-        const auto fetch = [&](int job, int& a, double& sw, double& sa, uint4& wa, int& row, int& b) {
-          b = job / nr;
-          const int rr = job - b * nr;
-          row = r0 + rr;
-          float fw, fa = 0.0f;
+        // the row's parameters: W_A bytes, sW, sA (stage copy, or global memory past the copied rows)
+        const auto row_params = [&](int rr, uint4& wa, float& fw, float& fa) {
+          const int row = r0 + rr;
+          fa = 0.0f;
           wa = make_uint4(0u, 0u, 0u, 0u);
           if (L.ptma) {
             wa = wa_st[rr];
@@ -584,10 +581,69 @@ __global__ void __launch_bounds__(NT, 1) stream_kernel(const __grid_constant__ P
               wa = load_wa(L, row);
             }
           }
+        };
+        if constexpr (MMA) {
+          // lane = row: sW and sA are converted once per row and shared by every token; four tokens' LoRA
+          // chains run interleaved, each W_A entry reaching fp64 once per four tokens, the tf rows read as
+          // broadcasts
+          const int rstart = (epi_split ? e * 32 : 0) + lane, rstride = epi_split ? NEP * 32 : 32;
+          const int rk = L.rank;
+          for (int rr = rstart; rr < nr; rr += rstride) {
+            uint4 wa;
+            float fw, fa;
+            row_params(rr, wa, fw, fa);
+            const double sw = (double)fw, sa = (double)fa;
+            const uint32_t w4[4] = {wa.x, wa.y, wa.z, wa.w};
+            const int row = r0 + rr;
+            for (int b0 = 0; b0 < B; b0 += 4) {
+              double lora[4] = {0.0, 0.0, 0.0, 0.0};
+              if (rk == R) {
+#pragma unroll 2
+                for (int r = 0; r < R; r += 2) {
+                  const double w0 = int_to_f64((int)(int8_t)(w4[r >> 2] >> (8 * (r & 3))));
+                  const double w1 = int_to_f64((int)(int8_t)(w4[r >> 2] >> (8 * ((r + 1) & 3))));
+#pragma unroll
+                  for (int k = 0; k < 4; ++k) {
+                    const double2 t = *reinterpret_cast<const double2*>(tf + (b0 + k) * R + r);
+                    lora[k] = fma(w0, t.x, lora[k]);
+                    lora[k] = fma(w1, t.y, lora[k]);
+                  }
+                }
+              } else {
+#pragma unroll
+                for (int r = 0; r < R; ++r)
+                  if (r < rk) {
+                    const double w = int_to_f64((int)(int8_t)(w4[r >> 2] >> (8 * (r & 3))));
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) lora[k] = fma(w, tf[(b0 + k) * R + r], lora[k]);
+                  }
+              }
+#pragma unroll
+              for (int k = 0; k < 4; ++k) {
+                const int b = b0 + k;  // slots past B (inside BT, a multiple of 4) are read, never stored
+                const int a = acc[b * TR + rr];
+                acc[b * TR + rr] = 0;  // the next tile of this stage adds into zero
+                const double scaffold = dmul(dmul(int_to_f64(a), s_tokd[b]), sw);
+                const double corr = rk > 0 ? dmul(sa, lora[k]) : 0.0;
+                if (b < B) {
+                  L.y[(size_t)b * L.d_out + row] = __double2float_rn(dadd(scaffold, corr));
+                  if (p.dbg_acc) p.dbg_acc[(size_t)b * L.d_out + row] = a;
+                }
+              }
+            }
+          }
+        } else {
+        // two (token, row) jobs per lane per step, their fp64 chains interleaved; consecutive lanes take
+        // consecutive rows of one token (coalesced outputs, one broadcast tf row)
+        const auto fetch = [&](int job, int& a, double& sw, double& sa, uint4& wa, int& row, int& b) {
+          b = job / nr;
+          const int rr = job - b * nr;
+          row = r0 + rr;
+          float fw, fa;
+          row_params(rr, wa, fw, fa);
           sw = (double)fw;
           sa = (double)fa;
           a = acc[b * TR + rr];
-          if constexpr (MMA) acc[b * TR + rr] = 0;  // the next tile of this stage adds into zero
         };
         const int jstride = epi_split ? NEP * 32 : 32;
         for (int job = (epi_split ? e * 32 : 0) + lane; job < nr * B; job += 2 * jstride) {
@@ -610,6 +666,7 @@ __global__ void __launch_bounds__(NT, 1) stream_kernel(const __grid_constant__ P
               if (p.dbg_acc) p.dbg_acc[(size_t)b[n] * L.d_out + row[n]] = a[n];
             }
           }
+        }
         }
       }
       __syncwarp();

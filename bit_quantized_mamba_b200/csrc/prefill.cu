@@ -320,8 +320,8 @@ __global__ void __launch_bounds__(PNT, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
                 const EpiArgs ep) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
-  unsigned char* smem = reinterpret_cast<unsigned char*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // aligned by an offset from the array itself, so that every access stays a shared-memory access
+  unsigned char* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + OFF_BARS);
   uint64_t* empty = full + STAGES;
   uint64_t* acc_full = empty + STAGES;     // [2] MMA -> epilogue
