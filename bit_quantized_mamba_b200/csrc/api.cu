@@ -83,7 +83,7 @@ struct PrefillLayerWs {
 PrefillLayerWs prefill_layer_ws(int M, int d_model, int E) {
   PrefillLayerWs w;
   const size_t C = (size_t)E + 2048, d_ip = 2 * (size_t)E + 2048 + 1024;
-  w.zx = 0;
+  w.zx = dfssm::kStatusBytes;  // the status word comes first
   w.xc = w.zx + align256(sizeof(float) * (size_t)M * d_ip);
   w.g = w.xc + align256(sizeof(float) * (size_t)M * C);
   w.sz = w.g + align256(sizeof(float) * (size_t)M * E);
@@ -122,19 +122,16 @@ int enqueue_head(const int8_t* W, const float* s_row, int V, int d, const float*
 // Clock budget of one device-side wait of the fused decode kernel (about 1 s at 2 GHz).
 constexpr long long kSpinLimitCycles = 2000000000LL;
 
+// The current device is an sm_100 part (asked every call: the answer depends on the calling thread's
+// current device, and the two runtime queries cost well under a microsecond).
 bool device_ok() {
-  static int ok = -1;
-  if (ok < 0) {
-    int dev = 0, major = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) {
-      cudaGetLastError();
-      ok = 0;
-    } else {
-      ok = (major == 10) ? 1 : 0;
-    }
+  int dev = 0, major = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
   }
-  return ok == 1;
+  return major == 10;
 }
 
 dfssm::GemvArgs gemv_args(const dfssm_linear_t* L, int B, const dfssm::QuantScratch& qs) {
@@ -623,10 +620,11 @@ int dfssm_layer_prefill(const dfssm_layer_t* layers, int n_layers, const dfssm_d
   float* g = reinterpret_cast<float*>(base + w.g);
   void* lin_ws = base + w.lin;
   const size_t lin_bytes = ws_bytes - w.lin;
+  int* status = reinterpret_cast<int*>(base);
   for (int l = 0; l < n_layers; ++l) {
     const dfssm_layer_t& Ly = layers[l];
     int st = dfssm::linear_prefill_impl(&Ly.in_proj, hidden, M, zx, Ly.norm_w, false, lin_ws, lin_bytes,
-                                        nullptr, stream);
+                                        status, nullptr, stream);
     if (st) return st;
     dfssm::ConvSeqArgs ca{zx, d_ip, E, conv_states[l], Ly.conv_w, Ly.conv_b, xc, M, C};
     cudaError_t e = dfssm::launch_conv_seq(ca, s);
@@ -654,7 +652,7 @@ int dfssm_layer_prefill(const dfssm_layer_t* layers, int n_layers, const dfssm_d
     e = dfssm::launch_ssm_scan(sa, s);
     if (e != cudaSuccess) return cuda_fail(e);
     st = dfssm::linear_prefill_impl(&Ly.out_proj, g, M, hidden, Ly.gnorm_w, true, lin_ws, lin_bytes,
-                                    nullptr, stream);
+                                    status, nullptr, stream);
     if (st) return st;
   }
   return DFSSM_OK;

@@ -168,8 +168,9 @@ size_t fused_decode_workspace_bytes();
 
 // dfssm_linear_prefill with two options for the layer prefill: a norm weight folded into the per-token
 // quantizer (norm_w, may be NULL), and a residual epilogue (y[m][n] = fl32(y[m][n] + out)).
+// status: the word a timed-out wait is recorded in (NULL: the first word of `workspace`).
 int linear_prefill_impl(const dfssm_linear_t* lin, const float* x, int M, float* y, const float* norm_w,
-                        bool resid, void* workspace, size_t ws_bytes, const dfssm_debug_t* dbg,
+                        bool resid, void* workspace, size_t ws_bytes, int* status, const dfssm_debug_t* dbg,
                         void* stream);
 bool fused_decode_supported(const dfssm_dims_t& d, int B, const dfssm_layer_t* layers, int n,
                             float* const* conv_states);

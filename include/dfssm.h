@@ -17,8 +17,8 @@
  *     word in fixed arrays of the library's own device memory.
  *   - Device-side errors (a wait that ran out of its clock budget, an embedding id out of range) are
  *     recorded in a status word at the start of the call's workspace (for dfssm_linear_decode,
- *     dfssm_linear_decode_multi, dfssm_embed, dfssm_layer_decode and dfssm_generate), read and cleared
- *     by dfssm_device_status.
+ *     dfssm_linear_decode_multi, dfssm_linear_prefill, dfssm_embed, dfssm_layer_decode,
+ *     dfssm_layer_prefill and dfssm_generate), read and cleared by dfssm_device_status.
  *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy default stream).  Inputs
  *     must not be modified, and outputs not read, until the stream reaches the call.  Weights and
  *     parameters must be fully written before the call is enqueued (kernels may read them before they
@@ -159,9 +159,11 @@ int dfssm_linear_decode_noalloc(const dfssm_linear_t* lin, const float* x, int B
                                 const dfssm_debug_t* dbg, void* stream);
 
 /*
- * M-token prefill of one linear on int8 tcgen05 tensor cores (technical summary §2.C: the scaffold
- * matmul on INT8 tensor cores).  Same math as dfssm_linear_decode, per row of x.
+ * M-token prefill of one linear on int8 tcgen05 tensor cores (technical summary §2.C: the 1-bit weights
+ * expanded on the fly to int8 for the INT8 tensor cores; here the expansion happens in shared memory and
+ * never reaches global memory).  Same math as dfssm_linear_decode, per row of x.
  *   x device f32 [M][d_in], y device f32 [M][d_out], M >= 1.  d_in % 128 == 0 required.
+ *   workspace: dfssm_workspace_size(DFSSM_OP_LINEAR_PREFILL, M, d_in, d_out) bytes (status word first).
  *   dbg->acc, dbg->xq, dbg->xscale and dbg->lora_t are exact, and y is bit-identical to the decode path
  *   (the epilogue evaluates the definition in fp64 with the decode rounding sequence).
  */

@@ -408,7 +408,7 @@ def _prefill_compare(dev, lin_host, x, rows):
 
 
 def test_prefill_ragged_small(dev):
-    """M and d_out not multiples of the 128 x 256 tile; every row checked."""
+    """M and d_out not multiples of the 128-row x 256-token tile; every row checked."""
     gen = np.random.default_rng(61)
     lin = inputs.linear(gen, 300, 256, 16)
     x = inputs.normal(gen, (200, 256)) * np.float32(2)
@@ -421,6 +421,37 @@ def test_prefill_rank_below_16(dev):
     lin = inputs.linear(gen, 256, 384, 5)
     x = inputs.normal(gen, (130, 384))
     _prefill_compare(dev, lin, x, range(130))
+
+
+def test_prefill_lora_sum_exactness_paths(dev):
+    """The prefill epilogue takes a token block's LoRA sum on the fp64 tensor core only when every partial
+    sum is exact (the token's nonzero tf span at most 18 binades), else the sequential chain.  W_B row 15
+    picks one input, so t_15 = q[i0]: tokens whose x[i0] quantizes to +-1 get a tf_15 far below the
+    others (sequential path for their block), tokens with x[i0] = 0 get tf_15 = 0 (still exact).  Every
+    output is compared bit for bit."""
+    gen = np.random.default_rng(63)
+    lin = inputs.linear(gen, 300, 256, 16)
+    i0 = 17
+    lin["lora_b"][15] = 0
+    lin["lora_b"][15, i0] = 1
+    lin["lora_b_scale"][15] = np.float32(1e-5)
+    x = inputs.normal(gen, (200, 256))
+    x[::2, i0] = 0.0
+    for m in range(1, 200, 2):
+        x[m, i0] = np.abs(x[m]).max()  # code 127: tf_15 within 2^17 of the largest tf
+    for m in (3, 41, 42, 100, 199):
+        x[m, i0] = np.abs(x[m]).max() / 127.0  # code +-1: tf_15 about 2^-22 of the largest tf
+    _prefill_compare(dev, lin, x, range(200))
+
+
+def test_prefill_lora_wide_scales(dev):
+    """LoRA-down scales spread over ~2^40: no token's sum is provably exact, every block takes the
+    sequential chain."""
+    gen = np.random.default_rng(64)
+    lin = inputs.linear(gen, 260, 384, 16)
+    lin["lora_b_scale"] = (2.0 ** np.linspace(-30, 10, 16)).astype(np.float32)
+    x = inputs.normal(gen, (70, 384))
+    _prefill_compare(dev, lin, x, range(70))
 
 
 @pytest.mark.parametrize("which", ["in_proj", "out_proj"])
