@@ -194,9 +194,9 @@ def run_reference(args, rank):
 # ---------------------------------------------------------------------------------- our arm
 
 # DRAM traffic of one decode_kernel launch (dram__bytes_read.sum + dram__bytes_write.sum, one ncu capture
-# of the fourth launch of `bench.py --ncu --warmup 3`: 280.58 MB + 57.18 MB), valid only for the kernel
+# of the fourth launch of `bench.py --ncu --warmup 3`: 280.89 MB + 52.80 MB), valid only for the kernel
 # source it was measured on; reported as null once that source changes.
-TRAFFIC_MEASURED = {"sha": "941fff55c4bb", "bytes": 337_766_912}
+TRAFFIC_MEASURED = {"sha": "53d0d9f55b17", "bytes": 333_697_280}
 
 
 def src_sha(*names):
@@ -598,15 +598,16 @@ def run_prefill_profile(args):
 
 
 def run_gemv_profile(args):
-    """Eager dfssm_linear_decode_multi calls over the 48 in_proj copies at batch 1, for ncu."""
+    """Eager dfssm_linear_decode_multi calls over the 48 in_proj copies (batch --gemv-batch), for ncu."""
     import torch
     from bit_quantized_mamba_b200 import build, dfssm, inputs
     build.build()
     dev = torch.device("cuda", 0)
     data = inputs.in_proj_stack()
     lins = [dfssm.Linear.from_host(l, dev) for l in data["linears"]]
-    x = torch.from_numpy(data["x"][:1].copy()).to(dev)
-    ys = [torch.empty((1, L.d_out), dtype=torch.float32, device=dev) for L in lins]
+    B = args.gemv_batch
+    x = torch.from_numpy(data["x"][:B].copy()).to(dev)
+    ys = [torch.empty((B, L.d_out), dtype=torch.float32, device=dev) for L in lins]
     ws = dfssm.workspace(dfssm.workspace_size(dfssm.OP_LINEAR_MULTI, 0, 0, 0), dev)
     for _ in range(args.warmup + 1):
         dfssm.linear_decode_multi(lins, x, ys, ws=ws)
@@ -666,6 +667,8 @@ def main():
                     help="profiling mode: run the 2048-token in_proj prefill --warmup + 1 times and exit")
     ap.add_argument("--ncu-gemv", action="store_true",
                     help="profiling mode: the 48-copy in_proj multi-linear decode --warmup + 1 times and exit")
+    ap.add_argument("--gemv-batch", type=int, default=1, choices=[1, 4, 16],
+                    help="token count of the --ncu-gemv profiling mode")
     ap.add_argument("--ncu-layer-prefill", action="store_true",
                     help="profiling mode: a 2048-token prompt through one layer --warmup + 1 times and exit")
     ap.add_argument("--ncu-head", action="store_true",
