@@ -194,9 +194,9 @@ def run_reference(args, rank):
 # ---------------------------------------------------------------------------------- our arm
 
 # DRAM traffic of one decode_kernel launch (dram__bytes_read.sum + dram__bytes_write.sum, one ncu capture
-# of the fourth launch of `bench.py --ncu --warmup 3`: 280.89 MB + 52.80 MB), valid only for the kernel
+# of the fourth launch of `bench.py --ncu --warmup 3`: 280.51 MB + 53.51 MB), valid only for the kernel
 # source it was measured on; reported as null once that source changes.
-TRAFFIC_MEASURED = {"sha": "53d0d9f55b17", "bytes": 333_697_280}
+TRAFFIC_MEASURED = {"sha": "57db9d3cbb95", "bytes": 334_023_680}
 
 
 def src_sha(*names):

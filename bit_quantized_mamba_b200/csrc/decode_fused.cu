@@ -87,6 +87,30 @@ struct Params {
   long long spin_limit;
 };
 
+// ------------------------------------------------------------------------------ phase trace
+// Built only with -DDFSSM_TRACE_DECODE (bit_quantized_mamba_b200/trace_decode.py): thread 0 of CTAs 0 and
+// kTraceCta2 stamps the global timer (ns) at eleven points of every layer, read by
+// dfssm_decode_trace_ptr().  The default build has no stamps.
+#ifdef DFSSM_TRACE_DECODE
+constexpr int kTraceCta2 = 74;  // a CTA on the other die
+constexpr int kTracePoints = 12;
+__device__ unsigned long long g_decode_trace[2 * 64 * kTracePoints];
+__device__ __forceinline__ unsigned long long trace_now() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+#define DTR(k)                                                                                          \
+  do {                                                                                                  \
+    if (threadIdx.x == 0 && (blockIdx.x == 0 || blockIdx.x == kTraceCta2) && l < 64)                    \
+      g_decode_trace[((blockIdx.x == 0 ? 0 : 1) * 64 + l) * kTracePoints + (k)] = trace_now();          \
+  } while (0)
+#else
+#define DTR(k) \
+  do {         \
+  } while (0)
+#endif
+
 // ------------------------------------------------------------------------------ workspace layout
 // [status word 128 B][abort word 128 B][hx DM x 8 B][gx E x 8 B][bcx (2N + 2H) x 8 B]
 // Everything from the abort word on is cleared before every launch (tag 0 = not yet written); the
@@ -657,6 +681,7 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ P
     const uint32_t tag_h = (uint32_t)l, tag_l = (uint32_t)(l + 1);
 
     // ---------------------------------------------------------------- phase A: h -> in_proj
+    DTR(0);
     float hv[4];
     bool ok = true;
     if (l == 0) {
@@ -672,6 +697,7 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ P
       __syncthreads();
       ok = poll_pairs<2>(p.hx, hoff, tag_h, hv, p.err, p.status, p.spin_limit);
     }
+    DTR(1);
     cp_async_wait<0>();  // this thread's row parameters; the quantizer's barriers publish them
     if (ok && !mbar_wait(&inbar[l & 1], (l >> 1) & 1, p.spin_limit)) {  // in_proj W_B and the norm weight
       fail();
@@ -684,6 +710,7 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ P
       drain(l, false);
       return;
     }
+    DTR(2);
     if (tid == 0) any_flag[1] = 0;  // the gated norm's flag (last read in the previous layer)
     const int sumq = block_sum16(red_i);
     // scaffold GEMV over the owned rows, pass 0 (the shared rows first), then LoRA-down row `warp`
@@ -698,6 +725,7 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ P
       lora_slice<DM>(wb_in(l), q_nat, warp, lane, red_t);
     }
     __syncthreads();
+    DTR(3);
     const auto pass1 = [&]() {
       int S = bits_dot_reg(w_in[1], qreg);
 #pragma unroll
@@ -738,6 +766,7 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ P
     }
 
     // ---------------------------------------------------------------- phase B: z/x epilogues + SSM
+    DTR(4);
     if (tid >= kZxBase && tid - kZxBase < n_ssm) {
       // the owned z rows (gate value SiLU(z) kept) and x rows (conv of the owned x channels)
       const int j = tid - kZxBase;
@@ -791,6 +820,7 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ P
       drain(l, has_next);
       return;
     }
+    DTR(5);
     float4 snew[2];
 #pragma unroll
     for (int ps = 0; ps < 2; ++ps) {
@@ -827,9 +857,11 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ P
       if (ssm_slot[ps] < n_ssm) st_f4(Lp.ssm_state + (size_t)(rs0 + ssm_slot[ps]) * N + lane * 4, snew[ps]);
 
     // ---------------------------------------------------------------- phase C: gated norm -> out_proj
+    DTR(6);
     float gv[8];
     __syncthreads();  // as before the h poll: no thread spins while others still work on this phase
     ok = poll_pairs<4>(p.gx, goff, tag_l, gv, p.err, p.status, p.spin_limit);
+    DTR(7);
     if (ok && !mbar_wait(&outbar, l & 1, p.spin_limit)) {  // out_proj W_B and the gated-norm weight
       fail();
       ok = false;
@@ -840,6 +872,7 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ P
       drain(l, has_next);
       return;
     }
+    DTR(8);
     if (tid == 0) any_flag[0] = 0;  // the next layer's pre-norm flag
     {
       // LoRA down of the codes (by input slices); every warp with an out_proj row then takes it
@@ -852,6 +885,7 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ P
       }
     }
     __syncthreads();
+    DTR(9);
     if (warp == 0) {
       // lanes r < R form the LoRA intermediate tf[r]; every epilogue lane takes all sixteen by shuffle
       const double tf_r = lane < R ? (double)lora_tf(lora_t_sum(red_t, lane), lbs_o[l & 1][lane], s_out) : 0.0;
@@ -866,7 +900,9 @@ __global__ void __launch_bounds__(NT, 1) decode_kernel(const __grid_constant__ P
         else p.hidden[ro0 + tid] = h_own;
       }
     }
+    DTR(10);
     if (has_next) issue_loads(l + 1);
+    DTR(11);
   }
 }
 
@@ -972,5 +1008,12 @@ cudaError_t launch_timeout_selftest(void* ws, cudaStream_t st, long long spin_li
   fused::timeout_selftest_kernel<<<1, 32, 0, st>>>(word, err, status, spin_limit);
   return cudaGetLastError();
 }
+
+#ifdef DFSSM_TRACE_DECODE
+extern "C" void* dfssm_decode_trace_ptr() {
+  void* q = nullptr;
+  return cudaGetSymbolAddress(&q, fused::g_decode_trace) == cudaSuccess ? q : nullptr;
+}
+#endif
 
 }  // namespace dfssm
