@@ -576,9 +576,39 @@ def run_ours(args, rank, world, local_rank):
                                           f"zero state, on {cores} threads",
                                 "single_thread": {"value": n1 / dt1, "unit": "tokens/s", "cores": 1,
                                                   "sample": f"first {n1} token(s), 1 thread"}}
+        vnni = vnni_engine_rate(cores)
+        if vnni is not None:
+            line["cpu_baseline"]["vnni_engine"] = vnni
     if rank == 0:
         print(json.dumps(line), flush=True)
     graph = None
+
+
+def vnni_engine_rate(cores, n_tokens=8):
+    """The host-CPU engine (libdfssm_cpu, AVX-512 VNNI scaffold GEMV; bit-identical to the oracle) on the
+    first tokens of the same 48-layer decode, all host cores; None when the CPU lacks VNNI."""
+    import numpy as np
+    import torch
+    from bit_quantized_mamba_b200 import build, dfssm, inputs
+    build.build_cpu()
+    if not dfssm.cpu_available():
+        return None
+    dfssm.cpu_set_threads(cores)
+    model = inputs.decode_model(seed=3, n_layers=48, n_tokens=n_tokens)
+    conv, ssm = inputs.zero_states(1, 48)
+    layers = [dfssm.Layer.from_host(x, "cpu") for x in model["layers"]]
+    stack = dfssm.LayerStack(layers, dict(d_model=2048, nheads=64, headdim=64, d_state=128, ngroups=1),
+                             [torch.from_numpy(conv[i]) for i in range(48)],
+                             [torch.from_numpy(ssm[i]) for i in range(48)])
+    h = torch.from_numpy(np.array(model["emb"][0], dtype=np.float32))
+    dfssm.cpu_layer_decode(stack, h)  # first token: page-in, not timed
+    t0 = time.perf_counter()
+    for t in range(1, n_tokens):
+        h = torch.from_numpy(np.array(model["emb"][t], dtype=np.float32))
+        dfssm.cpu_layer_decode(stack, h)
+    dt = time.perf_counter() - t0
+    return {"value": (n_tokens - 1) / dt, "unit": "tokens/s", "cores": cores, "kind": "vnni_engine",
+            "sample": f"tokens 1..{n_tokens - 1} of the 64-token decode, 48 layers, on {cores} threads"}
 
 
 def run_prefill_profile(args):

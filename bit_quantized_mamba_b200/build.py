@@ -61,6 +61,27 @@ def build(force: bool = False, verbose: bool = False) -> str:
     return LIB
 
 
+CPU_SRC = os.path.join(HERE, "cpu", "dfssm_cpu.cpp")
+CPU_LIB = os.path.join(HERE, "libdfssm_cpu.so")
+
+
+def build_cpu(force: bool = False) -> str:
+    """libdfssm_cpu.so: the host-CPU (AVX-512 VNNI) engine (include/dfssm_cpu.h).  The VNNI code sits in
+    functions compiled for that target and is entered only after a run-time CPU check; the rest is
+    built for the baseline x86-64 target with no contraction of products and sums."""
+    deps = [CPU_SRC, os.path.join(INCLUDE, "dfssm_cpu.h"), os.path.join(INCLUDE, "dfssm.h")]
+    if not force and os.path.exists(CPU_LIB) and all(os.path.getmtime(d) <= os.path.getmtime(CPU_LIB) for d in deps):
+        return CPU_LIB
+    tmp = CPU_LIB + f".tmp{os.getpid()}"
+    cmd = ["g++", "-O3", "-std=c++17", "-fopenmp", "-ffp-contract=off", "-fPIC", "-shared",
+           "-I", INCLUDE, CPU_SRC, "-o", tmp]
+    r = subprocess.run(cmd, capture_output=True, text=True)
+    if r.returncode != 0:
+        raise RuntimeError(f"g++ failed for {CPU_SRC}:\n{r.stdout}\n{r.stderr}")
+    os.replace(tmp, CPU_LIB)
+    return CPU_LIB
+
+
 def build_trace() -> str:
     """libdfssm_trace.so: the same library with the fused decode kernel's phase stamps compiled in
     (-DDFSSM_TRACE_DECODE); used by trace_decode.py only."""
@@ -77,3 +98,4 @@ def build_trace() -> str:
 
 if __name__ == "__main__":
     print(build(force="--force" in sys.argv, verbose="-v" in sys.argv))
+    print(build_cpu(force="--force" in sys.argv))

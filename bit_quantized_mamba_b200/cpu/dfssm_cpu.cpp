@@ -1,0 +1,336 @@
+// Host-CPU engine of the DF-SSM decode step (include/dfssm_cpu.h): the pages' CPU path (gist.science
+// technical summary of DF-SSM, §2.C "CPU path": the 1-bit packed weights are expanded to int8 for the
+// VNNI dot product, loading 8x less weight data than int8 weights).
+//
+// Scaffold GEMV: 64 sign bits (two consecutive u32 words of a row; bit k is input 64c + k) become a
+// 64-bit mask, `vmovdqu8` with zero-masking turns it into 64 bytes of 0 or 1, and `vpdpbusd` multiplies
+// them (as u8) with 64 int8 codes of each token, accumulating four products per 32-bit lane.  The sum
+// over the set bits gives the +-1 scaffold sum as acc = 2 sum_{bit=1} q - sum q (exact integers).  The
+// expanded bytes serve every token of the call.
+//
+// Every other step follows the library's definition and rounding sequence: fp32 values are single
+// IEEE operations or the fp32 rounding of an fp64 expression, sums of more than two terms are fp64 in
+// index order, transcendental functions are fp64 and rounded once.  Built with -ffp-contract=off so
+// that no product and sum are fused where the definition rounds them separately.
+
+#include <immintrin.h>
+#include <omp.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdint>
+#include <cstdlib>
+#include <cstring>
+#include <vector>
+
+#include "dfssm_cpu.h"
+
+namespace {
+
+constexpr double kEps = 1e-5;
+
+inline float f32(double v) { return (float)v; }
+inline double silu(double v) { return v / (1.0 + std::exp(-v)); }
+
+bool has_vnni() {
+  __builtin_cpu_init();
+  return __builtin_cpu_supports("avx512f") && __builtin_cpu_supports("avx512bw") &&
+         __builtin_cpu_supports("avx512vnni");
+}
+
+// 64-byte aligned scratch that lives for one call.
+struct Buf {
+  void* p = nullptr;
+  explicit Buf(size_t bytes) { p = std::aligned_alloc(64, (bytes + 63) / 64 * 64 + 64); }
+  ~Buf() { std::free(p); }
+  template <class T>
+  T* as() const { return static_cast<T*>(p); }
+};
+
+// ---------------------------------------------------------------------------------------- quantizer
+
+// Per-token absmax int8 quantizer: s = fl32(m / 127), q = clamp(rint(fl32(v / s)), +-127) with round
+// half to even; an all-zero row gives s = 0, q = 0.  Returns s; writes the code sum.
+float quantize(const float* v, int n, int8_t* q, int* sumq) {
+  float m = 0.0f;
+  for (int i = 0; i < n; ++i) m = std::max(m, std::fabs(v[i]));
+  int sq = 0;
+  if (m == 0.0f) {
+    std::memset(q, 0, (size_t)n);
+    *sumq = 0;
+    return 0.0f;
+  }
+  const float s = m / 127.0f;
+  for (int i = 0; i < n; ++i) {
+    float k = std::nearbyint(v[i] / s);
+    k = std::min(127.0f, std::max(-127.0f, k));
+    q[i] = (int8_t)k;
+    sq += (int)q[i];
+  }
+  *sumq = sq;
+  return s;
+}
+
+// RMSNorm (eps 1e-5, weight w), then the quantizer on the normalised row:
+//   r = fl32(1 / sqrt(sum h^2 / n + eps)) (the fp64 sum in index order, the squares exact),
+//   u = fl32(fl32(h r) w).
+float norm_quantize(const float* h, const float* w, int n, float* u, int8_t* q, int* sumq) {
+  double ss = 0.0;
+  for (int i = 0; i < n; ++i) ss += (double)h[i] * (double)h[i];
+  const float r = f32(1.0 / std::sqrt(ss / (double)n + kEps));
+  for (int i = 0; i < n; ++i) u[i] = (h[i] * r) * w[i];
+  return quantize(u, n, q, sumq);
+}
+
+// ---------------------------------------------------------------------------------------- linear
+
+// acc[b][o] for rows [o0, o1): BT token slots (codes zero-padded to BT tokens and to whole 64-byte
+// chunks), the expanded sign bytes shared by all of them.
+template <int BT>
+__attribute__((target("avx512f,avx512bw,avx512vnni"))) void scaffold_rows(
+    const uint32_t* bits, int d_in, int o0, int o1, const int8_t* qpad, int dpad, const int* sumq, int B,
+    int32_t* acc, int d_out) {
+  const __m512i ones = _mm512_set1_epi8(1);
+  const int words = d_in / 32, full = d_in / 64;
+  for (int o = o0; o < o1; ++o) {
+    const uint32_t* w = bits + (size_t)o * words;
+    __m512i a[BT];
+#pragma GCC unroll 16
+    for (int b = 0; b < BT; ++b) a[b] = _mm512_setzero_si512();
+    for (int c = 0; c < full; ++c) {
+      const uint64_t m = (uint64_t)w[2 * c] | ((uint64_t)w[2 * c + 1] << 32);
+      const __m512i v = _mm512_maskz_mov_epi8((__mmask64)m, ones);
+#pragma GCC unroll 16
+      for (int b = 0; b < BT; ++b)
+        a[b] = _mm512_dpbusd_epi32(a[b], v, _mm512_load_si512(qpad + (size_t)b * dpad + 64 * c));
+    }
+    if (words & 1) {  // d_in % 64 == 32: the last word alone (the codes beyond d_in are zero)
+      const uint64_t m = (uint64_t)w[words - 1];
+      const __m512i v = _mm512_maskz_mov_epi8((__mmask64)m, ones);
+#pragma GCC unroll 16
+      for (int b = 0; b < BT; ++b)
+        a[b] = _mm512_dpbusd_epi32(a[b], v, _mm512_load_si512(qpad + (size_t)b * dpad + 64 * full));
+    }
+    for (int b = 0; b < B; ++b) acc[(size_t)b * d_out + o] = 2 * _mm512_reduce_add_epi32(a[b]) - sumq[b];
+  }
+}
+
+using RowsFn = void (*)(const uint32_t*, int, int, int, const int8_t*, int, const int*, int, int32_t*, int);
+RowsFn rows_fn(int B) {
+  if (B <= 1) return scaffold_rows<1>;
+  if (B <= 2) return scaffold_rows<2>;
+  if (B <= 4) return scaffold_rows<4>;
+  if (B <= 8) return scaffold_rows<8>;
+  return scaffold_rows<16>;
+}
+int slots(int B) { return B <= 1 ? 1 : B <= 2 ? 2 : B <= 4 ? 4 : B <= 8 ? 8 : 16; }
+
+// One linear on B already-quantized tokens: codes q [B][d_in] (natural order), scales s, code sums.
+//   t[r] = sum_i W_B[r,i] q[i] (int32), tf[r] = fl32(t sB s) (fp64, this order)
+//   y[o] = fl32(acc s sW + sA sum_r W_A[o,r] tf[r])  (fp64, left to right; the LoRA sum in r order)
+// out_add: y = fl32(out_add + y) when not null (the residual add), else y is written as is.
+void linear(const dfssm_linear_t& L, const int8_t* q, const float* s, const int* sumq, int B, float* y,
+            const float* out_add, int32_t* dbg_acc, int32_t* dbg_t) {
+  const int d_in = L.d_in, d_out = L.d_out, rank = L.rank;
+  const int BT = slots(B);
+  const int dpad = (d_in + 63) / 64 * 64;
+  Buf qb((size_t)BT * dpad);
+  int8_t* qpad = qb.as<int8_t>();
+  std::memset(qpad, 0, (size_t)BT * dpad);
+  for (int b = 0; b < B; ++b) std::memcpy(qpad + (size_t)b * dpad, q + (size_t)b * d_in, (size_t)d_in);
+  int sq[16] = {0};
+  for (int b = 0; b < B; ++b) sq[b] = sumq[b];
+  // LoRA down-projection
+  std::vector<float> tf((size_t)B * DFSSM_MAX_RANK, 0.0f);
+  for (int b = 0; b < B; ++b)
+    for (int r = 0; r < rank; ++r) {
+      const int8_t* wb = L.lora_b + (size_t)r * d_in;
+      const int8_t* qb8 = q + (size_t)b * d_in;
+      int32_t t = 0;
+      for (int i = 0; i < d_in; ++i) t += (int32_t)wb[i] * (int32_t)qb8[i];
+      if (dbg_t) dbg_t[(size_t)b * rank + r] = t;
+      tf[(size_t)b * DFSSM_MAX_RANK + r] = f32((double)t * (double)L.lora_b_scale[r] * (double)s[b]);
+    }
+  // scaffold accumulators
+  Buf ab((size_t)B * d_out * 4);
+  int32_t* acc = ab.as<int32_t>();
+  const RowsFn fn = rows_fn(B);
+#pragma omp parallel
+  {
+    const int nt = omp_get_num_threads(), it = omp_get_thread_num();
+    const int o0 = (int)((long long)d_out * it / nt), o1 = (int)((long long)d_out * (it + 1) / nt);
+    fn(L.bits, d_in, o0, o1, qpad, dpad, sq, B, acc, d_out);
+  }
+  // epilogue
+#pragma omp parallel for schedule(static)
+  for (int o = 0; o < d_out; ++o) {
+    for (int b = 0; b < B; ++b) {
+      const int a = acc[(size_t)b * d_out + o];
+      double lora = 0.0;
+      for (int r = 0; r < rank; ++r)
+        lora += (double)L.lora_a[(size_t)o * rank + r] * (double)tf[(size_t)b * DFSSM_MAX_RANK + r];
+      const double scaffold = (double)a * (double)s[b] * (double)L.w_scale[o];
+      const double corr = rank > 0 ? (double)L.lora_a_scale[o] * lora : 0.0;
+      const float v = f32(scaffold + corr);
+      const size_t k = (size_t)b * d_out + o;
+      y[k] = out_add ? out_add[k] + v : v;
+      if (dbg_acc) dbg_acc[k] = a;
+    }
+  }
+}
+
+int check_linear(const dfssm_linear_t* L) {
+  if (!L || L->d_out < 1 || L->d_in < 32 || L->d_in % 32 || L->rank < 0 || L->rank > DFSSM_MAX_RANK)
+    return DFSSM_EINVAL;
+  if (L->d_in > 8192) return DFSSM_EUNSUPPORTED;
+  if (!L->bits || !L->w_scale) return DFSSM_EINVAL;
+  if (L->rank > 0 && (!L->lora_b || !L->lora_b_scale || !L->lora_a || !L->lora_a_scale)) return DFSSM_EINVAL;
+  return DFSSM_OK;
+}
+
+// ---------------------------------------------------------------------------------------- stateful
+
+// Width-4 conv step with SiLU on C channels: fl32(b + w0 s0 + w1 s1 + w2 s2 + w3 x) (fp64, this order),
+// then fl32(SiLU), the state shifted by one.
+void conv_step(float* st_all, const float* w, const float* bias, const float* x, float* out, int C) {
+#pragma omp parallel for schedule(static)
+  for (int c = 0; c < C; ++c) {
+    float* st = st_all + (size_t)c * 3;
+    const float* wc = w + (size_t)c * 4;
+    double e = (double)bias[c];
+    e += (double)wc[0] * (double)st[0];
+    e += (double)wc[1] * (double)st[1];
+    e += (double)wc[2] * (double)st[2];
+    e += (double)wc[3] * (double)x[c];
+    out[c] = f32(silu((double)f32(e)));
+    st[0] = st[1];
+    st[1] = st[2];
+    st[2] = x[c];
+  }
+}
+
+// SSM state update and readout of one token:
+//   dt = fl32(softplus(fl32(dt_raw + dt_bias))), A = fl32(-exp(A_log)), dA = fl32(exp(fl32(dt A)))
+//   S <- fl32(fl32(dA S) + fl32(fl32(dt x) B));  y = fl32(sum_n S C + D x) (fp64, n in order)
+// The update is three IEEE fp32 operations per element (vectorised); the readout keeps each row's fp64
+// sum in index order and interleaves eight rows for instruction-level parallelism.
+void ssm_step(float* S_all, const float* x, const float* dt_raw, const float* A_log, const float* dt_bias,
+              const float* Dv, const float* Bm, const float* Cm, float* y, int H, int P, int N, int G) {
+  const int hpg = H / G;
+#pragma omp parallel for schedule(static)
+  for (int h = 0; h < H; ++h) {
+    const int g = h / hpg;
+    const float v = dt_raw[h] + dt_bias[h];
+    const float dt = f32(v > 20.0f ? (double)v : std::log1p(std::exp((double)v)));
+    const float A = f32(-std::exp((double)A_log[h]));
+    const float dA = f32(std::exp((double)(dt * A)));
+    const float* Bg = Bm + (size_t)g * N;
+    const float* Cg = Cm + (size_t)g * N;
+    for (int p0 = 0; p0 < P; p0 += 8) {
+      const int np = std::min(8, P - p0);
+      double acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+      for (int k = 0; k < np; ++k) {
+        const int p = p0 + k;
+        const float dtx = dt * x[(size_t)h * P + p];
+        float* S = S_all + ((size_t)h * P + p) * N;
+        for (int n = 0; n < N; ++n) S[n] = (dA * S[n]) + (dtx * Bg[n]);
+      }
+      for (int n = 0; n < N; ++n) {
+        const double c = (double)Cg[n];
+        for (int k = 0; k < np; ++k) acc[k] += (double)S_all[((size_t)h * P + p0 + k) * N + n] * c;
+      }
+      for (int k = 0; k < np; ++k) {
+        const float xv = x[(size_t)h * P + p0 + k];
+        y[(size_t)h * P + p0 + k] = f32(acc[k] + (double)Dv[h] * (double)xv);
+      }
+    }
+  }
+}
+
+}  // namespace
+
+extern "C" {
+
+int dfssm_cpu_abi_version(void) { return DFSSM_CPU_ABI_VERSION; }
+
+int dfssm_cpu_available(void) { return has_vnni() ? 1 : 0; }
+
+int dfssm_cpu_set_threads(int n) {
+  if (n > 0) omp_set_num_threads(n);
+  else omp_set_num_threads(omp_get_num_procs());
+  return omp_get_max_threads();
+}
+
+int dfssm_cpu_linear_decode(const dfssm_linear_t* lin, const float* x, int B, float* y,
+                            const dfssm_debug_t* dbg) {
+  const int st = check_linear(lin);
+  if (st) return st;
+  if (!x || !y || B < 1 || B > DFSSM_MAX_BATCH) return DFSSM_EINVAL;
+  if (!has_vnni()) return DFSSM_EUNSUPPORTED;
+  const int d_in = lin->d_in;
+  std::vector<int8_t> q((size_t)B * d_in);
+  std::vector<float> s(B);
+  std::vector<int> sq(B);
+  for (int b = 0; b < B; ++b) {
+    s[b] = quantize(x + (size_t)b * d_in, d_in, q.data() + (size_t)b * d_in, &sq[b]);
+    if (dbg && dbg->xscale) dbg->xscale[b] = s[b];
+  }
+  if (dbg && dbg->xq) std::memcpy(dbg->xq, q.data(), q.size());
+  linear(*lin, q.data(), s.data(), sq.data(), B, y, nullptr, dbg ? dbg->acc : nullptr,
+         dbg ? dbg->lora_t : nullptr);
+  return DFSSM_OK;
+}
+
+int dfssm_cpu_layer_decode(const dfssm_layer_t* layers, int n_layers, const dfssm_dims_t* dims,
+                           float* hidden, float* const* conv_states, float* const* ssm_states, int B) {
+  if (!layers || !dims || !hidden || !conv_states || !ssm_states || n_layers < 1 || B < 1 ||
+      B > DFSSM_MAX_BATCH)
+    return DFSSM_EINVAL;
+  if (n_layers > DFSSM_MAX_LAYERS) return DFSSM_EUNSUPPORTED;
+  const int Dm = dims->d_model, H = dims->nheads, P = dims->headdim, N = dims->d_state, G = dims->ngroups;
+  if (Dm < 32 || Dm % 32 || H < 1 || P < 1 || N < 1 || G < 1 || H % G) return DFSSM_EINVAL;
+  const int E = H * P, C = E + 2 * G * N, d_ip = 2 * E + 2 * G * N + H;
+  if (E % 32) return DFSSM_EINVAL;
+  for (int l = 0; l < n_layers; ++l) {
+    const dfssm_layer_t& Ly = layers[l];
+    int st = check_linear(&Ly.in_proj);
+    if (st) return st;
+    st = check_linear(&Ly.out_proj);
+    if (st) return st;
+    if (Ly.in_proj.d_out != d_ip || Ly.in_proj.d_in != Dm || Ly.out_proj.d_out != Dm || Ly.out_proj.d_in != E)
+      return DFSSM_EINVAL;
+    if (!Ly.conv_w || !Ly.conv_b || !Ly.A_log || !Ly.dt_bias || !Ly.D || !Ly.norm_w || !Ly.gnorm_w ||
+        !conv_states[l] || !ssm_states[l])
+      return DFSSM_EINVAL;
+  }
+  if (!has_vnni()) return DFSSM_EUNSUPPORTED;
+  const int nmax = std::max(Dm, E);
+  std::vector<float> u((size_t)nmax), zx((size_t)B * d_ip), xc((size_t)C), y((size_t)E), g((size_t)B * E);
+  std::vector<int8_t> q((size_t)B * nmax);
+  std::vector<float> s(B);
+  std::vector<int> sq(B);
+  for (int l = 0; l < n_layers; ++l) {
+    const dfssm_layer_t& Ly = layers[l];
+    // pre-norm + quantize, in_proj
+    for (int b = 0; b < B; ++b)
+      s[b] = norm_quantize(hidden + (size_t)b * Dm, Ly.norm_w, Dm, u.data(), q.data() + (size_t)b * Dm, &sq[b]);
+    linear(Ly.in_proj, q.data(), s.data(), sq.data(), B, zx.data(), nullptr, nullptr, nullptr);
+    for (int b = 0; b < B; ++b) {
+      const float* zb = zx.data() + (size_t)b * d_ip;
+      // conv on x|B|C, SSM step, gate y SiLU(z)
+      conv_step(conv_states[l] + (size_t)b * C * 3, Ly.conv_w, Ly.conv_b, zb + E, xc.data(), C);
+      ssm_step(ssm_states[l] + (size_t)b * H * P * N, xc.data(), zb + E + C, Ly.A_log, Ly.dt_bias, Ly.D,
+               xc.data() + E, xc.data() + E + G * N, y.data(), H, P, N, G);
+      float* gb = g.data() + (size_t)b * E;
+#pragma omp parallel for schedule(static)
+      for (int i = 0; i < E; ++i) gb[i] = y[i] * f32(silu((double)zb[i]));
+    }
+    // gated norm + quantize, out_proj with the residual add
+    for (int b = 0; b < B; ++b)
+      s[b] = norm_quantize(g.data() + (size_t)b * E, Ly.gnorm_w, E, u.data(), q.data() + (size_t)b * E, &sq[b]);
+    linear(Ly.out_proj, q.data(), s.data(), sq.data(), B, hidden, hidden, nullptr, nullptr);
+  }
+  return DFSSM_OK;
+}
+
+}  // extern "C"

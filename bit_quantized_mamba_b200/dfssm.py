@@ -119,6 +119,27 @@ def _ptr(t):
     return t.data_ptr()
 
 
+def _hptr(t):
+    """Host pointer of a contiguous CPU tensor (the host-CPU engine's arguments)."""
+    if t is None:
+        return None
+    if t.device.type != "cpu":
+        raise ValueError("expected a host (CPU) tensor")
+    if not t.is_contiguous():
+        raise ValueError("expected a contiguous tensor")
+    return t.data_ptr()
+
+
+def _aptr(t, host: bool):
+    return _hptr(t) if host else _ptr(t)
+
+
+def _side(obj, host: bool):
+    if obj.host != host:
+        raise ValueError(f"{type(obj).__name__} lives in {'host' if obj.host else 'device'} memory; "
+                         f"{'the cpu_* calls' if obj.host else 'the CUDA calls'} take it")
+
+
 def _stream(stream):
     if stream is None:
         return torch.cuda.current_stream().cuda_stream
@@ -146,10 +167,11 @@ class Linear:
         self.d_out = bits.shape[0]
         self.d_in = bits.shape[1] * 32
         self.rank = lora_b.shape[0] if lora_b is not None else 0
-        self._c = LinearT(self.d_out, self.d_in, self.rank, _ptr(bits), _ptr(w_scale),
-                          _ptr(lora_b) if self.rank else None,
-                          _ptr(lora_b_scale) if self.rank else None,
-                          _ptr(lora_a) if self.rank else None, _ptr(lora_a_scale) if self.rank else None)
+        self.host = bits.device.type == "cpu"
+        P = lambda t: _aptr(t, self.host)  # noqa: E731
+        self._c = LinearT(self.d_out, self.d_in, self.rank, P(bits), P(w_scale),
+                          P(lora_b) if self.rank else None, P(lora_b_scale) if self.rank else None,
+                          P(lora_a) if self.rank else None, P(lora_a_scale) if self.rank else None)
 
     @classmethod
     def from_host(cls, d: dict, device="cuda"):
@@ -159,7 +181,8 @@ class Linear:
         bits = torch.from_numpy(np.ascontiguousarray(d["bits"]).view(np.int32)).to(device)
         return cls(bits, t["w_scale"], t["lora_b"], t["lora_b_scale"], t["lora_a"], t["lora_a_scale"])
 
-    def cstruct(self) -> LinearT:
+    def cstruct(self, host: bool = False) -> LinearT:
+        _side(self, host)
         return self._c
 
 
@@ -254,7 +277,9 @@ class Layer:
         self.in_proj, self.out_proj = in_proj, out_proj
         for k in self.VEC:
             setattr(self, k, vec[k])
-        self._c = LayerT(in_proj.cstruct(), out_proj.cstruct(), *(_ptr(vec[k]) for k in self.VEC))
+        self.host = in_proj.host
+        self._c = LayerT(in_proj.cstruct(self.host), out_proj.cstruct(self.host),
+                         *(_aptr(vec[k], self.host) for k in self.VEC))
 
     @classmethod
     def from_host(cls, d: dict, device="cuda"):
@@ -262,7 +287,8 @@ class Layer:
         return cls(Linear.from_host(d["in_proj"], device), Linear.from_host(d["out_proj"], device),
                    **vec)
 
-    def cstruct(self) -> LayerT:
+    def cstruct(self, host: bool = False) -> LayerT:
+        _side(self, host)
         return self._c
 
 
@@ -276,10 +302,16 @@ class LayerStack:
                           dims["ngroups"])
         self.d_model = dims["d_model"]
         self.d_inner = dims["nheads"] * dims["headdim"]
-        self._layers = (LayerT * n)(*(L.cstruct() for L in layers))
-        self._conv = (C.c_void_p * n)(*(_ptr(t) for t in conv_states))
-        self._ssm = (C.c_void_p * n)(*(_ptr(t) for t in ssm_states))
+        self.host = layers[0].host
+        self._layers = (LayerT * n)(*(L.cstruct(self.host) for L in layers))
+        self._conv = (C.c_void_p * n)(*(_aptr(t, self.host) for t in conv_states))
+        self._ssm = (C.c_void_p * n)(*(_aptr(t, self.host) for t in ssm_states))
         self.n = n
+
+    def c(self, host: bool = False):
+        """(layers, conv state pointers, SSM state pointers) for a call on that side of the bus."""
+        _side(self, host)
+        return self._layers, self._conv, self._ssm
 
 
 def layer_decode(stack: LayerStack, hidden: torch.Tensor, ws=None, stream=None) -> torch.Tensor:
@@ -289,7 +321,7 @@ def layer_decode(stack: LayerStack, hidden: torch.Tensor, ws=None, stream=None) 
         ws = workspace(workspace_size(OP_LAYER_DECODE, B, stack.d_model, stack.d_inner),
                        hidden.device)
     _check("dfssm_layer_decode", lib().dfssm_layer_decode(
-        stack._layers, stack.n, C.byref(stack.dims), _ptr(hidden), stack._conv, stack._ssm, B,
+        *stack.c()[:1], stack.n, C.byref(stack.dims), _ptr(hidden), *stack.c()[1:], B,
         _ptr(ws), ws.numel(), _stream(stream)))
     return hidden
 
@@ -301,7 +333,7 @@ def layer_prefill(stack: LayerStack, hidden: torch.Tensor, ws=None, stream=None)
     if ws is None:
         ws = workspace(workspace_size(OP_LAYER_PREFILL, M, stack.d_model, stack.d_inner), hidden.device)
     _check("dfssm_layer_prefill", lib().dfssm_layer_prefill(
-        stack._layers, stack.n, C.byref(stack.dims), _ptr(hidden), stack._conv, stack._ssm, M,
+        *stack.c()[:1], stack.n, C.byref(stack.dims), _ptr(hidden), *stack.c()[1:], M,
         _ptr(ws), ws.numel(), _stream(stream)))
     return hidden
 
@@ -367,8 +399,8 @@ def generate(stack: "LayerStack", W, s_row, final_norm_w, tokens, hidden_taps=No
     if ws is None:
         ws = workspace(workspace_size(OP_GENERATE, V, stack.d_model, stack.d_inner), W.device)
     _check("dfssm_generate", lib().dfssm_generate(
-        stack._layers, stack.n, C.byref(stack.dims), _ptr(W), _ptr(s_row), V, _ptr(final_norm_w),
-        _ptr(tokens), n, stack._conv, stack._ssm, _ptr(hidden_taps), _ptr(logits), _ptr(ws),
+        stack.c()[0], stack.n, C.byref(stack.dims), _ptr(W), _ptr(s_row), V, _ptr(final_norm_w),
+        _ptr(tokens), n, stack.c()[1], stack.c()[2], _ptr(hidden_taps), _ptr(logits), _ptr(ws),
         ws.numel(), _stream(stream)))
     return tokens
 
@@ -381,3 +413,61 @@ def pack_signs(signs: np.ndarray) -> np.ndarray:
     _check("dfssm_pack_signs", lib().dfssm_pack_signs(signs.ctypes.data, d_out, d_in,
                                                       bits.ctypes.data))
     return bits
+
+
+# ------------------------------------------------------------------ host-CPU engine (include/dfssm_cpu.h)
+
+CPU_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libdfssm_cpu.so")
+_cpu_lib = None
+
+
+def cpu_lib():
+    """Load libdfssm_cpu.so (built in-tree by bit_quantized_mamba_b200.build.build_cpu); raise if missing."""
+    global _cpu_lib
+    if _cpu_lib is None:
+        if not os.path.exists(CPU_LIB_PATH):
+            raise RuntimeError(f"libdfssm_cpu.so not built ({CPU_LIB_PATH}); run __graft_entry__.build()")
+        L = C.CDLL(CPU_LIB_PATH)
+        L.dfssm_cpu_abi_version.restype = C.c_int
+        L.dfssm_cpu_available.restype = C.c_int
+        L.dfssm_cpu_set_threads.restype = C.c_int
+        L.dfssm_cpu_set_threads.argtypes = [C.c_int]
+        L.dfssm_cpu_linear_decode.restype = C.c_int
+        L.dfssm_cpu_linear_decode.argtypes = [C.POINTER(LinearT), C.c_void_p, C.c_int, C.c_void_p,
+                                              C.POINTER(DebugT)]
+        L.dfssm_cpu_layer_decode.restype = C.c_int
+        L.dfssm_cpu_layer_decode.argtypes = [C.POINTER(LayerT), C.c_int, C.POINTER(DimsT), C.c_void_p,
+                                             C.POINTER(C.c_void_p), C.POINTER(C.c_void_p), C.c_int]
+        _cpu_lib = L
+    return _cpu_lib
+
+
+def cpu_available() -> bool:
+    """True when the host CPU runs the VNNI engine (AVX-512 F/BW and VNNI)."""
+    return bool(cpu_lib().dfssm_cpu_available())
+
+
+def cpu_set_threads(n: int = 0) -> int:
+    return int(cpu_lib().dfssm_cpu_set_threads(n))
+
+
+def cpu_linear_decode(lin: Linear, x: torch.Tensor, y: torch.Tensor | None = None,
+                      debug: dict | None = None) -> torch.Tensor:
+    """dfssm_cpu_linear_decode: lin built with host tensors (Linear.from_host(d, "cpu")), x host f32."""
+    B = x.shape[0]
+    if y is None:
+        y = torch.empty((B, lin.d_out), dtype=torch.float32)
+    dbg = None
+    if debug is not None:
+        dbg = DebugT(*(_hptr(debug.get(k)) for k in ("acc", "lora_t", "xq", "xscale")))
+    _check("dfssm_cpu_linear_decode", cpu_lib().dfssm_cpu_linear_decode(
+        C.byref(lin.cstruct(host=True)), _hptr(x), B, _hptr(y), C.byref(dbg) if dbg is not None else None))
+    return y
+
+
+def cpu_layer_decode(stack: LayerStack, hidden: torch.Tensor) -> torch.Tensor:
+    """dfssm_cpu_layer_decode over a LayerStack of host tensors; hidden [B][d_model] updated in place."""
+    _check("dfssm_cpu_layer_decode", cpu_lib().dfssm_cpu_layer_decode(
+        *stack.c(host=True)[:1], stack.n, C.byref(stack.dims), _hptr(hidden), *stack.c(host=True)[1:],
+        hidden.shape[0]))
+    return hidden

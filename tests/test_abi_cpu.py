@@ -40,6 +40,23 @@ def test_library_exports_every_declared_symbol(L):
     assert L.dfssm_abi_version() == 4
 
 
+def test_cpu_engine_exports_every_declared_symbol():
+    """libdfssm_cpu.so (the host-CPU engine) exports every function include/dfssm_cpu.h declares and
+    validates its arguments before computing (no AVX-512 needed for these calls)."""
+    from bit_quantized_mamba_b200 import build, dfssm
+    build.build_cpu()
+    text = re.sub(r"/\*.*?\*/", "", open(os.path.join(ROOT, "include", "dfssm_cpu.h")).read(), flags=re.S)
+    names = sorted(set(re.findall(r"\b(dfssm_cpu_[a-z0-9_]+)\s*\(", text)))
+    assert len(names) >= 5
+    Lc = dfssm.cpu_lib()
+    for n in names:
+        assert hasattr(Lc, n), f"{n} declared in dfssm_cpu.h but not exported"
+    assert Lc.dfssm_cpu_abi_version() == 1
+    assert Lc.dfssm_cpu_available() in (0, 1)
+    assert Lc.dfssm_cpu_linear_decode(None, None, 1, None, None) == -1
+    assert Lc.dfssm_cpu_layer_decode(None, 0, None, None, None, None, 1) == -1
+
+
 def test_status_strings(L):
     assert L.dfssm_status_string(0) == b"ok"
     assert L.dfssm_status_string(-7).startswith(b"workspace")
