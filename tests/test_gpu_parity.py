@@ -96,6 +96,41 @@ def test_linear_shapes(dev, d_out, d_in, rank, B):
     assert compare_linear(g, r, f"{d_out}x{d_in} r{rank} B{B}") == 0
 
 
+@pytest.mark.parametrize("d_out,d_in,B", [(700, 2048, 16), (300, 1024, 4), (130, 4096, 16)])
+def test_linear_lora_sum_exactness_paths(dev, d_out, d_in, B):
+    """The multi-token epilogue takes a block of eight tokens' LoRA sums on the fp64 tensor core only
+    when every partial sum is exact (each token's nonzero tf within 18 binades), else the sequential
+    chain.  W_B row 15 picks one input (t_15 = q[i0], sB_15 = 1e-5): tokens whose x[i0] quantizes to 127
+    stay exact, tokens with a code of +-1 do not, and x[i0] = 0 gives tf_15 = 0 (exact)."""
+    gen = np.random.default_rng(d_in + B)
+    lin = inputs.linear(gen, d_out, d_in, 16)
+    i0 = 5
+    lin["lora_b"][15] = 0
+    lin["lora_b"][15, i0] = 1
+    lin["lora_b_scale"][15] = np.float32(1e-5)
+    x = inputs.normal(gen, (B, d_in))
+    for b in range(B):
+        x[b, i0] = np.abs(x[b]).max() if b % 3 else 0.0
+    x[B - 1, i0] = np.abs(x[B - 1]).max() / 127.0  # code +-1: its block takes the chain
+    g = run_linear(lin, x, dev)
+    r = oracle.linear_decode(oracle.Linear.from_dict(lin), x)
+    assert compare_linear(g, r, f"exactness paths {d_out}x{d_in} B{B}") == 0
+    assert np.array_equal(g["y"], r["y"])
+
+
+def test_linear_lora_wide_scales(dev):
+    """LoRA-down scales spread over 2^40: every block of the multi-token epilogue takes the sequential
+    chain; outputs bit-identical."""
+    gen = np.random.default_rng(65)
+    lin = inputs.linear(gen, 900, 2048, 16)
+    lin["lora_b_scale"] = (2.0 ** np.linspace(-30, 10, 16)).astype(np.float32)
+    x = inputs.normal(gen, (16, 2048))
+    g = run_linear(lin, x, dev)
+    r = oracle.linear_decode(oracle.Linear.from_dict(lin), x)
+    assert compare_linear(g, r, "wide LoRA scales") == 0
+    assert np.array_equal(g["y"], r["y"])
+
+
 @pytest.mark.parametrize("which", ["in_proj", "out_proj"])
 def test_linear_full_stacks(dev, which):
     """The 48-copy in_proj / out_proj workloads at B = 1, 4, 16: every copy's codes checked, copies
