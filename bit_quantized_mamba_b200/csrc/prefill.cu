@@ -137,17 +137,6 @@ __device__ __forceinline__ void umma_commit(uint64_t* bar) {
                    smem_u32(bar))
                : "memory");
 }
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, "
-      "[%16];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
-        "=r"(r[15])
-      : "r"(taddr));
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-}
-
 // d += A (16 x 4) B (4 x 8) in fp64 on the tensor core (the warp-wide legacy MMA).  Fragments: lane (g, t4)
 // = (lane / 4, lane % 4) holds A[g][t4] (a0) and A[g + 8][t4] (a1), B[t4][g] (b), and D[g][2 t4 + {0, 1}]
 // (d[0], d[1]) and D[g + 8][2 t4 + {0, 1}] (d[2], d[3]).
