@@ -164,6 +164,7 @@ __device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t (&r)[8]) {
 constexpr int QW = 8;  // tokens (warps) per CTA
 static_assert(BN % QW == 0, "the quantizer's CTAs cover whole token tables");
 constexpr int QU = 8;  // float4 loads in flight per lane
+template <bool XREG>  // XREG: K <= 2048, the token's values stay in registers between the passes
 __global__ void __launch_bounds__(QW * 32) prefill_quant_kernel(const float* __restrict__ x, int M, int K,
                                                                const int8_t* __restrict__ lora_b,
                                                                const float* __restrict__ lora_b_scale,
@@ -174,57 +175,55 @@ __global__ void __launch_bounds__(QW * 32) prefill_quant_kernel(const float* __r
   extern __shared__ __align__(16) unsigned char sm[];
   int8_t* wb = reinterpret_cast<int8_t*>(sm);  // [16][K]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // W_B into shared memory: 16-byte loads when W_B is 16-byte aligned (rank K is a multiple of 16),
-  // else eight 4-byte loads in flight per thread
-  if ((reinterpret_cast<uintptr_t>(lora_b) & 15) == 0) {
-    for (int i0 = threadIdx.x * 16; i0 < DFSSM_MAX_RANK * K; i0 += 8 * QW * 32 * 16) {
-      uint4 w[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int i = i0 + u * QW * 32 * 16;
-        w[u] = i < rank * K ? __ldg(reinterpret_cast<const uint4*>(lora_b + i)) : make_uint4(0u, 0u, 0u, 0u);
+  // W_B into shared memory by asynchronous copies (16 bytes when W_B is 16-byte aligned, else 4), rows
+  // past the rank zeroed; awaited just before the codes pass, so the copies overlap the first passes
+  {
+    const bool a16 = (reinterpret_cast<uintptr_t>(lora_b) & 15) == 0;
+    const int step = a16 ? 16 : 4;
+    for (int i = threadIdx.x * step; i < DFSSM_MAX_RANK * K; i += QW * 32 * step) {
+      const uint32_t d = (uint32_t)__cvta_generic_to_shared(wb + i);
+      if (i >= rank * K) {
+        if (a16) *reinterpret_cast<uint4*>(wb + i) = make_uint4(0u, 0u, 0u, 0u);
+        else *reinterpret_cast<uint32_t*>(wb + i) = 0u;
+      } else if (a16) {
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(lora_b + i) : "memory");
+      } else {
+        asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(d), "l"(lora_b + i) : "memory");
       }
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int i = i0 + u * QW * 32 * 16;
-        if (i < DFSSM_MAX_RANK * K) *reinterpret_cast<uint4*>(wb + i) = w[u];
-      }
     }
-  } else
-  for (int i0 = threadIdx.x * 4; i0 < DFSSM_MAX_RANK * K; i0 += 8 * QW * 32 * 4) {
-    uint32_t w[8];
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int i = i0 + u * QW * 32 * 4;
-      w[u] = i < rank * K ? __ldg(reinterpret_cast<const uint32_t*>(lora_b + i)) : 0u;
-    }
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int i = i0 + u * QW * 32 * 4;
-      if (i < DFSSM_MAX_RANK * K) *reinterpret_cast<uint32_t*>(wb + i) = w[u];
-    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
   }
-  __syncthreads();
   const int m = blockIdx.x * QW + warp;
   unsigned char* tb = tab + (size_t)(m / BN) * TAB_BYTES;
   const int mi = m % BN;
-  if (m >= M) {
-    // the last table's tokens past M: zero parameters, trivially exact
-    if (lane < DFSSM_MAX_RANK) reinterpret_cast<float*>(tb + TAB_TF)[mi * DFSSM_MAX_RANK + lane] = 0.0f;
-    if (lane == 0) {
-      reinterpret_cast<double*>(tb + TAB_S)[mi] = 0.0;
-      reinterpret_cast<int*>(tb + TAB_SQ)[mi] = 0;
-      reinterpret_cast<int*>(tb + TAB_EX)[mi] = 1;
-    }
-    return;
-  }
-  const float4* xr = reinterpret_cast<const float4*>(x + (size_t)m * K);
+  const bool active = m < M;  // warps past M reach the staging barrier, then write zero parameters
+  const float4* xr = reinterpret_cast<const float4*>(x + (size_t)(active ? m : 0) * K);
   const float4* wr = reinterpret_cast<const float4*>(norm_w);
   const int K4 = K / 4;  // a multiple of 32: the bounds tests below are uniform over the warp
   constexpr int UB = QU;  // float4 per lane per batch
-  // RMSNorm factor (with a norm weight): a first pass for the sum of squares (exact squares in fp64)
+  constexpr int VR = XREG ? 16 : 1;  // float4 per lane kept in registers (K <= 2048)
+  const int V = K4 / 32;
+  float4 xv[VR];
+  if (XREG && active) {
+#pragma unroll
+    for (int k = 0; k < VR; ++k) xv[k] = k < V ? __ldg(xr + lane + 32 * k) : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  // RMSNorm factor (with a norm weight): a first pass for the sum of squares (exact squares in fp64, each
+  // lane's in increasing index order)
   float rn = 1.0f;
-  if (wr) {
+  if (XREG) {
+    if (wr && active) {
+      double ss = 0.0;
+#pragma unroll
+      for (int k = 0; k < VR; ++k) {
+        ss = fma((double)xv[k].x, (double)xv[k].x, ss);
+        ss = fma((double)xv[k].y, (double)xv[k].y, ss);
+        ss = fma((double)xv[k].z, (double)xv[k].z, ss);
+        ss = fma((double)xv[k].w, (double)xv[k].w, ss);
+      }
+      rn = rms_factor(warp_sum(ss), K);
+    }
+  } else if (wr && active) {
     double ss = 0.0;
     for (int i0 = lane; i0 < K4; i0 += 32 * UB) {
       float4 v[UB];
@@ -249,6 +248,15 @@ __global__ void __launch_bounds__(QW * 32) prefill_quant_kernel(const float* __r
                        norm_value(a.w, rn, w.w));
   };
   float m_abs = 0.0f;
+  if (XREG) {
+    if (active) {
+#pragma unroll
+      for (int k = 0; k < VR; ++k) {
+        if (wr && k < V) xv[k] = scale4(xv[k], lane + 32 * k);
+        m_abs = fmaxf(m_abs, fmaxf(fmaxf(fabsf(xv[k].x), fabsf(xv[k].y)), fmaxf(fabsf(xv[k].z), fabsf(xv[k].w))));
+      }
+    }
+  } else if (active)
   for (int i0 = lane; i0 < K4; i0 += 32 * UB) {
     float4 v[UB];
 #pragma unroll
@@ -275,6 +283,46 @@ __global__ void __launch_bounds__(QW * 32) prefill_quant_kernel(const float* __r
   // inputs l', 8 + l', 16 + l', 24 + l', i.e. byte (l' & 3) of lanes 2b + (l' >> 2) of the block
   const int lb = lane & ~7, lj = lane & 7;
   const uint32_t bsel = (uint32_t)(lj & 3);
+  asm volatile("cp.async.wait_all;" ::: "memory");
+  __syncthreads();  // W_B staged
+  if (!active) {
+    // the last table's tokens past M: zero parameters, trivially exact
+    if (lane < DFSSM_MAX_RANK) reinterpret_cast<float*>(tb + TAB_TF)[mi * DFSSM_MAX_RANK + lane] = 0.0f;
+    if (lane == 0) {
+      reinterpret_cast<double*>(tb + TAB_S)[mi] = 0.0;
+      reinterpret_cast<int*>(tb + TAB_SQ)[mi] = 0;
+      reinterpret_cast<int*>(tb + TAB_EX)[mi] = 1;
+    }
+    return;
+  }
+  // one token group of four values: codes, the bit-sliced gather, the LoRA-down dot products
+  const auto codes4 = [&](const float4 vs, int i) {
+    const float vv[4] = {vs.x, vs.y, vs.z, vs.w};
+    int cd[4];
+    quant_codes<4>(vv, s0, inv_s0, cd);
+    uint32_t packed = 0;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      packed |= ((uint32_t)cd[j] & 0xFFu) << (8 * j);
+      sq += cd[j];
+    }
+    uint32_t g = 0;
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+      const uint32_t v = __shfl_sync(0xffffffffu, packed, lb + 2 * b + (lj >> 2));
+      g |= ((v >> (8 * bsel)) & 0xFFu) << (8 * b);
+    }
+    reinterpret_cast<uint32_t*>(xq + (size_t)m * K)[i] = g;
+    if (dbg_xq) reinterpret_cast<uint32_t*>(dbg_xq + (size_t)m * K)[i] = packed;
+#pragma unroll
+    for (int r = 0; r < DFSSM_MAX_RANK; ++r)
+      u[r] = dp4a_ss(reinterpret_cast<const uint32_t*>(wb + (size_t)r * K)[i], packed, u[r]);
+  };
+  if (XREG) {
+#pragma unroll
+    for (int k = 0; k < VR; ++k)
+      if (k < V) codes4(xv[k], lane + 32 * k);
+  } else
   for (int i0 = lane; i0 < K4; i0 += 32 * UB) {
     float4 v[UB];
 #pragma unroll
@@ -283,29 +331,7 @@ __global__ void __launch_bounds__(QW * 32) prefill_quant_kernel(const float* __r
 #pragma unroll
     for (int q = 0; q < UB; ++q) {
       const int i = i0 + 32 * q;
-      if (i < K4) {
-        const float4 vs = scale4(v[q], i);
-        const float vv[4] = {vs.x, vs.y, vs.z, vs.w};
-        int cd[4];
-        quant_codes<4>(vv, s0, inv_s0, cd);
-        uint32_t packed = 0;
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          packed |= ((uint32_t)cd[j] & 0xFFu) << (8 * j);
-          sq += cd[j];
-        }
-        uint32_t g = 0;
-#pragma unroll
-        for (int b = 0; b < 4; ++b) {
-          const uint32_t v = __shfl_sync(0xffffffffu, packed, lb + 2 * b + (lj >> 2));
-          g |= ((v >> (8 * bsel)) & 0xFFu) << (8 * b);
-        }
-        reinterpret_cast<uint32_t*>(xq + (size_t)m * K)[i] = g;
-        if (dbg_xq) reinterpret_cast<uint32_t*>(dbg_xq + (size_t)m * K)[i] = packed;
-#pragma unroll
-        for (int r = 0; r < DFSSM_MAX_RANK; ++r)
-          u[r] = dp4a_ss(reinterpret_cast<const uint32_t*>(wb + (size_t)r * K)[i], packed, u[r]);
-      }
+      if (i < K4) codes4(scale4(v[q], i), i);
     }
   }
 #pragma unroll
@@ -811,10 +837,11 @@ int dfssm::linear_prefill_impl(const dfssm_linear_t* lin, const float* x, int M,
 
   // 1. per-token quantization and LoRA down-projection (one warp per token)
   const size_t qsmem = (size_t)DFSSM_MAX_RANK * K;  // W_B padded to sixteen rows
-  const cudaError_t ea = set_max_dynamic_smem(reinterpret_cast<const void*>(prefill::prefill_quant_kernel), 16 * 8192);
+  const auto qk = K <= 2048 ? prefill::prefill_quant_kernel<true> : prefill::prefill_quant_kernel<false>;
+  const cudaError_t ea = set_max_dynamic_smem(reinterpret_cast<const void*>(qk), 16 * 8192);
   if (ea != cudaSuccess) return record_cuda_failure(ea);
   const int m_pad = (M + prefill::BN - 1) / prefill::BN * prefill::BN;  // whole token tables
-  prefill::prefill_quant_kernel<<<m_pad / prefill::QW, prefill::QW * 32, qsmem, st>>>(
+  qk<<<m_pad / prefill::QW, prefill::QW * 32, qsmem, st>>>(
       x, M, K, lin->lora_b, lin->lora_b_scale, lin->rank, norm_w, w.xq, w.tab, dbg ? dbg->xq : nullptr,
       dbg ? dbg->xscale : nullptr, dbg ? dbg->lora_t : nullptr);
   cudaError_t e = cudaGetLastError();
