@@ -85,33 +85,76 @@ float norm_quantize(const float* h, const float* w, int n, float* u, int8_t* q, 
 // ---------------------------------------------------------------------------------------- linear
 
 // acc[b][o] for rows [o0, o1): BT token slots (codes zero-padded to BT tokens and to whole 64-byte
-// chunks), the expanded sign bytes shared by all of them.
+// chunks), the expanded sign bytes shared by all of them.  With fewer than four tokens each token keeps
+// U = 4 / BT partial sums over alternating chunks, so that U vpdpbusd chains run side by side (integer
+// sums: the order does not change the result).
 template <int BT>
 __attribute__((target("avx512f,avx512bw,avx512vnni"))) void scaffold_rows(
     const uint32_t* bits, int d_in, int o0, int o1, const int8_t* qpad, int dpad, const int* sumq, int B,
     int32_t* acc, int d_out) {
+  constexpr int U = BT >= 4 ? 1 : 4 / BT;
   const __m512i ones = _mm512_set1_epi8(1);
   const int words = d_in / 32, full = d_in / 64;
   for (int o = o0; o < o1; ++o) {
     const uint32_t* w = bits + (size_t)o * words;
-    __m512i a[BT];
+    __m512i a[U][BT];
 #pragma GCC unroll 16
-    for (int b = 0; b < BT; ++b) a[b] = _mm512_setzero_si512();
-    for (int c = 0; c < full; ++c) {
+    for (int u = 0; u < U; ++u)
+#pragma GCC unroll 16
+      for (int b = 0; b < BT; ++b) a[u][b] = _mm512_setzero_si512();
+    int c = 0;
+    for (; c + U <= full; c += U) {
+#pragma GCC unroll 4
+      for (int u = 0; u < U; ++u) {
+        const uint64_t m = (uint64_t)w[2 * (c + u)] | ((uint64_t)w[2 * (c + u) + 1] << 32);
+        const __m512i v = _mm512_maskz_mov_epi8((__mmask64)m, ones);
+#pragma GCC unroll 16
+        for (int b = 0; b < BT; ++b)
+          a[u][b] = _mm512_dpbusd_epi32(a[u][b], v, _mm512_load_si512(qpad + (size_t)b * dpad + 64 * (c + u)));
+      }
+    }
+    for (; c < full; ++c) {
       const uint64_t m = (uint64_t)w[2 * c] | ((uint64_t)w[2 * c + 1] << 32);
       const __m512i v = _mm512_maskz_mov_epi8((__mmask64)m, ones);
 #pragma GCC unroll 16
       for (int b = 0; b < BT; ++b)
-        a[b] = _mm512_dpbusd_epi32(a[b], v, _mm512_load_si512(qpad + (size_t)b * dpad + 64 * c));
+        a[0][b] = _mm512_dpbusd_epi32(a[0][b], v, _mm512_load_si512(qpad + (size_t)b * dpad + 64 * c));
     }
     if (words & 1) {  // d_in % 64 == 32: the last word alone (the codes beyond d_in are zero)
       const uint64_t m = (uint64_t)w[words - 1];
       const __m512i v = _mm512_maskz_mov_epi8((__mmask64)m, ones);
 #pragma GCC unroll 16
       for (int b = 0; b < BT; ++b)
-        a[b] = _mm512_dpbusd_epi32(a[b], v, _mm512_load_si512(qpad + (size_t)b * dpad + 64 * full));
+        a[0][b] = _mm512_dpbusd_epi32(a[0][b], v, _mm512_load_si512(qpad + (size_t)b * dpad + 64 * full));
     }
-    for (int b = 0; b < B; ++b) acc[(size_t)b * d_out + o] = 2 * _mm512_reduce_add_epi32(a[b]) - sumq[b];
+    for (int b = 0; b < B; ++b) {
+      __m512i t = a[0][b];
+#pragma GCC unroll 4
+      for (int u = 1; u < U; ++u) t = _mm512_add_epi32(t, a[u][b]);
+      acc[(size_t)b * d_out + o] = 2 * _mm512_reduce_add_epi32(t) - sumq[b];
+    }
+  }
+}
+
+// t[r] = sum_i W_B[r,i] q[i] for one token (exact int32): vpdpbusd multiplies unsigned by signed bytes,
+// so the codes enter as q + 128 (1..255) and 128 sum_i W_B[r,i] is taken off afterwards.
+__attribute__((target("avx512f,avx512bw,avx512vnni"))) void lora_down_vnni(const int8_t* wb, int rank,
+                                                                            int d_in, const int8_t* qpad,
+                                                                            int32_t* t) {
+  const __m512i bias = _mm512_set1_epi8((char)0x80), ones = _mm512_set1_epi8(1);
+  const int chunks = (d_in + 63) / 64;
+  for (int r = 0; r < rank; ++r) {
+    const int8_t* w = wb + (size_t)r * d_in;
+    __m512i acc = _mm512_setzero_si512(), wsum = _mm512_setzero_si512();
+    for (int c = 0; c < chunks; ++c) {
+      const int n = std::min(64, d_in - 64 * c);
+      const __mmask64 k = n == 64 ? ~0ull : ((1ull << n) - 1ull);
+      const __m512i wv = _mm512_maskz_loadu_epi8(k, w + 64 * c);
+      const __m512i qv = _mm512_xor_si512(_mm512_load_si512(qpad + 64 * c), bias);  // q + 128 as u8
+      acc = _mm512_dpbusd_epi32(acc, qv, wv);
+      wsum = _mm512_dpbusd_epi32(wsum, ones, wv);
+    }
+    t[r] = _mm512_reduce_add_epi32(acc) - 128 * _mm512_reduce_add_epi32(wsum);
   }
 }
 
@@ -140,42 +183,49 @@ void linear(const dfssm_linear_t& L, const int8_t* q, const float* s, const int*
   for (int b = 0; b < B; ++b) std::memcpy(qpad + (size_t)b * dpad, q + (size_t)b * d_in, (size_t)d_in);
   int sq[16] = {0};
   for (int b = 0; b < B; ++b) sq[b] = sumq[b];
-  // LoRA down-projection
+  // LoRA down-projection (the padded codes past d_in are zero and the masked W_B loads read nothing there)
   std::vector<float> tf((size_t)B * DFSSM_MAX_RANK, 0.0f);
-  for (int b = 0; b < B; ++b)
+  for (int b = 0; b < B; ++b) {
+    int32_t t[DFSSM_MAX_RANK];
+    lora_down_vnni(L.lora_b, rank, d_in, qpad + (size_t)b * dpad, t);
     for (int r = 0; r < rank; ++r) {
-      const int8_t* wb = L.lora_b + (size_t)r * d_in;
-      const int8_t* qb8 = q + (size_t)b * d_in;
-      int32_t t = 0;
-      for (int i = 0; i < d_in; ++i) t += (int32_t)wb[i] * (int32_t)qb8[i];
-      if (dbg_t) dbg_t[(size_t)b * rank + r] = t;
-      tf[(size_t)b * DFSSM_MAX_RANK + r] = f32((double)t * (double)L.lora_b_scale[r] * (double)s[b]);
+      if (dbg_t) dbg_t[(size_t)b * rank + r] = t[r];
+      tf[(size_t)b * DFSSM_MAX_RANK + r] = f32((double)t[r] * (double)L.lora_b_scale[r] * (double)s[b]);
     }
-  // scaffold accumulators
+  }
+  // scaffold accumulators, then the epilogue of the same rows, in chunks of 64 rows handed out as threads
+  // come free (the cores of a shared host run at uneven speeds)
   Buf ab((size_t)B * d_out * 4);
   int32_t* acc = ab.as<int32_t>();
   const RowsFn fn = rows_fn(B);
-#pragma omp parallel
-  {
-    const int nt = omp_get_num_threads(), it = omp_get_thread_num();
-    const int o0 = (int)((long long)d_out * it / nt), o1 = (int)((long long)d_out * (it + 1) / nt);
+  constexpr int kChunk = 64;
+  const int chunks = (d_out + kChunk - 1) / kChunk;
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int ci = 0; ci < chunks; ++ci) {
+    const int o0 = ci * kChunk, o1 = std::min(d_out, o0 + kChunk);
     fn(L.bits, d_in, o0, o1, qpad, dpad, sq, B, acc, d_out);
-  }
-  // epilogue
-#pragma omp parallel for schedule(static)
-  for (int o = 0; o < d_out; ++o) {
-    for (int b = 0; b < B; ++b) {
-      const int a = acc[(size_t)b * d_out + o];
-      double lora = 0.0;
-      for (int r = 0; r < rank; ++r)
-        lora += (double)L.lora_a[(size_t)o * rank + r] * (double)tf[(size_t)b * DFSSM_MAX_RANK + r];
-      const double scaffold = (double)a * (double)s[b] * (double)L.w_scale[o];
-      const double corr = rank > 0 ? (double)L.lora_a_scale[o] * lora : 0.0;
-      const float v = f32(scaffold + corr);
-      const size_t k = (size_t)b * d_out + o;
-      y[k] = out_add ? out_add[k] + v : v;
-      if (dbg_acc) dbg_acc[k] = a;
+  // epilogue, eight outputs at a time so that their LoRA sums (each in r order) run side by side
+  for (int b = 0; b < B; ++b) {
+    const float* tb = tf.data() + (size_t)b * DFSSM_MAX_RANK;
+    for (int ob = o0; ob < o1; ob += 8) {
+      const int no = std::min(8, o1 - ob);
+      double lora[8] = {};
+      for (int r = 0; r < rank; ++r) {
+        const double t = (double)tb[r];
+        for (int k = 0; k < no; ++k) lora[k] += (double)L.lora_a[(size_t)(ob + k) * rank + r] * t;
+      }
+      for (int k = 0; k < no; ++k) {
+        const int o = ob + k;
+        const size_t i = (size_t)b * d_out + o;
+        const int a = acc[i];
+        const double scaffold = (double)a * (double)s[b] * (double)L.w_scale[o];
+        const double corr = rank > 0 ? (double)L.lora_a_scale[o] * lora[k] : 0.0;
+        const float v = f32(scaffold + corr);
+        y[i] = out_add ? out_add[i] + v : v;
+        if (dbg_acc) dbg_acc[i] = a;
+      }
     }
+  }
   }
 }
 
@@ -209,14 +259,70 @@ void conv_step(float* st_all, const float* w, const float* bias, const float* x,
   }
 }
 
+// 8 R rows of one head (R groups of eight), n in [0, N8) with N8 a multiple of 8: the update as three
+// fp32 vector operations per element (no fusion), the readout products fl64(S) fl64(C) (exact) turned
+// from row-major 8 x 8 blocks into columns by an 8 x 8 transpose, so that lane k of group j accumulates
+// row 8j + k's sum in index order.  The R groups' add chains run side by side.
+template <int R>
+__attribute__((target("avx512f"))) void ssm_rows8(float* S, int N, int N8, float dA, const float* dtx,
+                                                   const float* Bg, const float* Cg, double* acc_out) {
+  const __m256 vdA = _mm256_set1_ps(dA);
+  __m512d acc[R];
+#pragma GCC unroll 2
+  for (int j = 0; j < R; ++j) acc[j] = _mm512_setzero_pd();
+  const __m512i lo2 = _mm512_setr_epi64(0, 1, 8, 9, 4, 5, 12, 13), hi2 = _mm512_setr_epi64(2, 3, 10, 11, 6, 7, 14, 15);
+  const __m512i lo4 = _mm512_setr_epi64(0, 1, 2, 3, 8, 9, 10, 11), hi4 = _mm512_setr_epi64(4, 5, 6, 7, 12, 13, 14, 15);
+  for (int n = 0; n < N8; n += 8) {
+    const __m256 vb = _mm256_loadu_ps(Bg + n);
+    const __m512d vc = _mm512_cvtps_pd(_mm256_loadu_ps(Cg + n));
+#pragma GCC unroll 2
+    for (int j = 0; j < R; ++j) {
+      __m512d r[8];
+#pragma GCC unroll 8
+      for (int k = 0; k < 8; ++k) {
+        float* Sk = S + (size_t)(8 * j + k) * N + n;
+        const __m256 upd = _mm256_add_ps(_mm256_mul_ps(vdA, _mm256_loadu_ps(Sk)),
+                                         _mm256_mul_ps(_mm256_set1_ps(dtx[8 * j + k]), vb));
+        _mm256_storeu_ps(Sk, upd);
+        r[k] = _mm512_mul_pd(_mm512_cvtps_pd(upd), vc);
+      }
+      __m512d a[8], b[8];
+#pragma GCC unroll 4
+      for (int k = 0; k < 8; k += 2) {
+        a[k] = _mm512_unpacklo_pd(r[k], r[k + 1]);      // columns 0, 2, 4, 6 of rows k, k+1
+        a[k + 1] = _mm512_unpackhi_pd(r[k], r[k + 1]);  // columns 1, 3, 5, 7
+      }
+#pragma GCC unroll 2
+      for (int k = 0; k < 8; k += 4) {
+        b[k] = _mm512_permutex2var_pd(a[k], lo2, a[k + 2]);          // columns 0, 4 of rows k..k+3
+        b[k + 2] = _mm512_permutex2var_pd(a[k], hi2, a[k + 2]);      // columns 2, 6
+        b[k + 1] = _mm512_permutex2var_pd(a[k + 1], lo2, a[k + 3]);  // columns 1, 5
+        b[k + 3] = _mm512_permutex2var_pd(a[k + 1], hi2, a[k + 3]);  // columns 3, 7
+      }
+      __m512d t = acc[j];
+      t = _mm512_add_pd(t, _mm512_permutex2var_pd(b[0], lo4, b[4]));  // column 0
+      t = _mm512_add_pd(t, _mm512_permutex2var_pd(b[1], lo4, b[5]));  // column 1
+      t = _mm512_add_pd(t, _mm512_permutex2var_pd(b[2], lo4, b[6]));  // column 2
+      t = _mm512_add_pd(t, _mm512_permutex2var_pd(b[3], lo4, b[7]));  // column 3
+      t = _mm512_add_pd(t, _mm512_permutex2var_pd(b[0], hi4, b[4]));  // column 4
+      t = _mm512_add_pd(t, _mm512_permutex2var_pd(b[1], hi4, b[5]));  // column 5
+      t = _mm512_add_pd(t, _mm512_permutex2var_pd(b[2], hi4, b[6]));  // column 6
+      t = _mm512_add_pd(t, _mm512_permutex2var_pd(b[3], hi4, b[7]));  // column 7
+      acc[j] = t;
+    }
+  }
+#pragma GCC unroll 2
+  for (int j = 0; j < R; ++j) _mm512_storeu_pd(acc_out + 8 * j, acc[j]);
+}
+
 // SSM state update and readout of one token:
 //   dt = fl32(softplus(fl32(dt_raw + dt_bias))), A = fl32(-exp(A_log)), dA = fl32(exp(fl32(dt A)))
 //   S <- fl32(fl32(dA S) + fl32(fl32(dt x) B));  y = fl32(sum_n S C + D x) (fp64, n in order)
-// The update is three IEEE fp32 operations per element (vectorised); the readout keeps each row's fp64
-// sum in index order and interleaves eight rows for instruction-level parallelism.
+// Rows go sixteen (or eight) at a time through ssm_rows8 for the whole multiple of 8 in n; the rest of n,
+// and the rows left over when P % 8 != 0, continue each row's sum one term at a time.
 void ssm_step(float* S_all, const float* x, const float* dt_raw, const float* A_log, const float* dt_bias,
               const float* Dv, const float* Bm, const float* Cm, float* y, int H, int P, int N, int G) {
-  const int hpg = H / G;
+  const int hpg = H / G, N8 = N / 8 * 8;
 #pragma omp parallel for schedule(static)
   for (int h = 0; h < H; ++h) {
     const int g = h / hpg;
@@ -226,22 +332,29 @@ void ssm_step(float* S_all, const float* x, const float* dt_raw, const float* A_
     const float dA = f32(std::exp((double)(dt * A)));
     const float* Bg = Bm + (size_t)g * N;
     const float* Cg = Cm + (size_t)g * N;
-    for (int p0 = 0; p0 < P; p0 += 8) {
-      const int np = std::min(8, P - p0);
-      double acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-      for (int k = 0; k < np; ++k) {
-        const int p = p0 + k;
-        const float dtx = dt * x[(size_t)h * P + p];
-        float* S = S_all + ((size_t)h * P + p) * N;
-        for (int n = 0; n < N; ++n) S[n] = (dA * S[n]) + (dtx * Bg[n]);
+    for (int p0 = 0; p0 < P; p0 += 16) {
+      const int np = std::min(16, P - p0);
+      double acc[16] = {};
+      float dtx[16];
+      for (int k = 0; k < np; ++k) dtx[k] = dt * x[(size_t)h * P + p0 + k];
+      float* S0 = S_all + ((size_t)h * P + p0) * N;
+      int n0 = 0, nv = 0;  // the first nv rows went through ssm_rows8 for n < n0
+      if (N8 > 0 && np == 16) {
+        ssm_rows8<2>(S0, N, N8, dA, dtx, Bg, Cg, acc);
+        n0 = N8, nv = 16;
+      } else if (N8 > 0 && np >= 8) {
+        ssm_rows8<1>(S0, N, N8, dA, dtx, Bg, Cg, acc);
+        n0 = N8, nv = 8;
       }
-      for (int n = 0; n < N; ++n) {
-        const double c = (double)Cg[n];
-        for (int k = 0; k < np; ++k) acc[k] += (double)S_all[((size_t)h * P + p0 + k) * N + n] * c;
-      }
       for (int k = 0; k < np; ++k) {
+        float* S = S0 + (size_t)k * N;
+        double a = acc[k];
+        for (int n = k < nv ? n0 : 0; n < N; ++n) {
+          S[n] = (dA * S[n]) + (dtx[k] * Bg[n]);
+          a += (double)S[n] * (double)Cg[n];
+        }
         const float xv = x[(size_t)h * P + p0 + k];
-        y[(size_t)h * P + p0 + k] = f32(acc[k] + (double)Dv[h] * (double)xv);
+        y[(size_t)h * P + p0 + k] = f32(a + (double)Dv[h] * (double)xv);
       }
     }
   }

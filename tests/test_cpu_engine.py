@@ -77,10 +77,12 @@ def _stack(model, conv, ssm, dims):
     (dict(d_model=256, nheads=4, headdim=32, d_state=16, ngroups=1, rank=16), 1, 3, 4),
     (dict(d_model=128, nheads=4, headdim=32, d_state=24, ngroups=2, rank=5), 3, 2, 3),
     (dict(d_model=2048, nheads=64, headdim=64, d_state=128, ngroups=1, rank=16), 1, 2, 2),
+    (dict(d_model=64, nheads=8, headdim=28, d_state=12, ngroups=2, rank=3), 2, 2, 3),
 ])
 def test_layer_decode_matches_oracle(engine, dims, B, n_layers, n_tokens):
     """Several tokens through a stack: the residual stream and both states bit-identical to the oracle
-    after every token (the 1.3B layer shape included)."""
+    after every token (the 1.3B layer shape included; headdim 28 and d_state 12 take every branch of
+    the SSM step: sixteen rows, eight rows, single rows, and state columns past the eight-wide blocks)."""
     d = dict(dims)
     model = inputs.decode_model(seed=21, n_layers=n_layers, n_tokens=n_tokens, batch=B, **d)
     conv, ssm = inputs.zero_states(B, n_layers, d["nheads"], d["headdim"], d["d_state"], d["ngroups"])
