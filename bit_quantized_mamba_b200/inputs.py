@@ -18,6 +18,8 @@ no distribution is given):
   LM head W                      int8 uniform on [-127, 127];  row scales* U(1e-4, 1e-3)
   tied embedding / LM head*      one int8 matrix as the LM head;  final RMSNorm weight* U(0.5, 1.5)
   first token of a generation*   uniform on [0, vocab)
+  SSM state rows (density field)* N(0, 1) times a per-row magnitude 10^U(-3, 1); every 64th row all
+                                 zero, every 64th (offset 32) one nonzero value (a spike)
 """
 from __future__ import annotations
 
@@ -149,3 +151,19 @@ def zero_states(batch: int = 1, n_layers: int = N_LAYERS, nheads: int = N_HEADS,
     conv = np.zeros((n_layers, batch, c, D_CONV - 1), np.float32)
     ssm = np.zeros((n_layers, batch, nheads, headdim, d_state), np.float32)
     return conv, ssm
+
+
+def ssm_state_rows(seed: int, rows: int, d_state: int = D_STATE) -> np.ndarray:
+    """State rows [rows][d_state] for the density-field encoding: per-row magnitudes spread over four
+    decades, with all-zero rows and single-spike rows mixed in (fixed positions)."""
+    g = rng(seed)
+    mag = (10.0 ** g.uniform(-3.0, 1.0, size=(rows, 1))).astype(np.float32)
+    S = (g.standard_normal((rows, d_state), dtype=np.float32) * mag).astype(np.float32)
+    S[0::64] = 0.0
+    spikes = np.arange(32, rows, 64)
+    if len(spikes):
+        pos = g.integers(0, d_state, size=len(spikes))
+        val = g.standard_normal(len(spikes), dtype=np.float32)
+        S[spikes] = 0.0
+        S[spikes, pos] = val
+    return S

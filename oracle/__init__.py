@@ -49,6 +49,8 @@ def _declare(L):
     L.oracle_embed.argtypes = [_P, _P, _I, _I, _I, _P]
     L.oracle_embed.restype = _I
     L.oracle_final_head.argtypes = [_P, _P, _I, _I, _P, _P, _P, _I, _P, _P]
+    L.oracle_field_encode.argtypes = [_P, _I, _I, _P, _P]
+    L.oracle_field_decode.argtypes = [_P, _P, _I, _I, _P]
 
 
 def _p(a):
@@ -323,3 +325,28 @@ def layer_prefill(layers, h, conv_states, ssm_states):
         for t in range(h.shape[0]):
             layer_decode(L, h[t:t + 1], cs, ss)
     return h
+
+
+def field_encode(state):
+    """Density-field encoding of state rows [..., N] (N % 8 == 0): returns (field uint32 [rows, N/8],
+    scale float32 [rows]) with rows = the product of the leading dimensions."""
+    S = _c(state, np.float32)
+    N = S.shape[-1]
+    assert N % 8 == 0 and N > 0
+    S = S.reshape(-1, N)
+    rows = S.shape[0]
+    field = np.zeros((rows, N // 8), np.uint32)
+    scale = np.zeros(rows, np.float32)
+    lib().oracle_field_encode(_p(S), rows, N, _p(field), _p(scale))
+    return field, scale
+
+
+def field_decode(field, scale, N: int):
+    """Popcount readout of density fields [rows, N/8] with their scales [rows] -> state rows [rows, N]."""
+    F = _c(field, np.uint32).reshape(-1, N // 8)
+    sc = _c(scale, np.float32).reshape(-1)
+    rows = F.shape[0]
+    assert sc.shape[0] == rows
+    out = np.zeros((rows, N), np.float32)
+    lib().oracle_field_decode(_p(F), _p(sc), rows, N, _p(out))
+    return out

@@ -10,6 +10,7 @@
 //           Organization in Mamba-2" (arXiv 2606.10932), abstract.
 //   [TS-2B] gist.science technical summary of the same paper, §2.B "Frozen Scaffold with LoRA Correction".
 //   [TS-2C] same summary, §2.C "Optimized Inference Pipeline".
+//   [TS-2D] same summary, §2.D "Density Field State Representation".
 //   [TS-3]  same summary, §3 "Key Results" (model size and composition).
 //   [MAP]   mlsanity.com citation map of the paper, "Builds on": Mamba; "Transformers are SSMs ...
 //           Structured State Space Duality" (Mamba-2 / SSD).  The Mamba-2 block itself is only cited,
@@ -130,7 +131,7 @@ inline double silu64(double v) { return v / (1.0 + std::exp(-v)); }
 
 extern "C" {
 
-int oracle_abi_version(void) { return 5; }
+int oracle_abi_version(void) { return 6; }
 
 // Host threads the OpenMP loops of this library use (timing of the CPU baseline); returns the previous
 // maximum.  No arithmetic.
@@ -415,6 +416,72 @@ void oracle_final_head(const int8_t* W, const float* s_row, int V, int d, const 
     for (int i = 0; i < d; ++i) a += (int64_t)W[(size_t)vrow * d + i] * (int64_t)q[i];
     if (acc_out) acc_out[k] = (int32_t)a;
     logits[k] = r32((double)a * (double)s * (double)s_row[vrow]);
+  }
+}
+
+// ---------------------------------------------------------------------------------- density field
+//
+// [TS-2D]: the SSM hidden state is kept as a K x K binary field per state element with K^2 about
+// 4 d_state; normalization, sigma-delta injection (error feedback), binarization, and a popcount readout
+// that recovers continuous values, at chunk boundaries.  Reading (F4): a "state element" is one state
+// row S[h][p][0..N) (N = d_state values), its field is 4N cells (four per value, so K^2 = 4N), and:
+//   normalization   c = max_n |S_n| (fp32); x_n = fl32(S_n / c), x_n = 0 when c = 0;
+//                   d_n = fl32(x_n + 1) / 2, a density in [0, 1];
+//   injection       the cells j = 4n + k (k = 0..3) in order, each fed its value's density d_n, through
+//                   a first-order sigma-delta modulator: v = d + e, b_j = [v >= 1/2], e = v - b_j,
+//                   with e = 0 before the first cell of the row;
+//   binarization    b_j, stored least significant bit first: cell j is bit j % 32 of word j / 32 (value
+//                   n is nibble n % 8 of word n / 8), N / 8 words per row, beside c;
+//   readout         p_n = popcount of value n's four cells, S^_n = fl32(c (p_n / 2 - 1)).
+// Every density is a multiple of 2^-25 (fl32(x + 1) is a multiple of 2^-24 for |x| <= 1) and |v| < 2,
+// so the modulator below runs exactly in fp64.
+// Pinned by: a hand-derived row (tests/golden/density_field.txt); the closed form of the first-order
+// modulator (ones among the first j + 1 cells = floor(P_j + 1/2), P_j the exact sum of their
+// densities); exact round trips of the five levels c {-1, -1/2, 0, 1/2, 1}; the running readout error
+// bounded by c / 4; the zero row.
+void oracle_field_encode(const float* state, int rows, int N, uint32_t* field, float* scale) {
+  const int words = N / 8;
+#pragma omp parallel for schedule(static)
+  for (int r = 0; r < rows; ++r) {
+    const float* S = state + (size_t)r * N;
+    uint32_t* F = field + (size_t)r * words;
+    float c = 0.0f;
+    for (int n = 0; n < N; ++n) {
+      const float a = std::fabs(S[n]);
+      if (a > c) c = a;
+    }
+    for (int w = 0; w < words; ++w) F[w] = 0u;
+    double e = 0.0;
+    for (int n = 0; n < N; ++n) {
+      const float x = c > 0.0f ? r32((double)S[n] / (double)c) : 0.0f;
+      const float d = r32((double)r32((double)x + 1.0) * 0.5);
+      for (int k = 0; k < 4; ++k) {
+        const double v = (double)d + e;
+        const int b = v >= 0.5 ? 1 : 0;
+        e = v - (double)b;
+        const int j = 4 * n + k;
+        F[j / 32] |= (uint32_t)b << (j % 32);
+      }
+    }
+    scale[r] = c;
+  }
+}
+
+// The readout of oracle_field_encode's fields: S^_n = fl32(c (popcount(cells of n) / 2 - 1)).
+// Pinned with oracle_field_encode (above).
+void oracle_field_decode(const uint32_t* field, const float* scale, int rows, int N, float* state) {
+  const int words = N / 8;
+#pragma omp parallel for schedule(static)
+  for (int r = 0; r < rows; ++r) {
+    const uint32_t* F = field + (size_t)r * words;
+    for (int n = 0; n < N; ++n) {
+      int p = 0;
+      for (int k = 0; k < 4; ++k) {
+        const int j = 4 * n + k;
+        p += (int)((F[j / 32] >> (j % 32)) & 1u);
+      }
+      state[(size_t)r * N + n] = r32((double)scale[r] * ((double)p * 0.5 - 1.0));
+    }
   }
 }
 
