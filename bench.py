@@ -526,6 +526,7 @@ def run_ours(args, rank, world, local_rank):
                     "last_token": int(toks[-1].item())}
         ggraph = None
         del GW
+    state_field = measure_state_field(dev, flush, hbm) if not args.no_extras else {}
     del flush
     torch.cuda.synchronize()
 
@@ -554,6 +555,7 @@ def run_ours(args, rank, world, local_rank):
         "prefill": prefill,
         "prefill_layers": prefill_layers,
         "generate": generate,
+        "state_field": state_field,
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": N_TOKENS * 2048 * 4,
                 "d2h_bytes_per_step": 2048 * 4},
         "gpu_launches": args.steps * N_TOKENS,
@@ -609,6 +611,84 @@ def vnni_engine_rate(cores, n_tokens=8):
     dt = time.perf_counter() - t0
     return {"value": (n_tokens - 1) / dt, "unit": "tokens/s", "cores": cores, "kind": "vnni_engine",
             "sample": f"tokens 1..{n_tokens - 1} of the 64-token decode, 48 layers, on {cores} threads"}
+
+
+FIELD_ROWS = 48 * 64 * 64   # the 48-layer Mamba-2-1.3B SSM state at batch 1: 196,608 rows of d_state 128
+FIELD_N = 128
+
+
+def measure_state_field(dev, flush, hbm, reps=10):
+    """Density-field encode, readout and in-place round trip of the whole 48-layer SSM state (technical
+    summary §2.D), each call timed alone with CUDA events on its stream, L2 flushed before each.
+    Algorithmic bytes per row: encode 4N read + N/2 + 4 written; readout N/2 + 4 read + 4N written;
+    round trip 4N read + 4N written."""
+    import torch
+    from bit_quantized_mamba_b200 import dfssm, inputs
+    state = torch.from_numpy(inputs.ssm_state_rows(seed=77, rows=FIELD_ROWS, d_state=FIELD_N)).to(dev)
+    work = state.clone()
+    field = torch.empty((FIELD_ROWS, FIELD_N // 8), dtype=torch.int32, device=dev)
+    scale = torch.empty(FIELD_ROWS, dtype=torch.float32, device=dev)
+    out = torch.empty_like(state)
+    per_row = {"encode": 4 * FIELD_N + FIELD_N // 2 + 4, "decode": 4 * FIELD_N + FIELD_N // 2 + 4,
+               "roundtrip": 8 * FIELD_N}
+    calls = {"encode": lambda st: dfssm.state_field_encode(state, field, scale, stream=st),
+             "decode": lambda st: dfssm.state_field_decode(field, scale, FIELD_N, out, stream=st),
+             "roundtrip": lambda st: dfssm.state_field_roundtrip(work, stream=st)}
+    res = {"rows": FIELD_ROWS, "d_state": FIELD_N, "bits_per_value": 4,
+           "kernels": "dfssm::field_encode_kernel, dfssm::field_decode_kernel (one launch per call)"}
+    stream = torch.cuda.Stream(dev)
+    with torch.cuda.stream(stream):
+        st = torch.cuda.current_stream()
+        for name, fn in calls.items():
+            for _ in range(3):
+                work.copy_(state)
+                fn(st)
+            tot = 0.0
+            for r in range(reps):
+                work.copy_(state)
+                flush.fill_(r & 0xFF)
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(st)
+                fn(st)
+                b.record(st)
+                b.synchronize()
+                tot += a.elapsed_time(b)
+            us = tot * 1e3 / reps
+            gbs = per_row[name] * FIELD_ROWS / (us * 1e-6) / 1e9
+            res[name] = {"us_per_call": round(us, 2), "GB_s": round(gbs, 1),
+                         "frac_of_measured_hbm": round(gbs / hbm, 3),
+                         "bytes_per_call": per_row[name] * FIELD_ROWS}
+    torch.cuda.synchronize()
+    return res
+
+
+def run_field_only(args):
+    """Only the density-field measurement, printed as one JSON object (no decode line)."""
+    import torch
+    from bit_quantized_mamba_b200 import build
+    build.build()
+    dev = torch.device("cuda", 0)
+    hbm, peak_kind = peaks()
+    flush = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    res = measure_state_field(dev, flush, hbm)
+    res["peak"], res["peak_kind"] = hbm, peak_kind
+    print(json.dumps({"state_field": res}), flush=True)
+
+
+def run_field_profile(args):
+    """Eager density-field encodes of the 48-layer state for an ncu capture (no timing is reported)."""
+    import torch
+    from bit_quantized_mamba_b200 import build, dfssm, inputs
+    build.build()
+    dev = torch.device("cuda", 0)
+    state = torch.from_numpy(inputs.ssm_state_rows(seed=77, rows=FIELD_ROWS, d_state=FIELD_N)).to(dev)
+    field = torch.empty((FIELD_ROWS, FIELD_N // 8), dtype=torch.int32, device=dev)
+    scale = torch.empty(FIELD_ROWS, dtype=torch.float32, device=dev)
+    out = torch.empty_like(state)
+    for _ in range(args.warmup + 1):
+        dfssm.state_field_encode(state, field, scale)
+        dfssm.state_field_decode(field, scale, FIELD_N, out)
+    torch.cuda.synchronize()
 
 
 def run_prefill_profile(args):
@@ -703,10 +783,16 @@ def main():
                     help="profiling mode: a 2048-token prompt through one layer --warmup + 1 times and exit")
     ap.add_argument("--ncu-head", action="store_true",
                     help="profiling mode: the final norm + LM head + greedy choice --warmup + 1 times and exit")
+    ap.add_argument("--field-only", action="store_true",
+                    help="time only the density-field encode / readout / round trip and print them")
+    ap.add_argument("--ncu-field", action="store_true",
+                    help="profiling mode: density-field encode + readout of the 48-layer state --warmup + 1 "
+                         "times and exit")
     ap.add_argument("--ncu", action="store_true",
                     help="profiling mode: decode --warmup tokens then one more token, eagerly, and exit")
     args = ap.parse_args()
-    profiling = args.ncu or args.ncu_gemv or args.ncu_prefill or args.ncu_layer_prefill or args.ncu_head
+    profiling = (args.ncu or args.ncu_gemv or args.ncu_prefill or args.ncu_layer_prefill or args.ncu_head
+                 or args.ncu_field)
     if args.warmup < 3 and not profiling:
         args.warmup = 3
     rank = int(os.environ.get("RANK", 0))
@@ -726,6 +812,12 @@ def main():
         return
     if args.ncu_head:
         run_head_profile(args)
+        return
+    if args.ncu_field:
+        run_field_profile(args)
+        return
+    if args.field_only:
+        run_field_only(args)
         return
     if world > 1:
         import datetime

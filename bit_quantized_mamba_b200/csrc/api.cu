@@ -260,6 +260,13 @@ int layer_decode_impl(const dfssm_layer_t* layers, int n_layers, const dfssm_dim
   return e == cudaSuccess ? DFSSM_OK : cuda_fail(e);
 }
 
+// Shared checks of the density-field entry points: DFSSM_OK or the status to return.
+int check_field(int rows, int N) {
+  if (rows < 0 || N < 8 || N % 8) return DFSSM_EINVAL;
+  if (N > 256) return DFSSM_EUNSUPPORTED;
+  return DFSSM_OK;
+}
+
 }  // namespace
 
 // Argument checks of one linear descriptor: d_in a multiple of 32 (above 8192: unsupported), rank 0..16,
@@ -429,6 +436,40 @@ int dfssm_conv_step(float* conv_state, const float* w, const float* b, const flo
   if (!device_ok()) return DFSSM_EDEVICE;
   dfssm::ConvArgs a{conv_state, w, b, x_in, C, x_out, C, B, C};
   cudaError_t e = dfssm::launch_conv(a, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? DFSSM_OK : cuda_fail(e);
+}
+
+int dfssm_state_field_encode(const float* state, int rows, int N, uint32_t* field, float* scale,
+                             void* stream) {
+  const int st = check_field(rows, N);
+  if (st || rows == 0) return st;
+  if (!state || !field || !scale) return DFSSM_EINVAL;
+  if (!aligned(state, 16) || !aligned(field, 4) || !aligned(scale, 4)) return DFSSM_EALIGN;
+  if (!device_ok()) return DFSSM_EDEVICE;
+  cudaError_t e = dfssm::launch_field_encode(state, nullptr, field, scale, rows, N,
+                                             static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? DFSSM_OK : cuda_fail(e);
+}
+
+int dfssm_state_field_decode(const uint32_t* field, const float* scale, int rows, int N, float* state,
+                             void* stream) {
+  const int st = check_field(rows, N);
+  if (st || rows == 0) return st;
+  if (!state || !field || !scale) return DFSSM_EINVAL;
+  if (!aligned(state, 16) || !aligned(field, 4) || !aligned(scale, 4)) return DFSSM_EALIGN;
+  if (!device_ok()) return DFSSM_EDEVICE;
+  cudaError_t e = dfssm::launch_field_decode(field, scale, rows, N, state, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? DFSSM_OK : cuda_fail(e);
+}
+
+int dfssm_state_field_roundtrip(float* state, int rows, int N, uint32_t* field, float* scale, void* stream) {
+  const int st = check_field(rows, N);
+  if (st || rows == 0) return st;
+  if (!state || (field == nullptr) != (scale == nullptr)) return DFSSM_EINVAL;
+  if (!aligned(state, 16) || !aligned(field, 4) || !aligned(scale, 4)) return DFSSM_EALIGN;
+  if (!device_ok()) return DFSSM_EDEVICE;
+  cudaError_t e = dfssm::launch_field_encode(state, state, field, scale, rows, N,
+                                             static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? DFSSM_OK : cuda_fail(e);
 }
 

@@ -150,6 +150,14 @@ struct EmbedArgs {
 };
 cudaError_t launch_embed(const EmbedArgs& a, cudaStream_t st);
 
+// Density-field state representation of state rows [rows][N] (8 <= N <= 256, N % 8 == 0; rows 16-byte
+// aligned): encode to field [rows][N/8] + scale [rows] (either both or neither stored) and/or write the
+// popcount readout to `out` (may equal `in`, or be NULL); decode a field back to rows.
+cudaError_t launch_field_encode(const float* in, float* out, uint32_t* field, float* scale, int rows, int N,
+                                cudaStream_t st);
+cudaError_t launch_field_decode(const uint32_t* field, const float* scale, int rows, int N, float* out,
+                                cudaStream_t st);
+
 // Streaming multiprocessors of the current device.
 int num_sms();
 // Sets the dynamic shared-memory limit of a kernel on the current device, once per (kernel, device): the

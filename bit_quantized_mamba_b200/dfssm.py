@@ -80,6 +80,9 @@ SIGNATURES = {
     "dfssm_embed": (_I, [_P, _P, _I, _I, _P, _P, _P, C.c_size_t, _P]),
     "dfssm_head_greedy": (_I, [_P, _P, _I, _I, _P, _P, _P, _P, _P, _P, _Z, _P]),
     "dfssm_generate": (_I, [_P, _I, _P, _P, _P, _I, _P, _P, _I, _P, _P, _P, _P, _P, _Z, _P]),
+    "dfssm_state_field_encode": (_I, [_P, _I, _I, _P, _P, _P]),
+    "dfssm_state_field_decode": (_I, [_P, _P, _I, _I, _P, _P]),
+    "dfssm_state_field_roundtrip": (_I, [_P, _I, _I, _P, _P, _P]),
     "dfssm_pack_signs": (_I, [_P, _I, _I, _P]),
     "dfssm_device_status": (_I, [_P, _P]),
     "dfssm_selftest_timeout": (_I, [_P, _Z, _P]),
@@ -266,6 +269,43 @@ def ssm_step(ssm_state, x, dt_raw, A_log, dt_bias, D, Bm, Cm, y=None, stream=Non
         _ptr(ssm_state), _ptr(x), _ptr(dt_raw), _ptr(A_log), _ptr(dt_bias), _ptr(D), _ptr(Bm),
         _ptr(Cm), _ptr(y), B, H, P, N, G, _stream(stream)))
     return y
+
+
+def _field_rows(state):
+    N = state.shape[-1]
+    return state.numel() // N if N else 0, N
+
+
+def state_field_encode(state, field=None, scale=None, stream=None):
+    """Density-field encoding of the state rows [..., N] (dfssm_state_field_encode): returns (field int32
+    [rows, N/8] holding the u32 words, scale float32 [rows])."""
+    rows, N = _field_rows(state)
+    if field is None:
+        field = torch.empty((rows, N // 8), dtype=torch.int32, device=state.device)
+    if scale is None:
+        scale = torch.empty(rows, dtype=torch.float32, device=state.device)
+    _check("dfssm_state_field_encode", lib().dfssm_state_field_encode(
+        _ptr(state), rows, N, _ptr(field), _ptr(scale), _stream(stream)))
+    return field, scale
+
+
+def state_field_decode(field, scale, N: int, out=None, stream=None):
+    """Popcount readout of density fields [rows, N/8] (dfssm_state_field_decode) into rows [rows, N]."""
+    rows = scale.numel()
+    if out is None:
+        out = torch.empty((rows, N), dtype=torch.float32, device=scale.device)
+    _check("dfssm_state_field_decode", lib().dfssm_state_field_decode(
+        _ptr(field), _ptr(scale), rows, N, _ptr(out), _stream(stream)))
+    return out
+
+
+def state_field_roundtrip(state, field=None, scale=None, stream=None):
+    """state <- readout(encode(state)) in place (dfssm_state_field_roundtrip); field and scale, when
+    given, receive the encoding too."""
+    rows, N = _field_rows(state)
+    _check("dfssm_state_field_roundtrip", lib().dfssm_state_field_roundtrip(
+        _ptr(state), rows, N, _ptr(field), _ptr(scale), _stream(stream)))
+    return state
 
 
 class Layer:

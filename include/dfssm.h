@@ -43,7 +43,7 @@
 extern "C" {
 #endif
 
-#define DFSSM_ABI_VERSION 4
+#define DFSSM_ABI_VERSION 5
 #define DFSSM_MAX_RANK 16
 #define DFSSM_MAX_BATCH 16
 #define DFSSM_MAX_LAYERS 64
@@ -190,6 +190,32 @@ int dfssm_conv_step(float* conv_state, const float* w, const float* b, const flo
 int dfssm_ssm_step(float* ssm_state, const float* x, const float* dt_raw, const float* A_log,
                    const float* dt_bias, const float* D, const float* Bm, const float* Cm, float* y,
                    int B, int H, int P, int N, int G, void* stream);
+
+/*
+ * Density-field state representation (technical summary §2.D "Density Field State Representation": the
+ * SSM hidden state kept as a binary field per state element, K^2 about 4 d_state cells, built by
+ * normalization, sigma-delta injection with error feedback and binarization, read back by popcount, at
+ * chunk boundaries).  One state row S[0..N) (N = d_state; an SSM state [B][H][P][N] is B*H*P rows) is
+ * 4N cells, four per value, plus c = max |S|:
+ *   x_n = fl32(S_n / c) (0 when c = 0), d_n = fl32(x_n + 1) / 2;
+ *   cells j = 4n + k, in order, fed d_n through v = d + e, b_j = [v >= 1/2], e = v - b_j (e = 0 at the row
+ *   start; exact arithmetic: every d_n is a multiple of 2^-25);
+ *   readout S^_n = fl32(c (popcount(cells of n) / 2 - 1)), one of {-c, -c/2, 0, c/2, c}.
+ *   state device f32 [rows][N] (16-byte aligned), finite values;
+ *   field device u32 [rows][N/8]: cell j is bit j % 32 of word j / 32 (value n is nibble n % 8 of word n / 8);
+ *   scale device f32 [rows]: c.
+ * Requires 8 <= N, N % 8 == 0 (else DFSSM_EINVAL), N <= 256 (else DFSSM_EUNSUPPORTED), rows >= 0; with
+ * rows == 0 nothing is read or launched (the pointers may be NULL), otherwise NULL pointers give
+ * DFSSM_EINVAL.  The library applies no schedule: the caller calls these at its chunk boundaries.
+ */
+int dfssm_state_field_encode(const float* state, int rows, int N, uint32_t* field, float* scale,
+                             void* stream);
+/* The popcount readout of a field into state rows (state written, field and scale read). */
+int dfssm_state_field_decode(const uint32_t* field, const float* scale, int rows, int N, float* state,
+                             void* stream);
+/* Encode and read back in place in one pass: state <- readout(encode(state)); field and scale are
+ * stored too when both are non-NULL (both NULL: not stored; one NULL: DFSSM_EINVAL). */
+int dfssm_state_field_roundtrip(float* state, int rows, int N, uint32_t* field, float* scale, void* stream);
 
 /* Shape of a DF-SSM Mamba-2 layer.  d_inner = nheads*headdim; conv channels = d_inner + 2*ngroups*d_state;
  * in_proj rows = 2*d_inner + 2*ngroups*d_state + nheads, ordered z | x | B | C | dt. */

@@ -37,7 +37,7 @@ def test_library_exports_every_declared_symbol(L):
     for n in names:
         assert hasattr(L, n), f"{n} declared in dfssm.h but not exported"
     assert set(names) == set(dfssm.SIGNATURES), "binding and header disagree"
-    assert L.dfssm_abi_version() == 4
+    assert L.dfssm_abi_version() == 5
 
 
 def test_cpu_engine_exports_every_declared_symbol():
@@ -113,6 +113,31 @@ def test_argument_validation_precedes_device_use(L):
                             256, 1024, None) == -7                                    # workspace
     assert L.dfssm_generate(None, 48, C.byref(dims), 16, 16, 10, 16, 16, 4, None, None, None, None,
                             256, 1 << 30, None) == -1                                 # no layers
+
+
+def test_state_field_validation_precedes_device_use(L):
+    """The density-field calls reject bad sizes, pointers and alignment on the host."""
+    for enc in (lambda st, r, n, f, s: L.dfssm_state_field_encode(st, r, n, f, s, None),
+                lambda st, r, n, f, s: L.dfssm_state_field_decode(f, s, r, n, st, None)):
+        assert enc(None, 4, 128, 256, 256) == -1      # no state
+        assert enc(256, 4, 128, None, 256) == -1      # no field
+        assert enc(256, 4, 128, 256, None) == -1      # no scale
+        assert enc(256, -1, 128, 256, 256) == -1      # rows < 0
+        assert enc(256, 4, 12, 256, 256) == -1        # N % 8
+        assert enc(256, 4, 0, 256, 256) == -1         # N < 8
+        assert enc(256, 4, 264, 256, 256) == -3       # N > 256
+        assert enc(8, 4, 128, 256, 256) == -2         # state not 16-byte aligned
+        assert enc(256, 4, 128, 2, 256) == -2         # field misaligned
+    assert L.dfssm_state_field_roundtrip(256, 4, 128, 256, None, None) == -1  # field without scale
+    assert L.dfssm_state_field_roundtrip(256, 4, 128, None, 256, None) == -1  # scale without field
+    assert L.dfssm_state_field_roundtrip(None, 4, 128, None, None, None) == -1
+    assert L.dfssm_state_field_roundtrip(8, 4, 128, None, None, None) == -2
+    assert L.dfssm_state_field_roundtrip(256, 4, 304, None, None, None) == -3
+    # no rows: nothing to read, NULL pointers accepted, no device touched
+    assert L.dfssm_state_field_encode(None, 0, 128, None, None, None) == 0
+    assert L.dfssm_state_field_decode(None, None, 0, 128, None, None) == 0
+    assert L.dfssm_state_field_roundtrip(None, 0, 128, None, None, None) == 0
+    assert L.dfssm_state_field_encode(None, 0, 12, None, None, None) == -1
 
 
 def _linears(dfssm, *descs):
