@@ -95,11 +95,13 @@ __device__ __forceinline__ float encode_row(const float (&s)[V], int N, int lane
   const float c = __uint_as_float(__reduce_max_sync(kFull, __float_as_uint(m)));
   uint32_t D[V];
   uint32_t own = 0;
+  const bool whole = V % 4 == 0 && lane * V < N;  // with V % 4 == 0 a lane's range is whole or empty
 #pragma unroll
   for (int i = 0; i < V; ++i) {
     const float x = c > 0.0f ? __fdiv_rn(s[i], c) : 0.0f;
     const float d = __fmul_rn(__fadd_rn(x, 1.0f), 0.5f);
-    D[i] = lane * V + i < N ? __float2uint_rn(__fmul_rn(d, kUnits)) : 0u;  // exact: d 2^25 <= 2^25
+    const bool in = V % 4 == 0 ? whole : lane * V + i < N;
+    D[i] = in ? __float2uint_rn(__fmul_rn(d, kUnits)) : 0u;  // exact: d 2^25 <= 2^25
     own += D[i];
   }
   uint32_t inc = own;  // inclusive scan over the lanes, modulo 2^32
@@ -111,10 +113,11 @@ __device__ __forceinline__ float encode_row(const float (&s)[V], int N, int lane
   uint32_t q = inc - own;  // Q of the lane's first value, modulo 2^32
 #pragma unroll
   for (int i = 0; i < V; ++i) {
-    const uint32_t lo = (4u * q + kHalfUnit) & kUnitMask;
-    const uint32_t t1 = (lo + D[i]) >> 25, t2 = (lo + 2u * D[i]) >> 25;
-    const uint32_t t3 = (lo + 3u * D[i]) >> 25, t4 = (lo + 4u * D[i]) >> 25;  // lo + 4 D < 2^28
-    nib[i] = t1 | ((t2 - t1) << 1) | ((t3 - t2) << 2) | ((t4 - t3) << 3);
+    const uint32_t a1 = ((4u * q + kHalfUnit) & kUnitMask) + D[i];
+    const uint32_t a2 = a1 + D[i], a3 = a2 + D[i], a4 = a3 + D[i];  // below 2^28
+    const uint32_t t1 = a1 >> 25, t2 = a2 >> 25, t3 = a3 >> 25, t4 = a4 >> 25;
+    // bit k is t_{k+1} - t_k (0 or 1), so the nibble is sum_k 2^k (t_{k+1} - t_k) = 8 t4 - 4 t3 - 2 t2 - t1
+    nib[i] = 8u * t4 - 4u * t3 - 2u * t2 - t1;
     pop[i] = (int)t4;
     q += D[i];
   }
@@ -155,17 +158,28 @@ __global__ void __launch_bounds__(kWarps * 32) field_encode_kernel(const float* 
       int pop[V];
       const float c = encode_row<V>(s[j], N, lane, nib, pop);
       if constexpr (kField) {
+        if constexpr (V == 8) {  // the lane's eight values are word `lane`
+          uint32_t wd = 0;
 #pragma unroll
-        for (int i = 0; i < V; ++i)
-          if (lane * V + i < N) nbuf[warp][lane * V + i] = (uint8_t)nib[i];
-        __syncwarp();
-        if (lane < W) {
-          const uint32_t lo = *reinterpret_cast<const uint32_t*>(&nbuf[warp][8 * lane]);
-          const uint32_t hi = *reinterpret_cast<const uint32_t*>(&nbuf[warp][8 * lane + 4]);
-          __stcs(field + r * W + lane, pack4(lo) | (pack4(hi) << 16));
+          for (int i = 0; i < 8; ++i) wd |= nib[i] << (4 * i);
+          if (lane < W) __stcs(field + r * W + lane, wd);
+        } else if constexpr (V == 4) {  // lanes 2t and 2t + 1 hold the two halves of word t
+          const uint32_t half = nib[0] | (nib[1] << 4) | (nib[2] << 8) | (nib[3] << 12);
+          const uint32_t up = __shfl_down_sync(kFull, half, 1);
+          if ((lane & 1) == 0 && (lane >> 1) < W) __stcs(field + r * W + (lane >> 1), half | (up << 16));
+        } else {
+#pragma unroll
+          for (int i = 0; i < V; ++i)
+            if (lane * V + i < N) nbuf[warp][lane * V + i] = (uint8_t)nib[i];
+          __syncwarp();
+          if (lane < W) {
+            const uint32_t lo = *reinterpret_cast<const uint32_t*>(&nbuf[warp][8 * lane]);
+            const uint32_t hi = *reinterpret_cast<const uint32_t*>(&nbuf[warp][8 * lane + 4]);
+            __stcs(field + r * W + lane, pack4(lo) | (pack4(hi) << 16));
+          }
+          __syncwarp();  // nbuf is rewritten for the next row
         }
         if (lane == 0) scale[r] = c;
-        __syncwarp();  // nbuf is rewritten for the next row
       }
       if constexpr (kReadout) {
         float y[V];
