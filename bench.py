@@ -581,6 +581,7 @@ def run_ours(args, rank, world, local_rank):
         vnni = vnni_engine_rate(cores)
         if vnni is not None:
             line["cpu_baseline"]["vnni_engine"] = vnni
+        line["cpu_baseline"]["state_field_encode"] = field_cpu_times(cores)
     if rank == 0:
         print(json.dumps(line), flush=True)
     graph = None
@@ -659,6 +660,32 @@ def measure_state_field(dev, flush, hbm, reps=10):
                          "frac_of_measured_hbm": round(gbs / hbm, 3),
                          "bytes_per_call": per_row[name] * FIELD_ROWS}
     torch.cuda.synchronize()
+    return res
+
+
+def field_cpu_times(cores):
+    """The density-field encode of the same 48-layer state on the host: the oracle (cell-by-cell
+    sigma-delta loop) and the host-CPU engine, best of three, all cores."""
+    import oracle
+    import torch
+    from bit_quantized_mamba_b200 import build, dfssm, inputs
+    S = inputs.ssm_state_rows(seed=77, rows=FIELD_ROWS, d_state=FIELD_N)
+
+    def best(fn):
+        ts = []
+        for _ in range(3):
+            t0 = time.perf_counter()
+            fn()
+            ts.append(time.perf_counter() - t0)
+        return round(min(ts) * 1e6, 1)
+
+    res = {"rows": FIELD_ROWS, "d_state": FIELD_N, "cores": cores,
+           "oracle_us_per_call": best(lambda: oracle.field_encode(S))}
+    build.build_cpu()
+    if dfssm.cpu_available():
+        dfssm.cpu_set_threads(cores)
+        St = torch.from_numpy(S)
+        res["cpu_engine_us_per_call"] = best(lambda: dfssm.cpu_state_field_encode(St))
     return res
 
 

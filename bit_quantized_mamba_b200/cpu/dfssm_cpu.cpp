@@ -360,6 +360,46 @@ void ssm_step(float* S_all, const float* x, const float* dt_raw, const float* A_
   }
 }
 
+// ------------------------------------------------------------------------------------ density field
+
+// One state row of the density-field representation (libdfssm's dfssm_state_field_encode): c = max |S|,
+// densities as integers D_n = fl32(fl32(S_n / c) + 1) 2^24 (exact: multiples of 2^-25 times 2^25), and
+// the four cells of value n the carries of lo + k D_n past 2^25, k = 1..4, lo = (4 Q_n + 2^24) mod 2^25
+// with Q_n the prefix sum of D (only Q mod 2^23 enters, so wrapping 32-bit arithmetic is exact).  The
+// divisions and conversions of a row are vectorised; the prefix sum runs in index order.  field and
+// readout may each be NULL.
+__attribute__((target("avx512f"))) void field_row(const float* S, int N, uint32_t* field, float* scale,
+                                                  float* readout) {
+  alignas(64) uint32_t D[256];
+  float c = 0.0f;
+  for (int n = 0; n < N; ++n) c = std::max(c, std::fabs(S[n]));
+  const __m512 vc = _mm512_set1_ps(c), one = _mm512_set1_ps(1.0f), k24 = _mm512_set1_ps(16777216.0f);
+  for (int n = 0; n < N; n += 16) {
+    const __mmask16 m = N - n >= 16 ? (__mmask16)0xFFFF : (__mmask16)((1u << (N - n)) - 1u);
+    const __m512 x = c > 0.0f ? _mm512_div_ps(_mm512_maskz_loadu_ps(m, S + n), vc) : _mm512_setzero_ps();
+    // fl32(x + 1) 2^24: the sum rounds once, the product by 2^24 is exact, the conversion is exact
+    const __m512i d = _mm512_cvtps_epu32(_mm512_mul_ps(_mm512_add_ps(x, one), k24));
+    _mm512_mask_storeu_epi32(D + n, m, d);
+  }
+  uint32_t q = 0;
+  for (int w = 0; w < N / 8; ++w) {
+    uint32_t word = 0;
+    for (int i = 0; i < 8; ++i) {
+      const int n = 8 * w + i;
+      const uint32_t a1 = ((4u * q + (1u << 24)) & ((1u << 25) - 1u)) + D[n];
+      const uint32_t a2 = a1 + D[n], a3 = a2 + D[n], a4 = a3 + D[n];
+      const uint32_t t1 = a1 >> 25, t2 = a2 >> 25, t3 = a3 >> 25, t4 = a4 >> 25;
+      word |= (8u * t4 - 4u * t3 - 2u * t2 - t1) << (4 * i);
+      if (readout) readout[n] = c * ((float)t4 * 0.5f - 1.0f);
+      q += D[n];
+    }
+    if (field) field[w] = word;
+  }
+  if (scale) *scale = c;
+}
+
+bool field_args_ok(int rows, int N) { return rows >= 0 && N >= 8 && N % 8 == 0; }
+
 }  // namespace
 
 extern "C" {
@@ -391,6 +431,51 @@ int dfssm_cpu_linear_decode(const dfssm_linear_t* lin, const float* x, int B, fl
   if (dbg && dbg->xq) std::memcpy(dbg->xq, q.data(), q.size());
   linear(*lin, q.data(), s.data(), sq.data(), B, y, nullptr, dbg ? dbg->acc : nullptr,
          dbg ? dbg->lora_t : nullptr);
+  return DFSSM_OK;
+}
+
+int dfssm_cpu_state_field_encode(const float* state, int rows, int N, uint32_t* field, float* scale) {
+  if (!field_args_ok(rows, N)) return DFSSM_EINVAL;
+  if (N > 256) return DFSSM_EUNSUPPORTED;
+  if (rows == 0) return DFSSM_OK;
+  if (!state || !field || !scale) return DFSSM_EINVAL;
+  if (!has_vnni()) return DFSSM_EUNSUPPORTED;
+#pragma omp parallel for schedule(static)
+  for (int r = 0; r < rows; ++r)
+    field_row(state + (size_t)r * N, N, field + (size_t)r * (N / 8), scale + r, nullptr);
+  return DFSSM_OK;
+}
+
+int dfssm_cpu_state_field_decode(const uint32_t* field, const float* scale, int rows, int N, float* state) {
+  if (!field_args_ok(rows, N)) return DFSSM_EINVAL;
+  if (N > 256) return DFSSM_EUNSUPPORTED;
+  if (rows == 0) return DFSSM_OK;
+  if (!state || !field || !scale) return DFSSM_EINVAL;
+#pragma omp parallel for schedule(static)
+  for (int r = 0; r < rows; ++r) {
+    const uint32_t* F = field + (size_t)r * (N / 8);
+    const float c = scale[r];
+    for (int n = 0; n < N; ++n) {
+      const int p = __builtin_popcount((F[n / 8] >> (4 * (n % 8))) & 0xFu);
+      state[(size_t)r * N + n] = c * ((float)p * 0.5f - 1.0f);
+    }
+  }
+  return DFSSM_OK;
+}
+
+int dfssm_cpu_state_field_roundtrip(float* state, int rows, int N, uint32_t* field, float* scale) {
+  if (!field_args_ok(rows, N)) return DFSSM_EINVAL;
+  if (N > 256) return DFSSM_EUNSUPPORTED;
+  if (rows == 0) return DFSSM_OK;
+  if (!state || (field == nullptr) != (scale == nullptr)) return DFSSM_EINVAL;
+  if (!has_vnni()) return DFSSM_EUNSUPPORTED;
+#pragma omp parallel for schedule(static)
+  for (int r = 0; r < rows; ++r) {
+    float* S = state + (size_t)r * N;
+    alignas(64) float tmp[256];
+    field_row(S, N, field ? field + (size_t)r * (N / 8) : nullptr, scale ? scale + r : nullptr, tmp);
+    std::memcpy(S, tmp, (size_t)N * 4);
+  }
   return DFSSM_OK;
 }
 

@@ -478,6 +478,9 @@ def cpu_lib():
         L.dfssm_cpu_layer_decode.restype = C.c_int
         L.dfssm_cpu_layer_decode.argtypes = [C.POINTER(LayerT), C.c_int, C.POINTER(DimsT), C.c_void_p,
                                              C.POINTER(C.c_void_p), C.POINTER(C.c_void_p), C.c_int]
+        L.dfssm_cpu_state_field_encode.argtypes = [C.c_void_p, C.c_int, C.c_int, C.c_void_p, C.c_void_p]
+        L.dfssm_cpu_state_field_decode.argtypes = [C.c_void_p, C.c_void_p, C.c_int, C.c_int, C.c_void_p]
+        L.dfssm_cpu_state_field_roundtrip.argtypes = [C.c_void_p, C.c_int, C.c_int, C.c_void_p, C.c_void_p]
         _cpu_lib = L
     return _cpu_lib
 
@@ -511,3 +514,34 @@ def cpu_layer_decode(stack: LayerStack, hidden: torch.Tensor) -> torch.Tensor:
         *stack.c(host=True)[:1], stack.n, C.byref(stack.dims), _hptr(hidden), *stack.c(host=True)[1:],
         hidden.shape[0]))
     return hidden
+
+
+def cpu_state_field_encode(state: torch.Tensor, field=None, scale=None):
+    """dfssm_cpu_state_field_encode on host rows [..., N]: returns (field int32 [rows, N/8] holding the u32
+    words, scale float32 [rows])."""
+    rows, N = _field_rows(state)
+    if field is None:
+        field = torch.empty((rows, N // 8), dtype=torch.int32)
+    if scale is None:
+        scale = torch.empty(rows, dtype=torch.float32)
+    _check("dfssm_cpu_state_field_encode", cpu_lib().dfssm_cpu_state_field_encode(
+        _hptr(state), rows, N, _hptr(field), _hptr(scale)))
+    return field, scale
+
+
+def cpu_state_field_decode(field: torch.Tensor, scale: torch.Tensor, N: int, out=None):
+    """dfssm_cpu_state_field_decode: the popcount readout of host fields into rows [rows, N]."""
+    rows = scale.numel()
+    if out is None:
+        out = torch.empty((rows, N), dtype=torch.float32)
+    _check("dfssm_cpu_state_field_decode", cpu_lib().dfssm_cpu_state_field_decode(
+        _hptr(field), _hptr(scale), rows, N, _hptr(out)))
+    return out
+
+
+def cpu_state_field_roundtrip(state: torch.Tensor, field=None, scale=None):
+    """dfssm_cpu_state_field_roundtrip: host rows replaced in place by the readout of their encoding."""
+    rows, N = _field_rows(state)
+    _check("dfssm_cpu_state_field_roundtrip", cpu_lib().dfssm_cpu_state_field_roundtrip(
+        _hptr(state), rows, N, _hptr(field), _hptr(scale)))
+    return state

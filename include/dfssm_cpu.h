@@ -28,7 +28,7 @@
 extern "C" {
 #endif
 
-#define DFSSM_CPU_ABI_VERSION 1
+#define DFSSM_CPU_ABI_VERSION 2
 
 int dfssm_cpu_abi_version(void);
 
@@ -54,6 +54,17 @@ int dfssm_cpu_linear_decode(const dfssm_linear_t* lin, const float* x, int B, fl
  */
 int dfssm_cpu_layer_decode(const dfssm_layer_t* layers, int n_layers, const dfssm_dims_t* dims,
                            float* hidden, float* const* conv_states, float* const* ssm_states, int B);
+
+/*
+ * Density-field state representation (dfssm_state_field_encode / _decode / _roundtrip's definition,
+ * technical summary §2.D "Density Field State Representation"), on host rows [rows][N]:
+ *   state host f32 [rows][N], field host u32 [rows][N/8], scale host f32 [rows];
+ *   8 <= N, N % 8 == 0 (else DFSSM_EINVAL), N <= 256 (else DFSSM_EUNSUPPORTED); rows == 0 does nothing.
+ * The readout needs no AVX-512; encode and round trip return DFSSM_EUNSUPPORTED without it.
+ */
+int dfssm_cpu_state_field_encode(const float* state, int rows, int N, uint32_t* field, float* scale);
+int dfssm_cpu_state_field_decode(const uint32_t* field, const float* scale, int rows, int N, float* state);
+int dfssm_cpu_state_field_roundtrip(float* state, int rows, int N, uint32_t* field, float* scale);
 
 #ifdef __cplusplus
 }

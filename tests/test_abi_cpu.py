@@ -51,10 +51,15 @@ def test_cpu_engine_exports_every_declared_symbol():
     Lc = dfssm.cpu_lib()
     for n in names:
         assert hasattr(Lc, n), f"{n} declared in dfssm_cpu.h but not exported"
-    assert Lc.dfssm_cpu_abi_version() == 1
+    assert Lc.dfssm_cpu_abi_version() == 2
     assert Lc.dfssm_cpu_available() in (0, 1)
     assert Lc.dfssm_cpu_linear_decode(None, None, 1, None, None) == -1
     assert Lc.dfssm_cpu_layer_decode(None, 0, None, None, None, None, 1) == -1
+    assert Lc.dfssm_cpu_state_field_encode(None, 4, 12, None, None) == -1      # N % 8
+    assert Lc.dfssm_cpu_state_field_encode(None, 4, 264, None, None) == -3     # N > 256
+    assert Lc.dfssm_cpu_state_field_encode(None, 4, 128, None, None) == -1     # NULL rows
+    assert Lc.dfssm_cpu_state_field_decode(None, None, 0, 128, None) == 0      # no rows
+    assert Lc.dfssm_cpu_state_field_roundtrip(None, -1, 128, None, None) == -1
 
 
 def test_status_strings(L):

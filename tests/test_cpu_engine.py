@@ -112,3 +112,43 @@ def test_rejects_bad_arguments(engine):
     dev_like = _host_linear(inputs.linear(gen, 64, 64, 4))
     with pytest.raises(ValueError):
         dfssm.linear_decode(dev_like, x[:1, :64])  # a host linear on the CUDA entry point
+
+
+@pytest.mark.parametrize("N,rows", [(8, 65), (24, 130), (72, 33), (128, 4097), (200, 70), (256, 129)])
+def test_state_field_matches_oracle(engine, N, rows):
+    """Density-field encode, readout and round trip bit-identical to the oracle's sigma-delta loop."""
+    S = inputs.ssm_state_rows(seed=500 + N, rows=rows, d_state=N)
+    f_ref, s_ref = oracle.field_encode(S)
+    back_ref = oracle.field_decode(f_ref, s_ref, N)
+    field, scale = engine.cpu_state_field_encode(torch.from_numpy(S))
+    assert np.array_equal(field.numpy().view(np.uint32), f_ref)
+    assert np.array_equal(scale.numpy(), s_ref)
+    assert np.array_equal(engine.cpu_state_field_decode(field, scale, N).numpy(), back_ref)
+    st = torch.from_numpy(S.copy())
+    f2, s2 = torch.zeros_like(field), torch.zeros_like(scale)
+    engine.cpu_state_field_roundtrip(st, f2, s2)
+    assert np.array_equal(st.numpy(), back_ref)
+    assert np.array_equal(f2.numpy().view(np.uint32), f_ref) and np.array_equal(s2.numpy(), s_ref)
+    st = torch.from_numpy(S.copy())
+    engine.cpu_state_field_roundtrip(st)
+    assert np.array_equal(st.numpy(), back_ref)
+
+
+def test_state_field_edge_rows(engine):
+    g = np.random.default_rng(6)
+    N = 128
+    rows = [np.zeros(N, np.float32),
+            ((g.integers(0, 5, N) * 0.5 - 1) * 3.0).astype(np.float32),
+            (g.standard_normal(N) * 1e37).astype(np.float32),
+            (g.standard_normal(N) * 1e-38).astype(np.float32),
+            np.full(N, -2.5, np.float32)]
+    den = (g.standard_normal(N) * 1e-10).astype(np.float32)
+    den[0] = 1e30
+    rows.append(den)
+    S = np.stack(rows)
+    f_ref, s_ref = oracle.field_encode(S)
+    field, scale = engine.cpu_state_field_encode(torch.from_numpy(S))
+    assert np.array_equal(field.numpy().view(np.uint32), f_ref)
+    assert np.array_equal(scale.numpy(), s_ref)
+    assert np.array_equal(engine.cpu_state_field_decode(field, scale, N).numpy(),
+                          oracle.field_decode(f_ref, s_ref, N))
