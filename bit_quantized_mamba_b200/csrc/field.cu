@@ -14,9 +14,10 @@
 // densities as integers D_n = d_n 2^25 and Q_n = D_0 + ... + D_{n-1}, the ones among the first k cells of
 // value n number floor((4 Q_n + k D_n + 2^24) / 2^25) - floor((4 Q_n + 2^24) / 2^25) = (lo + k D_n) >> 25
 // with lo = (4 Q_n + 2^24) mod 2^25.  Only Q_n mod 2^23 enters lo, so the prefix sums run in wrapping
-// 32-bit integers, exactly.  A warp takes a row: each lane its ceil(N / 32) consecutive values, one warp
-// scan for the Q of its first value; no serial chain.  HBM-bound: the state row is read once (and, for
-// the round trip, written once), the field and scale written once.
+// 32-bit integers, exactly.  A row goes to LPR lanes (16 for N <= 128, two rows per warp; else 32): each
+// lane its ceil(N / LPR) consecutive values, one scan over the row's lanes for the Q of its first value;
+// no serial chain.  The state row is read once (and, for the round trip, written once), the field and
+// scale written once.
 
 #include <cstdint>
 #include <cuda_runtime.h>
@@ -83,32 +84,40 @@ __device__ __forceinline__ float readout(float c, int p) {
   return __fmul_rn(c, __fadd_rn(__fmul_rn((float)p, 0.5f), -1.0f));
 }
 
-// Normalization and injection of one row held by a warp: returns c (every lane), the nibble of each of
-// the lane's values (cell k of the value in bit k) and its popcount.
-template <int V>
-__device__ __forceinline__ float encode_row(const float (&s)[V], int N, int lane, uint32_t (&nib)[V],
+// Normalization and injection of one row held by LPR lanes (a whole warp, or one half): returns c (every
+// lane of the row), the nibble of each of the lane's values (cell k of the value in bit k) and its
+// popcount.  li = the lane's index within the row.
+template <int V, int LPR>
+__device__ __forceinline__ float encode_row(const float (&s)[V], int N, int li, uint32_t (&nib)[V],
                                             int (&pop)[V]) {
   float m = 0.0f;
 #pragma unroll
   for (int i = 0; i < V; ++i) m = fmaxf(m, fabsf(s[i]));
   // non-negative floats order like their bit patterns
-  const float c = __uint_as_float(__reduce_max_sync(kFull, __float_as_uint(m)));
+  uint32_t mb = __float_as_uint(m);
+  if constexpr (LPR == 32) {
+    mb = __reduce_max_sync(kFull, mb);
+  } else {
+#pragma unroll
+    for (int o = LPR / 2; o > 0; o >>= 1) mb = max(mb, __shfl_xor_sync(kFull, mb, o));
+  }
+  const float c = __uint_as_float(mb);
   uint32_t D[V];
   uint32_t own = 0;
-  const bool whole = V % 4 == 0 && lane * V < N;  // with V % 4 == 0 a lane's range is whole or empty
+  const bool whole = V % 4 == 0 && li * V < N;  // with V % 4 == 0 a lane's range is whole or empty
 #pragma unroll
   for (int i = 0; i < V; ++i) {
     const float x = c > 0.0f ? __fdiv_rn(s[i], c) : 0.0f;
     const float d = __fmul_rn(__fadd_rn(x, 1.0f), 0.5f);
-    const bool in = V % 4 == 0 ? whole : lane * V + i < N;
+    const bool in = V % 4 == 0 ? whole : li * V + i < N;
     D[i] = in ? __float2uint_rn(__fmul_rn(d, kUnits)) : 0u;  // exact: d 2^25 <= 2^25
     own += D[i];
   }
-  uint32_t inc = own;  // inclusive scan over the lanes, modulo 2^32
+  uint32_t inc = own;  // inclusive scan over the row's lanes, modulo 2^32
 #pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const uint32_t t = __shfl_up_sync(kFull, inc, o);
-    if (lane >= o) inc += t;
+  for (int o = 1; o < LPR; o <<= 1) {
+    const uint32_t t = __shfl_up_sync(kFull, inc, o, LPR);
+    if (li >= o) inc += t;
   }
   uint32_t q = inc - own;  // Q of the lane's first value, modulo 2^32
 #pragma unroll
@@ -130,21 +139,27 @@ __device__ __forceinline__ uint32_t pack4(uint32_t b) {
 }
 
 // Encode rows of `in`; kField: store the field and scale; kReadout: store the readout to `out` (which
-// may be `in`: every row is read before it is written, by the same warp).
-template <int V, bool kField, bool kReadout>
+// may be `in`: every row is read before it is written, by the same lanes).  LPR lanes per row, so a
+// warp holds 32 / LPR rows side by side and R such groups at once.
+template <int V, int LPR, bool kField, bool kReadout>
 __global__ void __launch_bounds__(kWarps * 32) field_encode_kernel(const float* in, float* out, int rows,
                                                                    int N, uint32_t* field, float* scale) {
+  constexpr int RPW = 32 / LPR;
   constexpr int R = rows_per_warp<V>();
   __shared__ __align__(16) uint8_t nbuf[kWarps][256];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int li = lane & (LPR - 1), sub = lane / LPR;  // lane within the row; which of the warp's rows
+  uint8_t* const nb = &nbuf[warp][sub * (256 / RPW)];  // N <= 256 / RPW bytes of this row
   const int W = N / 8;
-  const long long step = (long long)gridDim.x * kWarps * R;
-  for (long long r0 = ((long long)blockIdx.x * kWarps + warp) * R; r0 < rows; r0 += step) {
+  const long long per_warp = (long long)R * RPW;
+  const long long step = (long long)gridDim.x * kWarps * per_warp;
+  for (long long r0 = ((long long)blockIdx.x * kWarps + warp) * per_warp; r0 < rows; r0 += step) {
     float s[R][V];
 #pragma unroll
     for (int j = 0; j < R; ++j) {
-      if (r0 + j < rows) {
-        load_vals<V>(in + (r0 + j) * N, N, lane, s[j]);
+      const long long r = r0 + (long long)j * RPW + sub;
+      if (r < rows) {
+        load_vals<V>(in + r * N, N, li, s[j]);
       } else {
 #pragma unroll
         for (int i = 0; i < V; ++i) s[j][i] = 0.0f;
@@ -152,40 +167,42 @@ __global__ void __launch_bounds__(kWarps * 32) field_encode_kernel(const float* 
     }
 #pragma unroll
     for (int j = 0; j < R; ++j) {
-      const long long r = r0 + j;
-      if (r >= rows) break;  // the same for the whole warp
+      const long long rb = r0 + (long long)j * RPW;
+      if (rb >= rows) break;  // the same for the whole warp
+      const long long r = rb + sub;
+      const bool valid = r < rows;  // the second row of a pair may lie past the end
       uint32_t nib[V];
       int pop[V];
-      const float c = encode_row<V>(s[j], N, lane, nib, pop);
+      const float c = encode_row<V, LPR>(s[j], N, li, nib, pop);
       if constexpr (kField) {
-        if constexpr (V == 8) {  // the lane's eight values are word `lane`
+        if constexpr (V == 8) {  // the lane's eight values are word li
           uint32_t wd = 0;
 #pragma unroll
           for (int i = 0; i < 8; ++i) wd |= nib[i] << (4 * i);
-          if (lane < W) __stcs(field + r * W + lane, wd);
-        } else if constexpr (V == 4) {  // lanes 2t and 2t + 1 hold the two halves of word t
+          if (valid && li < W) __stcs(field + r * W + li, wd);
+        } else if constexpr (V == 4) {  // lanes 2t and 2t + 1 of a row hold the two halves of word t
           const uint32_t half = nib[0] | (nib[1] << 4) | (nib[2] << 8) | (nib[3] << 12);
           const uint32_t up = __shfl_down_sync(kFull, half, 1);
-          if ((lane & 1) == 0 && (lane >> 1) < W) __stcs(field + r * W + (lane >> 1), half | (up << 16));
+          if (valid && (li & 1) == 0 && (li >> 1) < W) __stcs(field + r * W + (li >> 1), half | (up << 16));
         } else {
 #pragma unroll
           for (int i = 0; i < V; ++i)
-            if (lane * V + i < N) nbuf[warp][lane * V + i] = (uint8_t)nib[i];
+            if (li * V + i < N) nb[li * V + i] = (uint8_t)nib[i];
           __syncwarp();
-          if (lane < W) {
-            const uint32_t lo = *reinterpret_cast<const uint32_t*>(&nbuf[warp][8 * lane]);
-            const uint32_t hi = *reinterpret_cast<const uint32_t*>(&nbuf[warp][8 * lane + 4]);
-            __stcs(field + r * W + lane, pack4(lo) | (pack4(hi) << 16));
+          if (valid && li < W) {
+            const uint32_t lo = *reinterpret_cast<const uint32_t*>(nb + 8 * li);
+            const uint32_t hi = *reinterpret_cast<const uint32_t*>(nb + 8 * li + 4);
+            __stcs(field + r * W + li, pack4(lo) | (pack4(hi) << 16));
           }
           __syncwarp();  // nbuf is rewritten for the next row
         }
-        if (lane == 0) scale[r] = c;
+        if (valid && li == 0) scale[r] = c;
       }
       if constexpr (kReadout) {
-        float y[V];
+        float yv[V];
 #pragma unroll
-        for (int i = 0; i < V; ++i) y[i] = readout(c, pop[i]);
-        store_vals<V>(out + r * N, N, lane, y);
+        for (int i = 0; i < V; ++i) yv[i] = readout(c, pop[i]);
+        if (valid) store_vals<V>(out + r * N, N, li, yv);
       }
     }
   }
@@ -229,16 +246,16 @@ int grid_for(int rows, int rows_per_cta) {
   return (int)(need < cap ? need : cap);
 }
 
-template <int V>
+template <int V, int LPR>
 cudaError_t encode_v(const float* in, float* out, uint32_t* field, float* scale, int rows, int N,
                      cudaStream_t st) {
-  const int grid = grid_for(rows, kWarps * rows_per_warp<V>());
+  const int grid = grid_for(rows, kWarps * rows_per_warp<V>() * (32 / LPR));
   if (field && out)
-    field_encode_kernel<V, true, true><<<grid, kWarps * 32, 0, st>>>(in, out, rows, N, field, scale);
+    field_encode_kernel<V, LPR, true, true><<<grid, kWarps * 32, 0, st>>>(in, out, rows, N, field, scale);
   else if (field)
-    field_encode_kernel<V, true, false><<<grid, kWarps * 32, 0, st>>>(in, nullptr, rows, N, field, scale);
+    field_encode_kernel<V, LPR, true, false><<<grid, kWarps * 32, 0, st>>>(in, nullptr, rows, N, field, scale);
   else
-    field_encode_kernel<V, false, true><<<grid, kWarps * 32, 0, st>>>(in, out, rows, N, nullptr, nullptr);
+    field_encode_kernel<V, LPR, false, true><<<grid, kWarps * 32, 0, st>>>(in, out, rows, N, nullptr, nullptr);
   return cudaGetLastError();
 }
 
@@ -254,15 +271,24 @@ cudaError_t decode_v(const uint32_t* field, const float* scale, int rows, int N,
 cudaError_t launch_field_encode(const float* in, float* out, uint32_t* field, float* scale, int rows, int N,
                                 cudaStream_t st) {
   if (rows == 0) return cudaSuccess;
+  if (N <= 128) {  // sixteen lanes per row, two rows per warp
+    switch ((N + 15) / 16) {
+      case 1: return encode_v<1, 16>(in, out, field, scale, rows, N, st);
+      case 2: return encode_v<2, 16>(in, out, field, scale, rows, N, st);
+      case 3: return encode_v<3, 16>(in, out, field, scale, rows, N, st);
+      case 4: return encode_v<4, 16>(in, out, field, scale, rows, N, st);
+      case 5: return encode_v<5, 16>(in, out, field, scale, rows, N, st);
+      case 6: return encode_v<6, 16>(in, out, field, scale, rows, N, st);
+      case 7: return encode_v<7, 16>(in, out, field, scale, rows, N, st);
+      case 8: return encode_v<8, 16>(in, out, field, scale, rows, N, st);
+      default: return cudaErrorInvalidValue;
+    }
+  }
   switch ((N + 31) / 32) {
-    case 1: return encode_v<1>(in, out, field, scale, rows, N, st);
-    case 2: return encode_v<2>(in, out, field, scale, rows, N, st);
-    case 3: return encode_v<3>(in, out, field, scale, rows, N, st);
-    case 4: return encode_v<4>(in, out, field, scale, rows, N, st);
-    case 5: return encode_v<5>(in, out, field, scale, rows, N, st);
-    case 6: return encode_v<6>(in, out, field, scale, rows, N, st);
-    case 7: return encode_v<7>(in, out, field, scale, rows, N, st);
-    case 8: return encode_v<8>(in, out, field, scale, rows, N, st);
+    case 5: return encode_v<5, 32>(in, out, field, scale, rows, N, st);
+    case 6: return encode_v<6, 32>(in, out, field, scale, rows, N, st);
+    case 7: return encode_v<7, 32>(in, out, field, scale, rows, N, st);
+    case 8: return encode_v<8, 32>(in, out, field, scale, rows, N, st);
     default: return cudaErrorInvalidValue;
   }
 }
