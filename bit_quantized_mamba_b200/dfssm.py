@@ -276,9 +276,20 @@ def _field_rows(state):
     return state.numel() // N if N else 0, N
 
 
+def _field_dtypes(state=None, field=None, scale=None):
+    """The density-field calls take f32 rows and scales and 32-bit field words (int32 or uint32)."""
+    if state is not None and state.dtype != torch.float32:
+        raise ValueError(f"state rows must be float32, not {state.dtype}")
+    if field is not None and field.dtype not in (torch.int32, getattr(torch, "uint32", torch.int32)):
+        raise ValueError(f"field words must be int32 or uint32, not {field.dtype}")
+    if scale is not None and scale.dtype != torch.float32:
+        raise ValueError(f"scales must be float32, not {scale.dtype}")
+
+
 def state_field_encode(state, field=None, scale=None, stream=None):
     """Density-field encoding of the state rows [..., N] (dfssm_state_field_encode): returns (field int32
     [rows, N/8] holding the u32 words, scale float32 [rows])."""
+    _field_dtypes(state, field, scale)
     rows, N = _field_rows(state)
     if field is None:
         field = torch.empty((rows, N // 8), dtype=torch.int32, device=state.device)
@@ -291,6 +302,7 @@ def state_field_encode(state, field=None, scale=None, stream=None):
 
 def state_field_decode(field, scale, N: int, out=None, stream=None):
     """Popcount readout of density fields [rows, N/8] (dfssm_state_field_decode) into rows [rows, N]."""
+    _field_dtypes(out, field, scale)
     rows = scale.numel()
     if out is None:
         out = torch.empty((rows, N), dtype=torch.float32, device=scale.device)
@@ -302,6 +314,7 @@ def state_field_decode(field, scale, N: int, out=None, stream=None):
 def state_field_roundtrip(state, field=None, scale=None, stream=None):
     """state <- readout(encode(state)) in place (dfssm_state_field_roundtrip); field and scale, when
     given, receive the encoding too."""
+    _field_dtypes(state, field, scale)
     rows, N = _field_rows(state)
     _check("dfssm_state_field_roundtrip", lib().dfssm_state_field_roundtrip(
         _ptr(state), rows, N, _ptr(field), _ptr(scale), _stream(stream)))
@@ -519,6 +532,7 @@ def cpu_layer_decode(stack: LayerStack, hidden: torch.Tensor) -> torch.Tensor:
 def cpu_state_field_encode(state: torch.Tensor, field=None, scale=None):
     """dfssm_cpu_state_field_encode on host rows [..., N]: returns (field int32 [rows, N/8] holding the u32
     words, scale float32 [rows])."""
+    _field_dtypes(state, field, scale)
     rows, N = _field_rows(state)
     if field is None:
         field = torch.empty((rows, N // 8), dtype=torch.int32)
@@ -531,6 +545,7 @@ def cpu_state_field_encode(state: torch.Tensor, field=None, scale=None):
 
 def cpu_state_field_decode(field: torch.Tensor, scale: torch.Tensor, N: int, out=None):
     """dfssm_cpu_state_field_decode: the popcount readout of host fields into rows [rows, N]."""
+    _field_dtypes(out, field, scale)
     rows = scale.numel()
     if out is None:
         out = torch.empty((rows, N), dtype=torch.float32)
@@ -541,6 +556,7 @@ def cpu_state_field_decode(field: torch.Tensor, scale: torch.Tensor, N: int, out
 
 def cpu_state_field_roundtrip(state: torch.Tensor, field=None, scale=None):
     """dfssm_cpu_state_field_roundtrip: host rows replaced in place by the readout of their encoding."""
+    _field_dtypes(state, field, scale)
     rows, N = _field_rows(state)
     _check("dfssm_cpu_state_field_roundtrip", cpu_lib().dfssm_cpu_state_field_roundtrip(
         _hptr(state), rows, N, _hptr(field), _hptr(scale)))

@@ -6,6 +6,7 @@ AVX-512 VNNI.
 """
 import numpy as np
 import pytest
+from hypothesis import given, settings, strategies as st
 import torch
 
 import oracle
@@ -152,3 +153,31 @@ def test_state_field_edge_rows(engine):
     assert np.array_equal(scale.numpy(), s_ref)
     assert np.array_equal(engine.cpu_state_field_decode(field, scale, N).numpy(),
                           oracle.field_decode(f_ref, s_ref, N))
+
+
+def test_state_field_binding_rejects_wrong_dtypes(engine):
+    with pytest.raises(ValueError):
+        engine.cpu_state_field_encode(torch.zeros((4, 128), dtype=torch.float64))
+    with pytest.raises(ValueError):
+        engine.cpu_state_field_decode(torch.zeros((4, 16), dtype=torch.int64), torch.zeros(4), 128)
+    with pytest.raises(ValueError):
+        engine.cpu_state_field_decode(torch.zeros((4, 16), dtype=torch.int32),
+                                      torch.zeros(4, dtype=torch.float64), 128)
+    with pytest.raises(ValueError):
+        engine.state_field_encode(torch.zeros((4, 128)))  # a host tensor on the CUDA entry point
+
+
+@settings(max_examples=200, deadline=None)
+@given(st.sampled_from([8, 16, 40, 128]).flatmap(
+    lambda n: st.lists(st.floats(width=32, allow_nan=False, allow_infinity=False), min_size=n, max_size=n)))
+def test_state_field_arbitrary_rows(vals):
+    """The engine's integer closed form against the oracle's loop on arbitrary finite fp32 rows."""
+    build.build_cpu()
+    if not dfssm.cpu_available():
+        pytest.skip("host CPU has no AVX-512 VNNI")
+    S = np.array([vals], np.float32)
+    N = S.shape[1]
+    f_ref, s_ref = oracle.field_encode(S)
+    field, scale = dfssm.cpu_state_field_encode(torch.from_numpy(S))
+    assert np.array_equal(field.numpy().view(np.uint32), f_ref)
+    assert np.array_equal(scale.numpy(), s_ref)

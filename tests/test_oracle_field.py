@@ -14,6 +14,7 @@ import os
 
 import numpy as np
 import pytest
+from hypothesis import given, settings, strategies as st
 
 import oracle
 from bit_quantized_mamba_b200 import inputs
@@ -114,3 +115,23 @@ def test_readout_levels_of_arbitrary_fields():
     back = oracle.field_decode(field, scale, N)
     p = _cells(field, N).reshape(rows, N, 4).sum(axis=2)
     assert np.array_equal(back / scale[:, None], p * 0.5 - 1.0)
+
+
+_f32 = st.floats(width=32, allow_nan=False, allow_infinity=False)
+
+
+@settings(max_examples=300, deadline=None)
+@given(st.sampled_from([8, 16, 24, 32, 64]).flatmap(lambda n: st.lists(_f32, min_size=n, max_size=n)))
+def test_closed_form_on_arbitrary_rows(vals):
+    """Any finite fp32 row, extremes and subnormals included: the closed form holds cell by cell and
+    every readout lies on one of the five levels of the row's absmax."""
+    S = np.array([vals], np.float32)
+    N = S.shape[1]
+    field, scale = oracle.field_encode(S)
+    D, c = _densities_units(S)
+    assert scale[0] == c[0]
+    P = np.cumsum(np.repeat(D, 4, axis=1), axis=1)
+    assert np.array_equal(np.cumsum(_cells(field, N), axis=1), (P + (1 << 24)) >> 25)
+    back = oracle.field_decode(field, scale, N)
+    levels = np.array([-1.0, -0.5, 0.0, 0.5, 1.0], np.float32) * scale[0]
+    assert np.all(np.isin(back[0], levels))
