@@ -204,28 +204,28 @@ void linear(const dfssm_linear_t& L, const int8_t* q, const float* s, const int*
   for (int ci = 0; ci < chunks; ++ci) {
     const int o0 = ci * kChunk, o1 = std::min(d_out, o0 + kChunk);
     fn(L.bits, d_in, o0, o1, qpad, dpad, sq, B, acc, d_out);
-  // epilogue, eight outputs at a time so that their LoRA sums (each in r order) run side by side
-  for (int b = 0; b < B; ++b) {
-    const float* tb = tf.data() + (size_t)b * DFSSM_MAX_RANK;
-    for (int ob = o0; ob < o1; ob += 8) {
-      const int no = std::min(8, o1 - ob);
-      double lora[8] = {};
-      for (int r = 0; r < rank; ++r) {
-        const double t = (double)tb[r];
-        for (int k = 0; k < no; ++k) lora[k] += (double)L.lora_a[(size_t)(ob + k) * rank + r] * t;
-      }
-      for (int k = 0; k < no; ++k) {
-        const int o = ob + k;
-        const size_t i = (size_t)b * d_out + o;
-        const int a = acc[i];
-        const double scaffold = (double)a * (double)s[b] * (double)L.w_scale[o];
-        const double corr = rank > 0 ? (double)L.lora_a_scale[o] * lora[k] : 0.0;
-        const float v = f32(scaffold + corr);
-        y[i] = out_add ? out_add[i] + v : v;
-        if (dbg_acc) dbg_acc[i] = a;
+    // epilogue, eight outputs at a time so that their LoRA sums (each in r order) run side by side
+    for (int b = 0; b < B; ++b) {
+      const float* tb = tf.data() + (size_t)b * DFSSM_MAX_RANK;
+      for (int ob = o0; ob < o1; ob += 8) {
+        const int no = std::min(8, o1 - ob);
+        double lora[8] = {};
+        for (int r = 0; r < rank; ++r) {
+          const double t = (double)tb[r];
+          for (int k = 0; k < no; ++k) lora[k] += (double)L.lora_a[(size_t)(ob + k) * rank + r] * t;
+        }
+        for (int k = 0; k < no; ++k) {
+          const int o = ob + k;
+          const size_t i = (size_t)b * d_out + o;
+          const int a = acc[i];
+          const double scaffold = (double)a * (double)s[b] * (double)L.w_scale[o];
+          const double corr = rank > 0 ? (double)L.lora_a_scale[o] * lora[k] : 0.0;
+          const float v = f32(scaffold + corr);
+          y[i] = out_add ? out_add[i] + v : v;
+          if (dbg_acc) dbg_acc[i] = a;
+        }
       }
     }
-  }
   }
 }
 
