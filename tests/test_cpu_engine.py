@@ -181,3 +181,31 @@ def test_state_field_arbitrary_rows(vals):
     field, scale = dfssm.cpu_state_field_encode(torch.from_numpy(S))
     assert np.array_equal(field.numpy().view(np.uint32), f_ref)
     assert np.array_equal(scale.numpy(), s_ref)
+
+
+def test_decode_with_field_round_trips_at_chunk_boundaries(engine):
+    """The density field applied at chunk boundaries of a decode: every 3 tokens each layer's SSM state
+    is replaced by the readout of its encoding, on the engine (dfssm_cpu_state_field_roundtrip) and on
+    the oracle (its encode, then its readout).  Residual stream and states stay bit-identical."""
+    dims = dict(d_model=256, nheads=4, headdim=32, d_state=64, ngroups=1)
+    n_layers, n_tokens, chunk = 2, 7, 3
+    model = inputs.decode_model(seed=31, n_layers=n_layers, n_tokens=n_tokens, batch=1, rank=16, **dims)
+    conv, ssm = inputs.zero_states(1, n_layers, 4, 32, 64, 1)
+    stack, cs, ss = _stack(model, conv.copy(), ssm.copy(), dims)
+    olayers = [dict(l, in_proj=oracle.Linear.from_dict(l["in_proj"]),
+                    out_proj=oracle.Linear.from_dict(l["out_proj"])) for l in model["layers"]]
+    oconv, ossm = conv.copy(), ssm.copy()
+    for t in range(n_tokens):
+        hr = np.array(model["emb"][t], dtype=np.float32)
+        h = torch.from_numpy(hr.copy())
+        engine.cpu_layer_decode(stack, h)
+        for i, ol in enumerate(olayers):
+            oracle.layer_decode(ol, hr, oconv[i], ossm[i])
+        if (t + 1) % chunk == 0:
+            for i in range(n_layers):
+                engine.cpu_state_field_roundtrip(ss[i])
+                f, sc = oracle.field_encode(ossm[i])
+                ossm[i][...] = oracle.field_decode(f, sc, 64).reshape(ossm[i].shape)
+        assert np.array_equal(h.numpy(), hr), f"token {t}: hidden rows differ"
+        for i in range(n_layers):
+            assert np.array_equal(ss[i].numpy(), ossm[i]), f"token {t} layer {i}: SSM state differs"
