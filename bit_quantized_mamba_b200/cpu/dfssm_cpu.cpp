@@ -35,7 +35,7 @@ inline double silu(double v) { return v / (1.0 + std::exp(-v)); }
 bool has_vnni() {
   __builtin_cpu_init();
   return __builtin_cpu_supports("avx512f") && __builtin_cpu_supports("avx512bw") &&
-         __builtin_cpu_supports("avx512vnni");
+         __builtin_cpu_supports("avx512vl") && __builtin_cpu_supports("avx512vnni");
 }
 
 // 64-byte aligned scratch that lives for one call.
@@ -50,35 +50,50 @@ struct Buf {
 // ---------------------------------------------------------------------------------------- quantizer
 
 // Per-token absmax int8 quantizer: s = fl32(m / 127), q = clamp(rint(fl32(v / s)), +-127) with round
-// half to even; an all-zero row gives s = 0, q = 0.  Returns s; writes the code sum.
-float quantize(const float* v, int n, int8_t* q, int* sumq) {
-  float m = 0.0f;
-  for (int i = 0; i < n; ++i) m = std::max(m, std::fabs(v[i]));
-  int sq = 0;
+// half to even; an all-zero row gives s = 0, q = 0.  Returns s; writes the code sum.  Sixteen values at a
+// time: the IEEE division and the rounding to nearest even are single AVX-512 operations.
+__attribute__((target("avx512f,avx512bw,avx512vl"))) float quantize(const float* v, int n, int8_t* q, int* sumq) {
+  __m512 vm = _mm512_setzero_ps();
+  for (int i = 0; i < n; i += 16) {
+    const __mmask16 k = n - i >= 16 ? (__mmask16)0xFFFF : (__mmask16)((1u << (n - i)) - 1u);
+    vm = _mm512_max_ps(vm, _mm512_abs_ps(_mm512_maskz_loadu_ps(k, v + i)));
+  }
+  const float m = _mm512_reduce_max_ps(vm);
   if (m == 0.0f) {
     std::memset(q, 0, (size_t)n);
     *sumq = 0;
     return 0.0f;
   }
   const float s = m / 127.0f;
-  for (int i = 0; i < n; ++i) {
-    float k = std::nearbyint(v[i] / s);
-    k = std::min(127.0f, std::max(-127.0f, k));
-    q[i] = (int8_t)k;
-    sq += (int)q[i];
+  const __m512 vs = _mm512_set1_ps(s), hi = _mm512_set1_ps(127.0f), lo = _mm512_set1_ps(-127.0f);
+  __m512i vsum = _mm512_setzero_si512();
+  for (int i = 0; i < n; i += 16) {
+    const __mmask16 k = n - i >= 16 ? (__mmask16)0xFFFF : (__mmask16)((1u << (n - i)) - 1u);
+    __m512 t = _mm512_div_ps(_mm512_maskz_loadu_ps(k, v + i), vs);
+    t = _mm512_roundscale_ps(t, _MM_FROUND_TO_NEAREST_INT | _MM_FROUND_NO_EXC);
+    t = _mm512_min_ps(hi, _mm512_max_ps(lo, t));
+    const __m512i c = _mm512_maskz_cvtps_epi32(k, t);
+    _mm_mask_storeu_epi8(q + i, k, _mm512_cvtepi32_epi8(c));
+    vsum = _mm512_add_epi32(vsum, c);
   }
-  *sumq = sq;
+  *sumq = _mm512_reduce_add_epi32(vsum);
   return s;
 }
 
 // RMSNorm (eps 1e-5, weight w), then the quantizer on the normalised row:
 //   r = fl32(1 / sqrt(sum h^2 / n + eps)) (the fp64 sum in index order, the squares exact),
 //   u = fl32(fl32(h r) w).
-float norm_quantize(const float* h, const float* w, int n, float* u, int8_t* q, int* sumq) {
+__attribute__((target("avx512f,avx512bw,avx512vl"))) float norm_quantize(const float* h, const float* w, int n,
+                                                                 float* u, int8_t* q, int* sumq) {
   double ss = 0.0;
   for (int i = 0; i < n; ++i) ss += (double)h[i] * (double)h[i];
   const float r = f32(1.0 / std::sqrt(ss / (double)n + kEps));
-  for (int i = 0; i < n; ++i) u[i] = (h[i] * r) * w[i];
+  const __m512 vr = _mm512_set1_ps(r);
+  for (int i = 0; i < n; i += 16) {
+    const __mmask16 k = n - i >= 16 ? (__mmask16)0xFFFF : (__mmask16)((1u << (n - i)) - 1u);
+    const __m512 hr = _mm512_mul_ps(_mm512_maskz_loadu_ps(k, h + i), vr);
+    _mm512_mask_storeu_ps(u + i, k, _mm512_mul_ps(hr, _mm512_maskz_loadu_ps(k, w + i)));
+  }
   return quantize(u, n, q, sumq);
 }
 
@@ -315,13 +330,15 @@ __attribute__((target("avx512f"))) void ssm_rows8(float* S, int N, int N8, float
   for (int j = 0; j < R; ++j) _mm512_storeu_pd(acc_out + 8 * j, acc[j]);
 }
 
-// SSM state update and readout of one token:
+// SSM state update and readout of one token, then the gate:
 //   dt = fl32(softplus(fl32(dt_raw + dt_bias))), A = fl32(-exp(A_log)), dA = fl32(exp(fl32(dt A)))
 //   S <- fl32(fl32(dA S) + fl32(fl32(dt x) B));  y = fl32(sum_n S C + D x) (fp64, n in order)
+//   gate = fl32(y fl32(SiLU(z)))  (y itself is not stored)
 // Rows go sixteen (or eight) at a time through ssm_rows8 for the whole multiple of 8 in n; the rest of n,
 // and the rows left over when P % 8 != 0, continue each row's sum one term at a time.
 void ssm_step(float* S_all, const float* x, const float* dt_raw, const float* A_log, const float* dt_bias,
-              const float* Dv, const float* Bm, const float* Cm, float* y, int H, int P, int N, int G) {
+              const float* Dv, const float* Bm, const float* Cm, const float* z, float* gate, int H, int P,
+              int N, int G) {
   const int hpg = H / G, N8 = N / 8 * 8;
 #pragma omp parallel for schedule(static)
   for (int h = 0; h < H; ++h) {
@@ -353,8 +370,9 @@ void ssm_step(float* S_all, const float* x, const float* dt_raw, const float* A_
           S[n] = (dA * S[n]) + (dtx[k] * Bg[n]);
           a += (double)S[n] * (double)Cg[n];
         }
-        const float xv = x[(size_t)h * P + p0 + k];
-        y[(size_t)h * P + p0 + k] = f32(a + (double)Dv[h] * (double)xv);
+        const size_t idx = (size_t)h * P + p0 + k;
+        const float yv = f32(a + (double)Dv[h] * (double)x[idx]);
+        gate[idx] = yv * f32(silu((double)z[idx]));
       }
     }
   }
@@ -503,7 +521,7 @@ int dfssm_cpu_layer_decode(const dfssm_layer_t* layers, int n_layers, const dfss
   }
   if (!has_vnni()) return DFSSM_EUNSUPPORTED;
   const int nmax = std::max(Dm, E);
-  std::vector<float> u((size_t)nmax), zx((size_t)B * d_ip), xc((size_t)C), y((size_t)E), g((size_t)B * E);
+  std::vector<float> u((size_t)nmax), zx((size_t)B * d_ip), xc((size_t)C), g((size_t)B * E);
   std::vector<int8_t> q((size_t)B * nmax);
   std::vector<float> s(B);
   std::vector<int> sq(B);
@@ -518,10 +536,7 @@ int dfssm_cpu_layer_decode(const dfssm_layer_t* layers, int n_layers, const dfss
       // conv on x|B|C, SSM step, gate y SiLU(z)
       conv_step(conv_states[l] + (size_t)b * C * 3, Ly.conv_w, Ly.conv_b, zb + E, xc.data(), C);
       ssm_step(ssm_states[l] + (size_t)b * H * P * N, xc.data(), zb + E + C, Ly.A_log, Ly.dt_bias, Ly.D,
-               xc.data() + E, xc.data() + E + G * N, y.data(), H, P, N, G);
-      float* gb = g.data() + (size_t)b * E;
-#pragma omp parallel for schedule(static)
-      for (int i = 0; i < E; ++i) gb[i] = y[i] * f32(silu((double)zb[i]));
+               xc.data() + E, xc.data() + E + G * N, zb, g.data() + (size_t)b * E, H, P, N, G);
     }
     // gated norm + quantize, out_proj with the residual add
     for (int b = 0; b < B; ++b)

@@ -15,7 +15,7 @@
  *   - All pointers are HOST pointers (the dfssm_linear_t / dfssm_layer_t structs of dfssm.h filled with
  *     host addresses).  The caller owns every buffer; calls are synchronous; no global state besides the
  *     OpenMP thread count.
- *   - Each entry point checks at run time that the CPU supports AVX-512 F/BW and VNNI and returns
+ *   - Each entry point checks at run time that the CPU supports AVX-512 F/BW/VL and VNNI and returns
  *     DFSSM_EUNSUPPORTED otherwise (dfssm_cpu_available() tells in advance).
  *   - Arguments are validated first; on a negative status nothing was written.
  */
@@ -32,7 +32,7 @@ extern "C" {
 
 int dfssm_cpu_abi_version(void);
 
-/* 1 when the host CPU has AVX-512 F, BW and VNNI, else 0. */
+/* 1 when the host CPU has AVX-512 F, BW, VL and VNNI, else 0. */
 int dfssm_cpu_available(void);
 
 /* OpenMP threads used by the following calls (n <= 0: all available).  Returns the count in use. */
