@@ -16,8 +16,8 @@
 // with lo = (4 Q_n + 2^24) mod 2^25.  Only Q_n mod 2^23 enters lo, so the prefix sums run in wrapping
 // 32-bit integers, exactly.  A row goes to LPR lanes (16 for N <= 128, two rows per warp; else 32): each
 // lane its ceil(N / LPR) consecutive values, one scan over the row's lanes for the Q of its first value;
-// no serial chain.  The state row is read once (and, for the round trip, written once), the field and
-// scale written once.
+// no serial chain.  The readout kernel keeps one warp per row.  The state row is read once (and, for the
+// round trip, written once), the field and scale written once.
 
 #include <cstdint>
 #include <cuda_runtime.h>
@@ -28,13 +28,14 @@
 namespace dfssm {
 namespace {
 
-constexpr int kWarps = 8;                    // warps per CTA, one row each at a time
+constexpr int kWarps = 8;                    // warps per CTA
 constexpr unsigned kFull = 0xffffffffu;
 constexpr float kUnits = 33554432.0f;        // 2^25
 constexpr uint32_t kHalfUnit = 1u << 24;
 constexpr uint32_t kUnitMask = (1u << 25) - 1u;
 
-// Rows a warp holds at once (loads of all of them issued before the first is processed).
+// Row groups a warp holds at once (the loads of all of them are issued before the first is processed); a
+// group is one row, or two for the sixteen-lane split of the encoder.
 template <int V>
 constexpr int rows_per_warp() { return V <= 4 ? 4 : 2; }
 
