@@ -209,3 +209,26 @@ def test_decode_with_field_round_trips_at_chunk_boundaries(engine):
         assert np.array_equal(h.numpy(), hr), f"token {t}: hidden rows differ"
         for i in range(n_layers):
             assert np.array_equal(ss[i].numpy(), ossm[i]), f"token {t} layer {i}: SSM state differs"
+
+
+@settings(max_examples=40, deadline=None)
+@given(d_out=st.integers(1, 300), d_in_words=st.integers(1, 48), rank=st.integers(0, 16),
+       B=st.integers(1, 16), seed=st.integers(0, 2 ** 31 - 1))
+def test_linear_random_shapes(d_out, d_in_words, rank, B, seed):
+    """Random linear shapes (d_out across partial 64-row chunks, d_in = 32..1536 with odd 32-word tails,
+    every rank and token count): codes, scales, accumulators, t and outputs bit-identical to the oracle."""
+    build.build_cpu()
+    if not dfssm.cpu_available():
+        pytest.skip("host CPU has no AVX-512 VNNI")
+    d_in = 32 * d_in_words
+    gen = np.random.default_rng(seed)
+    lin = inputs.linear(gen, d_out, d_in, rank)
+    x = inputs.normal(gen, (B, d_in)) * np.float32(2)
+    dbg = dict(acc=torch.zeros((B, d_out), dtype=torch.int32),
+               lora_t=torch.zeros((B, max(rank, 1)), dtype=torch.int32))
+    y = dfssm.cpu_linear_decode(dfssm.Linear.from_host(lin, "cpu"), torch.from_numpy(x), debug=dbg).numpy()
+    ref = oracle.linear_decode(oracle.Linear.from_dict(lin), x)
+    assert np.array_equal(dbg["acc"].numpy(), ref["acc"])
+    if rank:
+        assert np.array_equal(dbg["lora_t"].numpy()[:, :rank], ref["t"])
+    assert np.array_equal(y, ref["y"])
